@@ -1,0 +1,242 @@
+/*
+ * sma.h -- C ABI of libsma: scaled-dot-product attention forward under
+ * structured masks on NVIDIA B200 (sm_100a).
+ *
+ * Four operations, all asynchronous on the caller's CUDA stream:
+ *
+ *   dfa_block_map      full / partial / empty key-tile lists of the DFlash
+ *                      draft-training mask, computed from the block anchors
+ *                      alone (no dense mask is ever built).
+ *   dfa_attn_fwd       attention forward under that mask.
+ *   masked_attn_fwd    attention forward with a broadcastable 4D boolean mask
+ *                      and/or additive bias, optional causal masking, and the
+ *                      single-query grouped-head ("swapped") decode path.
+ *   dynamic_topk_mask  boolean keep mask of the window_size largest entries
+ *                      of an attention bias per row, after a pre-mask.
+ *
+ * plus mask_tile_summary (the tile classifier masked_attn_fwd runs on an
+ * explicit mask), workspace queries and error reporting.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor arguments are DEVICE pointers owned by the caller; the library
+ *   allocates no device memory and keeps no state besides a thread-local
+ *   error string and one device error word per device.
+ * - Strides are in ELEMENTS.  Q/K/V/O are [batch, length, heads, head_dim]
+ *   with head_dim contiguous; their strides arrays give the batch, length and
+ *   head strides in that order.  Every stride and base address must be a
+ *   multiple of 16 bytes (TMA requirement) for bf16/fp16 inputs.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ * - Arguments are validated on the host before anything is launched; an
+ *   invalid call returns a nonzero status and launches nothing.  The message
+ *   is available from sma_last_error() on the calling thread.
+ * - Faults found on the device (an anchor out of range, a pipeline wait that
+ *   ran out of time) set the device error word; read and clear it with
+ *   sma_device_status().  Kernels never trap.
+ * - Query head h uses key/value head h / (heads / kv_heads) (contiguous
+ *   groups).
+ * - scale <= 0 selects 1/sqrt(head_dim).
+ * - lse (nullable) receives the natural-log log-sum-exp of each row's kept
+ *   scores, float32 [batch, heads, q_len] contiguous; a row with no kept key
+ *   gets -inf and a zero output row.
+ */
+#ifndef SMA_H_
+#define SMA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t sma_status;
+
+#define SMA_OK 0
+#define SMA_ERR_INVALID_ARG 1    /* shape, stride, pointer or value rejected */
+#define SMA_ERR_UNSUPPORTED 2    /* valid but not implemented (e.g. head_dim 96) */
+#define SMA_ERR_CUDA 3           /* a CUDA runtime/driver call failed */
+#define SMA_ERR_WORKSPACE 4      /* workspace smaller than the size query says */
+#define SMA_ERR_DEVICE_TIMEOUT 5 /* a kernel's bounded pipeline wait expired */
+#define SMA_ERR_DEVICE_INPUT 6   /* a device-resident input was out of range */
+
+#define SMA_BF16 0
+#define SMA_FP16 1
+#define SMA_FP32 2
+
+/* Tiles of the block maps and summaries are SMA_TILE x SMA_TILE
+ * (queries x keys). */
+#define SMA_TILE 128
+#define SMA_TILE_EMPTY 0
+#define SMA_TILE_PARTIAL 1
+#define SMA_TILE_FULL 2
+
+#define SMA_IS_CAUSAL_UNSET (-1)
+#define SMA_LAYER_FULL 0
+#define SMA_LAYER_SLIDING 1
+
+/* Message for the last nonzero status returned on this thread ("" if none). */
+const char* sma_last_error(void);
+
+/* ABI version of this header (bumped on any signature change). */
+int32_t sma_abi_version(void);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device into *device_error (SMA_OK if no kernel reported a fault).
+ * Returns SMA_ERR_CUDA if the synchronisation itself failed. */
+sma_status sma_device_status(void* stream, int32_t* device_error);
+
+/* ------------------------------------------------------------------------
+ * DFlash mask description.
+ *
+ * Source: SpecForge issue #452 "flex_attention BlockMask incorrectly created
+ * with H=num_heads", Problem paragraph -- every draft query sees the context
+ * that precedes its block plus the tokens of its own block, identically for
+ * every head (so the maps here have no head dimension).  SpecForge PR #905
+ * "Fix DFlash attention masking", Motivation list -- is_causal absent:
+ * bidirectional inside the block on full-attention layers, causal on
+ * sliding-attention layers; False: bidirectional on both; True: causal on
+ * both.  Same page, reply item 1 (#934): the in-block sliding window keeps
+ * only its left bound.
+ *
+ * Keys are laid out as [context 0..ctx_len) [block 0] ... [block N-1], so
+ * k_len = ctx_len + n_blocks * block_size and q_len = n_blocks * block_size.
+ * Query i of block j sits at position anchor[b][j] + i, context key k at
+ * position k.  Query (j, i) keeps
+ *   context key k  iff k < anchor[b][j]  and (sliding: anchor[b][j]+i-k < W)
+ *   draft key of block j' at offset t  iff j' == j and (causal: t <= i)
+ *                                        and (sliding: i - t < W).
+ * ---------------------------------------------------------------------- */
+typedef struct dfa_mask_desc {
+  int32_t batch;          /* B >= 1 */
+  int32_t n_blocks;       /* N >= 1 draft blocks per sequence */
+  int32_t block_size;     /* tokens per draft block, >= 1 */
+  int32_t ctx_len;        /* context keys, >= 0 */
+  int32_t is_causal;      /* SMA_IS_CAUSAL_UNSET, 0 or 1 */
+  int32_t layer_type;     /* SMA_LAYER_FULL or SMA_LAYER_SLIDING */
+  int32_t sliding_window; /* W >= 1; read only when layer_type is sliding */
+} dfa_mask_desc;
+
+/* Tile-grid size of the block map: q_tiles = ceil(q_len/128),
+ * kv_tiles = ceil(k_len/128). */
+sma_status dfa_block_map_dims(const dfa_mask_desc* desc, int32_t* q_tiles, int32_t* kv_tiles);
+
+/* DFlash block map, computed analytically from the anchors.
+ *
+ * anchors   int32 [batch, n_blocks] device, row-major; each in [0, ctx_len]
+ *           (need not be sorted or distinct).  Out-of-range anchors are
+ *           clamped and raise SMA_ERR_DEVICE_INPUT in the device error word.
+ * num_full  int32 [batch, q_tiles]           number of FULL key tiles
+ * full_idx  int32 [batch, q_tiles, kv_tiles] their indices, ascending, then -1
+ * num_part  int32 [batch, q_tiles]           number of PARTIAL key tiles
+ * part_idx  int32 [batch, q_tiles, kv_tiles] their indices, ascending, then -1
+ * A tile is FULL iff it lies inside [0, k_len) and every (valid query, key)
+ * pair in it is kept, EMPTY iff none is, PARTIAL otherwise.  This is the
+ * flex_attention BlockMask with a head dim of 1 that issue #452 asks for. */
+sma_status dfa_block_map(const dfa_mask_desc* desc, const int32_t* anchors, int32_t* num_full,
+                         int32_t* full_idx, int32_t* num_part, int32_t* part_idx, void* stream);
+
+/* Workspace bytes dfa_attn_fwd needs for this problem (block map and tile
+ * schedule).  The caller allocates it; it may be reused across calls that are
+ * ordered on one stream. */
+sma_status dfa_attn_fwd_workspace_size(const dfa_mask_desc* desc, int32_t heads, int32_t kv_heads,
+                                       int32_t head_dim, size_t* bytes);
+
+/* Attention forward under the DFlash mask.
+ *
+ * q    [batch, q_len, heads, head_dim]     strides q_strides (batch, row, head)
+ * k, v [batch, k_len, kv_heads, head_dim]  strides k_strides / v_strides
+ * out  [batch, q_len, heads, head_dim]     strides o_strides; same dtype as q
+ * dtype SMA_BF16 / SMA_FP16 (tensor cores, fp32 accumulation and softmax) or
+ *       SMA_FP32 (fp32 FFMA throughout).  head_dim 64 or 128; heads a
+ *       multiple of kv_heads.
+ * Only key tiles the block map marks FULL or PARTIAL are computed; the mask is
+ * evaluated per element on PARTIAL tiles only. */
+sma_status dfa_attn_fwd(const dfa_mask_desc* desc, const int32_t* anchors, int32_t dtype,
+                        int32_t heads, int32_t kv_heads, int32_t head_dim, float scale,
+                        const void* q, const int64_t q_strides[3], const void* k,
+                        const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
+                        void* out, const int64_t o_strides[3], float* lse, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Broadcastable 4D mask / bias contract.
+ *
+ * Source: flash-sparse-attention PR #190 "Broadcastable 4D mask/bias,
+ * 128-rounded key length, stride-0 broadcasting, and dbias reductions",
+ * Design and Changes sections.  mask (uint8 0/1, True = keep) and bias
+ * (additive, SMA_BF16/SMA_FP16/SMA_FP32) are rank 4 with sizes
+ *   ({batch|1}, {heads|kv_heads|1}, {q_len|1}, round_up(k_len, 128))
+ * and a contiguous last dim (stride 1).  Size-1 dims broadcast with stride 0
+ * whatever stride is passed; there is no implicit 3D form.  A head dim of
+ * kv_heads (when kv_heads != heads) is indexed by the query head's KV head.
+ * Columns in [k_len, round_up(k_len,128)) are never read as meaningful: they
+ * are never attended whatever they hold.
+ * ---------------------------------------------------------------------- */
+
+/* Tile codes of an explicit mask at its own broadcast shape:
+ * codes uint8 [m0, m1, ceil(m2/128), ceil(k_len/128)] contiguous (device),
+ * where (m0, m1, m2, m3) = mask_sizes; columns >= k_len count as not kept.
+ * mask must be 16-byte aligned with 16-byte-multiple strides (or 0). */
+sma_status mask_tile_summary(const uint8_t* mask, const int64_t mask_sizes[4],
+                             const int64_t mask_strides[4], int32_t k_len, uint8_t* codes,
+                             void* stream);
+
+/* Workspace bytes masked_attn_fwd needs (tile summary, tile lists and the
+ * split-KV partials of the single-query path).  mask_sizes may be NULL when
+ * no mask will be passed. */
+sma_status masked_attn_fwd_workspace_size(int32_t batch, int32_t heads, int32_t kv_heads,
+                                          int32_t q_len, int32_t k_len, int32_t head_dim,
+                                          const int64_t mask_sizes[4], size_t* bytes);
+
+/* Attention forward with optional mask, bias and causal masking.
+ *
+ * s = scale * q.k + bias[...];  key k is kept iff k < k_len and
+ * mask[...] (when given) and (is_causal -> k <= q + k_len - q_len, i.e.
+ * bottom-right aligned).
+ * mask / bias: NULL or the 4D contract above; their sizes/strides arrays are
+ * ignored when the pointer is NULL.
+ * When q_len == 1 (decode) the grouped query heads of each KV head are
+ * processed together as rows of one problem (the "swapped" path of PR #190,
+ * Swapped path bullets); mask/bias keep their original batch/head meaning.
+ * The result is the same as the unswapped definition. */
+sma_status masked_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t q_len, int32_t k_len, int32_t head_dim, float scale,
+                           int32_t is_causal, const void* q, const int64_t q_strides[3],
+                           const void* k, const int64_t k_strides[3], const void* v,
+                           const int64_t v_strides[3], const uint8_t* mask,
+                           const int64_t mask_sizes[4], const int64_t mask_strides[4],
+                           const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+                           const int64_t bias_strides[4], void* out, const int64_t o_strides[3],
+                           float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Dynamic top-k keep mask.
+ *
+ * Source: flash-sparse-attention PR #197 "Centralize dynamic mask creation
+ * for FDMA" -- Design (dynamic_mask / create_mask) and Implementation Notes:
+ * positions the pre-mask marks invalid are set to the minimum finite value of
+ * the BIAS dtype before choosing the window_size largest entries of each row,
+ * so they are never selected.
+ *
+ * bias      [b, h, q, round_up(k_len,128)] dtype bias_dtype, strides given,
+ *           last dim contiguous.  Only columns < k_len take part.
+ * pre_mask  NULL or uint8 0/1 4D with sizes (pb, ph, pq, pk): pb in {1, b},
+ *           ph in {1, h}, pq in {1, q}, pk >= 1, last stride 1; columns
+ *           >= pk are invalid.  A 2D (batch, k_len) pre-mask is passed as
+ *           sizes (batch, 1, 1, k_len).
+ * out_mask  uint8 [b, h, q, round_up(k_len,128)] contiguous (device); columns
+ *           >= k_len are written 0.
+ * Per row: entry k is kept iff it is among the window_size largest masked
+ * values (equal values: lower k first; -0 equals +0) and the pre-mask keeps
+ * it.  window_size >= k_len keeps exactly the pre-mask. */
+sma_status dynamic_topk_mask(int32_t bias_dtype, const void* bias, const int64_t bias_sizes[4],
+                             const int64_t bias_strides[4], int32_t k_len, const uint8_t* pre_mask,
+                             const int64_t pre_mask_sizes[4], const int64_t pre_mask_strides[4],
+                             int32_t window_size, uint8_t* out_mask, void* stream);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* SMA_H_ */

@@ -1,0 +1,21 @@
+"""Structured-mask attention forward for NVIDIA B200 (sm_100a).
+
+Thin Python binding over libsma (C ABI in include/sma.h): DFlash draft-training
+masks computed analytically from block anchors, broadcastable 4D mask/bias
+attention with the grouped-head decode path, and the dynamic top-k keep mask.
+"""
+from ._native import NativeLibraryMissing, SmaError  # noqa: F401
+from .ops import (  # noqa: F401
+    LAYER_FULL,
+    LAYER_SLIDING,
+    device_status,
+    dfa_attn_fwd,
+    dfa_attn_fwd_workspace_size,
+    dfa_block_map,
+    dfa_block_map_dims,
+    dynamic_topk_mask,
+    mask_tile_summary,
+    masked_attn_fwd,
+    masked_attn_fwd_workspace_size,
+    round_up_k,
+)

@@ -1,0 +1,682 @@
+// Attention forward on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// One persistent CTA per SM walks "units" (batch, KV head, pair of query
+// heads, 128-row query tile).  The two query heads of a unit share the KV
+// head, so they share every K/V tile and -- because both mask families here
+// are identical across the heads of a group -- the same key-tile list.  Only
+// tiles on that list are visited (empty tiles are skipped); the per-element
+// mask is evaluated only on tiles flagged PARTIAL.
+//
+// Warp roles (384 threads, three warpgroups):
+//   warps 0-3  softmax for query tile 0 (one thread per query row)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer: Q tiles, K/V tiles into a ring of smem stages
+//   warp  9    MMA issuer (one thread): S_i = Q_i K^T into TMEM (SS form),
+//              O_i += P_i V with P_i read from TMEM (TS form)
+//   warps 10-11 idle
+// The kernel is launched with kLaunchRegs registers per thread; the producer
+// warpgroup gives registers back (setmaxnreg.dec to kProducerRegs) and the two
+// softmax warpgroups take them (setmaxnreg.inc to kSoftmaxRegs).  The shares
+// add up to exactly the launch allocation:
+//   2 * 128 * kSoftmaxRegs + 128 * kProducerRegs == 384 * kLaunchRegs
+// and the host refuses to launch if the compiled register count differs.
+// TMEM (512 columns): S_0 | S_1 | O_0 | O_1; P_i (bf16/f16 pairs) overwrites
+// the first half of S_i's columns once the softmax has read S_i.
+//
+// Online softmax in the log2 domain with a lazily rescaled reference max: O
+// is rescaled in TMEM only when a row's max grows by more than 2^8.
+//
+// Mask sources (template policy):
+//   DFlash   -- SpecForge issue #452 (Problem paragraph) and PR #905
+//               (Motivation list; reply item 1 on the left-only window): a
+//               row keeps its context prefix [clo, chi) and its own block's
+//               slots [dlo, dhi); evaluated from the anchors.
+//   Explicit -- flash-sparse-attention PR #190 (Design: boolean mask, True =
+//               keep, additive bias, stride-0 broadcast dims), plus
+//               bottom-right causal masking; the bias is added on every kept
+//               tile, the mask read on PARTIAL tiles only.
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <type_traits>
+
+#include "device_common.cuh"
+#include "kernels.h"
+
+namespace sma {
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kProducerRegs = 56;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kProducerRegs == kThreads * kLaunchRegs,
+              "register split must equal the launch allocation");
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct Layout {
+  static constexpr int kStages = D == 128 ? 2 : 4;
+  static constexpr uint32_t kChunkBytes = kTile * 128;  // 64 columns x 128 rows, 128B-swizzled
+  static constexpr uint32_t kTileBytes = kTile * D * 2;
+  static constexpr int kChunks = D / 64;
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kK = kQ + 2 * kTileBytes;
+  static constexpr uint32_t kV = kK + kStages * kTileBytes;
+  static constexpr uint32_t kBars = kV + kStages * kTileBytes;
+  // barrier slots
+  static constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + kStages,
+                       kVFull = kKEmpty + kStages, kVEmpty = kVFull + kStages,
+                       kSBar = kVEmpty + kStages, kPBar = kSBar + 2, kOBar = kPBar + 2,
+                       kOFree = kOBar + 2, kDrain = kOFree + 2, kNumBars = kDrain + 1;
+  static constexpr uint32_t kTmemSlot = kBars + 8 * kNumBars;
+  static constexpr uint32_t kAbort = kTmemSlot + 4;
+  static constexpr uint32_t kBytes = kAbort + 4;
+  static constexpr uint32_t kAlloc = kBytes + 1024;  // base is rounded up to 1024
+  // TMEM columns
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+};
+
+struct Unit {
+  int b, hk, pair, qt, h0, h1valid;
+  int64_t list_row;
+  int n_full, n_part;
+};
+
+__device__ __forceinline__ Unit decode_unit(const AttnProblem& p, int u) {
+  Unit w;
+  const int per_qt = p.B * p.KVH * p.npairs;
+  w.qt = p.QT - 1 - u / per_qt;  // later query tiles first: they see the most keys
+  int r = u % per_qt;
+  w.pair = r % p.npairs;
+  r /= p.npairs;
+  w.hk = r % p.KVH;
+  w.b = r / p.KVH;
+  w.h0 = w.hk * p.group + 2 * w.pair;
+  w.h1valid = (2 * w.pair + 1) < p.group;
+  const int lb = p.lists.LB > 1 ? w.b : 0;
+  int lh = 0;
+  if (p.lists.head_mode == 1) lh = w.hk;
+  else if (p.lists.head_mode == 2) lh = w.hk * p.npairs + w.pair;
+  w.list_row = (static_cast<int64_t>(lb) * p.lists.LH + lh) * p.QT + w.qt;
+  w.n_full = p.lists.num_full[w.list_row];
+  w.n_part = p.lists.num_part[w.list_row];
+  return w;
+}
+
+__device__ __forceinline__ int tile_at(const AttnProblem& p, const Unit& w, int j, bool* partial) {
+  if (j < w.n_full) {
+    *partial = false;
+    return p.lists.full_idx[w.list_row * p.KT + j];
+  }
+  *partial = true;
+  return p.lists.part_idx[w.list_row * p.KT + (j - w.n_full)];
+}
+
+// Waits that ignore the abort flag (used only while draining after an abort).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* err) {
+  int never = 0;
+  volatile int* nv = &never;
+  mbar_wait(bar, parity, nv, err);
+}
+
+template <int D, int POLICY, int DT>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
+               const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+               int n_units) {
+  using L = Layout<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * static_cast<uint32_t>(i); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::kQFull), 1);
+    mbar_init(bar(L::kQEmpty), 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar(L::kKFull + s), 1);
+      mbar_init(bar(L::kKEmpty + s), 1);
+      mbar_init(bar(L::kVFull + s), 1);
+      mbar_init(bar(L::kVEmpty + s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(L::kSBar + i), 1);
+      mbar_init(bar(L::kPBar + i), 128);
+      mbar_init(bar(L::kOBar + i), 1);
+      mbar_init(bar(L::kOFree + i), 128);
+    }
+    mbar_init(bar(L::kDrain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+   if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_map(&map_q);
+      tma_prefetch_map(&map_k);
+      tma_prefetch_map(&map_v);
+      uint32_t kv_k = 0, kv_v = 0, q_it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(p, u);
+        const int n = w.n_full + w.n_part;
+        if (n == 0) continue;
+        if (q_it > 0 && !mbar_wait(bar(L::kQEmpty), (q_it - 1) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(L::kQFull), (1 + w.h1valid) * L::kTileBytes);
+        for (int i = 0; i < 1 + w.h1valid; ++i)
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_4d(sbase + L::kQ + i * L::kTileBytes + c * L::kChunkBytes, &map_q,
+                        bar(L::kQFull), c * 64, w.h0 + i, w.qt * kTile, w.b);
+        ++q_it;
+        for (int j = 0; j < n && ok; ++j) {
+          bool partial;
+          const int kt = tile_at(p, w, j, &partial);
+          const int stage = kv_k % L::kStages;
+          const uint32_t use = kv_k / L::kStages;
+          if (use > 0 && !mbar_wait(bar(L::kKEmpty + stage), (use - 1) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(L::kKFull + stage), L::kTileBytes);
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_4d(sbase + L::kK + stage * L::kTileBytes + c * L::kChunkBytes, &map_k,
+                        bar(L::kKFull + stage), c * 64, w.hk, kt * kTile, w.b);
+          ++kv_k;
+          if (use > 0 && !mbar_wait(bar(L::kVEmpty + stage), (use - 1) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(L::kVFull + stage), L::kTileBytes);
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_4d(sbase + L::kV + stage * L::kTileBytes + c * L::kChunkBytes, &map_v,
+                        bar(L::kVFull + stage), c * 64, w.hk, kt * kTile, w.b);
+          ++kv_v;
+        }
+      }
+      if (!ok) {
+        // Drain: every copy this thread issued must land before the CTA exits.
+        for (uint32_t t = 0; t < static_cast<uint32_t>(L::kStages); ++t) {
+          if (kv_k > t) {
+            const uint32_t nn = kv_k - 1 - t;
+            drain_wait(bar(L::kKFull + nn % L::kStages), (nn / L::kStages) & 1, p.err);
+          }
+          if (kv_v > t) {
+            const uint32_t nn = kv_v - 1 - t;
+            drain_wait(bar(L::kVFull + nn % L::kStages), (nn / L::kStages) & 1, p.err);
+          }
+        }
+        if (q_it > 0) drain_wait(bar(L::kQFull), (q_it - 1) & 1, p.err);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t fmt = DT == SMA_BF16 ? 1u : 0u;
+      constexpr uint32_t idesc_qk = mma_idesc_f16(fmt, 128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = mma_idesc_f16(fmt, 128, D, 0, 1);
+      uint32_t kv_it = 0, q_it = 0;
+      uint32_t pv_it[2] = {0, 0}, units[2] = {0, 0};
+      bool ok = true;
+      // Descriptors are built once per operand tile; a k-step only moves the
+      // start-address field (bits 0-13, in 16-byte units).
+      auto issue_qk = [&](int i, int stage) {
+        const uint64_t qd = smem_desc_sw128(sbase + L::kQ + i * L::kTileBytes, 16, 1024);
+        const uint64_t kd = smem_desc_sw128(sbase + L::kK + stage * L::kTileBytes, 16, 1024);
+        const uint32_t d_col = tmem + (i == 0 ? L::kColS0 : L::kColS1);
+#pragma unroll 1
+        for (int s = 0; s < D / 16; ++s) {
+          const uint64_t off = ((s >> 2) * L::kChunkBytes + (s & 3) * 32) >> 4;
+          tc_mma_ss(d_col, qd + off, kd + off, idesc_qk, s > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int i, int stage, bool first) {
+        const uint64_t vd =
+            smem_desc_sw128(sbase + L::kV + stage * L::kTileBytes, L::kChunkBytes, 1024);
+        const uint32_t d_col = tmem + (i == 0 ? L::kColO0 : L::kColO1);
+        const uint32_t p_col = tmem + (i == 0 ? L::kColS0 : L::kColS1);
+#pragma unroll 1
+        for (int s = 0; s < kTile / 16; ++s) {
+          tc_mma_ts(d_col, p_col + 8 * s, vd + static_cast<uint64_t>(s * 2048 >> 4), idesc_pv,
+                    (first && s == 0) ? 0u : 1u);
+        }
+      };
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(p, u);
+        const int n = w.n_full + w.n_part;
+        const int nq = 1 + w.h1valid;
+        if (n > 0) {
+          if (!mbar_wait(bar(L::kQFull), q_it & 1, abort_flag, p.err)) { ok = false; break; }
+          ++q_it;
+          // S_i(0) = Q_i K(0)^T
+          {
+            const int stage = kv_it % L::kStages;
+            if (!mbar_wait(bar(L::kKFull + stage), (kv_it / L::kStages) & 1, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            for (int i = 0; i < nq && ok; ++i) {
+              if (pv_it[i] > 0 &&
+                  !mbar_wait(bar(L::kOBar + i), (pv_it[i] - 1) & 1, abort_flag, p.err)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              issue_qk(i, stage);
+              tc_commit(bar(L::kSBar + i));
+            }
+            if (!ok) break;
+            tc_commit(bar(L::kKEmpty + stage));
+            if (n == 1) tc_commit(bar(L::kQEmpty));
+          }
+          for (int j = 0; j < n && ok; ++j) {
+            const int stage = kv_it % L::kStages;
+            const uint32_t ph = (kv_it / L::kStages) & 1;
+            const int nstage = (kv_it + 1) % L::kStages;
+            const uint32_t nph = ((kv_it + 1) / L::kStages) & 1;
+            if (!mbar_wait(bar(L::kVFull + stage), ph, abort_flag, p.err)) { ok = false; break; }
+            if (j + 1 < n &&
+                !mbar_wait(bar(L::kKFull + nstage), nph, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            for (int i = 0; i < nq && ok; ++i) {
+              // O_i += P_i(j) V(j)
+              if (!mbar_wait(bar(L::kPBar + i), pv_it[i] & 1, abort_flag, p.err)) { ok = false; break; }
+              if (j == 0 && units[i] > 0 &&
+                  !mbar_wait(bar(L::kOFree + i), (units[i] - 1) & 1, abort_flag, p.err)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              issue_pv(i, stage, j == 0);
+              tc_commit(bar(L::kOBar + i));
+              ++pv_it[i];
+              // S_i(j+1) = Q_i K(j+1)^T once P_i(j) has been consumed
+              if (j + 1 < n) {
+                if (!mbar_wait(bar(L::kOBar + i), (pv_it[i] - 1) & 1, abort_flag, p.err)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+                issue_qk(i, nstage);
+                tc_commit(bar(L::kSBar + i));
+              }
+            }
+            if (!ok) break;
+            tc_commit(bar(L::kVEmpty + stage));
+            if (j + 1 < n) {
+              tc_commit(bar(L::kKEmpty + nstage));
+              if (j + 2 == n) tc_commit(bar(L::kQEmpty));
+            }
+            ++kv_it;
+          }
+        }
+        units[0] += 1;
+        units[1] += w.h1valid;
+      }
+      if (!ok) {
+        tc_commit(bar(L::kDrain));
+        drain_wait(bar(L::kDrain), 0, p.err);
+      }
+    }
+   }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    // ------------------------------------------------------------ softmax
+    const int qi = warp >> 2;        // which query tile of the unit
+    const int quad = warp & 3;       // TMEM lane quadrant
+    const int r = quad * 32 + lane;  // row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t s_col = tmem + lane_off + (qi == 0 ? L::kColS0 : L::kColS1);
+    const uint32_t o_col = tmem + lane_off + (qi == 0 ? L::kColO0 : L::kColO1);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit w = decode_unit(p, u);
+      if (qi == 1 && !w.h1valid) continue;
+      const int h = w.h0 + qi;
+      const int q = w.qt * kTile + r;
+      const bool row_valid = q < p.Lq;
+      const int n = w.n_full + w.n_part;
+
+      // Per-row mask parameters.
+      int clo = 0, chi = 0, dlo = 0, dhi = 0;  // DFlash keep intervals
+      const uint8_t* mrow = nullptr;
+      const uint8_t* brow = nullptr;
+      int causal_lim = 0x7fffffff;
+      if (POLICY == kPolicyDflash) {
+        if (row_valid) {
+          const int j = q / p.bs, i = q - j * p.bs;
+          int a = p.anchors[static_cast<int64_t>(w.b) * p.N + j];
+          a = a < 0 ? 0 : (a > p.Lc ? p.Lc : a);
+          chi = a;
+          clo = p.window > 0 ? max(0, a + i - p.window + 1) : 0;
+          if (clo > chi) clo = chi;
+          const int base = p.Lc + j * p.bs;
+          dlo = base + (p.window > 0 ? max(0, i - p.window + 1) : 0);
+          dhi = base + (p.causal_in_block ? i + 1 : p.bs);
+        }
+      } else {
+        const int qq = row_valid ? q : 0;
+        if (p.has_mask) {
+          const int hm = p.mask.head_per_query ? h : w.hk;
+          mrow = reinterpret_cast<const uint8_t*>(p.mask.ptr) + w.b * p.mask.sb + hm * p.mask.sh +
+                 static_cast<int64_t>(qq) * p.mask.sq;
+        }
+        if (p.has_bias) {
+          const int hb = p.bias.head_per_query ? h : w.hk;
+          const int esz = p.bias.dtype == SMA_FP32 ? 4 : 2;
+          brow = reinterpret_cast<const uint8_t*>(p.bias.ptr) +
+                 (w.b * p.bias.sb + hb * p.bias.sh + static_cast<int64_t>(qq) * p.bias.sq) * esz;
+        }
+        if (p.causal) causal_lim = q + p.Lk - p.Lq;
+      }
+
+      float m_ref = -INFINITY, l_sum = 0.f;
+      for (int j = 0; j < n && ok; ++j) {
+        bool partial;
+        const int kt = tile_at(p, w, j, &partial);
+        const int k0 = kt * kTile;
+        if (!mbar_wait(bar(L::kSBar + qi), it & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        float x[kTile];
+#pragma unroll
+        for (int c = 0; c < kTile / 32; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(s_col + 32 * c, raw);
+          tc_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[32 * c + e] = __uint_as_float(raw[e]) * p.scale_log2;
+        }
+        if (POLICY == kPolicyExplicit && p.has_bias) {
+          if (p.bias.dtype == SMA_FP32) {
+#pragma unroll
+            for (int c = 0; c < kTile; c += 4) {
+              const float4 a = *reinterpret_cast<const float4*>(brow + (k0 + c) * 4);
+              x[c] = fmaf(a.x, kLog2e, x[c]);
+              x[c + 1] = fmaf(a.y, kLog2e, x[c + 1]);
+              x[c + 2] = fmaf(a.z, kLog2e, x[c + 2]);
+              x[c + 3] = fmaf(a.w, kLog2e, x[c + 3]);
+            }
+          } else if (p.bias.dtype == SMA_BF16) {
+#pragma unroll
+            for (int c = 0; c < kTile; c += 8) {
+              const uint4 a = *reinterpret_cast<const uint4*>(brow + (k0 + c) * 2);
+              const uint32_t wv[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                x[c + 2 * e] = fmaf(__uint_as_float(wv[e] << 16), kLog2e, x[c + 2 * e]);
+                x[c + 2 * e + 1] = fmaf(__uint_as_float(wv[e] & 0xffff0000u), kLog2e, x[c + 2 * e + 1]);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < kTile; c += 8) {
+              const uint4 a = *reinterpret_cast<const uint4*>(brow + (k0 + c) * 2);
+              const uint32_t wv[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[e]));
+                x[c + 2 * e] = fmaf(f.x, kLog2e, x[c + 2 * e]);
+                x[c + 2 * e + 1] = fmaf(f.y, kLog2e, x[c + 2 * e + 1]);
+              }
+            }
+          }
+        }
+        if (partial || !row_valid) {
+          if (POLICY == kPolicyDflash) {
+            const uint32_t wc = static_cast<uint32_t>(chi - clo);
+            const uint32_t wd = static_cast<uint32_t>(dhi - dlo);
+            const int ac = k0 - clo, ad = k0 - dlo;
+#pragma unroll
+            for (int c = 0; c < kTile; ++c) {
+              const bool keep = static_cast<uint32_t>(c + ac) < wc ||
+                                static_cast<uint32_t>(c + ad) < wd;
+              x[c] = (keep && row_valid) ? x[c] : -INFINITY;
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < kTile; c += 16) {
+              uint4 mv = make_uint4(0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u);
+              if (p.has_mask) mv = *reinterpret_cast<const uint4*>(mrow + k0 + c);
+              const uint32_t wv[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int k = k0 + c + e;
+                const bool keep = ((wv[e >> 2] >> (8 * (e & 3))) & 0xffu) != 0u && k < p.Lk &&
+                                  k <= causal_lim && row_valid;
+                x[c + e] = keep ? x[c + e] : -INFINITY;
+              }
+            }
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, x[c]);
+        const float m_new = fmaxf(m_ref, mx);
+        // Lazy rescale of O: only when the max grew by more than 2^8.
+        const bool need = (m_ref != -INFINITY) && (m_new > m_ref + 8.0f);
+        if (__any_sync(0xffffffffu, need)) {
+          if (!mbar_wait(bar(L::kOBar + qi), (it - 1) & 1, abort_flag, p.err)) { ok = false; }
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          tc_fence_after();
+          const float alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(o_col + 32 * c, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(o_col + 32 * c, o);
+          }
+          tc_wait_st();
+          if (need) {
+            l_sum *= alpha;
+            m_ref = m_new;
+          }
+        }
+        if (m_ref == -INFINITY) m_ref = m_new;
+        const float msub = m_ref == -INFINITY ? 0.f : m_ref;
+        float ls = 0.f;
+#pragma unroll
+        for (int c = 0; c < kTile / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = fast_exp2(x[32 * c + 2 * e] - msub);
+            const float p1 = fast_exp2(x[32 * c + 2 * e + 1] - msub);
+            ls += p0 + p1;
+            pk[e] = DT == SMA_BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+          }
+          // P columns [16c, 16c+16) of the packed pairs
+          asm volatile(
+              "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+              "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(
+                  s_col + 16 * c),
+              "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]),
+              "r"(pk[6]), "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]),
+              "r"(pk[12]), "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
+              : "memory");
+        }
+        l_sum += ls;
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::kPBar + qi));
+        ++it;
+      }
+      if (!ok) break;
+
+      // Epilogue: O / l, lse.
+      typedef typename std::conditional<DT == SMA_BF16, __nv_bfloat16, __half>::type OutT;
+      OutT* orow = reinterpret_cast<OutT*>(p.o) + w.b * p.o_sb + static_cast<int64_t>(q) * p.o_sr +
+                   h * p.o_sh;
+      const float inv_l = l_sum > 0.f ? 1.0f / l_sum : 0.f;
+      if (n > 0) {
+        if (!mbar_wait(bar(L::kOBar + qi), (it - 1) & 1, abort_flag, p.err)) ok = false;
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_col + 32 * c, o);
+          tc_wait_ld();
+          if (row_valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float a = __uint_as_float(o[2 * e]) * inv_l;
+              const float bq = __uint_as_float(o[2 * e + 1]) * inv_l;
+              pk[e] = DT == SMA_BF16 ? pack_bf16x2(a, bq) : pack_f16x2(a, bq);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
+        }
+      } else if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(orow);
+        for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
+      }
+      if (row_valid && p.lse != nullptr) {
+        p.lse[(static_cast<int64_t>(w.b) * p.H + h) * p.Lq + q] =
+            l_sum > 0.f ? (m_ref + __log2f(l_sum)) * kLn2 : -INFINITY;
+      }
+      tc_fence_before();
+      mbar_arrive(bar(L::kOFree + qi));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// 4D map over [B][len][heads][d] (d contiguous), box = 64 x 1 x 128 x 1,
+// 128-byte swizzle, zero fill outside the tensor.
+bool encode_map(CUtensorMap* map, const void* ptr, int dtype, int d, int heads, int len, int batch,
+                int64_t s_head, int64_t s_row, int64_t s_batch, char* msg, size_t msg_len) {
+  auto enc = get_encode_fn();
+  if (enc == nullptr) {
+    snprintf(msg, msg_len, "cuTensorMapEncodeTiled is unavailable");
+    return false;
+  }
+  const int esz = 2;
+  // A size-1 dim's stride is never used; give it a legal value.
+  if (heads == 1) s_head = d;
+  if (len == 1) s_row = s_head * heads;
+  if (batch == 1) s_batch = s_row * len;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(len), static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(s_head * esz),
+                           static_cast<cuuint64_t>(s_row * esz),
+                           static_cast<cuuint64_t>(s_batch * esz)};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kTile), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, dtype == SMA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   4, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(msg, msg_len, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return false;
+  }
+  return true;
+}
+
+template <int D, int POLICY, int DT>
+cudaError_t launch_typed(const AttnProblem& p, const CUtensorMap& mq, const CUtensorMap& mk,
+                         const CUtensorMap& mv, cudaStream_t stream) {
+  using L = Layout<D>;
+  auto kern = attn_tc_kernel<D, POLICY, DT>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    // The setmaxnreg split assumes exactly kLaunchRegs registers per thread.
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(L::kAlloc));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int n_units = p.B * p.KVH * p.npairs * p.QT;
+  if (n_units == 0) return cudaSuccess;
+  const int grid = n_units < num_sms() ? n_units : num_sms();
+  kern<<<grid, kThreads, L::kAlloc, stream>>>(p, mq, mk, mv, n_units);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int launch_attn_tc(const AttnProblem& p, cudaStream_t stream, char* msg, size_t msg_len) {
+  CUtensorMap mq, mk, mv;
+  if (!encode_map(&mq, p.q, p.dtype, p.d, p.H, p.Lq, p.B, p.q_sh, p.q_sr, p.q_sb, msg, msg_len) ||
+      !encode_map(&mk, p.k, p.dtype, p.d, p.KVH, p.Lk, p.B, p.k_sh, p.k_sr, p.k_sb, msg, msg_len) ||
+      !encode_map(&mv, p.v, p.dtype, p.d, p.KVH, p.Lk, p.B, p.v_sh, p.v_sr, p.v_sb, msg, msg_len))
+    return SMA_ERR_CUDA;
+  cudaError_t e = cudaErrorInvalidValue;
+  const bool bf = p.dtype == SMA_BF16;
+  if (p.policy == kPolicyDflash) {
+    if (p.d == 128) e = bf ? launch_typed<128, kPolicyDflash, SMA_BF16>(p, mq, mk, mv, stream)
+                           : launch_typed<128, kPolicyDflash, SMA_FP16>(p, mq, mk, mv, stream);
+    else e = bf ? launch_typed<64, kPolicyDflash, SMA_BF16>(p, mq, mk, mv, stream)
+                : launch_typed<64, kPolicyDflash, SMA_FP16>(p, mq, mk, mv, stream);
+  } else {
+    if (p.d == 128) e = bf ? launch_typed<128, kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, stream)
+                           : launch_typed<128, kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, stream);
+    else e = bf ? launch_typed<64, kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, stream)
+                : launch_typed<64, kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, stream);
+  }
+  if (e != cudaSuccess) {
+    snprintf(msg, msg_len, "attention launch failed: %s", cudaGetErrorString(e));
+    return SMA_ERR_CUDA;
+  }
+  return SMA_OK;
+}
+
+}  // namespace sma

@@ -1,0 +1,129 @@
+// Internal (non-ABI) description of the problems the kernels solve, and the
+// host-side launchers the C ABI calls.  Plain C++ structs; no torch types.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sma {
+
+constexpr int kTile = 128;
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up(int64_t a, int64_t m) { return ceil_div(a, m) * m; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// DFlash mask geometry after is_causal / window resolution.
+struct DflashGeom {
+  int B, N, bs, Lc;  // batch, blocks, block size, context keys
+  int Nq, Lk;        // queries, keys
+  int QT, KT;        // 128-tiles of queries / keys
+  int causal;        // 1: causal inside the block
+  int window;        // left window W, 0 = none
+};
+
+// Mask or bias operand after stride-0 folding of its size-1 dims.
+struct AuxView {
+  const void* ptr = nullptr;
+  int dtype = 0;        // bias dtype (SMA_BF16/FP16/FP32); unused for masks
+  int64_t sb = 0, sh = 0, sq = 0;  // element strides, 0 for broadcast dims
+  int head_per_query = 0;          // 1: head index is the query head, 0: the KV head
+  int64_t sizes[4] = {0, 0, 0, 0};
+};
+
+// Ascending key-tile lists; list row = (lb * LH + lh) * QT + qt.
+struct TileLists {
+  const int32_t* num_full = nullptr;
+  const int32_t* full_idx = nullptr;
+  const int32_t* num_part = nullptr;
+  const int32_t* part_idx = nullptr;
+  int LB = 1;         // batch rows (1 = shared by every batch entry)
+  int LH = 1;         // head rows
+  int head_mode = 0;  // 0: lh = 0; 1: lh = kv head; 2: lh = kv head * npairs + pair
+};
+
+enum MaskPolicy { kPolicyDflash = 0, kPolicyExplicit = 1 };
+
+// One attention forward problem: O[b, q, h] over keys of head h / group.
+struct AttnProblem {
+  int dtype;  // SMA_BF16 / SMA_FP16 / SMA_FP32 (q, k, v, out)
+  int B, H, KVH, Lq, Lk, d;
+  int group, npairs, QT, KT;
+  float scale_log2;  // scale * log2(e)
+  const void* q; int64_t q_sb, q_sr, q_sh;
+  const void* k; int64_t k_sb, k_sr, k_sh;
+  const void* v; int64_t v_sb, v_sr, v_sh;
+  void* o; int64_t o_sb, o_sr, o_sh;
+  float* lse;  // [B, H, Lq] contiguous or null
+  TileLists lists;
+  int policy;
+  // DFlash policy
+  const int32_t* anchors; int N, bs, Lc, causal_in_block, window;
+  // explicit policy
+  int causal;
+  int has_mask, has_bias;
+  AuxView mask, bias;
+  int* err;  // device error word
+};
+
+// Single-query (decode) problem after the grouped-head swap: for each
+// (b, kv head) the `group` query heads are the rows.
+struct DecodeProblem {
+  int dtype;
+  int B, H, KVH, Lk, d, group;
+  float scale_log2;
+  const void* q; int64_t q_sb, q_sh;
+  const void* k; int64_t k_sb, k_sr, k_sh;
+  const void* v; int64_t v_sb, v_sr, v_sh;
+  void* o; int64_t o_sb, o_sh;
+  float* lse;  // [B, H] (q_len 1) or null
+  int has_mask, has_bias;
+  AuxView mask, bias;
+  int splits, chunk;       // split-KV: keys [s*chunk, min((s+1)*chunk, Lk))
+  float* part_o;           // [B, H, splits, d]
+  float* part_ml;          // [B, H, splits, 2]  (max in log2 units, sum)
+  int* err;
+};
+
+struct TopkProblem {
+  int bias_dtype;
+  const void* bias; int64_t b_sizes[4]; int64_t b_strides[4];
+  int Lk, Kpad;
+  const uint8_t* pre; int64_t p_sizes[4]; int64_t p_strides[4];  // strides 0 on broadcast dims
+  int window;
+  uint8_t* out;
+};
+
+// ---- launchers (return cudaSuccess or the launch error)
+cudaError_t launch_dfa_block_map(const DflashGeom& g, const int32_t* anchors, int32_t* num_full,
+                                 int32_t* full_idx, int32_t* num_part, int32_t* part_idx, int* err,
+                                 cudaStream_t stream);
+
+cudaError_t launch_mask_tile_summary(const uint8_t* mask, const int64_t sizes[4],
+                                     const int64_t strides[4], int Lk, uint8_t* codes,
+                                     cudaStream_t stream);
+
+// Tile lists of the explicit-mask path from the summary codes (may be null),
+// causal flag and key length.  Writes LB*LH*QT lists.
+cudaError_t launch_explicit_lists(const AttnProblem& p, const uint8_t* codes, int codes_q_tiles,
+                                  int32_t* num_full, int32_t* full_idx, int32_t* num_part,
+                                  int32_t* part_idx, cudaStream_t stream);
+
+// tcgen05 forward (bf16 / fp16).  Returns a nonzero SMA status on a host-side
+// failure (tensor map encoding) and writes a message to `msg`.
+int launch_attn_tc(const AttnProblem& p, cudaStream_t stream, char* msg, size_t msg_len);
+
+// fp32 FFMA forward.
+cudaError_t launch_attn_simt(const AttnProblem& p, cudaStream_t stream);
+
+cudaError_t launch_decode(const DecodeProblem& p, cudaStream_t stream);
+
+cudaError_t launch_topk(const TopkProblem& p, cudaStream_t stream);
+
+// Device error word of the current device.
+int* device_error_word(cudaError_t* status);
+
+int num_sms();
+
+}  // namespace sma

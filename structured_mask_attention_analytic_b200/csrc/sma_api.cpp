@@ -1,0 +1,557 @@
+// C ABI of libsma (declared in include/sma.h): argument validation, stride-0
+// folding of broadcast dims, workspace layout and stream-ordered launches.
+// Nothing here allocates device memory or synchronises the stream (except
+// sma_device_status, whose job is to synchronise).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "kernels.h"
+#include "sma.h"
+
+using namespace sma;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+sma_status fail(sma_status code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+sma_status ok() {
+  g_last_error.clear();
+  return SMA_OK;
+}
+
+sma_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SMA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int elem_size(int32_t dtype) { return dtype == SMA_FP32 ? 4 : 2; }
+
+bool valid_dtype(int32_t dt) { return dt == SMA_BF16 || dt == SMA_FP16 || dt == SMA_FP32; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+float resolve_scale(float scale, int d) {
+  return scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
+}
+
+constexpr float kLog2eHost = 1.4426950408889634f;
+
+// Q/K/V/O operand: [batch, len, heads, d], d contiguous.
+sma_status check_operand(const char* name, const void* ptr, const int64_t* strides, int32_t dtype,
+                         int64_t len) {
+  if (ptr == nullptr) return fail(SMA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (strides == nullptr) return fail(SMA_ERR_INVALID_ARG, "%s strides are NULL", name);
+  if (!aligned16(ptr)) return fail(SMA_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);
+  const int es = elem_size(dtype);
+  for (int i = 0; i < 3; ++i) {
+    if (strides[i] < 0) return fail(SMA_ERR_INVALID_ARG, "%s stride %d is negative", name, i);
+    if ((strides[i] * es) % 16 != 0)
+      return fail(SMA_ERR_INVALID_ARG, "%s stride %d (%lld elements) is not a multiple of 16 bytes",
+                  name, i, static_cast<long long>(strides[i]));
+  }
+  (void)len;
+  return SMA_OK;
+}
+
+sma_status check_heads(int32_t heads, int32_t kv_heads, int32_t head_dim) {
+  if (heads < 1 || kv_heads < 1) return fail(SMA_ERR_INVALID_ARG, "heads and kv_heads must be >= 1");
+  if (heads % kv_heads != 0)
+    return fail(SMA_ERR_INVALID_ARG, "heads (%d) must be a multiple of kv_heads (%d)", heads, kv_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(SMA_ERR_UNSUPPORTED, "head_dim %d is not supported (64 or 128)", head_dim);
+  return SMA_OK;
+}
+
+// Mask/bias operand of the 4D broadcast contract; fills `view`.
+sma_status check_aux(const char* name, const void* ptr, const int64_t* sizes,
+                     const int64_t* strides, int esz, int32_t B, int32_t H, int32_t KVH,
+                     int32_t Lq, int32_t Lk, bool need_full_k, AuxView* view) {
+  if (sizes == nullptr || strides == nullptr)
+    return fail(SMA_ERR_INVALID_ARG, "%s sizes/strides are NULL", name);
+  const int64_t kpad = round_up(Lk, kTile);
+  if (sizes[0] != B && sizes[0] != 1)
+    return fail(SMA_ERR_INVALID_ARG, "%s batch dim %lld must be %d or 1", name,
+                static_cast<long long>(sizes[0]), B);
+  if (sizes[1] != H && sizes[1] != KVH && sizes[1] != 1)
+    return fail(SMA_ERR_INVALID_ARG, "%s head dim %lld must be %d, %d or 1", name,
+                static_cast<long long>(sizes[1]), H, KVH);
+  if (sizes[2] != Lq && sizes[2] != 1)
+    return fail(SMA_ERR_INVALID_ARG, "%s query dim %lld must be %d or 1", name,
+                static_cast<long long>(sizes[2]), Lq);
+  if (need_full_k && sizes[3] != kpad)
+    return fail(SMA_ERR_INVALID_ARG, "%s key dim %lld must be round_up(k_len, 128) = %lld", name,
+                static_cast<long long>(sizes[3]), static_cast<long long>(kpad));
+  if (strides[3] != 1) return fail(SMA_ERR_INVALID_ARG, "%s last dim must be contiguous", name);
+  if (!aligned16(ptr)) return fail(SMA_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);
+  view->ptr = ptr;
+  view->sb = sizes[0] == 1 ? 0 : strides[0];
+  view->sh = sizes[1] == 1 ? 0 : strides[1];
+  view->sq = sizes[2] == 1 ? 0 : strides[2];
+  for (int64_t s : {view->sb, view->sh, view->sq}) {
+    if (s < 0) return fail(SMA_ERR_INVALID_ARG, "%s has a negative stride", name);
+    if ((s * esz) % 16 != 0)
+      return fail(SMA_ERR_INVALID_ARG, "%s strides must be multiples of 16 bytes", name);
+  }
+  view->head_per_query = sizes[1] == H ? 1 : 0;
+  for (int i = 0; i < 4; ++i) view->sizes[i] = sizes[i];
+  return SMA_OK;
+}
+
+sma_status check_desc(const dfa_mask_desc* d) {
+  if (d == nullptr) return fail(SMA_ERR_INVALID_ARG, "desc is NULL");
+  if (d->batch < 1 || d->n_blocks < 1 || d->block_size < 1 || d->ctx_len < 0)
+    return fail(SMA_ERR_INVALID_ARG, "batch, n_blocks, block_size must be >= 1 and ctx_len >= 0");
+  if (d->is_causal != SMA_IS_CAUSAL_UNSET && d->is_causal != 0 && d->is_causal != 1)
+    return fail(SMA_ERR_INVALID_ARG, "is_causal must be -1, 0 or 1");
+  if (d->layer_type != SMA_LAYER_FULL && d->layer_type != SMA_LAYER_SLIDING)
+    return fail(SMA_ERR_INVALID_ARG, "layer_type must be 0 (full) or 1 (sliding)");
+  if (d->layer_type == SMA_LAYER_SLIDING && d->sliding_window < 1)
+    return fail(SMA_ERR_INVALID_ARG, "sliding layers need sliding_window >= 1");
+  const int64_t nq = static_cast<int64_t>(d->n_blocks) * d->block_size;
+  if (nq + d->ctx_len > (1LL << 30)) return fail(SMA_ERR_INVALID_ARG, "key length too large");
+  return SMA_OK;
+}
+
+DflashGeom make_geom(const dfa_mask_desc* d) {
+  DflashGeom g;
+  g.B = d->batch;
+  g.N = d->n_blocks;
+  g.bs = d->block_size;
+  g.Lc = d->ctx_len;
+  g.Nq = d->n_blocks * d->block_size;
+  g.Lk = g.Lc + g.Nq;
+  g.QT = static_cast<int>(ceil_div(g.Nq, kTile));
+  g.KT = static_cast<int>(ceil_div(g.Lk, kTile));
+  // SpecForge PR #905, Motivation list.
+  if (d->is_causal == SMA_IS_CAUSAL_UNSET) g.causal = d->layer_type == SMA_LAYER_SLIDING ? 1 : 0;
+  else g.causal = d->is_causal;
+  g.window = d->layer_type == SMA_LAYER_SLIDING ? d->sliding_window : 0;
+  return g;
+}
+
+struct ListsLayout {
+  size_t nf, np, fi, pi, end;
+};
+
+ListsLayout lists_layout(size_t base, int64_t rows, int KT) {
+  ListsLayout l;
+  l.nf = base;
+  l.np = align256(l.nf + rows * 4);
+  l.fi = align256(l.np + rows * 4);
+  l.pi = align256(l.fi + rows * KT * 4);
+  l.end = align256(l.pi + rows * KT * 4);
+  return l;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+sma_status check_workspace(void* ws, size_t have, size_t need) {
+  if (have < need)
+    return fail(SMA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", have,
+                need);
+  if (need > 0 && ws == nullptr) return fail(SMA_ERR_INVALID_ARG, "workspace is NULL");
+  if (need > 0 && (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(SMA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  return SMA_OK;
+}
+
+// ---- masked path geometry
+struct MaskedGeom {
+  int LB, LH, head_mode, npairs, QT, KT, codes_qt;
+  bool decode;
+  int splits, chunk;
+  size_t codes_bytes;
+  ListsLayout lists;
+  size_t part_o, part_ml, total;
+};
+
+MaskedGeom masked_geom(int32_t B, int32_t H, int32_t KVH, int32_t Lq, int32_t Lk, int32_t d,
+                       const int64_t* mask_sizes) {
+  MaskedGeom g{};
+  const int group = H / KVH;
+  g.npairs = (group + 1) / 2;
+  g.QT = static_cast<int>(ceil_div(Lq, kTile));
+  g.KT = static_cast<int>(ceil_div(Lk, kTile));
+  g.decode = Lq == 1;
+  if (g.decode) {
+    // split-KV: about two CTAs per SM of a 148-SM part, chunks of >= 256 keys
+    const int rows_groups = (group + 7) / 8;
+    const int64_t base_ctas = static_cast<int64_t>(B) * KVH * rows_groups;
+    int splits = static_cast<int>(ceil_div(296, base_ctas));
+    const int max_splits = static_cast<int>(ceil_div(Lk, 256));
+    if (splits > max_splits) splits = max_splits;
+    if (splits > 64) splits = 64;
+    if (splits < 1) splits = 1;
+    g.splits = splits;
+    g.chunk = static_cast<int>(ceil_div(Lk, splits));
+    g.part_o = 0;
+    g.part_ml = align256(static_cast<size_t>(B) * H * splits * d * 4);
+    g.total = align256(g.part_ml + static_cast<size_t>(B) * H * splits * 2 * 4);
+    return g;
+  }
+  const bool has_mask = mask_sizes != nullptr;
+  g.LB = (has_mask && mask_sizes[0] > 1) ? B : 1;
+  if (!has_mask || mask_sizes[1] == 1) {
+    g.head_mode = 0;
+    g.LH = 1;
+  } else if (mask_sizes[1] == H) {
+    g.head_mode = 2;
+    g.LH = KVH * g.npairs;
+  } else {
+    g.head_mode = 1;
+    g.LH = KVH;
+  }
+  g.codes_qt = has_mask ? static_cast<int>(ceil_div(mask_sizes[2], kTile)) : 0;
+  g.codes_bytes =
+      has_mask ? align256(static_cast<size_t>(mask_sizes[0] * mask_sizes[1]) * g.codes_qt * g.KT) : 0;
+  g.lists = lists_layout(g.codes_bytes, static_cast<int64_t>(g.LB) * g.LH * g.QT, g.KT);
+  g.total = g.lists.end;
+  return g;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sma_last_error(void) { return g_last_error.c_str(); }
+
+int32_t sma_abi_version(void) { return 1; }
+
+sma_status sma_device_status(void* stream, int32_t* device_error) {
+  if (device_error == nullptr) return fail(SMA_ERR_INVALID_ARG, "device_error is NULL");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronisation failed");
+  int* word = device_error_word(&e);
+  if (word == nullptr) return cuda_fail(e, "device error word unavailable");
+  int v = 0;
+  e = cudaMemcpy(&v, word, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word failed");
+  const int zero = 0;
+  e = cudaMemcpy(word, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word failed");
+  *device_error = v;
+  return ok();
+}
+
+sma_status dfa_block_map_dims(const dfa_mask_desc* desc, int32_t* q_tiles, int32_t* kv_tiles) {
+  sma_status s = check_desc(desc);
+  if (s != SMA_OK) return s;
+  if (q_tiles == nullptr || kv_tiles == nullptr)
+    return fail(SMA_ERR_INVALID_ARG, "output pointers are NULL");
+  const DflashGeom g = make_geom(desc);
+  *q_tiles = g.QT;
+  *kv_tiles = g.KT;
+  return ok();
+}
+
+sma_status dfa_block_map(const dfa_mask_desc* desc, const int32_t* anchors, int32_t* num_full,
+                         int32_t* full_idx, int32_t* num_part, int32_t* part_idx, void* stream) {
+  sma_status s = check_desc(desc);
+  if (s != SMA_OK) return s;
+  if (!anchors || !num_full || !full_idx || !num_part || !part_idx)
+    return fail(SMA_ERR_INVALID_ARG, "a device pointer is NULL");
+  const DflashGeom g = make_geom(desc);
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (err == nullptr) return cuda_fail(e, "device error word unavailable");
+  e = launch_dfa_block_map(g, anchors, num_full, full_idx, num_part, part_idx, err,
+                           static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "block map launch failed");
+  return ok();
+}
+
+sma_status dfa_attn_fwd_workspace_size(const dfa_mask_desc* desc, int32_t heads, int32_t kv_heads,
+                                       int32_t head_dim, size_t* bytes) {
+  sma_status s = check_desc(desc);
+  if (s != SMA_OK) return s;
+  s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (bytes == nullptr) return fail(SMA_ERR_INVALID_ARG, "bytes is NULL");
+  const DflashGeom g = make_geom(desc);
+  *bytes = lists_layout(0, static_cast<int64_t>(g.B) * g.QT, g.KT).end;
+  return ok();
+}
+
+sma_status dfa_attn_fwd(const dfa_mask_desc* desc, const int32_t* anchors, int32_t dtype,
+                        int32_t heads, int32_t kv_heads, int32_t head_dim, float scale,
+                        const void* q, const int64_t q_strides[3], const void* k,
+                        const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
+                        void* out, const int64_t o_strides[3], float* lse, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  sma_status s = check_desc(desc);
+  if (s != SMA_OK) return s;
+  if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (anchors == nullptr) return fail(SMA_ERR_INVALID_ARG, "anchors is NULL");
+  const DflashGeom g = make_geom(desc);
+  if ((s = check_operand("q", q, q_strides, dtype, g.Nq)) != SMA_OK) return s;
+  if ((s = check_operand("k", k, k_strides, dtype, g.Lk)) != SMA_OK) return s;
+  if ((s = check_operand("v", v, v_strides, dtype, g.Lk)) != SMA_OK) return s;
+  if ((s = check_operand("out", out, o_strides, dtype, g.Nq)) != SMA_OK) return s;
+  const ListsLayout lay = lists_layout(0, static_cast<int64_t>(g.B) * g.QT, g.KT);
+  if ((s = check_workspace(workspace, workspace_bytes, lay.end)) != SMA_OK) return s;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (err == nullptr) return cuda_fail(e, "device error word unavailable");
+  int32_t* nf = at<int32_t>(workspace, lay.nf);
+  int32_t* np = at<int32_t>(workspace, lay.np);
+  int32_t* fi = at<int32_t>(workspace, lay.fi);
+  int32_t* pi = at<int32_t>(workspace, lay.pi);
+  e = launch_dfa_block_map(g, anchors, nf, fi, np, pi, err, st);
+  if (e != cudaSuccess) return cuda_fail(e, "block map launch failed");
+
+  AttnProblem p{};
+  p.dtype = dtype;
+  p.B = g.B; p.H = heads; p.KVH = kv_heads; p.Lq = g.Nq; p.Lk = g.Lk; p.d = head_dim;
+  p.group = heads / kv_heads;
+  p.npairs = (p.group + 1) / 2;
+  p.QT = g.QT; p.KT = g.KT;
+  p.scale_log2 = resolve_scale(scale, head_dim) * kLog2eHost;
+  p.q = q; p.q_sb = q_strides[0]; p.q_sr = q_strides[1]; p.q_sh = q_strides[2];
+  p.k = k; p.k_sb = k_strides[0]; p.k_sr = k_strides[1]; p.k_sh = k_strides[2];
+  p.v = v; p.v_sb = v_strides[0]; p.v_sr = v_strides[1]; p.v_sh = v_strides[2];
+  p.o = out; p.o_sb = o_strides[0]; p.o_sr = o_strides[1]; p.o_sh = o_strides[2];
+  p.lse = lse;
+  p.lists.num_full = nf; p.lists.full_idx = fi; p.lists.num_part = np; p.lists.part_idx = pi;
+  p.lists.LB = g.B; p.lists.LH = 1; p.lists.head_mode = 0;
+  p.policy = kPolicyDflash;
+  p.anchors = anchors; p.N = g.N; p.bs = g.bs; p.Lc = g.Lc;
+  p.causal_in_block = g.causal; p.window = g.window;
+  p.err = err;
+  if (dtype == SMA_FP32) {
+    e = launch_attn_simt(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch failed");
+    return ok();
+  }
+  char msg[256];
+  const int rc = launch_attn_tc(p, st, msg, sizeof(msg));
+  if (rc != SMA_OK) return fail(rc, "%s", msg);
+  return ok();
+}
+
+sma_status mask_tile_summary(const uint8_t* mask, const int64_t mask_sizes[4],
+                             const int64_t mask_strides[4], int32_t k_len, uint8_t* codes,
+                             void* stream) {
+  if (mask == nullptr || codes == nullptr) return fail(SMA_ERR_INVALID_ARG, "NULL pointer");
+  if (k_len < 1) return fail(SMA_ERR_INVALID_ARG, "k_len must be >= 1");
+  if (mask_sizes == nullptr || mask_strides == nullptr)
+    return fail(SMA_ERR_INVALID_ARG, "mask sizes/strides are NULL");
+  for (int i = 0; i < 3; ++i)
+    if (mask_sizes[i] < 1) return fail(SMA_ERR_INVALID_ARG, "mask dims must be >= 1");
+  AuxView view;
+  // Shape checks that involve B/H/Lq do not apply here; use the mask's own dims.
+  sma_status s = check_aux("mask", mask, mask_sizes, mask_strides, 1,
+                           static_cast<int32_t>(mask_sizes[0]), static_cast<int32_t>(mask_sizes[1]),
+                           static_cast<int32_t>(mask_sizes[1]), static_cast<int32_t>(mask_sizes[2]),
+                           k_len, true, &view);
+  if (s != SMA_OK) return s;
+  const int64_t folded[4] = {view.sb, view.sh, view.sq, 1};
+  cudaError_t e = launch_mask_tile_summary(mask, mask_sizes, folded, k_len, codes,
+                                           static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "mask summary launch failed");
+  return ok();
+}
+
+sma_status masked_attn_fwd_workspace_size(int32_t batch, int32_t heads, int32_t kv_heads,
+                                          int32_t q_len, int32_t k_len, int32_t head_dim,
+                                          const int64_t mask_sizes[4], size_t* bytes) {
+  if (bytes == nullptr) return fail(SMA_ERR_INVALID_ARG, "bytes is NULL");
+  sma_status s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (batch < 1 || q_len < 1 || k_len < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, q_len and k_len must be >= 1");
+  *bytes = masked_geom(batch, heads, kv_heads, q_len, k_len, head_dim, mask_sizes).total;
+  return ok();
+}
+
+sma_status masked_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t q_len, int32_t k_len, int32_t head_dim, float scale,
+                           int32_t is_causal, const void* q, const int64_t q_strides[3],
+                           const void* k, const int64_t k_strides[3], const void* v,
+                           const int64_t v_strides[3], const uint8_t* mask,
+                           const int64_t mask_sizes[4], const int64_t mask_strides[4],
+                           const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+                           const int64_t bias_strides[4], void* out, const int64_t o_strides[3],
+                           float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  sma_status s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (batch < 1 || q_len < 1 || k_len < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, q_len and k_len must be >= 1");
+  if (is_causal != 0 && is_causal != 1) return fail(SMA_ERR_INVALID_ARG, "is_causal must be 0 or 1");
+  if ((s = check_operand("q", q, q_strides, dtype, q_len)) != SMA_OK) return s;
+  if ((s = check_operand("k", k, k_strides, dtype, k_len)) != SMA_OK) return s;
+  if ((s = check_operand("v", v, v_strides, dtype, k_len)) != SMA_OK) return s;
+  if ((s = check_operand("out", out, o_strides, dtype, q_len)) != SMA_OK) return s;
+  AuxView mview, bview;
+  const bool has_mask = mask != nullptr, has_bias = bias != nullptr;
+  if (has_mask && (s = check_aux("mask", mask, mask_sizes, mask_strides, 1, batch, heads, kv_heads,
+                                 q_len, k_len, true, &mview)) != SMA_OK)
+    return s;
+  if (has_bias) {
+    if (!valid_dtype(bias_dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown bias dtype %d", bias_dtype);
+    if ((s = check_aux("bias", bias, bias_sizes, bias_strides, elem_size(bias_dtype), batch, heads,
+                       kv_heads, q_len, k_len, true, &bview)) != SMA_OK)
+      return s;
+    bview.dtype = bias_dtype;
+  }
+  const MaskedGeom mg =
+      masked_geom(batch, heads, kv_heads, q_len, k_len, head_dim, has_mask ? mask_sizes : nullptr);
+  if ((s = check_workspace(workspace, workspace_bytes, mg.total)) != SMA_OK) return s;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (err == nullptr) return cuda_fail(e, "device error word unavailable");
+  const float scale_log2 = resolve_scale(scale, head_dim) * kLog2eHost;
+
+  if (mg.decode) {
+    // PR #190 swapped path: rows of one problem are the query heads of a KV head.
+    DecodeProblem dp{};
+    dp.dtype = dtype;
+    dp.B = batch; dp.H = heads; dp.KVH = kv_heads; dp.Lk = k_len; dp.d = head_dim;
+    dp.group = heads / kv_heads;
+    dp.scale_log2 = scale_log2;
+    dp.q = q; dp.q_sb = q_strides[0]; dp.q_sh = q_strides[2];
+    dp.k = k; dp.k_sb = k_strides[0]; dp.k_sr = k_strides[1]; dp.k_sh = k_strides[2];
+    dp.v = v; dp.v_sb = v_strides[0]; dp.v_sr = v_strides[1]; dp.v_sh = v_strides[2];
+    dp.o = out; dp.o_sb = o_strides[0]; dp.o_sh = o_strides[2];
+    dp.lse = lse;
+    dp.has_mask = has_mask; dp.has_bias = has_bias;
+    if (has_mask) dp.mask = mview;
+    if (has_bias) dp.bias = bview;
+    dp.splits = mg.splits;
+    dp.chunk = mg.chunk;
+    dp.part_o = at<float>(workspace, mg.part_o);
+    dp.part_ml = at<float>(workspace, mg.part_ml);
+    dp.err = err;
+    e = launch_decode(dp, st);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch failed");
+    return ok();
+  }
+
+  AttnProblem p{};
+  p.dtype = dtype;
+  p.B = batch; p.H = heads; p.KVH = kv_heads; p.Lq = q_len; p.Lk = k_len; p.d = head_dim;
+  p.group = heads / kv_heads;
+  p.npairs = mg.npairs;
+  p.QT = mg.QT; p.KT = mg.KT;
+  p.scale_log2 = scale_log2;
+  p.q = q; p.q_sb = q_strides[0]; p.q_sr = q_strides[1]; p.q_sh = q_strides[2];
+  p.k = k; p.k_sb = k_strides[0]; p.k_sr = k_strides[1]; p.k_sh = k_strides[2];
+  p.v = v; p.v_sb = v_strides[0]; p.v_sr = v_strides[1]; p.v_sh = v_strides[2];
+  p.o = out; p.o_sb = o_strides[0]; p.o_sr = o_strides[1]; p.o_sh = o_strides[2];
+  p.lse = lse;
+  p.policy = kPolicyExplicit;
+  p.causal = is_causal;
+  p.has_mask = has_mask;
+  p.has_bias = has_bias;
+  if (has_mask) p.mask = mview;
+  if (has_bias) p.bias = bview;
+  p.err = err;
+  p.lists.LB = mg.LB;
+  p.lists.LH = mg.LH;
+  p.lists.head_mode = mg.head_mode;
+  p.lists.num_full = at<int32_t>(workspace, mg.lists.nf);
+  p.lists.num_part = at<int32_t>(workspace, mg.lists.np);
+  p.lists.full_idx = at<int32_t>(workspace, mg.lists.fi);
+  p.lists.part_idx = at<int32_t>(workspace, mg.lists.pi);
+  uint8_t* codes = has_mask ? at<uint8_t>(workspace, 0) : nullptr;
+  if (has_mask) {
+    const int64_t folded[4] = {mview.sb, mview.sh, mview.sq, 1};
+    e = launch_mask_tile_summary(mask, mask_sizes, folded, k_len, codes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "mask summary launch failed");
+  }
+  e = launch_explicit_lists(p, codes, mg.codes_qt, at<int32_t>(workspace, mg.lists.nf),
+                            at<int32_t>(workspace, mg.lists.fi), at<int32_t>(workspace, mg.lists.np),
+                            at<int32_t>(workspace, mg.lists.pi), st);
+  if (e != cudaSuccess) return cuda_fail(e, "tile list launch failed");
+  if (dtype == SMA_FP32) {
+    e = launch_attn_simt(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch failed");
+    return ok();
+  }
+  char msg[256];
+  const int rc = launch_attn_tc(p, st, msg, sizeof(msg));
+  if (rc != SMA_OK) return fail(rc, "%s", msg);
+  return ok();
+}
+
+sma_status dynamic_topk_mask(int32_t bias_dtype, const void* bias, const int64_t bias_sizes[4],
+                             const int64_t bias_strides[4], int32_t k_len, const uint8_t* pre_mask,
+                             const int64_t pre_mask_sizes[4], const int64_t pre_mask_strides[4],
+                             int32_t window_size, uint8_t* out_mask, void* stream) {
+  if (!valid_dtype(bias_dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown bias dtype %d", bias_dtype);
+  if (bias == nullptr || out_mask == nullptr) return fail(SMA_ERR_INVALID_ARG, "NULL pointer");
+  if (bias_sizes == nullptr || bias_strides == nullptr)
+    return fail(SMA_ERR_INVALID_ARG, "bias sizes/strides are NULL");
+  if (k_len < 1) return fail(SMA_ERR_INVALID_ARG, "k_len must be >= 1");
+  if (window_size < 1) return fail(SMA_ERR_INVALID_ARG, "window_size must be >= 1");
+  for (int i = 0; i < 3; ++i)
+    if (bias_sizes[i] < 1) return fail(SMA_ERR_INVALID_ARG, "bias dims must be >= 1");
+  const int64_t kpad = round_up(k_len, kTile);
+  if (bias_sizes[3] != kpad)
+    return fail(SMA_ERR_INVALID_ARG, "bias key dim must be round_up(k_len, 128) = %lld",
+                static_cast<long long>(kpad));
+  if (bias_strides[3] != 1) return fail(SMA_ERR_INVALID_ARG, "bias last dim must be contiguous");
+  if (!aligned16(bias)) return fail(SMA_ERR_INVALID_ARG, "bias must be 16-byte aligned");
+  const int es = elem_size(bias_dtype);
+  TopkProblem p{};
+  p.bias_dtype = bias_dtype;
+  p.bias = bias;
+  for (int i = 0; i < 4; ++i) {
+    p.b_sizes[i] = bias_sizes[i];
+    p.b_strides[i] = (i < 3 && bias_sizes[i] == 1) ? 0 : bias_strides[i];
+    if (p.b_strides[i] < 0 || (i < 3 && (p.b_strides[i] * es) % 16 != 0))
+      return fail(SMA_ERR_INVALID_ARG, "bias strides must be non-negative multiples of 16 bytes");
+  }
+  p.Lk = k_len;
+  p.Kpad = static_cast<int>(kpad);
+  p.pre = pre_mask;
+  if (pre_mask != nullptr) {
+    if (pre_mask_sizes == nullptr || pre_mask_strides == nullptr)
+      return fail(SMA_ERR_INVALID_ARG, "pre_mask sizes/strides are NULL");
+    for (int i = 0; i < 3; ++i) {
+      if (pre_mask_sizes[i] != 1 && pre_mask_sizes[i] != bias_sizes[i])
+        return fail(SMA_ERR_INVALID_ARG, "pre_mask dim %d must be 1 or %lld", i,
+                    static_cast<long long>(bias_sizes[i]));
+    }
+    if (pre_mask_sizes[3] < 1) return fail(SMA_ERR_INVALID_ARG, "pre_mask key dim must be >= 1");
+    if (pre_mask_strides[3] != 1)
+      return fail(SMA_ERR_INVALID_ARG, "pre_mask last dim must be contiguous");
+    for (int i = 0; i < 4; ++i) {
+      p.p_sizes[i] = pre_mask_sizes[i];
+      p.p_strides[i] = (i < 3 && pre_mask_sizes[i] == 1) ? 0 : pre_mask_strides[i];
+      if (p.p_strides[i] < 0) return fail(SMA_ERR_INVALID_ARG, "pre_mask strides must be >= 0");
+    }
+  }
+  p.window = window_size;
+  p.out = out_mask;
+  if ((reinterpret_cast<uintptr_t>(out_mask) & 7u) != 0)
+    return fail(SMA_ERR_INVALID_ARG, "out_mask must be 8-byte aligned");
+  cudaError_t e = launch_topk(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "top-k launch failed");
+  return ok();
+}
+
+}  // extern "C"

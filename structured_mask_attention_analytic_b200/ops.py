@@ -1,0 +1,251 @@
+"""Python binding of libsma: the same entry points as include/sma.h, taking
+torch CUDA tensors.
+
+Only argument marshalling happens here (pointers, strides, the current
+stream, workspace buffers from the torch allocator); every step of the
+computation runs in the library's CUDA kernels.  Nothing falls back to
+PyTorch or the CPU: a missing library or a rejected argument raises.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _native as nat
+
+_DTYPE = {torch.bfloat16: nat.SMA_BF16, torch.float16: nat.SMA_FP16, torch.float32: nat.SMA_FP32}
+
+LAYER_FULL = 0
+LAYER_SLIDING = 1
+
+
+def _lib():
+    return nat.load()
+
+
+def _stream(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libsma ops take CUDA tensors")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _DTYPE[t.dtype]
+    except KeyError:
+        raise ValueError(f"unsupported dtype {t.dtype}") from None
+
+
+def round_up_k(k_len: int) -> int:
+    """Key dim of a mask/bias under the broadcast contract: round_up(k_len, 128)."""
+    return (k_len + 127) // 128 * 128
+
+
+def _is_causal_code(is_causal) -> int:
+    if is_causal is None:
+        return -1
+    return 1 if int(is_causal) == 1 else (0 if int(is_causal) == 0 else -1)
+
+
+def _desc(batch, n_blocks, block_size, ctx_len, is_causal, layer_type, sliding_window):
+    return nat.DfaMaskDesc(int(batch), int(n_blocks), int(block_size), int(ctx_len),
+                           _is_causal_code(is_causal), int(layer_type), int(sliding_window))
+
+
+def dfa_block_map_dims(batch, n_blocks, block_size, ctx_len, is_causal=None, layer_type=LAYER_FULL,
+                       sliding_window=0):
+    d = _desc(batch, n_blocks, block_size, ctx_len, is_causal, layer_type, sliding_window)
+    qt, kt = ctypes.c_int32(), ctypes.c_int32()
+    nat.check(_lib().dfa_block_map_dims(ctypes.byref(d), ctypes.byref(qt), ctypes.byref(kt)))
+    return qt.value, kt.value
+
+
+def dfa_block_map(anchors: torch.Tensor, ctx_len: int, block_size: int, is_causal=None,
+                  layer_type: int = LAYER_FULL, sliding_window: int = 0):
+    """DFlash block map of ``anchors`` (int32 [B, N], CUDA).
+
+    Returns ``(num_full [B,QT], full_idx [B,QT,KT], num_part [B,QT],
+    part_idx [B,QT,KT])`` int32 tensors."""
+    _require_cuda(anchors)
+    if anchors.dtype != torch.int32 or anchors.dim() != 2:
+        raise ValueError("anchors must be int32 [batch, n_blocks]")
+    anchors = anchors.contiguous()
+    b, n = anchors.shape
+    d = _desc(b, n, block_size, ctx_len, is_causal, layer_type, sliding_window)
+    qt, kt = dfa_block_map_dims(b, n, block_size, ctx_len, is_causal, layer_type, sliding_window)
+    dev = anchors.device
+    nf = torch.empty((b, qt), dtype=torch.int32, device=dev)
+    npart = torch.empty((b, qt), dtype=torch.int32, device=dev)
+    fi = torch.empty((b, qt, kt), dtype=torch.int32, device=dev)
+    pi = torch.empty((b, qt, kt), dtype=torch.int32, device=dev)
+    nat.check(_lib().dfa_block_map(ctypes.byref(d), _ptr(anchors), _ptr(nf), _ptr(fi), _ptr(npart),
+                                   _ptr(pi), _stream(anchors)))
+    return nf, fi, npart, pi
+
+
+def dfa_attn_fwd_workspace_size(batch, n_blocks, block_size, ctx_len, heads, kv_heads, head_dim,
+                                is_causal=None, layer_type=LAYER_FULL, sliding_window=0) -> int:
+    d = _desc(batch, n_blocks, block_size, ctx_len, is_causal, layer_type, sliding_window)
+    n = ctypes.c_size_t()
+    nat.check(_lib().dfa_attn_fwd_workspace_size(ctypes.byref(d), heads, kv_heads, head_dim,
+                                                 ctypes.byref(n)))
+    return n.value
+
+
+def _strides3(t: torch.Tensor):
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("q/k/v/out must be 4D [batch, len, heads, head_dim] with head_dim contiguous")
+    return nat.i64_array(t.stride()[:3])
+
+
+def dfa_attn_fwd(q, k, v, anchors, ctx_len: int, block_size: int, is_causal=None,
+                 layer_type: int = LAYER_FULL, sliding_window: int = 0, scale=None, out=None,
+                 return_lse: bool = True, workspace=None):
+    """Attention forward under the DFlash draft-training mask.
+
+    q ``[B, N*block_size, H, d]``, k/v ``[B, ctx_len + N*block_size, KVH, d]``,
+    anchors int32 ``[B, N]``.  Returns ``(out, lse)`` (lse None unless
+    requested)."""
+    _require_cuda(q, k, v, anchors)
+    b, nq, h, dh = q.shape
+    kvh = k.shape[2]
+    if anchors.dtype != torch.int32 or anchors.dim() != 2 or anchors.shape[0] != b:
+        raise ValueError("anchors must be int32 [batch, n_blocks]")
+    anchors = anchors.contiguous()
+    n = anchors.shape[1]
+    if nq != n * block_size or k.shape[1] != ctx_len + nq or v.shape != k.shape:
+        raise ValueError("q/k/v lengths do not match ctx_len, n_blocks and block_size")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k and v must share a dtype")
+    d = _desc(b, n, block_size, ctx_len, is_causal, layer_type, sliding_window)
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((b, h, nq), dtype=torch.float32, device=q.device) if return_lse else None
+    ws_bytes = dfa_attn_fwd_workspace_size(b, n, block_size, ctx_len, h, kvh, dh, is_causal,
+                                           layer_type, sliding_window)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    nat.check(_lib().dfa_attn_fwd(
+        ctypes.byref(d), _ptr(anchors), _dtype_code(q), h, kvh, dh,
+        ctypes.c_float(0.0 if scale is None else float(scale)),
+        _ptr(q), _strides3(q), _ptr(k), _strides3(k), _ptr(v), _strides3(v), _ptr(out), _strides3(out),
+        _ptr(lse), _ptr(workspace), workspace.numel(), _stream(q)))
+    return out, lse
+
+
+def _aux_args(t, k_len):
+    if t is None:
+        return ctypes.c_void_p(0), None, None
+    if t.dim() != 4:
+        raise ValueError("mask/bias must be 4D ({B|1}, {H|KVH|1}, {Lq|1}, round_up(Lk,128))")
+    return _ptr(t), nat.i64_array(t.shape), nat.i64_array(t.stride())
+
+
+def mask_tile_summary(mask: torch.Tensor, k_len: int) -> torch.Tensor:
+    """uint8 codes ``[m0, m1, ceil(m2/128), ceil(k_len/128)]`` of a 4D bool mask."""
+    _require_cuda(mask)
+    if mask.dtype not in (torch.bool, torch.uint8):
+        raise ValueError("mask must be bool")
+    m0, m1, m2, _ = mask.shape
+    codes = torch.empty((m0, m1, (m2 + 127) // 128, (k_len + 127) // 128), dtype=torch.uint8,
+                        device=mask.device)
+    p, sz, st = _aux_args(mask, k_len)
+    nat.check(_lib().mask_tile_summary(p, sz, st, int(k_len), _ptr(codes), _stream(mask)))
+    return codes
+
+
+def masked_attn_fwd_workspace_size(batch, heads, kv_heads, q_len, k_len, head_dim, mask_shape=None) -> int:
+    n = ctypes.c_size_t()
+    ms = nat.i64_array(mask_shape) if mask_shape is not None else None
+    nat.check(_lib().masked_attn_fwd_workspace_size(batch, heads, kv_heads, q_len, k_len, head_dim, ms,
+                                                    ctypes.byref(n)))
+    return n.value
+
+
+def masked_attn_fwd(q, k, v, mask=None, bias=None, is_causal: bool = False, scale=None, out=None,
+                    return_lse: bool = True, workspace=None):
+    """Attention forward with a broadcastable 4D bool mask and/or additive bias.
+
+    mask / bias follow ``({B|1}, {H|KVH|1}, {Lq|1}, round_up(Lk, 128))`` with a
+    contiguous last dim; broadcast dims may have any stride (they are read
+    with stride 0).  ``q_len == 1`` takes the grouped-head decode path.
+    Returns ``(out, lse)``."""
+    _require_cuda(q, k, v, mask, bias)
+    b, lq, h, dh = q.shape
+    lk, kvh = k.shape[1], k.shape[2]
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k and v must share a dtype")
+    if mask is not None and mask.dtype not in (torch.bool, torch.uint8):
+        raise ValueError("mask must be bool")
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((b, h, lq), dtype=torch.float32, device=q.device) if return_lse else None
+    ws_bytes = masked_attn_fwd_workspace_size(b, h, kvh, lq, lk, dh,
+                                              tuple(mask.shape) if mask is not None else None)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    mp, msz, mst = _aux_args(mask, lk)
+    bp, bsz, bst = _aux_args(bias, lk)
+    nat.check(_lib().masked_attn_fwd(
+        _dtype_code(q), b, h, kvh, lq, lk, dh, ctypes.c_float(0.0 if scale is None else float(scale)),
+        1 if is_causal else 0,
+        _ptr(q), _strides3(q), _ptr(k), _strides3(k), _ptr(v), _strides3(v),
+        mp, msz, mst,
+        bp, _dtype_code(bias) if bias is not None else 0, bsz, bst,
+        _ptr(out), _strides3(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(q)))
+    return out, lse
+
+
+def _pre_mask_view(pre_mask: torch.Tensor, batch: int, q_len: int, k_len: int):
+    """create_mask's shape step as a view: a 2D (batch, L) pre-mask becomes
+    sizes (batch, 1, 1, L); columns >= L count as invalid, which equals
+    padding with False (L == q_len < k_len) or cutting (L > k_len)."""
+    if pre_mask.dim() == 2:
+        if pre_mask.shape[0] != batch:
+            raise ValueError("2D pre-mask must be (batch, seq_len)")
+        if pre_mask.shape[1] not in (k_len, q_len):
+            raise ValueError("2D pre-mask length must be key_len or query_len")
+        return pre_mask.view(batch, 1, 1, pre_mask.shape[1])
+    if pre_mask.dim() == 4:
+        return pre_mask
+    raise ValueError("pre-mask must be 2D or 4D")
+
+
+def dynamic_topk_mask(bias: torch.Tensor, k_len: int, window_size: int, pre_mask=None, q_len=None,
+                      out=None) -> torch.Tensor:
+    """Bool keep mask of ``bias``'s shape: per row the ``window_size`` largest
+    entries among the first ``k_len`` columns after the pre-mask, and'ed with
+    the pre-mask."""
+    _require_cuda(bias, pre_mask)
+    if bias.dim() != 4:
+        raise ValueError("bias must be 4D")
+    if out is None:
+        out = torch.empty(bias.shape, dtype=torch.bool, device=bias.device)
+    pp, psz, pst = ctypes.c_void_p(0), None, None
+    if pre_mask is not None:
+        if pre_mask.dtype not in (torch.bool, torch.uint8):
+            raise ValueError("pre-mask must be bool")
+        pm = _pre_mask_view(pre_mask, bias.shape[0], bias.shape[2] if q_len is None else q_len, k_len)
+        pp, psz, pst = _ptr(pm), nat.i64_array(pm.shape), nat.i64_array(pm.stride())
+    nat.check(_lib().dynamic_topk_mask(_dtype_code(bias), _ptr(bias), nat.i64_array(bias.shape),
+                                       nat.i64_array(bias.stride()), int(k_len), pp, psz, pst,
+                                       int(window_size), _ptr(out), _stream(bias)))
+    return out
+
+
+def device_status(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device error word."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    v = ctypes.c_int32()
+    s = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    nat.check(_lib().sma_device_status(s, ctypes.byref(v)))
+    return v.value

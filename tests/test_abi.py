@@ -1,0 +1,135 @@
+"""The C-ABI library loads, exports every symbol include/sma.h declares, and
+its host-side validation rejects bad arguments before touching the GPU.
+CPU only: no call here reaches a CUDA API (validation runs first)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from structured_mask_attention_analytic_b200 import _native as nat
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "sma.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_][a-z0-9_]*)\s*\(", text,
+                       flags=re.M)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for want in ["dfa_block_map", "dfa_attn_fwd", "masked_attn_fwd", "dynamic_topk_mask",
+                 "mask_tile_summary", "sma_last_error", "sma_device_status"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = nat.load()
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.sma_abi_version() == 1
+
+
+def test_block_map_dims_on_host():
+    d = nat.DfaMaskDesc(2, 256, 16, 4096, -1, 0, 0)
+    qt, kt = ctypes.c_int32(), ctypes.c_int32()
+    assert nat.load().dfa_block_map_dims(ctypes.byref(d), ctypes.byref(qt), ctypes.byref(kt)) == 0
+    assert (qt.value, kt.value) == (32, 64)
+    d = nat.DfaMaskDesc(1, 4, 16, 64, -1, 0, 0)
+    assert nat.load().dfa_block_map_dims(ctypes.byref(d), ctypes.byref(qt), ctypes.byref(kt)) == 0
+    assert (qt.value, kt.value) == (1, 1)
+
+
+@pytest.mark.parametrize("fields,msg", [
+    ((0, 4, 16, 64, -1, 0, 0), "batch"),
+    ((1, 4, 16, 64, 2, 0, 0), "is_causal"),
+    ((1, 4, 16, 64, -1, 3, 0), "layer_type"),
+    ((1, 4, 16, 64, -1, 1, 0), "sliding_window"),
+    ((1, 4, 0, 64, -1, 0, 0), "block_size"),
+])
+def test_bad_descriptors_are_rejected(fields, msg):
+    d = nat.DfaMaskDesc(*fields)
+    qt, kt = ctypes.c_int32(), ctypes.c_int32()
+    st = nat.load().dfa_block_map_dims(ctypes.byref(d), ctypes.byref(qt), ctypes.byref(kt))
+    assert st == nat.SMA_ERR_INVALID_ARG
+    assert msg in nat.load().sma_last_error().decode()
+
+
+def test_workspace_sizes_on_host():
+    lib = nat.load()
+    d = nat.DfaMaskDesc(1, 2048, 16, 32768, 1, 0, 0)
+    n = ctypes.c_size_t()
+    assert lib.dfa_attn_fwd_workspace_size(ctypes.byref(d), 32, 8, 128, ctypes.byref(n)) == 0
+    # num_full + num_part (256 each) + two 256 x 512 index arrays, 256-byte aligned
+    assert n.value >= 2 * 256 * 4 + 2 * 256 * 512 * 4
+    assert lib.dfa_attn_fwd_workspace_size(ctypes.byref(d), 32, 8, 96, ctypes.byref(n)) == nat.SMA_ERR_UNSUPPORTED
+    assert lib.dfa_attn_fwd_workspace_size(ctypes.byref(d), 30, 8, 128, ctypes.byref(n)) == nat.SMA_ERR_INVALID_ARG
+    ms = nat.i64_array([1, 1, 8192, 8064])
+    assert lib.masked_attn_fwd_workspace_size(4, 16, 4, 8192, 8000, 128, ms, ctypes.byref(n)) == 0
+    assert n.value > 0
+    assert lib.masked_attn_fwd_workspace_size(8, 32, 8, 1, 16384, 128, None, ctypes.byref(n)) == 0
+    assert n.value > 0
+
+
+def _masked_call(**over):
+    """masked_attn_fwd with fake (never dereferenced) aligned pointers."""
+    a = dict(dtype=0, batch=2, heads=4, kv_heads=2, q_len=256, k_len=200, head_dim=128,
+             q=0x10000, k=0x20000, v=0x30000, out=0x40000,
+             qs=[256 * 4 * 128, 4 * 128, 128], ks=[200 * 2 * 128, 2 * 128, 128],
+             mask=None, msz=None, mst=None, bias=None, bsz=None, bst=None, ws=0x50000, wsb=1 << 30)
+    a.update(over)
+    return nat.load().masked_attn_fwd(
+        a["dtype"], a["batch"], a["heads"], a["kv_heads"], a["q_len"], a["k_len"], a["head_dim"],
+        ctypes.c_float(0.0), 0,
+        ctypes.c_void_p(a["q"]), nat.i64_array(a["qs"]), ctypes.c_void_p(a["k"]), nat.i64_array(a["ks"]),
+        ctypes.c_void_p(a["v"]), nat.i64_array(a["ks"]),
+        ctypes.c_void_p(a["mask"]), a["msz"] and nat.i64_array(a["msz"]), a["mst"] and nat.i64_array(a["mst"]),
+        ctypes.c_void_p(a["bias"]), 0, a["bsz"] and nat.i64_array(a["bsz"]), a["bst"] and nat.i64_array(a["bst"]),
+        ctypes.c_void_p(a["out"]), nat.i64_array(a["qs"]), None, ctypes.c_void_p(a["ws"]), a["wsb"], None)
+
+
+@pytest.mark.parametrize("over,status,msg", [
+    (dict(q=0x10002), nat.SMA_ERR_INVALID_ARG, "aligned"),
+    (dict(qs=[256 * 4 * 128, 4 * 128 + 1, 128]), nat.SMA_ERR_INVALID_ARG, "16 bytes"),
+    (dict(heads=3), nat.SMA_ERR_INVALID_ARG, "multiple"),
+    (dict(head_dim=80), nat.SMA_ERR_UNSUPPORTED, "head_dim"),
+    (dict(mask=0x60000, msz=[1, 1, 256, 200], mst=[0, 0, 200, 1]), nat.SMA_ERR_INVALID_ARG, "round_up"),
+    (dict(mask=0x60000, msz=[1, 3, 256, 256], mst=[0, 0, 256, 1]), nat.SMA_ERR_INVALID_ARG, "head dim"),
+    (dict(mask=0x60000, msz=[2, 1, 7, 256], mst=[256, 0, 256, 1]), nat.SMA_ERR_INVALID_ARG, "query dim"),
+    (dict(mask=0x60000, msz=[1, 1, 256, 256], mst=[0, 0, 1, 256]), nat.SMA_ERR_INVALID_ARG, "contiguous"),
+    (dict(bias=0x60000, bsz=[3, 1, 1, 256], bst=[256, 0, 0, 1]), nat.SMA_ERR_INVALID_ARG, "batch dim"),
+    (dict(wsb=16), nat.SMA_ERR_WORKSPACE, "workspace"),
+])
+def test_masked_attn_validation(over, status, msg):
+    assert _masked_call(**over) == status
+    assert msg in nat.load().sma_last_error().decode()
+
+
+def test_topk_validation():
+    lib = nat.load()
+    bad_window = lib.dynamic_topk_mask(0, ctypes.c_void_p(0x10000), nat.i64_array([1, 1, 1, 256]),
+                                       nat.i64_array([256, 256, 256, 1]), 200, None, None, None, 0,
+                                       ctypes.c_void_p(0x20000), None)
+    assert bad_window == nat.SMA_ERR_INVALID_ARG
+    bad_k = lib.dynamic_topk_mask(0, ctypes.c_void_p(0x10000), nat.i64_array([1, 1, 1, 200]),
+                                  nat.i64_array([200, 200, 200, 1]), 200, None, None, None, 8,
+                                  ctypes.c_void_p(0x20000), None)
+    assert bad_k == nat.SMA_ERR_INVALID_ARG
+    assert "round_up" in lib.sma_last_error().decode()
+    bad_pm = lib.dynamic_topk_mask(0, ctypes.c_void_p(0x10000), nat.i64_array([2, 1, 1, 256]),
+                                   nat.i64_array([256, 256, 256, 1]), 200, ctypes.c_void_p(0x30000),
+                                   nat.i64_array([3, 1, 1, 200]), nat.i64_array([200, 0, 0, 1]), 8,
+                                   ctypes.c_void_p(0x20000), None)
+    assert bad_pm == nat.SMA_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(nat, "LIB_PATH", str(tmp_path / "libsma.so"))
+    monkeypatch.setattr(nat, "_lib", None)
+    with pytest.raises(nat.NativeLibraryMissing):
+        nat.load()
