@@ -136,14 +136,27 @@ sma_status dfa_block_map_dims(const dfa_mask_desc* desc, int32_t* q_tiles, int32
 sma_status dfa_block_map(const dfa_mask_desc* desc, const int32_t* anchors, int32_t* num_full,
                          int32_t* full_idx, int32_t* num_part, int32_t* part_idx, void* stream);
 
-/* Workspace bytes dfa_attn_fwd needs for this problem (block map and tile
- * schedule).  The caller allocates it; it may be reused across calls that are
- * ordered on one stream. */
+/* A block map produced by dfa_block_map for the same descriptor (device
+ * pointers, layouts as documented there). */
+typedef struct dfa_block_map_ptrs {
+  const int32_t* num_full;
+  const int32_t* full_idx;
+  const int32_t* num_part;
+  const int32_t* part_idx;
+} dfa_block_map_ptrs;
+
+/* Workspace bytes dfa_attn_fwd needs for this problem when it computes the
+ * block map itself (0 is enough when a precomputed map is passed).  The
+ * caller allocates it; it may be reused across calls ordered on one stream. */
 sma_status dfa_attn_fwd_workspace_size(const dfa_mask_desc* desc, int32_t heads, int32_t kv_heads,
                                        int32_t head_dim, size_t* bytes);
 
 /* Attention forward under the DFlash mask.
  *
+ * block_map  NULL: the map is computed into `workspace` first (one extra
+ *            kernel).  Otherwise a map from dfa_block_map for the same desc
+ *            and anchors, e.g. shared by the layers of one training step;
+ *            `workspace` may then be NULL with 0 bytes.
  * q    [batch, q_len, heads, head_dim]     strides q_strides (batch, row, head)
  * k, v [batch, k_len, kv_heads, head_dim]  strides k_strides / v_strides
  * out  [batch, q_len, heads, head_dim]     strides o_strides; same dtype as q
@@ -156,7 +169,8 @@ sma_status dfa_attn_fwd(const dfa_mask_desc* desc, const int32_t* anchors, int32
                         int32_t heads, int32_t kv_heads, int32_t head_dim, float scale,
                         const void* q, const int64_t q_strides[3], const void* k,
                         const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
-                        void* out, const int64_t o_strides[3], float* lse, void* workspace,
+                        void* out, const int64_t o_strides[3], float* lse,
+                        const dfa_block_map_ptrs* block_map, void* workspace,
                         size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------

@@ -36,6 +36,10 @@ class DfaMaskDesc(ctypes.Structure):
                 ("is_causal", c_i32), ("layer_type", c_i32), ("sliding_window", c_i32)]
 
 
+class DfaBlockMapPtrs(ctypes.Structure):
+    _fields_ = [("num_full", c_vp), ("full_idx", c_vp), ("num_part", c_vp), ("part_idx", c_vp)]
+
+
 class NativeLibraryMissing(RuntimeError):
     pass
 
@@ -54,8 +58,8 @@ _SIGNATURES = {
     "dfa_block_map": (c_i32, [ctypes.POINTER(DfaMaskDesc), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "dfa_attn_fwd_workspace_size": (c_i32, [ctypes.POINTER(DfaMaskDesc), c_i32, c_i32, c_i32, c_sizep]),
     "dfa_attn_fwd": (c_i32, [ctypes.POINTER(DfaMaskDesc), c_vp, c_i32, c_i32, c_i32, c_i32, ctypes.c_float,
-                             c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_vp, c_size,
-                             c_vp]),
+                             c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp,
+                             ctypes.POINTER(DfaBlockMapPtrs), c_vp, c_size, c_vp]),
     "mask_tile_summary": (c_i32, [c_vp, c_i64p, c_i64p, c_i32, c_vp, c_vp]),
     "masked_attn_fwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64p, c_sizep]),
     "masked_attn_fwd": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.c_float, c_i32,

@@ -293,7 +293,8 @@ sma_status dfa_attn_fwd(const dfa_mask_desc* desc, const int32_t* anchors, int32
                         int32_t heads, int32_t kv_heads, int32_t head_dim, float scale,
                         const void* q, const int64_t q_strides[3], const void* k,
                         const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
-                        void* out, const int64_t o_strides[3], float* lse, void* workspace,
+                        void* out, const int64_t o_strides[3], float* lse,
+                        const dfa_block_map_ptrs* block_map, void* workspace,
                         size_t workspace_bytes, void* stream) {
   sma_status s = check_desc(desc);
   if (s != SMA_OK) return s;
@@ -307,18 +308,32 @@ sma_status dfa_attn_fwd(const dfa_mask_desc* desc, const int32_t* anchors, int32
   if ((s = check_operand("v", v, v_strides, dtype, g.Lk)) != SMA_OK) return s;
   if ((s = check_operand("out", out, o_strides, dtype, g.Nq)) != SMA_OK) return s;
   const ListsLayout lay = lists_layout(0, static_cast<int64_t>(g.B) * g.QT, g.KT);
-  if ((s = check_workspace(workspace, workspace_bytes, lay.end)) != SMA_OK) return s;
+  if (block_map != nullptr) {
+    if (!block_map->num_full || !block_map->full_idx || !block_map->num_part || !block_map->part_idx)
+      return fail(SMA_ERR_INVALID_ARG, "block_map has a NULL pointer");
+  } else if ((s = check_workspace(workspace, workspace_bytes, lay.end)) != SMA_OK) {
+    return s;
+  }
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   int* err = device_error_word(&e);
   if (err == nullptr) return cuda_fail(e, "device error word unavailable");
-  int32_t* nf = at<int32_t>(workspace, lay.nf);
-  int32_t* np = at<int32_t>(workspace, lay.np);
-  int32_t* fi = at<int32_t>(workspace, lay.fi);
-  int32_t* pi = at<int32_t>(workspace, lay.pi);
-  e = launch_dfa_block_map(g, anchors, nf, fi, np, pi, err, st);
-  if (e != cudaSuccess) return cuda_fail(e, "block map launch failed");
+  const int32_t *nf, *np, *fi, *pi;
+  if (block_map != nullptr) {
+    nf = block_map->num_full;
+    np = block_map->num_part;
+    fi = block_map->full_idx;
+    pi = block_map->part_idx;
+  } else {
+    int32_t* wnf = at<int32_t>(workspace, lay.nf);
+    int32_t* wnp = at<int32_t>(workspace, lay.np);
+    int32_t* wfi = at<int32_t>(workspace, lay.fi);
+    int32_t* wpi = at<int32_t>(workspace, lay.pi);
+    e = launch_dfa_block_map(g, anchors, wnf, wfi, wnp, wpi, err, st);
+    if (e != cudaSuccess) return cuda_fail(e, "block map launch failed");
+    nf = wnf; np = wnp; fi = wfi; pi = wpi;
+  }
 
   AttnProblem p{};
   p.dtype = dtype;

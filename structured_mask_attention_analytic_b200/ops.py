@@ -109,12 +109,13 @@ def _strides3(t: torch.Tensor):
 
 def dfa_attn_fwd(q, k, v, anchors, ctx_len: int, block_size: int, is_causal=None,
                  layer_type: int = LAYER_FULL, sliding_window: int = 0, scale=None, out=None,
-                 return_lse: bool = True, workspace=None):
+                 return_lse: bool = True, workspace=None, block_map=None):
     """Attention forward under the DFlash draft-training mask.
 
     q ``[B, N*block_size, H, d]``, k/v ``[B, ctx_len + N*block_size, KVH, d]``,
-    anchors int32 ``[B, N]``.  Returns ``(out, lse)`` (lse None unless
-    requested)."""
+    anchors int32 ``[B, N]``.  ``block_map`` optionally passes the 4-tuple
+    returned by ``dfa_block_map`` for the same mask (the map is then not
+    recomputed).  Returns ``(out, lse)`` (lse None unless requested)."""
     _require_cuda(q, k, v, anchors)
     b, nq, h, dh = q.shape
     kvh = k.shape[2]
@@ -130,15 +131,23 @@ def dfa_attn_fwd(q, k, v, anchors, ctx_len: int, block_size: int, is_causal=None
     if out is None:
         out = torch.empty_like(q)
     lse = torch.empty((b, h, nq), dtype=torch.float32, device=q.device) if return_lse else None
-    ws_bytes = dfa_attn_fwd_workspace_size(b, n, block_size, ctx_len, h, kvh, dh, is_causal,
-                                           layer_type, sliding_window)
-    if workspace is None:
-        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    map_ptrs = None
+    if block_map is not None:
+        nf, fi, npart, pi = block_map
+        map_ptrs = ctypes.byref(nat.DfaBlockMapPtrs(nf.data_ptr(), fi.data_ptr(), npart.data_ptr(),
+                                                    pi.data_ptr()))
+        ws_ptr, ws_len = ctypes.c_void_p(0), 0
+    else:
+        ws_bytes = dfa_attn_fwd_workspace_size(b, n, block_size, ctx_len, h, kvh, dh, is_causal,
+                                               layer_type, sliding_window)
+        if workspace is None:
+            workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+        ws_ptr, ws_len = _ptr(workspace), workspace.numel()
     nat.check(_lib().dfa_attn_fwd(
         ctypes.byref(d), _ptr(anchors), _dtype_code(q), h, kvh, dh,
         ctypes.c_float(0.0 if scale is None else float(scale)),
         _ptr(q), _strides3(q), _ptr(k), _strides3(k), _ptr(v), _strides3(v), _ptr(out), _strides3(out),
-        _ptr(lse), _ptr(workspace), workspace.numel(), _stream(q)))
+        _ptr(lse), map_ptrs, ws_ptr, ws_len, _stream(q)))
     return out, lse
 
 
