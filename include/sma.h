@@ -173,6 +173,31 @@ sma_status dfa_attn_fwd(const dfa_mask_desc* desc, const int32_t* anchors, int32
                         const dfa_block_map_ptrs* block_map, void* workspace,
                         size_t workspace_bytes, void* stream);
 
+/* dfa_attn_fwd for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot give the library a device workspace -- a plain C host program
+ * without a CUDA memory manager of its own, or a runtime whose device memory
+ * is fully pre-reserved by another allocator, where one more cudaMalloc
+ * would fail or fragment that pool.
+ *
+ * Same arguments and result as dfa_attn_fwd, without block_map and
+ * workspace: the block map goes to a fixed 4 MiB device array inside the
+ * library (held by every GPU that loads the library until process exit).
+ * Problems whose block map needs more than 4 MiB return SMA_ERR_WORKSPACE
+ * (about batch * q_tiles * (kv_tiles + 1) * 8 bytes; the 32768-query,
+ * 65536-key long-context problem needs 1.05 MB).  Calls share the array:
+ * calls that may overlap on the GPU (unordered streams) race, so order them
+ * on one stream.  The first call on a device looks up the array's address
+ * with that device current; make it before any stream capture starts.  No
+ * device memory is allocated or freed. */
+sma_status dfa_attn_fwd_noalloc(const dfa_mask_desc* desc, const int32_t* anchors, int32_t dtype,
+                                int32_t heads, int32_t kv_heads, int32_t head_dim, float scale,
+                                const void* q, const int64_t q_strides[3], const void* k,
+                                const int64_t k_strides[3], const void* v,
+                                const int64_t v_strides[3], void* out, const int64_t o_strides[3],
+                                float* lse, void* stream);
+
 /* ------------------------------------------------------------------------
  * Broadcastable 4D mask / bias contract.
  *

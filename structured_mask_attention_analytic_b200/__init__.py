@@ -10,6 +10,7 @@ from .ops import (  # noqa: F401
     LAYER_SLIDING,
     device_status,
     dfa_attn_fwd,
+    dfa_attn_fwd_noalloc,
     dfa_attn_fwd_workspace_size,
     dfa_block_map,
     dfa_block_map_dims,

@@ -60,6 +60,9 @@ _SIGNATURES = {
     "dfa_attn_fwd": (c_i32, [ctypes.POINTER(DfaMaskDesc), c_vp, c_i32, c_i32, c_i32, c_i32, ctypes.c_float,
                              c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp,
                              ctypes.POINTER(DfaBlockMapPtrs), c_vp, c_size, c_vp]),
+    "dfa_attn_fwd_noalloc": (c_i32, [ctypes.POINTER(DfaMaskDesc), c_vp, c_i32, c_i32, c_i32, c_i32,
+                                     ctypes.c_float, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp,
+                                     c_i64p, c_vp, c_vp]),
     "mask_tile_summary": (c_i32, [c_vp, c_i64p, c_i64p, c_i32, c_vp, c_vp]),
     "masked_attn_fwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64p, c_sizep]),
     "masked_attn_fwd": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.c_float, c_i32,

@@ -121,6 +121,10 @@ cudaError_t launch_decode(const DecodeProblem& p, cudaStream_t stream);
 
 cudaError_t launch_topk(const TopkProblem& p, cudaStream_t stream);
 
+// Records `message` as the calling thread's last error (read back through
+// sma_last_error) and returns `code`.
+int set_last_error(int code, const char* message);
+
 // Device error word of the current device.
 int* device_error_word(cudaError_t* status);
 

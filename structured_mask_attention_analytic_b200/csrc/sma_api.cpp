@@ -228,6 +228,11 @@ MaskedGeom masked_geom(int32_t B, int32_t H, int32_t KVH, int32_t Lq, int32_t Lk
 
 }  // namespace
 
+int sma::set_last_error(int code, const char* message) {
+  g_last_error = message;
+  return code;
+}
+
 extern "C" {
 
 const char* sma_last_error(void) { return g_last_error.c_str(); }

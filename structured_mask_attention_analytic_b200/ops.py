@@ -151,6 +151,31 @@ def dfa_attn_fwd(q, k, v, anchors, ctx_len: int, block_size: int, is_causal=None
     return out, lse
 
 
+def dfa_attn_fwd_noalloc(q, k, v, anchors, ctx_len: int, block_size: int, is_causal=None,
+                         layer_type: int = LAYER_FULL, sliding_window: int = 0, scale=None, out=None,
+                         return_lse: bool = True):
+    """dfa_attn_fwd without a workspace, for callers that cannot allocate
+    device scratch: the block map goes to a fixed 4 MiB array inside libsma
+    (larger problems raise).  Calls share that array, so calls that may run
+    concurrently on the GPU race; keep them on one stream."""
+    _require_cuda(q, k, v, anchors)
+    b, nq, h, dh = q.shape
+    kvh = k.shape[2]
+    if anchors.dtype != torch.int32 or anchors.dim() != 2 or anchors.shape[0] != b:
+        raise ValueError("anchors must be int32 [batch, n_blocks]")
+    anchors = anchors.contiguous()
+    d = _desc(b, anchors.shape[1], block_size, ctx_len, is_causal, layer_type, sliding_window)
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((b, h, nq), dtype=torch.float32, device=q.device) if return_lse else None
+    nat.check(_lib().dfa_attn_fwd_noalloc(
+        ctypes.byref(d), _ptr(anchors), _dtype_code(q), h, kvh, dh,
+        ctypes.c_float(0.0 if scale is None else float(scale)),
+        _ptr(q), _strides3(q), _ptr(k), _strides3(k), _ptr(v), _strides3(v), _ptr(out), _strides3(out),
+        _ptr(lse), _stream(q)))
+    return out, lse
+
+
 def _aux_args(t, k_len):
     if t is None:
         return ctypes.c_void_p(0), None, None
