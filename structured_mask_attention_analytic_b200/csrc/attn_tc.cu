@@ -171,178 +171,215 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
    if (warp == kLoadWarp) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane issues the copies.
+    if (elect_one()) {
       tma_prefetch_map(&map_q);
       tma_prefetch_map(&map_k);
       tma_prefetch_map(&map_v);
-      uint32_t kv_k = 0, kv_v = 0, q_it = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const Unit w = decode_unit(p, u);
-        const int n = w.n_full + w.n_part;
-        if (n == 0) continue;
-        if (q_it > 0 && !mbar_wait(bar(L::kQEmpty), (q_it - 1) & 1, abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
+    }
+    __syncwarp();
+    uint32_t kv_k = 0, kv_v = 0, q_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit w = decode_unit(p, u);
+      const int n = w.n_full + w.n_part;
+      if (n == 0) continue;
+      if (q_it > 0 && !mbar_wait_warp(bar(L::kQEmpty), (q_it - 1) & 1, abort_flag, p.err)) {
+        ok = false;
+        break;
+      }
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar(L::kQFull), (1 + w.h1valid) * L::kTileBytes);
         for (int i = 0; i < 1 + w.h1valid; ++i)
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sbase + L::kQ + i * L::kTileBytes + c * L::kChunkBytes, &map_q,
                         bar(L::kQFull), c * 64, w.h0 + i, w.qt * kTile, w.b);
-        ++q_it;
-        for (int j = 0; j < n && ok; ++j) {
-          bool partial;
-          const int kt = tile_at(p, w, j, &partial);
-          const int stage = kv_k % L::kStages;
-          const uint32_t use = kv_k / L::kStages;
-          if (use > 0 && !mbar_wait(bar(L::kKEmpty + stage), (use - 1) & 1, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
+      }
+      __syncwarp();
+      ++q_it;
+      bool partial_next = false;
+      int kt_next = tile_at(p, w, 0, &partial_next);
+      for (int j = 0; j < n && ok; ++j) {
+        const int kt = kt_next;
+        if (j + 1 < n) kt_next = tile_at(p, w, j + 1, &partial_next);
+        const int stage = kv_k % L::kStages;
+        const uint32_t use = kv_k / L::kStages;
+        if (use > 0 && !mbar_wait_warp(bar(L::kKEmpty + stage), (use - 1) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
           mbar_arrive_expect_tx(bar(L::kKFull + stage), L::kTileBytes);
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sbase + L::kK + stage * L::kTileBytes + c * L::kChunkBytes, &map_k,
                         bar(L::kKFull + stage), c * 64, w.hk, kt * kTile, w.b);
-          ++kv_k;
-          if (use > 0 && !mbar_wait(bar(L::kVEmpty + stage), (use - 1) & 1, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
+        }
+        __syncwarp();
+        ++kv_k;
+        if (use > 0 && !mbar_wait_warp(bar(L::kVEmpty + stage), (use - 1) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
           mbar_arrive_expect_tx(bar(L::kVFull + stage), L::kTileBytes);
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sbase + L::kV + stage * L::kTileBytes + c * L::kChunkBytes, &map_v,
                         bar(L::kVFull + stage), c * 64, w.hk, kt * kTile, w.b);
-          ++kv_v;
+        }
+        __syncwarp();
+        ++kv_v;
+      }
+    }
+    if (!ok) {
+      // Drain: every copy this warp issued must land before the CTA exits.
+      for (uint32_t t = 0; t < static_cast<uint32_t>(L::kStages); ++t) {
+        if (kv_k > t) {
+          const uint32_t nn = kv_k - 1 - t;
+          drain_wait(bar(L::kKFull + nn % L::kStages), (nn / L::kStages) & 1, p.err);
+        }
+        if (kv_v > t) {
+          const uint32_t nn = kv_v - 1 - t;
+          drain_wait(bar(L::kVFull + nn % L::kStages), (nn / L::kStages) & 1, p.err);
         }
       }
-      if (!ok) {
-        // Drain: every copy this thread issued must land before the CTA exits.
-        for (uint32_t t = 0; t < static_cast<uint32_t>(L::kStages); ++t) {
-          if (kv_k > t) {
-            const uint32_t nn = kv_k - 1 - t;
-            drain_wait(bar(L::kKFull + nn % L::kStages), (nn / L::kStages) & 1, p.err);
-          }
-          if (kv_v > t) {
-            const uint32_t nn = kv_v - 1 - t;
-            drain_wait(bar(L::kVFull + nn % L::kStages), (nn / L::kStages) & 1, p.err);
-          }
-        }
-        if (q_it > 0) drain_wait(bar(L::kQFull), (q_it - 1) & 1, p.err);
-      }
+      if (q_it > 0) drain_wait(bar(L::kQFull), (q_it - 1) & 1, p.err);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t fmt = DT == SMA_BF16 ? 1u : 0u;
-      constexpr uint32_t idesc_qk = mma_idesc_f16(fmt, 128, 128, 0, 0);
-      constexpr uint32_t idesc_pv = mma_idesc_f16(fmt, 128, D, 0, 1);
-      uint32_t kv_it = 0, q_it = 0;
-      uint32_t pv_it[2] = {0, 0}, units[2] = {0, 0};
-      bool ok = true;
-      // Descriptors are built once per operand tile; a k-step only moves the
-      // start-address field (bits 0-13, in 16-byte units).
-      auto issue_qk = [&](int i, int stage) {
-        const uint64_t qd = smem_desc_sw128(sbase + L::kQ + i * L::kTileBytes, 16, 1024);
-        const uint64_t kd = smem_desc_sw128(sbase + L::kK + stage * L::kTileBytes, 16, 1024);
-        const uint32_t d_col = tmem + (i == 0 ? L::kColS0 : L::kColS1);
+    // The whole warp runs the loop and waits; one elected lane issues every
+    // tcgen05.mma and tcgen05.commit (commits track that lane's MMAs).
+    constexpr uint32_t fmt = DT == SMA_BF16 ? 1u : 0u;
+    constexpr uint32_t idesc_qk = mma_idesc_f16(fmt, 128, 128, 0, 0);
+    constexpr uint32_t idesc_pv = mma_idesc_f16(fmt, 128, D, 0, 1);
+    uint32_t kv_it = 0, q_it = 0;
+    uint32_t pv_it0 = 0, pv_it1 = 0, units0 = 0, units1 = 0;
+    bool ok = true;
+    // Descriptors are built once per operand tile; a k-step only moves the
+    // start-address field (bits 0-13, in 16-byte units).
+    auto issue_qk = [&](int i, int stage) {
+      const uint64_t qd = smem_desc_sw128(sbase + L::kQ + i * L::kTileBytes, 16, 1024);
+      const uint64_t kd = smem_desc_sw128(sbase + L::kK + stage * L::kTileBytes, 16, 1024);
+      const uint32_t d_col = tmem + (i == 0 ? L::kColS0 : L::kColS1);
 #pragma unroll 1
-        for (int s = 0; s < D / 16; ++s) {
-          const uint64_t off = ((s >> 2) * L::kChunkBytes + (s & 3) * 32) >> 4;
-          tc_mma_ss(d_col, qd + off, kd + off, idesc_qk, s > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int i, int stage, bool first) {
-        const uint64_t vd =
-            smem_desc_sw128(sbase + L::kV + stage * L::kTileBytes, L::kChunkBytes, 1024);
-        const uint32_t d_col = tmem + (i == 0 ? L::kColO0 : L::kColO1);
-        const uint32_t p_col = tmem + (i == 0 ? L::kColS0 : L::kColS1);
+      for (int s = 0; s < D / 16; ++s) {
+        const uint64_t off = ((s >> 2) * L::kChunkBytes + (s & 3) * 32) >> 4;
+        tc_mma_ss(d_col, qd + off, kd + off, idesc_qk, s > 0 ? 1u : 0u);
+      }
+    };
+    // Both query tiles against one K tile, k-steps interleaved: two
+    // independent accumulator chains keep the tensor pipe full.
+    auto issue_qk_pair = [&](int stage) {
+      const uint64_t qd0 = smem_desc_sw128(sbase + L::kQ, 16, 1024);
+      const uint64_t qd1 = smem_desc_sw128(sbase + L::kQ + L::kTileBytes, 16, 1024);
+      const uint64_t kd = smem_desc_sw128(sbase + L::kK + stage * L::kTileBytes, 16, 1024);
 #pragma unroll 1
-        for (int s = 0; s < kTile / 16; ++s) {
-          tc_mma_ts(d_col, p_col + 8 * s, vd + static_cast<uint64_t>(s * 2048 >> 4), idesc_pv,
-                    (first && s == 0) ? 0u : 1u);
-        }
-      };
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const Unit w = decode_unit(p, u);
-        const int n = w.n_full + w.n_part;
-        const int nq = 1 + w.h1valid;
-        if (n > 0) {
-          if (!mbar_wait(bar(L::kQFull), q_it & 1, abort_flag, p.err)) { ok = false; break; }
-          ++q_it;
-          // S_i(0) = Q_i K(0)^T
-          {
-            const int stage = kv_it % L::kStages;
-            if (!mbar_wait(bar(L::kKFull + stage), (kv_it / L::kStages) & 1, abort_flag, p.err)) {
-              ok = false;
-              break;
+      for (int s = 0; s < D / 16; ++s) {
+        const uint64_t off = ((s >> 2) * L::kChunkBytes + (s & 3) * 32) >> 4;
+        tc_mma_ss(tmem + L::kColS0, qd0 + off, kd + off, idesc_qk, s > 0 ? 1u : 0u);
+        tc_mma_ss(tmem + L::kColS1, qd1 + off, kd + off, idesc_qk, s > 0 ? 1u : 0u);
+      }
+    };
+    auto issue_pv = [&](int i, int stage, bool first) {
+      const uint64_t vd =
+          smem_desc_sw128(sbase + L::kV + stage * L::kTileBytes, L::kChunkBytes, 1024);
+      const uint32_t d_col = tmem + (i == 0 ? L::kColO0 : L::kColO1);
+      const uint32_t p_col = tmem + (i == 0 ? L::kColS0 : L::kColS1);
+#pragma unroll 1
+      for (int s = 0; s < kTile / 16; ++s) {
+        tc_mma_ts(d_col, p_col + 8 * s, vd + static_cast<uint64_t>(s * 2048 >> 4), idesc_pv,
+                  (first && s == 0) ? 0u : 1u);
+      }
+    };
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit w = decode_unit(p, u);
+      const int n = w.n_full + w.n_part;
+      const int nq = 1 + w.h1valid;
+      if (n > 0) {
+        if (!mbar_wait_warp(bar(L::kQFull), q_it & 1, abort_flag, p.err)) { ok = false; break; }
+        ++q_it;
+        // S_i(0) = Q_i K(0)^T.  The previous unit's last PV_i read P_i from
+        // S_i's columns; it was issued earlier by this lane, and the MMAs of
+        // one issuing thread execute in order.
+        {
+          const int stage = kv_it % L::kStages;
+          if (!mbar_wait_warp(bar(L::kKFull + stage), (kv_it / L::kStages) & 1, abort_flag,
+                              p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+            if (nq == 2) {
+              issue_qk_pair(stage);
+              tc_commit(bar(L::kSBar + 0));
+              tc_commit(bar(L::kSBar + 1));
+            } else {
+              issue_qk(0, stage);
+              tc_commit(bar(L::kSBar + 0));
             }
-            tc_fence_after();
-            for (int i = 0; i < nq && ok; ++i) {
-              if (pv_it[i] > 0 &&
-                  !mbar_wait(bar(L::kOBar + i), (pv_it[i] - 1) & 1, abort_flag, p.err)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              issue_qk(i, stage);
-              tc_commit(bar(L::kSBar + i));
-            }
-            if (!ok) break;
             tc_commit(bar(L::kKEmpty + stage));
             if (n == 1) tc_commit(bar(L::kQEmpty));
           }
-          for (int j = 0; j < n && ok; ++j) {
-            const int stage = kv_it % L::kStages;
-            const uint32_t ph = (kv_it / L::kStages) & 1;
-            const int nstage = (kv_it + 1) % L::kStages;
-            const uint32_t nph = ((kv_it + 1) / L::kStages) & 1;
-            if (!mbar_wait(bar(L::kVFull + stage), ph, abort_flag, p.err)) { ok = false; break; }
-            if (j + 1 < n &&
-                !mbar_wait(bar(L::kKFull + nstage), nph, abort_flag, p.err)) {
+          __syncwarp();
+        }
+        for (int j = 0; j < n && ok; ++j) {
+          const int stage = kv_it % L::kStages;
+          const uint32_t ph = (kv_it / L::kStages) & 1;
+          const int nstage = (kv_it + 1) % L::kStages;
+          const uint32_t nph = ((kv_it + 1) / L::kStages) & 1;
+          if (!mbar_wait_warp(bar(L::kVFull + stage), ph, abort_flag, p.err)) { ok = false; break; }
+          for (int i = 0; i < nq && ok; ++i) {
+            const uint32_t pvi = i == 0 ? pv_it0 : pv_it1;
+            const uint32_t uni = i == 0 ? units0 : units1;
+            if (!mbar_wait_warp(bar(L::kPBar + i), pvi & 1, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
+            if (j == 0 && uni > 0 &&
+                !mbar_wait_warp(bar(L::kOFree + i), (uni - 1) & 1, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
+            if (i == 0 && j + 1 < n &&
+                !mbar_wait_warp(bar(L::kKFull + nstage), nph, abort_flag, p.err)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            for (int i = 0; i < nq && ok; ++i) {
+            if (elect_one()) {
               // O_i += P_i(j) V(j)
-              if (!mbar_wait(bar(L::kPBar + i), pv_it[i] & 1, abort_flag, p.err)) { ok = false; break; }
-              if (j == 0 && units[i] > 0 &&
-                  !mbar_wait(bar(L::kOFree + i), (units[i] - 1) & 1, abort_flag, p.err)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
               issue_pv(i, stage, j == 0);
               tc_commit(bar(L::kOBar + i));
-              ++pv_it[i];
-              // S_i(j+1) = Q_i K(j+1)^T once P_i(j) has been consumed
+              // S_i(j+1) = Q_i K(j+1)^T right behind it: the MMAs of one
+              // issuing thread execute in order, so PV_i(j) has read P_i(j)
+              // before QK_i(j+1) rewrites those TMEM columns.
               if (j + 1 < n) {
-                if (!mbar_wait(bar(L::kOBar + i), (pv_it[i] - 1) & 1, abort_flag, p.err)) {
-                  ok = false;
-                  break;
-                }
-                tc_fence_after();
                 issue_qk(i, nstage);
                 tc_commit(bar(L::kSBar + i));
               }
             }
-            if (!ok) break;
+            __syncwarp();
+            if (i == 0) ++pv_it0; else ++pv_it1;
+          }
+          if (!ok) break;
+          if (elect_one()) {
             tc_commit(bar(L::kVEmpty + stage));
             if (j + 1 < n) {
               tc_commit(bar(L::kKEmpty + nstage));
               if (j + 2 == n) tc_commit(bar(L::kQEmpty));
             }
-            ++kv_it;
           }
+          __syncwarp();
+          ++kv_it;
         }
-        units[0] += 1;
-        units[1] += w.h1valid;
       }
-      if (!ok) {
-        tc_commit(bar(L::kDrain));
-        drain_wait(bar(L::kDrain), 0, p.err);
-      }
+      units0 += 1;
+      units1 += w.h1valid;
+    }
+    if (!ok) {
+      if (elect_one()) tc_commit(bar(L::kDrain));
+      __syncwarp();
+      drain_wait(bar(L::kDrain), 0, p.err);
     }
    }
   } else {
@@ -397,21 +434,29 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
         if (p.causal) causal_lim = q + p.Lk - p.Lq;
       }
 
+      // DFlash scores are scaled inside the exponent (one FFMA per element);
+      // explicit-policy scores are scaled when the bias is added.
+      const float exp_scale = POLICY == kPolicyDflash ? p.scale_log2 : 1.0f;
       float m_ref = -INFINITY, l_sum = 0.f;
+      bool partial_next = false;
+      int kt_next = n > 0 ? tile_at(p, w, 0, &partial_next) : 0;
       for (int j = 0; j < n && ok; ++j) {
-        bool partial;
-        const int kt = tile_at(p, w, j, &partial);
+        const int kt = kt_next;
+        const bool partial = partial_next;
+        if (j + 1 < n) kt_next = tile_at(p, w, j + 1, &partial_next);  // prefetch
         const int k0 = kt * kTile;
         if (!mbar_wait(bar(L::kSBar + qi), it & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         float x[kTile];
+        {
+          uint32_t* xr = reinterpret_cast<uint32_t*>(x);
 #pragma unroll
-        for (int c = 0; c < kTile / 32; ++c) {
-          uint32_t raw[32];
-          tmem_ld32(s_col + 32 * c, raw);
+          for (int c = 0; c < kTile / 32; ++c) tmem_ld32_at(s_col + 32 * c, xr + 32 * c);
           tc_wait_ld();
+        }
+        if (POLICY == kPolicyExplicit) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) x[32 * c + e] = __uint_as_float(raw[e]) * p.scale_log2;
+          for (int c = 0; c < kTile; ++c) x[c] *= p.scale_log2;
         }
         if (POLICY == kPolicyExplicit && p.has_bias) {
           if (p.bias.dtype == SMA_FP32) {
@@ -475,10 +520,17 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
             }
           }
         }
-        float mx = -INFINITY;
+        // Row max: eight independent chains, then a tree.
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, x[c]);
-        const float m_new = fmaxf(m_ref, mx);
+        for (int e = 0; e < 8; ++e) mx8[e] = x[e];
+#pragma unroll
+        for (int c = 8; c < kTile; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
+#pragma unroll
+        for (int w2 = 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+          for (int e = 0; e < w2; ++e) mx8[e] = fmaxf(mx8[e], mx8[e + w2]);
+        const float m_new = fmaxf(m_ref, mx8[0] * exp_scale);
         // Lazy rescale of O: only when the max grew by more than 2^8.
         const bool need = (m_ref != -INFINITY) && (m_new > m_ref + 8.0f);
         if (__any_sync(0xffffffffu, need)) {
@@ -503,15 +555,18 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
         }
         if (m_ref == -INFINITY) m_ref = m_new;
         const float msub = m_ref == -INFINITY ? 0.f : m_ref;
-        float ls = 0.f;
+        float ls8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ls8[e] = 0.f;
 #pragma unroll
         for (int c = 0; c < kTile / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(x[32 * c + 2 * e] - msub);
-            const float p1 = fast_exp2(x[32 * c + 2 * e + 1] - msub);
-            ls += p0 + p1;
+            const float p0 = fast_exp2(fmaf(x[32 * c + 2 * e], exp_scale, -msub));
+            const float p1 = fast_exp2(fmaf(x[32 * c + 2 * e + 1], exp_scale, -msub));
+            ls8[(2 * e) & 7] += p0;
+            ls8[(2 * e + 1) & 7] += p1;
             pk[e] = DT == SMA_BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
           }
           // P columns [16c, 16c+16) of the packed pairs
@@ -524,7 +579,11 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
               "r"(pk[12]), "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
               : "memory");
         }
-        l_sum += ls;
+#pragma unroll
+        for (int w2 = 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+          for (int e = 0; e < w2; ++e) ls8[e] += ls8[e + w2];
+        l_sum += ls8[0];
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(bar(L::kPBar + qi));
