@@ -58,18 +58,19 @@ constexpr uint32_t kTmemCols = 512;
 
 template <int D>
 struct Layout {
-  static constexpr int kStages = D == 128 ? 2 : 4;
+  static constexpr int kKStages = D == 128 ? 3 : 4;  // K runs ahead of V
+  static constexpr int kVStages = D == 128 ? 2 : 4;
   static constexpr uint32_t kChunkBytes = kTile * 128;  // 64 columns x 128 rows, 128B-swizzled
   static constexpr uint32_t kTileBytes = kTile * D * 2;
   static constexpr int kChunks = D / 64;
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kK = kQ + 2 * kTileBytes;
-  static constexpr uint32_t kV = kK + kStages * kTileBytes;
-  static constexpr uint32_t kBars = kV + kStages * kTileBytes;
+  static constexpr uint32_t kV = kK + kKStages * kTileBytes;
+  static constexpr uint32_t kBars = kV + kVStages * kTileBytes;
   // barrier slots
-  static constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + kStages,
-                       kVFull = kKEmpty + kStages, kVEmpty = kVFull + kStages,
-                       kSBar = kVEmpty + kStages, kPBar = kSBar + 2, kOBar = kPBar + 2,
+  static constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + kKStages,
+                       kVFull = kKEmpty + kKStages, kVEmpty = kVFull + kVStages,
+                       kSBar = kVEmpty + kVStages, kPBar = kSBar + 2, kOBar = kPBar + 2,
                        kOFree = kOBar + 2, kDrain = kOFree + 2, kNumBars = kDrain + 1;
   static constexpr uint32_t kTmemSlot = kBars + 8 * kNumBars;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
@@ -142,9 +143,11 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
   if (threadIdx.x == 0) {
     mbar_init(bar(L::kQFull), 1);
     mbar_init(bar(L::kQEmpty), 1);
-    for (int s = 0; s < L::kStages; ++s) {
+    for (int s = 0; s < L::kKStages; ++s) {
       mbar_init(bar(L::kKFull + s), 1);
       mbar_init(bar(L::kKEmpty + s), 1);
+    }
+    for (int s = 0; s < L::kVStages; ++s) {
       mbar_init(bar(L::kVFull + s), 1);
       mbar_init(bar(L::kVEmpty + s), 1);
     }
@@ -202,29 +205,33 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
       for (int j = 0; j < n && ok; ++j) {
         const int kt = kt_next;
         if (j + 1 < n) kt_next = tile_at(p, w, j + 1, &partial_next);
-        const int stage = kv_k % L::kStages;
-        const uint32_t use = kv_k / L::kStages;
-        if (use > 0 && !mbar_wait_warp(bar(L::kKEmpty + stage), (use - 1) & 1, abort_flag, p.err)) {
+        const int kstage = kv_k % L::kKStages;
+        const uint32_t kuse = kv_k / L::kKStages;
+        if (kuse > 0 &&
+            !mbar_wait_warp(bar(L::kKEmpty + kstage), (kuse - 1) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
         if (elect_one()) {
-          mbar_arrive_expect_tx(bar(L::kKFull + stage), L::kTileBytes);
+          mbar_arrive_expect_tx(bar(L::kKFull + kstage), L::kTileBytes);
           for (int c = 0; c < L::kChunks; ++c)
-            tma_load_4d(sbase + L::kK + stage * L::kTileBytes + c * L::kChunkBytes, &map_k,
-                        bar(L::kKFull + stage), c * 64, w.hk, kt * kTile, w.b);
+            tma_load_4d(sbase + L::kK + kstage * L::kTileBytes + c * L::kChunkBytes, &map_k,
+                        bar(L::kKFull + kstage), c * 64, w.hk, kt * kTile, w.b);
         }
         __syncwarp();
         ++kv_k;
-        if (use > 0 && !mbar_wait_warp(bar(L::kVEmpty + stage), (use - 1) & 1, abort_flag, p.err)) {
+        const int vstage = kv_v % L::kVStages;
+        const uint32_t vuse = kv_v / L::kVStages;
+        if (vuse > 0 &&
+            !mbar_wait_warp(bar(L::kVEmpty + vstage), (vuse - 1) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
         if (elect_one()) {
-          mbar_arrive_expect_tx(bar(L::kVFull + stage), L::kTileBytes);
+          mbar_arrive_expect_tx(bar(L::kVFull + vstage), L::kTileBytes);
           for (int c = 0; c < L::kChunks; ++c)
-            tma_load_4d(sbase + L::kV + stage * L::kTileBytes + c * L::kChunkBytes, &map_v,
-                        bar(L::kVFull + stage), c * 64, w.hk, kt * kTile, w.b);
+            tma_load_4d(sbase + L::kV + vstage * L::kTileBytes + c * L::kChunkBytes, &map_v,
+                        bar(L::kVFull + vstage), c * 64, w.hk, kt * kTile, w.b);
         }
         __syncwarp();
         ++kv_v;
@@ -232,14 +239,16 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
     }
     if (!ok) {
       // Drain: every copy this warp issued must land before the CTA exits.
-      for (uint32_t t = 0; t < static_cast<uint32_t>(L::kStages); ++t) {
+      for (uint32_t t = 0; t < static_cast<uint32_t>(L::kKStages); ++t) {
         if (kv_k > t) {
           const uint32_t nn = kv_k - 1 - t;
-          drain_wait(bar(L::kKFull + nn % L::kStages), (nn / L::kStages) & 1, p.err);
+          drain_wait(bar(L::kKFull + nn % L::kKStages), (nn / L::kKStages) & 1, p.err);
         }
+      }
+      for (uint32_t t = 0; t < static_cast<uint32_t>(L::kVStages); ++t) {
         if (kv_v > t) {
           const uint32_t nn = kv_v - 1 - t;
-          drain_wait(bar(L::kVFull + nn % L::kStages), (nn / L::kStages) & 1, p.err);
+          drain_wait(bar(L::kVFull + nn % L::kVStages), (nn / L::kVStages) & 1, p.err);
         }
       }
       if (q_it > 0) drain_wait(bar(L::kQFull), (q_it - 1) & 1, p.err);
@@ -301,8 +310,8 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
         // S_i's columns; it was issued earlier by this lane, and the MMAs of
         // one issuing thread execute in order.
         {
-          const int stage = kv_it % L::kStages;
-          if (!mbar_wait_warp(bar(L::kKFull + stage), (kv_it / L::kStages) & 1, abort_flag,
+          const int stage = kv_it % L::kKStages;
+          if (!mbar_wait_warp(bar(L::kKFull + stage), (kv_it / L::kKStages) & 1, abort_flag,
                               p.err)) {
             ok = false;
             break;
@@ -323,10 +332,10 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           __syncwarp();
         }
         for (int j = 0; j < n && ok; ++j) {
-          const int stage = kv_it % L::kStages;
-          const uint32_t ph = (kv_it / L::kStages) & 1;
-          const int nstage = (kv_it + 1) % L::kStages;
-          const uint32_t nph = ((kv_it + 1) / L::kStages) & 1;
+          const int stage = kv_it % L::kVStages;
+          const uint32_t ph = (kv_it / L::kVStages) & 1;
+          const int nstage = (kv_it + 1) % L::kKStages;
+          const uint32_t nph = ((kv_it + 1) / L::kKStages) & 1;
           if (!mbar_wait_warp(bar(L::kVFull + stage), ph, abort_flag, p.err)) { ok = false; break; }
           for (int i = 0; i < nq && ok; ++i) {
             const uint32_t pvi = i == 0 ? pv_it0 : pv_it1;

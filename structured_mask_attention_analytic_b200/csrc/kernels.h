@@ -71,7 +71,7 @@ struct AttnProblem {
 // (b, kv head) the `group` query heads are the rows.
 struct DecodeProblem {
   int dtype;
-  int B, H, KVH, Lk, d, group;
+  int B, H, KVH, Lk, Kpad, d, group;
   float scale_log2;
   const void* q; int64_t q_sb, q_sh;
   const void* k; int64_t k_sb, k_sr, k_sh;
@@ -80,7 +80,7 @@ struct DecodeProblem {
   float* lse;  // [B, H] (q_len 1) or null
   int has_mask, has_bias;
   AuxView mask, bias;
-  int splits, chunk;       // split-KV: keys [s*chunk, min((s+1)*chunk, Lk))
+  int splits, chunk;       // split-KV: keys [s*chunk, min((s+1)*chunk, Lk)), chunk % 128 == 0
   float* part_o;           // [B, H, splits, d]
   float* part_ml;          // [B, H, splits, 2]  (max in log2 units, sum)
   int* err;

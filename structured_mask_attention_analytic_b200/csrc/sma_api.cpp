@@ -191,16 +191,17 @@ MaskedGeom masked_geom(int32_t B, int32_t H, int32_t KVH, int32_t Lq, int32_t Lk
   g.KT = static_cast<int>(ceil_div(Lk, kTile));
   g.decode = Lq == 1;
   if (g.decode) {
-    // split-KV: about two CTAs per SM of a 148-SM part, chunks of >= 256 keys
+    // split-KV: up to about two CTAs per SM of a 148-SM part (one wave), each
+    // streaming a chunk of at least 1024 keys
     const int rows_groups = (group + 7) / 8;
     const int64_t base_ctas = static_cast<int64_t>(B) * KVH * rows_groups;
-    int splits = static_cast<int>(ceil_div(296, base_ctas));
-    const int max_splits = static_cast<int>(ceil_div(Lk, 256));
+    int splits = static_cast<int>(296 / base_ctas);
+    const int max_splits = static_cast<int>(ceil_div(Lk, 1024));
     if (splits > max_splits) splits = max_splits;
     if (splits > 64) splits = 64;
     if (splits < 1) splits = 1;
     g.splits = splits;
-    g.chunk = static_cast<int>(ceil_div(Lk, splits));
+    g.chunk = static_cast<int>(round_up(ceil_div(Lk, splits), kTile));
     g.part_o = 0;
     g.part_ml = align256(static_cast<size_t>(B) * H * splits * d * 4);
     g.total = align256(g.part_ml + static_cast<size_t>(B) * H * splits * 2 * 4);
@@ -450,6 +451,7 @@ sma_status masked_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
     DecodeProblem dp{};
     dp.dtype = dtype;
     dp.B = batch; dp.H = heads; dp.KVH = kv_heads; dp.Lk = k_len; dp.d = head_dim;
+    dp.Kpad = static_cast<int>(round_up(k_len, kTile));
     dp.group = heads / kv_heads;
     dp.scale_log2 = scale_log2;
     dp.q = q; dp.q_sb = q_strides[0]; dp.q_sh = q_strides[2];

@@ -19,10 +19,7 @@
 namespace sma {
 namespace {
 
-constexpr int kTkThreads = 256;
-constexpr int kTkWarps = kTkThreads / 32;
 constexpr int kPerThread = 8;
-constexpr int kRowStep = kTkThreads * kPerThread;
 
 template <int DT>
 struct KeyTraits;
@@ -99,10 +96,14 @@ __device__ __forceinline__ void row_keys(const RowCtx& rc, int c, uint32_t (&key
   }
 }
 
-template <int DT>
-__global__ void __launch_bounds__(kTkThreads)
+// NT threads per row: 1024 when there are few rows (latency), 256 otherwise.
+template <int DT, int NT>
+__global__ void __launch_bounds__(NT)
 topk_mask_kernel(const TopkProblem p) {
   using T = KeyTraits<DT>;
+  constexpr int kTkThreads = NT;
+  constexpr int kTkWarps = NT / 32;
+  constexpr int kRowStep = NT * kPerThread;
   __shared__ uint32_t hist[kTkWarps][256];
   __shared__ uint32_t total[256];
   __shared__ uint32_t s_digit, s_remaining, s_scan[kTkWarps];
@@ -150,8 +151,8 @@ topk_mask_kernel(const TopkProblem p) {
       }
       __syncthreads();
       // total[d] and the digit where the running count from the top reaches `remaining`.
-      {
-        const int d = threadIdx.x;  // 256 threads, one per digit value
+      if (threadIdx.x < 256) {
+        const int d = threadIdx.x;
         uint32_t cnt = 0;
 #pragma unroll
         for (int w = 0; w < kTkWarps; ++w) cnt += hist[w][d];
@@ -159,23 +160,26 @@ topk_mask_kernel(const TopkProblem p) {
       }
       __syncthreads();
       {
-        // suffix sums: above[d] = sum of total[d'] for d' > d
-        const int d = 255 - threadIdx.x;  // reversed so an inclusive prefix scan gives suffixes
-        uint32_t v = total[d];
+        // suffix sums over digits: above[d] = sum of total[d'] for d' > d
+        // (threads 0..255 take digits 255..0, so a prefix scan gives suffixes)
+        const int d = 255 - threadIdx.x;
+        const uint32_t v = threadIdx.x < 256 ? total[d] : 0u;
         uint32_t incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
           if (lane >= o) incl += t;
         }
-        if (lane == 31) s_scan[warp] = incl;
+        if (lane == 31 && warp < 8) s_scan[warp] = incl;
         __syncthreads();
-        uint32_t wbase = 0;
-        for (int w = 0; w < warp; ++w) wbase += s_scan[w];
-        const uint32_t above = wbase + incl - v;
-        if (above < remaining && remaining <= above + v) {
-          s_digit = static_cast<uint32_t>(d);
-          s_remaining = remaining - above;
+        if (threadIdx.x < 256) {
+          uint32_t wbase = 0;
+          for (int w = 0; w < warp; ++w) wbase += s_scan[w];
+          const uint32_t above = wbase + incl - v;
+          if (above < remaining && remaining <= above + v) {
+            s_digit = static_cast<uint32_t>(d);
+            s_remaining = remaining - above;
+          }
         }
       }
       __syncthreads();
@@ -239,15 +243,22 @@ topk_mask_kernel(const TopkProblem p) {
   }
 }
 
+template <int NT>
+void launch_nt(const TopkProblem& p, unsigned grid, cudaStream_t stream) {
+  if (p.bias_dtype == SMA_BF16) topk_mask_kernel<SMA_BF16, NT><<<grid, NT, 0, stream>>>(p);
+  else if (p.bias_dtype == SMA_FP16) topk_mask_kernel<SMA_FP16, NT><<<grid, NT, 0, stream>>>(p);
+  else topk_mask_kernel<SMA_FP32, NT><<<grid, NT, 0, stream>>>(p);
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const TopkProblem& p, cudaStream_t stream) {
   const int64_t rows = p.b_sizes[0] * p.b_sizes[1] * p.b_sizes[2];
   if (rows == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>(rows);
-  if (p.bias_dtype == SMA_BF16) topk_mask_kernel<SMA_BF16><<<grid, kTkThreads, 0, stream>>>(p);
-  else if (p.bias_dtype == SMA_FP16) topk_mask_kernel<SMA_FP16><<<grid, kTkThreads, 0, stream>>>(p);
-  else topk_mask_kernel<SMA_FP32><<<grid, kTkThreads, 0, stream>>>(p);
+  // Few rows: one wide CTA per row finishes each row sooner.
+  if (rows < 2 * num_sms()) launch_nt<1024>(p, grid, stream);
+  else launch_nt<256>(p, grid, stream);
   return cudaGetLastError();
 }
 
