@@ -443,9 +443,13 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
         if (p.causal) causal_lim = q + p.Lk - p.Lq;
       }
 
-      // DFlash scores are scaled inside the exponent (one FFMA per element);
-      // explicit-policy scores are scaled when the bias is added.
-      const float exp_scale = POLICY == kPolicyDflash ? p.scale_log2 : 1.0f;
+      // Scores are scaled inside the exponent (one FFMA per element).  A bias
+      // is added as b / scale beforehand, so that scale * (s + b / scale) *
+      // log2(e) = (scale * s + b) * log2(e).
+      const float exp_scale = p.scale_log2;
+      const float bias_mul = kLog2e / p.scale_log2;
+      const int causal_off = p.Lk - p.Lq;
+      const bool mask_bcast_q = POLICY == kPolicyExplicit && p.has_mask && p.mask.sq == 0;
       float m_ref = -INFINITY, l_sum = 0.f;
       bool partial_next = false;
       int kt_next = n > 0 ? tile_at(p, w, 0, &partial_next) : 0;
@@ -463,19 +467,15 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           for (int c = 0; c < kTile / 32; ++c) tmem_ld32_at(s_col + 32 * c, xr + 32 * c);
           tc_wait_ld();
         }
-        if (POLICY == kPolicyExplicit) {
-#pragma unroll
-          for (int c = 0; c < kTile; ++c) x[c] *= p.scale_log2;
-        }
         if (POLICY == kPolicyExplicit && p.has_bias) {
           if (p.bias.dtype == SMA_FP32) {
 #pragma unroll
             for (int c = 0; c < kTile; c += 4) {
               const float4 a = *reinterpret_cast<const float4*>(brow + (k0 + c) * 4);
-              x[c] = fmaf(a.x, kLog2e, x[c]);
-              x[c + 1] = fmaf(a.y, kLog2e, x[c + 1]);
-              x[c + 2] = fmaf(a.z, kLog2e, x[c + 2]);
-              x[c + 3] = fmaf(a.w, kLog2e, x[c + 3]);
+              x[c] = fmaf(a.x, bias_mul, x[c]);
+              x[c + 1] = fmaf(a.y, bias_mul, x[c + 1]);
+              x[c + 2] = fmaf(a.z, bias_mul, x[c + 2]);
+              x[c + 3] = fmaf(a.w, bias_mul, x[c + 3]);
             }
           } else if (p.bias.dtype == SMA_BF16) {
 #pragma unroll
@@ -484,8 +484,9 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
               const uint32_t wv[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                x[c + 2 * e] = fmaf(__uint_as_float(wv[e] << 16), kLog2e, x[c + 2 * e]);
-                x[c + 2 * e + 1] = fmaf(__uint_as_float(wv[e] & 0xffff0000u), kLog2e, x[c + 2 * e + 1]);
+                x[c + 2 * e] = fmaf(__uint_as_float(wv[e] << 16), bias_mul, x[c + 2 * e]);
+                x[c + 2 * e + 1] =
+                    fmaf(__uint_as_float(wv[e] & 0xffff0000u), bias_mul, x[c + 2 * e + 1]);
               }
             }
           } else {
@@ -496,13 +497,13 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[e]));
-                x[c + 2 * e] = fmaf(f.x, kLog2e, x[c + 2 * e]);
-                x[c + 2 * e + 1] = fmaf(f.y, kLog2e, x[c + 2 * e + 1]);
+                x[c + 2 * e] = fmaf(f.x, bias_mul, x[c + 2 * e]);
+                x[c + 2 * e + 1] = fmaf(f.y, bias_mul, x[c + 2 * e + 1]);
               }
             }
           }
         }
-        if (partial || !row_valid) {
+        if (partial) {  // warp-uniform
           if (POLICY == kPolicyDflash) {
             const uint32_t wc = static_cast<uint32_t>(chi - clo);
             const uint32_t wd = static_cast<uint32_t>(dhi - dlo);
@@ -511,23 +512,48 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
             for (int c = 0; c < kTile; ++c) {
               const bool keep = static_cast<uint32_t>(c + ac) < wc ||
                                 static_cast<uint32_t>(c + ad) < wd;
-              x[c] = (keep && row_valid) ? x[c] : -INFINITY;
+              x[c] = keep ? x[c] : -INFINITY;
             }
           } else {
+            // Columns c >= lim fail the key-length or causal bound; both bounds
+            // are checked only on tiles they can cut (uniform per tile).
+            int lim = kTile;
+            if (k0 + kTile > p.Lk) lim = min(lim, p.Lk - k0);
+            if (p.causal && k0 + kTile - 1 > w.qt * kTile + causal_off)
+              lim = min(lim, causal_lim - k0 + 1);
+            if (mask_bcast_q) {
+              // One mask row for every query row: 4 ballots turn the tile's 128
+              // bytes into bits, bit l of word j = column 4 l + j.
+              const uint32_t mw = *reinterpret_cast<const uint32_t*>(mrow + k0 + 4 * lane);
+              uint32_t bits[4];
 #pragma unroll
-            for (int c = 0; c < kTile; c += 16) {
-              uint4 mv = make_uint4(0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u);
-              if (p.has_mask) mv = *reinterpret_cast<const uint4*>(mrow + k0 + c);
-              const uint32_t wv[4] = {mv.x, mv.y, mv.z, mv.w};
+              for (int j = 0; j < 4; ++j)
+                bits[j] = __ballot_sync(0xffffffffu, ((mw >> (8 * j)) & 0xffu) != 0u);
 #pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const int k = k0 + c + e;
-                const bool keep = ((wv[e >> 2] >> (8 * (e & 3))) & 0xffu) != 0u && k < p.Lk &&
-                                  k <= causal_lim && row_valid;
-                x[c + e] = keep ? x[c + e] : -INFINITY;
+              for (int c = 0; c < kTile; ++c) {
+                const bool keep = ((bits[c & 3] >> (c >> 2)) & 1u) != 0u && c < lim;
+                x[c] = keep ? x[c] : -INFINITY;
               }
+            } else if (p.has_mask) {
+#pragma unroll
+              for (int c = 0; c < kTile; c += 16) {
+                const uint4 mv = *reinterpret_cast<const uint4*>(mrow + k0 + c);
+                const uint32_t wv[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  const bool keep = ((wv[e >> 2] >> (8 * (e & 3))) & 0xffu) != 0u && (c + e) < lim;
+                  x[c + e] = keep ? x[c + e] : -INFINITY;
+                }
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < kTile; ++c) x[c] = c < lim ? x[c] : -INFINITY;
             }
           }
+        }
+        if (!row_valid) {
+#pragma unroll
+          for (int c = 0; c < kTile; ++c) x[c] = -INFINITY;
         }
         // Row max: eight independent chains, then a tree.
         float mx8[8];
