@@ -281,13 +281,20 @@ def run_ours(args, rank, world, dev):
     return res
 
 
-def run_details(sma, dev, stream, peaks):
-    """Other workloads, each timed alone (events on the launch stream)."""
+DETAILS = ("dflash", "broadcast_prefill", "broadcast_decode", "topk", "topk_wide")
+
+
+def run_details(sma, dev, stream, peaks, only=None):
+    """Other workloads, each timed alone (events on the launch stream).
+    ``only`` restricts the run to one group of DETAILS."""
     out = {}
     pk_t, pk_b = float(peaks["bf16_tflops"]), float(peaks["hbm_gbs"])
 
+    def want(name):
+        return only is None or only == name
+
     # DFlash: sliding layer of the long-context workload, both training layers
-    for w in (wl.DFLASH_LONG_SLIDING, wl.DFLASH_TRAIN_FULL, wl.DFLASH_TRAIN_SLIDING):
+    for w in ((wl.DFLASH_LONG_SLIDING, wl.DFLASH_TRAIN_FULL, wl.DFLASH_TRAIN_SLIDING) if want("dflash") else ()):
         q, k, v, anchors = dflash_case(w, dev)
         bmap = sma.dfa_block_map(anchors, w.ctx_len, w.block_size, w.is_causal, w.layer_type, w.sliding_window)
         kept = int((bmap[0] + bmap[2]).sum().item())
@@ -298,7 +305,21 @@ def run_details(sma, dev, stream, peaks):
         out[w.name] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / pk_t, "kept_tiles": kept}
         del q, k, v, o
 
-    # broadcast mask/bias prefill
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    if want("broadcast_prefill"):
+        _detail_prefill(sma, dev, stream, out, pk_t)
+    if want("broadcast_decode"):
+        _detail_decode(sma, dev, stream, out, pk_b, flush)
+    if want("topk"):
+        _detail_topk(sma, dev, stream, out, pk_t, pk_b, flush)
+    if want("topk_wide"):
+        _detail_topk_wide(sma, dev, stream, out, pk_b)
+    del flush
+    torch.cuda.empty_cache()
+    return out
+
+
+def _detail_prefill(sma, dev, stream, out, pk_t):
     w = wl.BROADCAST_PREFILL
     q, k, v, mask, bias = (None if t is None else t.to(dev) for t in wl.masked_inputs(w))
     codes = sma.mask_tile_summary(mask, w.n_k)
@@ -314,13 +335,14 @@ def run_details(sma, dev, stream, peaks):
                    "mask_summary_ms": ms_sum, "mask_summary_GB/s": mbytes / (ms_sum * 1e-3) / 1e9}
     del q, k, v, mask, bias, o
 
+
+def _detail_decode(sma, dev, stream, out, pk_b, flush):
     # decode (swapped grouped-head path): HBM-bound
     w = wl.BROADCAST_DECODE
     q, k, v, mask, bias = (None if t is None else t.to(dev) for t in wl.masked_inputs(w))
     o = torch.empty_like(q)
     ws = torch.empty(sma.masked_attn_fwd_workspace_size(w.batch, w.heads, w.kv_heads, 1, w.n_k, w.head_dim),
                      dtype=torch.uint8, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def dec():
         sma.masked_attn_fwd(q, k, v, None, bias, False, out=o, workspace=ws)
@@ -341,6 +363,8 @@ def run_details(sma, dev, stream, peaks):
     out[w.name] = {"ms": ms, "GB/s": gbs, "frac_hbm_peak": gbs / pk_b, "bytes": nbytes}
     del q, k, v, bias, o
 
+
+def _detail_topk(sma, dev, stream, out, pk_t, pk_b, flush):
     # top-k mask, then attention under it
     w = wl.TOPK
     bias, pre = (t.to(dev) for t in wl.topk_inputs(w))
@@ -369,6 +393,8 @@ def run_details(sma, dev, stream, peaks):
     out[w.name + "_attention"] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / pk_t, "kept_tiles_per_bh": kept}
     del q, k, v, o, bias, pre, keep
 
+
+def _detail_topk_wide(sma, dev, stream, out, pk_b):
     w = wl.TOPK_WIDE
     bias, pre = (t.to(dev) for t in wl.topk_inputs(w))
     keep = torch.empty(bias.shape, dtype=torch.bool, device=dev)
@@ -376,9 +402,7 @@ def run_details(sma, dev, stream, peaks):
     nbytes = bias.numel() * 2 + pre.numel() + keep.numel()
     out[w.name + "_mask"] = {"ms": ms, "GB/s": nbytes / (ms * 1e-3) / 1e9, "frac_hbm_peak": nbytes / (ms * 1e-3) / 1e9 / pk_b,
                              "bytes": nbytes}
-    del bias, pre, keep, flush
-    torch.cuda.empty_cache()
-    return out
+    del bias, pre, keep
 
 
 # ---------------------------------------------------------------- oracle arm
@@ -492,6 +516,8 @@ def main():
     ap.add_argument("--no-details", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=DETAILS, default=None,
+                    help="time only this group of secondary workloads and print their JSON (profiling aid)")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture (reported as roofline.traffic)")
     args = ap.parse_args()
@@ -510,6 +536,12 @@ def main():
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.only is not None:
+        import structured_mask_attention_analytic_b200 as sma
+        peaks, _ = load_peaks()
+        print(json.dumps({"only": args.only,
+                          "details": run_details(sma, dev, torch.cuda.current_stream(dev), peaks, args.only)}))
+        return 0
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
