@@ -86,6 +86,15 @@ int32_t sma_abi_version(void);
  * Returns SMA_ERR_CUDA if the synchronisation itself failed. */
 sma_status sma_device_status(void* stream, int32_t* device_error);
 
+/* Diagnostic: launches one tiny kernel that waits, with the bounded wait every
+ * pipeline kernel of the library uses, on a barrier that nothing completes.
+ * After `timeout_ns` (1 ms .. 2 s) the wait gives up, the kernel records
+ * SMA_ERR_DEVICE_TIMEOUT in the device error word and returns normally, so
+ * the CUDA context stays usable.  dev_out (device, int64[2]) receives
+ * {1 if the wait gave up else 0, nanoseconds waited}.  Not part of the
+ * method; it checks the failure-reporting path without faulting the GPU. */
+sma_status sma_selftest_wait_timeout(int64_t timeout_ns, int64_t* dev_out, void* stream);
+
 /* ------------------------------------------------------------------------
  * DFlash mask description.
  *

@@ -19,4 +19,5 @@ from .ops import (  # noqa: F401
     masked_attn_fwd,
     masked_attn_fwd_workspace_size,
     round_up_k,
+    selftest_wait_timeout,
 )

@@ -67,7 +67,7 @@ __device__ __forceinline__ void global8(const void* base, int64_t idx, float (&f
 
 // grid: (splits, KVH * row_groups, B); rows [rg*G, rg*G+G) of the group.
 template <int D, int G, int DT>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(kDecThreads, G <= 4 ? 2 : 1)
 decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v) {
   using L = DecLayout<D, DT>;
@@ -199,62 +199,66 @@ decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap m
     // Per tile: every score of this warp's keys first, then one max / sum /
     // rescale per row, then the P.V pass -- no branch, so the G rows overlap.
     constexpr int kSteps = T / (kConsumerWarps * KPW);
+    constexpr int kSub = kSteps < 4 ? kSteps : 4;  // key-steps per online-softmax update
     bool ok = true;
     for (int t = 0; t < n_tiles && ok; ++t) {
       const int s = t % kRing;
       if (!mbar_wait_warp(full(s), (t / kRing) & 1, abort_flag, p.err)) { ok = false; break; }
       const uint8_t* kt = ring + s * kStageBytes;
       const uint8_t* vt = kt + kTileBytes;
-      float sc[kSteps][G];
 #pragma unroll
-      for (int st = 0; st < kSteps; ++st) {
-        const int c = (st * kConsumerWarps + warp) * KPW + slot;
-        float kf[8];
-        smem8<DT>(kt + (c * D + e0) * L::kEsz, kf);
+      for (int st0 = 0; st0 < kSteps; st0 += kSub) {
+        float sc[kSub][G];
+#pragma unroll
+        for (int st = 0; st < kSub; ++st) {
+          const int c = ((st0 + st) * kConsumerWarps + warp) * KPW + slot;
+          float kf[8];
+          smem8<DT>(kt + (c * D + e0) * L::kEsz, kf);
+#pragma unroll
+          for (int r = 0; r < G; ++r) {
+            float d = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) d = fmaf(qf[r][e], kf[e], d);
+#pragma unroll
+            for (int off = 1; off < LPK; off <<= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+            const bool keep = s_keep[(s * G + r) * T + c] != 0;
+            sc[st][r] = keep ? d + s_bias[(s * G + r) * T + c] : -INFINITY;
+          }
+        }
 #pragma unroll
         for (int r = 0; r < G; ++r) {
-          float d = 0.f;
+          float mx = sc[0][r];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) d = fmaf(qf[r][e], kf[e], d);
+          for (int st = 1; st < kSub; ++st) mx = fmaxf(mx, sc[st][r]);
 #pragma unroll
-          for (int off = 1; off < LPK; off <<= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-          const bool keep = s_keep[(s * G + r) * T + c] != 0;
-          sc[st][r] = keep ? d + s_bias[(s * G + r) * T + c] : -INFINITY;
-        }
-      }
+          for (int off = LPK; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+          const float m_new = fmaxf(m[r], mx);
+          const bool dead = m_new == -INFINITY;
+          const float alpha = dead ? 1.f : fast_exp2(m[r] - m_new);  // exp2(-inf) = 0
+          const float msub = dead ? 0.f : m_new;
+          float ps = 0.f;
 #pragma unroll
-      for (int r = 0; r < G; ++r) {
-        float mx = sc[0][r];
+          for (int st = 0; st < kSub; ++st) {
+            sc[st][r] = fast_exp2(sc[st][r] - msub);
+            ps += sc[st][r];
+          }
 #pragma unroll
-        for (int st = 1; st < kSteps; ++st) mx = fmaxf(mx, sc[st][r]);
+          for (int off = LPK; off < 32; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+          l[r] = l[r] * alpha + ps;
+          m[r] = m_new;
 #pragma unroll
-        for (int off = LPK; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float m_new = fmaxf(m[r], mx);
-        const bool dead = m_new == -INFINITY;
-        const float alpha = dead ? 1.f : fast_exp2(m[r] - m_new);  // exp2(-inf) = 0
-        const float msub = dead ? 0.f : m_new;
-        float ps = 0.f;
-#pragma unroll
-        for (int st = 0; st < kSteps; ++st) {
-          sc[st][r] = fast_exp2(sc[st][r] - msub);
-          ps += sc[st][r];
+          for (int e = 0; e < 8; ++e) o[r][e] *= alpha;
         }
 #pragma unroll
-        for (int off = LPK; off < 32; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-        l[r] = l[r] * alpha + ps;
-        m[r] = m_new;
+        for (int st = 0; st < kSub; ++st) {
+          const int c = ((st0 + st) * kConsumerWarps + warp) * KPW + slot;
+          float vf[8];
+          smem8<DT>(vt + (c * D + e0) * L::kEsz, vf);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[r][e] *= alpha;
-      }
+          for (int r = 0; r < G; ++r)
 #pragma unroll
-      for (int st = 0; st < kSteps; ++st) {
-        const int c = (st * kConsumerWarps + warp) * KPW + slot;
-        float vf[8];
-        smem8<DT>(vt + (c * D + e0) * L::kEsz, vf);
-#pragma unroll
-        for (int r = 0; r < G; ++r)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) o[r][e] = fmaf(sc[st][r], vf[e], o[r][e]);
+            for (int e = 0; e < 8; ++e) o[r][e] = fmaf(sc[st][r], vf[e], o[r][e]);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty(s));

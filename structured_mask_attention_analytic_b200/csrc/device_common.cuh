@@ -68,23 +68,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with parity `parity` to complete.  Returns
-// false (after recording the timeout) if it did not within the time limit or
-// if another role of the CTA already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* err) {
+// false (after recording the timeout) if it did not within `timeout_ns` of
+// %globaltimer time or if another role of the CTA already aborted.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity,
+                                              volatile int* abort_flag, int* err,
+                                              uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0u) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > SMA_WAIT_TIMEOUT_NS) {
+      if (global_timer_ns() - t0 > timeout_ns) {
         report_error(err, SMA_ERR_DEVICE_TIMEOUT);
         *abort_flag = 1;
         return false;
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int* err) {
+  return mbar_wait_for(bar, parity, abort_flag, err, SMA_WAIT_TIMEOUT_NS);
 }
 
 // Warp-uniform form: every lane waits, and the result is the same in all lanes.

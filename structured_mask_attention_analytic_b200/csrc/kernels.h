@@ -125,6 +125,9 @@ cudaError_t launch_topk(const TopkProblem& p, cudaStream_t stream);
 // sma_last_error) and returns `code`.
 int set_last_error(int code, const char* message);
 
+cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, int* err, int64_t* out,
+                                         cudaStream_t stream);
+
 // Device error word of the current device.
 int* device_error_word(cudaError_t* status);
 

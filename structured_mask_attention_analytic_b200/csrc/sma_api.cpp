@@ -256,6 +256,19 @@ sma_status sma_device_status(void* stream, int32_t* device_error) {
   return ok();
 }
 
+sma_status sma_selftest_wait_timeout(int64_t timeout_ns, int64_t* dev_out, void* stream) {
+  if (dev_out == nullptr) return fail(SMA_ERR_INVALID_ARG, "dev_out is NULL");
+  if (timeout_ns < 1000000 || timeout_ns > 2000000000)
+    return fail(SMA_ERR_INVALID_ARG, "timeout_ns must be in [1 ms, 2 s]");
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (err == nullptr) return cuda_fail(e, "device error word unavailable");
+  e = launch_wait_timeout_selftest(static_cast<uint64_t>(timeout_ns), err, dev_out,
+                                   static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch failed");
+  return ok();
+}
+
 sma_status dfa_block_map_dims(const dfa_mask_desc* desc, int32_t* q_tiles, int32_t* kv_tiles) {
   sma_status s = check_desc(desc);
   if (s != SMA_OK) return s;

@@ -283,3 +283,14 @@ def device_status(device=None) -> int:
     s = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     nat.check(_lib().sma_device_status(s, ctypes.byref(v)))
     return v.value
+
+
+def selftest_wait_timeout(timeout_ns: int, out: torch.Tensor) -> None:
+    """Diagnostic: a kernel waits on a barrier nothing completes, gives up
+    after ``timeout_ns`` and reports SMA_ERR_DEVICE_TIMEOUT in the device error
+    word (read it with ``device_status``).  ``out`` is int64[2] on the device:
+    {1 if the wait gave up, nanoseconds waited}."""
+    _require_cuda(out)
+    if out.dtype != torch.int64 or out.numel() < 2:
+        raise ValueError("out must be a CUDA int64 tensor with 2 elements")
+    nat.check(_lib().sma_selftest_wait_timeout(int(timeout_ns), _ptr(out), _stream(out)))
