@@ -263,29 +263,32 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
     uint32_t kv_it = 0, q_it = 0;
     uint32_t pv_it0 = 0, pv_it1 = 0, units0 = 0, units1 = 0;
     bool ok = true;
-    // Descriptors are built once per operand tile; a k-step only moves the
-    // start-address field (bits 0-13, in 16-byte units).
+    // Descriptors are built once per operand tile; a k-step only adds to the
+    // start-address field (bits 0-13 of the low word, in 16-byte units), so
+    // each MMA of the fully unrolled issue sequences costs one 32-bit add.
+    auto with_lo = [](uint64_t d, uint32_t add) -> uint64_t {
+      return (d & 0xffffffff00000000ull) | static_cast<uint32_t>(static_cast<uint32_t>(d) + add);
+    };
     auto issue_qk = [&](int i, int stage) {
       const uint64_t qd = smem_desc_sw128(sbase + L::kQ + i * L::kTileBytes, 16, 1024);
       const uint64_t kd = smem_desc_sw128(sbase + L::kK + stage * L::kTileBytes, 16, 1024);
       const uint32_t d_col = tmem + (i == 0 ? L::kColS0 : L::kColS1);
-#pragma unroll 1
+#pragma unroll
       for (int s = 0; s < D / 16; ++s) {
-        const uint64_t off = ((s >> 2) * L::kChunkBytes + (s & 3) * 32) >> 4;
-        tc_mma_ss(d_col, qd + off, kd + off, idesc_qk, s > 0 ? 1u : 0u);
+        const uint32_t off = ((s >> 2) * L::kChunkBytes + (s & 3) * 32) >> 4;
+        tc_mma_ss(d_col, with_lo(qd, off), with_lo(kd, off), idesc_qk, s > 0 ? 1u : 0u);
       }
     };
-    // Both query tiles against one K tile, k-steps interleaved: two
-    // independent accumulator chains keep the tensor pipe full.
+    // Both query tiles against one K tile, k-steps interleaved.
     auto issue_qk_pair = [&](int stage) {
       const uint64_t qd0 = smem_desc_sw128(sbase + L::kQ, 16, 1024);
       const uint64_t qd1 = smem_desc_sw128(sbase + L::kQ + L::kTileBytes, 16, 1024);
       const uint64_t kd = smem_desc_sw128(sbase + L::kK + stage * L::kTileBytes, 16, 1024);
-#pragma unroll 1
+#pragma unroll
       for (int s = 0; s < D / 16; ++s) {
-        const uint64_t off = ((s >> 2) * L::kChunkBytes + (s & 3) * 32) >> 4;
-        tc_mma_ss(tmem + L::kColS0, qd0 + off, kd + off, idesc_qk, s > 0 ? 1u : 0u);
-        tc_mma_ss(tmem + L::kColS1, qd1 + off, kd + off, idesc_qk, s > 0 ? 1u : 0u);
+        const uint32_t off = ((s >> 2) * L::kChunkBytes + (s & 3) * 32) >> 4;
+        tc_mma_ss(tmem + L::kColS0, with_lo(qd0, off), with_lo(kd, off), idesc_qk, s > 0 ? 1u : 0u);
+        tc_mma_ss(tmem + L::kColS1, with_lo(qd1, off), with_lo(kd, off), idesc_qk, s > 0 ? 1u : 0u);
       }
     };
     auto issue_pv = [&](int i, int stage, bool first) {
@@ -293,9 +296,9 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           smem_desc_sw128(sbase + L::kV + stage * L::kTileBytes, L::kChunkBytes, 1024);
       const uint32_t d_col = tmem + (i == 0 ? L::kColO0 : L::kColO1);
       const uint32_t p_col = tmem + (i == 0 ? L::kColS0 : L::kColS1);
-#pragma unroll 1
+#pragma unroll
       for (int s = 0; s < kTile / 16; ++s) {
-        tc_mma_ts(d_col, p_col + 8 * s, vd + static_cast<uint64_t>(s * 2048 >> 4), idesc_pv,
+        tc_mma_ts(d_col, p_col + 8 * s, with_lo(vd, (s * 2048) >> 4), idesc_pv,
                   (first && s == 0) ? 0u : 1u);
       }
     };
