@@ -391,7 +391,27 @@ def _detail_topk(sma, dev, stream, out, pk_t, pk_b, flush):
     kept = sum(1 for a in range(qt_n) for c in range(kt_n) if c * TILE <= min((a + 1) * TILE, w.n_q) - 1 + off)
     tf = tile_flops(w.head_dim, w.heads * w.batch, kept) / (ms * 1e-3) / 1e12
     out[w.name + "_attention"] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / pk_t, "kept_tiles_per_bh": kept}
-    del q, k, v, o, bias, pre, keep
+    # index-gather path over the same mask: compacted key tiles per (b, kv head, q tile)
+    ws = torch.empty(sma.sparse_attn_fwd_workspace_size(q.dtype, w.batch, w.heads, w.kv_heads, w.n_q, w.n_k,
+                                                        w.head_dim, tuple(keep.shape), max_keys=w.window),
+                     dtype=torch.uint8, device=dev)
+    ms_g = timed(lambda: sma.sparse_attn_fwd(q, k, v, keep, None, True, max_keys=w.window, out=o, workspace=ws),
+                 stream, 10, 3)
+    km = keep[:, :, 0, :w.n_k].cpu()
+    ctiles = 0
+    for row in km.reshape(-1, w.n_k):
+        idx = torch.nonzero(row).flatten()
+        for a in range(qt_n):
+            lim = int(torch.searchsorted(idx, min((a + 1) * TILE, w.n_q) - 1 + off, right=True))
+            ctiles += -(-lim // TILE)
+    group = w.heads // w.kv_heads
+    tf_c = tile_flops(w.head_dim, group, ctiles) / (ms_g * 1e-3) / 1e12
+    out[w.name + "_attention_gather"] = {
+        "ms": ms_g, "speedup_vs_dense_walk": ms / ms_g,
+        "TFLOP/s_compacted_tiles": tf_c, "frac_bf16_peak": tf_c / pk_t,
+        "TFLOP/s_dense_tile_equivalent": tile_flops(w.head_dim, w.heads * w.batch, kept) / (ms_g * 1e-3) / 1e12,
+        "compacted_tiles": ctiles}
+    del q, k, v, o, bias, pre, keep, ws
 
 
 def _detail_topk_wide(sma, dev, stream, out, pk_b):

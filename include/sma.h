@@ -283,6 +283,49 @@ sma_status dynamic_topk_mask(int32_t bias_dtype, const void* bias, const int64_t
                              const int64_t pre_mask_sizes[4], const int64_t pre_mask_strides[4],
                              int32_t window_size, uint8_t* out_mask, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Index-gather attention under a query-broadcast keep mask.
+ *
+ * Source: flash-sparse-attention PR #197 (Design: the top-k keep mask of a
+ * bias row, broadcast over the query dim in its Usage) with the mask/bias
+ * contract and causal rule of PR #190.  Computes exactly what
+ * masked_attn_fwd computes for the same arguments, but only over the kept
+ * keys: per (batch row, head row) of the mask the kept key indices are
+ * listed in ascending order, the K/V rows (and bias columns) they name are
+ * copied into compacted operands in the workspace, and attention runs over
+ * those with the causal bound applied to the original indices.  Work scales
+ * with the kept keys, not with k_len.
+ *
+ * mask      required; the 4D contract above with sizes[2] == 1 (one row for
+ *           every query) and sizes[1] in {1, kv_heads} (or heads when heads
+ *           == kv_heads): rows shared by the query heads of a KV head.
+ *           Other masks return SMA_ERR_UNSUPPORTED (use masked_attn_fwd).
+ * bias      NULL or the 4D contract above (any broadcast shape).
+ * max_keys  upper bound on the kept keys of any mask row (e.g. the top-k
+ *           window_size); <= 0 or > k_len means k_len.  It sizes the
+ *           compacted operands.  A row with more kept keys is cut to its
+ *           first max_keys and raises SMA_ERR_DEVICE_INPUT in the device
+ *           error word (read with sma_device_status).
+ * dtype     SMA_BF16 / SMA_FP16 (tensor cores) or SMA_FP32 (FFMA).
+ * Other arguments as masked_attn_fwd; all q_len >= 1 run the prefill kernel.
+ * A row that keeps no key gives out = 0 and lse = -inf. */
+sma_status sparse_attn_fwd_workspace_size(int32_t dtype, int32_t batch, int32_t heads,
+                                          int32_t kv_heads, int32_t q_len, int32_t k_len,
+                                          int32_t head_dim, const int64_t mask_sizes[4],
+                                          int32_t bias_dtype, const int64_t bias_sizes[4],
+                                          int32_t max_keys, size_t* bytes);
+
+sma_status sparse_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t q_len, int32_t k_len, int32_t head_dim, float scale,
+                           int32_t is_causal, const void* q, const int64_t q_strides[3],
+                           const void* k, const int64_t k_strides[3], const void* v,
+                           const int64_t v_strides[3], const uint8_t* mask,
+                           const int64_t mask_sizes[4], const int64_t mask_strides[4],
+                           const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+                           const int64_t bias_strides[4], int32_t max_keys, void* out,
+                           const int64_t o_strides[3], float* lse, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

@@ -2,7 +2,8 @@
 
 Thin Python binding over libsma (C ABI in include/sma.h): DFlash draft-training
 masks computed analytically from block anchors, broadcastable 4D mask/bias
-attention with the grouped-head decode path, and the dynamic top-k keep mask.
+attention with the grouped-head decode path, the dynamic top-k keep mask, and
+index-gather attention over the keys such a mask keeps.
 """
 from ._native import NativeLibraryMissing, SmaError  # noqa: F401
 from .ops import (  # noqa: F401
@@ -20,4 +21,6 @@ from .ops import (  # noqa: F401
     masked_attn_fwd_workspace_size,
     round_up_k,
     selftest_wait_timeout,
+    sparse_attn_fwd,
+    sparse_attn_fwd_workspace_size,
 )

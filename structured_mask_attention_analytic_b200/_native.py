@@ -73,6 +73,13 @@ _SIGNATURES = {
                                 c_vp, c_i64p, c_vp, c_vp, c_size, c_vp]),
     "dynamic_topk_mask": (c_i32, [c_i32, c_vp, c_i64p, c_i64p, c_i32, c_vp, c_i64p, c_i64p, c_i32, c_vp,
                                   c_vp]),
+    "sparse_attn_fwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64p,
+                                               c_i32, c_i64p, c_i32, c_sizep]),
+    "sparse_attn_fwd": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.c_float, c_i32,
+                                c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
+                                c_vp, c_i64p, c_i64p,
+                                c_vp, c_i32, c_i64p, c_i64p, c_i32,
+                                c_vp, c_i64p, c_vp, c_vp, c_size, c_vp]),
 }
 
 _lib = None

@@ -7,6 +7,7 @@
 // each owning the even or odd half of head_dim; keys in chunks of 32 staged
 // through shared memory.
 #include "device_common.cuh"
+#include "gather.cuh"
 #include "kernels.h"
 
 namespace sma {
@@ -75,7 +76,10 @@ attn_simt_kernel(const AttnProblem p) {
       brow = reinterpret_cast<const uint8_t*>(p.bias.ptr) +
              (b * p.bias.sb + hb * p.bias.sh + static_cast<int64_t>(qq) * p.bias.sq) * esz;
     }
-    if (p.causal) causal_lim = q + p.Lk - p.Lq;
+    if (p.gather.idx != nullptr)  // compacted keys: the row's limit on the compacted index
+      causal_lim = row_valid ? gather_row_limit(p, static_cast<int64_t>(lb) * p.lists.LH + lh, q) - 1 : -1;
+    else if (p.causal)
+      causal_lim = q + p.Lk - p.Lq;
   }
 
   float m = -INFINITY, l = 0.f;
@@ -106,7 +110,7 @@ attn_simt_kernel(const AttnProblem p) {
         for (int e = 0; e < E; ++e) acc = fmaf(qr[e], sk[kk][2 * e + hf], acc);
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
         const int k = c0 + kk;
-        if (POLICY == kPolicyExplicit && p.has_bias && k < p.Lk)
+        if (POLICY != kPolicyDflash && p.has_bias && k < p.Lk)
           acc = fmaf(load_any_as_float(brow, p.bias.dtype, k), kLog2e, acc);
         bool keep = row_valid;
         if (partial) {

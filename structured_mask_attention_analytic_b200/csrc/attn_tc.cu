@@ -35,12 +35,17 @@
 //               keep, additive bias, stride-0 broadcast dims), plus
 //               bottom-right causal masking; the bias is added on every kept
 //               tile, the mask read on PARTIAL tiles only.
+//   Gather   -- the explicit policy over keys compacted by a query-broadcast
+//               mask (PR #197 top-k masks): K/V/bias are the compacted
+//               operands and each row's causal bound is a limit on the
+//               compacted index.
 #include <cudaTypedefs.h>
 
 #include <cstdio>
 #include <type_traits>
 
 #include "device_common.cuh"
+#include "gather.cuh"
 #include "kernels.h"
 
 namespace sma {
@@ -443,7 +448,10 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           brow = reinterpret_cast<const uint8_t*>(p.bias.ptr) +
                  (w.b * p.bias.sb + hb * p.bias.sh + static_cast<int64_t>(qq) * p.bias.sq) * esz;
         }
-        if (p.causal) causal_lim = q + p.Lk - p.Lq;
+        if (POLICY == kPolicyGather)  // compacted keys: the row's limit on the compacted index
+          causal_lim = row_valid ? gather_row_limit(p, w.list_row / p.QT, q) - 1 : -1;
+        else if (p.causal)
+          causal_lim = q + p.Lk - p.Lq;
       }
 
       // Scores are scaled inside the exponent (one FFMA per element).  A bias
@@ -451,7 +459,8 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
       // log2(e) = (scale * s + b) * log2(e).
       const float exp_scale = p.scale_log2;
       const float bias_mul = kLog2e / p.scale_log2;
-      const int causal_off = p.Lk - p.Lq;
+      // With compacted keys every PARTIAL tile is cut by the row limit.
+      const int causal_off = POLICY == kPolicyGather ? -(1 << 30) : p.Lk - p.Lq;
       const bool mask_bcast_q = POLICY == kPolicyExplicit && p.has_mask && p.mask.sq == 0;
       float m_ref = -INFINITY, l_sum = 0.f;
       bool partial_next = false;
@@ -470,7 +479,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           for (int c = 0; c < kTile / 32; ++c) tmem_ld32_at(s_col + 32 * c, xr + 32 * c);
           tc_wait_ld();
         }
-        if (POLICY == kPolicyExplicit && p.has_bias) {
+        if (POLICY != kPolicyDflash && p.has_bias) {
           if (p.bias.dtype == SMA_FP32) {
 #pragma unroll
             for (int c = 0; c < kTile; c += 4) {
@@ -537,7 +546,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
                 const bool keep = ((bits[c & 3] >> (c >> 2)) & 1u) != 0u && c < lim;
                 x[c] = keep ? x[c] : -INFINITY;
               }
-            } else if (p.has_mask) {
+            } else if (POLICY == kPolicyExplicit && p.has_mask) {
 #pragma unroll
               for (int c = 0; c < kTile; c += 16) {
                 const uint4 mv = *reinterpret_cast<const uint4*>(mrow + k0 + c);
@@ -763,6 +772,11 @@ int launch_attn_tc(const AttnProblem& p, cudaStream_t stream, char* msg, size_t 
                            : launch_typed<128, kPolicyDflash, SMA_FP16>(p, mq, mk, mv, stream);
     else e = bf ? launch_typed<64, kPolicyDflash, SMA_BF16>(p, mq, mk, mv, stream)
                 : launch_typed<64, kPolicyDflash, SMA_FP16>(p, mq, mk, mv, stream);
+  } else if (p.policy == kPolicyGather) {
+    if (p.d == 128) e = bf ? launch_typed<128, kPolicyGather, SMA_BF16>(p, mq, mk, mv, stream)
+                           : launch_typed<128, kPolicyGather, SMA_FP16>(p, mq, mk, mv, stream);
+    else e = bf ? launch_typed<64, kPolicyGather, SMA_BF16>(p, mq, mk, mv, stream)
+                : launch_typed<64, kPolicyGather, SMA_FP16>(p, mq, mk, mv, stream);
   } else {
     if (p.d == 128) e = bf ? launch_typed<128, kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, stream)
                            : launch_typed<128, kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, stream);

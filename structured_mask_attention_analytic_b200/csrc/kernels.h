@@ -43,7 +43,21 @@ struct TileLists {
   int head_mode = 0;  // 0: lh = 0; 1: lh = kv head; 2: lh = kv head * npairs + pair
 };
 
-enum MaskPolicy { kPolicyDflash = 0, kPolicyExplicit = 1 };
+// Gather: explicit policy over compacted keys (GatherView set, no mask).
+enum MaskPolicy { kPolicyDflash = 0, kPolicyExplicit = 1, kPolicyGather = 2 };
+
+// Index-gather view of a query-broadcast keep mask: per gather row (batch
+// row LB x head row LH of the mask, the same rows as the tile lists) the
+// ascending original indices of the kept keys.  When set, the problem's k, v
+// and bias are the compacted operands (compacted key j of a row is original
+// key idx[row][j]) and Lk is the compacted capacity.
+struct GatherView {
+  const int32_t* idx = nullptr;    // [rows, cap]
+  const int32_t* count = nullptr;  // [rows], <= cap
+  int cap = 0;                     // multiple of 128
+  int k_len = 0;                   // original key length
+  int causal = 0;                  // bottom-right causal bound on original indices
+};
 
 // One attention forward problem: O[b, q, h] over keys of head h / group.
 struct AttnProblem {
@@ -64,6 +78,7 @@ struct AttnProblem {
   int causal;
   int has_mask, has_bias;
   AuxView mask, bias;
+  GatherView gather;  // idx == nullptr: keys are not compacted
   int* err;  // device error word
 };
 
@@ -118,6 +133,22 @@ int launch_attn_tc(const AttnProblem& p, cudaStream_t stream, char* msg, size_t 
 cudaError_t launch_attn_simt(const AttnProblem& p, cudaStream_t stream);
 
 cudaError_t launch_decode(const DecodeProblem& p, cudaStream_t stream);
+
+// Index-gather preparation.  `mask` is a query-broadcast keep mask with
+// element strides m_sb / m_sh (0 on broadcast dims) and Kpad columns; gather
+// row (lb, lh) reads mask row lb * m_sb + lh * m_sh.
+cudaError_t launch_select_keys(const uint8_t* mask, int64_t m_sb, int64_t m_sh, int LB, int LH,
+                               int Lk, int cap, int32_t* idx, int32_t* count, int* err,
+                               cudaStream_t stream);
+// Compacted K and V ([B, cap, KVH, d], the strides in p.k/p.v) from the
+// original operands; rows from count to the next multiple of 128 are zeroed.
+cudaError_t launch_gather_kv(const AttnProblem& p, const void* k, const int64_t k_strides[3],
+                             const void* v, const int64_t v_strides[3], cudaStream_t stream);
+// Compacted bias (the view in p.bias, cap columns) from the original view.
+cudaError_t launch_gather_bias(const AttnProblem& p, const AuxView& bias, int rows_h, int rows_q,
+                               cudaStream_t stream);
+// FULL / PARTIAL key-tile lists over the compacted keys.
+cudaError_t launch_gather_lists(const AttnProblem& p, cudaStream_t stream);
 
 cudaError_t launch_topk(const TopkProblem& p, cudaStream_t stream);
 

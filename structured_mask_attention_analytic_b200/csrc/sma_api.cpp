@@ -227,6 +227,61 @@ MaskedGeom masked_geom(int32_t B, int32_t H, int32_t KVH, int32_t Lq, int32_t Lk
   return g;
 }
 
+
+// ---- index-gather path geometry: kept-key lists, tile lists over the
+// compacted keys, compacted K/V and bias, all in the workspace.
+struct SparseGeom {
+  int LB, LH, QT, KT, cap, Hc, Qc;
+  size_t idx, count;
+  ListsLayout lists;
+  size_t kc, vc, bias, total;
+};
+
+sma_status sparse_geom(int32_t dtype, int32_t B, int32_t H, int32_t KVH, int32_t Lq, int32_t Lk,
+                       int32_t d, const int64_t* mask_sizes, int32_t bias_dtype,
+                       const int64_t* bias_sizes, int32_t max_keys, SparseGeom* g) {
+  if (mask_sizes == nullptr) return fail(SMA_ERR_INVALID_ARG, "the index-gather path needs a mask");
+  if (mask_sizes[2] != 1)
+    return fail(SMA_ERR_UNSUPPORTED,
+                "index-gather attention needs a mask broadcast over queries (size 1 in dim 2, "
+                "got %lld); use masked_attn_fwd",
+                static_cast<long long>(mask_sizes[2]));
+  if (mask_sizes[1] != 1 && mask_sizes[1] != KVH)
+    return fail(SMA_ERR_UNSUPPORTED,
+                "index-gather attention needs mask rows shared by the query heads of a KV head "
+                "(head dim 1 or %d, got %lld); use masked_attn_fwd",
+                KVH, static_cast<long long>(mask_sizes[1]));
+  if (mask_sizes[0] != 1 && mask_sizes[0] != B)
+    return fail(SMA_ERR_INVALID_ARG, "mask batch dim must be %d or 1", B);
+  g->LB = mask_sizes[0] > 1 ? B : 1;
+  g->LH = mask_sizes[1] > 1 ? KVH : 1;
+  g->QT = static_cast<int>(ceil_div(Lq, kTile));
+  const int keys = (max_keys <= 0 || max_keys > Lk) ? Lk : max_keys;
+  g->cap = static_cast<int>(round_up(keys, kTile));
+  g->KT = g->cap / kTile;
+  const int64_t rows = static_cast<int64_t>(g->LB) * g->LH;
+  g->idx = 0;
+  g->count = align256(static_cast<size_t>(rows) * g->cap * 4);
+  g->lists = lists_layout(align256(g->count + rows * 4), rows * g->QT, g->KT);
+  const size_t kv_bytes = static_cast<size_t>(B) * g->cap * KVH * d * elem_size(dtype);
+  g->kc = g->lists.end;
+  g->vc = align256(g->kc + kv_bytes);
+  g->bias = align256(g->vc + kv_bytes);
+  g->Hc = g->Qc = 0;
+  g->total = g->bias;
+  if (bias_sizes != nullptr) {
+    if (bias_sizes[1] != H && bias_sizes[1] != KVH && bias_sizes[1] != 1)
+      return fail(SMA_ERR_INVALID_ARG, "bias head dim must be %d, %d or 1", H, KVH);
+    if (bias_sizes[2] != Lq && bias_sizes[2] != 1)
+      return fail(SMA_ERR_INVALID_ARG, "bias query dim must be %d or 1", Lq);
+    g->Hc = bias_sizes[1] == H ? H : KVH;
+    g->Qc = static_cast<int>(bias_sizes[2]);
+    g->total = align256(g->bias + static_cast<size_t>(B) * g->Hc * g->Qc * g->cap *
+                                      elem_size(bias_dtype));
+  }
+  return SMA_OK;
+}
+
 }  // namespace
 
 int sma::set_last_error(int code, const char* message) {
@@ -586,6 +641,138 @@ sma_status dynamic_topk_mask(int32_t bias_dtype, const void* bias, const int64_t
     return fail(SMA_ERR_INVALID_ARG, "out_mask must be 8-byte aligned");
   cudaError_t e = launch_topk(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "top-k launch failed");
+  return ok();
+}
+
+sma_status sparse_attn_fwd_workspace_size(int32_t dtype, int32_t batch, int32_t heads,
+                                          int32_t kv_heads, int32_t q_len, int32_t k_len,
+                                          int32_t head_dim, const int64_t mask_sizes[4],
+                                          int32_t bias_dtype, const int64_t bias_sizes[4],
+                                          int32_t max_keys, size_t* bytes) {
+  if (bytes == nullptr) return fail(SMA_ERR_INVALID_ARG, "bytes is NULL");
+  if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (bias_sizes != nullptr && !valid_dtype(bias_dtype))
+    return fail(SMA_ERR_INVALID_ARG, "unknown bias dtype %d", bias_dtype);
+  sma_status s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (batch < 1 || q_len < 1 || k_len < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, q_len and k_len must be >= 1");
+  SparseGeom g;
+  if ((s = sparse_geom(dtype, batch, heads, kv_heads, q_len, k_len, head_dim, mask_sizes, bias_dtype,
+                       bias_sizes, max_keys, &g)) != SMA_OK)
+    return s;
+  *bytes = g.total;
+  return ok();
+}
+
+sma_status sparse_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t q_len, int32_t k_len, int32_t head_dim, float scale,
+                           int32_t is_causal, const void* q, const int64_t q_strides[3],
+                           const void* k, const int64_t k_strides[3], const void* v,
+                           const int64_t v_strides[3], const uint8_t* mask,
+                           const int64_t mask_sizes[4], const int64_t mask_strides[4],
+                           const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+                           const int64_t bias_strides[4], int32_t max_keys, void* out,
+                           const int64_t o_strides[3], float* lse, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  sma_status s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (batch < 1 || q_len < 1 || k_len < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, q_len and k_len must be >= 1");
+  if (is_causal != 0 && is_causal != 1) return fail(SMA_ERR_INVALID_ARG, "is_causal must be 0 or 1");
+  if ((s = check_operand("q", q, q_strides, dtype, q_len)) != SMA_OK) return s;
+  if ((s = check_operand("k", k, k_strides, dtype, k_len)) != SMA_OK) return s;
+  if ((s = check_operand("v", v, v_strides, dtype, k_len)) != SMA_OK) return s;
+  if ((s = check_operand("out", out, o_strides, dtype, q_len)) != SMA_OK) return s;
+  if (mask == nullptr) return fail(SMA_ERR_INVALID_ARG, "the index-gather path needs a mask");
+  AuxView mview, bview;
+  if ((s = check_aux("mask", mask, mask_sizes, mask_strides, 1, batch, heads, kv_heads, q_len, k_len,
+                     true, &mview)) != SMA_OK)
+    return s;
+  const bool has_bias = bias != nullptr;
+  if (has_bias) {
+    if (!valid_dtype(bias_dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown bias dtype %d", bias_dtype);
+    if ((s = check_aux("bias", bias, bias_sizes, bias_strides, elem_size(bias_dtype), batch, heads,
+                       kv_heads, q_len, k_len, true, &bview)) != SMA_OK)
+      return s;
+    bview.dtype = bias_dtype;
+  }
+  SparseGeom g;
+  if ((s = sparse_geom(dtype, batch, heads, kv_heads, q_len, k_len, head_dim, mask_sizes, bias_dtype,
+                       has_bias ? bias_sizes : nullptr, max_keys, &g)) != SMA_OK)
+    return s;
+  if ((s = check_workspace(workspace, workspace_bytes, g.total)) != SMA_OK) return s;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (err == nullptr) return cuda_fail(e, "device error word unavailable");
+
+  AttnProblem p{};
+  p.dtype = dtype;
+  p.B = batch; p.H = heads; p.KVH = kv_heads; p.Lq = q_len; p.Lk = g.cap; p.d = head_dim;
+  p.group = heads / kv_heads;
+  p.npairs = (p.group + 1) / 2;
+  p.QT = g.QT; p.KT = g.KT;
+  p.scale_log2 = resolve_scale(scale, head_dim) * kLog2eHost;
+  p.q = q; p.q_sb = q_strides[0]; p.q_sr = q_strides[1]; p.q_sh = q_strides[2];
+  // compacted K / V: [batch, cap, kv_heads, head_dim] contiguous
+  p.k = at<uint8_t>(workspace, g.kc);
+  p.v = at<uint8_t>(workspace, g.vc);
+  p.k_sh = p.v_sh = head_dim;
+  p.k_sr = p.v_sr = static_cast<int64_t>(kv_heads) * head_dim;
+  p.k_sb = p.v_sb = static_cast<int64_t>(g.cap) * kv_heads * head_dim;
+  p.o = out; p.o_sb = o_strides[0]; p.o_sr = o_strides[1]; p.o_sh = o_strides[2];
+  p.lse = lse;
+  p.policy = kPolicyGather;
+  p.causal = 1;  // every PARTIAL tile is cut by its row's limit
+  p.has_mask = 0;
+  p.has_bias = has_bias;
+  p.err = err;
+  p.lists.LB = g.LB;
+  p.lists.LH = g.LH;
+  p.lists.head_mode = g.LH > 1 ? 1 : 0;
+  p.lists.num_full = at<int32_t>(workspace, g.lists.nf);
+  p.lists.num_part = at<int32_t>(workspace, g.lists.np);
+  p.lists.full_idx = at<int32_t>(workspace, g.lists.fi);
+  p.lists.part_idx = at<int32_t>(workspace, g.lists.pi);
+  int32_t* idx = at<int32_t>(workspace, g.idx);
+  int32_t* count = at<int32_t>(workspace, g.count);
+  p.gather.idx = idx;
+  p.gather.count = count;
+  p.gather.cap = g.cap;
+  p.gather.k_len = k_len;
+  p.gather.causal = is_causal;
+  if (has_bias) {
+    AuxView cb;
+    cb.ptr = at<uint8_t>(workspace, g.bias);
+    cb.dtype = bias_dtype;
+    cb.sq = g.Qc > 1 ? g.cap : 0;
+    cb.sh = static_cast<int64_t>(g.Qc) * g.cap;
+    cb.sb = static_cast<int64_t>(g.Hc) * g.Qc * g.cap;
+    cb.head_per_query = g.Hc == heads && bview.head_per_query ? 1 : 0;
+    p.bias = cb;
+  }
+
+  e = launch_select_keys(mask, mview.sb, mview.sh, g.LB, g.LH, k_len, g.cap, idx, count, err, st);
+  if (e != cudaSuccess) return cuda_fail(e, "key selection launch failed");
+  e = launch_gather_kv(p, k, k_strides, v, v_strides, st);
+  if (e != cudaSuccess) return cuda_fail(e, "K/V gather launch failed");
+  if (has_bias) {
+    e = launch_gather_bias(p, bview, g.Hc, g.Qc, st);
+    if (e != cudaSuccess) return cuda_fail(e, "bias gather launch failed");
+  }
+  e = launch_gather_lists(p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "tile list launch failed");
+  if (dtype == SMA_FP32) {
+    e = launch_attn_simt(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch failed");
+    return ok();
+  }
+  char msg[256];
+  const int rc = launch_attn_tc(p, st, msg, sizeof(msg));
+  if (rc != SMA_OK) return fail(rc, "%s", msg);
   return ok();
 }
 

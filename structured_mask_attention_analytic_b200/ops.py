@@ -239,6 +239,54 @@ def masked_attn_fwd(q, k, v, mask=None, bias=None, is_causal: bool = False, scal
     return out, lse
 
 
+def sparse_attn_fwd_workspace_size(dtype, batch, heads, kv_heads, q_len, k_len, head_dim, mask_shape,
+                                   bias_dtype=None, bias_shape=None, max_keys=None) -> int:
+    n = ctypes.c_size_t()
+    bdt = _DTYPE[bias_dtype] if bias_dtype is not None else 0
+    nat.check(_lib().sparse_attn_fwd_workspace_size(
+        _DTYPE[dtype], batch, heads, kv_heads, q_len, k_len, head_dim, nat.i64_array(mask_shape), bdt,
+        nat.i64_array(bias_shape) if bias_shape is not None else None,
+        0 if max_keys is None else int(max_keys), ctypes.byref(n)))
+    return n.value
+
+
+def sparse_attn_fwd(q, k, v, mask, bias=None, is_causal: bool = False, scale=None, max_keys=None,
+                    out=None, return_lse: bool = True, workspace=None):
+    """Index-gather attention under a keep mask shared by every query.
+
+    ``mask`` follows the 4D contract with a query dim of 1 and a head dim of
+    1 or KVH (e.g. a dynamic top-k mask); ``max_keys`` bounds the kept keys of
+    any mask row (the top-k window size).  The result equals
+    ``masked_attn_fwd`` on the same arguments; only the kept keys are read.
+    Returns ``(out, lse)``."""
+    _require_cuda(q, k, v, mask, bias)
+    b, lq, h, dh = q.shape
+    lk, kvh = k.shape[1], k.shape[2]
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k and v must share a dtype")
+    if mask is None or mask.dtype not in (torch.bool, torch.uint8):
+        raise ValueError("mask must be a bool tensor")
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((b, h, lq), dtype=torch.float32, device=q.device) if return_lse else None
+    ws_bytes = sparse_attn_fwd_workspace_size(q.dtype, b, h, kvh, lq, lk, dh, tuple(mask.shape),
+                                              bias.dtype if bias is not None else None,
+                                              tuple(bias.shape) if bias is not None else None, max_keys)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    mp, msz, mst = _aux_args(mask, lk)
+    bp, bsz, bst = _aux_args(bias, lk)
+    nat.check(_lib().sparse_attn_fwd(
+        _dtype_code(q), b, h, kvh, lq, lk, dh, ctypes.c_float(0.0 if scale is None else float(scale)),
+        1 if is_causal else 0,
+        _ptr(q), _strides3(q), _ptr(k), _strides3(k), _ptr(v), _strides3(v),
+        mp, msz, mst,
+        bp, _dtype_code(bias) if bias is not None else 0, bsz, bst,
+        0 if max_keys is None else int(max_keys),
+        _ptr(out), _strides3(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(q)))
+    return out, lse
+
+
 def _pre_mask_view(pre_mask: torch.Tensor, batch: int, q_len: int, k_len: int):
     """create_mask's shape step as a view: a 2D (batch, L) pre-mask becomes
     sizes (batch, 1, 1, L); columns >= L count as invalid, which equals

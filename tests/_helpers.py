@@ -47,6 +47,20 @@ def assert_attention_close(out_gpu, lse_gpu, out_ref, lse_ref, dtype, rows=None,
             assert lerr <= LSE_TOL[dtype], f"{what}: lse err {lerr:.3e}"
 
 
+def masked_oracle(q, k, v, mask, bias, causal, rows=None, workers=8):
+    """Dense definition of attention under the 4D mask/bias contract (the
+    keep set is mask AND k < Lk AND, if causal, k <= q + Lk - Lq)."""
+    b, lq, h, d = q.shape
+    lk, kvh = k.shape[1], k.shape[2]
+    keep = at.aux_view(mask.cpu().numpy(), h, kvh, lk) if mask is not None else None
+    if causal:
+        ck = at.causal_keep(lq, lk)[None, None]
+        keep = ck if keep is None else (keep & ck)
+    bb = at.aux_view(f64(bias), h, kvh, lk) if bias is not None else None
+    return at.attention(f64(q), f64(k), f64(v), keep=keep, bias=bb, rows=rows, workers=workers,
+                        row_chunk=128)
+
+
 def dflash_oracle(q, k, v, anchors, ctx_len, block_size, is_causal, layer_type, window, rows=None,
                   workers=8):
     causal = dm.resolve_in_block_causal(is_causal, layer_type)

@@ -133,3 +133,47 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(nat, "_lib", None)
     with pytest.raises(nat.NativeLibraryMissing):
         nat.load()
+
+
+def test_sparse_workspace_and_validation_on_host():
+    lib = nat.load()
+    n = ctypes.c_size_t()
+    ms = nat.i64_array([2, 8, 1, 16384])
+    assert lib.sparse_attn_fwd_workspace_size(0, 2, 32, 8, 4096, 16384, 128, ms, 0, None, 2048,
+                                              ctypes.byref(n)) == 0
+    # compacted K and V: 2 x (batch 2, 2048 keys, 8 kv heads, 128) bf16, plus index and tile lists
+    kv = 2 * 2 * 2048 * 8 * 128 * 2
+    assert kv < n.value < kv + (1 << 20)
+    small = n.value
+    assert lib.sparse_attn_fwd_workspace_size(0, 2, 32, 8, 4096, 16384, 128, ms, 0, None, 0,
+                                              ctypes.byref(n)) == 0
+    assert n.value > 7 * small            # unbounded: capacity k_len
+    bs = nat.i64_array([1, 32, 4096, 16384])
+    assert lib.sparse_attn_fwd_workspace_size(0, 2, 32, 8, 4096, 16384, 128, ms, 2, bs, 2048,
+                                              ctypes.byref(n)) == 0
+    assert n.value >= small + 2 * 32 * 4096 * 2048 * 4     # compacted fp32 bias
+    per_query = nat.i64_array([1, 1, 4096, 16384])
+    assert lib.sparse_attn_fwd_workspace_size(0, 2, 32, 8, 4096, 16384, 128, per_query, 0, None, 0,
+                                              ctypes.byref(n)) == nat.SMA_ERR_UNSUPPORTED
+    assert "broadcast over queries" in lib.sma_last_error().decode()
+    per_qhead = nat.i64_array([1, 32, 1, 16384])
+    assert lib.sparse_attn_fwd_workspace_size(0, 2, 32, 8, 4096, 16384, 128, per_qhead, 0, None, 0,
+                                              ctypes.byref(n)) == nat.SMA_ERR_UNSUPPORTED
+    mha = nat.i64_array([1, 8, 1, 16384])
+    assert lib.sparse_attn_fwd_workspace_size(0, 2, 8, 8, 4096, 16384, 128, mha, 0, None, 0,
+                                              ctypes.byref(n)) == 0
+    assert lib.sparse_attn_fwd_workspace_size(0, 2, 32, 8, 4096, 16384, 128, None, 0, None, 0,
+                                              ctypes.byref(n)) == nat.SMA_ERR_INVALID_ARG
+
+
+def test_sparse_attn_needs_a_mask():
+    qs = [256 * 4 * 128, 4 * 128, 128]
+    ks = [200 * 2 * 128, 2 * 128, 128]
+    st = nat.load().sparse_attn_fwd(
+        0, 2, 4, 2, 256, 200, 128, ctypes.c_float(0.0), 0,
+        ctypes.c_void_p(0x10000), nat.i64_array(qs), ctypes.c_void_p(0x20000), nat.i64_array(ks),
+        ctypes.c_void_p(0x30000), nat.i64_array(ks), ctypes.c_void_p(0), None, None,
+        ctypes.c_void_p(0), 0, None, None, 0,
+        ctypes.c_void_p(0x40000), nat.i64_array(qs), None, ctypes.c_void_p(0x50000), 1 << 30, None)
+    assert st == nat.SMA_ERR_INVALID_ARG
+    assert "needs a mask" in nat.load().sma_last_error().decode()
