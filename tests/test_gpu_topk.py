@@ -94,3 +94,64 @@ def test_topk_then_attention_sampled():
     q, k, v = wl.topk_attention_inputs(w)
     rows = sample_tiles(w.n_q, picks=(0.25, 1.0))
     _run(q, k, v, keep.cpu(), None, True, rows=rows, what="topk attention")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_many_rows_random_full_check(dtype):
+    """Enough rows for the many-rows launch shape; N(0,1) values, ragged key
+    length, 2D pre-mask; every row checked."""
+    rng = np.random.default_rng(6)
+    bias = torch.from_numpy(rng.standard_normal((2, 4, 40, 3072), dtype=np.float32)).to(dtype)
+    pre = torch.from_numpy(rng.random((2, 3000)) < 0.85)
+    for window in (1, 37, 375, 2000, 2999):
+        _check(bias, 3000, window, pre)
+    _check(bias, 3000, 700, None)
+
+
+@pytest.mark.parametrize("rows", [(1, 1, 4), (2, 4, 40)], ids=["few", "many"])
+def test_heavy_ties_take_the_exact_fallback(rows):
+    """Eight distinct values: the sample bracket cannot isolate the threshold
+    and the full bisection decides."""
+    rng = np.random.default_rng(7)
+    levels = torch.tensor([-3.0, -1.0, -0.0, 0.0, 0.25, 1.0, 2.0, 9.0])
+    bias = levels[torch.from_numpy(rng.integers(0, 8, size=rows + (2048,)))].to(torch.bfloat16)
+    for window in (1, 300, 1024, 2047):
+        _check(bias, 2048, window, None)
+
+
+@pytest.mark.parametrize("rows", [(1, 1, 4), (2, 4, 40)], ids=["few", "many"])
+def test_infinities_below_the_sentinel(rows):
+    """-inf values rank below the pre-mask sentinel: when the window reaches
+    them, pre-masked positions (holding the sentinel) pass the threshold and
+    the pre-mask must still clear them."""
+    rng = np.random.default_rng(8)
+    vals = rng.standard_normal(rows + (1024,), dtype=np.float32)
+    vals[rng.random(vals.shape) < 0.3] = -np.inf
+    vals[rng.random(vals.shape) < 0.05] = np.inf
+    bias = torch.from_numpy(vals).to(torch.bfloat16)
+    pre = torch.from_numpy(rng.random((rows[0], 1000)) < 0.7)
+    for window in (10, 400, 700, 900):
+        _check(bias, 1000, window, pre)
+
+
+def test_longest_register_row_and_the_next():
+    """16384 columns (the register-resident kernel's limit) and 16512 (the
+    radix-select kernel) give the oracle's masks."""
+    rng = np.random.default_rng(9)
+    for k_len in (16384, 16500):
+        kp = sma.round_up_k(k_len)
+        bias = torch.from_numpy(rng.standard_normal((1, 2, 3, kp), dtype=np.float32)).to(torch.bfloat16)
+        pre = torch.from_numpy(rng.random((1, k_len)) < 0.9)
+        _check(bias, k_len, 2048, pre)
+
+
+def test_output_aligned_to_8_bytes_only():
+    """An output that is 8- but not 16-byte aligned takes the radix-select
+    kernel and gives the same mask."""
+    rng = np.random.default_rng(10)
+    bias = torch.from_numpy(rng.standard_normal((1, 1, 2, 512), dtype=np.float32)).to(torch.bfloat16).cuda()
+    buf = torch.empty(2 * 512 + 8, dtype=torch.bool, device="cuda")
+    out = buf[8:].view(1, 1, 2, 512)
+    got = sma.dynamic_topk_mask(bias, 500, 64, None, out=out)
+    ref = sma.dynamic_topk_mask(bias, 500, 64, None)
+    assert torch.equal(got, ref)
