@@ -15,6 +15,9 @@ Each module writes out the plain definition of one thing the pages describe:
 * ``attention``    -- dense softmax attention with an explicit keep mask and
   additive bias, including the broadcastable 4D mask/bias contract
   (flash-sparse-attention PR #190, Design: "Contract for aux tensors").
+* ``attention_grad`` -- the gradients dQ, dK, dV and the broadcast-reduced
+  dbias of that attention for an upstream gradient dO (flash-sparse-attention
+  PR #190, Changes: mha_bwd and its dbias reductions).
 * ``topk``         -- the dynamic top-k keep mask built from an attention bias
   (flash-sparse-attention PR #197, Design and Implementation Notes).
 * ``tiles``        -- full / partial / empty classification of 128x128 tiles
@@ -23,6 +26,7 @@ Each module writes out the plain definition of one thing the pages describe:
 Every function is pinned by ``tests/test_oracle_*.py`` to hand-worked
 fixtures under ``tests/golden/``, to library routines
 (``torch.nn.functional.scaled_dot_product_attention``, ``torch.topk``,
-``scipy.special.logsumexp``) on special cases, and to brute-force
+``scipy.special.logsumexp``, float64 autograd) on special cases, to central
+finite differences of the forward (the gradients), and to brute-force
 enumeration on tiny inputs.  No function here is "parity unpinned".
 """
