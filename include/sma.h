@@ -284,6 +284,66 @@ sma_status dynamic_topk_mask(int32_t bias_dtype, const void* bias, const int64_t
                              int32_t window_size, uint8_t* out_mask, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Backward (gradients) of the two attention entry points.
+ *
+ * Source: flash-sparse-attention PR #190, Changes (mha_bwd): the backward
+ * returns dQ, dK, dV under the same 4D mask/bias contract; SpecForge issue
+ * #452 (Problem) for the DFlash mask it is trained with.  With the forward's
+ * P (softmax over the kept keys) and O, and the upstream gradient dO:
+ *   dV = P^T dO,  dS = P * (dO V^T - rowsum(dO * O)),
+ *   dQ = scale * dS K,  dK = scale * dS^T Q
+ * (dK, dV summed over the query heads of each KV head).  Keys that no query
+ * attends get zero gradients; rows with no kept key contribute nothing.
+ *
+ * out, lse  the forward's output and log-sum-exp (natural log, [B, H, Lq]
+ *           contiguous float32, -inf for rows with no kept key), as the
+ *           forward call wrote them with the same arguments.
+ * dout      the upstream gradient, [B, Lq, H, d] like out.
+ * dq        [B, Lq, H, d]; dk, dv [B, Lk, KVH, d]: written, caller-owned,
+ *           strides as for q/k/v (last dim contiguous, 16-byte multiples).
+ * dtype     SMA_BF16 or SMA_FP16 (tensor cores, fp32 accumulation; dQ is
+ *           accumulated in fp32 in the workspace); SMA_FP32 returns
+ *           SMA_ERR_UNSUPPORTED.  head_dim 64 or 128.
+ * The workspace holds the tile lists, rowsum(dO * O) and the fp32 dQ
+ * accumulator (B * Lq * H * d * 4 bytes); query its size first.
+ * ---------------------------------------------------------------------- */
+
+sma_status dfa_attn_bwd_workspace_size(const dfa_mask_desc* desc, int32_t heads, int32_t kv_heads,
+                                       int32_t head_dim, size_t* bytes);
+
+sma_status dfa_attn_bwd(const dfa_mask_desc* desc, const int32_t* anchors, int32_t dtype,
+                        int32_t heads, int32_t kv_heads, int32_t head_dim, float scale,
+                        const void* q, const int64_t q_strides[3], const void* k,
+                        const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
+                        const void* out, const int64_t o_strides[3], const float* lse,
+                        const void* dout, const int64_t do_strides[3], void* dq,
+                        const int64_t dq_strides[3], void* dk, const int64_t dk_strides[3],
+                        void* dv, const int64_t dv_strides[3], void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+sma_status masked_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t kv_heads,
+                                          int32_t q_len, int32_t k_len, int32_t head_dim,
+                                          const int64_t mask_sizes[4], size_t* bytes);
+
+/* mask / bias / is_causal / scale exactly as given to masked_attn_fwd (any
+ * q_len; single-query problems run the general kernel).  dbias must be NULL:
+ * the broadcast-reduced bias gradient of PR #190 is not produced by this
+ * build (SMA_ERR_UNSUPPORTED otherwise). */
+sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t q_len, int32_t k_len, int32_t head_dim, float scale,
+                           int32_t is_causal, const void* q, const int64_t q_strides[3],
+                           const void* k, const int64_t k_strides[3], const void* v,
+                           const int64_t v_strides[3], const uint8_t* mask,
+                           const int64_t mask_sizes[4], const int64_t mask_strides[4],
+                           const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+                           const int64_t bias_strides[4], const void* out,
+                           const int64_t o_strides[3], const float* lse, const void* dout,
+                           const int64_t do_strides[3], void* dq, const int64_t dq_strides[3],
+                           void* dk, const int64_t dk_strides[3], void* dv,
+                           const int64_t dv_strides[3], float* dbias, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Index-gather attention under a query-broadcast keep mask.
  *
  * Source: flash-sparse-attention PR #197 (Design: the top-k keep mask of a

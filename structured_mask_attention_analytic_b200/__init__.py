@@ -1,4 +1,4 @@
-"""Structured-mask attention forward for NVIDIA B200 (sm_100a).
+"""Structured-mask attention forward and backward for NVIDIA B200 (sm_100a).
 
 Thin Python binding over libsma (C ABI in include/sma.h): DFlash draft-training
 masks computed analytically from block anchors, broadcastable 4D mask/bias
@@ -10,6 +10,8 @@ from .ops import (  # noqa: F401
     LAYER_FULL,
     LAYER_SLIDING,
     device_status,
+    dfa_attn_bwd,
+    dfa_attn_bwd_workspace_size,
     dfa_attn_fwd,
     dfa_attn_fwd_noalloc,
     dfa_attn_fwd_workspace_size,
@@ -17,6 +19,8 @@ from .ops import (  # noqa: F401
     dfa_block_map_dims,
     dynamic_topk_mask,
     mask_tile_summary,
+    masked_attn_bwd,
+    masked_attn_bwd_workspace_size,
     masked_attn_fwd,
     masked_attn_fwd_workspace_size,
     round_up_k,

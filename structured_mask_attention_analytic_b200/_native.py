@@ -73,6 +73,20 @@ _SIGNATURES = {
                                 c_vp, c_i64p, c_vp, c_vp, c_size, c_vp]),
     "dynamic_topk_mask": (c_i32, [c_i32, c_vp, c_i64p, c_i64p, c_i32, c_vp, c_i64p, c_i64p, c_i32, c_vp,
                                   c_vp]),
+    "dfa_attn_bwd_workspace_size": (c_i32, [ctypes.POINTER(DfaMaskDesc), c_i32, c_i32, c_i32, c_sizep]),
+    "dfa_attn_bwd": (c_i32, [ctypes.POINTER(DfaMaskDesc), c_vp, c_i32, c_i32, c_i32, c_i32, ctypes.c_float,
+                             c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
+                             c_vp, c_i64p, c_vp, c_vp, c_i64p,
+                             c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
+                             c_vp, c_size, c_vp]),
+    "masked_attn_bwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64p, c_sizep]),
+    "masked_attn_bwd": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.c_float, c_i32,
+                                c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
+                                c_vp, c_i64p, c_i64p,
+                                c_vp, c_i32, c_i64p, c_i64p,
+                                c_vp, c_i64p, c_vp, c_vp, c_i64p,
+                                c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
+                                c_vp, c_vp, c_size, c_vp]),
     "sparse_attn_fwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64p,
                                                c_i32, c_i64p, c_i32, c_sizep]),
     "sparse_attn_fwd": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.c_float, c_i32,

@@ -1,0 +1,883 @@
+// Attention backward on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Gradients of the forward in attn_tc.cu for an upstream gradient dO, under
+// the same mask families (DFlash analytic intervals, explicit mask / bias /
+// causal): flash-sparse-attention PR #190 (Changes, mha_bwd) names the
+// outputs dQ, dK, dV; the formulas are the derivative of softmax attention:
+//   P  = exp(scale * Q K^T + bias - lse)          (recomputed from the forward's lse)
+//   dV = P^T dO              dP = dO V^T          D = rowsum(dO * O)
+//   dS = P * (dP - D)        dQ = scale * dS K    dK = scale * dS^T Q
+//
+// One persistent CTA per SM walks units (batch, KV head, 128-key tile).  A
+// unit loops over the (query head of the group, 128-row query tile) pairs
+// that attend its key tile -- the transposed tile lists -- accumulating dK
+// and dV in TMEM over the whole group; each pair's dQ contribution is added
+// into an fp32 accumulator in global memory.
+//
+// Per pair, five 128-row products on the tensor cores (bf16/f16 operands
+// from shared memory, fp32 accumulators in TMEM):
+//   S  = Q K^T        A = Q  (K-major)      B = K  (K-major)       -> cols [0, 128)
+//   dP = dO V^T       A = dO (K-major)      B = V  (K-major)       -> cols [128, 256)
+//   dV += P^T dO      A = P^T (MN-major)    B = dO (MN-major)      -> cols [256, 256+D)
+//   dK += dS^T Q      A = dS^T (MN-major)   B = Q  (MN-major)      -> cols [256+D, 256+2D)
+//   dQ  = dS K        A = dS (K-major)      B = K  (MN-major)      -> cols [128, 128+D)
+// P and dS are written by the compute warps into shared memory in the same
+// 128-byte swizzled layout TMA gives a [128][128] tile, so one tile serves as
+// both a K-major operand and (transposed) an MN-major one.  dQ reuses dP's
+// columns once dS is formed.
+//
+// Warp roles (320 threads):
+//   warps 0-3  compute: row r of a query tile; phase A forms P from S (mask,
+//              bias, lse) and stores it; phase B forms dS = P (dP - D) and
+//              stores it.  dS uses P as stored (rounded to the operand type,
+//              as the dV product sees it).
+//   warps 4-7  dQ drain (TMEM -> vector atomic adds into the fp32 dQ
+//              accumulator) and the unit's dK / dV epilogue.
+//   warp  8    TMA producer: K, V once per unit; Q (2 stages), dO (1 stage)
+//   warp  9    MMA issuer (one elected lane), in the order
+//              S(0) dP(0) | dV(p) S(p+1) | dK(p) dQ(p) | dP(p+1) ...
+// Every mbarrier wait is bounded; on expiry the CTA raises its abort flag,
+// drains its own copies and products, frees TMEM and returns.
+#include <cstdio>
+#include <type_traits>
+
+#include "device_common.cuh"
+#include "kernels.h"
+#include "tma_map.h"
+
+namespace sma {
+namespace {
+
+constexpr int kBwdThreads = 320;
+constexpr int kBLoadWarp = 8;
+constexpr int kBMmaWarp = 9;
+constexpr uint32_t kBTmemCols = 512;
+
+template <int D>
+struct BLayout {
+  static constexpr uint32_t kChunk = kTile * 128;   // 64 columns x 128 rows, 128B-swizzled
+  static constexpr uint32_t kTileD = kTile * D * 2;  // [128][D] 16-bit tile
+  static constexpr uint32_t kTileK = kTile * kTile * 2;  // [128][128] 16-bit tile (P, dS)
+  static constexpr int kChunksD = D / 64;
+  static constexpr uint32_t kK = 0;
+  static constexpr uint32_t kV = kK + kTileD;
+  static constexpr uint32_t kQ = kV + kTileD;       // 2 stages
+  static constexpr uint32_t kDO = kQ + 2 * kTileD;  // 1 stage
+  static constexpr uint32_t kP = kDO + kTileD;
+  static constexpr uint32_t kDS = kP + kTileK;
+  static constexpr uint32_t kBars = kDS + kTileK;
+  enum : int {
+    kKVFull = 0, kKVEmpty, kQFull, kQEmpty = kQFull + 2, kOFull = kQEmpty + 2, kOEmpty,
+    kSFull, kPDone, kDPFull, kDSDone, kDQFull, kDQFree, kPFree, kDSFree, kAccDone, kAccFree,
+    kDrain, kNumBars
+  };
+  static constexpr uint32_t kTmemSlot = kBars + 8 * kNumBars;
+  static constexpr uint32_t kAbort = kTmemSlot + 4;
+  static constexpr uint32_t kBytes = kAbort + 4;
+  static constexpr uint32_t kAlloc = kBytes + 1024;  // base rounded up to 1024
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+  static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+// Transposed-list row of the query heads g of a unit.
+__device__ __forceinline__ int64_t bwd_row(const BwdProblem& p, int b, int hk, int g) {
+  const int lb = p.f.lists.LB > 1 ? b : 0;
+  int lh = 0;
+  if (p.f.lists.head_mode == 1) lh = hk;
+  else if (p.f.lists.head_mode == 2) lh = hk * p.f.npairs + g / 2;
+  return static_cast<int64_t>(lb) * p.f.lists.LH + lh;
+}
+
+struct BUnit {
+  int b, hk, kt, n_pairs;
+};
+
+__device__ __forceinline__ BUnit bwd_unit(const BwdProblem& p, int u) {
+  BUnit w;
+  const int per_kt = p.f.B * p.f.KVH;
+  w.kt = u / per_kt;  // key tiles in ascending order: early (context) tiles carry the most pairs
+  const int r = u - w.kt * per_kt;
+  w.b = r / p.f.KVH;
+  w.hk = r - w.b * p.f.KVH;
+  int n = 0;
+  for (int g = 0; g < p.f.group; ++g) {
+    const int64_t row = bwd_row(p, w.b, w.hk, g);
+    n += p.t_num_full[row * p.f.KT + w.kt] + p.t_num_part[row * p.f.KT + w.kt];
+  }
+  w.n_pairs = n;
+  return w;
+}
+
+// Walks the pairs of a unit in the order every role uses: heads of the group
+// outer, the key tile's query tiles (FULL first, then PARTIAL) inner.
+struct PairWalk {
+  int g, t, nf, np, G;
+  int64_t row;
+  __device__ __forceinline__ void begin(const BwdProblem& p, const BUnit& w) {
+    G = p.f.group;
+    g = 0;
+    t = 0;
+    load(p, w);
+    settle(p, w);
+  }
+  __device__ __forceinline__ void load(const BwdProblem& p, const BUnit& w) {
+    row = bwd_row(p, w.b, w.hk, g);
+    nf = p.t_num_full[row * p.f.KT + w.kt];
+    np = p.t_num_part[row * p.f.KT + w.kt];
+  }
+  __device__ __forceinline__ void settle(const BwdProblem& p, const BUnit& w) {
+    while (t >= nf + np && g + 1 < G) {
+      ++g;
+      t = 0;
+      load(p, w);
+    }
+  }
+  __device__ __forceinline__ void next(const BwdProblem& p, const BUnit& w) {
+    ++t;
+    settle(p, w);
+  }
+  __device__ __forceinline__ int head(const BUnit& w) const { return w.hk * G + g; }
+  __device__ __forceinline__ int qtile(const BwdProblem& p, const BUnit& w, bool* partial) const {
+    const int64_t base = (row * p.f.KT + w.kt) * p.f.QT;
+    if (t < nf) {
+      *partial = false;
+      return p.t_full[base + t];
+    }
+    *partial = true;
+    return p.t_part[base + (t - nf)];
+  }
+};
+
+__device__ __forceinline__ void bdrain_wait(uint32_t bar, uint32_t parity, int* err) {
+  int never = 0;
+  volatile int* nv = &never;
+  mbar_wait(bar, parity, nv, err);
+}
+
+// 16-byte unit u (8 columns) of row r of a 128-byte-swizzled [128][128] tile.
+__device__ __forceinline__ uint32_t sw128_unit(uint32_t base, int r, int u) {
+  return base + static_cast<uint32_t>((u >> 3) * (kTile * 128) + r * 128 + (((u & 7) ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int DT>
+__device__ __forceinline__ float2 unpack2(uint32_t w) {
+  if (DT == SMA_BF16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+
+template <int D, int POLICY, int DT>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
+                const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                const __grid_constant__ CUtensorMap map_do, int n_units) {
+  using L = BLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * static_cast<uint32_t>(i); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::kKVFull), 1);
+    mbar_init(bar(L::kKVEmpty), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(L::kQFull + s), 1);
+      mbar_init(bar(L::kQEmpty + s), 1);
+    }
+    mbar_init(bar(L::kOFull), 1);
+    mbar_init(bar(L::kOEmpty), 1);
+    mbar_init(bar(L::kSFull), 1);
+    mbar_init(bar(L::kPDone), 128);
+    mbar_init(bar(L::kDPFull), 1);
+    mbar_init(bar(L::kDSDone), 128);
+    mbar_init(bar(L::kDQFull), 1);
+    mbar_init(bar(L::kDQFree), 128);
+    mbar_init(bar(L::kPFree), 1);
+    mbar_init(bar(L::kDSFree), 1);
+    mbar_init(bar(L::kAccDone), 1);
+    mbar_init(bar(L::kAccFree), 128);
+    mbar_init(bar(L::kDrain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kBMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kBTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kBLoadWarp) {
+    // ------------------------------------------------------------ producer
+    if (elect_one()) {
+      tma_prefetch_map(&map_q);
+      tma_prefetch_map(&map_k);
+      tma_prefetch_map(&map_v);
+      tma_prefetch_map(&map_do);
+    }
+    __syncwarp();
+    uint32_t kv_it = 0, q_it = 0, o_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const BUnit w = bwd_unit(p, u);
+      if (w.n_pairs == 0) continue;
+      if (kv_it > 0 && !mbar_wait_warp(bar(L::kKVEmpty), (kv_it - 1) & 1, abort_flag, p.f.err)) {
+        ok = false;
+        break;
+      }
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar(L::kKVFull), 2 * L::kTileD);
+        for (int c = 0; c < L::kChunksD; ++c) {
+          tma_load_4d(sbase + L::kK + c * L::kChunk, &map_k, bar(L::kKVFull), c * 64, w.hk,
+                      w.kt * kTile, w.b);
+          tma_load_4d(sbase + L::kV + c * L::kChunk, &map_v, bar(L::kKVFull), c * 64, w.hk,
+                      w.kt * kTile, w.b);
+        }
+      }
+      __syncwarp();
+      ++kv_it;
+      PairWalk pw;
+      pw.begin(p, w);
+      for (int i = 0; i < w.n_pairs && ok; ++i, pw.next(p, w)) {
+        bool partial;
+        const int qt = pw.qtile(p, w, &partial);
+        const int h = pw.head(w);
+        const int s = q_it & 1;
+        const uint32_t use = q_it >> 1;
+        if (use > 0 && !mbar_wait_warp(bar(L::kQEmpty + s), (use - 1) & 1, abort_flag, p.f.err)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(L::kQFull + s), L::kTileD);
+          for (int c = 0; c < L::kChunksD; ++c)
+            tma_load_4d(sbase + L::kQ + s * L::kTileD + c * L::kChunk, &map_q, bar(L::kQFull + s),
+                        c * 64, h, qt * kTile, w.b);
+        }
+        __syncwarp();
+        ++q_it;
+        if (o_it > 0 && !mbar_wait_warp(bar(L::kOEmpty), (o_it - 1) & 1, abort_flag, p.f.err)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(L::kOFull), L::kTileD);
+          for (int c = 0; c < L::kChunksD; ++c)
+            tma_load_4d(sbase + L::kDO + c * L::kChunk, &map_do, bar(L::kOFull), c * 64, h,
+                        qt * kTile, w.b);
+        }
+        __syncwarp();
+        ++o_it;
+      }
+    }
+    if (!ok) {
+      // every copy this warp issued must land before the CTA exits
+      if (kv_it > 0) bdrain_wait(bar(L::kKVFull), (kv_it - 1) & 1, p.f.err);
+      for (uint32_t t = 0; t < 2; ++t) {
+        if (q_it > t) {
+          const uint32_t nn = q_it - 1 - t;
+          bdrain_wait(bar(L::kQFull + (nn & 1)), (nn >> 1) & 1, p.f.err);
+        }
+      }
+      if (o_it > 0) bdrain_wait(bar(L::kOFull), (o_it - 1) & 1, p.f.err);
+    }
+  } else if (warp == kBMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t fmt = DT == SMA_BF16 ? 1u : 0u;
+    constexpr uint32_t idesc_s = mma_idesc_f16(fmt, 128, 128, 0, 0);  // S, dP
+    constexpr uint32_t idesc_t = mma_idesc_f16(fmt, 128, D, 1, 1);    // dV, dK
+    constexpr uint32_t idesc_q = mma_idesc_f16(fmt, 128, D, 0, 1);    // dQ
+    auto with_lo = [](uint64_t d, uint32_t add) -> uint64_t {
+      return (d & 0xffffffff00000000ull) | static_cast<uint32_t>(static_cast<uint32_t>(d) + add);
+    };
+    // C[128][128] = A[128][D] B[128][D]^T, both K-major (K = head dim)
+    auto issue_kmajor = [&](uint32_t dcol, uint32_t a_addr, uint32_t b_addr) {
+      const uint64_t ad = smem_desc_sw128(a_addr, 16, 1024);
+      const uint64_t bd = smem_desc_sw128(b_addr, 16, 1024);
+#pragma unroll
+      for (int s = 0; s < D / 16; ++s) {
+        const uint32_t off = ((s >> 2) * L::kChunk + (s & 3) * 32) >> 4;
+        tc_mma_ss(tmem + dcol, with_lo(ad, off), with_lo(bd, off), idesc_s, s > 0 ? 1u : 0u);
+      }
+    };
+    // C[128][D] (+)= A^T B over the 128 query rows: A = P or dS [q][k], B = dO or Q [q][d]
+    auto issue_trans = [&](uint32_t dcol, uint32_t a_addr, uint32_t b_addr, bool acc) {
+      const uint64_t ad = smem_desc_sw128(a_addr, L::kChunk, 1024);
+      const uint64_t bd = smem_desc_sw128(b_addr, L::kChunk, 1024);
+#pragma unroll
+      for (int s = 0; s < kTile / 16; ++s) {
+        const uint32_t off = (s * 2048) >> 4;
+        tc_mma_ss(tmem + dcol, with_lo(ad, off), with_lo(bd, off), idesc_t,
+                  (acc || s > 0) ? 1u : 0u);
+      }
+    };
+    // dQ[128][D] = dS[q][k] K[k][d]
+    auto issue_dq = [&]() {
+      const uint64_t ad = smem_desc_sw128(sbase + L::kDS, 16, 1024);
+      const uint64_t bd = smem_desc_sw128(sbase + L::kK, L::kChunk, 1024);
+#pragma unroll
+      for (int s = 0; s < kTile / 16; ++s) {
+        const uint32_t aoff = ((s >> 2) * L::kChunk + (s & 3) * 32) >> 4;
+        const uint32_t boff = (s * 2048) >> 4;
+        tc_mma_ss(tmem + L::kColDP, with_lo(ad, aoff), with_lo(bd, boff), idesc_q,
+                  s > 0 ? 1u : 0u);
+      }
+    };
+    uint32_t kv_it = 0, q_it = 0, o_it = 0, pit = 0, uit = 0;
+    bool ok = true;
+    auto wait = [&](int b_, uint32_t parity) -> bool {
+      if (!mbar_wait_warp(bar(b_), parity, abort_flag, p.f.err)) ok = false;
+      return ok;
+    };
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const BUnit w = bwd_unit(p, u);
+      const int n = w.n_pairs;
+      if (n == 0) continue;
+      if (!wait(L::kKVFull, kv_it & 1)) break;
+      ++kv_it;
+      // S(0), dP(0)
+      if (!wait(L::kQFull + (q_it & 1), (q_it >> 1) & 1)) break;
+      tc_fence_after();
+      if (elect_one()) {
+        issue_kmajor(L::kColS, sbase + L::kQ + (q_it & 1) * L::kTileD, sbase + L::kK);
+        tc_commit(bar(L::kSFull));
+      }
+      __syncwarp();
+      if (!wait(L::kOFull, o_it & 1)) break;
+      if (pit > 0 && !wait(L::kDQFree, (pit - 1) & 1)) break;
+      tc_fence_after();
+      if (elect_one()) {
+        issue_kmajor(L::kColDP, sbase + L::kDO, sbase + L::kV);
+        tc_commit(bar(L::kDPFull));
+      }
+      __syncwarp();
+      for (int i = 0; i < n && ok; ++i) {
+        const int qs = q_it & 1;  // Q stage of pair i
+        // dV += P^T dO
+        if (!wait(L::kPDone, pit & 1)) break;
+        if (i == 0 && uit > 0 && !wait(L::kAccFree, (uit - 1) & 1)) break;
+        tc_fence_after();
+        if (elect_one()) {
+          issue_trans(L::kColDV, sbase + L::kP, sbase + L::kDO, i > 0);
+          tc_commit(bar(L::kPFree));
+          tc_commit(bar(L::kOEmpty));
+        }
+        __syncwarp();
+        ++o_it;
+        // S(i+1): S's columns are free once P(i) is formed
+        if (i + 1 < n) {
+          const uint32_t nq = q_it + 1;
+          if (!wait(L::kQFull + (nq & 1), (nq >> 1) & 1)) break;
+          tc_fence_after();
+          if (elect_one()) {
+            issue_kmajor(L::kColS, sbase + L::kQ + (nq & 1) * L::kTileD, sbase + L::kK);
+            tc_commit(bar(L::kSFull));
+          }
+          __syncwarp();
+        }
+        // dK += dS^T Q; dQ = dS K into dP's columns
+        if (!wait(L::kDSDone, pit & 1)) break;
+        tc_fence_after();
+        if (elect_one()) {
+          issue_trans(L::kColDK, sbase + L::kDS, sbase + L::kQ + qs * L::kTileD, i > 0);
+          issue_dq();
+          tc_commit(bar(L::kDQFull));
+          tc_commit(bar(L::kDSFree));
+          tc_commit(bar(L::kQEmpty + qs));
+        }
+        __syncwarp();
+        ++q_it;
+        ++pit;
+        // dP(i+1) once dO(i+1) is in and dQ(i) has left TMEM
+        if (i + 1 < n) {
+          if (!wait(L::kOFull, o_it & 1)) break;
+          if (!wait(L::kDQFree, (pit - 1) & 1)) break;
+          tc_fence_after();
+          if (elect_one()) {
+            issue_kmajor(L::kColDP, sbase + L::kDO, sbase + L::kV);
+            tc_commit(bar(L::kDPFull));
+          }
+          __syncwarp();
+        }
+      }
+      if (!ok) break;
+      if (elect_one()) {
+        tc_commit(bar(L::kAccDone));
+        tc_commit(bar(L::kKVEmpty));
+      }
+      __syncwarp();
+      ++uit;
+    }
+    if (!ok) {
+      if (elect_one()) tc_commit(bar(L::kDrain));
+      __syncwarp();
+      bdrain_wait(bar(L::kDrain), 0, p.f.err);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ compute (P, dS)
+    const int r = warp * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t s_col = tmem + lane_off + L::kColS;
+    const uint32_t dp_col = tmem + lane_off + L::kColDP;
+    const float scale_log2 = p.f.scale_log2;
+    const float bias_mul = kLog2e / p.f.scale_log2;
+    uint32_t pit = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const BUnit w = bwd_unit(p, u);
+      if (w.n_pairs == 0) continue;
+      const int k0 = w.kt * kTile;
+      PairWalk pw;
+      pw.begin(p, w);
+      for (int i = 0; i < w.n_pairs && ok; ++i, pw.next(p, w)) {
+        bool partial;
+        const int qt = pw.qtile(p, w, &partial);
+        const int h = pw.head(w);
+        const int q = qt * kTile + r;
+        const bool row_valid = q < p.f.Lq;
+        float neg_lse2 = -INFINITY, drow = 0.f;
+        if (row_valid) {
+          const float l = p.f.lse[(static_cast<int64_t>(w.b) * p.f.H + h) * p.f.Lq + q];
+          neg_lse2 = l == -INFINITY ? -INFINITY : -l * kLog2e;
+          drow = p.dvec[(static_cast<int64_t>(w.b) * p.f.H + h) * p.f.Lq + q];
+        }
+        const bool live = row_valid && neg_lse2 != -INFINITY;
+        // per-row mask parameters (as in the forward)
+        int clo = 0, chi = 0, dlo = 0, dhi = 0, lim = kTile;
+        const uint8_t* mrow = nullptr;
+        const uint8_t* brow = nullptr;
+        if (POLICY == kPolicyDflash) {
+          if (row_valid) {
+            const int j = q / p.f.bs, ii = q - j * p.f.bs;
+            int a = p.f.anchors[static_cast<int64_t>(w.b) * p.f.N + j];
+            a = a < 0 ? 0 : (a > p.f.Lc ? p.f.Lc : a);
+            chi = a;
+            clo = p.f.window > 0 ? max(0, a + ii - p.f.window + 1) : 0;
+            if (clo > chi) clo = chi;
+            const int base = p.f.Lc + j * p.f.bs;
+            dlo = base + (p.f.window > 0 ? max(0, ii - p.f.window + 1) : 0);
+            dhi = base + (p.f.causal_in_block ? ii + 1 : p.f.bs);
+          }
+        } else {
+          const int qq = row_valid ? q : 0;
+          if (p.f.has_mask) {
+            const int hm = p.f.mask.head_per_query ? h : w.hk;
+            mrow = reinterpret_cast<const uint8_t*>(p.f.mask.ptr) + w.b * p.f.mask.sb +
+                   hm * p.f.mask.sh + static_cast<int64_t>(qq) * p.f.mask.sq;
+          }
+          if (p.f.has_bias) {
+            const int hb = p.f.bias.head_per_query ? h : w.hk;
+            const int esz = p.f.bias.dtype == SMA_FP32 ? 4 : 2;
+            brow = reinterpret_cast<const uint8_t*>(p.f.bias.ptr) +
+                   (w.b * p.f.bias.sb + hb * p.f.bias.sh + static_cast<int64_t>(qq) * p.f.bias.sq) * esz;
+          }
+          if (k0 + kTile > p.f.Lk) lim = min(lim, p.f.Lk - k0);
+          if (p.f.causal) lim = min(lim, q + p.f.Lk - p.f.Lq - k0 + 1);
+        }
+
+        // ---- phase A: P from S
+        if (!mbar_wait(bar(L::kSFull), pit & 1, abort_flag, p.f.err)) { ok = false; break; }
+        if (pit > 0 && !mbar_wait(bar(L::kPFree), (pit - 1) & 1, abort_flag, p.f.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kTile / 32; ++c) {
+          uint32_t xr[32];
+          tmem_ld32_at(s_col + 32 * c, xr);
+          tc_wait_ld();
+          float x[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(xr[e]);
+          if (POLICY != kPolicyDflash && p.f.has_bias) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              x[e] = fmaf(load_any_as_float(brow, p.f.bias.dtype, k0 + 32 * c + e), bias_mul, x[e]);
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float pv[2];
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+              const int cc = 32 * c + e + z;
+              bool keep = live;
+              if (partial) {
+                if (POLICY == kPolicyDflash) {
+                  const int k = k0 + cc;
+                  keep = keep && ((k >= clo && k < chi) || (k >= dlo && k < dhi));
+                } else {
+                  keep = keep && cc < lim && (!p.f.has_mask || mrow[k0 + cc] != 0);
+                }
+              }
+              pv[z] = keep ? fast_exp2(fmaf(x[e + z], scale_log2, neg_lse2)) : 0.f;
+            }
+            pk[e >> 1] = DT == SMA_BF16 ? pack_bf16x2(pv[0], pv[1]) : pack_f16x2(pv[0], pv[1]);
+          }
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            st_shared_v4(sw128_unit(sbase + L::kP, r, 4 * c + v4), pk[4 * v4], pk[4 * v4 + 1],
+                         pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+        fence_async_shared();
+        tc_fence_before();
+        mbar_arrive(bar(L::kPDone));
+
+        // ---- phase B: dS = P (dP - D)
+        if (!mbar_wait(bar(L::kDPFull), pit & 1, abort_flag, p.f.err)) { ok = false; break; }
+        if (pit > 0 && !mbar_wait(bar(L::kDSFree), (pit - 1) & 1, abort_flag, p.f.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kTile / 32; ++c) {
+          uint32_t yr[32];
+          tmem_ld32_at(dp_col + 32 * c, yr);
+          tc_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            const uint4 pp = ld_shared_v4(sw128_unit(sbase + L::kP, r, 4 * c + v4));
+            const uint32_t pw4[4] = {pp.x, pp.y, pp.z, pp.w};
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+              const int e = 8 * v4 + 2 * z;
+              const float2 pf = unpack2<DT>(pw4[z]);
+              const float d0 = pf.x * (__uint_as_float(yr[e]) - drow);
+              const float d1 = pf.y * (__uint_as_float(yr[e + 1]) - drow);
+              pk[4 * v4 + z] = DT == SMA_BF16 ? pack_bf16x2(d0, d1) : pack_f16x2(d0, d1);
+            }
+          }
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            st_shared_v4(sw128_unit(sbase + L::kDS, r, 4 * c + v4), pk[4 * v4], pk[4 * v4 + 1],
+                         pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+        fence_async_shared();
+        tc_fence_before();
+        mbar_arrive(bar(L::kDSDone));
+        ++pit;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ drain, dK / dV epilogue
+    const int wq = warp - 4;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t dq_col = tmem + lane_off + L::kColDP;
+    const uint32_t dv_col = tmem + lane_off + L::kColDV;
+    const uint32_t dk_col = tmem + lane_off + L::kColDK;
+    typedef typename std::conditional<DT == SMA_BF16, __nv_bfloat16, __half>::type OutT;
+    uint32_t pit = 0, uit = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const BUnit w = bwd_unit(p, u);
+      const int key = w.kt * kTile + r;
+      OutT* dvrow = reinterpret_cast<OutT*>(p.dv) + w.b * p.dv_sb + static_cast<int64_t>(key) * p.dv_sr +
+                    w.hk * p.dv_sh;
+      OutT* dkrow = reinterpret_cast<OutT*>(p.dk) + w.b * p.dk_sb + static_cast<int64_t>(key) * p.dk_sr +
+                    w.hk * p.dk_sh;
+      if (w.n_pairs == 0) {  // keys no query attends: zero gradients
+        if (key < p.f.Lk) {
+          for (int e = 0; e < D / 8; ++e) {
+            reinterpret_cast<uint4*>(dvrow)[e] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4*>(dkrow)[e] = make_uint4(0, 0, 0, 0);
+          }
+        }
+        continue;
+      }
+      PairWalk pw;
+      pw.begin(p, w);
+      for (int i = 0; i < w.n_pairs && ok; ++i, pw.next(p, w)) {
+        bool partial;
+        const int qt = pw.qtile(p, w, &partial);
+        const int h = pw.head(w);
+        const int q = qt * kTile + r;
+        if (!mbar_wait(bar(L::kDQFull), pit & 1, abort_flag, p.f.err)) { ok = false; break; }
+        tc_fence_after();
+        float4* acc = reinterpret_cast<float4*>(
+            p.dq_acc + ((static_cast<int64_t>(w.b) * p.f.Lq + q) * p.f.H + h) * D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32_at(dq_col + 32 * c, v);
+          tc_wait_ld();
+          if (c == D / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(bar(L::kDQFree));
+          }
+          if (q < p.f.Lq) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              atomicAdd(acc + 8 * c + e,
+                        make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                    __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
+          }
+        }
+        ++pit;
+      }
+      if (!ok) break;
+      if (!mbar_wait(bar(L::kAccDone), uit & 1, abort_flag, p.f.err)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which == 0 ? dv_col : dk_col;
+        const float mul = which == 0 ? 1.f : p.scale;
+        OutT* dst = which == 0 ? dvrow : dkrow;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32_at(col + 32 * c, v);
+          tc_wait_ld();
+          if (key < p.f.Lk) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float a = __uint_as_float(v[2 * e]) * mul;
+              const float bq = __uint_as_float(v[2 * e + 1]) * mul;
+              pk[e] = DT == SMA_BF16 ? pack_bf16x2(a, bq) : pack_f16x2(a, bq);
+            }
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(L::kAccFree));
+      ++uit;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kBMmaWarp) tmem_dealloc(tmem, kBTmemCols);
+}
+
+// rowsum(dO * O) per (b, h, q) and the zeroed dQ accumulator; one warp per row.
+template <int DT>
+__global__ void bwd_prep_kernel(const BwdProblem p) {
+  const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = static_cast<int64_t>(p.f.B) * p.f.Lq * p.f.H;
+  if (gw >= rows) return;
+  const int h = static_cast<int>(gw % p.f.H);
+  const int64_t bq = gw / p.f.H;
+  const int q = static_cast<int>(bq % p.f.Lq);
+  const int b = static_cast<int>(bq / p.f.Lq);
+  const int d = p.f.d;
+  const void* orow = reinterpret_cast<const uint8_t*>(p.f.o) +
+                     (b * p.f.o_sb + static_cast<int64_t>(q) * p.f.o_sr + h * p.f.o_sh) * (DT == SMA_FP32 ? 4 : 2);
+  const void* grow = reinterpret_cast<const uint8_t*>(p.dout) +
+                     (b * p.do_sb + static_cast<int64_t>(q) * p.do_sr + h * p.do_sh) * (DT == SMA_FP32 ? 4 : 2);
+  float s = 0.f;
+  for (int e = lane; e < d; e += 32) s += load_as_float<DT>(orow, e) * load_as_float<DT>(grow, e);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) p.dvec[(static_cast<int64_t>(b) * p.f.H + h) * p.f.Lq + q] = s;
+  float* acc = p.dq_acc + gw * d;
+  for (int e = lane; e < d; e += 32) acc[e] = 0.f;
+}
+
+// codes[row][qt][kt] from the forward lists (2 = FULL, 1 = PARTIAL); the
+// buffer is zeroed first.
+__global__ void scatter_codes_kernel(const BwdProblem p, uint8_t* codes) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t rows = static_cast<int64_t>(p.f.lists.LB) * p.f.lists.LH * p.f.QT;
+  if (t >= rows * p.f.KT) return;
+  const int64_t lrow = t / p.f.KT;  // (row, qt)
+  const int j = static_cast<int>(t - lrow * p.f.KT);
+  const int nf = p.f.lists.num_full[lrow], np = p.f.lists.num_part[lrow];
+  uint8_t* c = codes + lrow * p.f.KT;
+  if (j < nf) {
+    const int kt = p.f.lists.full_idx[lrow * p.f.KT + j];
+    if (kt >= 0 && kt < p.f.KT) c[kt] = 2;
+  }
+  if (j < np) {
+    const int kt = p.f.lists.part_idx[lrow * p.f.KT + j];
+    if (kt >= 0 && kt < p.f.KT) c[kt] = 1;
+  }
+}
+
+// Per (row, key tile): ascending query tiles, FULL and PARTIAL lists.
+constexpr int kTrThreads = 128;
+__global__ void __launch_bounds__(kTrThreads) transpose_lists_kernel(const BwdProblem p,
+                                                                      const uint8_t* codes) {
+  const int kt = blockIdx.x;
+  const int64_t row = blockIdx.y;
+  __shared__ uint32_t s_warp[kTrThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t out = (row * p.f.KT + kt);
+  int32_t* tf = const_cast<int32_t*>(p.t_full) + out * p.f.QT;
+  int32_t* tp = const_cast<int32_t*>(p.t_part) + out * p.f.QT;
+  uint32_t nf = 0, np = 0;
+  for (int q0 = 0; q0 < p.f.QT; q0 += kTrThreads) {
+    const int qt = q0 + threadIdx.x;
+    const uint8_t code = qt < p.f.QT ? codes[(row * p.f.QT + qt) * p.f.KT + kt] : 0;
+    const uint32_t v = (code == 2 ? 1u : 0u) | (code == 1 ? 0x10000u : 0u);
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t2 = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t2;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    uint32_t base = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kTrThreads / 32; ++w) {
+      base += w < warp ? s_warp[w] : 0u;
+      tot += s_warp[w];
+    }
+    __syncthreads();
+    const uint32_t ex = base + incl - v;
+    if (code == 2) tf[nf + (ex & 0xffffu)] = qt;
+    if (code == 1) tp[np + (ex >> 16)] = qt;
+    nf += tot & 0xffffu;
+    np += tot >> 16;
+  }
+  for (int i = nf + threadIdx.x; i < p.f.QT; i += kTrThreads) tf[i] = -1;
+  for (int i = np + threadIdx.x; i < p.f.QT; i += kTrThreads) tp[i] = -1;
+  if (threadIdx.x == 0) {
+    const_cast<int32_t*>(p.t_num_full)[out] = static_cast<int32_t>(nf);
+    const_cast<int32_t*>(p.t_num_part)[out] = static_cast<int32_t>(np);
+  }
+}
+
+// dQ = scale * accumulator, in the output dtype; one thread per 4 elements.
+template <int DT>
+__global__ void dq_convert_kernel(const BwdProblem p) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int d4 = p.f.d / 4;
+  const int64_t total = static_cast<int64_t>(p.f.B) * p.f.Lq * p.f.H * d4;
+  if (t >= total) return;
+  const int e = static_cast<int>(t % d4) * 4;
+  const int64_t row = t / d4;  // (b, q, h)
+  const int h = static_cast<int>(row % p.f.H);
+  const int64_t bq = row / p.f.H;
+  const int q = static_cast<int>(bq % p.f.Lq);
+  const int b = static_cast<int>(bq / p.f.Lq);
+  const float4 a = reinterpret_cast<const float4*>(p.dq_acc + row * p.f.d + e)[0];
+  const int64_t off = b * p.dq_sb + static_cast<int64_t>(q) * p.dq_sr + h * p.dq_sh + e;
+  if (DT == SMA_FP32) {
+    float* dst = reinterpret_cast<float*>(p.dq) + off;
+    dst[0] = a.x * p.scale; dst[1] = a.y * p.scale; dst[2] = a.z * p.scale; dst[3] = a.w * p.scale;
+  } else {
+    const uint32_t w0 = DT == SMA_BF16 ? pack_bf16x2(a.x * p.scale, a.y * p.scale)
+                                       : pack_f16x2(a.x * p.scale, a.y * p.scale);
+    const uint32_t w1 = DT == SMA_BF16 ? pack_bf16x2(a.z * p.scale, a.w * p.scale)
+                                       : pack_f16x2(a.z * p.scale, a.w * p.scale);
+    *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.dq) + off) = make_uint2(w0, w1);
+  }
+}
+
+template <int D, int POLICY, int DT>
+cudaError_t launch_bwd_typed(const BwdProblem& p, const CUtensorMap& mq, const CUtensorMap& mk,
+                             const CUtensorMap& mv, const CUtensorMap& mdo, cudaStream_t stream) {
+  using L = BLayout<D>;
+  auto kern = attn_bwd_kernel<D, POLICY, DT>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(L::kAlloc));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int n_units = p.f.B * p.f.KVH * p.f.KT;
+  if (n_units == 0) return cudaSuccess;
+  const int grid = n_units < num_sms() ? n_units : num_sms();
+  kern<<<grid, kBwdThreads, L::kAlloc, stream>>>(p, mq, mk, mv, mdo, n_units);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_prep(const BwdProblem& p, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(p.f.B) * p.f.Lq * p.f.H;
+  const int block = 256;
+  const unsigned grid = static_cast<unsigned>((rows * 32 + block - 1) / block);
+  if (p.f.dtype == SMA_BF16) bwd_prep_kernel<SMA_BF16><<<grid, block, 0, stream>>>(p);
+  else if (p.f.dtype == SMA_FP16) bwd_prep_kernel<SMA_FP16><<<grid, block, 0, stream>>>(p);
+  else bwd_prep_kernel<SMA_FP32><<<grid, block, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_lists(const BwdProblem& p, uint8_t* codes, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(p.f.lists.LB) * p.f.lists.LH;
+  cudaError_t e = cudaMemsetAsync(codes, 0, static_cast<size_t>(rows * p.f.QT * p.f.KT), stream);
+  if (e != cudaSuccess) return e;
+  const int64_t n = rows * p.f.QT * p.f.KT;
+  scatter_codes_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(p, codes);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  transpose_lists_kernel<<<dim3(p.f.KT, static_cast<unsigned>(rows)), kTrThreads, 0, stream>>>(p, codes);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dq_convert(const BwdProblem& p, cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>(p.f.B) * p.f.Lq * p.f.H * (p.f.d / 4);
+  const unsigned grid = static_cast<unsigned>((total + 255) / 256);
+  if (p.f.dtype == SMA_BF16) dq_convert_kernel<SMA_BF16><<<grid, 256, 0, stream>>>(p);
+  else if (p.f.dtype == SMA_FP16) dq_convert_kernel<SMA_FP16><<<grid, 256, 0, stream>>>(p);
+  else dq_convert_kernel<SMA_FP32><<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+int launch_attn_bwd(const BwdProblem& p, cudaStream_t stream, char* msg, size_t msg_len) {
+  const AttnProblem& f = p.f;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!encode_map(&mq, f.q, f.dtype, f.d, f.H, f.Lq, f.B, f.q_sh, f.q_sr, f.q_sb, msg, msg_len) ||
+      !encode_map(&mk, f.k, f.dtype, f.d, f.KVH, f.Lk, f.B, f.k_sh, f.k_sr, f.k_sb, msg, msg_len) ||
+      !encode_map(&mv, f.v, f.dtype, f.d, f.KVH, f.Lk, f.B, f.v_sh, f.v_sr, f.v_sb, msg, msg_len) ||
+      !encode_map(&mdo, p.dout, f.dtype, f.d, f.H, f.Lq, f.B, p.do_sh, p.do_sr, p.do_sb, msg, msg_len))
+    return SMA_ERR_CUDA;
+  cudaError_t e = cudaErrorInvalidValue;
+  const bool bf = f.dtype == SMA_BF16;
+  if (f.policy == kPolicyDflash) {
+    if (f.d == 128) e = bf ? launch_bwd_typed<128, kPolicyDflash, SMA_BF16>(p, mq, mk, mv, mdo, stream)
+                           : launch_bwd_typed<128, kPolicyDflash, SMA_FP16>(p, mq, mk, mv, mdo, stream);
+    else e = bf ? launch_bwd_typed<64, kPolicyDflash, SMA_BF16>(p, mq, mk, mv, mdo, stream)
+                : launch_bwd_typed<64, kPolicyDflash, SMA_FP16>(p, mq, mk, mv, mdo, stream);
+  } else {
+    if (f.d == 128) e = bf ? launch_bwd_typed<128, kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, mdo, stream)
+                           : launch_bwd_typed<128, kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, mdo, stream);
+    else e = bf ? launch_bwd_typed<64, kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, mdo, stream)
+                : launch_bwd_typed<64, kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, mdo, stream);
+  }
+  if (e != cudaSuccess) {
+    snprintf(msg, msg_len, "attention backward launch failed: %s", cudaGetErrorString(e));
+    return SMA_ERR_CUDA;
+  }
+  return SMA_OK;
+}
+
+}  // namespace sma

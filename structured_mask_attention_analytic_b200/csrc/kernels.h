@@ -82,6 +82,23 @@ struct AttnProblem {
   int* err;  // device error word
 };
 
+// Backward of one attention problem.  `f` is the forward problem (q, k, v,
+// geometry, policy, masks and the forward tile lists, f.o = the forward
+// output O, f.lse = its log-sum-exp, read only); the transposed lists give,
+// per list row and key tile, the query tiles that attend it.
+struct BwdProblem {
+  AttnProblem f;
+  const void* dout; int64_t do_sb, do_sr, do_sh;   // upstream gradient dO [B, Lq, H, d]
+  void* dq; int64_t dq_sb, dq_sr, dq_sh;           // [B, Lq, H, d]
+  void* dk; int64_t dk_sb, dk_sr, dk_sh;           // [B, Lk, KVH, d]
+  void* dv; int64_t dv_sb, dv_sr, dv_sh;
+  float* dq_acc;   // [B, Lq, H, d] fp32, zeroed by the preparation kernel
+  float* dvec;     // [B, H, Lq]: rowsum(dO * O)
+  const int32_t* t_num_full; const int32_t* t_full;  // [rows, KT], [rows, KT, QT]
+  const int32_t* t_num_part; const int32_t* t_part;
+  float scale;     // softmax scale (dQ and dK carry it)
+};
+
 // Single-query (decode) problem after the grouped-head swap: for each
 // (b, kv head) the `group` query heads are the rows.
 struct DecodeProblem {
@@ -151,6 +168,14 @@ cudaError_t launch_gather_bias(const AttnProblem& p, const AuxView& bias, int ro
 cudaError_t launch_gather_lists(const AttnProblem& p, cudaStream_t stream);
 
 cudaError_t launch_topk(const TopkProblem& p, cudaStream_t stream);
+
+// Backward: rowsum(dO * O) and a zeroed dQ accumulator; the transposed tile
+// lists (codes: scratch of rows * QT * KT bytes); the tcgen05 kernel (dK, dV
+// and dQ partial sums); dQ = scale * accumulator in the output dtype.
+cudaError_t launch_bwd_prep(const BwdProblem& p, cudaStream_t stream);
+cudaError_t launch_transpose_lists(const BwdProblem& p, uint8_t* codes, cudaStream_t stream);
+int launch_attn_bwd(const BwdProblem& p, cudaStream_t stream, char* msg, size_t msg_len);
+cudaError_t launch_dq_convert(const BwdProblem& p, cudaStream_t stream);
 
 // Records `message` as the calling thread's last error (read back through
 // sma_last_error) and returns `code`.

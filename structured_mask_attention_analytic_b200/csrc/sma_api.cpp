@@ -228,6 +228,73 @@ MaskedGeom masked_geom(int32_t B, int32_t H, int32_t KVH, int32_t Lq, int32_t Lk
 }
 
 
+// ---- backward workspace: forward tile lists (unless given), transposed
+// lists, tile codes, rowsum(dO * O) and the fp32 dQ accumulator.
+struct BwdLayout {
+  ListsLayout fl;
+  size_t tnf, tnp, tf, tp, codes, dvec, dqacc, total;
+};
+
+BwdLayout bwd_layout(size_t base, int64_t rows, int QT, int KT, int B, int H, int Lq, int d) {
+  BwdLayout l;
+  l.fl = lists_layout(base, rows * QT, KT);
+  l.tnf = l.fl.end;
+  l.tnp = align256(l.tnf + static_cast<size_t>(rows) * KT * 4);
+  l.tf = align256(l.tnp + static_cast<size_t>(rows) * KT * 4);
+  l.tp = align256(l.tf + static_cast<size_t>(rows) * KT * QT * 4);
+  l.codes = align256(l.tp + static_cast<size_t>(rows) * KT * QT * 4);
+  l.dvec = align256(l.codes + static_cast<size_t>(rows) * QT * KT);
+  l.dqacc = align256(l.dvec + static_cast<size_t>(B) * H * Lq * 4);
+  l.total = align256(l.dqacc + static_cast<size_t>(B) * Lq * H * d * 4);
+  return l;
+}
+
+// Runs the backward launches for a filled problem (forward lists in place).
+sma_status run_backward(BwdProblem& b, void* ws, const BwdLayout& l, cudaStream_t st) {
+  b.t_num_full = at<int32_t>(ws, l.tnf);
+  b.t_num_part = at<int32_t>(ws, l.tnp);
+  b.t_full = at<int32_t>(ws, l.tf);
+  b.t_part = at<int32_t>(ws, l.tp);
+  b.dvec = at<float>(ws, l.dvec);
+  b.dq_acc = at<float>(ws, l.dqacc);
+  cudaError_t e = launch_bwd_prep(b, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward preparation launch failed");
+  e = launch_transpose_lists(b, at<uint8_t>(ws, l.codes), st);
+  if (e != cudaSuccess) return cuda_fail(e, "tile list transpose launch failed");
+  char msg[256];
+  const int rc = launch_attn_bwd(b, st, msg, sizeof(msg));
+  if (rc != SMA_OK) return fail(rc, "%s", msg);
+  e = launch_dq_convert(b, st);
+  if (e != cudaSuccess) return cuda_fail(e, "dQ conversion launch failed");
+  return SMA_OK;
+}
+
+sma_status check_grad_operands(int32_t dtype, int64_t lq, int64_t lk, const void* out,
+                               const int64_t* o_strides, const float* lse, const void* dout,
+                               const int64_t* do_strides, const void* dq, const int64_t* dq_strides,
+                               const void* dk, const int64_t* dk_strides, const void* dv,
+                               const int64_t* dv_strides) {
+  sma_status s;
+  if (dtype == SMA_FP32)
+    return fail(SMA_ERR_UNSUPPORTED, "the backward runs on the tensor cores: bf16 or fp16 only");
+  if ((s = check_operand("out", out, o_strides, dtype, lq)) != SMA_OK) return s;
+  if ((s = check_operand("dout", dout, do_strides, dtype, lq)) != SMA_OK) return s;
+  if ((s = check_operand("dq", dq, dq_strides, dtype, lq)) != SMA_OK) return s;
+  if ((s = check_operand("dk", dk, dk_strides, dtype, lk)) != SMA_OK) return s;
+  if ((s = check_operand("dv", dv, dv_strides, dtype, lk)) != SMA_OK) return s;
+  if (lse == nullptr) return fail(SMA_ERR_INVALID_ARG, "lse is NULL (the forward's log-sum-exp is required)");
+  return SMA_OK;
+}
+
+void set_grads(BwdProblem& b, const void* dout, const int64_t* ds, void* dq, const int64_t* qs,
+               void* dk, const int64_t* ks, void* dv, const int64_t* vs, float scale) {
+  b.dout = dout; b.do_sb = ds[0]; b.do_sr = ds[1]; b.do_sh = ds[2];
+  b.dq = dq; b.dq_sb = qs[0]; b.dq_sr = qs[1]; b.dq_sh = qs[2];
+  b.dk = dk; b.dk_sb = ks[0]; b.dk_sr = ks[1]; b.dk_sh = ks[2];
+  b.dv = dv; b.dv_sb = vs[0]; b.dv_sr = vs[1]; b.dv_sh = vs[2];
+  b.scale = scale;
+}
+
 // ---- index-gather path geometry: kept-key lists, tile lists over the
 // compacted keys, compacted K/V and bias, all in the workspace.
 struct SparseGeom {
@@ -773,6 +840,187 @@ sma_status sparse_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   char msg[256];
   const int rc = launch_attn_tc(p, st, msg, sizeof(msg));
   if (rc != SMA_OK) return fail(rc, "%s", msg);
+  return ok();
+}
+
+sma_status dfa_attn_bwd_workspace_size(const dfa_mask_desc* desc, int32_t heads, int32_t kv_heads,
+                                       int32_t head_dim, size_t* bytes) {
+  if (bytes == nullptr) return fail(SMA_ERR_INVALID_ARG, "bytes is NULL");
+  sma_status s = check_desc(desc);
+  if (s != SMA_OK) return s;
+  if ((s = check_heads(heads, kv_heads, head_dim)) != SMA_OK) return s;
+  const DflashGeom g = make_geom(desc);
+  *bytes = bwd_layout(0, g.B, g.QT, g.KT, g.B, heads, g.Nq, head_dim).total;
+  return ok();
+}
+
+sma_status dfa_attn_bwd(const dfa_mask_desc* desc, const int32_t* anchors, int32_t dtype,
+                        int32_t heads, int32_t kv_heads, int32_t head_dim, float scale,
+                        const void* q, const int64_t q_strides[3], const void* k,
+                        const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
+                        const void* out, const int64_t o_strides[3], const float* lse,
+                        const void* dout, const int64_t do_strides[3], void* dq,
+                        const int64_t dq_strides[3], void* dk, const int64_t dk_strides[3],
+                        void* dv, const int64_t dv_strides[3], void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  sma_status s = check_desc(desc);
+  if (s != SMA_OK) return s;
+  if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if ((s = check_heads(heads, kv_heads, head_dim)) != SMA_OK) return s;
+  if (anchors == nullptr) return fail(SMA_ERR_INVALID_ARG, "anchors is NULL");
+  const DflashGeom g = make_geom(desc);
+  if ((s = check_operand("q", q, q_strides, dtype, g.Nq)) != SMA_OK) return s;
+  if ((s = check_operand("k", k, k_strides, dtype, g.Lk)) != SMA_OK) return s;
+  if ((s = check_operand("v", v, v_strides, dtype, g.Lk)) != SMA_OK) return s;
+  if ((s = check_grad_operands(dtype, g.Nq, g.Lk, out, o_strides, lse, dout, do_strides, dq,
+                               dq_strides, dk, dk_strides, dv, dv_strides)) != SMA_OK)
+    return s;
+  const BwdLayout lay = bwd_layout(0, g.B, g.QT, g.KT, g.B, heads, g.Nq, head_dim);
+  if ((s = check_workspace(workspace, workspace_bytes, lay.total)) != SMA_OK) return s;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (err == nullptr) return cuda_fail(e, "device error word unavailable");
+  int32_t* nf = at<int32_t>(workspace, lay.fl.nf);
+  int32_t* np = at<int32_t>(workspace, lay.fl.np);
+  int32_t* fi = at<int32_t>(workspace, lay.fl.fi);
+  int32_t* pi = at<int32_t>(workspace, lay.fl.pi);
+  e = launch_dfa_block_map(g, anchors, nf, fi, np, pi, err, st);
+  if (e != cudaSuccess) return cuda_fail(e, "block map launch failed");
+
+  BwdProblem b{};
+  AttnProblem& p = b.f;
+  p.dtype = dtype;
+  p.B = g.B; p.H = heads; p.KVH = kv_heads; p.Lq = g.Nq; p.Lk = g.Lk; p.d = head_dim;
+  p.group = heads / kv_heads;
+  p.npairs = (p.group + 1) / 2;
+  p.QT = g.QT; p.KT = g.KT;
+  const float sc = resolve_scale(scale, head_dim);
+  p.scale_log2 = sc * kLog2eHost;
+  p.q = q; p.q_sb = q_strides[0]; p.q_sr = q_strides[1]; p.q_sh = q_strides[2];
+  p.k = k; p.k_sb = k_strides[0]; p.k_sr = k_strides[1]; p.k_sh = k_strides[2];
+  p.v = v; p.v_sb = v_strides[0]; p.v_sr = v_strides[1]; p.v_sh = v_strides[2];
+  p.o = const_cast<void*>(out); p.o_sb = o_strides[0]; p.o_sr = o_strides[1]; p.o_sh = o_strides[2];
+  p.lse = const_cast<float*>(lse);
+  p.lists.num_full = nf; p.lists.full_idx = fi; p.lists.num_part = np; p.lists.part_idx = pi;
+  p.lists.LB = g.B; p.lists.LH = 1; p.lists.head_mode = 0;
+  p.policy = kPolicyDflash;
+  p.anchors = anchors; p.N = g.N; p.bs = g.bs; p.Lc = g.Lc;
+  p.causal_in_block = g.causal; p.window = g.window;
+  p.err = err;
+  set_grads(b, dout, do_strides, dq, dq_strides, dk, dk_strides, dv, dv_strides, sc);
+  if ((s = run_backward(b, workspace, lay, st)) != SMA_OK) return s;
+  return ok();
+}
+
+sma_status masked_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t kv_heads,
+                                          int32_t q_len, int32_t k_len, int32_t head_dim,
+                                          const int64_t mask_sizes[4], size_t* bytes) {
+  if (bytes == nullptr) return fail(SMA_ERR_INVALID_ARG, "bytes is NULL");
+  sma_status s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (batch < 1 || q_len < 1 || k_len < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, q_len and k_len must be >= 1");
+  // the prefill geometry (tile lists), whatever q_len is
+  const MaskedGeom mg = masked_geom(batch, heads, kv_heads, q_len < 2 ? 2 : q_len, k_len, head_dim,
+                                    mask_sizes);
+  const int QT = static_cast<int>(ceil_div(q_len, kTile));
+  const int KT = static_cast<int>(ceil_div(k_len, kTile));
+  *bytes = bwd_layout(mg.codes_bytes, static_cast<int64_t>(mg.LB) * mg.LH, QT, KT, batch, heads,
+                      q_len, head_dim).total;
+  return ok();
+}
+
+sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t q_len, int32_t k_len, int32_t head_dim, float scale,
+                           int32_t is_causal, const void* q, const int64_t q_strides[3],
+                           const void* k, const int64_t k_strides[3], const void* v,
+                           const int64_t v_strides[3], const uint8_t* mask,
+                           const int64_t mask_sizes[4], const int64_t mask_strides[4],
+                           const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+                           const int64_t bias_strides[4], const void* out,
+                           const int64_t o_strides[3], const float* lse, const void* dout,
+                           const int64_t do_strides[3], void* dq, const int64_t dq_strides[3],
+                           void* dk, const int64_t dk_strides[3], void* dv,
+                           const int64_t dv_strides[3], float* dbias, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  sma_status s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (batch < 1 || q_len < 1 || k_len < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, q_len and k_len must be >= 1");
+  if (is_causal != 0 && is_causal != 1) return fail(SMA_ERR_INVALID_ARG, "is_causal must be 0 or 1");
+  if (dbias != nullptr) return fail(SMA_ERR_UNSUPPORTED, "dbias is not produced by this build");
+  if ((s = check_operand("q", q, q_strides, dtype, q_len)) != SMA_OK) return s;
+  if ((s = check_operand("k", k, k_strides, dtype, k_len)) != SMA_OK) return s;
+  if ((s = check_operand("v", v, v_strides, dtype, k_len)) != SMA_OK) return s;
+  if ((s = check_grad_operands(dtype, q_len, k_len, out, o_strides, lse, dout, do_strides, dq,
+                               dq_strides, dk, dk_strides, dv, dv_strides)) != SMA_OK)
+    return s;
+  AuxView mview, bview;
+  const bool has_mask = mask != nullptr, has_bias = bias != nullptr;
+  if (has_mask && (s = check_aux("mask", mask, mask_sizes, mask_strides, 1, batch, heads, kv_heads,
+                                 q_len, k_len, true, &mview)) != SMA_OK)
+    return s;
+  if (has_bias) {
+    if (!valid_dtype(bias_dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown bias dtype %d", bias_dtype);
+    if ((s = check_aux("bias", bias, bias_sizes, bias_strides, elem_size(bias_dtype), batch, heads,
+                       kv_heads, q_len, k_len, true, &bview)) != SMA_OK)
+      return s;
+    bview.dtype = bias_dtype;
+  }
+  const MaskedGeom mg = masked_geom(batch, heads, kv_heads, q_len < 2 ? 2 : q_len, k_len, head_dim,
+                                    has_mask ? mask_sizes : nullptr);
+  const int QT = static_cast<int>(ceil_div(q_len, kTile));
+  const int KT = static_cast<int>(ceil_div(k_len, kTile));
+  const BwdLayout lay = bwd_layout(mg.codes_bytes, static_cast<int64_t>(mg.LB) * mg.LH, QT, KT,
+                                   batch, heads, q_len, head_dim);
+  if ((s = check_workspace(workspace, workspace_bytes, lay.total)) != SMA_OK) return s;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (err == nullptr) return cuda_fail(e, "device error word unavailable");
+  BwdProblem b{};
+  AttnProblem& p = b.f;
+  p.dtype = dtype;
+  p.B = batch; p.H = heads; p.KVH = kv_heads; p.Lq = q_len; p.Lk = k_len; p.d = head_dim;
+  p.group = heads / kv_heads;
+  p.npairs = mg.npairs;
+  p.QT = QT; p.KT = KT;
+  const float sc = resolve_scale(scale, head_dim);
+  p.scale_log2 = sc * kLog2eHost;
+  p.q = q; p.q_sb = q_strides[0]; p.q_sr = q_strides[1]; p.q_sh = q_strides[2];
+  p.k = k; p.k_sb = k_strides[0]; p.k_sr = k_strides[1]; p.k_sh = k_strides[2];
+  p.v = v; p.v_sb = v_strides[0]; p.v_sr = v_strides[1]; p.v_sh = v_strides[2];
+  p.o = const_cast<void*>(out); p.o_sb = o_strides[0]; p.o_sr = o_strides[1]; p.o_sh = o_strides[2];
+  p.lse = const_cast<float*>(lse);
+  p.policy = kPolicyExplicit;
+  p.causal = is_causal;
+  p.has_mask = has_mask;
+  p.has_bias = has_bias;
+  if (has_mask) p.mask = mview;
+  if (has_bias) p.bias = bview;
+  p.err = err;
+  p.lists.LB = mg.LB;
+  p.lists.LH = mg.LH;
+  p.lists.head_mode = mg.head_mode;
+  int32_t* nf = at<int32_t>(workspace, lay.fl.nf);
+  int32_t* np = at<int32_t>(workspace, lay.fl.np);
+  int32_t* fi = at<int32_t>(workspace, lay.fl.fi);
+  int32_t* pi = at<int32_t>(workspace, lay.fl.pi);
+  p.lists.num_full = nf; p.lists.num_part = np; p.lists.full_idx = fi; p.lists.part_idx = pi;
+  uint8_t* codes = has_mask ? at<uint8_t>(workspace, 0) : nullptr;
+  if (has_mask) {
+    const int64_t folded[4] = {mview.sb, mview.sh, mview.sq, 1};
+    e = launch_mask_tile_summary(mask, mask_sizes, folded, k_len, codes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "mask summary launch failed");
+  }
+  e = launch_explicit_lists(p, codes, mg.codes_qt, nf, fi, np, pi, st);
+  if (e != cudaSuccess) return cuda_fail(e, "tile list launch failed");
+  set_grads(b, dout, do_strides, dq, dq_strides, dk, dk_strides, dv, dv_strides, sc);
+  if ((s = run_backward(b, workspace, lay, st)) != SMA_OK) return s;
   return ok();
 }
 

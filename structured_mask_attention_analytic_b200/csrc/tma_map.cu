@@ -1,0 +1,60 @@
+// TMA tensor-map encoding through the driver entry point (no libcuda link).
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+
+#include "sma.h"
+#include "tma_map.h"
+
+namespace sma {
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+}  // namespace
+
+// 4D map over [B][len][heads][d] (d contiguous), box = 64 x 1 x 128 x 1,
+// 128-byte swizzle, zero fill outside the tensor.
+bool encode_map(CUtensorMap* map, const void* ptr, int dtype, int d, int heads, int len, int batch,
+                int64_t s_head, int64_t s_row, int64_t s_batch, char* msg, size_t msg_len) {
+  auto enc = get_encode_fn();
+  if (enc == nullptr) {
+    snprintf(msg, msg_len, "cuTensorMapEncodeTiled is unavailable");
+    return false;
+  }
+  const int esz = 2;
+  // A size-1 dim's stride is never used; give it a legal value.
+  if (heads == 1) s_head = d;
+  if (len == 1) s_row = s_head * heads;
+  if (batch == 1) s_batch = s_row * len;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(len), static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(s_head * esz),
+                           static_cast<cuuint64_t>(s_row * esz),
+                           static_cast<cuuint64_t>(s_batch * esz)};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(SMA_TILE), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, dtype == SMA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   4, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(msg, msg_len, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return false;
+  }
+  return true;
+}
+
+}  // namespace sma

@@ -1,0 +1,17 @@
+// Host-side TMA tensor maps of the [batch][len][heads][d] operands.
+#pragma once
+
+#include <cuda.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sma {
+
+// 4D map over [B][len][heads][d] (d contiguous, 16-bit elements), box =
+// 64 x 1 x 128 x 1, 128-byte swizzle, zero fill outside the tensor.  Returns
+// false and writes a message if the driver entry point is missing or the
+// encoding is rejected.
+bool encode_map(CUtensorMap* map, const void* ptr, int dtype, int d, int heads, int len, int batch,
+                int64_t s_head, int64_t s_row, int64_t s_batch, char* msg, size_t msg_len);
+
+}  // namespace sma

@@ -151,6 +151,53 @@ def dfa_attn_fwd(q, k, v, anchors, ctx_len: int, block_size: int, is_causal=None
     return out, lse
 
 
+def dfa_attn_bwd_workspace_size(batch, n_blocks, block_size, ctx_len, heads, kv_heads, head_dim,
+                                is_causal=None, layer_type=LAYER_FULL, sliding_window=0) -> int:
+    d = _desc(batch, n_blocks, block_size, ctx_len, is_causal, layer_type, sliding_window)
+    n = ctypes.c_size_t()
+    nat.check(_lib().dfa_attn_bwd_workspace_size(ctypes.byref(d), heads, kv_heads, head_dim,
+                                                 ctypes.byref(n)))
+    return n.value
+
+
+def _grad_outputs(q, k, dq, dk, dv):
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(k) if dv is None else dv
+    return dq, dk, dv
+
+
+def dfa_attn_bwd(q, k, v, out, lse, dout, anchors, ctx_len: int, block_size: int, is_causal=None,
+                 layer_type: int = LAYER_FULL, sliding_window: int = 0, scale=None, dq=None, dk=None,
+                 dv=None, workspace=None):
+    """Gradients of ``dfa_attn_fwd``: ``out`` and ``lse`` are that call's
+    results for the same arguments, ``dout`` the upstream gradient.
+    Returns ``(dq, dk, dv)``."""
+    _require_cuda(q, k, v, out, lse, dout, anchors)
+    b, nq, h, dh = q.shape
+    kvh = k.shape[2]
+    if anchors.dtype != torch.int32 or anchors.dim() != 2 or anchors.shape[0] != b:
+        raise ValueError("anchors must be int32 [batch, n_blocks]")
+    anchors = anchors.contiguous()
+    n = anchors.shape[1]
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (b, h, nq) or not lse.is_contiguous():
+        raise ValueError("lse must be the forward's contiguous float32 [batch, heads, q_len]")
+    d = _desc(b, n, block_size, ctx_len, is_causal, layer_type, sliding_window)
+    dq, dk, dv = _grad_outputs(q, k, dq, dk, dv)
+    ws_bytes = dfa_attn_bwd_workspace_size(b, n, block_size, ctx_len, h, kvh, dh, is_causal, layer_type,
+                                           sliding_window)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    nat.check(_lib().dfa_attn_bwd(
+        ctypes.byref(d), _ptr(anchors), _dtype_code(q), h, kvh, dh,
+        ctypes.c_float(0.0 if scale is None else float(scale)),
+        _ptr(q), _strides3(q), _ptr(k), _strides3(k), _ptr(v), _strides3(v),
+        _ptr(out), _strides3(out), _ptr(lse), _ptr(dout), _strides3(dout),
+        _ptr(dq), _strides3(dq), _ptr(dk), _strides3(dk), _ptr(dv), _strides3(dv),
+        _ptr(workspace), workspace.numel(), _stream(q)))
+    return dq, dk, dv
+
+
 def dfa_attn_fwd_noalloc(q, k, v, anchors, ctx_len: int, block_size: int, is_causal=None,
                          layer_type: int = LAYER_FULL, sliding_window: int = 0, scale=None, out=None,
                          return_lse: bool = True):
@@ -237,6 +284,43 @@ def masked_attn_fwd(q, k, v, mask=None, bias=None, is_causal: bool = False, scal
         bp, _dtype_code(bias) if bias is not None else 0, bsz, bst,
         _ptr(out), _strides3(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(q)))
     return out, lse
+
+
+def masked_attn_bwd_workspace_size(batch, heads, kv_heads, q_len, k_len, head_dim, mask_shape=None) -> int:
+    n = ctypes.c_size_t()
+    ms = nat.i64_array(mask_shape) if mask_shape is not None else None
+    nat.check(_lib().masked_attn_bwd_workspace_size(batch, heads, kv_heads, q_len, k_len, head_dim, ms,
+                                                    ctypes.byref(n)))
+    return n.value
+
+
+def masked_attn_bwd(q, k, v, out, lse, dout, mask=None, bias=None, is_causal: bool = False, scale=None,
+                    dq=None, dk=None, dv=None, workspace=None):
+    """Gradients of ``masked_attn_fwd`` (same mask / bias / causal / scale):
+    ``out`` and ``lse`` are that call's results, ``dout`` the upstream
+    gradient.  Returns ``(dq, dk, dv)``; no bias gradient."""
+    _require_cuda(q, k, v, out, lse, dout, mask, bias)
+    b, lq, h, dh = q.shape
+    lk, kvh = k.shape[1], k.shape[2]
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (b, h, lq) or not lse.is_contiguous():
+        raise ValueError("lse must be the forward's contiguous float32 [batch, heads, q_len]")
+    dq, dk, dv = _grad_outputs(q, k, dq, dk, dv)
+    ws_bytes = masked_attn_bwd_workspace_size(b, h, kvh, lq, lk, dh,
+                                              tuple(mask.shape) if mask is not None else None)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    mp, msz, mst = _aux_args(mask, lk)
+    bp, bsz, bst = _aux_args(bias, lk)
+    nat.check(_lib().masked_attn_bwd(
+        _dtype_code(q), b, h, kvh, lq, lk, dh, ctypes.c_float(0.0 if scale is None else float(scale)),
+        1 if is_causal else 0,
+        _ptr(q), _strides3(q), _ptr(k), _strides3(k), _ptr(v), _strides3(v),
+        mp, msz, mst,
+        bp, _dtype_code(bias) if bias is not None else 0, bsz, bst,
+        _ptr(out), _strides3(out), _ptr(lse), _ptr(dout), _strides3(dout),
+        _ptr(dq), _strides3(dq), _ptr(dk), _strides3(dk), _ptr(dv), _strides3(dv),
+        ctypes.c_void_p(0), _ptr(workspace), workspace.numel(), _stream(q)))
+    return dq, dk, dv
 
 
 def sparse_attn_fwd_workspace_size(dtype, batch, heads, kv_heads, q_len, k_len, head_dim, mask_shape,

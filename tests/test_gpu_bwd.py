@@ -1,0 +1,135 @@
+"""GPU: dfa_attn_bwd / masked_attn_bwd (tcgen05 backward) agree with the
+float64 oracle's gradients (oracle.attention_grad, pinned by finite
+differences) under DFlash and explicit masks, grouped heads, ragged tiles,
+and keys that no query attends."""
+import numpy as np
+import pytest
+import torch
+
+import structured_mask_attention_analytic_b200 as sma
+import workloads as wl
+from oracle import attention as at
+from oracle import attention_grad as ag
+from oracle import dflash_mask as dm
+from tests._helpers import f64
+
+pytestmark = pytest.mark.gpu
+
+# Gradient agreement (bf16 / fp16 operands, fp32 accumulation): relative to
+# the largest reference magnitude m = max(1, max |ref|) of each tensor,
+# max-abs <= 2.5e-2 m and mean-abs <= 2.5e-3 m.
+GRAD_TOL = (2.5e-2, 2.5e-3)
+
+
+def _close(name, got, ref):
+    g = f64(got)
+    m = max(1.0, float(np.abs(ref).max()))
+    err = np.abs(g - ref)
+    assert np.isfinite(g).all(), f"{name}: non-finite"
+    assert err.max() <= GRAD_TOL[0] * m, f"{name}: max abs err {err.max():.3e} (scale {m:.2f})"
+    assert err.mean() <= GRAD_TOL[1] * m, f"{name}: mean abs err {err.mean():.3e} (scale {m:.2f})"
+
+
+def _dflash_case(seed, B, H, KVH, D, Lc, N, bs, is_causal, layer, window, dtype="bf16"):
+    rng = wl.rng_for(seed)
+    nq, lk = N * bs, Lc + N * bs
+    q = wl.normal(rng, (B, nq, H, D), dtype)
+    k = wl.normal(rng, (B, lk, KVH, D), dtype)
+    v = wl.normal(rng, (B, lk, KVH, D), dtype)
+    do = wl.normal(rng, (B, nq, H, D), dtype)
+    anchors = torch.from_numpy(np.sort(rng.integers(0, Lc + 1, size=(B, N)), axis=1).astype(np.int32))
+    return q, k, v, do, anchors
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("layer,is_causal,window", [(0, None, 0), (1, None, 40), (0, True, 0)], ids=str)
+def test_dflash_backward(D, layer, is_causal, window):
+    B, H, KVH, Lc, N, bs = 2, 4, 2, 300, 20, 16   # Nq 320, Lk 620: ragged query and key tiles
+    q, k, v, do, anchors = _dflash_case(31, B, H, KVH, D, Lc, N, bs, is_causal, layer, window)
+    qc, kc, vc, dc, ac = (t.cuda() for t in (q, k, v, do, anchors))
+    out, lse = sma.dfa_attn_fwd(qc, kc, vc, ac, Lc, bs, is_causal, layer, window)
+    dq, dk, dv = sma.dfa_attn_bwd(qc, kc, vc, out, lse, dc, ac, Lc, bs, is_causal, layer, window)
+    torch.cuda.synchronize()
+    assert sma.device_status() == 0
+    causal = dm.resolve_in_block_causal(is_causal, layer)
+    w = dm.resolve_window(layer, window) if layer == dm.LAYER_SLIDING else None
+    keep = dm.dflash_keep_mask(anchors.numpy(), Lc, bs, causal, w)[:, None]
+    rq, rk, rv, _ = ag.attention_grad(f64(q), f64(k), f64(v), f64(do), keep=keep, workers=8)
+    _close("dq", dq, rq)
+    _close("dk", dk, rk)
+    _close("dv", dv, rv)
+
+
+B, LQ, LK, H, KVH = 2, 300, 450, 8, 2
+KP = sma.round_up_k(LK)
+
+
+@pytest.mark.parametrize("mshape", [None, (1, 1, LQ, KP), (B, KVH, 1, KP), (B, H, LQ, KP)], ids=str)
+@pytest.mark.parametrize("bshape", [None, (B, KVH, 1, KP)], ids=str)
+@pytest.mark.parametrize("causal", [False, True])
+def test_masked_backward(mshape, bshape, causal):
+    rng = wl.rng_for(32)
+    q = wl.normal(rng, (B, LQ, H, 128), "bf16")
+    k = wl.normal(rng, (B, LK, KVH, 128), "bf16")
+    v = wl.normal(rng, (B, LK, KVH, 128), "bf16")
+    do = wl.normal(rng, (B, LQ, H, 128), "bf16")
+    mask = torch.from_numpy(rng.random(mshape) < 0.7) if mshape else None
+    bias = wl.normal(rng, bshape, "bf16") if bshape else None
+    qc, kc, vc, dc = (t.cuda() for t in (q, k, v, do))
+    mc = None if mask is None else mask.cuda()
+    bc = None if bias is None else bias.cuda()
+    out, lse = sma.masked_attn_fwd(qc, kc, vc, mc, bc, causal)
+    dq, dk, dv = sma.masked_attn_bwd(qc, kc, vc, out, lse, dc, mc, bc, causal)
+    torch.cuda.synchronize()
+    assert sma.device_status() == 0
+    keep = at.aux_view(mask.numpy(), H, KVH, LK) if mask is not None else None
+    if causal:
+        ck = at.causal_keep(LQ, LK)[None, None]
+        keep = ck if keep is None else (keep & ck)
+    bb = at.aux_view(f64(bias), H, KVH, LK) if bias is not None else None
+    rq, rk, rv, _ = ag.attention_grad(f64(q), f64(k), f64(v), f64(do), keep=keep, bias=bb, workers=8)
+    _close("dq", dq, rq)
+    _close("dk", dk, rk)
+    _close("dv", dv, rv)
+
+
+def test_unattended_keys_and_dead_rows():
+    """Keys no query keeps get zero dK / dV; rows with no kept key give zero dQ."""
+    rng = wl.rng_for(33)
+    q = wl.normal(rng, (1, 200, 4, 128), "bf16")
+    k = wl.normal(rng, (1, 500, 2, 128), "bf16")
+    v = wl.normal(rng, (1, 500, 2, 128), "bf16")
+    do = wl.normal(rng, (1, 200, 4, 128), "bf16")
+    kp = sma.round_up_k(500)
+    mask = torch.from_numpy(rng.random((1, 1, 200, kp)) < 0.5)
+    mask[..., 128:300] = False           # a whole key tile and more unattended
+    mask[0, 0, 7] = False                # a dead row
+    qc, kc, vc, dc, mc = (t.cuda() for t in (q, k, v, do, mask))
+    out, lse = sma.masked_attn_fwd(qc, kc, vc, mc, None, False)
+    dq, dk, dv = sma.masked_attn_bwd(qc, kc, vc, out, lse, dc, mc, None, False)
+    torch.cuda.synchronize()
+    assert sma.device_status() == 0
+    assert (dk[:, 128:300] == 0).all() and (dv[:, 128:300] == 0).all()
+    assert (dq[0, 7] == 0).all()
+    rq, rk, rv, _ = ag.attention_grad(f64(q), f64(k), f64(v), f64(do), keep=mask.numpy()[..., :500], workers=8)
+    _close("dq", dq, rq)
+    _close("dk", dk, rk)
+    _close("dv", dv, rv)
+
+
+def test_fp16_and_rejections():
+    rng = wl.rng_for(34)
+    q = wl.normal(rng, (1, 130, 2, 64), "fp16")
+    k = wl.normal(rng, (1, 260, 1, 64), "fp16")
+    v = wl.normal(rng, (1, 260, 1, 64), "fp16")
+    do = wl.normal(rng, (1, 130, 2, 64), "fp16")
+    qc, kc, vc, dc = (t.cuda() for t in (q, k, v, do))
+    out, lse = sma.masked_attn_fwd(qc, kc, vc, None, None, True)
+    dq, dk, dv = sma.masked_attn_bwd(qc, kc, vc, out, lse, dc, None, None, True)
+    torch.cuda.synchronize()
+    rq, rk, rv, _ = ag.attention_grad(f64(q), f64(k), f64(v), f64(do), keep=at.causal_keep(130, 260)[None, None])
+    _close("dq", dq, rq)
+    _close("dk", dk, rk)
+    _close("dv", dv, rv)
+    with pytest.raises(sma.SmaError, match="bf16 or fp16"):
+        sma.masked_attn_bwd(qc.float(), kc.float(), vc.float(), out.float(), lse, dc.float())
