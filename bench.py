@@ -281,7 +281,7 @@ def run_ours(args, rank, world, dev):
     return res
 
 
-DETAILS = ("dflash", "broadcast_prefill", "broadcast_decode", "topk", "topk_wide")
+DETAILS = ("dflash", "dflash_bwd", "broadcast_prefill", "broadcast_decode", "topk", "topk_wide")
 
 
 def run_details(sma, dev, stream, peaks, only=None):
@@ -304,6 +304,26 @@ def run_details(sma, dev, stream, peaks, only=None):
         tf = tile_flops(w.head_dim, w.heads, kept) / (ms * 1e-3) / 1e12
         out[w.name] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / pk_t, "kept_tiles": kept}
         del q, k, v, o
+
+    # backward of the DFlash layers: 5 products per kept tile (2.5x the forward's work)
+    for w in ((wl.DFLASH_TRAIN_FULL, wl.DFLASH_TRAIN_SLIDING, wl.DFLASH_LONG_FULL) if want("dflash_bwd") else ()):
+        q, k, v, anchors = dflash_case(w, dev)
+        args = (anchors, w.ctx_len, w.block_size, w.is_causal, w.layer_type, w.sliding_window)
+        bmap = sma.dfa_block_map(*args)
+        kept = int((bmap[0] + bmap[2]).sum().item())
+        o, lse = sma.dfa_attn_fwd(q, k, v, *args)
+        do = torch.randn_like(q)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(sma.dfa_attn_bwd_workspace_size(q.shape[0], anchors.shape[1], w.block_size, w.ctx_len,
+                                                         w.heads, w.kv_heads, w.head_dim, w.is_causal, w.layer_type,
+                                                         w.sliding_window), dtype=torch.uint8, device=dev)
+        ms = timed(lambda: sma.dfa_attn_bwd(q, k, v, o, lse, do, *args, dq=dq, dk=dk, dv=dv, workspace=ws),
+                   stream, 5, 2)
+        tf = 2.5 * tile_flops(w.head_dim, w.heads, kept) / (ms * 1e-3) / 1e12
+        out[w.name + "_bwd"] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / pk_t, "kept_tiles": kept,
+                                "status": sma.device_status()}
+        del q, k, v, o, lse, do, dq, dk, dv, ws
+        torch.cuda.empty_cache()
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     if want("broadcast_prefill"):

@@ -35,7 +35,8 @@
 //              accumulator) and the unit's dK / dV epilogue.
 //   warp  8    TMA producer: K, V once per unit; Q (2 stages), dO (1 stage)
 //   warp  9    MMA issuer (one elected lane), in the order
-//              S(0) dP(0) | dV(p) S(p+1) | dK(p) dQ(p) | dP(p+1) ...
+//              S(0) dP(0) | dV(p) S(p+1) | dK(p) dQ(p) | dP(p+1) ..., the two
+//              products of each group issued with their k-steps interleaved.
 // Every mbarrier wait is bounded; on expiry the CTA raises its abort flag,
 // drains its own copies and products, frees TMEM and returns.
 #include <cstdio>
@@ -316,37 +317,49 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     auto with_lo = [](uint64_t d, uint32_t add) -> uint64_t {
       return (d & 0xffffffff00000000ull) | static_cast<uint32_t>(static_cast<uint32_t>(d) + add);
     };
-    // C[128][128] = A[128][D] B[128][D]^T, both K-major (K = head dim)
-    auto issue_kmajor = [&](uint32_t dcol, uint32_t a_addr, uint32_t b_addr) {
-      const uint64_t ad = smem_desc_sw128(a_addr, 16, 1024);
-      const uint64_t bd = smem_desc_sw128(b_addr, 16, 1024);
+    // Two independent products issued with their k-steps interleaved: each
+    // k-step of a chain depends on the previous one through its accumulator,
+    // so alternating two chains keeps the tensor pipe busy.
+    auto issue_s_dp = [&](uint32_t q_addr, bool with_s, bool with_dp) {
+      const uint64_t qd = smem_desc_sw128(q_addr, 16, 1024);
+      const uint64_t kd = smem_desc_sw128(sbase + L::kK, 16, 1024);
+      const uint64_t od = smem_desc_sw128(sbase + L::kDO, 16, 1024);
+      const uint64_t vd = smem_desc_sw128(sbase + L::kV, 16, 1024);
 #pragma unroll
       for (int s = 0; s < D / 16; ++s) {
         const uint32_t off = ((s >> 2) * L::kChunk + (s & 3) * 32) >> 4;
-        tc_mma_ss(tmem + dcol, with_lo(ad, off), with_lo(bd, off), idesc_s, s > 0 ? 1u : 0u);
+        if (with_s) tc_mma_ss(tmem + L::kColS, with_lo(qd, off), with_lo(kd, off), idesc_s, s > 0 ? 1u : 0u);
+        if (with_dp) tc_mma_ss(tmem + L::kColDP, with_lo(od, off), with_lo(vd, off), idesc_s, s > 0 ? 1u : 0u);
       }
     };
-    // C[128][D] (+)= A^T B over the 128 query rows: A = P or dS [q][k], B = dO or Q [q][d]
-    auto issue_trans = [&](uint32_t dcol, uint32_t a_addr, uint32_t b_addr, bool acc) {
-      const uint64_t ad = smem_desc_sw128(a_addr, L::kChunk, 1024);
-      const uint64_t bd = smem_desc_sw128(b_addr, L::kChunk, 1024);
+    // dV += P^T dO interleaved with S(next) = Q(next) K^T (when there is one)
+    auto issue_dv_s = [&](bool acc, bool with_s, uint32_t q_addr) {
+      const uint64_t ad = smem_desc_sw128(sbase + L::kP, L::kChunk, 1024);
+      const uint64_t bd = smem_desc_sw128(sbase + L::kDO, L::kChunk, 1024);
+      const uint64_t qd = smem_desc_sw128(q_addr, 16, 1024);
+      const uint64_t kd = smem_desc_sw128(sbase + L::kK, 16, 1024);
 #pragma unroll
       for (int s = 0; s < kTile / 16; ++s) {
         const uint32_t off = (s * 2048) >> 4;
-        tc_mma_ss(tmem + dcol, with_lo(ad, off), with_lo(bd, off), idesc_t,
-                  (acc || s > 0) ? 1u : 0u);
+        tc_mma_ss(tmem + L::kColDV, with_lo(ad, off), with_lo(bd, off), idesc_t, (acc || s > 0) ? 1u : 0u);
+        if (with_s && s < D / 16) {
+          const uint32_t so = ((s >> 2) * L::kChunk + (s & 3) * 32) >> 4;
+          tc_mma_ss(tmem + L::kColS, with_lo(qd, so), with_lo(kd, so), idesc_s, s > 0 ? 1u : 0u);
+        }
       }
     };
-    // dQ[128][D] = dS[q][k] K[k][d]
-    auto issue_dq = [&]() {
-      const uint64_t ad = smem_desc_sw128(sbase + L::kDS, 16, 1024);
-      const uint64_t bd = smem_desc_sw128(sbase + L::kK, L::kChunk, 1024);
+    // dK += dS^T Q interleaved with dQ = dS K
+    auto issue_dk_dq = [&](bool acc, uint32_t q_addr) {
+      const uint64_t ad = smem_desc_sw128(sbase + L::kDS, L::kChunk, 1024);
+      const uint64_t bd = smem_desc_sw128(q_addr, L::kChunk, 1024);
+      const uint64_t sd = smem_desc_sw128(sbase + L::kDS, 16, 1024);
+      const uint64_t kd = smem_desc_sw128(sbase + L::kK, L::kChunk, 1024);
 #pragma unroll
       for (int s = 0; s < kTile / 16; ++s) {
+        const uint32_t off = (s * 2048) >> 4;
         const uint32_t aoff = ((s >> 2) * L::kChunk + (s & 3) * 32) >> 4;
-        const uint32_t boff = (s * 2048) >> 4;
-        tc_mma_ss(tmem + L::kColDP, with_lo(ad, aoff), with_lo(bd, boff), idesc_q,
-                  s > 0 ? 1u : 0u);
+        tc_mma_ss(tmem + L::kColDK, with_lo(ad, off), with_lo(bd, off), idesc_t, (acc || s > 0) ? 1u : 0u);
+        tc_mma_ss(tmem + L::kColDP, with_lo(sd, aoff), with_lo(kd, off), idesc_q, s > 0 ? 1u : 0u);
       }
     };
     uint32_t kv_it = 0, q_it = 0, o_it = 0, pit = 0, uit = 0;
@@ -361,52 +374,39 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
       if (n == 0) continue;
       if (!wait(L::kKVFull, kv_it & 1)) break;
       ++kv_it;
-      // S(0), dP(0)
+      // S(0) and dP(0)
       if (!wait(L::kQFull + (q_it & 1), (q_it >> 1) & 1)) break;
-      tc_fence_after();
-      if (elect_one()) {
-        issue_kmajor(L::kColS, sbase + L::kQ + (q_it & 1) * L::kTileD, sbase + L::kK);
-        tc_commit(bar(L::kSFull));
-      }
-      __syncwarp();
       if (!wait(L::kOFull, o_it & 1)) break;
       if (pit > 0 && !wait(L::kDQFree, (pit - 1) & 1)) break;
       tc_fence_after();
       if (elect_one()) {
-        issue_kmajor(L::kColDP, sbase + L::kDO, sbase + L::kV);
+        issue_s_dp(sbase + L::kQ + (q_it & 1) * L::kTileD, true, true);
+        tc_commit(bar(L::kSFull));
         tc_commit(bar(L::kDPFull));
       }
       __syncwarp();
       for (int i = 0; i < n && ok; ++i) {
         const int qs = q_it & 1;  // Q stage of pair i
-        // dV += P^T dO
+        const bool more = i + 1 < n;
+        const uint32_t nq = q_it + 1;
+        // dV += P^T dO, with S(i+1) alongside (S's columns are free once P(i) is formed)
         if (!wait(L::kPDone, pit & 1)) break;
         if (i == 0 && uit > 0 && !wait(L::kAccFree, (uit - 1) & 1)) break;
+        if (more && !wait(L::kQFull + (nq & 1), (nq >> 1) & 1)) break;
         tc_fence_after();
         if (elect_one()) {
-          issue_trans(L::kColDV, sbase + L::kP, sbase + L::kDO, i > 0);
+          issue_dv_s(i > 0, more, sbase + L::kQ + (nq & 1) * L::kTileD);
           tc_commit(bar(L::kPFree));
           tc_commit(bar(L::kOEmpty));
+          if (more) tc_commit(bar(L::kSFull));
         }
         __syncwarp();
         ++o_it;
-        // S(i+1): S's columns are free once P(i) is formed
-        if (i + 1 < n) {
-          const uint32_t nq = q_it + 1;
-          if (!wait(L::kQFull + (nq & 1), (nq >> 1) & 1)) break;
-          tc_fence_after();
-          if (elect_one()) {
-            issue_kmajor(L::kColS, sbase + L::kQ + (nq & 1) * L::kTileD, sbase + L::kK);
-            tc_commit(bar(L::kSFull));
-          }
-          __syncwarp();
-        }
-        // dK += dS^T Q; dQ = dS K into dP's columns
+        // dK += dS^T Q and dQ = dS K (into dP's columns)
         if (!wait(L::kDSDone, pit & 1)) break;
         tc_fence_after();
         if (elect_one()) {
-          issue_trans(L::kColDK, sbase + L::kDS, sbase + L::kQ + qs * L::kTileD, i > 0);
-          issue_dq();
+          issue_dk_dq(i > 0, sbase + L::kQ + qs * L::kTileD);
           tc_commit(bar(L::kDQFull));
           tc_commit(bar(L::kDSFree));
           tc_commit(bar(L::kQEmpty + qs));
@@ -415,12 +415,12 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         ++q_it;
         ++pit;
         // dP(i+1) once dO(i+1) is in and dQ(i) has left TMEM
-        if (i + 1 < n) {
+        if (more) {
           if (!wait(L::kOFull, o_it & 1)) break;
           if (!wait(L::kDQFree, (pit - 1) & 1)) break;
           tc_fence_after();
           if (elect_one()) {
-            issue_kmajor(L::kColDP, sbase + L::kDO, sbase + L::kV);
+            issue_s_dp(0, false, true);
             tc_commit(bar(L::kDPFull));
           }
           __syncwarp();
