@@ -683,6 +683,688 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
   if (warp == kBMmaWarp) tmem_dealloc(tmem, kBTmemCols);
 }
 
+
+// ---------------------------------------------------------------------------
+// Head dim 128: the transposed form.  The compute threads own key rows:
+//   S^T  = K Q^T        A = K (K-major)        B = Q (K-major)        SS
+//   dP^T = V dO^T       A = V (K-major)        B = dO (K-major)       SS
+//   dV  += P^T dO       A = P^T from TMEM      B = dO (MN-major)      TS
+//   dK  += dS^T Q       A = dS^T from TMEM     B = Q (MN-major)       TS
+//   dQ   = dS K         A = dS (MN-major)      B = K (MN-major)       SS
+// P^T and dS^T go to TMEM as packed 16-bit pairs over the first half of the
+// S^T / dP^T columns (as the forward's P does), so dV and dK read their A
+// operand from TMEM; only dS^T is also written to shared memory, where the
+// [key][query] tile read as an MN-major operand is dS itself (queries
+// contiguous), so dQ comes out with query rows in TMEM.
+// That halves the operand traffic the products and the compute threads put
+// on shared memory.  Two 128-column TMEM regions alternate between pairs:
+// pair i puts S^T / P^T and later dQ in region X_i, dP^T / dS^T in Y_i;
+// pair i+1 swaps them, so S^T(i+1) can be issued as soon as dK(i) has read
+// dS^T(i), and dP^T(i+1) once dQ(i) has been drained.
+// The producer stages, per pair, -lse * log2(e) and rowsum(dO * O) of the
+// 128 queries (and, for DFlash, each query's kept key intervals) in shared
+// memory next to the Q stage.
+// Bulk tensor reduction (add) of a swizzled shared-memory box into global
+// memory, tracked by the issuing thread's bulk group.
+__device__ __forceinline__ void bulk_reduce_add_4d(const CUtensorMap* map, uint32_t src, int c0,
+                                                   int c1, int c2, int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+      ::"l"(map), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+constexpr int kBwdTThreads = 352;  // + warp 10: per-query data of each pair
+constexpr int kBAuxWarp = 10;
+
+struct TLayout {
+  static constexpr int D = 128;
+  static constexpr uint32_t kChunk = kTile * 128;
+  static constexpr uint32_t kTileD = kTile * D * 2;
+  static constexpr uint32_t kK = 0;
+  static constexpr uint32_t kV = kK + kTileD;
+  static constexpr uint32_t kQ = kV + kTileD;        // 2 stages
+  static constexpr uint32_t kDO = kQ + 2 * kTileD;   // 1 stage
+  static constexpr uint32_t kDS = kDO + kTileD;      // dS^T [key][query]
+  static constexpr uint32_t kAux = kDS + kTileD;     // 2 stages of kAuxBytes
+  static constexpr uint32_t kAuxBytes = 6 * kTile * 4;  // nl, dd, clo, chi, dlo, dhi
+  // dQ staging for the bulk reductions: per drain warp 32 rows x 32 floats
+  static constexpr uint32_t kStage = (kAux + 2 * kAuxBytes + 1023) / 1024 * 1024;
+  static constexpr uint32_t kStageWarp = 32 * 32 * 4;
+  static constexpr uint32_t kBars = kStage + 4 * kStageWarp;
+  enum : int {
+    kKVFull = 0, kKVEmpty, kQFull, kQEmpty = kQFull + 2, kAuxFull = kQEmpty + 2,
+    kOFull = kAuxFull + 2, kOEmpty, kSFull, kPDone, kDPFull, kDSDone, kDQFull, kDQFree, kDSFree,
+    kAccDone, kAccFree, kDrain, kNumBars
+  };
+  static constexpr uint32_t kTmemSlot = kBars + 8 * kNumBars;
+  static constexpr uint32_t kAbort = kTmemSlot + 4;
+  static constexpr uint32_t kBytes = kAbort + 4;
+  static constexpr uint32_t kAlloc = kBytes + 1024;
+  static constexpr uint32_t kColDV = 256, kColDK = 384;
+  static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+template <int POLICY, int DT>
+__global__ void __launch_bounds__(kBwdTThreads, 1)
+attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
+                  const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                  const __grid_constant__ CUtensorMap map_do, const __grid_constant__ CUtensorMap map_dq,
+                  int n_units) {
+  using L = TLayout;
+  constexpr int D = L::D;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * static_cast<uint32_t>(i); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+  auto aux_f = [&](int stage, int which) -> float* {
+    return reinterpret_cast<float*>(smem + L::kAux + stage * L::kAuxBytes + which * kTile * 4);
+  };
+  auto aux_i = [&](int stage, int which) -> int* {
+    return reinterpret_cast<int*>(smem + L::kAux + stage * L::kAuxBytes + which * kTile * 4);
+  };
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::kKVFull), 1);
+    mbar_init(bar(L::kKVEmpty), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(L::kQFull + s), 1);
+      mbar_init(bar(L::kQEmpty + s), 1);
+      mbar_init(bar(L::kAuxFull + s), 32);
+    }
+    mbar_init(bar(L::kOFull), 1);
+    mbar_init(bar(L::kOEmpty), 1);
+    mbar_init(bar(L::kSFull), 1);
+    mbar_init(bar(L::kPDone), 128);
+    mbar_init(bar(L::kDPFull), 1);
+    mbar_init(bar(L::kDSDone), 128);
+    mbar_init(bar(L::kDQFull), 1);
+    mbar_init(bar(L::kDQFree), 128);
+    mbar_init(bar(L::kDSFree), 1);
+    mbar_init(bar(L::kAccDone), 1);
+    mbar_init(bar(L::kAccFree), 128);
+    mbar_init(bar(L::kDrain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kBMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kBTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kBLoadWarp) {
+    // ------------------------------------------------------------ producer
+    if (elect_one()) {
+      tma_prefetch_map(&map_q);
+      tma_prefetch_map(&map_k);
+      tma_prefetch_map(&map_v);
+      tma_prefetch_map(&map_do);
+    }
+    __syncwarp();
+    uint32_t kv_it = 0, q_it = 0, o_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const BUnit w = bwd_unit(p, u);
+      if (w.n_pairs == 0) continue;
+      if (kv_it > 0 && !mbar_wait_warp(bar(L::kKVEmpty), (kv_it - 1) & 1, abort_flag, p.f.err)) {
+        ok = false;
+        break;
+      }
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar(L::kKVFull), 2 * L::kTileD);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_4d(sbase + L::kK + c * L::kChunk, &map_k, bar(L::kKVFull), c * 64, w.hk,
+                      w.kt * kTile, w.b);
+          tma_load_4d(sbase + L::kV + c * L::kChunk, &map_v, bar(L::kKVFull), c * 64, w.hk,
+                      w.kt * kTile, w.b);
+        }
+      }
+      __syncwarp();
+      ++kv_it;
+      PairWalk pw;
+      pw.begin(p, w);
+      for (int i = 0; i < w.n_pairs && ok; ++i, pw.next(p, w)) {
+        bool partial;
+        const int qt = pw.qtile(p, w, &partial);
+        const int h = pw.head(w);
+        const int s = q_it & 1;
+        const uint32_t use = q_it >> 1;
+        if (use > 0 && !mbar_wait_warp(bar(L::kQEmpty + s), (use - 1) & 1, abort_flag, p.f.err)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(L::kQFull + s), L::kTileD);
+          for (int c = 0; c < 2; ++c)
+            tma_load_4d(sbase + L::kQ + s * L::kTileD + c * L::kChunk, &map_q, bar(L::kQFull + s),
+                        c * 64, h, qt * kTile, w.b);
+        }
+        __syncwarp();
+        ++q_it;
+        if (o_it > 0 && !mbar_wait_warp(bar(L::kOEmpty), (o_it - 1) & 1, abort_flag, p.f.err)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(L::kOFull), L::kTileD);
+          for (int c = 0; c < 2; ++c)
+            tma_load_4d(sbase + L::kDO + c * L::kChunk, &map_do, bar(L::kOFull), c * 64, h,
+                        qt * kTile, w.b);
+        }
+        __syncwarp();
+        ++o_it;
+      }
+    }
+    if (!ok) {
+      if (kv_it > 0) bdrain_wait(bar(L::kKVFull), (kv_it - 1) & 1, p.f.err);
+      for (uint32_t t = 0; t < 2; ++t) {
+        if (q_it > t) {
+          const uint32_t nn = q_it - 1 - t;
+          bdrain_wait(bar(L::kQFull + (nn & 1)), (nn >> 1) & 1, p.f.err);
+        }
+      }
+      if (o_it > 0) bdrain_wait(bar(L::kOFull), (o_it - 1) & 1, p.f.err);
+    }
+  } else if (warp == kBAuxWarp) {
+    // ------------------------------------------------------------ per-query data
+    // -lse * log2(e), rowsum(dO * O) and (DFlash) the kept key intervals of the
+    // pair's 128 queries, 4 per lane; the global reads of the next pair are in
+    // flight while the stage is still in use.
+    uint32_t q_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const BUnit w = bwd_unit(p, u);
+      if (w.n_pairs == 0) continue;
+      PairWalk pw;
+      pw.begin(p, w);
+      for (int i = 0; i < w.n_pairs && ok; ++i, pw.next(p, w)) {
+        bool partial;
+        const int qt = pw.qtile(p, w, &partial);
+        const int h = pw.head(w);
+        float n_l[4], d_v[4];
+        int clo[4], chi[4], dlo[4], dhi[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int q = qt * kTile + lane * 4 + j;
+          n_l[j] = -INFINITY;
+          d_v[j] = 0.f;
+          clo[j] = chi[j] = dlo[j] = dhi[j] = 0;
+          if (q < p.f.Lq) {
+            const int64_t row = (static_cast<int64_t>(w.b) * p.f.H + h) * p.f.Lq + q;
+            const float l = p.f.lse[row];
+            n_l[j] = l == -INFINITY ? -INFINITY : -l * kLog2e;
+            d_v[j] = p.dvec[row];
+            if (POLICY == kPolicyDflash) {
+              const int jb = q / p.f.bs, ii = q - jb * p.f.bs;
+              int a = p.f.anchors[static_cast<int64_t>(w.b) * p.f.N + jb];
+              a = a < 0 ? 0 : (a > p.f.Lc ? p.f.Lc : a);
+              chi[j] = a;
+              clo[j] = p.f.window > 0 ? max(0, a + ii - p.f.window + 1) : 0;
+              if (clo[j] > chi[j]) clo[j] = chi[j];
+              const int base = p.f.Lc + jb * p.f.bs;
+              dlo[j] = base + (p.f.window > 0 ? max(0, ii - p.f.window + 1) : 0);
+              dhi[j] = base + (p.f.causal_in_block ? ii + 1 : p.f.bs);
+            }
+          }
+        }
+        const int s = q_it & 1;
+        const uint32_t use = q_it >> 1;
+        if (use > 0 && !mbar_wait_warp(bar(L::kQEmpty + s), (use - 1) & 1, abort_flag, p.f.err)) {
+          ok = false;
+          break;
+        }
+        float4* nl4 = reinterpret_cast<float4*>(aux_f(s, 0)) + lane;
+        float4* dd4 = reinterpret_cast<float4*>(aux_f(s, 1)) + lane;
+        int4* iv4 = reinterpret_cast<int4*>(aux_i(s, 2)) + lane;
+        *nl4 = make_float4(n_l[0], n_l[1], n_l[2], n_l[3]);
+        *dd4 = make_float4(d_v[0], d_v[1], d_v[2], d_v[3]);
+        iv4[0] = make_int4(clo[0], clo[1], clo[2], clo[3]);
+        iv4[kTile / 4] = make_int4(chi[0], chi[1], chi[2], chi[3]);
+        iv4[2 * kTile / 4] = make_int4(dlo[0], dlo[1], dlo[2], dlo[3]);
+        iv4[3 * kTile / 4] = make_int4(dhi[0], dhi[1], dhi[2], dhi[3]);
+        mbar_arrive(bar(L::kAuxFull + s));
+        ++q_it;
+      }
+    }
+  } else if (warp == kBMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t fmt = DT == SMA_BF16 ? 1u : 0u;
+    constexpr uint32_t idesc_ss = mma_idesc_f16(fmt, 128, 128, 0, 0);  // S^T, dP^T
+    constexpr uint32_t idesc_ts = mma_idesc_f16(fmt, 128, D, 0, 1);    // dV, dK (A in TMEM)
+    constexpr uint32_t idesc_dq = mma_idesc_f16(fmt, 128, D, 1, 1);    // dQ (A = dS from dS^T, MN-major)
+    auto with_lo = [](uint64_t d, uint32_t add) -> uint64_t {
+      return (d & 0xffffffff00000000ull) | static_cast<uint32_t>(static_cast<uint32_t>(d) + add);
+    };
+    // C[128 keys][128 queries] = A[keys][d] B[queries][d]^T, both K-major
+    auto issue_t = [&](uint32_t col, uint32_t a_addr, uint32_t b_addr) {
+      const uint64_t ad = smem_desc_sw128(a_addr, 16, 1024);
+      const uint64_t bd = smem_desc_sw128(b_addr, 16, 1024);
+#pragma unroll
+      for (int s = 0; s < D / 16; ++s) {
+        const uint32_t off = ((s >> 2) * L::kChunk + (s & 3) * 32) >> 4;
+        tc_mma_ss(tmem + col, with_lo(ad, off), with_lo(bd, off), idesc_ss, s > 0 ? 1u : 0u);
+      }
+    };
+    // S^T and dP^T with k-steps interleaved
+    auto issue_st_dpt = [&](uint32_t xcol, uint32_t ycol, uint32_t q_addr) {
+      const uint64_t kd = smem_desc_sw128(sbase + L::kK, 16, 1024);
+      const uint64_t qd = smem_desc_sw128(q_addr, 16, 1024);
+      const uint64_t vd = smem_desc_sw128(sbase + L::kV, 16, 1024);
+      const uint64_t od = smem_desc_sw128(sbase + L::kDO, 16, 1024);
+#pragma unroll
+      for (int s = 0; s < D / 16; ++s) {
+        const uint32_t off = ((s >> 2) * L::kChunk + (s & 3) * 32) >> 4;
+        tc_mma_ss(tmem + xcol, with_lo(kd, off), with_lo(qd, off), idesc_ss, s > 0 ? 1u : 0u);
+        tc_mma_ss(tmem + ycol, with_lo(vd, off), with_lo(od, off), idesc_ss, s > 0 ? 1u : 0u);
+      }
+    };
+    // acc[keys][d] (+)= A^T[keys][queries] B[queries][d], A packed in TMEM
+    auto issue_ts = [&](uint32_t dcol, uint32_t acol, uint32_t b_addr, bool acc) {
+      const uint64_t bd = smem_desc_sw128(b_addr, L::kChunk, 1024);
+#pragma unroll
+      for (int s = 0; s < kTile / 16; ++s)
+        tc_mma_ts(tmem + dcol, tmem + acol + 8 * s, with_lo(bd, (s * 2048) >> 4), idesc_ts,
+                  (acc || s > 0) ? 1u : 0u);
+    };
+    // dK += dS^T Q (TS) interleaved with dQ = dS K (SS; the dS^T tile read as an
+    // MN-major A operand is dS with queries contiguous)
+    auto issue_dk_dq = [&](uint32_t ycol, uint32_t xcol, uint32_t q_addr, bool acc) {
+      const uint64_t qd = smem_desc_sw128(q_addr, L::kChunk, 1024);
+      const uint64_t kd = smem_desc_sw128(sbase + L::kK, L::kChunk, 1024);
+      const uint64_t sd = smem_desc_sw128(sbase + L::kDS, L::kChunk, 1024);
+#pragma unroll
+      for (int s = 0; s < kTile / 16; ++s) {
+        const uint32_t off = (s * 2048) >> 4;
+        tc_mma_ts(tmem + L::kColDK, tmem + ycol + 8 * s, with_lo(qd, off), idesc_ts,
+                  (acc || s > 0) ? 1u : 0u);
+        tc_mma_ss(tmem + xcol, with_lo(sd, off), with_lo(kd, off), idesc_dq, s > 0 ? 1u : 0u);
+      }
+    };
+    uint32_t kv_it = 0, q_it = 0, o_it = 0, pit = 0, uit = 0;
+    bool ok = true;
+    auto wait = [&](int b_, uint32_t parity) -> bool {
+      if (!mbar_wait_warp(bar(b_), parity, abort_flag, p.f.err)) ok = false;
+      return ok;
+    };
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const BUnit w = bwd_unit(p, u);
+      const int n = w.n_pairs;
+      if (n == 0) continue;
+      if (!wait(L::kKVFull, kv_it & 1)) break;
+      ++kv_it;
+      {  // S^T(0), dP^T(0)
+        const uint32_t X = (pit & 1) ? 128u : 0u, Y = 128u - X;
+        if (!wait(L::kQFull + (q_it & 1), (q_it >> 1) & 1)) break;
+        if (!wait(L::kOFull, o_it & 1)) break;
+        if (pit > 0 && !wait(L::kDQFree, (pit - 1) & 1)) break;  // Y held dQ of the last pair
+        tc_fence_after();
+        if (elect_one()) {
+          issue_st_dpt(X, Y, sbase + L::kQ + (q_it & 1) * L::kTileD);
+          tc_commit(bar(L::kSFull));
+          tc_commit(bar(L::kDPFull));
+        }
+        __syncwarp();
+      }
+      for (int i = 0; i < n && ok; ++i) {
+        const uint32_t X = (pit & 1) ? 128u : 0u, Y = 128u - X;
+        const int qs = q_it & 1;
+        // dV += P^T dO
+        if (!wait(L::kPDone, pit & 1)) break;
+        if (i == 0 && uit > 0 && !wait(L::kAccFree, (uit - 1) & 1)) break;
+        tc_fence_after();
+        if (elect_one()) {
+          issue_ts(L::kColDV, X, sbase + L::kDO, i > 0);
+          tc_commit(bar(L::kOEmpty));
+        }
+        __syncwarp();
+        ++o_it;
+        // dK += dS^T Q and dQ = dS K (into X, after dV has read P^T there)
+        if (!wait(L::kDSDone, pit & 1)) break;
+        tc_fence_after();
+        if (elect_one()) {
+          issue_dk_dq(Y, X, sbase + L::kQ + qs * L::kTileD, i > 0);
+          tc_commit(bar(L::kDQFull));
+          tc_commit(bar(L::kDSFree));
+          tc_commit(bar(L::kQEmpty + qs));
+        }
+        __syncwarp();
+        ++q_it;
+        ++pit;
+        if (i + 1 < n) {
+          // S^T(i+1) into Y (dK has read dS^T there); dP^T(i+1) into X once dQ is drained
+          if (!wait(L::kQFull + (q_it & 1), (q_it >> 1) & 1)) break;
+          tc_fence_after();
+          if (elect_one()) {
+            issue_t(Y, sbase + L::kK, sbase + L::kQ + (q_it & 1) * L::kTileD);
+            tc_commit(bar(L::kSFull));
+          }
+          __syncwarp();
+          if (!wait(L::kOFull, o_it & 1)) break;
+          if (!wait(L::kDQFree, (pit - 1) & 1)) break;
+          tc_fence_after();
+          if (elect_one()) {
+            issue_t(X, sbase + L::kV, sbase + L::kDO);
+            tc_commit(bar(L::kDPFull));
+          }
+          __syncwarp();
+        }
+      }
+      if (!ok) break;
+      if (elect_one()) {
+        tc_commit(bar(L::kAccDone));
+        tc_commit(bar(L::kKVEmpty));
+      }
+      __syncwarp();
+      ++uit;
+    }
+    if (!ok) {
+      if (elect_one()) tc_commit(bar(L::kDrain));
+      __syncwarp();
+      bdrain_wait(bar(L::kDrain), 0, p.f.err);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ compute (P^T, dS^T), key rows
+    const int r = warp * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float scale_log2 = p.f.scale_log2;
+    const float bias_mul = kLog2e / p.f.scale_log2;
+    uint32_t pit = 0, q_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const BUnit w = bwd_unit(p, u);
+      if (w.n_pairs == 0) continue;
+      const int key = w.kt * kTile + r;
+      PairWalk pw;
+      pw.begin(p, w);
+      for (int i = 0; i < w.n_pairs && ok; ++i, pw.next(p, w)) {
+        bool partial;
+        const int qt = pw.qtile(p, w, &partial);
+        const int h = pw.head(w);
+        const int q0 = qt * kTile;
+        const uint32_t X = (pit & 1) ? 128u : 0u, Y = 128u - X;
+        const uint32_t xcol = tmem + lane_off + X, ycol = tmem + lane_off + Y;
+        const int s = q_it & 1;
+        const float* nl = aux_f(s, 0);
+        const float* dd = aux_f(s, 1);
+        const int* iv = aux_i(s, 2);
+        const uint8_t* mcol = nullptr;  // mask[b, h?, q, key] at q = 0
+        const uint8_t* bcol = nullptr;
+        int64_t msq = 0, bsq = 0;
+        int bdt = 0;
+        if (POLICY != kPolicyDflash) {
+          if (p.f.has_mask) {
+            const int hm = p.f.mask.head_per_query ? h : w.hk;
+            mcol = reinterpret_cast<const uint8_t*>(p.f.mask.ptr) + w.b * p.f.mask.sb + hm * p.f.mask.sh + key;
+            msq = p.f.mask.sq;
+          }
+          if (p.f.has_bias) {
+            const int hb = p.f.bias.head_per_query ? h : w.hk;
+            bdt = p.f.bias.dtype;
+            const int esz = bdt == SMA_FP32 ? 4 : 2;
+            bcol = reinterpret_cast<const uint8_t*>(p.f.bias.ptr) +
+                   (w.b * p.f.bias.sb + hb * p.f.bias.sh + key) * esz;
+            bsq = p.f.bias.sq * esz;
+          }
+        }
+        if (!mbar_wait(bar(L::kAuxFull + s), (q_it >> 1) & 1, abort_flag, p.f.err)) { ok = false; break; }
+        if (!mbar_wait(bar(L::kSFull), pit & 1, abort_flag, p.f.err)) { ok = false; break; }
+        tc_fence_after();
+        // ---- phase A: P^T = exp2(S^T * scale * log2 e - lse * log2 e), packed into X
+        // FULL and PARTIAL pairs run separate copies of the loop, so that a
+        // FULL pair carries none of the mask evaluation.
+        auto phase_a = [&](auto masked_tag) {
+          constexpr bool MASKED = decltype(masked_tag)::value;
+  #pragma unroll 1
+          for (int c = 0; c < kTile / 32; ++c) {
+            uint32_t xr[32];
+            tmem_ld32_at(xcol + 32 * c, xr);
+            // keep bits of the chunk's 32 queries (PARTIAL pairs only; the loads
+            // are volatile so that FULL pairs never pay for them)
+            uint32_t kbits = 0xffffffffu;
+            if (MASKED) {
+              kbits = 0u;
+              if (POLICY == kPolicyDflash) {
+                const uint32_t ivs = sbase + L::kAux + s * L::kAuxBytes + 2 * kTile * 4 + 32 * c * 4;
+  #pragma unroll
+                for (int g4 = 0; g4 < 8; ++g4) {
+                  const uint4 lo = ld_shared_v4(ivs + 16 * g4);
+                  const uint4 hi = ld_shared_v4(ivs + kTile * 4 + 16 * g4);
+                  const uint4 dl = ld_shared_v4(ivs + 2 * kTile * 4 + 16 * g4);
+                  const uint4 dh = ld_shared_v4(ivs + 3 * kTile * 4 + 16 * g4);
+                  const int l4[4] = {static_cast<int>(lo.x), static_cast<int>(lo.y), static_cast<int>(lo.z), static_cast<int>(lo.w)};
+                  const int h4[4] = {static_cast<int>(hi.x), static_cast<int>(hi.y), static_cast<int>(hi.z), static_cast<int>(hi.w)};
+                  const int a4[4] = {static_cast<int>(dl.x), static_cast<int>(dl.y), static_cast<int>(dl.z), static_cast<int>(dl.w)};
+                  const int b4[4] = {static_cast<int>(dh.x), static_cast<int>(dh.y), static_cast<int>(dh.z), static_cast<int>(dh.w)};
+  #pragma unroll
+                  for (int z = 0; z < 4; ++z) {
+                    const bool keep = (key >= l4[z] && key < h4[z]) || (key >= a4[z] && key < b4[z]);
+                    kbits |= (keep ? 1u : 0u) << (4 * g4 + z);
+                  }
+                }
+              } else {
+                const volatile uint8_t* mv = mcol;
+  #pragma unroll 4
+                for (int z = 0; z < 32; ++z) {
+                  const int q = q0 + 32 * c + z;
+                  const int qc = q < p.f.Lq ? q : 0;
+                  const bool keep = key < p.f.Lk && (!p.f.causal || key <= q + p.f.Lk - p.f.Lq) &&
+                                    (!p.f.has_mask || mv[qc * msq] != 0);
+                  kbits |= (keep ? 1u : 0u) << z;
+                }
+              }
+            }
+            tc_wait_ld();
+            uint32_t pk[16];
+  #pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 n4 = *reinterpret_cast<const float4*>(nl + 32 * c + e);
+              const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
+              float pv[4];
+  #pragma unroll
+              for (int z = 0; z < 4; ++z) {
+                float x = __uint_as_float(xr[e + z]);
+                if (POLICY != kPolicyDflash && p.f.has_bias) {
+                  const int q = q0 + 32 * c + e + z;
+                  const int qc = q < p.f.Lq ? q : 0;  // rows past Lq read row 0 (their P is 0)
+                  x = fmaf(load_any_as_float(bcol + qc * bsq, bdt, 0), bias_mul, x);
+                }
+                pv[z] = ((kbits >> (e + z)) & 1u) ? fast_exp2(fmaf(x, scale_log2, nn[z])) : 0.f;
+              }
+              pk[e >> 1] = DT == SMA_BF16 ? pack_bf16x2(pv[0], pv[1]) : pack_f16x2(pv[0], pv[1]);
+              pk[(e >> 1) + 1] = DT == SMA_BF16 ? pack_bf16x2(pv[2], pv[3]) : pack_f16x2(pv[2], pv[3]);
+            }
+            tmem_st16_at(xcol + 16 * c, pk);
+          }
+        };
+        if (partial) phase_a(std::true_type{});
+        else phase_a(std::false_type{});
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::kPDone));
+
+        // ---- phase B: dS^T = P^T (dP^T - D), packed into Y and stored to shared memory
+        if (!mbar_wait(bar(L::kDPFull), pit & 1, abort_flag, p.f.err)) { ok = false; break; }
+        if (pit > 0 && !mbar_wait(bar(L::kDSFree), (pit - 1) & 1, abort_flag, p.f.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < kTile / 32; ++c) {
+          uint32_t yr[32], pr[16];
+          tmem_ld32_at(ycol + 32 * c, yr);
+          tmem_ld16_at(xcol + 16 * c, pr);
+          tc_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 d4 = *reinterpret_cast<const float4*>(dd + 32 * c + e);
+            const float2 p01 = unpack2<DT>(pr[e >> 1]);
+            const float2 p23 = unpack2<DT>(pr[(e >> 1) + 1]);
+            const float s0 = p01.x * (__uint_as_float(yr[e]) - d4.x);
+            const float s1 = p01.y * (__uint_as_float(yr[e + 1]) - d4.y);
+            const float s2 = p23.x * (__uint_as_float(yr[e + 2]) - d4.z);
+            const float s3 = p23.y * (__uint_as_float(yr[e + 3]) - d4.w);
+            pk[e >> 1] = DT == SMA_BF16 ? pack_bf16x2(s0, s1) : pack_f16x2(s0, s1);
+            pk[(e >> 1) + 1] = DT == SMA_BF16 ? pack_bf16x2(s2, s3) : pack_f16x2(s2, s3);
+          }
+          tmem_st16_at(ycol + 16 * c, pk);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            st_shared_v4(sw128_unit(sbase + L::kDS, r, 4 * c + v4), pk[4 * v4], pk[4 * v4 + 1],
+                         pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+        fence_async_shared();
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::kDSDone));
+        ++pit;
+        ++q_it;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ drain, dK / dV epilogue
+    const int wq = warp - 4;
+    const int r = wq * 32 + lane;  // dQ: query row; dK / dV: key row
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t dv_col = tmem + lane_off + L::kColDV;
+    const uint32_t dk_col = tmem + lane_off + L::kColDK;
+    typedef typename std::conditional<DT == SMA_BF16, __nv_bfloat16, __half>::type OutT;
+    uint32_t pit = 0, uit = 0;
+    bool ok = true;
+    bool bulk_pending = false;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const BUnit w = bwd_unit(p, u);
+      const int key = w.kt * kTile + r;
+      OutT* dvrow = reinterpret_cast<OutT*>(p.dv) + w.b * p.dv_sb + static_cast<int64_t>(key) * p.dv_sr +
+                    w.hk * p.dv_sh;
+      OutT* dkrow = reinterpret_cast<OutT*>(p.dk) + w.b * p.dk_sb + static_cast<int64_t>(key) * p.dk_sr +
+                    w.hk * p.dk_sh;
+      if (w.n_pairs == 0) {  // keys no query attends: zero gradients
+        if (key < p.f.Lk) {
+          for (int e = 0; e < D / 8; ++e) {
+            reinterpret_cast<uint4*>(dvrow)[e] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4*>(dkrow)[e] = make_uint4(0, 0, 0, 0);
+          }
+        }
+        continue;
+      }
+      PairWalk pw;
+      pw.begin(p, w);
+      for (int i = 0; i < w.n_pairs && ok; ++i, pw.next(p, w)) {
+        bool partial;
+        const int qt = pw.qtile(p, w, &partial);
+        const int h = pw.head(w);
+        const uint32_t X = (pit & 1) ? 128u : 0u;
+        const uint32_t qcol = tmem + lane_off + X;
+        if (!mbar_wait(bar(L::kDQFull), pit & 1, abort_flag, p.f.err)) { ok = false; break; }
+        tc_fence_after();
+        // dQ row q0 + r: all of it to registers, TMEM freed at once; then per
+        // 32-column chunk the warp's 32 rows go through its 4 KB staging box
+        // (128-byte swizzle) into a bulk tensor add on the fp32 accumulator.
+        // Rows past Lq fall outside the map and are not written.
+        uint32_t v[D];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_ld32_at(qcol + 32 * c, v + 32 * c);
+        tc_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(L::kDQFree));
+        const uint32_t stage = sbase + L::kStage + wq * L::kStageWarp;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          if (bulk_pending) {
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            st_shared_v4(stage + lane * 128 + ((u ^ (lane & 7)) << 4), v[32 * c + 4 * u],
+                         v[32 * c + 4 * u + 1], v[32 * c + 4 * u + 2], v[32 * c + 4 * u + 3]);
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            bulk_reduce_add_4d(&map_dq, stage, 32 * c, h, qt * kTile + 32 * wq, w.b);
+            bulk_commit();
+          }
+          bulk_pending = true;
+        }
+        ++pit;
+      }
+      if (!ok) break;
+      if (!mbar_wait(bar(L::kAccDone), uit & 1, abort_flag, p.f.err)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which == 0 ? dv_col : dk_col;
+        const float mul = which == 0 ? 1.f : p.scale;
+        OutT* dst = which == 0 ? dvrow : dkrow;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32_at(col + 32 * c, v);
+          tc_wait_ld();
+          if (key < p.f.Lk) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float a = __uint_as_float(v[2 * e]) * mul;
+              const float bq = __uint_as_float(v[2 * e + 1]) * mul;
+              pk[e] = DT == SMA_BF16 ? pack_bf16x2(a, bq) : pack_f16x2(a, bq);
+            }
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(L::kAccFree));
+      ++uit;
+    }
+    // the staging boxes must stay valid until the reductions are done
+    if (lane == 0) bulk_wait_all0();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kBMmaWarp) tmem_dealloc(tmem, kBTmemCols);
+}
+
+template <int POLICY, int DT>
+cudaError_t launch_bwd_t(const BwdProblem& p, const CUtensorMap& mq, const CUtensorMap& mk,
+                         const CUtensorMap& mv, const CUtensorMap& mdo, const CUtensorMap& mdq,
+                         cudaStream_t stream) {
+  auto kern = attn_bwd_t_kernel<POLICY, DT>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(TLayout::kAlloc));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int n_units = p.f.B * p.f.KVH * p.f.KT;
+  if (n_units == 0) return cudaSuccess;
+  const int grid = n_units < num_sms() ? n_units : num_sms();
+  kern<<<grid, kBwdTThreads, TLayout::kAlloc, stream>>>(p, mq, mk, mv, mdo, mdq, n_units);
+  return cudaGetLastError();
+}
+
 // rowsum(dO * O) per (b, h, q) and the zeroed dQ accumulator; one warp per row.
 template <int DT>
 __global__ void bwd_prep_kernel(const BwdProblem p) {
@@ -860,16 +1542,19 @@ int launch_attn_bwd(const BwdProblem& p, cudaStream_t stream, char* msg, size_t 
       !encode_map(&mv, f.v, f.dtype, f.d, f.KVH, f.Lk, f.B, f.v_sh, f.v_sr, f.v_sb, msg, msg_len) ||
       !encode_map(&mdo, p.dout, f.dtype, f.d, f.H, f.Lq, f.B, p.do_sh, p.do_sr, p.do_sb, msg, msg_len))
     return SMA_ERR_CUDA;
+  CUtensorMap mdq;
+  if (f.d == 128 && !encode_map_f32(&mdq, p.dq_acc, f.d, f.H, f.Lq, f.B, 32, 32, msg, msg_len))
+    return SMA_ERR_CUDA;
   cudaError_t e = cudaErrorInvalidValue;
   const bool bf = f.dtype == SMA_BF16;
   if (f.policy == kPolicyDflash) {
-    if (f.d == 128) e = bf ? launch_bwd_typed<128, kPolicyDflash, SMA_BF16>(p, mq, mk, mv, mdo, stream)
-                           : launch_bwd_typed<128, kPolicyDflash, SMA_FP16>(p, mq, mk, mv, mdo, stream);
+    if (f.d == 128) e = bf ? launch_bwd_t<kPolicyDflash, SMA_BF16>(p, mq, mk, mv, mdo, mdq, stream)
+                           : launch_bwd_t<kPolicyDflash, SMA_FP16>(p, mq, mk, mv, mdo, mdq, stream);
     else e = bf ? launch_bwd_typed<64, kPolicyDflash, SMA_BF16>(p, mq, mk, mv, mdo, stream)
                 : launch_bwd_typed<64, kPolicyDflash, SMA_FP16>(p, mq, mk, mv, mdo, stream);
   } else {
-    if (f.d == 128) e = bf ? launch_bwd_typed<128, kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, mdo, stream)
-                           : launch_bwd_typed<128, kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, mdo, stream);
+    if (f.d == 128) e = bf ? launch_bwd_t<kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, mdo, mdq, stream)
+                           : launch_bwd_t<kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, mdo, mdq, stream);
     else e = bf ? launch_bwd_typed<64, kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, mdo, stream)
                 : launch_bwd_typed<64, kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, mdo, stream);
   }

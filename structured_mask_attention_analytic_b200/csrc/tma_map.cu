@@ -57,4 +57,30 @@ bool encode_map(CUtensorMap* map, const void* ptr, int dtype, int d, int heads, 
   return true;
 }
 
+bool encode_map_f32(CUtensorMap* map, const void* ptr, int d, int heads, int len, int batch,
+                    int box_d, int box_rows, char* msg, size_t msg_len) {
+  auto enc = get_encode_fn();
+  if (enc == nullptr) {
+    snprintf(msg, msg_len, "cuTensorMapEncodeTiled is unavailable");
+    return false;
+  }
+  const uint64_t s_head = static_cast<uint64_t>(d) * 4;
+  const uint64_t s_row = s_head * heads;
+  const uint64_t s_batch = s_row * len;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(len), static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[3] = {s_head, s_row, s_batch};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(box_d), 1, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(msg, msg_len, "cuTensorMapEncodeTiled (float32 accumulator) failed (%d)",
+             static_cast<int>(r));
+    return false;
+  }
+  return true;
+}
+
 }  // namespace sma

@@ -14,4 +14,9 @@ namespace sma {
 bool encode_map(CUtensorMap* map, const void* ptr, int dtype, int d, int heads, int len, int batch,
                 int64_t s_head, int64_t s_row, int64_t s_batch, char* msg, size_t msg_len);
 
+// 4D map over a float32 [B][len][heads][d] accumulator for bulk reductions:
+// box = box_d x 1 x box_rows x 1, 128-byte swizzle (box_d * 4 must be 128).
+bool encode_map_f32(CUtensorMap* map, const void* ptr, int d, int heads, int len, int batch,
+                    int box_d, int box_rows, char* msg, size_t msg_len);
+
 }  // namespace sma
