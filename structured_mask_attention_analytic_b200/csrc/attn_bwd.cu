@@ -689,18 +689,18 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
 //   S^T  = K Q^T        A = K (K-major)        B = Q (K-major)        SS
 //   dP^T = V dO^T       A = V (K-major)        B = dO (K-major)       SS
 //   dV  += P^T dO       A = P^T from TMEM      B = dO (MN-major)      TS
-//   dK  += dS^T Q       A = dS^T from TMEM     B = Q (MN-major)       TS
+//   dK  += dS^T Q       A = dS^T (K-major)     B = Q (MN-major)       SS
 //   dQ   = dS K         A = dS (MN-major)      B = K (MN-major)       SS
-// P^T and dS^T go to TMEM as packed 16-bit pairs over the first half of the
-// S^T / dP^T columns (as the forward's P does), so dV and dK read their A
-// operand from TMEM; only dS^T is also written to shared memory, where the
-// [key][query] tile read as an MN-major operand is dS itself (queries
-// contiguous), so dQ comes out with query rows in TMEM.
+// P^T goes to TMEM as packed 16-bit pairs over S^T's columns (pcol below),
+// as the forward's P does, so dV reads its A operand from TMEM.
+// dS^T is written to shared memory only: read K-major it is dK's A operand,
+// read MN-major it is dS itself (queries contiguous), so dQ comes out with
+// query rows in TMEM.
 // That halves the operand traffic the products and the compute threads put
 // on shared memory.  Two 128-column TMEM regions alternate between pairs:
-// pair i puts S^T / P^T and later dQ in region X_i, dP^T / dS^T in Y_i;
-// pair i+1 swaps them, so S^T(i+1) can be issued as soon as dK(i) has read
-// dS^T(i), and dP^T(i+1) once dQ(i) has been drained.
+// pair i puts S^T / P^T and later dQ in region X_i, dP^T in Y_i; pair i+1
+// swaps them, so S^T(i+1) is issued as soon as dS^T(i) is formed (ahead of
+// dK(i) and dQ(i)), and dP^T(i+1) once dQ(i) has been drained.
 // The producer stages, per pair, -lse * log2(e) and rowsum(dO * O) of the
 // 128 queries (and, for DFlash, each query's kept key intervals) in shared
 // memory next to the Q stage.
@@ -719,8 +719,22 @@ __device__ __forceinline__ void bulk_wait_read0() {
 }
 __device__ __forceinline__ void bulk_wait_all0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-constexpr int kBwdTThreads = 352;  // + warp 10: per-query data of each pair
-constexpr int kBAuxWarp = 10;
+// 16 warps in four warpgroups: compute (0-3, 4-7; each key row's 128 queries
+// split in two halves), dQ drain + epilogue (8-11), and producer / MMA /
+// per-query data / idle (12-15).  setmaxnreg moves registers from the last
+// group to the drain group; the shares add up to at most the launch
+// allocation (512 x kTLaunchRegs), and the host refuses to launch if the
+// compiled register count differs.
+constexpr int kBwdTThreads = 512;
+constexpr int kTDrainWarp0 = 8;
+constexpr int kTLoadWarp = 12;
+constexpr int kTMmaWarp = 13;
+constexpr int kBAuxWarp = 14;
+constexpr int kTLaunchRegs = 128;
+constexpr int kTDrainRegs = 168;
+constexpr int kTCtrlRegs = 88;
+static_assert(256 * kTLaunchRegs + 128 * kTDrainRegs + 128 * kTCtrlRegs <= kBwdTThreads * kTLaunchRegs,
+              "register split must fit the launch allocation");
 
 struct TLayout {
   static constexpr int D = 128;
@@ -749,6 +763,14 @@ struct TLayout {
   static constexpr uint32_t kColDV = 256, kColDK = 384;
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
+
+// Packed P^T column of query column q: each 64-query half packs into the
+// first half of its own S^T columns (queries 0-63 -> columns 0-31, queries
+// 64-127 -> columns 64-95), so the two compute warps of a key row never
+// write columns the other has yet to read.
+__host__ __device__ constexpr uint32_t pcol(int q) {
+  return static_cast<uint32_t>((q & ~63) + (q & 63) / 2);
+}
 
 template <int POLICY, int DT>
 __global__ void __launch_bounds__(kBwdTThreads, 1)
@@ -785,9 +807,9 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     mbar_init(bar(L::kOFull), 1);
     mbar_init(bar(L::kOEmpty), 1);
     mbar_init(bar(L::kSFull), 1);
-    mbar_init(bar(L::kPDone), 128);
+    mbar_init(bar(L::kPDone), 256);
     mbar_init(bar(L::kDPFull), 1);
-    mbar_init(bar(L::kDSDone), 128);
+    mbar_init(bar(L::kDSDone), 256);
     mbar_init(bar(L::kDQFull), 1);
     mbar_init(bar(L::kDQFree), 128);
     mbar_init(bar(L::kDSFree), 1);
@@ -797,7 +819,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kBMmaWarp) {
+  if (warp == kTMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kBTmemCols);
     tmem_relinquish();
   }
@@ -806,7 +828,9 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kBLoadWarp) {
+  if (warp >= kTLoadWarp) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kTCtrlRegs));
+   if (warp == kTLoadWarp) {
     // ------------------------------------------------------------ producer
     if (elect_one()) {
       tma_prefetch_map(&map_q);
@@ -879,7 +903,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
       }
       if (o_it > 0) bdrain_wait(bar(L::kOFull), (o_it - 1) & 1, p.f.err);
     }
-  } else if (warp == kBAuxWarp) {
+   } else if (warp == kBAuxWarp) {
     // ------------------------------------------------------------ per-query data
     // -lse * log2(e), rowsum(dO * O) and (DFlash) the kept key intervals of the
     // pair's 128 queries, 4 per lane; the global reads of the next pair are in
@@ -940,7 +964,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         ++q_it;
       }
     }
-  } else if (warp == kBMmaWarp) {
+   } else if (warp == kTMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t fmt = DT == SMA_BF16 ? 1u : 0u;
     constexpr uint32_t idesc_ss = mma_idesc_f16(fmt, 128, 128, 0, 0);  // S^T, dP^T
@@ -973,23 +997,26 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
       }
     };
     // acc[keys][d] (+)= A^T[keys][queries] B[queries][d], A packed in TMEM
+    // (queries 16 s .. 16 s + 15 at packed column pcol(16 s))
     auto issue_ts = [&](uint32_t dcol, uint32_t acol, uint32_t b_addr, bool acc) {
       const uint64_t bd = smem_desc_sw128(b_addr, L::kChunk, 1024);
 #pragma unroll
       for (int s = 0; s < kTile / 16; ++s)
-        tc_mma_ts(tmem + dcol, tmem + acol + 8 * s, with_lo(bd, (s * 2048) >> 4), idesc_ts,
+        tc_mma_ts(tmem + dcol, tmem + acol + pcol(16 * s), with_lo(bd, (s * 2048) >> 4), idesc_ts,
                   (acc || s > 0) ? 1u : 0u);
     };
-    // dK += dS^T Q (TS) interleaved with dQ = dS K (SS; the dS^T tile read as an
-    // MN-major A operand is dS with queries contiguous)
-    auto issue_dk_dq = [&](uint32_t ycol, uint32_t xcol, uint32_t q_addr, bool acc) {
+    // dK += dS^T Q (A = the dS^T tile, K-major) interleaved with dQ = dS K
+    // (A = the same tile read MN-major: dS with queries contiguous)
+    auto issue_dk_dq = [&](uint32_t xcol, uint32_t q_addr, bool acc) {
       const uint64_t qd = smem_desc_sw128(q_addr, L::kChunk, 1024);
       const uint64_t kd = smem_desc_sw128(sbase + L::kK, L::kChunk, 1024);
+      const uint64_t st = smem_desc_sw128(sbase + L::kDS, 16, 1024);
       const uint64_t sd = smem_desc_sw128(sbase + L::kDS, L::kChunk, 1024);
 #pragma unroll
       for (int s = 0; s < kTile / 16; ++s) {
         const uint32_t off = (s * 2048) >> 4;
-        tc_mma_ts(tmem + L::kColDK, tmem + ycol + 8 * s, with_lo(qd, off), idesc_ts,
+        const uint32_t koff = ((s >> 2) * L::kChunk + (s & 3) * 32) >> 4;
+        tc_mma_ss(tmem + L::kColDK, with_lo(st, koff), with_lo(qd, off), idesc_ts,
                   (acc || s > 0) ? 1u : 0u);
         tc_mma_ss(tmem + xcol, with_lo(sd, off), with_lo(kd, off), idesc_dq, s > 0 ? 1u : 0u);
       }
@@ -1032,11 +1059,18 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         }
         __syncwarp();
         ++o_it;
-        // dK += dS^T Q and dQ = dS K (into X, after dV has read P^T there)
+        // dS^T(i) is formed: Y is free (dP^T(i) consumed), so S^T(i+1) goes
+        // first, then dK += dS^T Q and dQ = dS K (into X, after dV read P^T)
         if (!wait(L::kDSDone, pit & 1)) break;
+        const uint32_t nq = q_it + 1;
+        if (i + 1 < n && !wait(L::kQFull + (nq & 1), (nq >> 1) & 1)) break;
         tc_fence_after();
         if (elect_one()) {
-          issue_dk_dq(Y, X, sbase + L::kQ + qs * L::kTileD, i > 0);
+          if (i + 1 < n) {
+            issue_t(Y, sbase + L::kK, sbase + L::kQ + (nq & 1) * L::kTileD);
+            tc_commit(bar(L::kSFull));
+          }
+          issue_dk_dq(X, sbase + L::kQ + qs * L::kTileD, i > 0);
           tc_commit(bar(L::kDQFull));
           tc_commit(bar(L::kDSFree));
           tc_commit(bar(L::kQEmpty + qs));
@@ -1045,14 +1079,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         ++q_it;
         ++pit;
         if (i + 1 < n) {
-          // S^T(i+1) into Y (dK has read dS^T there); dP^T(i+1) into X once dQ is drained
-          if (!wait(L::kQFull + (q_it & 1), (q_it >> 1) & 1)) break;
-          tc_fence_after();
-          if (elect_one()) {
-            issue_t(Y, sbase + L::kK, sbase + L::kQ + (q_it & 1) * L::kTileD);
-            tc_commit(bar(L::kSFull));
-          }
-          __syncwarp();
+          // dP^T(i+1) into X once dQ(i) is drained
           if (!wait(L::kOFull, o_it & 1)) break;
           if (!wait(L::kDQFree, (pit - 1) & 1)) break;
           tc_fence_after();
@@ -1076,10 +1103,13 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
       __syncwarp();
       bdrain_wait(bar(L::kDrain), 0, p.f.err);
     }
-  } else if (warp < 4) {
+   }
+  } else if (warp < kTDrainWarp0) {
     // ------------------------------------------------------------ compute (P^T, dS^T), key rows
-    const int r = warp * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // warp w: key rows 32 (w % 4) .. +31, queries 64 (w / 4) .. +63
+    const int r = (warp & 3) * 32 + lane;
+    const int qb = (warp >> 2) * 64;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float scale_log2 = p.f.scale_log2;
     const float bias_mul = kLog2e / p.f.scale_log2;
     uint32_t pit = 0, q_it = 0;
@@ -1128,17 +1158,18 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         // FULL pair carries none of the mask evaluation.
         auto phase_a = [&](auto masked_tag) {
           constexpr bool MASKED = decltype(masked_tag)::value;
-  #pragma unroll 1
-          for (int c = 0; c < kTile / 32; ++c) {
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            const int cq = qb + 32 * c;  // first query column of the chunk
             uint32_t xr[32];
-            tmem_ld32_at(xcol + 32 * c, xr);
+            tmem_ld32_at(xcol + cq, xr);
             // keep bits of the chunk's 32 queries (PARTIAL pairs only; the loads
             // are volatile so that FULL pairs never pay for them)
             uint32_t kbits = 0xffffffffu;
             if (MASKED) {
               kbits = 0u;
               if (POLICY == kPolicyDflash) {
-                const uint32_t ivs = sbase + L::kAux + s * L::kAuxBytes + 2 * kTile * 4 + 32 * c * 4;
+                const uint32_t ivs = sbase + L::kAux + s * L::kAuxBytes + 2 * kTile * 4 + cq * 4;
   #pragma unroll
                 for (int g4 = 0; g4 < 8; ++g4) {
                   const uint4 lo = ld_shared_v4(ivs + 16 * g4);
@@ -1159,7 +1190,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
                 const volatile uint8_t* mv = mcol;
   #pragma unroll 4
                 for (int z = 0; z < 32; ++z) {
-                  const int q = q0 + 32 * c + z;
+                  const int q = q0 + cq + z;
                   const int qc = q < p.f.Lq ? q : 0;
                   const bool keep = key < p.f.Lk && (!p.f.causal || key <= q + p.f.Lk - p.f.Lq) &&
                                     (!p.f.has_mask || mv[qc * msq] != 0);
@@ -1171,14 +1202,14 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
             uint32_t pk[16];
   #pragma unroll
             for (int e = 0; e < 32; e += 4) {
-              const float4 n4 = *reinterpret_cast<const float4*>(nl + 32 * c + e);
+              const float4 n4 = *reinterpret_cast<const float4*>(nl + cq + e);
               const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
               float pv[4];
   #pragma unroll
               for (int z = 0; z < 4; ++z) {
                 float x = __uint_as_float(xr[e + z]);
                 if (POLICY != kPolicyDflash && p.f.has_bias) {
-                  const int q = q0 + 32 * c + e + z;
+                  const int q = q0 + cq + e + z;
                   const int qc = q < p.f.Lq ? q : 0;  // rows past Lq read row 0 (their P is 0)
                   x = fmaf(load_any_as_float(bcol + qc * bsq, bdt, 0), bias_mul, x);
                 }
@@ -1187,7 +1218,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
               pk[e >> 1] = DT == SMA_BF16 ? pack_bf16x2(pv[0], pv[1]) : pack_f16x2(pv[0], pv[1]);
               pk[(e >> 1) + 1] = DT == SMA_BF16 ? pack_bf16x2(pv[2], pv[3]) : pack_f16x2(pv[2], pv[3]);
             }
-            tmem_st16_at(xcol + 16 * c, pk);
+            tmem_st16_at(xcol + pcol(cq), pk);
           }
         };
         if (partial) phase_a(std::true_type{});
@@ -1196,7 +1227,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         tc_fence_before();
         mbar_arrive(bar(L::kPDone));
 
-        // ---- phase B: dS^T = P^T (dP^T - D), packed into Y and stored to shared memory
+        // ---- phase B: dS^T = P^T (dP^T - D), stored to shared memory
         if (!mbar_wait(bar(L::kDPFull), pit & 1, abort_flag, p.f.err)) { ok = false; break; }
         if (pit > 0 && !mbar_wait(bar(L::kDSFree), (pit - 1) & 1, abort_flag, p.f.err)) {
           ok = false;
@@ -1204,15 +1235,16 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         }
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < kTile / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
+          const int cq = qb + 32 * c;
           uint32_t yr[32], pr[16];
-          tmem_ld32_at(ycol + 32 * c, yr);
-          tmem_ld16_at(xcol + 16 * c, pr);
+          tmem_ld32_at(ycol + cq, yr);
+          tmem_ld16_at(xcol + pcol(cq), pr);
           tc_wait_ld();
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
-            const float4 d4 = *reinterpret_cast<const float4*>(dd + 32 * c + e);
+            const float4 d4 = *reinterpret_cast<const float4*>(dd + cq + e);
             const float2 p01 = unpack2<DT>(pr[e >> 1]);
             const float2 p23 = unpack2<DT>(pr[(e >> 1) + 1]);
             const float s0 = p01.x * (__uint_as_float(yr[e]) - d4.x);
@@ -1222,14 +1254,12 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
             pk[e >> 1] = DT == SMA_BF16 ? pack_bf16x2(s0, s1) : pack_f16x2(s0, s1);
             pk[(e >> 1) + 1] = DT == SMA_BF16 ? pack_bf16x2(s2, s3) : pack_f16x2(s2, s3);
           }
-          tmem_st16_at(ycol + 16 * c, pk);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
-            st_shared_v4(sw128_unit(sbase + L::kDS, r, 4 * c + v4), pk[4 * v4], pk[4 * v4 + 1],
+            st_shared_v4(sw128_unit(sbase + L::kDS, r, cq / 8 + v4), pk[4 * v4], pk[4 * v4 + 1],
                          pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }
         fence_async_shared();
-        tc_wait_st();
         tc_fence_before();
         mbar_arrive(bar(L::kDSDone));
         ++pit;
@@ -1238,7 +1268,8 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     }
   } else {
     // ------------------------------------------------------------ dQ drain, dK / dV epilogue
-    const int wq = warp - 4;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kTDrainRegs));
+    const int wq = warp - kTDrainWarp0;
     const int r = wq * 32 + lane;  // dQ: query row; dK / dV: key row
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t dv_col = tmem + lane_off + L::kColDV;
@@ -1343,7 +1374,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kBMmaWarp) tmem_dealloc(tmem, kBTmemCols);
+  if (warp == kTMmaWarp) tmem_dealloc(tmem, kBTmemCols);
 }
 
 template <int POLICY, int DT>
@@ -1353,8 +1384,13 @@ cudaError_t launch_bwd_t(const BwdProblem& p, const CUtensorMap& mq, const CUten
   auto kern = attn_bwd_t_kernel<POLICY, DT>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(TLayout::kAlloc));
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    // The setmaxnreg split assumes exactly kTLaunchRegs registers per thread.
+    if (fa.numRegs != kTLaunchRegs) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(TLayout::kAlloc));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
