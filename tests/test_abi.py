@@ -177,3 +177,38 @@ def test_sparse_attn_needs_a_mask():
         ctypes.c_void_p(0x40000), nat.i64_array(qs), None, ctypes.c_void_p(0x50000), 1 << 30, None)
     assert st == nat.SMA_ERR_INVALID_ARG
     assert "needs a mask" in nat.load().sma_last_error().decode()
+
+
+def test_backward_workspace_and_validation_on_host():
+    lib = nat.load()
+    n = ctypes.c_size_t()
+    d = nat.DfaMaskDesc(1, 2048, 16, 32768, 1, 0, 0)
+    assert lib.dfa_attn_bwd_workspace_size(ctypes.byref(d), 32, 8, 128, ctypes.byref(n)) == 0
+    # the fp32 dQ accumulator alone is B * Lq * H * d * 4 bytes
+    assert n.value >= 32768 * 32 * 128 * 4
+    ms = nat.i64_array([1, 1, 8192, 8064])
+    assert lib.masked_attn_bwd_workspace_size(4, 16, 4, 8192, 8000, 128, ms, ctypes.byref(n)) == 0
+    assert n.value >= 4 * 8192 * 16 * 128 * 4
+    assert lib.masked_attn_bwd_workspace_size(4, 16, 4, 8192, 8000, 96, ms, ctypes.byref(n)) == nat.SMA_ERR_UNSUPPORTED
+
+    qs = [256 * 4 * 128, 4 * 128, 128]
+    ks = [200 * 2 * 128, 2 * 128, 128]
+
+    def call(dtype=0, lse=0x70000, dbias=0):
+        return lib.masked_attn_bwd(
+            dtype, 2, 4, 2, 256, 200, 128, ctypes.c_float(0.0), 0,
+            ctypes.c_void_p(0x10000), nat.i64_array(qs), ctypes.c_void_p(0x20000), nat.i64_array(ks),
+            ctypes.c_void_p(0x30000), nat.i64_array(ks), ctypes.c_void_p(0), None, None,
+            ctypes.c_void_p(0), 0, None, None,
+            ctypes.c_void_p(0x40000), nat.i64_array(qs), ctypes.c_void_p(lse),
+            ctypes.c_void_p(0x50000), nat.i64_array(qs),
+            ctypes.c_void_p(0x60000), nat.i64_array(qs), ctypes.c_void_p(0x80000), nat.i64_array(ks),
+            ctypes.c_void_p(0x90000), nat.i64_array(ks), ctypes.c_void_p(dbias),
+            ctypes.c_void_p(0xa0000), 1 << 30, None)
+
+    assert call(dtype=2) == nat.SMA_ERR_UNSUPPORTED
+    assert "bf16 or fp16" in lib.sma_last_error().decode()
+    assert call(lse=0) == nat.SMA_ERR_INVALID_ARG
+    assert "lse" in lib.sma_last_error().decode()
+    assert call(dbias=0xb0000) == nat.SMA_ERR_UNSUPPORTED
+    assert "dbias" in lib.sma_last_error().decode()
