@@ -731,8 +731,8 @@ constexpr int kTLoadWarp = 12;
 constexpr int kTMmaWarp = 13;
 constexpr int kBAuxWarp = 14;
 constexpr int kTLaunchRegs = 128;
-constexpr int kTDrainRegs = 168;
-constexpr int kTCtrlRegs = 88;
+constexpr int kTDrainRegs = 144;
+constexpr int kTCtrlRegs = 112;
 static_assert(256 * kTLaunchRegs + 128 * kTDrainRegs + 128 * kTCtrlRegs <= kBwdTThreads * kTLaunchRegs,
               "register split must fit the launch allocation");
 
@@ -781,8 +781,9 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
   using L = TLayout;
   constexpr int D = L::D;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned by offsetting the shared array itself, so that pointers
+  // derived from it keep the shared state space (shared loads, not generic)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * static_cast<uint32_t>(i); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
