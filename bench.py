@@ -281,7 +281,7 @@ def run_ours(args, rank, world, dev):
     return res
 
 
-DETAILS = ("dflash", "dflash_bwd", "broadcast_prefill", "broadcast_decode", "topk", "topk_wide")
+DETAILS = ("dflash", "dflash_bwd", "spec_generate", "broadcast_prefill", "broadcast_decode", "topk", "topk_wide")
 
 
 def run_details(sma, dev, stream, peaks, only=None):
@@ -324,6 +324,22 @@ def run_details(sma, dev, stream, peaks, only=None):
                                 "status": sma.device_status()}
         del q, k, v, o, lse, do, dq, dk, dv, ws
         torch.cuda.empty_cache()
+
+    if want("spec_generate"):
+        # DFlash inference: one block of 16 draft queries after a 32k context (HBM-bound: K/V read once)
+        wd = wl.DFLASH_LONG_FULL
+        bs, lc = wd.block_size, wd.ctx_len
+        g = torch.Generator(device=dev).manual_seed(7)
+        q = torch.randn((1, bs, wd.heads, wd.head_dim), device=dev, generator=g).to(torch.bfloat16)
+        k = torch.randn((1, lc + bs, wd.kv_heads, wd.head_dim), device=dev, generator=g).to(torch.bfloat16)
+        v = torch.randn_like(k)
+        cl = torch.tensor([lc], dtype=torch.int32, device=dev)
+        o = torch.empty_like(q)
+        ms = timed(lambda: sma.dflash_spec_generate_fwd(q, k, v, cl, lc, True, out=o), stream, 20, 3)
+        nbytes = 2 * k.numel() * 2 + 2 * q.numel() * 2
+        out["spec_generate_32k"] = {"ms": ms, "GB/s": nbytes / (ms * 1e-3) / 1e9,
+                                    "frac_hbm_peak": nbytes / (ms * 1e-3) / 1e9 / pk_b, "bytes": nbytes}
+        del q, k, v, o
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     if want("broadcast_prefill"):

@@ -129,3 +129,18 @@ def dflash_keep_scalar(anchors, ctx_len: int, block_size: int, in_block_causal: 
             continue
         visible.add(block_first + t)
     return k in visible
+
+
+def spec_generate_keep_mask(ctx_lens, ctx_len: int, block_size: int, in_block_causal: bool,
+                            window) -> np.ndarray:
+    """Keep mask ``[B, block_size, ctx_len + block_size]`` of DFlash inference
+    (``spec_generate``): one draft block placed after each row's context.
+
+    SpecForge PR #905 (Motivation list and the maintainer's split note, item
+    2/3) moves the mask builders to a module shared by training and inference
+    and adds default masks for ``spec_generate``; the plainest reading is the
+    training rule above with a single block whose anchor is the row's context
+    length ``ctx_lens[b] <= ctx_len`` (keys ``[ctx_lens[b], ctx_len)`` are
+    padding and never kept)."""
+    anchors = np.asarray(ctx_lens).reshape(-1, 1)
+    return dflash_keep_mask(anchors, ctx_len, block_size, in_block_causal, window)

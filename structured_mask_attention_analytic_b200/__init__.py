@@ -17,6 +17,7 @@ from .ops import (  # noqa: F401
     dfa_attn_fwd_workspace_size,
     dfa_block_map,
     dfa_block_map_dims,
+    dflash_spec_generate_fwd,
     dynamic_topk_mask,
     mask_tile_summary,
     masked_attn_bwd,

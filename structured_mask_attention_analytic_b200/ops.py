@@ -151,6 +151,25 @@ def dfa_attn_fwd(q, k, v, anchors, ctx_len: int, block_size: int, is_causal=None
     return out, lse
 
 
+def dflash_spec_generate_fwd(q, k, v, ctx_lens, ctx_len: int, is_causal=None, layer_type: int = LAYER_FULL,
+                             sliding_window: int = 0, scale=None, out=None, return_lse: bool = True,
+                             workspace=None):
+    """Attention of DFlash inference (``spec_generate``): one draft block of
+    ``q.shape[1]`` queries after each row's context.
+
+    q ``[B, block_size, H, d]``; k/v ``[B, ctx_len + block_size, KVH, d]`` with
+    row b's context in keys ``[0, ctx_lens[b])`` (the rest of the first
+    ``ctx_len`` keys is padding) and the block's own keys last; ``ctx_lens``
+    int32 ``[B]`` on the device.  This is ``dfa_attn_fwd`` with one block
+    whose anchor is the row's context length (the same C entry point)."""
+    _require_cuda(ctx_lens)
+    if ctx_lens.dtype != torch.int32 or ctx_lens.dim() != 1 or ctx_lens.shape[0] != q.shape[0]:
+        raise ValueError("ctx_lens must be int32 [batch]")
+    anchors = ctx_lens.contiguous().view(-1, 1)
+    return dfa_attn_fwd(q, k, v, anchors, ctx_len, q.shape[1], is_causal, layer_type, sliding_window,
+                        scale=scale, out=out, return_lse=return_lse, workspace=workspace)
+
+
 def dfa_attn_bwd_workspace_size(batch, n_blocks, block_size, ctx_len, heads, kv_heads, head_dim,
                                 is_causal=None, layer_type=LAYER_FULL, sliding_window=0) -> int:
     d = _desc(batch, n_blocks, block_size, ctx_len, is_causal, layer_type, sliding_window)

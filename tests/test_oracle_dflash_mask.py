@@ -112,3 +112,27 @@ def test_sliding_window_requires_positive_size():
     with pytest.raises(ValueError):
         dm.resolve_window(dm.LAYER_SLIDING, 0)
     assert dm.resolve_window(dm.LAYER_FULL, 0) is None
+
+
+@pytest.mark.parametrize("causal,window", [(False, None), (True, None), (True, 5), (False, 3)])
+def test_spec_generate_mask_equals_position_walk(causal, window):
+    """Inference mask (one block after a padded context) against the scalar
+    position walk, plus its plain reading: every context key below the row's
+    length, nothing of the padding, the block by the in-block rule."""
+    ctx_lens = np.array([0, 7, 20, 13])
+    Lc, bs = 20, 6
+    m = dm.spec_generate_keep_mask(ctx_lens, Lc, bs, causal, window)
+    assert m.shape == (4, bs, Lc + bs)
+    for b in range(4):
+        for i in range(bs):
+            for k in range(Lc + bs):
+                want = dm.dflash_keep_scalar(ctx_lens.reshape(-1, 1), Lc, bs, causal, window, b, i, k)
+                assert m[b, i, k] == want
+            assert not m[b, i, ctx_lens[b]:Lc].any()          # padding never kept
+            if window is None:
+                assert m[b, i, :ctx_lens[b]].all()            # the whole context
+            t = np.arange(bs)
+            block = (t <= i) if causal else np.ones(bs, bool)
+            if window is not None:
+                block &= i - t < window
+            assert (m[b, i, Lc:] == block).all()
