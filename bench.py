@@ -281,7 +281,7 @@ def run_ours(args, rank, world, dev):
     return res
 
 
-DETAILS = ("dflash", "dflash_bwd", "spec_generate", "broadcast_prefill", "broadcast_decode", "topk", "topk_wide")
+DETAILS = ("dflash", "dflash_bwd", "spec_generate", "varlen", "broadcast_prefill", "broadcast_decode", "topk", "topk_wide")
 
 
 def run_details(sma, dev, stream, peaks, only=None):
@@ -339,6 +339,24 @@ def run_details(sma, dev, stream, peaks, only=None):
         nbytes = 2 * k.numel() * 2 + 2 * q.numel() * 2
         out["spec_generate_32k"] = {"ms": ms, "GB/s": nbytes / (ms * 1e-3) / 1e9,
                                     "frac_hbm_peak": nbytes / (ms * 1e-3) / 1e9 / pk_b, "bytes": nbytes}
+        del q, k, v, o
+
+    if want("varlen"):
+        # packed causal training batch: 12 sequences of random lengths up to 8192 (seed 5), H 32 / KVH 8, d 128
+        rng = np.random.default_rng(5)
+        lens = rng.integers(256, 8193, size=12).tolist()
+        cu = torch.tensor(np.cumsum([0] + lens), dtype=torch.int32, device=dev)
+        total = int(sum(lens))
+        g = torch.Generator(device=dev).manual_seed(5)
+        q = torch.randn((total, 32, 128), device=dev, generator=g).to(torch.bfloat16)
+        k = torch.randn((total, 8, 128), device=dev, generator=g).to(torch.bfloat16)
+        v = torch.randn_like(k)
+        o = torch.empty_like(q)
+        ms = timed(lambda: sma.varlen_attn_fwd(q, k, v, cu, cu, max(lens), max(lens), True, out=o), stream, 10, 3)
+        kept = sum(sum(1 for a in range(-(-L // TILE)) for c in range(-(-L // TILE)) if c <= a) for L in lens)
+        tf = tile_flops(128, 32, kept) / (ms * 1e-3) / 1e12
+        out["varlen_causal_12seq"] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / pk_t, "tokens": total,
+                                      "kept_tiles_per_head": kept}
         del q, k, v, o
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)

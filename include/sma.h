@@ -1,18 +1,25 @@
 /*
- * sma.h -- C ABI of libsma: scaled-dot-product attention forward under
- * structured masks on NVIDIA B200 (sm_100a).
+ * sma.h -- C ABI of libsma: scaled-dot-product attention under structured
+ * masks on NVIDIA B200 (sm_100a).
  *
- * Four operations, all asynchronous on the caller's CUDA stream:
+ * Operations, all asynchronous on the caller's CUDA stream:
  *
  *   dfa_block_map      full / partial / empty key-tile lists of the DFlash
  *                      draft-training mask, computed from the block anchors
  *                      alone (no dense mask is ever built).
- *   dfa_attn_fwd       attention forward under that mask.
+ *   dfa_attn_fwd       attention forward under that mask (also the DFlash
+ *                      inference mask: one block, anchor = context length).
  *   masked_attn_fwd    attention forward with a broadcastable 4D boolean mask
  *                      and/or additive bias, optional causal masking, and the
  *                      single-query grouped-head ("swapped") decode path.
  *   dynamic_topk_mask  boolean keep mask of the window_size largest entries
  *                      of an attention bias per row, after a pre-mask.
+ *   sparse_attn_fwd    masked_attn_fwd over only the keys a query-broadcast
+ *                      mask keeps (index gather), e.g. a top-k mask.
+ *   dfa_attn_bwd,      gradients dQ, dK, dV of the two attention forwards.
+ *   masked_attn_bwd
+ *   varlen_attn_fwd    attention over packed variable-length sequences, with
+ *                      varlen_pad / varlen_unpad.
  *
  * plus mask_tile_summary (the tile classifier masked_attn_fwd runs on an
  * explicit mask), workspace queries and error reporting.
@@ -342,6 +349,52 @@ sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
                            void* dk, const int64_t dk_strides[3], void* dv,
                            const int64_t dv_strides[3], float* dbias, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Variable-length (packed) batches.
+ *
+ * Source: flash-sparse-attention PR #197, Changes list: the integration's
+ * loader returns a varlen attention function and pad / unpad helpers next to
+ * the padded one; the pages give no interface, so this follows the packed
+ * layout those names denote.  Sequence b owns rows [cu_seqlens_q[b],
+ * cu_seqlens_q[b+1]) of the packed queries and [cu_seqlens_k[b],
+ * cu_seqlens_k[b+1]) of the packed keys (int32 [batch + 1], ascending, on the
+ * device); it attends only its own keys, bottom-right causal per sequence
+ * when is_causal (key k kept iff k <= q + len_k - len_q).  No mask or bias.
+ *
+ * q, out   [total_q, heads, d]; k, v [total_k, kv_heads, d]; strides[2] =
+ *          {row, head} in elements, d contiguous, 16-byte multiples.
+ * lse      NULL or float32 [heads, total_q] (natural log; -inf for rows
+ *          with no kept key, e.g. causal rows when len_q > len_k).
+ * max_q / max_k bound every sequence's lengths (host values, size the tile
+ *          lists); offsets that break a bound, are not ascending or exceed
+ *          the totals raise SMA_ERR_DEVICE_INPUT in the device error word and
+ *          leave that sequence's rows unwritten.
+ * dtype    SMA_BF16 / SMA_FP16; head_dim 64 or 128.
+ * ---------------------------------------------------------------------- */
+
+sma_status varlen_attn_fwd_workspace_size(int32_t batch, int32_t max_q, int32_t max_k, size_t* bytes);
+
+sma_status varlen_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t head_dim, int32_t total_q, int32_t total_k, int32_t max_q,
+                           int32_t max_k, float scale, int32_t is_causal, const int32_t* cu_seqlens_q,
+                           const int32_t* cu_seqlens_k, const void* q, const int64_t q_strides[2],
+                           const void* k, const int64_t k_strides[2], const void* v,
+                           const int64_t v_strides[2], void* out, const int64_t o_strides[2],
+                           float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* pad: padded [batch, max_len, heads, d] (strides[3] = batch, row, head) from
+ * packed rows, zero past each sequence's length; unpad: the reverse (rows
+ * past a length are not read).  Rows must be 16-byte multiples. */
+sma_status varlen_pad(int32_t dtype, int32_t batch, int32_t max_len, int32_t heads,
+                      int32_t head_dim, const int32_t* cu_seqlens, const void* packed,
+                      const int64_t packed_strides[2], void* padded,
+                      const int64_t padded_strides[3], void* stream);
+
+sma_status varlen_unpad(int32_t dtype, int32_t batch, int32_t max_len, int32_t heads,
+                        int32_t head_dim, const int32_t* cu_seqlens, const void* padded,
+                        const int64_t padded_strides[3], void* packed,
+                        const int64_t packed_strides[2], void* stream);
 
 /* ------------------------------------------------------------------------
  * Index-gather attention under a query-broadcast keep mask.

@@ -149,6 +149,31 @@ def attention(q, k, v, *, keep=None, keep_rows=None, bias=None, scale=None,
     return out, lse
 
 
+def varlen_attention(q, k, v, cu_q, cu_k, causal: bool = False, scale=None):
+    """Packed variable-length sequences: sequence b is rows ``cu_q[b]:cu_q[b+1]``
+    of q (``[total_q, H, d]``) and ``cu_k[b]:cu_k[b+1]`` of k / v and attends
+    only its own keys, bottom-right causal within the sequence when ``causal``.
+
+    The packed form behind flash-sparse-attention PR #197's varlen function
+    and pad / unpad helpers (Changes list); each sequence is the dense
+    attention above.  Returns ``out [total_q, H, d]`` and ``lse [H, total_q]``.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    out = np.zeros(q.shape)
+    lse = np.full((q.shape[1], q.shape[0]), -np.inf)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        if q1 == q0 or k1 == k0:
+            continue
+        keep = causal_keep(q1 - q0, k1 - k0)[None, None] if causal else None
+        o, l = attention(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], keep=keep, scale=scale)
+        out[q0:q1] = o[0]
+        lse[:, q0:q1] = l[0]
+    return out, lse
+
+
 def host_threads() -> int:
     """Cores this process may run on."""
     try:

@@ -87,6 +87,12 @@ _SIGNATURES = {
                                 c_vp, c_i64p, c_vp, c_vp, c_i64p,
                                 c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
                                 c_vp, c_vp, c_size, c_vp]),
+    "varlen_attn_fwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_sizep]),
+    "varlen_attn_fwd": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.c_float,
+                                c_i32, c_vp, c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
+                                c_vp, c_vp, c_size, c_vp]),
+    "varlen_pad": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp]),
+    "varlen_unpad": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp]),
     "sparse_attn_fwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64p,
                                                c_i32, c_i64p, c_i32, c_sizep]),
     "sparse_attn_fwd": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.c_float, c_i32,

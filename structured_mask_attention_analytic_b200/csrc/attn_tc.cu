@@ -35,6 +35,9 @@
 //               keep, additive bias, stride-0 broadcast dims), plus
 //               bottom-right causal masking; the bias is added on every kept
 //               tile, the mask read on PARTIAL tiles only.
+//   Varlen   -- packed sequences: the explicit policy without mask or bias,
+//               each unit's rows offset to its sequence and bounded by its
+//               lengths (bottom-right causal per sequence).
 //   Gather   -- the explicit policy over keys compacted by a query-broadcast
 //               mask (PR #197 top-k masks): K/V/bias are the compacted
 //               operands and each row's causal bound is a limit on the
@@ -90,8 +93,10 @@ struct Unit {
   int b, hk, pair, qt, h0, h1valid;
   int64_t list_row;
   int n_full, n_part;
+  int q_off, k_off, lq, lk;  // varlen: the sequence's first rows and lengths
 };
 
+template <int POLICY>
 __device__ __forceinline__ Unit decode_unit(const AttnProblem& p, int u) {
   Unit w;
   const int per_qt = p.B * p.KVH * p.npairs;
@@ -110,6 +115,24 @@ __device__ __forceinline__ Unit decode_unit(const AttnProblem& p, int u) {
   w.list_row = (static_cast<int64_t>(lb) * p.lists.LH + lh) * p.QT + w.qt;
   w.n_full = p.lists.num_full[w.list_row];
   w.n_part = p.lists.num_part[w.list_row];
+  if (POLICY == kPolicyVarlen) {
+    w.q_off = p.cu_q[w.b];
+    w.lq = p.cu_q[w.b + 1] - w.q_off;
+    w.k_off = p.cu_k[w.b];
+    w.lk = p.cu_k[w.b + 1] - w.k_off;
+    // malformed offsets (reported by the list kernel): the sequence is empty,
+    // so no row of it is read or written
+    if (w.lq < 0 || w.lq > p.Lq || w.q_off < 0 || w.q_off + w.lq > p.total_q || w.lk < 0 ||
+        w.lk > p.Lk || w.k_off < 0 || w.k_off + w.lk > p.total_k) {
+      w.q_off = w.k_off = w.lq = w.lk = 0;
+      w.n_full = w.n_part = 0;
+    }
+  } else {
+    w.q_off = 0;
+    w.k_off = 0;
+    w.lq = p.Lq;
+    w.lk = p.Lk;
+  }
   return w;
 }
 
@@ -190,7 +213,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
     uint32_t kv_k = 0, kv_v = 0, q_it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit w = decode_unit(p, u);
+      const Unit w = decode_unit<POLICY>(p, u);
       const int n = w.n_full + w.n_part;
       if (n == 0) continue;
       if (q_it > 0 && !mbar_wait_warp(bar(L::kQEmpty), (q_it - 1) & 1, abort_flag, p.err)) {
@@ -202,7 +225,8 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
         for (int i = 0; i < 1 + w.h1valid; ++i)
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sbase + L::kQ + i * L::kTileBytes + c * L::kChunkBytes, &map_q,
-                        bar(L::kQFull), c * 64, w.h0 + i, w.qt * kTile, w.b);
+                        bar(L::kQFull), c * 64, w.h0 + i, w.q_off + w.qt * kTile,
+                        POLICY == kPolicyVarlen ? 0 : w.b);
       }
       __syncwarp();
       ++q_it;
@@ -222,7 +246,8 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           mbar_arrive_expect_tx(bar(L::kKFull + kstage), L::kTileBytes);
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sbase + L::kK + kstage * L::kTileBytes + c * L::kChunkBytes, &map_k,
-                        bar(L::kKFull + kstage), c * 64, w.hk, kt * kTile, w.b);
+                        bar(L::kKFull + kstage), c * 64, w.hk, w.k_off + kt * kTile,
+                        POLICY == kPolicyVarlen ? 0 : w.b);
         }
         __syncwarp();
         ++kv_k;
@@ -237,7 +262,8 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           mbar_arrive_expect_tx(bar(L::kVFull + vstage), L::kTileBytes);
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sbase + L::kV + vstage * L::kTileBytes + c * L::kChunkBytes, &map_v,
-                        bar(L::kVFull + vstage), c * 64, w.hk, kt * kTile, w.b);
+                        bar(L::kVFull + vstage), c * 64, w.hk, w.k_off + kt * kTile,
+                        POLICY == kPolicyVarlen ? 0 : w.b);
         }
         __syncwarp();
         ++kv_v;
@@ -309,7 +335,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
       }
     };
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit w = decode_unit(p, u);
+      const Unit w = decode_unit<POLICY>(p, u);
       const int n = w.n_full + w.n_part;
       const int nq = 1 + w.h1valid;
       if (n > 0) {
@@ -412,11 +438,11 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
     uint32_t it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit w = decode_unit(p, u);
+      const Unit w = decode_unit<POLICY>(p, u);
       if (qi == 1 && !w.h1valid) continue;
       const int h = w.h0 + qi;
       const int q = w.qt * kTile + r;
-      const bool row_valid = q < p.Lq;
+      const bool row_valid = q < w.lq;
       const int n = w.n_full + w.n_part;
 
       // Per-row mask parameters.
@@ -452,7 +478,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
         if (POLICY == kPolicyGather)  // compacted keys: the row's limit on the compacted index
           causal_lim = row_valid ? gather_row_limit(p, w.list_row / p.QT, q) - 1 : -1;
         else if (p.causal)
-          causal_lim = q + p.Lk - p.Lq;
+          causal_lim = q + w.lk - w.lq;
       }
 
       // Scores are scaled inside the exponent (one FFMA per element).  A bias
@@ -461,7 +487,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
       const float exp_scale = p.scale_log2;
       const float bias_mul = kLog2e / p.scale_log2;
       // With compacted keys every PARTIAL tile is cut by the row limit.
-      const int causal_off = POLICY == kPolicyGather ? -(1 << 30) : p.Lk - p.Lq;
+      const int causal_off = POLICY == kPolicyGather ? -(1 << 30) : w.lk - w.lq;
       const bool mask_bcast_q = POLICY == kPolicyExplicit && p.has_mask && p.mask.sq == 0;
       float m_ref = -INFINITY, l_sum = 0.f;
       bool partial_next = false;
@@ -531,7 +557,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
             // Columns c >= lim fail the key-length or causal bound; both bounds
             // are checked only on tiles they can cut (uniform per tile).
             int lim = kTile;
-            if (k0 + kTile > p.Lk) lim = min(lim, p.Lk - k0);
+            if (k0 + kTile > w.lk) lim = min(lim, w.lk - k0);
             if (p.causal && k0 + kTile - 1 > w.qt * kTile + causal_off)
               lim = min(lim, causal_lim - k0 + 1);
             if (mask_bcast_q) {
@@ -641,7 +667,8 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
 
       // Epilogue: O / l, lse.
       typedef typename std::conditional<DT == SMA_BF16, __nv_bfloat16, __half>::type OutT;
-      OutT* orow = reinterpret_cast<OutT*>(p.o) + w.b * p.o_sb + static_cast<int64_t>(q) * p.o_sr +
+      OutT* orow = reinterpret_cast<OutT*>(p.o) + (POLICY == kPolicyVarlen ? 0 : w.b) * p.o_sb +
+                   static_cast<int64_t>(w.q_off + q) * p.o_sr +
                    h * p.o_sh;
       const float inv_l = l_sum > 0.f ? 1.0f / l_sum : 0.f;
       if (n > 0) {
@@ -672,7 +699,8 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
         for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
       }
       if (row_valid && p.lse != nullptr) {
-        p.lse[(static_cast<int64_t>(w.b) * p.H + h) * p.Lq + q] =
+        p.lse[POLICY == kPolicyVarlen ? static_cast<int64_t>(h) * p.total_q + w.q_off + q
+                                      : (static_cast<int64_t>(w.b) * p.H + h) * p.Lq + q] =
             l_sum > 0.f ? (m_ref + __log2f(l_sum)) * kLn2 : -INFINITY;
       }
       tc_fence_before();
@@ -716,9 +744,12 @@ cudaError_t launch_typed(const AttnProblem& p, const CUtensorMap& mq, const CUte
 
 int launch_attn_tc(const AttnProblem& p, cudaStream_t stream, char* msg, size_t msg_len) {
   CUtensorMap mq, mk, mv;
-  if (!encode_map(&mq, p.q, p.dtype, p.d, p.H, p.Lq, p.B, p.q_sh, p.q_sr, p.q_sb, msg, msg_len) ||
-      !encode_map(&mk, p.k, p.dtype, p.d, p.KVH, p.Lk, p.B, p.k_sh, p.k_sr, p.k_sb, msg, msg_len) ||
-      !encode_map(&mv, p.v, p.dtype, p.d, p.KVH, p.Lk, p.B, p.v_sh, p.v_sr, p.v_sb, msg, msg_len))
+  // packed sequences: one batch entry of total_q (total_k) rows
+  const bool packed = p.policy == kPolicyVarlen;
+  const int lq = packed ? p.total_q : p.Lq, lk = packed ? p.total_k : p.Lk, nb = packed ? 1 : p.B;
+  if (!encode_map(&mq, p.q, p.dtype, p.d, p.H, lq, nb, p.q_sh, p.q_sr, p.q_sb, msg, msg_len) ||
+      !encode_map(&mk, p.k, p.dtype, p.d, p.KVH, lk, nb, p.k_sh, p.k_sr, p.k_sb, msg, msg_len) ||
+      !encode_map(&mv, p.v, p.dtype, p.d, p.KVH, lk, nb, p.v_sh, p.v_sr, p.v_sb, msg, msg_len))
     return SMA_ERR_CUDA;
   cudaError_t e = cudaErrorInvalidValue;
   const bool bf = p.dtype == SMA_BF16;
@@ -732,6 +763,11 @@ int launch_attn_tc(const AttnProblem& p, cudaStream_t stream, char* msg, size_t 
                            : launch_typed<128, kPolicyGather, SMA_FP16>(p, mq, mk, mv, stream);
     else e = bf ? launch_typed<64, kPolicyGather, SMA_BF16>(p, mq, mk, mv, stream)
                 : launch_typed<64, kPolicyGather, SMA_FP16>(p, mq, mk, mv, stream);
+  } else if (p.policy == kPolicyVarlen) {
+    if (p.d == 128) e = bf ? launch_typed<128, kPolicyVarlen, SMA_BF16>(p, mq, mk, mv, stream)
+                           : launch_typed<128, kPolicyVarlen, SMA_FP16>(p, mq, mk, mv, stream);
+    else e = bf ? launch_typed<64, kPolicyVarlen, SMA_BF16>(p, mq, mk, mv, stream)
+                : launch_typed<64, kPolicyVarlen, SMA_FP16>(p, mq, mk, mv, stream);
   } else {
     if (p.d == 128) e = bf ? launch_typed<128, kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, stream)
                            : launch_typed<128, kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, stream);

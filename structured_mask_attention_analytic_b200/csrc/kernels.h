@@ -44,7 +44,8 @@ struct TileLists {
 };
 
 // Gather: explicit policy over compacted keys (GatherView set, no mask).
-enum MaskPolicy { kPolicyDflash = 0, kPolicyExplicit = 1, kPolicyGather = 2 };
+// Varlen: packed sequences (cu_q / cu_k set), causal or not, no mask / bias.
+enum MaskPolicy { kPolicyDflash = 0, kPolicyExplicit = 1, kPolicyGather = 2, kPolicyVarlen = 3 };
 
 // Index-gather view of a query-broadcast keep mask: per gather row (batch
 // row LB x head row LH of the mask, the same rows as the tile lists) the
@@ -79,6 +80,11 @@ struct AttnProblem {
   int has_mask, has_bias;
   AuxView mask, bias;
   GatherView gather;  // idx == nullptr: keys are not compacted
+  // varlen policy: sequence b holds query rows [cu_q[b], cu_q[b+1]) of the
+  // packed [total_q, H, d] operands (keys likewise); Lq / Lk are the maxima
+  const int32_t* cu_q = nullptr;
+  const int32_t* cu_k = nullptr;
+  int total_q = 0, total_k = 0;
   int* err;  // device error word
 };
 
@@ -141,6 +147,22 @@ cudaError_t launch_mask_tile_summary(const uint8_t* mask, const int64_t sizes[4]
 cudaError_t launch_explicit_lists(const AttnProblem& p, const uint8_t* codes, int codes_q_tiles,
                                   int32_t* num_full, int32_t* full_idx, int32_t* num_part,
                                   int32_t* part_idx, cudaStream_t stream);
+
+// Tile lists of packed sequences: per (sequence, query tile) the key tiles
+// of that sequence, causal (bottom-right per sequence) or not.  Malformed
+// offsets raise SMA_ERR_DEVICE_INPUT and give empty lists.
+cudaError_t launch_varlen_lists(const AttnProblem& p, int32_t* num_full, int32_t* full_idx,
+                                int32_t* num_part, int32_t* part_idx, cudaStream_t stream);
+
+// Packed <-> padded copies of [total, heads, d] rows (pad zero-fills rows past
+// each sequence's length).  esz: element size in bytes.
+cudaError_t launch_varlen_pad(const void* packed, void* padded, const int32_t* cu, int batch,
+                              int max_len, int heads, int d, int esz, int64_t p_row, int64_t p_head,
+                              int64_t d_sb, int64_t d_sr, int64_t d_sh, cudaStream_t stream);
+cudaError_t launch_varlen_unpad(const void* padded, void* packed, const int32_t* cu, int batch,
+                                int max_len, int heads, int d, int esz, int64_t p_row,
+                                int64_t p_head, int64_t s_sb, int64_t s_sr, int64_t s_sh,
+                                cudaStream_t stream);
 
 // tcgen05 forward (bf16 / fp16).  Returns a nonzero SMA status on a host-side
 // failure (tensor map encoding) and writes a message to `msg`.

@@ -1024,4 +1024,135 @@ sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   return ok();
 }
 
+sma_status varlen_attn_fwd_workspace_size(int32_t batch, int32_t max_q, int32_t max_k, size_t* bytes) {
+  if (bytes == nullptr) return fail(SMA_ERR_INVALID_ARG, "bytes is NULL");
+  if (batch < 1 || max_q < 1 || max_k < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, max_q and max_k must be >= 1");
+  *bytes = lists_layout(0, static_cast<int64_t>(batch) * ceil_div(max_q, kTile),
+                        static_cast<int>(ceil_div(max_k, kTile))).end;
+  return ok();
+}
+
+sma_status varlen_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t head_dim, int32_t total_q, int32_t total_k, int32_t max_q,
+                           int32_t max_k, float scale, int32_t is_causal, const int32_t* cu_seqlens_q,
+                           const int32_t* cu_seqlens_k, const void* q, const int64_t q_strides[2],
+                           const void* k, const int64_t k_strides[2], const void* v,
+                           const int64_t v_strides[2], void* out, const int64_t o_strides[2],
+                           float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (dtype == SMA_FP32)
+    return fail(SMA_ERR_UNSUPPORTED, "varlen attention runs on the tensor cores: bf16 or fp16 only");
+  sma_status s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (batch < 1 || total_q < 1 || total_k < 1 || max_q < 1 || max_k < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, totals and maxima must be >= 1");
+  if (is_causal != 0 && is_causal != 1) return fail(SMA_ERR_INVALID_ARG, "is_causal must be 0 or 1");
+  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr)
+    return fail(SMA_ERR_INVALID_ARG, "cu_seqlens_q / cu_seqlens_k are NULL");
+  if (q_strides == nullptr || k_strides == nullptr || v_strides == nullptr || o_strides == nullptr)
+    return fail(SMA_ERR_INVALID_ARG, "strides are NULL");
+  const int64_t qs[3] = {0, q_strides[0], q_strides[1]};
+  const int64_t ks[3] = {0, k_strides[0], k_strides[1]};
+  const int64_t vs[3] = {0, v_strides[0], v_strides[1]};
+  const int64_t os[3] = {0, o_strides[0], o_strides[1]};
+  if ((s = check_operand("q", q, qs, dtype, total_q)) != SMA_OK) return s;
+  if ((s = check_operand("k", k, ks, dtype, total_k)) != SMA_OK) return s;
+  if ((s = check_operand("v", v, vs, dtype, total_k)) != SMA_OK) return s;
+  if ((s = check_operand("out", out, os, dtype, total_q)) != SMA_OK) return s;
+  size_t need = 0;
+  if ((s = varlen_attn_fwd_workspace_size(batch, max_q, max_k, &need)) != SMA_OK) return s;
+  if ((s = check_workspace(workspace, workspace_bytes, need)) != SMA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (err == nullptr) return cuda_fail(e, "device error word unavailable");
+  AttnProblem p{};
+  p.dtype = dtype;
+  p.B = batch; p.H = heads; p.KVH = kv_heads; p.Lq = max_q; p.Lk = max_k; p.d = head_dim;
+  p.group = heads / kv_heads;
+  p.npairs = (p.group + 1) / 2;
+  p.QT = static_cast<int>(ceil_div(max_q, kTile));
+  p.KT = static_cast<int>(ceil_div(max_k, kTile));
+  p.scale_log2 = resolve_scale(scale, head_dim) * kLog2eHost;
+  p.q = q; p.q_sb = 0; p.q_sr = q_strides[0]; p.q_sh = q_strides[1];
+  p.k = k; p.k_sb = 0; p.k_sr = k_strides[0]; p.k_sh = k_strides[1];
+  p.v = v; p.v_sb = 0; p.v_sr = v_strides[0]; p.v_sh = v_strides[1];
+  p.o = out; p.o_sb = 0; p.o_sr = o_strides[0]; p.o_sh = o_strides[1];
+  p.lse = lse;
+  p.policy = kPolicyVarlen;
+  p.causal = is_causal;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.err = err;
+  const ListsLayout lay = lists_layout(0, static_cast<int64_t>(batch) * p.QT, p.KT);
+  p.lists.LB = batch; p.lists.LH = 1; p.lists.head_mode = 0;
+  p.lists.num_full = at<int32_t>(workspace, lay.nf);
+  p.lists.num_part = at<int32_t>(workspace, lay.np);
+  p.lists.full_idx = at<int32_t>(workspace, lay.fi);
+  p.lists.part_idx = at<int32_t>(workspace, lay.pi);
+  e = launch_varlen_lists(p, at<int32_t>(workspace, lay.nf), at<int32_t>(workspace, lay.fi),
+                          at<int32_t>(workspace, lay.np), at<int32_t>(workspace, lay.pi), st);
+  if (e != cudaSuccess) return cuda_fail(e, "tile list launch failed");
+  char msg[256];
+  const int rc = launch_attn_tc(p, st, msg, sizeof(msg));
+  if (rc != SMA_OK) return fail(rc, "%s", msg);
+  return ok();
+}
+
+static sma_status check_pad_args(int32_t dtype, int32_t batch, int32_t max_len, int32_t heads,
+                                 int32_t head_dim, const int32_t* cu, const void* packed,
+                                 const int64_t* p_strides, const void* padded,
+                                 const int64_t* d_strides) {
+  if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (batch < 1 || max_len < 0 || heads < 1 || head_dim < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, heads and head_dim must be >= 1, max_len >= 0");
+  const int es = elem_size(dtype);
+  if ((head_dim * es) % 16 != 0) return fail(SMA_ERR_INVALID_ARG, "rows must be multiples of 16 bytes");
+  if (cu == nullptr || packed == nullptr || padded == nullptr || p_strides == nullptr ||
+      d_strides == nullptr)
+    return fail(SMA_ERR_INVALID_ARG, "NULL argument");
+  if (!aligned16(packed) || !aligned16(padded))
+    return fail(SMA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  for (int i = 0; i < 2; ++i)
+    if (p_strides[i] < 0 || (p_strides[i] * es) % 16 != 0)
+      return fail(SMA_ERR_INVALID_ARG, "packed strides must be non-negative multiples of 16 bytes");
+  for (int i = 0; i < 3; ++i)
+    if (d_strides[i] < 0 || (d_strides[i] * es) % 16 != 0)
+      return fail(SMA_ERR_INVALID_ARG, "padded strides must be non-negative multiples of 16 bytes");
+  return SMA_OK;
+}
+
+sma_status varlen_pad(int32_t dtype, int32_t batch, int32_t max_len, int32_t heads,
+                      int32_t head_dim, const int32_t* cu_seqlens, const void* packed,
+                      const int64_t packed_strides[2], void* padded,
+                      const int64_t padded_strides[3], void* stream) {
+  sma_status s = check_pad_args(dtype, batch, max_len, heads, head_dim, cu_seqlens, packed,
+                                packed_strides, padded, padded_strides);
+  if (s != SMA_OK) return s;
+  cudaError_t e = launch_varlen_pad(packed, padded, cu_seqlens, batch, max_len, heads, head_dim,
+                                    elem_size(dtype), packed_strides[0], packed_strides[1],
+                                    padded_strides[0], padded_strides[1], padded_strides[2],
+                                    static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pad launch failed");
+  return ok();
+}
+
+sma_status varlen_unpad(int32_t dtype, int32_t batch, int32_t max_len, int32_t heads,
+                        int32_t head_dim, const int32_t* cu_seqlens, const void* padded,
+                        const int64_t padded_strides[3], void* packed,
+                        const int64_t packed_strides[2], void* stream) {
+  sma_status s = check_pad_args(dtype, batch, max_len, heads, head_dim, cu_seqlens, packed,
+                                packed_strides, padded, padded_strides);
+  if (s != SMA_OK) return s;
+  cudaError_t e = launch_varlen_unpad(padded, packed, cu_seqlens, batch, max_len, heads, head_dim,
+                                      elem_size(dtype), packed_strides[0], packed_strides[1],
+                                      padded_strides[0], padded_strides[1], padded_strides[2],
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "unpad launch failed");
+  return ok();
+}
+
 }  // extern "C"

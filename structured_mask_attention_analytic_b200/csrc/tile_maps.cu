@@ -270,6 +270,51 @@ cudaError_t launch_mask_tile_summary(const uint8_t* mask, const int64_t sizes[4]
   return cudaGetLastError();
 }
 
+namespace {
+// Lists of packed sequences: list row (b, qt) over the key tiles of sequence
+// b, from its lengths cu[b+1] - cu[b]; causal is bottom-right per sequence.
+__global__ void __launch_bounds__(kMapThreads)
+varlen_lists_kernel(AttnProblem p, int32_t* num_full, int32_t* full_idx, int32_t* num_part,
+                    int32_t* part_idx) {
+  const int qt = blockIdx.x, b = blockIdx.z;
+  int lq = p.cu_q[b + 1] - p.cu_q[b];
+  int lk = p.cu_k[b + 1] - p.cu_k[b];
+  if (lq < 0 || lk < 0 || lq > p.Lq || lk > p.Lk || p.cu_q[b] < 0 || p.cu_k[b] < 0 ||
+      p.cu_q[b + 1] > p.total_q || p.cu_k[b + 1] > p.total_k) {
+    if (threadIdx.x == 0 && qt == 0) report_error(p.err, SMA_ERR_DEVICE_INPUT);
+    lq = 0;
+    lk = 0;
+  }
+  const int q0 = qt * kTile;
+  const int q1 = min(q0 + kTile, lq);
+  const int off = lk - lq;
+  auto code_of = [&](int kt) -> int {
+    const int k0 = kt * kTile;
+    if (q0 >= lq || k0 >= lk) return SMA_TILE_EMPTY;
+    const int k1 = min(k0 + kTile, lk);
+    int c = ((kt + 1) * kTile <= lk) ? SMA_TILE_FULL : SMA_TILE_PARTIAL;
+    if (p.causal) {
+      int cc;
+      if (k1 - 1 <= q0 + off) cc = SMA_TILE_FULL;
+      else if (k0 > (q1 - 1) + off) cc = SMA_TILE_EMPTY;
+      else cc = SMA_TILE_PARTIAL;
+      c = combine_codes(c, cc);
+    }
+    return c;
+  };
+  const int64_t row = static_cast<int64_t>(b) * p.QT + qt;
+  emit_lists(p.KT, code_of, num_full + row, full_idx + row * p.KT, num_part + row,
+             part_idx + row * p.KT);
+}
+}  // namespace
+
+cudaError_t launch_varlen_lists(const AttnProblem& p, int32_t* num_full, int32_t* full_idx,
+                                int32_t* num_part, int32_t* part_idx, cudaStream_t stream) {
+  dim3 grid(p.QT, 1, p.B);
+  varlen_lists_kernel<<<grid, kMapThreads, 0, stream>>>(p, num_full, full_idx, num_part, part_idx);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_explicit_lists(const AttnProblem& p, const uint8_t* codes, int codes_q_tiles,
                                   int32_t* num_full, int32_t* full_idx, int32_t* num_part,
                                   int32_t* part_idx, cudaStream_t stream) {

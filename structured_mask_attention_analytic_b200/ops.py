@@ -390,6 +390,71 @@ def sparse_attn_fwd(q, k, v, mask, bias=None, is_causal: bool = False, scale=Non
     return out, lse
 
 
+def _strides2(t: torch.Tensor):
+    if t.dim() != 3 or t.stride(2) != 1:
+        raise ValueError("packed tensors must be 3D [total, heads, head_dim] with head_dim contiguous")
+    return nat.i64_array(t.stride()[:2])
+
+
+def _cu(t: torch.Tensor, batch=None) -> torch.Tensor:
+    if t.dtype != torch.int32 or t.dim() != 1 or (batch is not None and t.shape[0] != batch + 1):
+        raise ValueError("cu_seqlens must be int32 [batch + 1]")
+    return t.contiguous()
+
+
+def varlen_attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                    is_causal: bool = False, scale=None, out=None, return_lse: bool = True, workspace=None):
+    """Attention over packed variable-length sequences.
+
+    q ``[total_q, H, d]``, k/v ``[total_k, KVH, d]``; sequence b is rows
+    ``cu_seqlens_q[b]:cu_seqlens_q[b+1]`` of q (keys likewise) and attends
+    only its own keys (bottom-right causal per sequence when ``is_causal``).
+    Returns ``(out, lse)``, lse float32 ``[H, total_q]``."""
+    _require_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k)
+    total_q, h, dh = q.shape
+    total_k, kvh = k.shape[0], k.shape[1]
+    b = cu_seqlens_q.shape[0] - 1
+    cq, ck = _cu(cu_seqlens_q), _cu(cu_seqlens_k, b)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k and v must share a dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((h, total_q), dtype=torch.float32, device=q.device) if return_lse else None
+    n = ctypes.c_size_t()
+    nat.check(_lib().varlen_attn_fwd_workspace_size(b, int(max_seqlen_q), int(max_seqlen_k), ctypes.byref(n)))
+    if workspace is None:
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=q.device)
+    nat.check(_lib().varlen_attn_fwd(
+        _dtype_code(q), b, h, kvh, dh, total_q, total_k, int(max_seqlen_q), int(max_seqlen_k),
+        ctypes.c_float(0.0 if scale is None else float(scale)), 1 if is_causal else 0,
+        _ptr(cq), _ptr(ck), _ptr(q), _strides2(q), _ptr(k), _strides2(k), _ptr(v), _strides2(v),
+        _ptr(out), _strides2(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(q)))
+    return out, lse
+
+
+def varlen_pad(packed: torch.Tensor, cu_seqlens: torch.Tensor, max_len: int) -> torch.Tensor:
+    """``[batch, max_len, H, d]`` from packed ``[total, H, d]`` rows (zeros past each length)."""
+    _require_cuda(packed, cu_seqlens)
+    cu = _cu(cu_seqlens)
+    b = cu.shape[0] - 1
+    _, h, dh = packed.shape
+    padded = torch.empty((b, int(max_len), h, dh), dtype=packed.dtype, device=packed.device)
+    nat.check(_lib().varlen_pad(_dtype_code(packed), b, int(max_len), h, dh, _ptr(cu), _ptr(packed),
+                                _strides2(packed), _ptr(padded), _strides3(padded), _stream(packed)))
+    return padded
+
+
+def varlen_unpad(padded: torch.Tensor, cu_seqlens: torch.Tensor, total: int) -> torch.Tensor:
+    """Packed ``[total, H, d]`` rows from ``[batch, max_len, H, d]``."""
+    _require_cuda(padded, cu_seqlens)
+    cu = _cu(cu_seqlens, padded.shape[0])
+    b, max_len, h, dh = padded.shape
+    packed = torch.empty((int(total), h, dh), dtype=padded.dtype, device=padded.device)
+    nat.check(_lib().varlen_unpad(_dtype_code(padded), b, max_len, h, dh, _ptr(cu), _ptr(padded),
+                                  _strides3(padded), _ptr(packed), _strides2(packed), _stream(padded)))
+    return packed
+
+
 def _pre_mask_view(pre_mask: torch.Tensor, batch: int, q_len: int, k_len: int):
     """create_mask's shape step as a view: a 2D (batch, L) pre-mask becomes
     sizes (batch, 1, 1, L); columns >= L count as invalid, which equals

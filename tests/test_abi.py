@@ -212,3 +212,26 @@ def test_backward_workspace_and_validation_on_host():
     assert "lse" in lib.sma_last_error().decode()
     assert call(dbias=0xb0000) == nat.SMA_ERR_UNSUPPORTED
     assert "dbias" in lib.sma_last_error().decode()
+
+
+def test_varlen_validation_on_host():
+    lib = nat.load()
+    n = ctypes.c_size_t()
+    assert lib.varlen_attn_fwd_workspace_size(4, 1000, 2000, ctypes.byref(n)) == 0
+    assert n.value >= 2 * 4 * 8 * 16 * 4          # full and partial index arrays
+    st = lib.varlen_attn_fwd(2, 2, 4, 2, 128, 100, 100, 60, 60, ctypes.c_float(0.0), 0,
+                             ctypes.c_void_p(0x100), ctypes.c_void_p(0x200),
+                             ctypes.c_void_p(0x10000), nat.i64_array([512, 128]),
+                             ctypes.c_void_p(0x20000), nat.i64_array([256, 128]),
+                             ctypes.c_void_p(0x30000), nat.i64_array([256, 128]),
+                             ctypes.c_void_p(0x40000), nat.i64_array([512, 128]), None,
+                             ctypes.c_void_p(0x50000), 1 << 20, None)
+    assert st == nat.SMA_ERR_UNSUPPORTED
+    st = lib.varlen_attn_fwd(0, 2, 4, 2, 128, 100, 100, 60, 60, ctypes.c_float(0.0), 0,
+                             ctypes.c_void_p(0), ctypes.c_void_p(0x200),
+                             ctypes.c_void_p(0x10000), nat.i64_array([512, 128]),
+                             ctypes.c_void_p(0x20000), nat.i64_array([256, 128]),
+                             ctypes.c_void_p(0x30000), nat.i64_array([256, 128]),
+                             ctypes.c_void_p(0x40000), nat.i64_array([512, 128]), None,
+                             ctypes.c_void_p(0x50000), 1 << 20, None)
+    assert st == nat.SMA_ERR_INVALID_ARG and "cu_seqlens" in lib.sma_last_error().decode()

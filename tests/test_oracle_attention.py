@@ -225,3 +225,28 @@ def test_threaded_equals_serial(qkv):
     o2, l2 = at.attention(q, k, v, row_chunk=8, workers=4)
     np.testing.assert_array_equal(o1, o2)
     np.testing.assert_array_equal(l1, l2)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_equals_block_diagonal_mask(causal):
+    """Packed sequences equal one problem over the packed rows with a
+    block-diagonal keep mask (causal bottom-right inside each block)."""
+    rng = np.random.default_rng(21)
+    lq, lk = [3, 0, 5, 1, 4], [4, 2, 5, 0, 2]
+    cu_q, cu_k = np.cumsum([0] + lq), np.cumsum([0] + lk)
+    H, KVH, D = 4, 2, 3
+    q = rng.standard_normal((cu_q[-1], H, D))
+    k = rng.standard_normal((cu_k[-1], KVH, D))
+    v = rng.standard_normal((cu_k[-1], KVH, D))
+    out, lse = at.varlen_attention(q, k, v, cu_q, cu_k, causal)
+    keep = np.zeros((cu_q[-1], cu_k[-1]), bool)
+    for b in range(len(lq)):
+        blk = np.ones((lq[b], lk[b]), bool)
+        if causal:
+            blk = at.causal_keep(lq[b], lk[b])
+        keep[cu_q[b]:cu_q[b + 1], cu_k[b]:cu_k[b + 1]] = blk
+    ref, ref_lse = at.attention(q[None], k[None], v[None], keep=keep[None, None])
+    np.testing.assert_allclose(out, ref[0], atol=1e-13)
+    np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(ref_lse[0]))
+    fin = ~np.isneginf(lse)
+    np.testing.assert_allclose(lse[fin], ref_lse[0][fin], atol=1e-13)
