@@ -161,9 +161,12 @@ typedef struct dfa_block_map_ptrs {
   const int32_t* part_idx;
 } dfa_block_map_ptrs;
 
-/* Workspace bytes dfa_attn_fwd needs for this problem when it computes the
- * block map itself (0 is enough when a precomputed map is passed).  The
- * caller allocates it; it may be reused across calls ordered on one stream. */
+/* Workspace bytes dfa_attn_fwd uses for this problem: the block map (when
+ * the call computes it) and, for problems with too few (batch, KV head, head
+ * pair, 128-query tile) units to fill the SMs, the partial results of the
+ * key-range split (per segment and query row: fp32 O and the running max and
+ * sum).  The caller allocates it; it may be reused across calls ordered on
+ * one stream. */
 sma_status dfa_attn_fwd_workspace_size(const dfa_mask_desc* desc, int32_t heads, int32_t kv_heads,
                                        int32_t head_dim, size_t* bytes);
 
@@ -173,6 +176,14 @@ sma_status dfa_attn_fwd_workspace_size(const dfa_mask_desc* desc, int32_t heads,
  *            kernel).  Otherwise a map from dfa_block_map for the same desc
  *            and anchors, e.g. shared by the layers of one training step;
  *            `workspace` may then be NULL with 0 bytes.
+ * workspace  at least the block map's bytes when block_map is NULL
+ *            (SMA_ERR_WORKSPACE otherwise).  Short-query problems (e.g. one
+ *            draft block after a long context) cut each unit's key tiles
+ *            into contiguous segments run on separate SMs and merge the
+ *            segments' partial results in a second kernel; they do so only
+ *            when `workspace` holds dfa_attn_fwd_workspace_size bytes.  The
+ *            split changes the fp32 summation order, not the result beyond
+ *            rounding.
  * q    [batch, q_len, heads, head_dim]     strides q_strides (batch, row, head)
  * k, v [batch, k_len, kv_heads, head_dim]  strides k_strides / v_strides
  * out  [batch, q_len, heads, head_dim]     strides o_strides; same dtype as q
@@ -237,8 +248,10 @@ sma_status mask_tile_summary(const uint8_t* mask, const int64_t mask_sizes[4],
                              const int64_t mask_strides[4], int32_t k_len, uint8_t* codes,
                              void* stream);
 
-/* Workspace bytes masked_attn_fwd needs (tile summary, tile lists and the
- * split-KV partials of the single-query path).  mask_sizes may be NULL when
+/* Workspace bytes masked_attn_fwd needs (tile summary, tile lists, the
+ * split-KV partials of the single-query path, and for other short-query
+ * problems the partials of the key-range split: each unit's key tiles cut
+ * into segments run on separate SMs, merged by a second kernel).  mask_sizes may be NULL when
  * no mask will be passed. */
 sma_status masked_attn_fwd_workspace_size(int32_t batch, int32_t heads, int32_t kv_heads,
                                           int32_t q_len, int32_t k_len, int32_t head_dim,
@@ -333,9 +346,18 @@ sma_status masked_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t 
                                           const int64_t mask_sizes[4], size_t* bytes);
 
 /* mask / bias / is_causal / scale exactly as given to masked_attn_fwd (any
- * q_len; single-query problems run the general kernel).  dbias must be NULL:
- * the broadcast-reduced bias gradient of PR #190 is not produced by this
- * build (SMA_ERR_UNSUPPORTED otherwise). */
+ * q_len; single-query problems run the general kernel).
+ *
+ * dbias (nullable; device, 16-byte aligned, caller-owned): the bias gradient
+ * of PR #190 (Changes, mha_bwd), written as contiguous float32 with the
+ * bias's own sizes (b', h', q', round_up(k_len, 128)).  Element (b, h, q, k)
+ * of dS = P * (dP - D) (the gradient of the score, bias included) is summed
+ * into the dbias element its bias element broadcast from: over the batch
+ * when b' = 1, over the heads of a group when h' = kv_heads, over all heads
+ * when h' = 1, over the queries when q' = 1.  Columns >= k_len come out 0.
+ * The call zeroes dbias first; sums over broadcast dims use fp32 atomic
+ * adds, so their rounding order is not fixed.  Needs a bias (
+ * SMA_ERR_INVALID_ARG otherwise). */
 sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
                            int32_t q_len, int32_t k_len, int32_t head_dim, float scale,
                            int32_t is_causal, const void* q, const int64_t q_strides[3],
@@ -420,8 +442,9 @@ sma_status varlen_unpad(int32_t dtype, int32_t batch, int32_t max_len, int32_t h
  *           first max_keys and raises SMA_ERR_DEVICE_INPUT in the device
  *           error word (read with sma_device_status).
  * dtype     SMA_BF16 / SMA_FP16 (tensor cores) or SMA_FP32 (FFMA).
- * Other arguments as masked_attn_fwd; all q_len >= 1 run the prefill kernel.
- * A row that keeps no key gives out = 0 and lse = -inf. */
+ * Other arguments as masked_attn_fwd; all q_len >= 1 run the prefill kernel
+ * (with the key-range split over the compacted key tiles when too few units
+ * fill the SMs).  A row that keeps no key gives out = 0 and lse = -inf. */
 sma_status sparse_attn_fwd_workspace_size(int32_t dtype, int32_t batch, int32_t heads,
                                           int32_t kv_heads, int32_t q_len, int32_t k_len,
                                           int32_t head_dim, const int64_t mask_sizes[4],

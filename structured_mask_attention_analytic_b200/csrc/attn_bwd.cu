@@ -557,30 +557,75 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           break;
         }
         tc_fence_after();
+        // dbias: this thread's query row of dS over the tile's 128 keys
+        float* dbrow = nullptr;
+        if (POLICY != kPolicyDflash && p.db_mode != kDbiasNone)
+          dbrow = p.dbias + w.b * p.db_sb + (p.db_head_per_query ? h : w.hk) * p.db_sh +
+                  static_cast<int64_t>(row_valid ? q : 0) * p.db_sq + k0;
+        auto phase_b = [&](auto mode_tag) {
+          constexpr int MODE = decltype(mode_tag)::value;
 #pragma unroll
-        for (int c = 0; c < kTile / 32; ++c) {
-          uint32_t yr[32];
-          tmem_ld32_at(dp_col + 32 * c, yr);
-          tc_wait_ld();
-          uint32_t pk[16];
+          for (int c = 0; c < kTile / 32; ++c) {
+            uint32_t yr[32];
+            tmem_ld32_at(dp_col + 32 * c, yr);
+            tc_wait_ld();
+            uint32_t pk[16];
+            float dsv[32];
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            const uint4 pp = ld_shared_v4(sw128_unit(sbase + L::kP, r, 4 * c + v4));
-            const uint32_t pw4[4] = {pp.x, pp.y, pp.z, pp.w};
+            for (int v4 = 0; v4 < 4; ++v4) {
+              const uint4 pp = ld_shared_v4(sw128_unit(sbase + L::kP, r, 4 * c + v4));
+              const uint32_t pw4[4] = {pp.x, pp.y, pp.z, pp.w};
 #pragma unroll
-            for (int z = 0; z < 4; ++z) {
-              const int e = 8 * v4 + 2 * z;
-              const float2 pf = unpack2<DT>(pw4[z]);
-              const float d0 = pf.x * (__uint_as_float(yr[e]) - drow);
-              const float d1 = pf.y * (__uint_as_float(yr[e + 1]) - drow);
-              pk[4 * v4 + z] = DT == SMA_BF16 ? pack_bf16x2(d0, d1) : pack_f16x2(d0, d1);
+              for (int z = 0; z < 4; ++z) {
+                const int e = 8 * v4 + 2 * z;
+                const float2 pf = unpack2<DT>(pw4[z]);
+                const float d0 = pf.x * (__uint_as_float(yr[e]) - drow);
+                const float d1 = pf.y * (__uint_as_float(yr[e + 1]) - drow);
+                pk[4 * v4 + z] = DT == SMA_BF16 ? pack_bf16x2(d0, d1) : pack_f16x2(d0, d1);
+                dsv[e] = d0;
+                dsv[e + 1] = d1;
+              }
+            }
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              st_shared_v4(sw128_unit(sbase + L::kDS, r, 4 * c + v4), pk[4 * v4], pk[4 * v4 + 1],
+                           pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            if (MODE == kDbiasStore || MODE == kDbiasAdd) {
+              if (row_valid) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const float4 v =
+                      make_float4(dsv[4 * j], dsv[4 * j + 1], dsv[4 * j + 2], dsv[4 * j + 3]);
+                  float4* dst = reinterpret_cast<float4*>(dbrow + 32 * c + 4 * j);
+                  if (MODE == kDbiasStore) *dst = v;
+                  else atomicAdd(dst, v);
+                }
+              }
+            } else if (MODE == kDbiasRowSum) {
+              // Column sums over the warp's 32 query rows (rows past Lq hold
+              // 0): halving exchanges, after which lane l holds column l.
+#pragma unroll
+              for (int wd = 16; wd >= 1; wd >>= 1) {
+                const bool upper = (lane & wd) != 0;
+#pragma unroll
+                for (int i = 0; i < wd; ++i) {
+                  const float send = upper ? dsv[i] : dsv[i + wd];
+                  const float keep = upper ? dsv[i + wd] : dsv[i];
+                  dsv[i] = keep + __shfl_xor_sync(0xffffffffu, send, wd);
+                }
+              }
+              atomicAdd(dbrow + 32 * c + lane, dsv[0]);
             }
           }
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            st_shared_v4(sw128_unit(sbase + L::kDS, r, 4 * c + v4), pk[4 * v4], pk[4 * v4 + 1],
-                         pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        }
+        };
+        if (POLICY == kPolicyDflash || p.db_mode == kDbiasNone)
+          phase_b(std::integral_constant<int, kDbiasNone>{});
+        else if (p.db_mode == kDbiasStore)
+          phase_b(std::integral_constant<int, kDbiasStore>{});
+        else if (p.db_mode == kDbiasAdd)
+          phase_b(std::integral_constant<int, kDbiasAdd>{});
+        else
+          phase_b(std::integral_constant<int, kDbiasRowSum>{});
         fence_async_shared();
         tc_fence_before();
         mbar_arrive(bar(L::kDSDone));
@@ -1235,31 +1280,62 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           break;
         }
         tc_fence_after();
+        // dbias: this thread's key column of dS over its 64 queries, added
+        // where the bias broadcasts (or stored where each element is its own)
+        float* dbcol = nullptr;
+        if (POLICY != kPolicyDflash && p.db_mode != kDbiasNone)
+          dbcol = p.dbias + w.b * p.db_sb + (p.db_head_per_query ? h : w.hk) * p.db_sh + key;
+        auto phase_b = [&](auto mode_tag) {
+          constexpr int MODE = decltype(mode_tag)::value;
+          float rsum = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          const int cq = qb + 32 * c;
-          uint32_t yr[32], pr[16];
-          tmem_ld32_at(ycol + cq, yr);
-          tmem_ld16_at(xcol + pcol(cq), pr);
-          tc_wait_ld();
-          uint32_t pk[16];
+          for (int c = 0; c < 2; ++c) {
+            const int cq = qb + 32 * c;
+            uint32_t yr[32], pr[16];
+            tmem_ld32_at(ycol + cq, yr);
+            tmem_ld16_at(xcol + pcol(cq), pr);
+            tc_wait_ld();
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 d4 = *reinterpret_cast<const float4*>(dd + cq + e);
-            const float2 p01 = unpack2<DT>(pr[e >> 1]);
-            const float2 p23 = unpack2<DT>(pr[(e >> 1) + 1]);
-            const float s0 = p01.x * (__uint_as_float(yr[e]) - d4.x);
-            const float s1 = p01.y * (__uint_as_float(yr[e + 1]) - d4.y);
-            const float s2 = p23.x * (__uint_as_float(yr[e + 2]) - d4.z);
-            const float s3 = p23.y * (__uint_as_float(yr[e + 3]) - d4.w);
-            pk[e >> 1] = DT == SMA_BF16 ? pack_bf16x2(s0, s1) : pack_f16x2(s0, s1);
-            pk[(e >> 1) + 1] = DT == SMA_BF16 ? pack_bf16x2(s2, s3) : pack_f16x2(s2, s3);
+            for (int e = 0; e < 32; e += 4) {
+              const float4 d4 = *reinterpret_cast<const float4*>(dd + cq + e);
+              const float2 p01 = unpack2<DT>(pr[e >> 1]);
+              const float2 p23 = unpack2<DT>(pr[(e >> 1) + 1]);
+              const float s0 = p01.x * (__uint_as_float(yr[e]) - d4.x);
+              const float s1 = p01.y * (__uint_as_float(yr[e + 1]) - d4.y);
+              const float s2 = p23.x * (__uint_as_float(yr[e + 2]) - d4.z);
+              const float s3 = p23.y * (__uint_as_float(yr[e + 3]) - d4.w);
+              pk[e >> 1] = DT == SMA_BF16 ? pack_bf16x2(s0, s1) : pack_f16x2(s0, s1);
+              pk[(e >> 1) + 1] = DT == SMA_BF16 ? pack_bf16x2(s2, s3) : pack_f16x2(s2, s3);
+              if (MODE == kDbiasRowSum) {
+                rsum += (s0 + s1) + (s2 + s3);  // rows past Lq have P = 0, so dS = 0
+              } else if (MODE != kDbiasNone) {
+                const float sv[4] = {s0, s1, s2, s3};
+#pragma unroll
+                for (int z = 0; z < 4; ++z) {
+                  const int q = q0 + cq + e + z;
+                  if (q < p.f.Lq) {
+                    if (MODE == kDbiasStore) dbcol[q * p.db_sq] = sv[z];
+                    else atomicAdd(dbcol + q * p.db_sq, sv[z]);
+                  }
+                }
+              }
+            }
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              st_shared_v4(sw128_unit(sbase + L::kDS, r, cq / 8 + v4), pk[4 * v4], pk[4 * v4 + 1],
+                           pk[4 * v4 + 2], pk[4 * v4 + 3]);
           }
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            st_shared_v4(sw128_unit(sbase + L::kDS, r, cq / 8 + v4), pk[4 * v4], pk[4 * v4 + 1],
-                         pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        }
+          if (MODE == kDbiasRowSum) atomicAdd(dbcol, rsum);
+        };
+        if (POLICY == kPolicyDflash || p.db_mode == kDbiasNone)
+          phase_b(std::integral_constant<int, kDbiasNone>{});
+        else if (p.db_mode == kDbiasStore)
+          phase_b(std::integral_constant<int, kDbiasStore>{});
+        else if (p.db_mode == kDbiasAdd)
+          phase_b(std::integral_constant<int, kDbiasAdd>{});
+        else
+          phase_b(std::integral_constant<int, kDbiasRowSum>{});
         fence_async_shared();
         tc_fence_before();
         mbar_arrive(bar(L::kDSDone));

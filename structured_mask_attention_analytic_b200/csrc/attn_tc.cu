@@ -91,23 +91,53 @@ struct Layout {
 
 struct Unit {
   int b, hk, pair, qt, h0, h1valid;
+  int q0, q1off, h1off;  // first query of tile 0; tile 1's query and head offsets
   int64_t list_row;
   int n_full, n_part;
+  int split, j0, n;          // key-range segment: list entries [j0, j0 + n)
   int q_off, k_off, lq, lk;  // varlen: the sequence's first rows and lengths
 };
 
 template <int POLICY>
 __device__ __forceinline__ Unit decode_unit(const AttnProblem& p, int u) {
   Unit w;
-  const int per_qt = p.B * p.KVH * p.npairs;
-  w.qt = p.QT - 1 - u / per_qt;  // later query tiles first: they see the most keys
-  int r = u % per_qt;
-  w.pair = r % p.npairs;
-  r /= p.npairs;
-  w.hk = r % p.KVH;
-  w.b = r / p.KVH;
-  w.h0 = w.hk * p.group + 2 * w.pair;
-  w.h1valid = (2 * w.pair + 1) < p.group;
+  // the segments of one unit are adjacent unit indices (adjacent CTAs);
+  // packed sequences use neither the key-range split nor head packing
+  constexpr bool kSplitPack = POLICY != kPolicyVarlen;
+  w.split = kSplitPack ? u % p.n_split : 0;
+  if (kSplitPack) u /= p.n_split;
+  if (kSplitPack && p.pack > 1) {
+    // head-packed tiles: tile i of the unit holds every head of the group
+    // for queries [q0 + i * q1off, + 128 / pack); both blocks lie in one
+    // 128-query tile, whose key-tile list they share
+    const int rows = kTile / p.pack;
+    const int qblocks = (p.Lq + rows - 1) / rows;
+    const int per = p.B * p.KVH;
+    const int pi = (qblocks + 1) / 2 - 1 - u / per;
+    const int r = u % per;
+    w.hk = r % p.KVH;
+    w.b = r / p.KVH;
+    w.pair = 0;
+    w.h0 = w.hk * p.group;
+    w.q0 = 2 * pi * rows;
+    w.q1off = rows;
+    w.h1off = 0;
+    w.h1valid = w.q0 + rows < p.Lq;
+    w.qt = w.q0 / kTile;
+  } else {
+    const int per_qt = p.B * p.KVH * p.npairs;
+    w.qt = p.QT - 1 - u / per_qt;  // later query tiles first: they see the most keys
+    int r = u % per_qt;
+    w.pair = r % p.npairs;
+    r /= p.npairs;
+    w.hk = r % p.KVH;
+    w.b = r / p.KVH;
+    w.h0 = w.hk * p.group + 2 * w.pair;
+    w.h1valid = (2 * w.pair + 1) < p.group;
+    w.q0 = w.qt * kTile;
+    w.q1off = 0;
+    w.h1off = 1;
+  }
   const int lb = p.lists.LB > 1 ? w.b : 0;
   int lh = 0;
   if (p.lists.head_mode == 1) lh = w.hk;
@@ -133,10 +163,17 @@ __device__ __forceinline__ Unit decode_unit(const AttnProblem& p, int u) {
     w.lq = p.Lq;
     w.lk = p.Lk;
   }
+  const int nt = w.n_full + w.n_part;
+  const int ns = kSplitPack ? p.n_split : 1;
+  const int seg = (nt + ns - 1) / ns;
+  w.j0 = w.split * seg;
+  w.n = max(0, min(seg, nt - w.j0));
   return w;
 }
 
+// Key tile of the segment's j-th entry (FULL entries precede PARTIAL ones).
 __device__ __forceinline__ int tile_at(const AttnProblem& p, const Unit& w, int j, bool* partial) {
+  j += w.j0;
   if (j < w.n_full) {
     *partial = false;
     return p.lists.full_idx[w.list_row * p.KT + j];
@@ -214,7 +251,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit w = decode_unit<POLICY>(p, u);
-      const int n = w.n_full + w.n_part;
+      const int n = w.n;
       if (n == 0) continue;
       if (q_it > 0 && !mbar_wait_warp(bar(L::kQEmpty), (q_it - 1) & 1, abort_flag, p.err)) {
         ok = false;
@@ -225,8 +262,8 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
         for (int i = 0; i < 1 + w.h1valid; ++i)
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sbase + L::kQ + i * L::kTileBytes + c * L::kChunkBytes, &map_q,
-                        bar(L::kQFull), c * 64, w.h0 + i, w.q_off + w.qt * kTile,
-                        POLICY == kPolicyVarlen ? 0 : w.b);
+                        bar(L::kQFull), c * 64, w.h0 + i * w.h1off,
+                        w.q_off + w.q0 + i * w.q1off, POLICY == kPolicyVarlen ? 0 : w.b);
       }
       __syncwarp();
       ++q_it;
@@ -336,7 +373,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
     };
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit w = decode_unit<POLICY>(p, u);
-      const int n = w.n_full + w.n_part;
+      const int n = w.n;
       const int nq = 1 + w.h1valid;
       if (n > 0) {
         if (!mbar_wait_warp(bar(L::kQFull), q_it & 1, abort_flag, p.err)) { ok = false; break; }
@@ -440,10 +477,17 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit w = decode_unit<POLICY>(p, u);
       if (qi == 1 && !w.h1valid) continue;
-      const int h = w.h0 + qi;
-      const int q = w.qt * kTile + r;
+      const int qfirst = w.q0 + qi * w.q1off;  // first query of this tile
+      int h, q;
+      if (POLICY != kPolicyVarlen && p.pack > 1) {  // row r: head r % pack of query r / pack
+        h = w.h0 + (r & (p.pack - 1));
+        q = qfirst + (r >> (__ffs(p.pack) - 1));
+      } else {
+        h = w.h0 + qi;
+        q = qfirst + r;
+      }
       const bool row_valid = q < w.lq;
-      const int n = w.n_full + w.n_part;
+      const int n = w.n;
 
       // Per-row mask parameters.
       int clo = 0, chi = 0, dlo = 0, dhi = 0;  // DFlash keep intervals
@@ -558,7 +602,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
             // are checked only on tiles they can cut (uniform per tile).
             int lim = kTile;
             if (k0 + kTile > w.lk) lim = min(lim, w.lk - k0);
-            if (p.causal && k0 + kTile - 1 > w.qt * kTile + causal_off)
+            if (p.causal && k0 + kTile - 1 > qfirst + causal_off)
               lim = min(lim, causal_lim - k0 + 1);
             if (mask_bcast_q) {
               // One mask row for every query row: 4 ballots turn the tile's 128
@@ -671,6 +715,11 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
                    static_cast<int64_t>(w.q_off + q) * p.o_sr +
                    h * p.o_sh;
       const float inv_l = l_sum > 0.f ? 1.0f / l_sum : 0.f;
+      // Key-range segment: unnormalised O and (max, sum) go to the partials.
+      const bool seg_out = POLICY != kPolicyVarlen && p.n_split > 1;
+      const int64_t prow =
+          (static_cast<int64_t>(w.split) * p.part_rows + (static_cast<int64_t>(w.b) * p.H + h) * p.Lq +
+           q);
       if (n > 0) {
         if (!mbar_wait(bar(L::kOBar + qi), (it - 1) & 1, abort_flag, p.err)) ok = false;
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -680,7 +729,14 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           uint32_t o[32];
           tmem_ld32(o_col + 32 * c, o);
           tc_wait_ld();
-          if (row_valid) {
+          if (seg_out) {
+            if (row_valid) {
+              uint4* dst = reinterpret_cast<uint4*>(p.part_o + prow * D + 32 * c);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+            }
+          } else if (row_valid) {
             uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -694,11 +750,15 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
               dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
           }
         }
-      } else if (row_valid) {
+      } else if (row_valid && !seg_out) {
         uint4* dst = reinterpret_cast<uint4*>(orow);
         for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
       }
-      if (row_valid && p.lse != nullptr) {
+      if (seg_out) {
+        if (row_valid)
+          *reinterpret_cast<float2*>(p.part_ml + 2 * prow) =
+              make_float2(l_sum > 0.f ? m_ref : -INFINITY, l_sum);
+      } else if (row_valid && p.lse != nullptr) {
         p.lse[POLICY == kPolicyVarlen ? static_cast<int64_t>(h) * p.total_q + w.q_off + q
                                       : (static_cast<int64_t>(w.b) * p.H + h) * p.Lq + q] =
             l_sum > 0.f ? (m_ref + __log2f(l_sum)) * kLn2 : -INFINITY;
@@ -712,6 +772,68 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+// Merge of the key-range segments.  Segment s holds, per row, O_s = sum of
+// 2^(t - m_s) V over its keys (t = log2-domain score) and l_s = sum of
+// 2^(t - m_s); with M = max m_s over the segments that kept a key,
+//   O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,
+//   lse = ln 2 * (M + log2 sum_s 2^(m_s - M) l_s).
+// One warp per row, each lane D / 32 consecutive columns.
+template <int D, int DT>
+__global__ void __launch_bounds__(256) attn_combine_kernel(const AttnProblem p) {
+  typedef typename std::conditional<DT == SMA_BF16, __nv_bfloat16, __half>::type OutT;
+  constexpr int kPer = D / 32;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= p.part_rows) return;
+  const float2* ml = reinterpret_cast<const float2*>(p.part_ml);
+  float mx = -INFINITY;
+  for (int s = lane; s < p.n_split; s += 32) {
+    const float2 v = ml[static_cast<int64_t>(s) * p.part_rows + row];
+    if (v.y > 0.f) mx = fmaxf(mx, v.x);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float l = 0.f;
+  for (int s = 0; s < p.n_split; ++s) {
+    const int64_t sr = static_cast<int64_t>(s) * p.part_rows + row;
+    const float2 v = ml[sr];
+    if (!(v.y > 0.f)) continue;  // no kept key in this segment: O_s was not written
+    const float wgt = fast_exp2(v.x - mx);
+    l = fmaf(wgt, v.y, l);
+    const float* src = p.part_o + sr * D + lane * kPer;
+    if (kPer == 4) {
+      const float4 a = *reinterpret_cast<const float4*>(src);
+      acc[0] = fmaf(wgt, a.x, acc[0]);
+      acc[1] = fmaf(wgt, a.y, acc[1]);
+      acc[2] = fmaf(wgt, a.z, acc[2]);
+      acc[3] = fmaf(wgt, a.w, acc[3]);
+    } else {
+      const float2 a = *reinterpret_cast<const float2*>(src);
+      acc[0] = fmaf(wgt, a.x, acc[0]);
+      acc[1] = fmaf(wgt, a.y, acc[1]);
+    }
+  }
+  const float inv = l > 0.f ? 1.0f / l : 0.f;
+  const int q = static_cast<int>(row % p.Lq);
+  const int64_t bh = row / p.Lq;
+  const int h = static_cast<int>(bh % p.H);
+  const int b = static_cast<int>(bh / p.H);
+  OutT* orow = reinterpret_cast<OutT*>(p.o) + b * p.o_sb + static_cast<int64_t>(q) * p.o_sr +
+               h * p.o_sh + lane * kPer;
+  uint32_t pk[kPer / 2];
+#pragma unroll
+  for (int e = 0; e < kPer / 2; ++e)
+    pk[e] = DT == SMA_BF16 ? pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv)
+                           : pack_f16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+  if (kPer == 4) *reinterpret_cast<uint2*>(orow) = make_uint2(pk[0], pk[1]);
+  else *reinterpret_cast<uint32_t*>(orow) = pk[0];
+  if (lane == 0 && p.lse != nullptr)
+    p.lse[row] = l > 0.f ? (mx + __log2f(l)) * kLn2 : -INFINITY;
 }
 
 // ------------------------------------------------------------------ host side
@@ -733,21 +855,26 @@ cudaError_t launch_typed(const AttnProblem& p, const CUtensorMap& mq, const CUte
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int n_units = p.B * p.KVH * p.npairs * p.QT;
+  const int n_units =
+      static_cast<int>(fwd_units(p.B, p.KVH, p.npairs, p.QT, p.Lq, p.pack)) * p.n_split;
   if (n_units == 0) return cudaSuccess;
   const int grid = n_units < num_sms() ? n_units : num_sms();
   kern<<<grid, kThreads, L::kAlloc, stream>>>(p, mq, mk, mv, n_units);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || p.n_split == 1) return e;
+  const int64_t blocks = (p.part_rows + 7) / 8;
+  attn_combine_kernel<D, DT><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
-}  // namespace
-
-int launch_attn_tc(const AttnProblem& p, cudaStream_t stream, char* msg, size_t msg_len) {
+// Tensor maps and the typed launch of one problem (pack already set).
+int launch_problem(const AttnProblem& p, cudaStream_t stream, char* msg, size_t msg_len) {
   CUtensorMap mq, mk, mv;
   // packed sequences: one batch entry of total_q (total_k) rows
   const bool packed = p.policy == kPolicyVarlen;
   const int lq = packed ? p.total_q : p.Lq, lk = packed ? p.total_k : p.Lk, nb = packed ? 1 : p.B;
-  if (!encode_map(&mq, p.q, p.dtype, p.d, p.H, lq, nb, p.q_sh, p.q_sr, p.q_sb, msg, msg_len) ||
+  if (!encode_map(&mq, p.q, p.dtype, p.d, p.H, lq, nb, p.q_sh, p.q_sr, p.q_sb, msg, msg_len,
+                  p.pack) ||
       !encode_map(&mk, p.k, p.dtype, p.d, p.KVH, lk, nb, p.k_sh, p.k_sr, p.k_sb, msg, msg_len) ||
       !encode_map(&mv, p.v, p.dtype, p.d, p.KVH, lk, nb, p.v_sh, p.v_sr, p.v_sb, msg, msg_len))
     return SMA_ERR_CUDA;
@@ -779,6 +906,20 @@ int launch_attn_tc(const AttnProblem& p, cudaStream_t stream, char* msg, size_t 
     return SMA_ERR_CUDA;
   }
   return SMA_OK;
+}
+
+}  // namespace
+
+int launch_attn_tc(const AttnProblem& p, cudaStream_t stream, char* msg, size_t msg_len) {
+  if (p.n_split < 1 || (p.n_split > 1 && (p.policy == kPolicyVarlen || p.part_o == nullptr ||
+                                          p.part_ml == nullptr ||
+                                          p.part_rows != static_cast<int64_t>(p.B) * p.H * p.Lq))) {
+    snprintf(msg, msg_len, "invalid key-range split");
+    return SMA_ERR_INVALID_ARG;
+  }
+  AttnProblem pp = p;
+  pp.pack = fwd_pack(p.Lq, p.group, p.lists.head_mode, p.policy);
+  return launch_problem(pp, stream, msg, msg_len);
 }
 
 }  // namespace sma

@@ -85,8 +85,41 @@ struct AttnProblem {
   const int32_t* cu_q = nullptr;
   const int32_t* cu_k = nullptr;
   int total_q = 0, total_k = 0;
+  // Key-range split (tcgen05 path, not varlen): each unit's key-tile list is
+  // cut into n_split contiguous segments run as separate units.  Segment s
+  // writes its rows' unnormalised O to part_o[s][row] and (running max in
+  // log2 units, sum of exponentials) to part_ml[s][row]; a combine kernel
+  // merges them into o and lse.  row = (b * H + h) * Lq + q, part_rows =
+  // B * H * Lq.
+  int n_split = 1;
+  float* part_o = nullptr;   // [n_split, part_rows, d]
+  float* part_ml = nullptr;  // [n_split, part_rows, 2]
+  int64_t part_rows = 0;
+  // Head packing (tcgen05 path; set by the launcher, see fwd_pack): with
+  // pack = P > 1 a 128-row tile holds the P query heads of a KV head for
+  // 128 / P consecutive queries (row r: head r % P, query r / P).
+  int pack = 1;
   int* err;  // device error word
 };
+
+// Query heads per 128-row tile of the tcgen05 forward: the whole group when
+// the queries are few (<= 64, so a head-per-tile layout would leave most rows
+// empty), the group has 2, 4 or 8 heads and the tile lists are shared by the
+// group's heads; 1 otherwise.
+inline int fwd_pack(int Lq, int group, int head_mode, int policy) {
+  if (policy == kPolicyVarlen || head_mode == 2 || Lq > 64) return 1;
+  return (group == 2 || group == 4 || group == 8) ? group : 1;
+}
+
+// Units of the tcgen05 forward before any key-range split: (batch, KV head,
+// pair of query heads, 128-query tile), or with head packing (batch, KV head,
+// pair of 128 / pack-query blocks).
+inline int64_t fwd_units(int B, int KVH, int npairs, int QT, int Lq, int pack) {
+  if (pack == 1) return static_cast<int64_t>(B) * KVH * npairs * QT;
+  const int rows = kTile / pack;
+  const int qblocks = (Lq + rows - 1) / rows;
+  return static_cast<int64_t>(B) * KVH * ((qblocks + 1) / 2);
+}
 
 // Backward of one attention problem.  `f` is the forward problem (q, k, v,
 // geometry, policy, masks and the forward tile lists, f.o = the forward
@@ -103,7 +136,21 @@ struct BwdProblem {
   const int32_t* t_num_full; const int32_t* t_full;  // [rows, KT], [rows, KT, QT]
   const int32_t* t_num_part; const int32_t* t_part;
   float scale;     // softmax scale (dQ and dK carry it)
+  // Gradient of the bias (explicit policy only): fp32, the bias's broadcast
+  // shape (b', h', q', 128-rounded Lk), zeroed before the kernel runs; element
+  // (b, h, q, k) of dS adds into dbias[b * db_sb + hb * db_sh + q * db_sq + k]
+  // (strides 0 on broadcast dims; hb = h if db_head_per_query else h / group).
+  float* dbias = nullptr;
+  int64_t db_sb = 0, db_sh = 0, db_sq = 0;
+  int db_head_per_query = 0;
+  int db_mode = 0;  // kDbias* below
 };
+
+// How the backward writes dbias: not at all; one store per element (every
+// element of dS has its own dbias element); one atomic add per element
+// (several heads or batch rows share an element); one atomic add of each
+// thread's sum over its queries (dbias broadcast over the queries).
+enum DbiasMode { kDbiasNone = 0, kDbiasStore = 1, kDbiasAdd = 2, kDbiasRowSum = 3 };
 
 // Single-query (decode) problem after the grouped-head swap: for each
 // (b, kv head) the `group` query heads are the rows.

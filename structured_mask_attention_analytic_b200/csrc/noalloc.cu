@@ -15,7 +15,9 @@
 //   which loads the library holds until the process exits.  Problems whose
 //   block map needs more (batch * ceil(q_len/128) * (ceil(k_len/128) + 1) *
 //   8 bytes, plus alignment) are rejected with SMA_ERR_WORKSPACE; use
-//   dfa_attn_fwd with a caller workspace for those.
+//   dfa_attn_fwd with a caller workspace for those.  Short-query problems
+//   split each unit's key tiles over several SMs only when the partial
+//   results fit in the array beside the block map.
 // * Every call shares the array and overwrites it.  Calls that can run at the
 //   same time on the GPU (e.g. on two streams without ordering between them)
 //   race on it; order them on one stream.  Nothing in the array needs to start
@@ -31,6 +33,10 @@
 
 #include "kernels.h"
 #include "sma.h"
+
+namespace sma {
+size_t dfa_fwd_map_bytes(const dfa_mask_desc* desc);
+}
 
 namespace {
 
@@ -53,9 +59,12 @@ extern "C" sma_status dfa_attn_fwd_noalloc(const dfa_mask_desc* desc, const int3
                                            const int64_t k_strides[3], const void* v,
                                            const int64_t v_strides[3], void* out,
                                            const int64_t o_strides[3], float* lse, void* stream) {
-  size_t need = 0;
-  sma_status s = dfa_attn_fwd_workspace_size(desc, heads, kv_heads, head_dim, &need);
+  size_t full = 0;  // validates the arguments
+  sma_status s = dfa_attn_fwd_workspace_size(desc, heads, kv_heads, head_dim, &full);
   if (s != SMA_OK) return s;
+  // the block map must fit; the key-range split's partials are used only if
+  // they fit as well
+  const size_t need = sma::dfa_fwd_map_bytes(desc);
   if (need > kNoAllocScratchBytes) {
     char msg[256];
     snprintf(msg, sizeof(msg),

@@ -162,6 +162,44 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
+// ---- key-range split of short-query forwards.  When the (batch, KV head,
+// head pair, query tile) units of the tcgen05 forward fill at most half of
+// the SMs, each unit's key-tile list is cut into n_split segments that run on
+// separate SMs: as many segments per unit as whole units fit in one wave,
+// at most one segment per 4 key tiles of a full list, and at most 32.  The
+// partial results sit in the workspace after `base`.
+struct SplitLayout {
+  int n_split;
+  size_t part_o, part_ml, end;
+};
+
+SplitLayout split_layout(size_t base, int B, int H, int KVH, int Lq, int d, int QT, int KT,
+                         int head_mode, int policy) {
+  SplitLayout s{1, base, base, base};
+  const int group = H / KVH;
+  const int64_t units =
+      fwd_units(B, KVH, (group + 1) / 2, QT, Lq, fwd_pack(Lq, group, head_mode, policy));
+  int64_t ns = units > 0 ? num_sms() / units : 1;
+  if (ns > KT / 4) ns = KT / 4;
+  if (ns > 32) ns = 32;
+  if (ns < 2) return s;
+  s.n_split = static_cast<int>(ns);
+  const size_t rows = static_cast<size_t>(B) * H * Lq;
+  s.part_o = align256(base);
+  s.part_ml = align256(s.part_o + static_cast<size_t>(ns) * rows * d * 4);
+  s.end = align256(s.part_ml + static_cast<size_t>(ns) * rows * 8);
+  return s;
+}
+
+// Enables the split on a tensor-core problem whose workspace holds it.
+void apply_split(AttnProblem& p, const SplitLayout& s, void* ws) {
+  if (s.n_split < 2 || p.dtype == SMA_FP32) return;
+  p.n_split = s.n_split;
+  p.part_o = at<float>(ws, s.part_o);
+  p.part_ml = at<float>(ws, s.part_ml);
+  p.part_rows = static_cast<int64_t>(p.B) * p.H * p.Lq;
+}
+
 sma_status check_workspace(void* ws, size_t have, size_t need) {
   if (have < need)
     return fail(SMA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", have,
@@ -179,6 +217,7 @@ struct MaskedGeom {
   int splits, chunk;
   size_t codes_bytes;
   ListsLayout lists;
+  SplitLayout kv_split;  // key-range split of the tcgen05 forward
   size_t part_o, part_ml, total;
 };
 
@@ -223,7 +262,8 @@ MaskedGeom masked_geom(int32_t B, int32_t H, int32_t KVH, int32_t Lq, int32_t Lk
   g.codes_bytes =
       has_mask ? align256(static_cast<size_t>(mask_sizes[0] * mask_sizes[1]) * g.codes_qt * g.KT) : 0;
   g.lists = lists_layout(g.codes_bytes, static_cast<int64_t>(g.LB) * g.LH * g.QT, g.KT);
-  g.total = g.lists.end;
+  g.kv_split = split_layout(g.lists.end, B, H, KVH, Lq, d, g.QT, g.KT, g.head_mode, kPolicyExplicit);
+  g.total = g.kv_split.end;
   return g;
 }
 
@@ -301,7 +341,9 @@ struct SparseGeom {
   int LB, LH, QT, KT, cap, Hc, Qc;
   size_t idx, count;
   ListsLayout lists;
-  size_t kc, vc, bias, total;
+  size_t kc, vc, bias;
+  SplitLayout kv_split;
+  size_t total;
 };
 
 sma_status sparse_geom(int32_t dtype, int32_t B, int32_t H, int32_t KVH, int32_t Lq, int32_t Lk,
@@ -346,6 +388,9 @@ sma_status sparse_geom(int32_t dtype, int32_t B, int32_t H, int32_t KVH, int32_t
     g->total = align256(g->bias + static_cast<size_t>(B) * g->Hc * g->Qc * g->cap *
                                       elem_size(bias_dtype));
   }
+  g->kv_split = split_layout(g->total, B, H, KVH, Lq, d, g->QT, g->KT, g->LH > 1 ? 1 : 0,
+                             kPolicyGather);
+  g->total = g->kv_split.end;
   return SMA_OK;
 }
 
@@ -418,6 +463,19 @@ sma_status dfa_block_map(const dfa_mask_desc* desc, const int32_t* anchors, int3
   return ok();
 }
 
+}  // extern "C"
+
+namespace sma {
+// Bytes of the DFlash forward's block map in its workspace (the minimum
+// workspace of dfa_attn_fwd without a block map).
+size_t dfa_fwd_map_bytes(const dfa_mask_desc* desc) {
+  const DflashGeom g = make_geom(desc);
+  return lists_layout(0, static_cast<int64_t>(g.B) * g.QT, g.KT).end;
+}
+}  // namespace sma
+
+extern "C" {
+
 sma_status dfa_attn_fwd_workspace_size(const dfa_mask_desc* desc, int32_t heads, int32_t kv_heads,
                                        int32_t head_dim, size_t* bytes) {
   sma_status s = check_desc(desc);
@@ -426,7 +484,8 @@ sma_status dfa_attn_fwd_workspace_size(const dfa_mask_desc* desc, int32_t heads,
   if (s != SMA_OK) return s;
   if (bytes == nullptr) return fail(SMA_ERR_INVALID_ARG, "bytes is NULL");
   const DflashGeom g = make_geom(desc);
-  *bytes = lists_layout(0, static_cast<int64_t>(g.B) * g.QT, g.KT).end;
+  const ListsLayout lay = lists_layout(0, static_cast<int64_t>(g.B) * g.QT, g.KT);
+  *bytes = split_layout(lay.end, g.B, heads, kv_heads, g.Nq, head_dim, g.QT, g.KT, 0, kPolicyDflash).end;
   return ok();
 }
 
@@ -449,12 +508,17 @@ sma_status dfa_attn_fwd(const dfa_mask_desc* desc, const int32_t* anchors, int32
   if ((s = check_operand("v", v, v_strides, dtype, g.Lk)) != SMA_OK) return s;
   if ((s = check_operand("out", out, o_strides, dtype, g.Nq)) != SMA_OK) return s;
   const ListsLayout lay = lists_layout(0, static_cast<int64_t>(g.B) * g.QT, g.KT);
+  const SplitLayout sp = split_layout(lay.end, g.B, heads, kv_heads, g.Nq, head_dim, g.QT, g.KT, 0, kPolicyDflash);
+  // The workspace must hold the block map (unless one is given); the
+  // key-range split runs only when it also holds the split's partial results.
   if (block_map != nullptr) {
     if (!block_map->num_full || !block_map->full_idx || !block_map->num_part || !block_map->part_idx)
       return fail(SMA_ERR_INVALID_ARG, "block_map has a NULL pointer");
   } else if ((s = check_workspace(workspace, workspace_bytes, lay.end)) != SMA_OK) {
     return s;
   }
+  const bool split_ok = workspace != nullptr && workspace_bytes >= sp.end &&
+                        (reinterpret_cast<uintptr_t>(workspace) & 255u) == 0;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
@@ -494,6 +558,7 @@ sma_status dfa_attn_fwd(const dfa_mask_desc* desc, const int32_t* anchors, int32
   p.anchors = anchors; p.N = g.N; p.bs = g.bs; p.Lc = g.Lc;
   p.causal_in_block = g.causal; p.window = g.window;
   p.err = err;
+  if (split_ok) apply_split(p, sp, workspace);
   if (dtype == SMA_FP32) {
     e = launch_attn_simt(p, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch failed");
@@ -633,6 +698,7 @@ sma_status masked_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   p.lists.num_part = at<int32_t>(workspace, mg.lists.np);
   p.lists.full_idx = at<int32_t>(workspace, mg.lists.fi);
   p.lists.part_idx = at<int32_t>(workspace, mg.lists.pi);
+  apply_split(p, mg.kv_split, workspace);
   uint8_t* codes = has_mask ? at<uint8_t>(workspace, 0) : nullptr;
   if (has_mask) {
     const int64_t folded[4] = {mview.sb, mview.sh, mview.sq, 1};
@@ -811,6 +877,7 @@ sma_status sparse_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   p.gather.cap = g.cap;
   p.gather.k_len = k_len;
   p.gather.causal = is_causal;
+  apply_split(p, g.kv_split, workspace);
   if (has_bias) {
     AuxView cb;
     cb.ptr = at<uint8_t>(workspace, g.bias);
@@ -951,7 +1018,10 @@ sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   if (batch < 1 || q_len < 1 || k_len < 1)
     return fail(SMA_ERR_INVALID_ARG, "batch, q_len and k_len must be >= 1");
   if (is_causal != 0 && is_causal != 1) return fail(SMA_ERR_INVALID_ARG, "is_causal must be 0 or 1");
-  if (dbias != nullptr) return fail(SMA_ERR_UNSUPPORTED, "dbias is not produced by this build");
+  if (dbias != nullptr && bias == nullptr)
+    return fail(SMA_ERR_INVALID_ARG, "dbias needs the bias (it takes the bias's shape)");
+  if (dbias != nullptr && (reinterpret_cast<uintptr_t>(dbias) & 15u) != 0)
+    return fail(SMA_ERR_INVALID_ARG, "dbias must be 16-byte aligned");
   if ((s = check_operand("q", q, q_strides, dtype, q_len)) != SMA_OK) return s;
   if ((s = check_operand("k", k, k_strides, dtype, k_len)) != SMA_OK) return s;
   if ((s = check_operand("v", v, v_strides, dtype, k_len)) != SMA_OK) return s;
@@ -1020,6 +1090,21 @@ sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   e = launch_explicit_lists(p, codes, mg.codes_qt, nf, fi, np, pi, st);
   if (e != cudaSuccess) return cuda_fail(e, "tile list launch failed");
   set_grads(b, dout, do_strides, dq, dq_strides, dk, dk_strides, dv, dv_strides, sc);
+  if (dbias != nullptr) {
+    // contiguous fp32 at the bias's sizes (b', h', q', round_up(Lk, 128))
+    const int64_t kp = round_up(k_len, kTile);
+    const int64_t nb = bias_sizes[0], nh = bias_sizes[1], nq = bias_sizes[2];
+    b.dbias = dbias;
+    b.db_sq = nq > 1 ? kp : 0;
+    b.db_sh = nh > 1 ? nq * kp : 0;
+    b.db_sb = nb > 1 ? nh * nq * kp : 0;
+    b.db_head_per_query = bview.head_per_query;
+    const bool own_head = heads == 1 || (nh > 1 && (bview.head_per_query || p.group == 1));
+    const bool own_batch = batch == 1 || nb > 1;
+    b.db_mode = nq == 1 ? kDbiasRowSum : (own_head && own_batch ? kDbiasStore : kDbiasAdd);
+    e = cudaMemsetAsync(dbias, 0, static_cast<size_t>(nb * nh * nq * kp) * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "dbias zeroing failed");
+  }
   if ((s = run_backward(b, workspace, lay, st)) != SMA_OK) return s;
   return ok();
 }

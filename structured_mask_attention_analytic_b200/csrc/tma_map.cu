@@ -24,10 +24,11 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 }  // namespace
 
-// 4D map over [B][len][heads][d] (d contiguous), box = 64 x 1 x 128 x 1,
-// 128-byte swizzle, zero fill outside the tensor.
+// 4D map over [B][len][heads][d] (d contiguous), box = 64 x box_heads x
+// (128 / box_heads) x 1, 128-byte swizzle, zero fill outside the tensor.
 bool encode_map(CUtensorMap* map, const void* ptr, int dtype, int d, int heads, int len, int batch,
-                int64_t s_head, int64_t s_row, int64_t s_batch, char* msg, size_t msg_len) {
+                int64_t s_head, int64_t s_row, int64_t s_batch, char* msg, size_t msg_len,
+                int box_heads) {
   auto enc = get_encode_fn();
   if (enc == nullptr) {
     snprintf(msg, msg_len, "cuTensorMapEncodeTiled is unavailable");
@@ -43,7 +44,12 @@ bool encode_map(CUtensorMap* map, const void* ptr, int dtype, int d, int heads, 
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(s_head * esz),
                            static_cast<cuuint64_t>(s_row * esz),
                            static_cast<cuuint64_t>(s_batch * esz)};
-  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(SMA_TILE), 1};
+  if (box_heads < 1 || box_heads > heads || SMA_TILE % box_heads != 0) {
+    snprintf(msg, msg_len, "invalid heads per TMA box (%d)", box_heads);
+    return false;
+  }
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_heads),
+                       static_cast<cuuint32_t>(SMA_TILE / box_heads), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, dtype == SMA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,

@@ -314,10 +314,12 @@ def masked_attn_bwd_workspace_size(batch, heads, kv_heads, q_len, k_len, head_di
 
 
 def masked_attn_bwd(q, k, v, out, lse, dout, mask=None, bias=None, is_causal: bool = False, scale=None,
-                    dq=None, dk=None, dv=None, workspace=None):
+                    dq=None, dk=None, dv=None, workspace=None, return_dbias: bool = False, dbias=None):
     """Gradients of ``masked_attn_fwd`` (same mask / bias / causal / scale):
     ``out`` and ``lse`` are that call's results, ``dout`` the upstream
-    gradient.  Returns ``(dq, dk, dv)``; no bias gradient."""
+    gradient.  Returns ``(dq, dk, dv)``, or ``(dq, dk, dv, dbias)`` with
+    ``return_dbias`` (or a ``dbias`` buffer): float32 at the bias's shape,
+    reduced over the dims the bias broadcasts along."""
     _require_cuda(q, k, v, out, lse, dout, mask, bias)
     b, lq, h, dh = q.shape
     lk, kvh = k.shape[1], k.shape[2]
@@ -330,6 +332,14 @@ def masked_attn_bwd(q, k, v, out, lse, dout, mask=None, bias=None, is_causal: bo
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     mp, msz, mst = _aux_args(mask, lk)
     bp, bsz, bst = _aux_args(bias, lk)
+    want_db = return_dbias or dbias is not None
+    if want_db:
+        if bias is None:
+            raise ValueError("dbias needs a bias")
+        if dbias is None:
+            dbias = torch.empty(tuple(bias.shape), dtype=torch.float32, device=q.device)
+        elif dbias.dtype != torch.float32 or tuple(dbias.shape) != tuple(bias.shape) or not dbias.is_contiguous():
+            raise ValueError("dbias must be contiguous float32 with the bias's shape")
     nat.check(_lib().masked_attn_bwd(
         _dtype_code(q), b, h, kvh, lq, lk, dh, ctypes.c_float(0.0 if scale is None else float(scale)),
         1 if is_causal else 0,
@@ -338,8 +348,8 @@ def masked_attn_bwd(q, k, v, out, lse, dout, mask=None, bias=None, is_causal: bo
         bp, _dtype_code(bias) if bias is not None else 0, bsz, bst,
         _ptr(out), _strides3(out), _ptr(lse), _ptr(dout), _strides3(dout),
         _ptr(dq), _strides3(dq), _ptr(dk), _strides3(dk), _ptr(dv), _strides3(dv),
-        ctypes.c_void_p(0), _ptr(workspace), workspace.numel(), _stream(q)))
-    return dq, dk, dv
+        _ptr(dbias) if want_db else ctypes.c_void_p(0), _ptr(workspace), workspace.numel(), _stream(q)))
+    return (dq, dk, dv, dbias) if want_db else (dq, dk, dv)
 
 
 def sparse_attn_fwd_workspace_size(dtype, batch, heads, kv_heads, q_len, k_len, head_dim, mask_shape,

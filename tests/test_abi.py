@@ -76,6 +76,25 @@ def test_workspace_sizes_on_host():
     assert n.value > 0
 
 
+def test_workspace_holds_key_range_segments_for_short_queries():
+    """16 queries after an 8k context (4 units on a 148-SM part): the forward
+    workspace holds the partial results of 16 key-range segments per unit
+    (fp32 O and (max, sum) per segment and row); 64 batch rows fill the SMs
+    and need no segments."""
+    lib = nat.load()
+    n = ctypes.c_size_t()
+    short = nat.DfaMaskDesc(1, 1, 16, 8192, 1, 0, 0)
+    assert lib.dfa_attn_fwd_workspace_size(ctypes.byref(short), 8, 2, 128, ctypes.byref(n)) == 0
+    rows = 1 * 8 * 16
+    assert n.value >= 16 * rows * (128 * 4 + 8)
+    wide = nat.DfaMaskDesc(64, 1, 16, 8192, 1, 0, 0)
+    assert lib.dfa_attn_fwd_workspace_size(ctypes.byref(wide), 8, 2, 128, ctypes.byref(n)) == 0
+    assert n.value < 64 * 65 * 4 * 2 + 64 * 4 * 2 + 4096
+    ms = nat.i64_array([1, 1, 24, 5120])
+    assert lib.masked_attn_fwd_workspace_size(1, 8, 2, 24, 5000, 128, ms, ctypes.byref(n)) == 0
+    assert n.value >= 10 * (8 * 24) * (128 * 4 + 8)
+
+
 def _masked_call(**over):
     """masked_attn_fwd with fake (never dereferenced) aligned pointers."""
     a = dict(dtype=0, batch=2, heads=4, kv_heads=2, q_len=256, k_len=200, head_dim=128,
@@ -210,8 +229,8 @@ def test_backward_workspace_and_validation_on_host():
     assert "bf16 or fp16" in lib.sma_last_error().decode()
     assert call(lse=0) == nat.SMA_ERR_INVALID_ARG
     assert "lse" in lib.sma_last_error().decode()
-    assert call(dbias=0xb0000) == nat.SMA_ERR_UNSUPPORTED
-    assert "dbias" in lib.sma_last_error().decode()
+    assert call(dbias=0xb0000) == nat.SMA_ERR_INVALID_ARG  # no bias to take the gradient of
+    assert "dbias needs the bias" in lib.sma_last_error().decode()
 
 
 def test_varlen_validation_on_host():

@@ -133,3 +133,57 @@ def test_fp16_and_rejections():
     _close("dv", dv, rv)
     with pytest.raises(sma.SmaError, match="bf16 or fp16"):
         sma.masked_attn_bwd(qc.float(), kc.float(), vc.float(), out.float(), lse, dc.float())
+
+
+DB_SHAPES = [(B, H, LQ, KP), (B, KVH, LQ, KP), (1, 1, LQ, KP), (B, H, 1, KP), (1, KVH, 1, KP),
+             (1, 1, 1, KP)]
+
+
+@pytest.mark.parametrize("bshape", DB_SHAPES, ids=str)
+@pytest.mark.parametrize("D", [64, 128])
+def test_masked_backward_dbias(bshape, D):
+    """The bias gradient dS summed over every dim the bias broadcasts along
+    (batch, the heads of a group or all heads, the queries), against the
+    oracle's reduction onto the bias shape; padded key columns stay 0."""
+    rng = wl.rng_for(35)
+    q = wl.normal(rng, (B, LQ, H, D), "bf16")
+    k = wl.normal(rng, (B, LK, KVH, D), "bf16")
+    v = wl.normal(rng, (B, LK, KVH, D), "bf16")
+    do = wl.normal(rng, (B, LQ, H, D), "bf16")
+    mask = torch.from_numpy(rng.random((B, KVH, 1, KP)) < 0.8)
+    bias = wl.normal(rng, bshape, "bf16")
+    qc, kc, vc, dc, mc, bc = (t.cuda() for t in (q, k, v, do, mask, bias))
+    out, lse = sma.masked_attn_fwd(qc, kc, vc, mc, bc, True)
+    dq, dk, dv, db = sma.masked_attn_bwd(qc, kc, vc, out, lse, dc, mc, bc, True, return_dbias=True)
+    torch.cuda.synchronize()
+    assert sma.device_status() == 0
+    assert db.shape == bias.shape and db.dtype == torch.float32
+    keep = at.aux_view(mask.numpy(), H, KVH, LK) & at.causal_keep(LQ, LK)[None, None]
+    bb = at.aux_view(f64(bias), H, KVH, LK)
+    rq, rk, rv, rdb = ag.attention_grad(f64(q), f64(k), f64(v), f64(do), keep=keep, bias=bb,
+                                        dbias_shape=bshape, workers=8)
+    _close("dq", dq, rq)
+    _close("dk", dk, rk)
+    _close("dv", dv, rv)
+    _close("dbias", db, rdb)
+    assert (db[..., LK:] == 0).all()
+
+
+def test_dbias_fp16_per_query_bias_and_rejection():
+    rng = wl.rng_for(36)
+    q = wl.normal(rng, (1, 130, 4, 128), "fp16")
+    k = wl.normal(rng, (1, 260, 2, 128), "fp16")
+    v = wl.normal(rng, (1, 260, 2, 128), "fp16")
+    do = wl.normal(rng, (1, 130, 4, 128), "fp16")
+    kp = sma.round_up_k(260)
+    bias = wl.normal(rng, (1, 4, 130, kp), "fp32")
+    qc, kc, vc, dc, bc = (t.cuda() for t in (q, k, v, do, bias))
+    out, lse = sma.masked_attn_fwd(qc, kc, vc, None, bc, False)
+    dq, dk, dv, db = sma.masked_attn_bwd(qc, kc, vc, out, lse, dc, None, bc, False, return_dbias=True)
+    torch.cuda.synchronize()
+    rq, rk, rv, rdb = ag.attention_grad(f64(q), f64(k), f64(v), f64(do), bias=f64(bias)[..., :260],
+                                        dbias_shape=tuple(bias.shape))
+    _close("dbias", db, rdb)
+    _close("dq", dq, rq)
+    with pytest.raises(ValueError, match="needs a bias"):
+        sma.masked_attn_bwd(qc, kc, vc, out, lse, dc, None, None, False, return_dbias=True)

@@ -143,3 +143,56 @@ def test_decode_equals_unswapped_rows():
 def test_decode_workload(w):
     q, k, v, mask, bias = wl.masked_inputs(w)
     _run(q, k, v, mask, bias, False, what=w.name)
+
+
+# ------------------------------------------------- short queries, long keys
+
+
+LK_LONG = 5000
+KP_LONG = sma.round_up_k(LK_LONG)
+
+
+@pytest.mark.parametrize("mshape,bshape", [(None, None), ((1, 1, 24, KP_LONG), (1, 8, 1, KP_LONG)),
+                                           ((1, 8, 24, KP_LONG), None)], ids=str)
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_short_queries_long_keys(mshape, bshape, causal, d):
+    """24 queries against 5000 keys give 4 (batch, KV head, head pair, query
+    tile) units: each unit's key tiles are cut into segments run on separate
+    SMs and merged.  Row 3 keeps no key at all, row 5 none of the first 2500
+    keys (its early segments are empty)."""
+    rng = wl.rng_for(14)
+    q, k, v = _qkv(rng, 1, 24, LK_LONG, 8, 2, d)
+    mask = None
+    if mshape is not None:
+        mask = torch.from_numpy(rng.random(mshape) < 0.7)
+        if mshape[2] > 1:
+            mask[:, :, 3, :] = False
+            mask[:, :, 5, :2500] = False
+    bias = wl.normal(rng, bshape, "bf16") if bshape else None
+    out, lse = _run(q, k, v, mask, bias, causal, what=f"short {mshape} {bshape} {causal} {d}")
+    if mshape is not None and mshape[2] > 1:
+        assert (out[0, 3] == 0).all() and torch.isneginf(lse[0, :, 3]).all()
+
+
+def test_short_queries_fp16():
+    rng = wl.rng_for(15)
+    q, k, v = _qkv(rng, 2, 40, 3000, 4, 4, D, "fp16")
+    mask = torch.from_numpy(rng.random((2, 4, 1, sma.round_up_k(3000))) < 0.5)
+    _run(q, k, v, mask, None, True, what="short fp16")
+
+
+@pytest.mark.parametrize("h,kvh,lq", [(16, 2, 40), (4, 2, 64), (8, 4, 2), (16, 2, 16)], ids=str)
+@pytest.mark.parametrize("causal", [False, True])
+def test_short_queries_heads_packed_per_tile(h, kvh, lq, causal):
+    """Up to 64 queries with 2, 4 or 8 heads per KV head: one 128-row tile
+    holds every head of the group for 128 / group queries (group 8 and 40
+    queries: three blocks of 16, two tiles in one unit and one alone).  The
+    bias differs per query head and per query, the mask per KV head."""
+    rng = wl.rng_for(16)
+    lk = 3000
+    kp = sma.round_up_k(lk)
+    q, k, v = _qkv(rng, 2, lq, lk, h, kvh, D)
+    mask = torch.from_numpy(rng.random((2, kvh, lq, kp)) < 0.6)
+    bias = wl.normal(rng, (1, h, lq, kp), "bf16")
+    _run(q, k, v, mask, bias, causal, what=f"packed {h}/{kvh} lq={lq} {causal}")

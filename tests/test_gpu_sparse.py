@@ -54,6 +54,17 @@ def test_dtypes_and_head_dims(dtype, d):
     _run(q, k, v, mask, bias, True, what=f"{dtype} d={d}")
 
 
+def test_short_queries_many_keys():
+    """16 queries over ~10k kept of 20k keys: 4 units, so the compacted key
+    tiles of each are cut into segments on separate SMs and merged."""
+    rng = wl.rng_for(26)
+    q, k, v = _qkv(rng, 1, 16, 20000, 8, 2, D)
+    kp = sma.round_up_k(20000)
+    mask = torch.from_numpy(rng.random((1, 2, 1, kp)) < 0.5)
+    bias = wl.normal(rng, (1, 8, 16, kp), "bf16")
+    _run(q, k, v, mask, bias, True, what="short gather")
+
+
 def test_mha_mask_per_head():
     """heads == kv_heads: a mask row per head."""
     rng = wl.rng_for(23)
@@ -64,15 +75,16 @@ def test_mha_mask_per_head():
 
 def test_max_keys_exact_bound():
     """max_keys equal to the largest kept count sizes the compacted operands
-    exactly; the result does not change."""
+    exactly; both capacities give the oracle's result.  (They need not agree
+    bit for bit: the capacity sets how many key-range segments a unit's tiles
+    are cut into, and so the order of the fp32 sums.)"""
     rng = wl.rng_for(24)
     q, k, v = _qkv(rng, B, LQ, LK, H, KVH, D)
     mask = torch.from_numpy(rng.random((B, KVH, 1, KP)) < 0.25)
     mask[..., LK:] = False
     top = int(mask.sum(-1).max())
-    o1, l1 = _run(q, k, v, mask, None, True, max_keys=top, what="exact max_keys")
-    o2, l2 = sma.sparse_attn_fwd(q.cuda(), k.cuda(), v.cuda(), mask.cuda(), None, True)
-    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    _run(q, k, v, mask, None, True, max_keys=top, what="exact max_keys")
+    _run(q, k, v, mask, None, True, what="default max_keys")
 
 
 def test_rows_over_max_keys_raise_device_input():

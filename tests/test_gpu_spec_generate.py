@@ -47,3 +47,24 @@ def test_spec_generate_long_context_sampled_heads():
     keep = dm.spec_generate_keep_mask(ctx_lens.numpy(), Lc, bs, True, None)[:, None]
     ref_o, ref_l = at.attention(f64(q), f64(k), f64(v), keep=keep, workers=8)
     assert_attention_close(out, lse, ref_o, ref_l, q.dtype, what="spec long")
+
+
+@pytest.mark.parametrize("H,KVH", [(8, 2), (16, 2), (4, 2)], ids=str)
+@pytest.mark.parametrize("is_causal", [True, False])
+def test_spec_generate_segments_of_mixed_lengths(is_causal, H, KVH):
+    """An 8k context with one block of 16 queries: the group's heads share a
+    128-row tile (4, 8 or 2 heads of 32, 16 or 64 queries) and every unit's
+    key tiles are cut into segments.  Row 0's list holds two tiles (most
+    segments empty), row 1's about 64."""
+    rng = wl.rng_for(43)
+    B, D, Lc, bs = 2, 128, 8192, 16
+    q = wl.normal(rng, (B, bs, H, D), "bf16")
+    k = wl.normal(rng, (B, Lc + bs, KVH, D), "bf16")
+    v = wl.normal(rng, (B, Lc + bs, KVH, D), "bf16")
+    ctx_lens = torch.tensor([37, 8000], dtype=torch.int32)
+    out, lse = sma.dflash_spec_generate_fwd(q.cuda(), k.cuda(), v.cuda(), ctx_lens.cuda(), Lc, is_causal)
+    torch.cuda.synchronize()
+    assert sma.device_status() == 0
+    keep = dm.spec_generate_keep_mask(ctx_lens.numpy(), Lc, bs, is_causal, None)[:, None]
+    ref_o, ref_l = at.attention(f64(q), f64(k), f64(v), keep=keep, workers=8)
+    assert_attention_close(out, lse, ref_o, ref_l, q.dtype, what=f"spec segments {is_causal}")
