@@ -196,3 +196,26 @@ def test_short_queries_heads_packed_per_tile(h, kvh, lq, causal):
     mask = torch.from_numpy(rng.random((2, kvh, lq, kp)) < 0.6)
     bias = wl.normal(rng, (1, h, lq, kp), "bf16")
     _run(q, k, v, mask, bias, causal, what=f"packed {h}/{kvh} lq={lq} {causal}")
+
+
+@pytest.mark.parametrize("bshape", [(2, 2, 1, KP), (1, 1, 1, KP), (2, 1, 1, KP)], ids=str)
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("fp16", 64)])
+def test_query_broadcast_bias_large_values(bshape, dtype, d):
+    """A bias shared by every query and query head of a KV head, with values
+    of +-30 (peaked rows, where the dominant key's probability is exactly
+    representable only if the row max includes the bias), keys at -inf (never
+    kept), and, where the bias has a row per (batch, KV head), one row at
+    -inf everywhere (its queries keep nothing: O = 0, lse = -inf)."""
+    rng = wl.rng_for(17)
+    q, k, v = _qkv(rng, B, LQ, LK, H, KVH, d, dtype)
+    mask = torch.from_numpy(rng.random((1, 1, LQ, KP)) < 0.8)
+    bias = (wl.normal(rng, bshape, "fp32") * 10.0).clamp(-30, 30)
+    bias[..., ::7] = -float("inf")
+    dead = bshape[0] == 2 and bshape[1] == 2
+    if dead:
+        bias[1, 1] = -float("inf")
+    bias = bias.to(torch.bfloat16 if dtype == "bf16" else torch.float16)
+    out, lse = _run(q, k, v, mask, bias, True, what=f"large bias {bshape} {dtype} {d}")
+    if dead:
+        heads = slice(1 * (H // KVH), 2 * (H // KVH))
+        assert (out[1, :, heads] == 0).all() and torch.isneginf(lse[1, heads]).all()
