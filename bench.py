@@ -131,6 +131,37 @@ def timed(fn, stream, reps, warmup):
     return s.elapsed_time(e) / reps
 
 
+# DRAM bytes (read + write) of one attention launch of a workload, from one
+# ncu capture of dram__bytes_read.sum / dram__bytes_write.sum on the current
+# attn_tc_kernel (profiles/attn_tc_dflash_long_full_traffic.md).  Remove an
+# entry when that kernel changes.
+MEASURED_TRAFFIC = {"dflash_long_full": 2.11e9 + 0.24844e9}
+
+
+def timed_graph(fn, reps, warmup):
+    """Average ms of one replay of a CUDA graph holding one fn() call (the
+    same launches without the Python / ctypes issue time between them)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    side = torch.cuda.current_stream()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(side)
+    for _ in range(reps):
+        g.replay()
+    e.record(side)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / reps
+    del g
+    return ms
+
+
 def dflash_case(w, dev, seed=None):
     q, k, v, anchors = wl.dflash_inputs(w, seed)
     return tuple(t.to(dev) for t in (q, k, v, anchors))
@@ -243,10 +274,10 @@ def run_ours(args, rank, world, dev):
         def e2e_step():
             for d_, h_ in ((qd, qh), (kd, kh), (vd, vh), (ad, ah)):
                 d_.copy_(h_, non_blocking=True)
-            sma.dfa_attn_fwd(qd, kd, vd, ad, w.ctx_len, w.block_size, w.is_causal, w.layer_type,
-                             w.sliding_window, out=out, workspace=ws)
+            _, lse_step = sma.dfa_attn_fwd(qd, kd, vd, ad, w.ctx_len, w.block_size, w.is_causal,
+                                           w.layer_type, w.sliding_window, out=out, workspace=ws)
             oh.copy_(out, non_blocking=True)
-            lh.copy_(lse, non_blocking=True)
+            lh.copy_(lse_step, non_blocking=True)
 
         e_ms = timed(e2e_step, stream, args.e2e_steps, 2)
         h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, ah))
@@ -270,7 +301,9 @@ def run_ours(args, rank, world, dev):
         "config": config_dict(w, {"parallelism": f"replicas x{world} (one long-context batch per GPU)",
                                   "kept_tiles": kept, "flops_per_step": flops}),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": args.traffic_bytes,
+                     "frac": achieved / peak,
+                     "traffic": args.traffic_bytes if args.traffic_bytes is not None
+                     else MEASURED_TRAFFIC.get(w.name),
                      "kernel": "attn_tc_kernel<128, DFlash, bf16>",
                      "peak_source": f"{peak_src} bf16 dense burst",
                      "frac_of_spec_2250": achieved / 2250.0,
@@ -335,10 +368,14 @@ def run_details(sma, dev, stream, peaks, only=None):
         v = torch.randn_like(k)
         cl = torch.tensor([lc], dtype=torch.int32, device=dev)
         o = torch.empty_like(q)
-        ms = timed(lambda: sma.dflash_spec_generate_fwd(q, k, v, cl, lc, True, out=o), stream, 20, 3)
+        call = lambda: sma.dflash_spec_generate_fwd(q, k, v, cl, lc, True, out=o)
+        ms_eager = timed(call, stream, 20, 3)
+        ms = timed_graph(call, 20, 3)  # block map, attention, combine: one graph replay
         nbytes = 2 * k.numel() * 2 + 2 * q.numel() * 2
         out["spec_generate_32k"] = {"ms": ms, "GB/s": nbytes / (ms * 1e-3) / 1e9,
-                                    "frac_hbm_peak": nbytes / (ms * 1e-3) / 1e9 / pk_b, "bytes": nbytes}
+                                    "frac_hbm_peak": nbytes / (ms * 1e-3) / 1e9 / pk_b, "bytes": nbytes,
+                                    "timing": "CUDA graph replay of the call's 3 launches",
+                                    "ms_python_calls": ms_eager}
         del q, k, v, o
 
     if want("varlen"):

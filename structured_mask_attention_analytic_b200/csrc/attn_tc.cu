@@ -779,7 +779,11 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
 // 2^(t - m_s); with M = max m_s over the segments that kept a key,
 //   O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,
 //   lse = ln 2 * (M + log2 sum_s 2^(m_s - M) l_s).
-// One warp per row, each lane D / 32 consecutive columns.
+// One warp per row: lane s reads segment s's (m_s, l_s) (at most 32
+// segments), the warp reduces M and the sum, then every lane accumulates its
+// D / 32 columns over the segments, four independent loads at a time.  A
+// segment that kept no key of the row (l_s = 0) may not have written O_s and
+// is never read.
 template <int D, int DT>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnProblem p) {
   typedef typename std::conditional<DT == SMA_BF16, __nv_bfloat16, __half>::type OutT;
@@ -787,36 +791,47 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnProblem p) 
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= p.part_rows) return;
-  const float2* ml = reinterpret_cast<const float2*>(p.part_ml);
-  float mx = -INFINITY;
-  for (int s = lane; s < p.n_split; s += 32) {
-    const float2 v = ml[static_cast<int64_t>(s) * p.part_rows + row];
-    if (v.y > 0.f) mx = fmaxf(mx, v.x);
-  }
+  const int ns = p.n_split;
+  const float2 v = lane < ns
+                       ? reinterpret_cast<const float2*>(p.part_ml)[static_cast<int64_t>(lane) * p.part_rows + row]
+                       : make_float2(-INFINITY, 0.f);
+  const bool live = v.y > 0.f;
+  float mx = live ? v.x : -INFINITY;
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float wgt = live ? fast_exp2(v.x - mx) : 0.f;
+  float l = wgt * v.y;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-  float l = 0.f;
-  for (int s = 0; s < p.n_split; ++s) {
-    const int64_t sr = static_cast<int64_t>(s) * p.part_rows + row;
-    const float2 v = ml[sr];
-    if (!(v.y > 0.f)) continue;  // no kept key in this segment: O_s was not written
-    const float wgt = fast_exp2(v.x - mx);
-    l = fmaf(wgt, v.y, l);
-    const float* src = p.part_o + sr * D + lane * kPer;
-    if (kPer == 4) {
-      const float4 a = *reinterpret_cast<const float4*>(src);
-      acc[0] = fmaf(wgt, a.x, acc[0]);
-      acc[1] = fmaf(wgt, a.y, acc[1]);
-      acc[2] = fmaf(wgt, a.z, acc[2]);
-      acc[3] = fmaf(wgt, a.w, acc[3]);
-    } else {
-      const float2 a = *reinterpret_cast<const float2*>(src);
-      acc[0] = fmaf(wgt, a.x, acc[0]);
-      acc[1] = fmaf(wgt, a.y, acc[1]);
+  const float* src = p.part_o + row * D + lane * kPer;
+  const int64_t seg_stride = p.part_rows * D;
+  for (int s0 = 0; s0 < ns; s0 += 4) {
+    float ws[4];
+    float vals[4][kPer];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ws[i] = __shfl_sync(0xffffffffu, wgt, (s0 + i) & 31);
+      if (s0 + i >= ns) ws[i] = 0.f;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) vals[i][e] = 0.f;
+      if (ws[i] != 0.f) {
+        const float* sp = src + (s0 + i) * seg_stride;
+        if (kPer == 4) {
+          const float4 a = *reinterpret_cast<const float4*>(sp);
+          vals[i][0] = a.x; vals[i][1] = a.y; vals[i][2] = a.z; vals[i][3] = a.w;
+        } else {
+          const float2 a = *reinterpret_cast<const float2*>(sp);
+          vals[i][0] = a.x; vals[i][1] = a.y;
+        }
+      }
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) acc[e] = fmaf(ws[i], vals[i][e], acc[e]);
   }
   const float inv = l > 0.f ? 1.0f / l : 0.f;
   const int q = static_cast<int>(row % p.Lq);
@@ -911,9 +926,10 @@ int launch_problem(const AttnProblem& p, cudaStream_t stream, char* msg, size_t 
 }  // namespace
 
 int launch_attn_tc(const AttnProblem& p, cudaStream_t stream, char* msg, size_t msg_len) {
-  if (p.n_split < 1 || (p.n_split > 1 && (p.policy == kPolicyVarlen || p.part_o == nullptr ||
-                                          p.part_ml == nullptr ||
-                                          p.part_rows != static_cast<int64_t>(p.B) * p.H * p.Lq))) {
+  // the combine kernel reads one segment per lane: at most 32 segments
+  if (p.n_split < 1 || p.n_split > 32 ||
+      (p.n_split > 1 && (p.policy == kPolicyVarlen || p.part_o == nullptr || p.part_ml == nullptr ||
+                         p.part_rows != static_cast<int64_t>(p.B) * p.H * p.Lq))) {
     snprintf(msg, msg_len, "invalid key-range split");
     return SMA_ERR_INVALID_ARG;
   }
