@@ -781,7 +781,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
 //   lse = ln 2 * (M + log2 sum_s 2^(m_s - M) l_s).
 // One warp per row: lane s reads segment s's (m_s, l_s) (at most 32
 // segments), the warp reduces M and the sum, then every lane accumulates its
-// D / 32 columns over the segments, four independent loads at a time.  A
+// D / 32 columns over the segments, eight independent loads at a time.  A
 // segment that kept no key of the row (l_s = 0) may not have written O_s and
 // is never read.
 template <int D, int DT>
@@ -808,11 +808,12 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnProblem p) 
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
   const float* src = p.part_o + row * D + lane * kPer;
   const int64_t seg_stride = p.part_rows * D;
-  for (int s0 = 0; s0 < ns; s0 += 4) {
-    float ws[4];
-    float vals[4][kPer];
+  constexpr int kGroup = 8;
+  for (int s0 = 0; s0 < ns; s0 += kGroup) {
+    float ws[kGroup];
+    float vals[kGroup][kPer];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kGroup; ++i) {
       ws[i] = __shfl_sync(0xffffffffu, wgt, (s0 + i) & 31);
       if (s0 + i >= ns) ws[i] = 0.f;
 #pragma unroll
@@ -829,7 +830,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnProblem p) 
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < kGroup; ++i)
 #pragma unroll
       for (int e = 0; e < kPer; ++e) acc[e] = fmaf(ws[i], vals[i][e], acc[e]);
   }
