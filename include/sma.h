@@ -405,6 +405,32 @@ sma_status varlen_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
                            const int64_t v_strides[2], void* out, const int64_t o_strides[2],
                            float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Workspace bytes varlen_attn_bwd needs: the per-sequence tile lists and
+ * their transpose, rowsum(dO * O) [heads, total_q] and the fp32 dQ
+ * accumulator [total_q, heads, head_dim]. */
+sma_status varlen_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t total_q,
+                                          int32_t max_q, int32_t max_k, int32_t head_dim,
+                                          size_t* bytes);
+
+/* Gradients of varlen_attn_fwd for an upstream gradient dout (the packed
+ * counterpart of masked_attn_bwd; the derivative of softmax attention as in
+ * flash-sparse-attention PR #190, Changes: mha_bwd, per sequence).  out and
+ * lse are that forward's results for the same arguments (lse required);
+ * dout, dq [total_q, heads, d], dk, dv [total_k, kv_heads, d] with strides[2]
+ * = {row, head}.  Keys of a sequence that none of its queries keeps get zero
+ * dK / dV; rows with no kept key get zero dQ.  bf16 / fp16 only
+ * (SMA_ERR_UNSUPPORTED for SMA_FP32); offsets as in varlen_attn_fwd. */
+sma_status varlen_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t head_dim, int32_t total_q, int32_t total_k, int32_t max_q,
+                           int32_t max_k, float scale, int32_t is_causal, const int32_t* cu_seqlens_q,
+                           const int32_t* cu_seqlens_k, const void* q, const int64_t q_strides[2],
+                           const void* k, const int64_t k_strides[2], const void* v,
+                           const int64_t v_strides[2], const void* out, const int64_t o_strides[2],
+                           const float* lse, const void* dout, const int64_t do_strides[2],
+                           void* dq, const int64_t dq_strides[2], void* dk,
+                           const int64_t dk_strides[2], void* dv, const int64_t dv_strides[2],
+                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* pad: padded [batch, max_len, heads, d] (strides[3] = batch, row, head) from
  * packed rows, zero past each sequence's length; unpad: the reverse (rows
  * past a length are not read).  Rows must be 16-byte multiples. */

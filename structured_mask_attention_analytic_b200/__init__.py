@@ -28,6 +28,7 @@ from .ops import (  # noqa: F401
     selftest_wait_timeout,
     sparse_attn_fwd,
     sparse_attn_fwd_workspace_size,
+    varlen_attn_bwd,
     varlen_attn_fwd,
     varlen_pad,
     varlen_unpad,

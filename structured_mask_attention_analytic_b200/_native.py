@@ -91,6 +91,11 @@ _SIGNATURES = {
     "varlen_attn_fwd": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.c_float,
                                 c_i32, c_vp, c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
                                 c_vp, c_vp, c_size, c_vp]),
+    "varlen_attn_bwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_sizep]),
+    "varlen_attn_bwd": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.c_float,
+                                c_i32, c_vp, c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
+                                c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
+                                c_vp, c_size, c_vp]),
     "varlen_pad": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp]),
     "varlen_unpad": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp]),
     "sparse_attn_fwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64p,

@@ -89,8 +89,13 @@ __device__ __forceinline__ int64_t bwd_row(const BwdProblem& p, int b, int hk, i
   return static_cast<int64_t>(lb) * p.f.lists.LH + lh;
 }
 
+// A unit's rows: padded batches read batch b's rows [0, Lq) / [0, Lk) at
+// batch coordinate b; packed batches (cu_q / cu_k set) read sequence b's rows
+// [q_off, q_off + lq) / [k_off, k_off + lk) of the one packed batch.
 struct BUnit {
   int b, hk, kt, n_pairs;
+  int bt;                    // batch coordinate of the operands
+  int q_off, k_off, lq, lk;  // the unit's first rows and lengths
 };
 
 __device__ __forceinline__ BUnit bwd_unit(const BwdProblem& p, int u) {
@@ -100,13 +105,40 @@ __device__ __forceinline__ BUnit bwd_unit(const BwdProblem& p, int u) {
   const int r = u - w.kt * per_kt;
   w.b = r / p.f.KVH;
   w.hk = r - w.b * p.f.KVH;
+  bool empty = false;
+  if (p.f.cu_q != nullptr) {
+    w.bt = 0;
+    w.q_off = p.f.cu_q[w.b];
+    w.lq = p.f.cu_q[w.b + 1] - w.q_off;
+    w.k_off = p.f.cu_k[w.b];
+    w.lk = p.f.cu_k[w.b + 1] - w.k_off;
+    // malformed offsets (reported by the list kernel): nothing of the sequence
+    // is read or written
+    if (w.lq < 0 || w.lq > p.f.Lq || w.q_off < 0 || w.q_off + w.lq > p.f.total_q || w.lk < 0 ||
+        w.lk > p.f.Lk || w.k_off < 0 || w.k_off + w.lk > p.f.total_k) {
+      w.q_off = w.k_off = w.lq = w.lk = 0;
+      empty = true;
+    }
+  } else {
+    w.bt = w.b;
+    w.q_off = w.k_off = 0;
+    w.lq = p.f.Lq;
+    w.lk = p.f.Lk;
+  }
   int n = 0;
   for (int g = 0; g < p.f.group; ++g) {
     const int64_t row = bwd_row(p, w.b, w.hk, g);
     n += p.t_num_full[row * p.f.KT + w.kt] + p.t_num_part[row * p.f.KT + w.kt];
   }
-  w.n_pairs = n;
+  w.n_pairs = empty ? 0 : n;
   return w;
+}
+
+// Index of (head h, query q of the unit) in the [B, H, rows] per-query arrays
+// (lse, rowsum(dO * O)); packed batches: [H, total_q].
+__device__ __forceinline__ int64_t qrow(const BwdProblem& p, const BUnit& w, int h, int q) {
+  const int rows = p.f.cu_q != nullptr ? p.f.total_q : p.f.Lq;
+  return (static_cast<int64_t>(w.bt) * p.f.H + h) * rows + w.q_off + q;
 }
 
 // Walks the pairs of a unit in the order every role uses: heads of the group
@@ -256,9 +288,9 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         mbar_arrive_expect_tx(bar(L::kKVFull), 2 * L::kTileD);
         for (int c = 0; c < L::kChunksD; ++c) {
           tma_load_4d(sbase + L::kK + c * L::kChunk, &map_k, bar(L::kKVFull), c * 64, w.hk,
-                      w.kt * kTile, w.b);
+                      w.k_off + w.kt * kTile, w.bt);
           tma_load_4d(sbase + L::kV + c * L::kChunk, &map_v, bar(L::kKVFull), c * 64, w.hk,
-                      w.kt * kTile, w.b);
+                      w.k_off + w.kt * kTile, w.bt);
         }
       }
       __syncwarp();
@@ -279,7 +311,7 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           mbar_arrive_expect_tx(bar(L::kQFull + s), L::kTileD);
           for (int c = 0; c < L::kChunksD; ++c)
             tma_load_4d(sbase + L::kQ + s * L::kTileD + c * L::kChunk, &map_q, bar(L::kQFull + s),
-                        c * 64, h, qt * kTile, w.b);
+                        c * 64, h, w.q_off + qt * kTile, w.bt);
         }
         __syncwarp();
         ++q_it;
@@ -291,7 +323,7 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           mbar_arrive_expect_tx(bar(L::kOFull), L::kTileD);
           for (int c = 0; c < L::kChunksD; ++c)
             tma_load_4d(sbase + L::kDO + c * L::kChunk, &map_do, bar(L::kOFull), c * 64, h,
-                        qt * kTile, w.b);
+                        w.q_off + qt * kTile, w.bt);
         }
         __syncwarp();
         ++o_it;
@@ -460,12 +492,12 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         const int qt = pw.qtile(p, w, &partial);
         const int h = pw.head(w);
         const int q = qt * kTile + r;
-        const bool row_valid = q < p.f.Lq;
+        const bool row_valid = q < w.lq;
         float neg_lse2 = -INFINITY, drow = 0.f;
         if (row_valid) {
-          const float l = p.f.lse[(static_cast<int64_t>(w.b) * p.f.H + h) * p.f.Lq + q];
+          const float l = p.f.lse[qrow(p, w, h, q)];
           neg_lse2 = l == -INFINITY ? -INFINITY : -l * kLog2e;
-          drow = p.dvec[(static_cast<int64_t>(w.b) * p.f.H + h) * p.f.Lq + q];
+          drow = p.dvec[qrow(p, w, h, q)];
         }
         const bool live = row_valid && neg_lse2 != -INFINITY;
         // per-row mask parameters (as in the forward)
@@ -497,8 +529,8 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
             brow = reinterpret_cast<const uint8_t*>(p.f.bias.ptr) +
                    (w.b * p.f.bias.sb + hb * p.f.bias.sh + static_cast<int64_t>(qq) * p.f.bias.sq) * esz;
           }
-          if (k0 + kTile > p.f.Lk) lim = min(lim, p.f.Lk - k0);
-          if (p.f.causal) lim = min(lim, q + p.f.Lk - p.f.Lq - k0 + 1);
+          if (k0 + kTile > w.lk) lim = min(lim, w.lk - k0);
+          if (p.f.causal) lim = min(lim, q + w.lk - w.lq - k0 + 1);
         }
 
         // ---- phase A: P from S
@@ -646,12 +678,12 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const BUnit w = bwd_unit(p, u);
       const int key = w.kt * kTile + r;
-      OutT* dvrow = reinterpret_cast<OutT*>(p.dv) + w.b * p.dv_sb + static_cast<int64_t>(key) * p.dv_sr +
+      OutT* dvrow = reinterpret_cast<OutT*>(p.dv) + w.bt * p.dv_sb + static_cast<int64_t>(w.k_off + key) * p.dv_sr +
                     w.hk * p.dv_sh;
-      OutT* dkrow = reinterpret_cast<OutT*>(p.dk) + w.b * p.dk_sb + static_cast<int64_t>(key) * p.dk_sr +
+      OutT* dkrow = reinterpret_cast<OutT*>(p.dk) + w.bt * p.dk_sb + static_cast<int64_t>(w.k_off + key) * p.dk_sr +
                     w.hk * p.dk_sh;
       if (w.n_pairs == 0) {  // keys no query attends: zero gradients
-        if (key < p.f.Lk) {
+        if (key < w.lk) {
           for (int e = 0; e < D / 8; ++e) {
             reinterpret_cast<uint4*>(dvrow)[e] = make_uint4(0, 0, 0, 0);
             reinterpret_cast<uint4*>(dkrow)[e] = make_uint4(0, 0, 0, 0);
@@ -669,7 +701,8 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         if (!mbar_wait(bar(L::kDQFull), pit & 1, abort_flag, p.f.err)) { ok = false; break; }
         tc_fence_after();
         float4* acc = reinterpret_cast<float4*>(
-            p.dq_acc + ((static_cast<int64_t>(w.b) * p.f.Lq + q) * p.f.H + h) * D);
+            p.dq_acc + ((static_cast<int64_t>(w.bt) * (p.f.cu_q != nullptr ? p.f.total_q : p.f.Lq) +
+                         w.q_off + q) * p.f.H + h) * D);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
@@ -679,7 +712,7 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
             tc_fence_before();
             mbar_arrive(bar(L::kDQFree));
           }
-          if (q < p.f.Lq) {
+          if (q < w.lq) {
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               atomicAdd(acc + 8 * c + e,
@@ -702,7 +735,7 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           uint32_t v[32];
           tmem_ld32_at(col + 32 * c, v);
           tc_wait_ld();
-          if (key < p.f.Lk) {
+          if (key < w.lk) {
             uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -898,9 +931,9 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         mbar_arrive_expect_tx(bar(L::kKVFull), 2 * L::kTileD);
         for (int c = 0; c < 2; ++c) {
           tma_load_4d(sbase + L::kK + c * L::kChunk, &map_k, bar(L::kKVFull), c * 64, w.hk,
-                      w.kt * kTile, w.b);
+                      w.k_off + w.kt * kTile, w.bt);
           tma_load_4d(sbase + L::kV + c * L::kChunk, &map_v, bar(L::kKVFull), c * 64, w.hk,
-                      w.kt * kTile, w.b);
+                      w.k_off + w.kt * kTile, w.bt);
         }
       }
       __syncwarp();
@@ -921,7 +954,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           mbar_arrive_expect_tx(bar(L::kQFull + s), L::kTileD);
           for (int c = 0; c < 2; ++c)
             tma_load_4d(sbase + L::kQ + s * L::kTileD + c * L::kChunk, &map_q, bar(L::kQFull + s),
-                        c * 64, h, qt * kTile, w.b);
+                        c * 64, h, w.q_off + qt * kTile, w.bt);
         }
         __syncwarp();
         ++q_it;
@@ -933,7 +966,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           mbar_arrive_expect_tx(bar(L::kOFull), L::kTileD);
           for (int c = 0; c < 2; ++c)
             tma_load_4d(sbase + L::kDO + c * L::kChunk, &map_do, bar(L::kOFull), c * 64, h,
-                        qt * kTile, w.b);
+                        w.q_off + qt * kTile, w.bt);
         }
         __syncwarp();
         ++o_it;
@@ -973,8 +1006,8 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           n_l[j] = -INFINITY;
           d_v[j] = 0.f;
           clo[j] = chi[j] = dlo[j] = dhi[j] = 0;
-          if (q < p.f.Lq) {
-            const int64_t row = (static_cast<int64_t>(w.b) * p.f.H + h) * p.f.Lq + q;
+          if (q < w.lq) {
+            const int64_t row = qrow(p, w, h, q);
             const float l = p.f.lse[row];
             n_l[j] = l == -INFINITY ? -INFINITY : -l * kLog2e;
             d_v[j] = p.dvec[row];
@@ -1238,7 +1271,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
                 for (int z = 0; z < 32; ++z) {
                   const int q = q0 + cq + z;
                   const int qc = q < p.f.Lq ? q : 0;
-                  const bool keep = key < p.f.Lk && (!p.f.causal || key <= q + p.f.Lk - p.f.Lq) &&
+                  const bool keep = q < w.lq && key < w.lk && (!p.f.causal || key <= q + w.lk - w.lq) &&
                                     (!p.f.has_mask || mv[qc * msq] != 0);
                   kbits |= (keep ? 1u : 0u) << z;
                 }
@@ -1358,12 +1391,12 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const BUnit w = bwd_unit(p, u);
       const int key = w.kt * kTile + r;
-      OutT* dvrow = reinterpret_cast<OutT*>(p.dv) + w.b * p.dv_sb + static_cast<int64_t>(key) * p.dv_sr +
+      OutT* dvrow = reinterpret_cast<OutT*>(p.dv) + w.bt * p.dv_sb + static_cast<int64_t>(w.k_off + key) * p.dv_sr +
                     w.hk * p.dv_sh;
-      OutT* dkrow = reinterpret_cast<OutT*>(p.dk) + w.b * p.dk_sb + static_cast<int64_t>(key) * p.dk_sr +
+      OutT* dkrow = reinterpret_cast<OutT*>(p.dk) + w.bt * p.dk_sb + static_cast<int64_t>(w.k_off + key) * p.dk_sr +
                     w.hk * p.dk_sh;
       if (w.n_pairs == 0) {  // keys no query attends: zero gradients
-        if (key < p.f.Lk) {
+        if (key < w.lk) {
           for (int e = 0; e < D / 8; ++e) {
             reinterpret_cast<uint4*>(dvrow)[e] = make_uint4(0, 0, 0, 0);
             reinterpret_cast<uint4*>(dkrow)[e] = make_uint4(0, 0, 0, 0);
@@ -1405,7 +1438,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           fence_async_shared();
           __syncwarp();
           if (lane == 0) {
-            bulk_reduce_add_4d(&map_dq, stage, 32 * c, h, qt * kTile + 32 * wq, w.b);
+            bulk_reduce_add_4d(&map_dq, stage, 32 * c, h, w.q_off + qt * kTile + 32 * wq, w.bt);
             bulk_commit();
           }
           bulk_pending = true;
@@ -1425,7 +1458,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           uint32_t v[32];
           tmem_ld32_at(col + 32 * c, v);
           tc_wait_ld();
-          if (key < p.f.Lk) {
+          if (key < w.lk) {
             uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -1616,7 +1649,19 @@ cudaError_t launch_bwd_typed(const BwdProblem& p, const CUtensorMap& mq, const C
 
 }  // namespace
 
-cudaError_t launch_bwd_prep(const BwdProblem& p, cudaStream_t stream) {
+// Packed batches are one batch entry of total_q rows for the row-wise kernels
+// (their per-query arrays are [H, total_q], the dQ accumulator [total_q, H, d]).
+BwdProblem flat_view(const BwdProblem& p) {
+  BwdProblem f = p;
+  if (p.f.cu_q != nullptr) {
+    f.f.B = 1;
+    f.f.Lq = p.f.total_q;
+  }
+  return f;
+}
+
+cudaError_t launch_bwd_prep(const BwdProblem& pin, cudaStream_t stream) {
+  const BwdProblem p = flat_view(pin);
   const int64_t rows = static_cast<int64_t>(p.f.B) * p.f.Lq * p.f.H;
   const int block = 256;
   const unsigned grid = static_cast<unsigned>((rows * 32 + block - 1) / block);
@@ -1638,7 +1683,8 @@ cudaError_t launch_transpose_lists(const BwdProblem& p, uint8_t* codes, cudaStre
   return cudaGetLastError();
 }
 
-cudaError_t launch_dq_convert(const BwdProblem& p, cudaStream_t stream) {
+cudaError_t launch_dq_convert(const BwdProblem& pin, cudaStream_t stream) {
+  const BwdProblem p = flat_view(pin);
   const int64_t total = static_cast<int64_t>(p.f.B) * p.f.Lq * p.f.H * (p.f.d / 4);
   const unsigned grid = static_cast<unsigned>((total + 255) / 256);
   if (p.f.dtype == SMA_BF16) dq_convert_kernel<SMA_BF16><<<grid, 256, 0, stream>>>(p);
@@ -1649,14 +1695,17 @@ cudaError_t launch_dq_convert(const BwdProblem& p, cudaStream_t stream) {
 
 int launch_attn_bwd(const BwdProblem& p, cudaStream_t stream, char* msg, size_t msg_len) {
   const AttnProblem& f = p.f;
+  // packed batches: one batch entry of total_q (total_k) rows
+  const bool packed = f.cu_q != nullptr;
+  const int lq = packed ? f.total_q : f.Lq, lk = packed ? f.total_k : f.Lk, nb = packed ? 1 : f.B;
   CUtensorMap mq, mk, mv, mdo;
-  if (!encode_map(&mq, f.q, f.dtype, f.d, f.H, f.Lq, f.B, f.q_sh, f.q_sr, f.q_sb, msg, msg_len) ||
-      !encode_map(&mk, f.k, f.dtype, f.d, f.KVH, f.Lk, f.B, f.k_sh, f.k_sr, f.k_sb, msg, msg_len) ||
-      !encode_map(&mv, f.v, f.dtype, f.d, f.KVH, f.Lk, f.B, f.v_sh, f.v_sr, f.v_sb, msg, msg_len) ||
-      !encode_map(&mdo, p.dout, f.dtype, f.d, f.H, f.Lq, f.B, p.do_sh, p.do_sr, p.do_sb, msg, msg_len))
+  if (!encode_map(&mq, f.q, f.dtype, f.d, f.H, lq, nb, f.q_sh, f.q_sr, f.q_sb, msg, msg_len) ||
+      !encode_map(&mk, f.k, f.dtype, f.d, f.KVH, lk, nb, f.k_sh, f.k_sr, f.k_sb, msg, msg_len) ||
+      !encode_map(&mv, f.v, f.dtype, f.d, f.KVH, lk, nb, f.v_sh, f.v_sr, f.v_sb, msg, msg_len) ||
+      !encode_map(&mdo, p.dout, f.dtype, f.d, f.H, lq, nb, p.do_sh, p.do_sr, p.do_sb, msg, msg_len))
     return SMA_ERR_CUDA;
   CUtensorMap mdq;
-  if (f.d == 128 && !encode_map_f32(&mdq, p.dq_acc, f.d, f.H, f.Lq, f.B, 32, 32, msg, msg_len))
+  if (f.d == 128 && !encode_map_f32(&mdq, p.dq_acc, f.d, f.H, lq, nb, 32, 32, msg, msg_len))
     return SMA_ERR_CUDA;
   cudaError_t e = cudaErrorInvalidValue;
   const bool bf = f.dtype == SMA_BF16;

@@ -1187,6 +1187,98 @@ sma_status varlen_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   return ok();
 }
 
+sma_status varlen_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t total_q,
+                                          int32_t max_q, int32_t max_k, int32_t head_dim,
+                                          size_t* bytes) {
+  if (bytes == nullptr) return fail(SMA_ERR_INVALID_ARG, "bytes is NULL");
+  if (batch < 1 || heads < 1 || total_q < 1 || max_q < 1 || max_k < 1 || head_dim < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, heads, total_q, maxima and head_dim must be >= 1");
+  const int QT = static_cast<int>(ceil_div(max_q, kTile));
+  const int KT = static_cast<int>(ceil_div(max_k, kTile));
+  // lists per sequence; per-query data and the dQ accumulator over the packed rows
+  *bytes = bwd_layout(0, batch, QT, KT, 1, heads, total_q, head_dim).total;
+  return ok();
+}
+
+sma_status varlen_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t head_dim, int32_t total_q, int32_t total_k, int32_t max_q,
+                           int32_t max_k, float scale, int32_t is_causal, const int32_t* cu_seqlens_q,
+                           const int32_t* cu_seqlens_k, const void* q, const int64_t q_strides[2],
+                           const void* k, const int64_t k_strides[2], const void* v,
+                           const int64_t v_strides[2], const void* out, const int64_t o_strides[2],
+                           const float* lse, const void* dout, const int64_t do_strides[2],
+                           void* dq, const int64_t dq_strides[2], void* dk,
+                           const int64_t dk_strides[2], void* dv, const int64_t dv_strides[2],
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  sma_status s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (batch < 1 || total_q < 1 || total_k < 1 || max_q < 1 || max_k < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, totals and maxima must be >= 1");
+  if (is_causal != 0 && is_causal != 1) return fail(SMA_ERR_INVALID_ARG, "is_causal must be 0 or 1");
+  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr)
+    return fail(SMA_ERR_INVALID_ARG, "cu_seqlens_q / cu_seqlens_k are NULL");
+  const int64_t* s2[7] = {q_strides, k_strides, v_strides, o_strides, do_strides, dq_strides, dk_strides};
+  for (const int64_t* a : s2)
+    if (a == nullptr) return fail(SMA_ERR_INVALID_ARG, "strides are NULL");
+  if (dv_strides == nullptr) return fail(SMA_ERR_INVALID_ARG, "strides are NULL");
+  // [rows, heads, d] operands as one batch entry: strides {0, row, head}
+  const int64_t qs[3] = {0, q_strides[0], q_strides[1]}, ks[3] = {0, k_strides[0], k_strides[1]};
+  const int64_t vs[3] = {0, v_strides[0], v_strides[1]}, os[3] = {0, o_strides[0], o_strides[1]};
+  const int64_t gs[3] = {0, do_strides[0], do_strides[1]}, dqs[3] = {0, dq_strides[0], dq_strides[1]};
+  const int64_t dks[3] = {0, dk_strides[0], dk_strides[1]}, dvs[3] = {0, dv_strides[0], dv_strides[1]};
+  if ((s = check_operand("q", q, qs, dtype, total_q)) != SMA_OK) return s;
+  if ((s = check_operand("k", k, ks, dtype, total_k)) != SMA_OK) return s;
+  if ((s = check_operand("v", v, vs, dtype, total_k)) != SMA_OK) return s;
+  if ((s = check_grad_operands(dtype, total_q, total_k, out, os, lse, dout, gs, dq, dqs, dk, dks, dv,
+                               dvs)) != SMA_OK)
+    return s;
+  size_t need = 0;
+  if ((s = varlen_attn_bwd_workspace_size(batch, heads, total_q, max_q, max_k, head_dim, &need)) !=
+      SMA_OK)
+    return s;
+  if ((s = check_workspace(workspace, workspace_bytes, need)) != SMA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (err == nullptr) return cuda_fail(e, "device error word unavailable");
+  const int QT = static_cast<int>(ceil_div(max_q, kTile));
+  const int KT = static_cast<int>(ceil_div(max_k, kTile));
+  const BwdLayout lay = bwd_layout(0, batch, QT, KT, 1, heads, total_q, head_dim);
+  BwdProblem b{};
+  AttnProblem& p = b.f;
+  p.dtype = dtype;
+  p.B = batch; p.H = heads; p.KVH = kv_heads; p.Lq = max_q; p.Lk = max_k; p.d = head_dim;
+  p.group = heads / kv_heads;
+  p.npairs = (p.group + 1) / 2;
+  p.QT = QT; p.KT = KT;
+  const float sc = resolve_scale(scale, head_dim);
+  p.scale_log2 = sc * kLog2eHost;
+  p.q = q; p.q_sb = 0; p.q_sr = qs[1]; p.q_sh = qs[2];
+  p.k = k; p.k_sb = 0; p.k_sr = ks[1]; p.k_sh = ks[2];
+  p.v = v; p.v_sb = 0; p.v_sr = vs[1]; p.v_sh = vs[2];
+  p.o = const_cast<void*>(out); p.o_sb = 0; p.o_sr = os[1]; p.o_sh = os[2];
+  p.lse = const_cast<float*>(lse);
+  p.policy = kPolicyVarlen;
+  p.causal = is_causal;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.err = err;
+  p.lists.LB = batch; p.lists.LH = 1; p.lists.head_mode = 0;
+  int32_t* nf = at<int32_t>(workspace, lay.fl.nf);
+  int32_t* np = at<int32_t>(workspace, lay.fl.np);
+  int32_t* fi = at<int32_t>(workspace, lay.fl.fi);
+  int32_t* pi = at<int32_t>(workspace, lay.fl.pi);
+  p.lists.num_full = nf; p.lists.num_part = np; p.lists.full_idx = fi; p.lists.part_idx = pi;
+  e = launch_varlen_lists(p, nf, fi, np, pi, st);
+  if (e != cudaSuccess) return cuda_fail(e, "tile list launch failed");
+  set_grads(b, dout, gs, dq, dqs, dk, dks, dv, dvs, sc);
+  if ((s = run_backward(b, workspace, lay, st)) != SMA_OK) return s;
+  return ok();
+}
+
 static sma_status check_pad_args(int32_t dtype, int32_t batch, int32_t max_len, int32_t heads,
                                  int32_t head_dim, const int32_t* cu, const void* packed,
                                  const int64_t* p_strides, const void* padded,

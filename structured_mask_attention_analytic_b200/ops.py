@@ -442,6 +442,37 @@ def varlen_attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
     return out, lse
 
 
+def varlen_attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                    max_seqlen_k: int, is_causal: bool = False, scale=None, dq=None, dk=None, dv=None,
+                    workspace=None):
+    """Gradients of ``varlen_attn_fwd`` (same sequences, causal flag and
+    scale): ``out`` and ``lse`` are that call's results, ``dout`` the upstream
+    gradient ``[total_q, H, d]``.  Returns ``(dq, dk, dv)`` in the packed
+    layouts of q and k."""
+    _require_cuda(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k)
+    total_q, h, dh = q.shape
+    total_k, kvh = k.shape[0], k.shape[1]
+    b = cu_seqlens_q.shape[0] - 1
+    cq, ck = _cu(cu_seqlens_q), _cu(cu_seqlens_k, b)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (h, total_q) or not lse.is_contiguous():
+        raise ValueError("lse must be the forward's contiguous float32 [heads, total_q]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(k) if dv is None else dv
+    n = ctypes.c_size_t()
+    nat.check(_lib().varlen_attn_bwd_workspace_size(b, h, total_q, int(max_seqlen_q), int(max_seqlen_k), dh,
+                                                    ctypes.byref(n)))
+    if workspace is None:
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=q.device)
+    nat.check(_lib().varlen_attn_bwd(
+        _dtype_code(q), b, h, kvh, dh, total_q, total_k, int(max_seqlen_q), int(max_seqlen_k),
+        ctypes.c_float(0.0 if scale is None else float(scale)), 1 if is_causal else 0,
+        _ptr(cq), _ptr(ck), _ptr(q), _strides2(q), _ptr(k), _strides2(k), _ptr(v), _strides2(v),
+        _ptr(out), _strides2(out), _ptr(lse), _ptr(dout), _strides2(dout), _ptr(dq), _strides2(dq),
+        _ptr(dk), _strides2(dk), _ptr(dv), _strides2(dv), _ptr(workspace), workspace.numel(), _stream(q)))
+    return dq, dk, dv
+
+
 def varlen_pad(packed: torch.Tensor, cu_seqlens: torch.Tensor, max_len: int) -> torch.Tensor:
     """``[batch, max_len, H, d]`` from packed ``[total, H, d]`` rows (zeros past each length)."""
     _require_cuda(packed, cu_seqlens)

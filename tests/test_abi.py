@@ -237,6 +237,12 @@ def test_varlen_validation_on_host():
     lib = nat.load()
     n = ctypes.c_size_t()
     assert lib.varlen_attn_fwd_workspace_size(4, 1000, 2000, ctypes.byref(n)) == 0
+    nf = n.value
+    # backward: the same lists plus their transpose, rowsum(dO * O) and the
+    # fp32 dQ accumulator over the packed rows
+    assert lib.varlen_attn_bwd_workspace_size(4, 8, 3000, 1000, 2000, 128, ctypes.byref(n)) == 0
+    assert n.value >= nf + 3000 * 8 * 4 + 3000 * 8 * 128 * 4
+    assert lib.varlen_attn_bwd_workspace_size(0, 8, 3000, 1000, 2000, 128, ctypes.byref(n)) == nat.SMA_ERR_INVALID_ARG
     assert n.value >= 2 * 4 * 8 * 16 * 4          # full and partial index arrays
     st = lib.varlen_attn_fwd(2, 2, 4, 2, 128, 100, 100, 60, 60, ctypes.c_float(0.0), 0,
                              ctypes.c_void_p(0x100), ctypes.c_void_p(0x200),

@@ -98,3 +98,50 @@ def test_malformed_offsets_are_reported():
     assert sma.device_status() == 6   # SMA_ERR_DEVICE_INPUT
     assert sma.device_status() == 0
     assert (out[:120] == 7.0).all()   # the malformed sequence's rows are left untouched
+
+
+# Gradient agreement as for the padded backward: relative to m = max(1,
+# max |ref|) of each tensor, max-abs <= 2.5e-2 m and mean-abs <= 2.5e-3 m.
+def _close_grad(name, got, ref):
+    g = f64(got)
+    m = max(1.0, float(np.abs(ref).max()))
+    err = np.abs(g - ref)
+    assert np.isfinite(g).all(), f"{name}: non-finite"
+    assert err.max() <= 2.5e-2 * m, f"{name}: max abs err {err.max():.3e} (scale {m:.2f})"
+    assert err.mean() <= 2.5e-3 * m, f"{name}: mean abs err {err.mean():.3e} (scale {m:.2f})"
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("D,dtype", [(128, "bf16"), (64, "bf16"), (128, "fp16")])
+def test_varlen_backward(causal, D, dtype):
+    """dQ, dK, dV of packed sequences against the float64 gradients of each
+    sequence on its own: lengths spanning several tiles and ragged tails, one
+    query over 40 keys, an empty sequence, different query and key lengths
+    (bottom-right causal), and tiles that straddle sequence boundaries."""
+    from oracle import attention_grad as ag
+    rng = wl.rng_for(61)
+    H, KVH = 8, 2
+    lq = [130, 1, 257, 0, 100, 64]
+    lk = [130, 40, 257, 0, 300, 64]
+    cu_q, cu_k, q, k, v = _case(rng, lq, lk, H, KVH, D, dtype)
+    do = wl.normal(rng, tuple(q.shape), dtype)
+    cq, ck = torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda()
+    qc, kc, vc, dc = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    out, lse = sma.varlen_attn_fwd(qc, kc, vc, cq, ck, max(lq), max(lk), causal)
+    dq, dk, dv = sma.varlen_attn_bwd(qc, kc, vc, out, lse, dc, cq, ck, max(lq), max(lk), causal)
+    torch.cuda.synchronize()
+    assert sma.device_status() == 0
+    rq = np.zeros(tuple(q.shape))
+    rk = np.zeros(tuple(k.shape))
+    rv = np.zeros(tuple(k.shape))
+    for i in range(len(lq)):
+        q0, q1, k0, k1 = cu_q[i], cu_q[i + 1], cu_k[i], cu_k[i + 1]
+        if q1 == q0 or k1 == k0:
+            continue
+        keep = at.causal_keep(q1 - q0, k1 - k0)[None, None] if causal else None
+        gq, gk, gv, _ = ag.attention_grad(f64(q[q0:q1])[None], f64(k[k0:k1])[None], f64(v[k0:k1])[None],
+                                          f64(do[q0:q1])[None], keep=keep)
+        rq[q0:q1], rk[k0:k1], rv[k0:k1] = gq[0], gk[0], gv[0]
+    _close_grad("dq", dq, rq)
+    _close_grad("dk", dk, rk)
+    _close_grad("dv", dv, rv)
