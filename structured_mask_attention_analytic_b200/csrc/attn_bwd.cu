@@ -1283,17 +1283,23 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
             for (int e = 0; e < 32; e += 4) {
               const float4 n4 = *reinterpret_cast<const float4*>(nl + cq + e);
               const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
-              float pv[4];
+              float xs[4], pv[4];
   #pragma unroll
               for (int z = 0; z < 4; ++z) {
-                float x = __uint_as_float(xr[e + z]);
+                xs[z] = __uint_as_float(xr[e + z]);
                 if (POLICY != kPolicyDflash && p.f.has_bias) {
                   const int q = q0 + cq + e + z;
                   const int qc = q < p.f.Lq ? q : 0;  // rows past Lq read row 0 (their P is 0)
-                  x = fmaf(load_any_as_float(bcol + qc * bsq, bdt, 0), bias_mul, x);
+                  xs[z] = fmaf(load_any_as_float(bcol + qc * bsq, bdt, 0), bias_mul, xs[z]);
                 }
-                pv[z] = ((kbits >> (e + z)) & 1u) ? fast_exp2(fmaf(x, scale_log2, nn[z])) : 0.f;
               }
+              // exponent arguments two at a time (packed fp32 pairs)
+              const float2 sl2 = make_float2(scale_log2, scale_log2);
+              const float2 t01 = fma2(make_float2(xs[0], xs[1]), sl2, make_float2(nn[0], nn[1]));
+              const float2 t23 = fma2(make_float2(xs[2], xs[3]), sl2, make_float2(nn[2], nn[3]));
+              const float ts[4] = {t01.x, t01.y, t23.x, t23.y};
+  #pragma unroll
+              for (int z = 0; z < 4; ++z) pv[z] = ((kbits >> (e + z)) & 1u) ? fast_exp2(ts[z]) : 0.f;
               pk[e >> 1] = DT == SMA_BF16 ? pack_bf16x2(pv[0], pv[1]) : pack_f16x2(pv[0], pv[1]);
               pk[(e >> 1) + 1] = DT == SMA_BF16 ? pack_bf16x2(pv[2], pv[3]) : pack_f16x2(pv[2], pv[3]);
             }
@@ -1334,10 +1340,12 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
               const float4 d4 = *reinterpret_cast<const float4*>(dd + cq + e);
               const float2 p01 = unpack2<DT>(pr[e >> 1]);
               const float2 p23 = unpack2<DT>(pr[(e >> 1) + 1]);
-              const float s0 = p01.x * (__uint_as_float(yr[e]) - d4.x);
-              const float s1 = p01.y * (__uint_as_float(yr[e + 1]) - d4.y);
-              const float s2 = p23.x * (__uint_as_float(yr[e + 2]) - d4.z);
-              const float s3 = p23.y * (__uint_as_float(yr[e + 3]) - d4.w);
+              // dS = P (dP - D), two at a time (packed fp32 pairs)
+              const float2 s01 = mul2(p01, sub2(make_float2(__uint_as_float(yr[e]), __uint_as_float(yr[e + 1])),
+                                                make_float2(d4.x, d4.y)));
+              const float2 s23 = mul2(p23, sub2(make_float2(__uint_as_float(yr[e + 2]), __uint_as_float(yr[e + 3])),
+                                                make_float2(d4.z, d4.w)));
+              const float s0 = s01.x, s1 = s01.y, s2 = s23.x, s3 = s23.y;
               pk[e >> 1] = DT == SMA_BF16 ? pack_bf16x2(s0, s1) : pack_f16x2(s0, s1);
               pk[(e >> 1) + 1] = DT == SMA_BF16 ? pack_bf16x2(s2, s3) : pack_f16x2(s2, s3);
               if (MODE == kDbiasRowSum) {
