@@ -322,8 +322,9 @@ sma_status dynamic_topk_mask(int32_t bias_dtype, const void* bias, const int64_t
  * dq        [B, Lq, H, d]; dk, dv [B, Lk, KVH, d]: written, caller-owned,
  *           strides as for q/k/v (last dim contiguous, 16-byte multiples).
  * dtype     SMA_BF16 or SMA_FP16 (tensor cores, fp32 accumulation; dQ is
- *           accumulated in fp32 in the workspace); SMA_FP32 returns
- *           SMA_ERR_UNSUPPORTED.  head_dim 64 or 128.
+ *           accumulated in fp32 in the workspace), or SMA_FP32 (fp32 FFMA
+ *           throughout, the gradients of the fp32 forward; no tensor cores,
+ *           a correctness path).  head_dim 64 or 128.
  * The workspace holds the tile lists, rowsum(dO * O) and the fp32 dQ
  * accumulator (B * Lq * H * d * 4 bytes); query its size first.
  * ---------------------------------------------------------------------- */

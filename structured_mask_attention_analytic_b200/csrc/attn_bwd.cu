@@ -1703,6 +1703,14 @@ cudaError_t launch_dq_convert(const BwdProblem& pin, cudaStream_t stream) {
 
 int launch_attn_bwd(const BwdProblem& p, cudaStream_t stream, char* msg, size_t msg_len) {
   const AttnProblem& f = p.f;
+  if (f.dtype == SMA_FP32) {  // FFMA path (no tensor maps)
+    const cudaError_t e = launch_attn_bwd_simt(p, stream);
+    if (e != cudaSuccess) {
+      snprintf(msg, msg_len, "fp32 attention backward launch failed: %s", cudaGetErrorString(e));
+      return SMA_ERR_CUDA;
+    }
+    return SMA_OK;
+  }
   // packed batches: one batch entry of total_q (total_k) rows
   const bool packed = f.cu_q != nullptr;
   const int lq = packed ? f.total_q : f.Lq, lk = packed ? f.total_k : f.Lk, nb = packed ? 1 : f.B;

@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsma.so")
 
-SOURCES = ["runtime.cu", "tile_maps.cu", "attn_tc.cu", "attn_simt.cu", "decode.cu", "topk.cu", "gather.cu", "tma_map.cu", "attn_bwd.cu", "varlen.cu",
+SOURCES = ["runtime.cu", "tile_maps.cu", "attn_tc.cu", "attn_simt.cu", "decode.cu", "topk.cu", "gather.cu", "tma_map.cu", "attn_bwd.cu", "attn_bwd_simt.cu", "varlen.cu",
            "noalloc.cu", "sma_api.cpp"]
 HEADERS = ["device_common.cuh", "kernels.h", "gather.cuh", "tma_map.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

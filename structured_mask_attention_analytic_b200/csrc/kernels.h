@@ -245,6 +245,9 @@ cudaError_t launch_bwd_prep(const BwdProblem& p, cudaStream_t stream);
 cudaError_t launch_transpose_lists(const BwdProblem& p, uint8_t* codes, cudaStream_t stream);
 int launch_attn_bwd(const BwdProblem& p, cudaStream_t stream, char* msg, size_t msg_len);
 cudaError_t launch_dq_convert(const BwdProblem& p, cudaStream_t stream);
+// fp32 FFMA backward (dQ accumulator, dK, dV, dbias), after launch_bwd_prep
+// and launch_transpose_lists; launch_dq_convert follows.
+cudaError_t launch_attn_bwd_simt(const BwdProblem& p, cudaStream_t stream);
 
 // Records `message` as the calling thread's last error (read back through
 // sma_last_error) and returns `code`.

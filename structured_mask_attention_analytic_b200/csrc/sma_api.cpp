@@ -315,8 +315,6 @@ sma_status check_grad_operands(int32_t dtype, int64_t lq, int64_t lk, const void
                                const void* dk, const int64_t* dk_strides, const void* dv,
                                const int64_t* dv_strides) {
   sma_status s;
-  if (dtype == SMA_FP32)
-    return fail(SMA_ERR_UNSUPPORTED, "the backward runs on the tensor cores: bf16 or fp16 only");
   if ((s = check_operand("out", out, o_strides, dtype, lq)) != SMA_OK) return s;
   if ((s = check_operand("dout", dout, do_strides, dtype, lq)) != SMA_OK) return s;
   if ((s = check_operand("dq", dq, dq_strides, dtype, lq)) != SMA_OK) return s;
@@ -1213,6 +1211,8 @@ sma_status varlen_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   sma_status s = check_heads(heads, kv_heads, head_dim);
   if (s != SMA_OK) return s;
+  if (dtype == SMA_FP32)
+    return fail(SMA_ERR_UNSUPPORTED, "varlen attention runs on the tensor cores: bf16 or fp16 only");
   if (batch < 1 || total_q < 1 || total_k < 1 || max_q < 1 || max_k < 1)
     return fail(SMA_ERR_INVALID_ARG, "batch, totals and maxima must be >= 1");
   if (is_causal != 0 && is_causal != 1) return fail(SMA_ERR_INVALID_ARG, "is_causal must be 0 or 1");

@@ -225,7 +225,13 @@ def test_backward_workspace_and_validation_on_host():
             ctypes.c_void_p(0x90000), nat.i64_array(ks), ctypes.c_void_p(dbias),
             ctypes.c_void_p(0xa0000), 1 << 30, None)
 
-    assert call(dtype=2) == nat.SMA_ERR_UNSUPPORTED
+    # packed batches have no fp32 backward: rejected before anything runs
+    s2 = nat.i64_array([1024, 128])
+    assert lib.varlen_attn_bwd(2, 2, 8, 2, 128, 100, 100, 64, 64, ctypes.c_float(0.0), 0,
+                               ctypes.c_void_p(0x10000), ctypes.c_void_p(0x11000),
+                               *([ctypes.c_void_p(0x20000), s2] * 4), ctypes.c_void_p(0x70000),
+                               *([ctypes.c_void_p(0x20000), s2] * 4), ctypes.c_void_p(0xa0000),
+                               1 << 30, None) == nat.SMA_ERR_UNSUPPORTED
     assert "bf16 or fp16" in lib.sma_last_error().decode()
     assert call(lse=0) == nat.SMA_ERR_INVALID_ARG
     assert "lse" in lib.sma_last_error().decode()

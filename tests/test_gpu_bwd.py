@@ -131,8 +131,59 @@ def test_fp16_and_rejections():
     _close("dq", dq, rq)
     _close("dk", dk, rk)
     _close("dv", dv, rv)
-    with pytest.raises(sma.SmaError, match="bf16 or fp16"):
-        sma.masked_attn_bwd(qc.float(), kc.float(), vc.float(), out.float(), lse, dc.float())
+
+
+def _close_fp32(name, got, ref):
+    """fp32 FFMA gradients: max-abs <= 1e-4 m, mean-abs <= 1e-5 m (m as above)."""
+    g = f64(got)
+    m = max(1.0, float(np.abs(ref).max()))
+    err = np.abs(g - ref)
+    assert err.max() <= 1e-4 * m, f"{name}: max abs err {err.max():.3e} (scale {m:.2f})"
+    assert err.mean() <= 1e-5 * m, f"{name}: mean abs err {err.mean():.3e} (scale {m:.2f})"
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp32_masked_backward_with_bias_and_dbias(d):
+    """fp32 inputs take the FFMA backward: explicit mask (PARTIAL tiles), a
+    per-query-head bias (per-element dbias) and causal masking."""
+    rng = wl.rng_for(37)
+    q = wl.normal(rng, (B, LQ, H, d), "fp32")
+    k = wl.normal(rng, (B, LK, KVH, d), "fp32")
+    v = wl.normal(rng, (B, LK, KVH, d), "fp32")
+    do = wl.normal(rng, (B, LQ, H, d), "fp32")
+    mask = torch.from_numpy(rng.random((1, 1, LQ, KP)) < 0.7)
+    bias = wl.normal(rng, (1, H, 1, KP), "fp32")
+    qc, kc, vc, dc, mc, bc = (t.cuda() for t in (q, k, v, do, mask, bias))
+    out, lse = sma.masked_attn_fwd(qc, kc, vc, mc, bc, True)
+    dq, dk, dv, db = sma.masked_attn_bwd(qc, kc, vc, out, lse, dc, mc, bc, True, return_dbias=True)
+    torch.cuda.synchronize()
+    assert sma.device_status() == 0
+    keep = at.aux_view(mask.numpy(), H, KVH, LK) & at.causal_keep(LQ, LK)[None, None]
+    bb = at.aux_view(f64(bias), H, KVH, LK)
+    rq, rk, rv, rdb = ag.attention_grad(f64(q), f64(k), f64(v), f64(do), keep=keep, bias=bb,
+                                        dbias_shape=tuple(bias.shape), workers=8)
+    _close_fp32("dq", dq, rq)
+    _close_fp32("dk", dk, rk)
+    _close_fp32("dv", dv, rv)
+    _close_fp32("dbias", db, rdb)
+
+
+def test_fp32_dflash_backward():
+    """fp32 inputs, DFlash sliding layer (in-block causal, window 40)."""
+    Lc, bs = 200, 16
+    q, k, v, do, anchors = _dflash_case(38, 2, 4, 2, 64, Lc, 12, bs, None, 1, 40, "fp32")
+    causal = dm.resolve_in_block_causal(None, 1)
+    w = dm.resolve_window(1, 40)
+    qc, kc, vc, dc, ac = (t.cuda() for t in (q, k, v, do, anchors))
+    out, lse = sma.dfa_attn_fwd(qc, kc, vc, ac, Lc, bs, None, 1, 40)
+    dq, dk, dv = sma.dfa_attn_bwd(qc, kc, vc, out, lse, dc, ac, Lc, bs, None, 1, 40)
+    torch.cuda.synchronize()
+    assert sma.device_status() == 0
+    keep = dm.dflash_keep_mask(anchors.numpy(), Lc, bs, causal, w)[:, None]
+    rq, rk, rv, _ = ag.attention_grad(f64(q), f64(k), f64(v), f64(do), keep=keep, workers=8)
+    _close_fp32("dq", dq, rq)
+    _close_fp32("dk", dk, rk)
+    _close_fp32("dv", dv, rv)
 
 
 DB_SHAPES = [(B, H, LQ, KP), (B, KVH, LQ, KP), (1, 1, LQ, KP), (B, H, 1, KP), (1, KVH, 1, KP),
