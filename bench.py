@@ -394,7 +394,16 @@ def run_details(sma, dev, stream, peaks, only=None):
         tf = tile_flops(128, 32, kept) / (ms * 1e-3) / 1e12
         out["varlen_causal_12seq"] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / pk_t, "tokens": total,
                                       "kept_tiles_per_head": kept}
-        del q, k, v, o
+        # backward of the same batch: 5 products per kept tile (2.5x the forward's work)
+        o, lse = sma.varlen_attn_fwd(q, k, v, cu, cu, max(lens), max(lens), True, out=o)
+        do = torch.randn(q.shape, device=dev, generator=g).to(torch.bfloat16)
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+        ms_b = timed(lambda: sma.varlen_attn_bwd(q, k, v, o, lse, do, cu, cu, max(lens), max(lens), True,
+                                                 dq=grads[0], dk=grads[1], dv=grads[2]), stream, 5, 2)
+        tf_b = 2.5 * tile_flops(128, 32, kept) / (ms_b * 1e-3) / 1e12
+        out["varlen_causal_12seq_bwd"] = {"ms": ms_b, "TFLOP/s": tf_b, "frac_bf16_peak": tf_b / pk_t,
+                                          "status": sma.device_status()}
+        del q, k, v, o, do, grads
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     if want("broadcast_prefill"):
