@@ -117,6 +117,22 @@ class ClockSampler:
 # ---------------------------------------------------------------- helpers
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The job's time: the slowest rank's, returned on every rank (one
+    all-reduce; a single process returns its own)."""
+    if world <= 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank: float, ms_per_step: float) -> float:
+    """Units per second of the whole job: every rank processes its own
+    units_per_rank each step (replicas, weak scaling) in ms_per_step."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
+
+
 def timed(fn, stream, reps, warmup):
     """Average ms of fn() over reps, CUDA events on `stream`."""
     for _ in range(warmup):
@@ -249,12 +265,9 @@ def run_ours(args, rank, world, dev):
     total_ms = t0.elapsed_time(t1)
     attn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
     map_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = job_throughput(world, flops, ms_per_step) / 1e12
     attn_avg = sum(attn_ms) / len(attn_ms)
     achieved = flops / (attn_avg * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
@@ -282,7 +295,8 @@ def run_ours(args, rank, world, dev):
         e_ms = timed(e2e_step, stream, args.e2e_steps, 2)
         h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, ah))
         d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
-        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+        e_ms = max_over_ranks(e_ms, world, dev)
+        e2e = {"value": job_throughput(world, flops, e_ms) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
         del qh, kh, vh, oh
 
