@@ -14,7 +14,7 @@ Sources
 * Same page, maintainer reply, item 1 (#934): the in-block sliding window
   keeps only its left bound.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 * keys are laid out as ``concat(context[0:Lc], block_0, ..., block_{N-1})``;
 * query ``i`` of block ``j`` sits at position ``anchor_j + i``; context key
   ``k`` sits at position ``k``; the window keeps a key iff

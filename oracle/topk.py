@@ -12,7 +12,7 @@ are never selected; a 2D mask of length key_len becomes ``(B, 1, 1, K)``, one
 of length query_len is padded or cut to key_len.  Changes: the sentinel is
 the minimum finite value of the *bias* dtype.
 
-Readings (listed in DESIGN.md):
+Readings where the pages are silent or loose:
 * only columns ``k < Lk`` take part; padded columns are never selected;
 * equal values are ordered by lower key index first (the page's selection is
   unsorted, so ties are left open there); ``-0.0 == +0.0``;
