@@ -8,9 +8,9 @@ from oracle import attention as at
 from oracle import dflash_mask as dm
 from oracle import tiles as tl
 
-# Agreement required of attention outputs (fixed by the benchmark spec for
-# this library): bf16/fp16 inputs max-abs <= 2e-2 and mean-abs <= 2e-3; fp32
-# inputs max-abs <= 1e-4.
+# Agreement required of attention outputs (the library's stated accuracy;
+# the pages fix none): bf16/fp16 inputs max-abs <= 2e-2 and mean-abs <= 2e-3;
+# fp32 inputs max-abs <= 1e-4.
 TOL = {torch.bfloat16: (2e-2, 2e-3), torch.float16: (2e-2, 2e-3), torch.float32: (1e-4, 1e-4)}
 # log-sum-exp is compared with the same absolute bounds scaled by 5 (lse is
 # O(log Lk) in magnitude, computed in fp32 from bf16-rounded scores).
