@@ -244,12 +244,12 @@ def test_varlen_validation_on_host():
     n = ctypes.c_size_t()
     assert lib.varlen_attn_fwd_workspace_size(4, 1000, 2000, ctypes.byref(n)) == 0
     nf = n.value
+    assert nf >= 2 * 4 * 8 * 16 * 4          # full and partial index arrays
     # backward: the same lists plus their transpose, rowsum(dO * O) and the
     # fp32 dQ accumulator over the packed rows
     assert lib.varlen_attn_bwd_workspace_size(4, 8, 3000, 1000, 2000, 128, ctypes.byref(n)) == 0
     assert n.value >= nf + 3000 * 8 * 4 + 3000 * 8 * 128 * 4
     assert lib.varlen_attn_bwd_workspace_size(0, 8, 3000, 1000, 2000, 128, ctypes.byref(n)) == nat.SMA_ERR_INVALID_ARG
-    assert n.value >= 2 * 4 * 8 * 16 * 4          # full and partial index arrays
     st = lib.varlen_attn_fwd(2, 2, 4, 2, 128, 100, 100, 60, 60, ctypes.c_float(0.0), 0,
                              ctypes.c_void_p(0x100), ctypes.c_void_p(0x200),
                              ctypes.c_void_p(0x10000), nat.i64_array([512, 128]),
@@ -266,3 +266,23 @@ def test_varlen_validation_on_host():
                              ctypes.c_void_p(0x40000), nat.i64_array([512, 128]), None,
                              ctypes.c_void_p(0x50000), 1 << 20, None)
     assert st == nat.SMA_ERR_INVALID_ARG and "cu_seqlens" in lib.sma_last_error().decode()
+
+
+def test_varlen_backward_validation_on_host():
+    """varlen_attn_bwd rejects a short workspace, a missing lse and missing
+    offsets before anything runs (fake, never dereferenced pointers)."""
+    lib = nat.load()
+    qs, ks = nat.i64_array([512, 128]), nat.i64_array([256, 128])
+
+    def call(ws_bytes=1 << 30, lse=0x60000, cu=0x100):
+        return lib.varlen_attn_bwd(
+            0, 2, 4, 2, 128, 100, 100, 60, 60, ctypes.c_float(0.0), 1,
+            ctypes.c_void_p(cu), ctypes.c_void_p(0x200),
+            ctypes.c_void_p(0x10000), qs, ctypes.c_void_p(0x20000), ks, ctypes.c_void_p(0x30000), ks,
+            ctypes.c_void_p(0x40000), qs, ctypes.c_void_p(lse), ctypes.c_void_p(0x50000), qs,
+            ctypes.c_void_p(0x70000), qs, ctypes.c_void_p(0x80000), ks, ctypes.c_void_p(0x90000), ks,
+            ctypes.c_void_p(0xa0000), ws_bytes, None)
+
+    assert call(ws_bytes=256) == nat.SMA_ERR_WORKSPACE
+    assert call(lse=0) == nat.SMA_ERR_INVALID_ARG and "lse" in lib.sma_last_error().decode()
+    assert call(cu=0) == nat.SMA_ERR_INVALID_ARG and "cu_seqlens" in lib.sma_last_error().decode()
