@@ -128,3 +128,29 @@ def test_matches_float64_autograd():
     np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-12)
     np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-12)
     np.testing.assert_allclose(db, tb.grad.numpy(), atol=1e-12)
+
+
+def test_per_sequence_gradients_equal_block_diagonal_mask():
+    """Packed sequences' gradients, computed one sequence at a time (how the
+    packed backward's parity test builds its reference), equal the gradients
+    of the concatenated batch under the block-diagonal keep mask with
+    bottom-right causality inside each block."""
+    rng = np.random.default_rng(21)
+    lq, lk = [3, 5, 2], [4, 5, 6]
+    H, KVH, d = 4, 2, 3
+    cq, ck = np.cumsum([0] + lq), np.cumsum([0] + lk)
+    q = rng.standard_normal((1, cq[-1], H, d))
+    k = rng.standard_normal((1, ck[-1], KVH, d))
+    v = rng.standard_normal((1, ck[-1], KVH, d))
+    do = rng.standard_normal((1, cq[-1], H, d))
+    keep = np.zeros((1, 1, cq[-1], ck[-1]), dtype=bool)
+    for i in range(3):
+        keep[0, 0, cq[i]:cq[i + 1], ck[i]:ck[i + 1]] = at.causal_keep(lq[i], lk[i])
+    dq, dk, dv, _ = ag.attention_grad(q, k, v, do, keep=keep)
+    for i in range(3):
+        s_q, s_k = slice(cq[i], cq[i + 1]), slice(ck[i], ck[i + 1])
+        gq, gk, gv, _ = ag.attention_grad(q[:, s_q], k[:, s_k], v[:, s_k], do[:, s_q],
+                                          keep=at.causal_keep(lq[i], lk[i])[None, None])
+        np.testing.assert_allclose(dq[:, s_q], gq, atol=1e-13)
+        np.testing.assert_allclose(dk[:, s_k], gk, atol=1e-13)
+        np.testing.assert_allclose(dv[:, s_k], gv, atol=1e-13)
