@@ -286,3 +286,19 @@ def test_varlen_backward_validation_on_host():
     assert call(ws_bytes=256) == nat.SMA_ERR_WORKSPACE
     assert call(lse=0) == nat.SMA_ERR_INVALID_ARG and "lse" in lib.sma_last_error().decode()
     assert call(cu=0) == nat.SMA_ERR_INVALID_ARG and "cu_seqlens" in lib.sma_last_error().decode()
+
+
+def test_sparse_workspace_includes_key_range_segments_for_short_queries():
+    """16 queries over compacted keys: the group's 4 heads share a tile, so
+    2 units on a 148-SM part, and the index-gather workspace also holds the
+    key-range split's partial results (32 segments, the cap)."""
+    lib = nat.load()
+    n_short, n_long = ctypes.c_size_t(), ctypes.c_size_t()
+    ms = nat.i64_array([1, 2, 1, 20096])
+    assert lib.sparse_attn_fwd_workspace_size(0, 1, 8, 2, 16, 20000, 128, ms, 0, None, 0,
+                                              ctypes.byref(n_short)) == 0
+    assert lib.sparse_attn_fwd_workspace_size(0, 1, 8, 2, 4096, 20000, 128, ms, 0, None, 0,
+                                              ctypes.byref(n_long)) == 0
+    segments = 32                       # 148 // 2 = 74 per unit, at most 157 // 4, at most 32
+    rows = 1 * 8 * 16
+    assert n_short.value >= segments * rows * (128 * 4 + 8)
