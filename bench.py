@@ -147,11 +147,41 @@ def timed(fn, stream, reps, warmup):
     return s.elapsed_time(e) / reps
 
 
-# DRAM bytes (read + write) of one attention launch of a workload, from one
-# ncu capture of dram__bytes_read.sum / dram__bytes_write.sum on the current
-# attn_tc_kernel (profiles/attn_tc_dflash_long_full_traffic.md).  Remove an
-# entry when that kernel changes.
-MEASURED_TRAFFIC = {"dflash_long_full": 2.11e9 + 0.24844e9}
+# Committed ncu summaries of the headline kernel's DRAM traffic carry two
+# machine-readable lines: the bytes (read + write) of one launch and a
+# SHA-256 of the kernel's sources when the counters were taken.  The figure is
+# reported only while the sources still hash the same; once the kernel
+# changes it is stale and roofline.traffic is null.
+KERNEL_SOURCES = ("structured_mask_attention_analytic_b200/csrc/attn_tc.cu",
+                  "structured_mask_attention_analytic_b200/csrc/device_common.cuh")
+
+
+def kernel_source_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload_name: str):
+    """(bytes per launch, profile file) from profiles/attn_tc_<workload>_traffic.md
+    if it was captured on the current kernel sources, else (None, reason)."""
+    path = os.path.join(ROOT, "profiles", f"attn_tc_{workload_name}_traffic.md")
+    if not os.path.exists(path):
+        return None, "no ncu traffic summary for this workload"
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.startswith("- "):
+                key, val = line[2:].split(":", 1)
+                vals[key.strip()] = val.strip().strip("`")
+    if "traffic_bytes_per_launch" not in vals or "kernel_source_sha256" not in vals:
+        return None, "summary lacks traffic_bytes_per_launch / kernel_source_sha256"
+    if vals["kernel_source_sha256"] != kernel_source_sha256():
+        return None, "stale: kernel sources changed since the capture"
+    return float(vals["traffic_bytes_per_launch"]), os.path.relpath(path, ROOT)
 
 
 def timed_graph(fn, reps, warmup):
@@ -271,6 +301,10 @@ def run_ours(args, rank, world, dev):
     attn_avg = sum(attn_ms) / len(attn_ms)
     achieved = flops / (attn_avg * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
+    if args.traffic_bytes is not None:
+        traffic, traffic_src = args.traffic_bytes, "--traffic-bytes"
+    else:
+        traffic, traffic_src = measured_traffic(w.name)
 
     # end to end: host buffers in pinned memory, copies inside the timed region
     e2e = None
@@ -316,8 +350,7 @@ def run_ours(args, rank, world, dev):
                                   "kept_tiles": kept, "flops_per_step": flops}),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
-                     "traffic": args.traffic_bytes if args.traffic_bytes is not None
-                     else MEASURED_TRAFFIC.get(w.name),
+                     "traffic": traffic, "traffic_source": traffic_src,
                      "kernel": "attn_tc_kernel<128, DFlash, bf16>",
                      "peak_source": f"{peak_src} bf16 dense burst",
                      "frac_of_spec_2250": achieved / 2250.0,

@@ -215,9 +215,11 @@ sma_status dfa_attn_fwd(const dfa_mask_desc* desc, const int32_t* anchors, int32
  * (about batch * q_tiles * (kv_tiles + 1) * 8 bytes; the 32768-query,
  * 65536-key long-context problem needs 1.05 MB).  Calls share the array:
  * calls that may overlap on the GPU (unordered streams) race, so order them
- * on one stream.  The first call on a device looks up the array's address
- * with that device current; make it before any stream capture starts.  No
- * device memory is allocated or freed. */
+ * on one stream.  The first call in a CUDA context looks up the array's
+ * address with that context current and caches it per context; make it
+ * before any stream capture starts.  A new context (after cudaDeviceReset,
+ * or a caller's own non-primary context) repeats the lookup on its first
+ * call.  No device memory is allocated or freed. */
 sma_status dfa_attn_fwd_noalloc(const dfa_mask_desc* desc, const int32_t* anchors, int32_t dtype,
                                 int32_t heads, int32_t kv_heads, int32_t head_dim, float scale,
                                 const void* q, const int64_t q_strides[3], const void* k,

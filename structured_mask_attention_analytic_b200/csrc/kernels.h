@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace sma {
 
 constexpr int kTile = 128;
@@ -256,8 +258,27 @@ int set_last_error(int code, const char* message);
 cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, int* err, int64_t* out,
                                          cudaStream_t stream);
 
-// Device error word of the current device.
+// Device error word in the current context (looked up once per context).
 int* device_error_word(cudaError_t* status);
+
+// Unique id of the CUDA context current on the calling thread (ids are never
+// reused within a process, so a context created after cudaDeviceReset, or a
+// caller's own non-primary context, gets a new one); 0 if none is current.
+unsigned long long current_context_id();
+
+// Device addresses of a __device__ symbol per CUDA context.  A symbol's
+// address belongs to the context the module is loaded in: it is not valid in
+// another context of the same device, nor after the context is destroyed.
+struct ContextAddressCache {
+  static constexpr int kSlots = 64;
+  std::mutex mutex;
+  unsigned long long ids[kSlots] = {};
+  void* ptrs[kSlots] = {};
+  int count = 0;
+  unsigned next_evict = 0;
+  void* find(unsigned long long ctx_id);  // nullptr if not cached (or ctx_id 0)
+  void insert(unsigned long long ctx_id, void* ptr);
+};
 
 int num_sms();
 

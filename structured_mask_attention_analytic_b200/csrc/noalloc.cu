@@ -22,14 +22,16 @@
 //   same time on the GPU (e.g. on two streams without ordering between them)
 //   race on it; order them on one stream.  Nothing in the array needs to start
 //   at zero: each call rewrites every entry it later reads.
-// * The first call on a device looks the array's device address up (with that
-//   device current) and caches it; make that first call before any stream
-//   capture begins.
+// * The first call in a CUDA context looks the array's device address up
+//   (with that context current) and caches it for that context; make that
+//   first call before any stream capture begins.  A new context (after
+//   cudaDeviceReset, or a caller's own non-primary context) gets its own
+//   lookup on its first call, since the address belongs to the context the
+//   library's module is loaded in.
 // * No cudaMalloc, cudaFree or other allocating routine is called.
 #include <cuda_runtime.h>
 
 #include <cstdio>
-#include <mutex>
 
 #include "kernels.h"
 #include "sma.h"
@@ -46,9 +48,7 @@ constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 // address; the address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_dfa_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
+sma::ContextAddressCache g_scratch_cache;
 
 }  // namespace
 
@@ -73,25 +73,17 @@ extern "C" sma_status dfa_attn_fwd_noalloc(const dfa_mask_desc* desc, const int3
              need, kNoAllocScratchBytes);
     return sma::set_last_error(SMA_ERR_WORKSPACE, msg);
   }
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    return sma::set_last_error(SMA_ERR_CUDA, "dfa_attn_fwd_noalloc: no usable current device");
-  }
-  void* ptr = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (g_scratch_ptr[dev] == nullptr) {
-      e = cudaGetSymbolAddress(&ptr, g_dfa_scratch);
-      if (e != cudaSuccess || ptr == nullptr) {
-        char msg[256];
-        snprintf(msg, sizeof(msg), "dfa_attn_fwd_noalloc: cudaGetSymbolAddress failed: %s",
-                 cudaGetErrorString(e));
-        return sma::set_last_error(SMA_ERR_CUDA, msg);
-      }
-      g_scratch_ptr[dev] = ptr;
+  void* ptr = g_scratch_cache.find(sma::current_context_id());
+  if (ptr == nullptr) {
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_dfa_scratch);
+    if (e != cudaSuccess || ptr == nullptr) {
+      char msg[256];
+      snprintf(msg, sizeof(msg), "dfa_attn_fwd_noalloc: cudaGetSymbolAddress failed: %s",
+               cudaGetErrorString(e));
+      return sma::set_last_error(SMA_ERR_CUDA, msg);
     }
-    ptr = g_scratch_ptr[dev];
+    // the lookup makes the device's primary context current if none was
+    g_scratch_cache.insert(sma::current_context_id(), ptr);
   }
   return dfa_attn_fwd(desc, anchors, dtype, heads, kv_heads, head_dim, scale, q, q_strides, k,
                       k_strides, v, v_strides, out, o_strides, lse, nullptr, ptr,

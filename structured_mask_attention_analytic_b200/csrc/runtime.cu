@@ -1,5 +1,7 @@
-// Per-device state of the library: the device error word kernels report
+// Per-context state of the library: the device error word kernels report
 // into, and the SM count used to size persistent grids.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "device_common.cuh"
@@ -11,30 +13,71 @@ namespace {
 __device__ int g_device_error;
 
 constexpr int kMaxDevices = 64;
-int* g_error_ptr[kMaxDevices] = {nullptr};
 int g_sm_count[kMaxDevices] = {0};
 std::mutex g_mutex;
+ContextAddressCache g_error_cache;
+
+PFN_cuCtxGetCurrent_v4000 g_ctx_get_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_get_id = nullptr;
+std::once_flag g_ctx_fns_once;
+
+void load_ctx_fns() {
+  cudaDriverEntryPointQueryResult q;
+  void* f = nullptr;
+  if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+  f = nullptr;
+  if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+}
 }  // namespace
 
+unsigned long long current_context_id() {
+  std::call_once(g_ctx_fns_once, load_ctx_fns);
+  if (g_ctx_get_current == nullptr || g_ctx_get_id == nullptr) return 0;
+  CUcontext c = nullptr;
+  if (g_ctx_get_current(&c) != CUDA_SUCCESS || c == nullptr) return 0;
+  unsigned long long id = 0;
+  if (g_ctx_get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+void* ContextAddressCache::find(unsigned long long ctx_id) {
+  if (ctx_id == 0) return nullptr;
+  std::lock_guard<std::mutex> lock(mutex);
+  for (int i = 0; i < count; ++i)
+    if (ids[i] == ctx_id) return ptrs[i];
+  return nullptr;
+}
+
+void ContextAddressCache::insert(unsigned long long ctx_id, void* ptr) {
+  if (ctx_id == 0) return;
+  std::lock_guard<std::mutex> lock(mutex);
+  for (int i = 0; i < count; ++i)
+    if (ids[i] == ctx_id) {
+      ptrs[i] = ptr;
+      return;
+    }
+  const int slot = count < kSlots ? count++ : static_cast<int>(next_evict++ % kSlots);
+  ids[slot] = ctx_id;
+  ptrs[slot] = ptr;
+}
+
 int* device_error_word(cudaError_t* status) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    if (status) *status = e != cudaSuccess ? e : cudaErrorInvalidDevice;
-    return nullptr;
-  }
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_error_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_device_error);
-    if (e != cudaSuccess) {
-      if (status) *status = e;
+  void* p = g_error_cache.find(current_context_id());
+  if (p == nullptr) {
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_device_error);
+    if (e != cudaSuccess || p == nullptr) {
+      if (status) *status = e != cudaSuccess ? e : cudaErrorInvalidSymbol;
       return nullptr;
     }
-    g_error_ptr[dev] = static_cast<int*>(p);
+    // the lookup makes the device's primary context current if none was
+    g_error_cache.insert(current_context_id(), p);
   }
   if (status) *status = cudaSuccess;
-  return g_error_ptr[dev];
+  return static_cast<int*>(p);
 }
 
 namespace {
