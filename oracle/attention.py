@@ -48,14 +48,21 @@ def aux_view(aux: np.ndarray, n_heads: int, n_kv_heads: int, n_k: int) -> np.nda
     """Turn a 4D mask/bias of the broadcast contract into an array that numpy
     broadcasts against ``[B, H, Lq, Lk]``.
 
-    ``aux`` has shape ``(b', h', q', K)`` with ``K >= n_k``; only the first
-    ``n_k`` columns are used.  A head dim equal to ``n_kv_heads`` (and not to
-    ``n_heads``) is indexed with the query head's KV head ``h // (H // KVH)``;
-    size-1 dims broadcast.
+    ``aux`` has shape ``(b', h', q', K)`` with ``K >= n_k`` (the padded
+    ``round_up(n_k, 128)`` or ``n_k`` itself), of which only the first ``n_k``
+    columns are used, or ``K == 1``: one value for every key, expanded over
+    the ``n_k`` keys as the page's interface expands a key dim of 1.  A head
+    dim equal to ``n_kv_heads`` (and not to ``n_heads``) is indexed with the
+    query head's KV head ``h // (H // KVH)``; size-1 dims broadcast.
     """
     if aux.ndim != 4:
         raise ValueError("mask/bias must be 4D")
-    x = aux[..., :n_k]
+    if aux.shape[-1] == 1:
+        x = np.broadcast_to(aux, aux.shape[:-1] + (n_k,))
+    elif aux.shape[-1] >= n_k:
+        x = aux[..., :n_k]
+    else:
+        raise ValueError("mask/bias key dim must be >= Lk or 1")
     h_aux = x.shape[1]
     if h_aux not in (1, n_heads, n_kv_heads):
         raise ValueError("mask/bias head dim must be 1, H or KVH")

@@ -80,9 +80,10 @@ def attention_grad(q, k, v, do, *, keep=None, keep_rows=None, bias=None, scale=N
 
     q, do: ``[B, Lq, H, d]``; k, v: ``[B, Lk, KVH, d]``.  keep / keep_rows /
     bias / scale as in ``attention``.  ``dbias_shape``: the 4D shape of the
-    bias as the caller holds it ``(b', h', q', K)`` with ``K >= Lk``; dbias is
-    reduced onto that shape (columns >= Lk are 0).  A head dim equal to KVH
-    (when KVH != H) sums the heads of each group.
+    bias as the caller holds it ``(b', h', q', K)`` with ``K >= Lk`` or
+    ``K == 1``; dbias is reduced onto that shape (columns >= Lk are 0; a key
+    dim of 1, one bias value for every key, sums dS over the keys as well).
+    A head dim equal to KVH (when KVH != H) sums the heads of each group.
     Returns ``dq [B, Lq, H, d], dk [B, Lk, KVH, d], dv [B, Lk, KVH, d]`` and
     ``dbias`` (None without ``dbias_shape``).
     """
@@ -123,8 +124,8 @@ def attention_grad(q, k, v, do, *, keep=None, keep_rows=None, bias=None, scale=N
     dbias = None
     if dbias_shape is not None:
         sb, sh, sq, kk = dbias_shape
-        if kk < n_k:
-            raise ValueError("dbias key dim must be at least Lk")
+        if kk < n_k and kk != 1:
+            raise ValueError("dbias key dim must be at least Lk, or 1")
         dbias = np.zeros(dbias_shape)
     for b, h, q0, q1, gq, gk, gv, ds in results:
         hk = h // group
@@ -139,8 +140,10 @@ def attention_grad(q, k, v, do, *, keep=None, keep_rows=None, bias=None, scale=N
                 hi = hk
             else:
                 hi = 0
+            if kk == 1 and n_k > 1:           # one bias value for every key
+                ds = ds.sum(axis=1, keepdims=True)
             if sq > 1:
-                dbias[bi, hi, q0:q1, :n_k] += ds
+                dbias[bi, hi, q0:q1, :ds.shape[1]] += ds
             else:
-                dbias[bi, hi, 0, :n_k] += ds.sum(axis=0)
+                dbias[bi, hi, 0, :ds.shape[1]] += ds.sum(axis=0)
     return dq, dk, dv, dbias

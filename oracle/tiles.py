@@ -88,8 +88,11 @@ def block_map_from_rows(keep_rows, n_batch: int, n_q: int, n_k: int, tile: int =
 def mask_tile_summary(mask: np.ndarray, n_k: int, tile: int = TILE) -> np.ndarray:
     """Codes of an explicit 4D bool mask at its own (broadcast) shape:
     ``uint8 [b', h', ceil(q'/tile), ceil(n_k/tile)]``; columns >= n_k count
-    as not kept."""
+    as not kept.  A key dim of 1 is one flag for every key (expanded over the
+    n_k keys)."""
     mask = np.asarray(mask, dtype=bool)
+    if mask.shape[-1] == 1:
+        mask = np.broadcast_to(mask, mask.shape[:-1] + (n_k,))
     b_, h_, q_, _ = mask.shape
     out = np.zeros((b_, h_, -(-q_ // tile), -(-n_k // tile)), dtype=np.uint8)
     for i in range(b_):

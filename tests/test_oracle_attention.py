@@ -250,3 +250,40 @@ def test_varlen_equals_block_diagonal_mask(causal):
     np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(ref_lse[0]))
     fin = ~np.isneginf(lse)
     np.testing.assert_allclose(lse[fin], ref_lse[0][fin], atol=1e-13)
+
+
+def test_key_dim_forms_of_mask_and_bias(qkv):
+    """The three key dims of PR #190's interface (padded to a multiple of 128
+    there; padded, Lk, or 1 which the interface expands).  A mask/bias of key
+    dim Lk equals the padded one's first Lk columns; a key dim of 1 equals its
+    explicit expansion over the keys.  A bias that is one value c per row
+    shifts every score of the row alike: the output is that of no bias at all
+    and lse grows by exactly c (softmax is shift invariant).  A one-column
+    mask keeps a row whole or kills it."""
+    q, k, v = qkv
+    b, lq, h, _ = q.shape
+    kvh, lk = k.shape[2], k.shape[1]
+    rng = np.random.default_rng(5)
+    pad = rng.standard_normal((b, kvh, lq, 64))
+    mpad = rng.random((b, kvh, lq, 64)) < 0.7
+    mpad[..., 0] = True
+    o1, l1 = at.attention(q, k, v, keep=at.aux_view(mpad, h, kvh, lk), bias=at.aux_view(pad, h, kvh, lk))
+    o2, l2 = at.attention(q, k, v, keep=at.aux_view(np.ascontiguousarray(mpad[..., :lk]), h, kvh, lk),
+                          bias=at.aux_view(np.ascontiguousarray(pad[..., :lk]), h, kvh, lk))
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+    c = rng.standard_normal((b, h, lq, 1)) * 3.0
+    o_c, l_c = at.attention(q, k, v, bias=at.aux_view(c, h, kvh, lk))
+    o_x, l_x = at.attention(q, k, v, bias=np.repeat(c, lk, axis=-1))
+    np.testing.assert_array_equal(o_c, o_x)
+    np.testing.assert_array_equal(l_c, l_x)
+    o_0, l_0 = at.attention(q, k, v)
+    np.testing.assert_allclose(o_c, o_0, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l_c, l_0 + c[..., 0], rtol=0, atol=1e-12)
+
+    flag = rng.random((1, 1, lq, 1)) < 0.5
+    o_f, l_f = at.attention(q, k, v, keep=at.aux_view(flag, h, kvh, lk))
+    rows = flag[0, 0, :, 0]
+    np.testing.assert_array_equal(o_f[:, rows], o_0[:, rows])
+    assert np.all(o_f[:, ~rows] == 0.0) and np.all(l_f[:, :, ~rows] == -np.inf)

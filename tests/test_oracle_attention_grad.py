@@ -154,3 +154,43 @@ def test_per_sequence_gradients_equal_block_diagonal_mask():
         np.testing.assert_allclose(dq[:, s_q], gq, atol=1e-13)
         np.testing.assert_allclose(dk[:, s_k], gk, atol=1e-13)
         np.testing.assert_allclose(dv[:, s_k], gv, atol=1e-13)
+
+
+def test_dbias_key_dim_forms():
+    """dbias at the bias's own key dim.  Key dim Lk: the padded dbias's first
+    Lk columns.  Key dim 1 (one value for every key of a row): the gradient of
+    a shift shared by every score of the row, which is exactly zero
+    (sum_k P (dP - D) = D - D), while dQ, dK and dV equal those without the
+    bias (softmax ignores the shift); also equal to the full-shape dbias of
+    the expanded bias summed over the keys, and to torch autograd."""
+    q, k, v, do, keep, bias_pad = _case(15, (2, 2, 5, 8))
+    lk = 7
+    pad = ag.attention_grad(q, k, v, do, keep=keep, bias=at.aux_view(bias_pad, 4, 2, lk),
+                            dbias_shape=bias_pad.shape)
+    unp = np.ascontiguousarray(bias_pad[..., :lk])
+    got = ag.attention_grad(q, k, v, do, keep=keep, bias=at.aux_view(unp, 4, 2, lk), dbias_shape=unp.shape)
+    for a, b in zip(pad[:3], got[:3]):
+        np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(pad[3][..., :lk], got[3])
+
+    rng = np.random.default_rng(16)
+    c = rng.standard_normal((2, 4, 5, 1)) * 2.0
+    dq, dk, dv, db = ag.attention_grad(q, k, v, do, keep=keep, bias=at.aux_view(c, 4, 2, lk),
+                                       dbias_shape=c.shape)
+    assert db.shape == c.shape and np.abs(db).max() < 1e-12
+    nq, nk, nv, _ = ag.attention_grad(q, k, v, do, keep=keep)
+    np.testing.assert_allclose(dq, nq, atol=1e-12)
+    np.testing.assert_allclose(dk, nk, atol=1e-12)
+    np.testing.assert_allclose(dv, nv, atol=1e-12)
+    full = np.repeat(c, lk, axis=-1)
+    _, _, _, dfull = ag.attention_grad(q, k, v, do, keep=keep, bias=full, dbias_shape=full.shape)
+    np.testing.assert_allclose(db[..., 0], dfull.sum(axis=-1), atol=1e-12)
+    tq = torch.tensor(q)
+    tc = torch.tensor(c, requires_grad=True)
+    kk = torch.tensor(k).repeat_interleave(2, dim=2)
+    vv = torch.tensor(v).repeat_interleave(2, dim=2)
+    s = torch.einsum("bqhd,bkhd->bhqk", tq, kk) / math.sqrt(3) + tc
+    s = s.masked_fill(~torch.from_numpy(keep), float("-inf"))
+    o = torch.einsum("bhqk,bkhd->bqhd", torch.softmax(s, dim=-1).nan_to_num(0.0), vv)
+    (o * torch.from_numpy(do)).sum().backward()
+    np.testing.assert_allclose(db, tc.grad.numpy(), atol=1e-12)

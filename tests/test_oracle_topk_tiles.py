@@ -169,3 +169,22 @@ def test_block_map_codes_agree_with_mask_content():
                 is_part = kt in pi[b, qt, : npart[b, qt]]
                 assert is_full == (blk.all() and (kt + 1) * 128 <= n_k)
                 assert (is_full or is_part) == bool(blk.any())
+
+
+def test_key_dim_forms_of_summary_and_topk():
+    """A mask of key dim 1 is one flag for every key: its summary equals that
+    of the explicit expansion.  A top-k bias of key dim Lk gives the padded
+    bias's mask, first Lk columns."""
+    rng = np.random.default_rng(21)
+    flags = rng.random((2, 1, 300, 1)) < 0.5
+    flags[0, 0, :128] = True
+    flags[1, 0, 128:256] = False
+    np.testing.assert_array_equal(tl.mask_tile_summary(flags, 333),
+                                  tl.mask_tile_summary(np.repeat(flags, 384, axis=-1), 333))
+    sent = float(np.finfo(np.float32).min)
+    bias = rng.standard_normal((2, 2, 3, 384)).astype(np.float32)
+    pm = rng.random((2, 1, 1, 333)) < 0.9
+    a = tk.dynamic_topk_keep(bias, 333, pm, 50, sent)
+    b = tk.dynamic_topk_keep(np.ascontiguousarray(bias[..., :333]), 333, pm, 50, sent)
+    assert b.shape == (2, 2, 3, 333)
+    np.testing.assert_array_equal(a[..., :333], b)
