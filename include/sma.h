@@ -102,6 +102,14 @@ sma_status sma_device_status(void* stream, int32_t* device_error);
  * method; it checks the failure-reporting path without faulting the GPU. */
 sma_status sma_selftest_wait_timeout(int64_t timeout_ns, int64_t* dev_out, void* stream);
 
+/* Diagnostic: dev_out[i] = 2^dev_in[i] (device float32 arrays of n floats,
+ * n even) as the attention softmax computes it on the FMA pipe for part of
+ * each row: t = round(t) + f, 2^f from a cubic (relative error <= 7.5e-5 on
+ * f in [-1/2, 1/2]), 2^round(t) added to the exponent field.  Arguments below
+ * -125 are clamped to -125 (so -inf gives 2^-125, not 0).  Not part of the
+ * method; it lets a test compare this exponential with CUDA's. */
+sma_status sma_selftest_exp2(const float* dev_in, float* dev_out, int64_t n, void* stream);
+
 /* ------------------------------------------------------------------------
  * DFlash mask description.
  *
@@ -234,12 +242,18 @@ sma_status dfa_attn_fwd_noalloc(const dfa_mask_desc* desc, const int32_t* anchor
  * 128-rounded key length, stride-0 broadcasting, and dbias reductions",
  * Design and Changes sections.  mask (uint8 0/1, True = keep) and bias
  * (additive, SMA_BF16/SMA_FP16/SMA_FP32) are rank 4 with sizes
- *   ({batch|1}, {heads|kv_heads|1}, {q_len|1}, round_up(k_len, 128))
+ *   ({batch|1}, {heads|kv_heads|1}, {q_len|1}, {round_up(k_len, 128)|k_len|1})
  * and a contiguous last dim (stride 1).  Size-1 dims broadcast with stride 0
  * whatever stride is passed; there is no implicit 3D form.  A head dim of
  * kv_heads (when kv_heads != heads) is indexed by the query head's KV head.
- * Columns in [k_len, round_up(k_len,128)) are never read as meaningful: they
- * are never attended whatever they hold.
+ * Key dim: the page's interface pads it to round_up(k_len, 128) and expands
+ * a key dim of 1 before its kernels run; here all three forms are read in
+ * place, with no copy.  Columns in [k_len, round_up(k_len,128)) are never
+ * read as meaningful: they are never attended whatever they hold.  A key dim
+ * of 1 is one value for every key (its last-dim stride is ignored).
+ * Alignment: base address and the batch / head / query strides must be
+ * multiples of 16 bytes (vector loads), except for a key dim of 1, which is
+ * read one element at a time and needs only element alignment.
  * ---------------------------------------------------------------------- */
 
 /* Tile codes of an explicit mask at its own broadcast shape:
@@ -289,13 +303,15 @@ sma_status masked_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
  * the BIAS dtype before choosing the window_size largest entries of each row,
  * so they are never selected.
  *
- * bias      [b, h, q, round_up(k_len,128)] dtype bias_dtype, strides given,
- *           last dim contiguous.  Only columns < k_len take part.
+ * bias      [b, h, q, kc] dtype bias_dtype, strides given, last dim
+ *           contiguous, kc = round_up(k_len,128) or k_len (a key dim of 1 is
+ *           refused: the output has one column per key).  Only columns
+ *           < k_len take part.
  * pre_mask  NULL or uint8 0/1 4D with sizes (pb, ph, pq, pk): pb in {1, b},
  *           ph in {1, h}, pq in {1, q}, pk >= 1, last stride 1; columns
  *           >= pk are invalid.  A 2D (batch, k_len) pre-mask is passed as
  *           sizes (batch, 1, 1, k_len).
- * out_mask  uint8 [b, h, q, round_up(k_len,128)] contiguous (device); columns
+ * out_mask  uint8 [b, h, q, kc] contiguous (device), 8-byte aligned; columns
  *           >= k_len are written 0.
  * Per row: entry k is kept iff it is among the window_size largest masked
  * values (equal values: lower k first; -0 equals +0) and the pre-mask keeps
@@ -353,11 +369,14 @@ sma_status masked_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t 
  *
  * dbias (nullable; device, 16-byte aligned, caller-owned): the bias gradient
  * of PR #190 (Changes, mha_bwd), written as contiguous float32 with the
- * bias's own sizes (b', h', q', round_up(k_len, 128)).  Element (b, h, q, k)
- * of dS = P * (dP - D) (the gradient of the score, bias included) is summed
- * into the dbias element its bias element broadcast from: over the batch
- * when b' = 1, over the heads of a group when h' = kv_heads, over all heads
- * when h' = 1, over the queries when q' = 1.  Columns >= k_len come out 0.
+ * bias's own sizes (b', h', q', kd), kd the bias's key dim.  Element
+ * (b, h, q, k) of dS = P * (dP - D) (the gradient of the score, bias
+ * included) is summed into the dbias element its bias element broadcast
+ * from: over the batch when b' = 1, over the heads of a group when
+ * h' = kv_heads, over all heads when h' = 1, over the queries when q' = 1,
+ * over the keys when kd = 1.  Columns >= k_len come out 0.  With kd = 1 (one
+ * bias value for every key of a row) the sum over the row's keys is exactly
+ * 0 (sum_k P (dP - D) = D - D): the call writes zeros.
  * The call zeroes dbias first; sums over broadcast dims use fp32 atomic
  * adds, so their rounding order is not fixed.  Needs a bias (
  * SMA_ERR_INVALID_ARG otherwise). */

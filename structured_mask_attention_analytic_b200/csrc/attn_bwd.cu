@@ -192,26 +192,6 @@ __device__ __forceinline__ uint32_t sw128_unit(uint32_t base, int r, int u) {
   return base + static_cast<uint32_t>((u >> 3) * (kTile * 128) + r * 128 + (((u & 7) ^ (r & 7)) << 4));
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void fence_async_shared() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 template <int DT>
 __device__ __forceinline__ float2 unpack2(uint32_t w) {
   if (DT == SMA_BF16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
@@ -551,7 +531,8 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           if (POLICY != kPolicyDflash && p.f.has_bias) {
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              x[e] = fmaf(load_any_as_float(brow, p.f.bias.dtype, k0 + 32 * c + e), bias_mul, x[e]);
+              x[e] = fmaf(load_any_as_float(brow, p.f.bias.dtype, aux_col(k0 + 32 * c + e, p.f.bias.kd)),
+                          bias_mul, x[e]);
           }
           uint32_t pk[16];
 #pragma unroll
@@ -566,7 +547,7 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
                   const int k = k0 + cc;
                   keep = keep && ((k >= clo && k < chi) || (k >= dlo && k < dhi));
                 } else {
-                  keep = keep && cc < lim && (!p.f.has_mask || mrow[k0 + cc] != 0);
+                  keep = keep && cc < lim && (!p.f.has_mask || mrow[aux_col(k0 + cc, p.f.mask.kd)] != 0);
                 }
               }
               pv[z] = keep ? fast_exp2(fmaf(x[e + z], scale_log2, neg_lse2)) : 0.f;
@@ -623,7 +604,7 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
               st_shared_v4(sw128_unit(sbase + L::kDS, r, 4 * c + v4), pk[4 * v4], pk[4 * v4 + 1],
                            pk[4 * v4 + 2], pk[4 * v4 + 3]);
             if (MODE == kDbiasStore || MODE == kDbiasAdd) {
-              if (row_valid) {
+              if (row_valid && k0 + kTile <= p.db_kd && p.db_kd % 4 == 0) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                   const float4 v =
@@ -631,6 +612,14 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
                   float4* dst = reinterpret_cast<float4*>(dbrow + 32 * c + 4 * j);
                   if (MODE == kDbiasStore) *dst = v;
                   else atomicAdd(dst, v);
+                }
+              } else if (row_valid) {  // a dbias row of Lk columns: element by element, inside it
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                  if (k0 + 32 * c + e < p.db_kd) {
+                    if (MODE == kDbiasStore) dbrow[32 * c + e] = dsv[e];
+                    else atomicAdd(dbrow + 32 * c + e, dsv[e]);
+                  }
                 }
               }
             } else if (MODE == kDbiasRowSum) {
@@ -646,7 +635,7 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
                   dsv[i] = keep + __shfl_xor_sync(0xffffffffu, send, wd);
                 }
               }
-              atomicAdd(dbrow + 32 * c + lane, dsv[0]);
+              if (k0 + 32 * c + lane < p.db_kd) atomicAdd(dbrow + 32 * c + lane, dsv[0]);
             }
           }
         };
@@ -1217,7 +1206,8 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         if (POLICY != kPolicyDflash) {
           if (p.f.has_mask) {
             const int hm = p.f.mask.head_per_query ? h : w.hk;
-            mcol = reinterpret_cast<const uint8_t*>(p.f.mask.ptr) + w.b * p.f.mask.sb + hm * p.f.mask.sh + key;
+            mcol = reinterpret_cast<const uint8_t*>(p.f.mask.ptr) + w.b * p.f.mask.sb + hm * p.f.mask.sh +
+                   aux_col(key, p.f.mask.kd);
             msq = p.f.mask.sq;
           }
           if (p.f.has_bias) {
@@ -1225,7 +1215,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
             bdt = p.f.bias.dtype;
             const int esz = bdt == SMA_FP32 ? 4 : 2;
             bcol = reinterpret_cast<const uint8_t*>(p.f.bias.ptr) +
-                   (w.b * p.f.bias.sb + hb * p.f.bias.sh + key) * esz;
+                   (w.b * p.f.bias.sb + hb * p.f.bias.sh + aux_col(key, p.f.bias.kd)) * esz;
             bsq = p.f.bias.sq * esz;
           }
         }
@@ -1322,8 +1312,11 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         // dbias: this thread's key column of dS over its 64 queries, added
         // where the bias broadcasts (or stored where each element is its own)
         float* dbcol = nullptr;
+        // (a dbias row of Lk columns has none for this thread's key past it)
+        const bool db_key = key < p.db_kd;
         if (POLICY != kPolicyDflash && p.db_mode != kDbiasNone)
-          dbcol = p.dbias + w.b * p.db_sb + (p.db_head_per_query ? h : w.hk) * p.db_sh + key;
+          dbcol = p.dbias + w.b * p.db_sb + (p.db_head_per_query ? h : w.hk) * p.db_sh +
+                  (db_key ? key : 0);
         auto phase_b = [&](auto mode_tag) {
           constexpr int MODE = decltype(mode_tag)::value;
           float rsum = 0.f;
@@ -1355,7 +1348,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
 #pragma unroll
                 for (int z = 0; z < 4; ++z) {
                   const int q = q0 + cq + e + z;
-                  if (q < p.f.Lq) {
+                  if (q < p.f.Lq && db_key) {
                     if (MODE == kDbiasStore) dbcol[q * p.db_sq] = sv[z];
                     else atomicAdd(dbcol + q * p.db_sq, sv[z]);
                   }
@@ -1367,7 +1360,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
               st_shared_v4(sw128_unit(sbase + L::kDS, r, cq / 8 + v4), pk[4 * v4], pk[4 * v4 + 1],
                            pk[4 * v4 + 2], pk[4 * v4 + 3]);
           }
-          if (MODE == kDbiasRowSum) atomicAdd(dbcol, rsum);
+          if (MODE == kDbiasRowSum && db_key) atomicAdd(dbcol, rsum);
         };
         if (POLICY == kPolicyDflash || p.db_mode == kDbiasNone)
           phase_b(std::integral_constant<int, kDbiasNone>{});

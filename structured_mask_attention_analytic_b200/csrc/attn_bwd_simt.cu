@@ -73,7 +73,7 @@ __device__ __forceinline__ bool keeps(const AttnProblem& p, const RowKeep& r, in
   if (!r.valid || k >= p.Lk) return false;
   if (!partial) return true;
   if (POLICY == kPolicyDflash) return (k >= r.clo && k < r.chi) || (k >= r.dlo && k < r.dhi);
-  return k <= r.causal_lim && (r.mrow == nullptr || r.mrow[k] != 0);
+  return k <= r.causal_lim && (r.mrow == nullptr || r.mrow[aux_col(k, p.mask.kd)] != 0);
 }
 
 // dS of one (query row, key): log2-domain score s2 (scale * log2 e folded
@@ -154,12 +154,12 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dq_kernel(const BwdP
         dp += __shfl_xor_sync(0xffffffffu, dp, 1);
         const int k = c0 + kk;
         if (POLICY != kPolicyDflash && rk.brow != nullptr && k < p.Lk)
-          s2 = fmaf(load_any_as_float(rk.brow, p.bias.dtype, k), kLog2e, s2);
+          s2 = fmaf(load_any_as_float(rk.brow, p.bias.dtype, aux_col(k, p.bias.kd)), kLog2e, s2);
         const bool keep = keeps<POLICY>(p, rk, k, partial) && lse2 != -INFINITY;
         const float ds = ds_of(s2, lse2, dp, dd, keep);
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] = fmaf(ds, sk[kk][2 * e + hf], acc[e]);
-        if (dbrow != nullptr && hf == 0 && k < p.Lk) {
+        if (dbrow != nullptr && hf == 0 && k < p.Lk && k < bp.db_kd) {
           if (bp.db_mode == kDbiasStore) dbrow[k] = ds;
           else if (ds != 0.f) atomicAdd(dbrow + k, ds);
         }
@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dkv_kernel(const Bwd
           s2 *= p.scale_log2;
           const RowKeep rk = row_keep<POLICY>(p, b, h, hk, q);
           if (POLICY != kPolicyDflash && rk.brow != nullptr && key_valid)
-            s2 = fmaf(load_any_as_float(rk.brow, p.bias.dtype, k), kLog2e, s2);
+            s2 = fmaf(load_any_as_float(rk.brow, p.bias.dtype, aux_col(k, p.bias.kd)), kLog2e, s2);
           const bool keep = key_valid && keeps<POLICY>(p, rk, k, partial) && sl[qq] != -INFINITY;
           const float pr = keep ? exp2f(s2 - sl[qq]) : 0.f;
           const float ds = pr * (dp - sd[qq]);

@@ -111,13 +111,13 @@ attn_simt_kernel(const AttnProblem p) {
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
         const int k = c0 + kk;
         if (POLICY != kPolicyDflash && p.has_bias && k < p.Lk)
-          acc = fmaf(load_any_as_float(brow, p.bias.dtype, k), kLog2e, acc);
+          acc = fmaf(load_any_as_float(brow, p.bias.dtype, aux_col(k, p.bias.kd)), kLog2e, acc);
         bool keep = row_valid;
         if (partial) {
           if (POLICY == kPolicyDflash) {
             keep = keep && ((k >= clo && k < chi) || (k >= dlo && k < dhi));
           } else {
-            keep = keep && k < p.Lk && k <= causal_lim && (!p.has_mask || mrow[k] != 0);
+            keep = keep && k < p.Lk && k <= causal_lim && (!p.has_mask || mrow[aux_col(k, p.mask.kd)] != 0);
           }
         }
         s[kk] = keep ? acc : -INFINITY;

@@ -13,7 +13,9 @@
 //   warp  8    TMA producer: Q tiles, K/V tiles into a ring of smem stages
 //   warp  9    MMA issuer (one thread): S_i = Q_i K^T into TMEM (SS form),
 //              O_i += P_i V with P_i read from TMEM (TS form)
-//   warps 10-11 idle
+//   warp  10   bias operand tiles when the bias goes through the tensor
+//              cores (BTC, see AttnProblem::bias_tc); otherwise idle
+//   warp  11   idle
 // The kernel is launched with kLaunchRegs registers per thread; the producer
 // warpgroup gives registers back (setmaxnreg.dec to kProducerRegs) and the two
 // softmax warpgroups take them (setmaxnreg.inc to kSoftmaxRegs).  The shares
@@ -45,6 +47,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdio>
+#include <cstring>
 #include <type_traits>
 
 #include "device_common.cuh"
@@ -58,6 +61,7 @@ namespace {
 constexpr int kThreads = 384;
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kBiasWarp = 10;  // bias operands of the tensor-core bias path
 constexpr int kLaunchRegs = 168;
 constexpr int kSoftmaxRegs = 224;
 constexpr int kProducerRegs = 56;
@@ -65,9 +69,17 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kProducerRegs == kThreads * kLaunch
               "register split must equal the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 
-template <int D>
+// Exponentials of a softmax row: MUFU ex2 (16 per clock per SM) would take as
+// long as the row's two products on the tensor cores, so the pairs of each
+// 32-column chunk selected here are computed on the FMA pipe instead
+// (exp2_fma2): 5 of 16 pairs, about 31 %.
+__device__ __forceinline__ constexpr bool exp2_pair_on_fma(int e) { return e % 3 == 2; }
+
+template <int D, bool BTC = false>
 struct Layout {
-  static constexpr int kKStages = D == 128 ? 3 : 4;  // K runs ahead of V
+  // K runs ahead of V; with the bias on the tensor cores at d = 128 the K ring
+  // gives up a stage to the bias operand tiles
+  static constexpr int kKStages = D == 128 ? (BTC ? 2 : 3) : 4;
   static constexpr int kVStages = D == 128 ? 2 : 4;
   static constexpr uint32_t kChunkBytes = kTile * 128;  // 64 columns x 128 rows, 128B-swizzled
   static constexpr uint32_t kTileBytes = kTile * D * 2;
@@ -75,7 +87,12 @@ struct Layout {
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kK = kQ + 2 * kTileBytes;
   static constexpr uint32_t kV = kK + kKStages * kTileBytes;
-  static constexpr uint32_t kBars = kV + kVStages * kTileBytes;
+  // bias operand tiles (BTC): A (128 query rows x one K step) and one B
+  // (128 keys x one K step) per K stage, 32-byte rows, 32-byte swizzle
+  static constexpr uint32_t kXBytes = BTC ? kTile * 32 : 0;
+  static constexpr uint32_t kAX = kV + kVStages * kTileBytes;
+  static constexpr uint32_t kBX = kAX + kXBytes;
+  static constexpr uint32_t kBars = kBX + kKStages * kXBytes;
   // barrier slots
   static constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + kKStages,
                        kVFull = kKEmpty + kKStages, kVEmpty = kVFull + kVStages,
@@ -189,12 +206,12 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* e
   mbar_wait(bar, parity, nv, err);
 }
 
-template <int D, int POLICY, int DT>
+template <int D, int POLICY, int DT, bool BTC>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
                const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                int n_units) {
-  using L = Layout<D>;
+  using L = Layout<D, BTC>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -210,7 +227,9 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
     mbar_init(bar(L::kQFull), 1);
     mbar_init(bar(L::kQEmpty), 1);
     for (int s = 0; s < L::kKStages; ++s) {
-      mbar_init(bar(L::kKFull + s), 1);
+      // (with the bias on the tensor cores the bias warp's 32 lanes also
+      // arrive, once its operand tile for the stage is written)
+      mbar_init(bar(L::kKFull + s), BTC ? 1 + 32 : 1);
       mbar_init(bar(L::kKEmpty + s), 1);
     }
     for (int s = 0; s < L::kVStages; ++s) {
@@ -338,6 +357,12 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
     auto with_lo = [](uint64_t d, uint32_t add) -> uint64_t {
       return (d & 0xffffffff00000000ull) | static_cast<uint32_t>(static_cast<uint32_t>(d) + add);
     };
+    // With the bias on the tensor cores, one more K step adds b[k] / scale.
+    auto issue_bias_step = [&](uint32_t d_col, int stage) {
+      if (BTC)
+        tc_mma_ss(d_col, smem_desc_sw32(sbase + L::kAX),
+                  smem_desc_sw32(sbase + L::kBX + stage * L::kXBytes), idesc_qk, 1u);
+    };
     auto issue_qk = [&](int i, int stage) {
       const uint64_t qd = smem_desc_sw128(sbase + L::kQ + i * L::kTileBytes, 16, 1024);
       const uint64_t kd = smem_desc_sw128(sbase + L::kK + stage * L::kTileBytes, 16, 1024);
@@ -347,6 +372,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
         const uint32_t off = ((s >> 2) * L::kChunkBytes + (s & 3) * 32) >> 4;
         tc_mma_ss(d_col, with_lo(qd, off), with_lo(kd, off), idesc_qk, s > 0 ? 1u : 0u);
       }
+      issue_bias_step(d_col, stage);
     };
     // Both query tiles against one K tile, k-steps interleaved.
     auto issue_qk_pair = [&](int stage) {
@@ -359,6 +385,8 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
         tc_mma_ss(tmem + L::kColS0, with_lo(qd0, off), with_lo(kd, off), idesc_qk, s > 0 ? 1u : 0u);
         tc_mma_ss(tmem + L::kColS1, with_lo(qd1, off), with_lo(kd, off), idesc_qk, s > 0 ? 1u : 0u);
       }
+      issue_bias_step(tmem + L::kColS0, stage);
+      issue_bias_step(tmem + L::kColS1, stage);
     };
     auto issue_pv = [&](int i, int stage, bool first) {
       const uint64_t vd =
@@ -462,6 +490,59 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
       __syncwarp();
       drain_wait(bar(L::kDrain), 0, p.err);
     }
+   } else if (BTC && warp == kBiasWarp) {
+    // ------------------------------------------------------------ bias operands
+    // A: every query row [hi, lo, 0, ...] (1 / scale in the operand type); B
+    // for each K stage: key row k [b[k], b[k], 0, ...].  Only the first
+    // 16-byte half of a row ever holds data; the other half is zeroed once.
+    // The bias row is shared by all queries and by both query tiles of a
+    // unit (the launcher takes this path only then).  Lane l writes key rows
+    // l, l + 32, l + 64, l + 96; the values of the next tile are loaded before
+    // waiting for its stage to free up.
+    const uint32_t ax = sbase + L::kAX;
+    for (int r = lane; r < kTile; r += 32) {
+      st_shared_v4(ax + sw32_chunk(r, 0), p.bias_tc_a, 0u, 0u, 0u);
+      st_shared_v4(ax + sw32_chunk(r, 1), 0u, 0u, 0u, 0u);
+      for (int s2 = 0; s2 < L::kKStages; ++s2)
+        st_shared_v4(sbase + L::kBX + s2 * L::kXBytes + sw32_chunk(r, 1), 0u, 0u, 0u, 0u);
+    }
+    const uint16_t* bias16 = static_cast<const uint16_t*>(p.bias.ptr);
+    const int kd = p.bias.kd;
+    const uint32_t two_cols = (p.bias_tc_a >> 16) != 0u ? 1u : 0u;  // A has a nonzero lo column
+    uint32_t kv_k = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit w = decode_unit<POLICY>(p, u);
+      const int n = w.n;
+      if (n == 0) continue;
+      const uint16_t* brow = bias16 + w.b * p.bias.sb + w.hk * p.bias.sh;
+      bool partial;
+      int kt = tile_at(p, w, 0, &partial);
+      uint32_t v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = brow[aux_col(kt * kTile + lane + 32 * i, kd)];
+      for (int j = 0; j < n && ok; ++j) {
+        const int stage = kv_k % L::kKStages;
+        const uint32_t kuse = kv_k / L::kKStages;
+        if (kuse > 0 &&
+            !mbar_wait_warp(bar(L::kKEmpty + stage), (kuse - 1) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        const uint32_t bx = sbase + L::kBX + stage * L::kXBytes;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          st_shared_v4(bx + sw32_chunk(lane + 32 * i, 0), v[i] | (v[i] << 16) * two_cols, 0u, 0u, 0u);
+        fence_async_shared();
+        mbar_arrive(bar(L::kKFull + stage));
+        ++kv_k;
+        if (j + 1 < n) {
+          kt = tile_at(p, w, j + 1, &partial);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) v[i] = brow[aux_col(kt * kTile + lane + 32 * i, kd)];
+        }
+      }
+    }
    }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
@@ -533,6 +614,22 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
       // With compacted keys every PARTIAL tile is cut by the row limit.
       const int causal_off = POLICY == kPolicyGather ? -(1 << 30) : w.lk - w.lq;
       const bool mask_bcast_q = POLICY == kPolicyExplicit && p.has_mask && p.mask.sq == 0;
+      // Mask / bias rows hold kd columns: round_up(Lk, 128), Lk, or 1.  Vector
+      // loads start at most at the row's last aligned chunk (a 16-byte block
+      // that holds column kd - 1), so none leaves the row's memory; columns
+      // past Lk are never kept whatever is read for them.  A row of one column
+      // holds one value for every key: a mask flag for the whole row, or a
+      // bias that shifts every score of the row alike, which the softmax
+      // ignores; it is added once, to the row's max (and so to lse).
+      const bool bias_cols = !BTC && p.has_bias && p.bias.kd > 1;
+      const int bias_vlast = (p.bias.kd - 1) & (p.bias.dtype == SMA_FP32 ? ~3 : ~7);
+      const bool mask_row1 = p.has_mask && p.mask.kd == 1;
+      const int mask_vlast16 = (p.mask.kd - 1) & ~15;
+      const int mask_vlast4 = (p.mask.kd - 1) & ~3;
+      const bool row_keep1 = mask_row1 && mrow[0] != 0;
+      const float bias_row_log2 =
+          (POLICY != kPolicyDflash && !BTC && p.has_bias && p.bias.kd == 1)
+              ? load_any_as_float(brow, p.bias.dtype, 0) * kLog2e : 0.f;
       float m_ref = -INFINITY, l_sum = 0.f;
       bool partial_next = false;
       int kt_next = n > 0 ? tile_at(p, w, 0, &partial_next) : 0;
@@ -550,11 +647,11 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           for (int c = 0; c < kTile / 32; ++c) tmem_ld32_at(s_col + 32 * c, xr + 32 * c);
           tc_wait_ld();
         }
-        if (POLICY != kPolicyDflash && p.has_bias) {
+        if (POLICY != kPolicyDflash && bias_cols) {
           if (p.bias.dtype == SMA_FP32) {
 #pragma unroll
             for (int c = 0; c < kTile; c += 4) {
-              const float4 a = *reinterpret_cast<const float4*>(brow + (k0 + c) * 4);
+              const float4 a = *reinterpret_cast<const float4*>(brow + min(k0 + c, bias_vlast) * 4);
               x[c] = fmaf(a.x, bias_mul, x[c]);
               x[c + 1] = fmaf(a.y, bias_mul, x[c + 1]);
               x[c + 2] = fmaf(a.z, bias_mul, x[c + 2]);
@@ -563,7 +660,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           } else if (p.bias.dtype == SMA_BF16) {
 #pragma unroll
             for (int c = 0; c < kTile; c += 8) {
-              const uint4 a = *reinterpret_cast<const uint4*>(brow + (k0 + c) * 2);
+              const uint4 a = *reinterpret_cast<const uint4*>(brow + min(k0 + c, bias_vlast) * 2);
               const uint32_t wv[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -575,7 +672,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           } else {
 #pragma unroll
             for (int c = 0; c < kTile; c += 8) {
-              const uint4 a = *reinterpret_cast<const uint4*>(brow + (k0 + c) * 2);
+              const uint4 a = *reinterpret_cast<const uint4*>(brow + min(k0 + c, bias_vlast) * 2);
               const uint32_t wv[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -604,10 +701,13 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
             if (k0 + kTile > w.lk) lim = min(lim, w.lk - k0);
             if (p.causal && k0 + kTile - 1 > qfirst + causal_off)
               lim = min(lim, causal_lim - k0 + 1);
-            if (mask_bcast_q) {
+            if (POLICY == kPolicyExplicit && mask_row1) {
+#pragma unroll
+              for (int c = 0; c < kTile; ++c) x[c] = (row_keep1 && c < lim) ? x[c] : -INFINITY;
+            } else if (mask_bcast_q) {
               // One mask row for every query row: 4 ballots turn the tile's 128
               // bytes into bits, bit l of word j = column 4 l + j.
-              const uint32_t mw = *reinterpret_cast<const uint32_t*>(mrow + k0 + 4 * lane);
+              const uint32_t mw = *reinterpret_cast<const uint32_t*>(mrow + min(k0 + 4 * lane, mask_vlast4));
               uint32_t bits[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j)
@@ -620,7 +720,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
             } else if (POLICY == kPolicyExplicit && p.has_mask) {
 #pragma unroll
               for (int c = 0; c < kTile; c += 16) {
-                const uint4 mv = *reinterpret_cast<const uint4*>(mrow + k0 + c);
+                const uint4 mv = *reinterpret_cast<const uint4*>(mrow + min(k0 + c, mask_vlast16));
                 const uint32_t wv[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -681,8 +781,17 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(fmaf(x[32 * c + 2 * e], exp_scale, -msub));
-            const float p1 = fast_exp2(fmaf(x[32 * c + 2 * e + 1], exp_scale, -msub));
+            const float2 t = fma2(make_float2(x[32 * c + 2 * e], x[32 * c + 2 * e + 1]),
+                                  make_float2(exp_scale, exp_scale), make_float2(-msub, -msub));
+            float p0, p1;
+            if (exp2_pair_on_fma(e)) {
+              const float2 pp = exp2_fma2(t);
+              p0 = pp.x;
+              p1 = pp.y;
+            } else {
+              p0 = fast_exp2(t.x);
+              p1 = fast_exp2(t.y);
+            }
             ls8[(2 * e) & 7] += p0;
             ls8[(2 * e + 1) & 7] += p1;
             pk[e] = DT == SMA_BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
@@ -714,7 +823,10 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
       OutT* orow = reinterpret_cast<OutT*>(p.o) + (POLICY == kPolicyVarlen ? 0 : w.b) * p.o_sb +
                    static_cast<int64_t>(w.q_off + q) * p.o_sr +
                    h * p.o_sh;
-      const float inv_l = l_sum > 0.f ? 1.0f / l_sum : 0.f;
+      // A row that kept no key has max -inf (its sum is not 0: exp2_fma2 of
+      // -inf is 2^-125).
+      const bool live = m_ref != -INFINITY;
+      const float inv_l = live ? 1.0f / l_sum : 0.f;
       // Key-range segment: unnormalised O and (max, sum) go to the partials.
       const bool seg_out = POLICY != kPolicyVarlen && p.n_split > 1;
       const int64_t prow =
@@ -757,11 +869,11 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
       if (seg_out) {
         if (row_valid)
           *reinterpret_cast<float2*>(p.part_ml + 2 * prow) =
-              make_float2(l_sum > 0.f ? m_ref : -INFINITY, l_sum);
+              make_float2(live ? m_ref + bias_row_log2 : -INFINITY, live ? l_sum : 0.f);
       } else if (row_valid && p.lse != nullptr) {
         p.lse[POLICY == kPolicyVarlen ? static_cast<int64_t>(h) * p.total_q + w.q_off + q
                                       : (static_cast<int64_t>(w.b) * p.H + h) * p.Lq + q] =
-            l_sum > 0.f ? (m_ref + __log2f(l_sum)) * kLn2 : -INFINITY;
+            live ? (m_ref + bias_row_log2 + __log2f(l_sum)) * kLn2 : -INFINITY;
       }
       tc_fence_before();
       mbar_arrive(bar(L::kOFree + qi));
@@ -854,11 +966,26 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnProblem p) 
 
 // ------------------------------------------------------------------ host side
 
-template <int D, int POLICY, int DT>
+// bf16 bits of x rounded to nearest even (finite x), and back.
+uint16_t float_to_bf16_bits(float x) {
+  uint32_t u;
+  memcpy(&u, &x, 4);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return static_cast<uint16_t>(u >> 16);
+}
+float bf16_bits_to_float(uint16_t h) {
+  const uint32_t u = static_cast<uint32_t>(h) << 16;
+  float x;
+  memcpy(&x, &u, 4);
+  return x;
+}
+
+template <int D, int POLICY, int DT, bool BTC = false>
 cudaError_t launch_typed(const AttnProblem& p, const CUtensorMap& mq, const CUtensorMap& mk,
                          const CUtensorMap& mv, cudaStream_t stream) {
-  using L = Layout<D>;
-  auto kern = attn_tc_kernel<D, POLICY, DT>;
+  using L = Layout<D, BTC>;
+  static_assert(L::kAlloc <= 232448, "shared memory of one CTA");
+  auto kern = attn_tc_kernel<D, POLICY, DT, BTC>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaFuncAttributes fa;
@@ -911,6 +1038,12 @@ int launch_problem(const AttnProblem& p, cudaStream_t stream, char* msg, size_t 
                            : launch_typed<128, kPolicyVarlen, SMA_FP16>(p, mq, mk, mv, stream);
     else e = bf ? launch_typed<64, kPolicyVarlen, SMA_BF16>(p, mq, mk, mv, stream)
                 : launch_typed<64, kPolicyVarlen, SMA_FP16>(p, mq, mk, mv, stream);
+  } else if (p.bias_tc) {
+    if (p.d == 128)
+      e = bf ? launch_typed<128, kPolicyExplicit, SMA_BF16, true>(p, mq, mk, mv, stream)
+             : launch_typed<128, kPolicyExplicit, SMA_FP16, true>(p, mq, mk, mv, stream);
+    else e = bf ? launch_typed<64, kPolicyExplicit, SMA_BF16, true>(p, mq, mk, mv, stream)
+                : launch_typed<64, kPolicyExplicit, SMA_FP16, true>(p, mq, mk, mv, stream);
   } else {
     if (p.d == 128) e = bf ? launch_typed<128, kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, stream)
                            : launch_typed<128, kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, stream);
@@ -936,6 +1069,32 @@ int launch_attn_tc(const AttnProblem& p, cudaStream_t stream, char* msg, size_t 
   }
   AttnProblem pp = p;
   pp.pack = fwd_pack(p.Lq, p.group, p.lists.head_mode, p.policy);
+  // The bias goes through the tensor cores when one bias row serves every
+  // query and both query heads of a unit: query stride 0, head dim 1 or KVH
+  // (or one head per KV head, or a head dim read with stride 0), more than
+  // one key column, the operands' dtype.
+  pp.bias_tc = 0;
+  if (pp.policy == kPolicyExplicit && pp.has_bias && pp.bias.kd > 1 && pp.bias.sq == 0 &&
+      pp.bias.dtype == pp.dtype &&
+      (pp.bias.head_per_query == 0 || pp.group == 1 || pp.bias.sh == 0)) {
+    pp.bias_tc = 1;
+    // hi is 1 / scale rounded toward zero, so that lo = 1 / scale - hi >= 0:
+    // a bias of -inf then gives -inf * hi + -inf * lo = -inf, never
+    // -inf + inf.  When lo is 0 (1 / scale exact, e.g. 8 at head dim 64) the
+    // operand has one column only, so that -inf never meets a zero factor.
+    const float inv_scale = 1.4426950408889634f / pp.scale_log2;  // as the kernel's bias_mul
+    uint16_t hi, lo;
+    if (pp.dtype == SMA_BF16) {
+      uint32_t u;
+      memcpy(&u, &inv_scale, 4);
+      hi = static_cast<uint16_t>(u >> 16);
+      lo = float_to_bf16_bits(inv_scale - bf16_bits_to_float(hi));
+    } else {
+      hi = __half_as_ushort(__float2half_rz(inv_scale));
+      lo = __half_as_ushort(__float2half_rn(inv_scale - __half2float(__ushort_as_half(hi))));
+    }
+    pp.bias_tc_a = static_cast<uint32_t>(hi) | (static_cast<uint32_t>(lo) << 16);
+  }
   return launch_problem(pp, stream, msg, msg_len);
 }
 

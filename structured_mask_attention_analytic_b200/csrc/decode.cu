@@ -138,23 +138,37 @@ decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap m
           const int gr = rg * G + r;
           const bool rv = gr < p.group;
           const int h = hk * p.group + (rv ? gr : 0);
-          const bool in_row = k < p.Kpad;
           uint2 mb = make_uint2(0x01010101u, 0x01010101u);
-          if (p.has_mask && in_row) {
+          if (p.has_mask) {
             const int hm = p.mask.head_per_query ? h : hk;
-            mb = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(p.mask.ptr) +
-                                                 b * p.mask.sb + hm * p.mask.sh + k);
+            const uint8_t* mrow =
+                reinterpret_cast<const uint8_t*>(p.mask.ptr) + b * p.mask.sb + hm * p.mask.sh;
+            if (k + 8 <= p.mask.kd) {
+              mb = *reinterpret_cast<const uint2*>(mrow + k);
+            } else {  // a row of Lk or 1 columns: column by column, inside the row
+              uint32_t w2[2] = {0u, 0u};
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                w2[e >> 2] |= (mrow[aux_col(k + e, p.mask.kd)] != 0 ? 1u : 0u) << (8 * (e & 3));
+              mb = make_uint2(w2[0], w2[1]);
+            }
           }
           float bv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          if (p.has_bias && in_row) {
+          if (p.has_bias) {
             const int hb = p.bias.head_per_query ? h : hk;
-            const int64_t bi = b * p.bias.sb + hb * p.bias.sh + k;
-            if (p.bias.dtype == SMA_FP32) {
-              global8<SMA_FP32>(p.bias.ptr, bi, bv);
-            } else if (p.bias.dtype == SMA_BF16) {
-              global8<SMA_BF16>(p.bias.ptr, bi, bv);
+            const int64_t bi = b * p.bias.sb + hb * p.bias.sh;
+            if (k + 8 <= p.bias.kd) {
+              if (p.bias.dtype == SMA_FP32) {
+                global8<SMA_FP32>(p.bias.ptr, bi + k, bv);
+              } else if (p.bias.dtype == SMA_BF16) {
+                global8<SMA_BF16>(p.bias.ptr, bi + k, bv);
+              } else {
+                global8<SMA_FP16>(p.bias.ptr, bi + k, bv);
+              }
             } else {
-              global8<SMA_FP16>(p.bias.ptr, bi, bv);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                bv[e] = load_any_as_float(p.bias.ptr, p.bias.dtype, bi + aux_col(k + e, p.bias.kd));
             }
           }
           const uint32_t mw[2] = {mb.x, mb.y};

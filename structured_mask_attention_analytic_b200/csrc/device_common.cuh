@@ -258,6 +258,28 @@ __device__ __forceinline__ void tmem_st16_at(uint32_t taddr, const uint32_t* r) 
       : "memory");
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// Orders this thread's earlier shared-memory writes (generic proxy) before
+// later reads of them by the tensor cores or TMA (async proxy).
+__device__ __forceinline__ void fence_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor of a tile stored the way a 128-byte-swizzled
 // TMA load leaves it: rows of 128 bytes, 8-row groups 1024 bytes apart.
 //   bits  0-13 start address >> 4     bits 16-29 leading byte offset >> 4
@@ -272,6 +294,24 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_
   d |= static_cast<uint64_t>(1) << 46;
   d |= static_cast<uint64_t>(2) << 61;
   return d;
+}
+
+// The same descriptor for a tile stored with a 32-byte swizzle: rows of 32
+// bytes (16 elements of 16 bits, one K step), 8-row groups 256 bytes apart,
+// the two 16-byte halves of row r swapped when bit 2 of r is set (swizzle
+// mode 6).
+__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(16u >> 4) << 16;
+  d |= static_cast<uint64_t>(256u >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(6) << 61;
+  return d;
+}
+// Byte offset of 16-byte chunk c (0 or 1) of row r in such a tile.
+__device__ __forceinline__ uint32_t sw32_chunk(int r, int c) {
+  return static_cast<uint32_t>((r >> 3) * 256 + (r & 7) * 32 + ((c ^ ((r >> 2) & 1)) << 4));
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16 with fp32 accumulation.
@@ -318,6 +358,12 @@ __device__ __forceinline__ float load_as_float<SMA_FP32>(const void* base, int64
   return reinterpret_cast<const float*>(base)[idx];
 }
 
+// Column of a mask / bias row that holds key k.  A row holds kd columns:
+// round_up(Lk, 128), Lk, or 1, where one value stands for every key (a key
+// dim broadcast with stride 0).  Keys at or past kd are never kept, so for
+// them the row's last column is read only to keep the access inside the row.
+__device__ __forceinline__ int aux_col(int k, int kd) { return k < kd ? k : kd - 1; }
+
 __device__ __forceinline__ float load_any_as_float(const void* base, int dtype, int64_t idx) {
   if (dtype == SMA_BF16) return load_as_float<SMA_BF16>(base, idx);
   if (dtype == SMA_FP16) return load_as_float<SMA_FP16>(base, idx);
@@ -354,6 +400,44 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
       : "=f"(r.x), "=f"(r.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return r;
+}
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
+// 2^t for a pair of arguments on the FMA and integer pipes, leaving the
+// MUFU unit (ex2.approx, 16 results per clock per SM) to the other columns
+// of a softmax row.  t = n + f with n = round(t): adding 1.5 * 2^23 rounds t
+// to an integer held in the low mantissa bits; f = t - n lies in [-1/2, 1/2];
+// 2^f is a cubic whose coefficients fit_exp2_poly.py derives (relative error
+// at most 7.5e-5 over [-1/2, 1/2] in float32, against 2^-9 for rounding P to
+// bf16); 2^n is added to the exponent field (the low bits of the rounded sum,
+// shifted left by 23, are n << 23).  Arguments are clamped at -125 from
+// below: -inf gives 2^-125 (2.4e-38) rather than 0, so a softmax using this
+// must tell an empty row by its max (-inf), not by its sum.  Arguments up to
+// +127 are exact in range.
+constexpr float kExp2C0 = 9.999280572e-01f;
+constexpr float kExp2C1 = 6.932609677e-01f;
+constexpr float kExp2C2 = 2.426111251e-01f;
+constexpr float kExp2C3 = 5.517166480e-02f;
+__device__ __forceinline__ float2 exp2_fma2(float2 t) {
+  t.x = fmaxf(t.x, -125.f);
+  t.y = fmaxf(t.y, -125.f);
+  const float2 magic = make_float2(12582912.f, 12582912.f);
+  const float2 j = add2(t, magic);
+  const float2 f = sub2(t, sub2(j, magic));
+  float2 p = fma2(f, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
+  p = fma2(p, f, make_float2(kExp2C1, kExp2C1));
+  p = fma2(p, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
 }
 
 constexpr float kLog2e = 1.4426950408889634f;

@@ -28,8 +28,8 @@ constexpr int kSelThreads = 256;
 // Stream compaction of one mask row: each thread takes 4 columns per step, a
 // block-wide exclusive scan of the kept counts gives the output positions.
 __global__ void __launch_bounds__(kSelThreads)
-select_keys_kernel(const uint8_t* __restrict__ mask, int64_t m_sb, int64_t m_sh, int LH, int Lk,
-                   int cap, int32_t* __restrict__ idx, int32_t* __restrict__ count, int* err) {
+select_keys_kernel(const uint8_t* __restrict__ mask, int64_t m_sb, int64_t m_sh, int m_kd, int LH,
+                   int Lk, int cap, int32_t* __restrict__ idx, int32_t* __restrict__ count, int* err) {
   const int grow = blockIdx.x;
   const int lb = grow / LH, lh = grow - lb * LH;
   const uint8_t* row = mask + lb * m_sb + lh * m_sh;
@@ -41,11 +41,15 @@ select_keys_kernel(const uint8_t* __restrict__ mask, int64_t m_sb, int64_t m_sh,
   for (int c0 = 0; c0 < kpad; c0 += kSelThreads * 4) {
     const int c = c0 + threadIdx.x * 4;
     uint32_t bits = 0;
-    if (c < kpad) {  // the row holds kpad columns, c is a multiple of 4
+    if (c + 4 <= m_kd) {  // c is a multiple of 4
       const uint32_t wv = *reinterpret_cast<const uint32_t*>(row + c);
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         if (((wv >> (8 * e)) & 0xffu) != 0u && c + e < Lk) bits |= 1u << e;
+    } else if (c < kpad) {  // a row of Lk columns ends here, or one column stands for every key
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (c + e < Lk && row[aux_col(c + e, m_kd)] != 0) bits |= 1u << e;
     }
     const uint32_t n = __popc(bits);
     uint32_t incl = n;
@@ -115,7 +119,7 @@ __global__ void gather_kv_kernel(const AttnProblem p, const uint8_t* __restrict_
 // the original column idx[j]; the rest are 0 (masked by the row limit).
 template <typename T>
 __global__ void gather_bias_kernel(const AttnProblem p, const T* __restrict__ src, int64_t s_sb,
-                                   int64_t s_sh, int64_t s_sq, int rows_h, int rows_q,
+                                   int64_t s_sh, int64_t s_sq, int s_kd, int rows_h, int rows_q,
                                    int heads_are_query) {
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   const int hq = blockIdx.y, b = blockIdx.z;
@@ -127,7 +131,7 @@ __global__ void gather_bias_kernel(const AttnProblem p, const T* __restrict__ sr
   T val = T(0.f);
   if (j < cnt) {
     const int64_t key = p.gather.idx[grow * p.gather.cap + j];
-    val = src[b * s_sb + hc * s_sh + qc * s_sq + key];
+    val = src[b * s_sb + hc * s_sh + qc * s_sq + aux_col(static_cast<int>(key), s_kd)];
   }
   T* dst = reinterpret_cast<T*>(const_cast<void*>(p.bias.ptr));
   dst[b * p.bias.sb + hc * p.bias.sh + qc * p.bias.sq + j] = val;
@@ -160,10 +164,10 @@ __global__ void __launch_bounds__(kGlThreads) gather_lists_kernel(const AttnProb
 
 }  // namespace
 
-cudaError_t launch_select_keys(const uint8_t* mask, int64_t m_sb, int64_t m_sh, int LB, int LH,
-                               int Lk, int cap, int32_t* idx, int32_t* count, int* err,
+cudaError_t launch_select_keys(const uint8_t* mask, int64_t m_sb, int64_t m_sh, int m_kd, int LB,
+                               int LH, int Lk, int cap, int32_t* idx, int32_t* count, int* err,
                                cudaStream_t stream) {
-  select_keys_kernel<<<LB * LH, kSelThreads, 0, stream>>>(mask, m_sb, m_sh, LH, Lk, cap, idx,
+  select_keys_kernel<<<LB * LH, kSelThreads, 0, stream>>>(mask, m_sb, m_sh, m_kd, LH, Lk, cap, idx,
                                                           count, err);
   return cudaGetLastError();
 }
@@ -188,10 +192,12 @@ cudaError_t launch_gather_bias(const AttnProblem& p, const AuxView& bias, int ro
   const int hq = bias.head_per_query;
   if (bias.dtype == SMA_FP32)
     gather_bias_kernel<float><<<grid, block, 0, stream>>>(
-        p, static_cast<const float*>(bias.ptr), bias.sb, bias.sh, bias.sq, rows_h, rows_q, hq);
+        p, static_cast<const float*>(bias.ptr), bias.sb, bias.sh, bias.sq, bias.kd, rows_h, rows_q,
+        hq);
   else  // bf16 / fp16 move as raw 16-bit words
     gather_bias_kernel<uint16_t><<<grid, block, 0, stream>>>(
-        p, static_cast<const uint16_t*>(bias.ptr), bias.sb, bias.sh, bias.sq, rows_h, rows_q, hq);
+        p, static_cast<const uint16_t*>(bias.ptr), bias.sb, bias.sh, bias.sq, bias.kd, rows_h, rows_q,
+        hq);
   return cudaGetLastError();
 }
 

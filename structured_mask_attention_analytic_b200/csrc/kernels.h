@@ -32,6 +32,10 @@ struct AuxView {
   int64_t sb = 0, sh = 0, sq = 0;  // element strides, 0 for broadcast dims
   int head_per_query = 0;          // 1: head index is the query head, 0: the KV head
   int64_t sizes[4] = {0, 0, 0, 0};
+  // Key columns each row holds: round_up(Lk, 128) (the padded form), Lk, or
+  // 1 (one value for every key: the key dim broadcasts with stride 0).
+  // Kernels read column min(k, kd - 1) for key k, so no access leaves a row.
+  int kd = 0;
 };
 
 // Ascending key-tile lists; list row = (lb * LH + lh) * QT + qt.
@@ -81,6 +85,14 @@ struct AttnProblem {
   int causal;
   int has_mask, has_bias;
   AuxView mask, bias;
+  // Bias on the tensor cores (tcgen05 explicit path, set by the launcher):
+  // a bias shared by every query of a row of S, b[k], enters S = Q K^T as one
+  // more K step whose A rows are [hi, lo, 0, ...] (1 / scale split into two
+  // values of the operand type, packed hi | lo << 16 here) and whose B rows are
+  // [b[k], b[k], 0, ...], so S holds q.k + b / scale and the softmax adds no
+  // bias itself.
+  int bias_tc = 0;
+  uint32_t bias_tc_a = 0;
   GatherView gather;  // idx == nullptr: keys are not compacted
   // varlen policy: sequence b holds query rows [cu_q[b], cu_q[b+1]) of the
   // packed [total_q, H, d] operands (keys likewise); Lq / Lk are the maxima
@@ -139,11 +151,13 @@ struct BwdProblem {
   const int32_t* t_num_part; const int32_t* t_part;
   float scale;     // softmax scale (dQ and dK carry it)
   // Gradient of the bias (explicit policy only): fp32, the bias's broadcast
-  // shape (b', h', q', 128-rounded Lk), zeroed before the kernel runs; element
-  // (b, h, q, k) of dS adds into dbias[b * db_sb + hb * db_sh + q * db_sq + k]
-  // (strides 0 on broadcast dims; hb = h if db_head_per_query else h / group).
+  // shape (b', h', q', db_kd) with db_kd the bias's key dim (128-rounded Lk, or
+  // Lk), zeroed before the kernel runs; element (b, h, q, k) of dS adds into
+  // dbias[b * db_sb + hb * db_sh + q * db_sq + k] for k < db_kd (strides 0 on
+  // broadcast dims; hb = h if db_head_per_query else h / group).
   float* dbias = nullptr;
   int64_t db_sb = 0, db_sh = 0, db_sq = 0;
+  int db_kd = 0;
   int db_head_per_query = 0;
   int db_mode = 0;  // kDbias* below
 };
@@ -167,6 +181,14 @@ struct DecodeProblem {
   float* lse;  // [B, H] (q_len 1) or null
   int has_mask, has_bias;
   AuxView mask, bias;
+  // Bias on the tensor cores (tcgen05 explicit path, set by the launcher):
+  // a bias shared by every query of a row of S, b[k], enters S = Q K^T as one
+  // more K step whose A rows are [hi, lo, 0, ...] (1 / scale split into two
+  // values of the operand type, packed hi | lo << 16 here) and whose B rows are
+  // [b[k], b[k], 0, ...], so S holds q.k + b / scale and the softmax adds no
+  // bias itself.
+  int bias_tc = 0;
+  uint32_t bias_tc_a = 0;
   int splits, chunk;       // split-KV: keys [s*chunk, min((s+1)*chunk, Lk)), chunk % 128 == 0
   float* part_o;           // [B, H, splits, d]
   float* part_ml;          // [B, H, splits, 2]  (max in log2 units, sum)
@@ -176,7 +198,8 @@ struct DecodeProblem {
 struct TopkProblem {
   int bias_dtype;
   const void* bias; int64_t b_sizes[4]; int64_t b_strides[4];
-  int Lk, Kpad;
+  int Lk;
+  int Kcols;  // columns of each bias / output row: round_up(Lk, 128) or Lk
   const uint8_t* pre; int64_t p_sizes[4]; int64_t p_strides[4];  // strides 0 on broadcast dims
   int window;
   uint8_t* out;
@@ -223,10 +246,11 @@ cudaError_t launch_attn_simt(const AttnProblem& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeProblem& p, cudaStream_t stream);
 
 // Index-gather preparation.  `mask` is a query-broadcast keep mask with
-// element strides m_sb / m_sh (0 on broadcast dims) and Kpad columns; gather
-// row (lb, lh) reads mask row lb * m_sb + lh * m_sh.
-cudaError_t launch_select_keys(const uint8_t* mask, int64_t m_sb, int64_t m_sh, int LB, int LH,
-                               int Lk, int cap, int32_t* idx, int32_t* count, int* err,
+// element strides m_sb / m_sh (0 on broadcast dims) and m_kd columns per row
+// (round_up(Lk, 128), Lk or 1); gather row (lb, lh) reads mask row
+// lb * m_sb + lh * m_sh.
+cudaError_t launch_select_keys(const uint8_t* mask, int64_t m_sb, int64_t m_sh, int m_kd, int LB,
+                               int LH, int Lk, int cap, int32_t* idx, int32_t* count, int* err,
                                cudaStream_t stream);
 // Compacted K and V ([B, cap, KVH, d], the strides in p.k/p.v) from the
 // original operands; rows from count to the next multiple of 128 are zeroed.
@@ -257,6 +281,8 @@ int set_last_error(int code, const char* message);
 
 cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, int* err, int64_t* out,
                                          cudaStream_t stream);
+// out[i] = the softmax's FMA-pipe 2^in[i] for n (even) floats on the device.
+cudaError_t launch_exp2_fma_selftest(const float* in, float* out, int64_t n, cudaStream_t stream);
 
 // Device error word in the current context (looked up once per context).
 int* device_error_word(cudaError_t* status);

@@ -79,7 +79,7 @@ sma_status check_heads(int32_t heads, int32_t kv_heads, int32_t head_dim) {
 // Mask/bias operand of the 4D broadcast contract; fills `view`.
 sma_status check_aux(const char* name, const void* ptr, const int64_t* sizes,
                      const int64_t* strides, int esz, int32_t B, int32_t H, int32_t KVH,
-                     int32_t Lq, int32_t Lk, bool need_full_k, AuxView* view) {
+                     int32_t Lq, int32_t Lk, bool allow_key_dim_1, AuxView* view) {
   if (sizes == nullptr || strides == nullptr)
     return fail(SMA_ERR_INVALID_ARG, "%s sizes/strides are NULL", name);
   const int64_t kpad = round_up(Lk, kTile);
@@ -92,22 +92,36 @@ sma_status check_aux(const char* name, const void* ptr, const int64_t* sizes,
   if (sizes[2] != Lq && sizes[2] != 1)
     return fail(SMA_ERR_INVALID_ARG, "%s query dim %lld must be %d or 1", name,
                 static_cast<long long>(sizes[2]), Lq);
-  if (need_full_k && sizes[3] != kpad)
-    return fail(SMA_ERR_INVALID_ARG, "%s key dim %lld must be round_up(k_len, 128) = %lld", name,
-                static_cast<long long>(sizes[3]), static_cast<long long>(kpad));
-  if (strides[3] != 1) return fail(SMA_ERR_INVALID_ARG, "%s last dim must be contiguous", name);
-  if (!aligned16(ptr)) return fail(SMA_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);
+  // PR #190's interface pads the key dim to round_up(Lk, 128) and expands a
+  // key dim of 1; the kernels read all three forms in place (no copy).
+  if (sizes[3] != kpad && sizes[3] != Lk && sizes[3] != 1)
+    return fail(SMA_ERR_INVALID_ARG,
+                "%s key dim %lld must be round_up(k_len, 128) = %lld, k_len = %d or 1", name,
+                static_cast<long long>(sizes[3]), static_cast<long long>(kpad), Lk);
+  if (!allow_key_dim_1 && sizes[3] == 1 && Lk > 1)
+    return fail(SMA_ERR_INVALID_ARG, "%s key dim 1 is not accepted here", name);
+  if (sizes[3] != 1 && strides[3] != 1)
+    return fail(SMA_ERR_INVALID_ARG, "%s last dim must be contiguous", name);
+  // Rows of more than one column are read with 16-byte vector loads; a row
+  // of one column is read one element at a time and needs only element
+  // alignment.
+  const bool one_col = sizes[3] == 1;
+  if (!one_col && !aligned16(ptr))
+    return fail(SMA_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);
+  if (one_col && (reinterpret_cast<uintptr_t>(ptr) % esz) != 0)
+    return fail(SMA_ERR_INVALID_ARG, "%s must be aligned to its element size", name);
   view->ptr = ptr;
   view->sb = sizes[0] == 1 ? 0 : strides[0];
   view->sh = sizes[1] == 1 ? 0 : strides[1];
   view->sq = sizes[2] == 1 ? 0 : strides[2];
   for (int64_t s : {view->sb, view->sh, view->sq}) {
     if (s < 0) return fail(SMA_ERR_INVALID_ARG, "%s has a negative stride", name);
-    if ((s * esz) % 16 != 0)
+    if (!one_col && (s * esz) % 16 != 0)
       return fail(SMA_ERR_INVALID_ARG, "%s strides must be multiples of 16 bytes", name);
   }
   view->head_per_query = sizes[1] == H ? 1 : 0;
   for (int i = 0; i < 4; ++i) view->sizes[i] = sizes[i];
+  view->kd = static_cast<int>(sizes[3]);
   return SMA_OK;
 }
 
@@ -434,6 +448,16 @@ sma_status sma_selftest_wait_timeout(int64_t timeout_ns, int64_t* dev_out, void*
   return ok();
 }
 
+sma_status sma_selftest_exp2(const float* dev_in, float* dev_out, int64_t n, void* stream) {
+  if (dev_in == nullptr || dev_out == nullptr) return fail(SMA_ERR_INVALID_ARG, "NULL pointer");
+  if (n < 0 || (n & 1) != 0) return fail(SMA_ERR_INVALID_ARG, "n must be even and >= 0");
+  if ((reinterpret_cast<uintptr_t>(dev_in) & 3u) != 0 || (reinterpret_cast<uintptr_t>(dev_out) & 3u) != 0)
+    return fail(SMA_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
+  cudaError_t e = launch_exp2_fma_selftest(dev_in, dev_out, n, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch failed");
+  return ok();
+}
+
 sma_status dfa_block_map_dims(const dfa_mask_desc* desc, int32_t* q_tiles, int32_t* kv_tiles) {
   sma_status s = check_desc(desc);
   if (s != SMA_OK) return s;
@@ -731,9 +755,14 @@ sma_status dynamic_topk_mask(int32_t bias_dtype, const void* bias, const int64_t
   for (int i = 0; i < 3; ++i)
     if (bias_sizes[i] < 1) return fail(SMA_ERR_INVALID_ARG, "bias dims must be >= 1");
   const int64_t kpad = round_up(k_len, kTile);
-  if (bias_sizes[3] != kpad)
-    return fail(SMA_ERR_INVALID_ARG, "bias key dim must be round_up(k_len, 128) = %lld",
-                static_cast<long long>(kpad));
+  // The padded key dim of PR #190's contract, or the true key length.  A key
+  // dim of 1 (one value for every key) would rank every key equal; its
+  // output would not have one column per key, so it is refused.
+  if (bias_sizes[3] != kpad && bias_sizes[3] != k_len)
+    return fail(SMA_ERR_INVALID_ARG,
+                "bias key dim must be round_up(k_len, 128) = %lld or k_len = %d (the output mask "
+                "has one column per key of the bias)",
+                static_cast<long long>(kpad), k_len);
   if (bias_strides[3] != 1) return fail(SMA_ERR_INVALID_ARG, "bias last dim must be contiguous");
   if (!aligned16(bias)) return fail(SMA_ERR_INVALID_ARG, "bias must be 16-byte aligned");
   const int es = elem_size(bias_dtype);
@@ -747,7 +776,7 @@ sma_status dynamic_topk_mask(int32_t bias_dtype, const void* bias, const int64_t
       return fail(SMA_ERR_INVALID_ARG, "bias strides must be non-negative multiples of 16 bytes");
   }
   p.Lk = k_len;
-  p.Kpad = static_cast<int>(kpad);
+  p.Kcols = static_cast<int>(bias_sizes[3]);
   p.pre = pre_mask;
   if (pre_mask != nullptr) {
     if (pre_mask_sizes == nullptr || pre_mask_strides == nullptr)
@@ -884,10 +913,12 @@ sma_status sparse_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
     cb.sh = static_cast<int64_t>(g.Qc) * g.cap;
     cb.sb = static_cast<int64_t>(g.Hc) * g.Qc * g.cap;
     cb.head_per_query = g.Hc == heads && bview.head_per_query ? 1 : 0;
+    cb.kd = g.cap;  // compacted rows hold every column up to cap
     p.bias = cb;
   }
 
-  e = launch_select_keys(mask, mview.sb, mview.sh, g.LB, g.LH, k_len, g.cap, idx, count, err, st);
+  e = launch_select_keys(mask, mview.sb, mview.sh, mview.kd, g.LB, g.LH, k_len, g.cap, idx, count,
+                         err, st);
   if (e != cudaSuccess) return cuda_fail(e, "key selection launch failed");
   e = launch_gather_kv(p, k, k_strides, v, v_strides, st);
   if (e != cudaSuccess) return cuda_fail(e, "K/V gather launch failed");
@@ -1089,19 +1120,30 @@ sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   if (e != cudaSuccess) return cuda_fail(e, "tile list launch failed");
   set_grads(b, dout, do_strides, dq, dq_strides, dk, dk_strides, dv, dv_strides, sc);
   if (dbias != nullptr) {
-    // contiguous fp32 at the bias's sizes (b', h', q', round_up(Lk, 128))
-    const int64_t kp = round_up(k_len, kTile);
+    // contiguous fp32 at the bias's sizes (b', h', q', kd), kd the bias's key
+    // dim: round_up(Lk, 128), Lk, or 1
+    const int64_t kd = bias_sizes[3];
     const int64_t nb = bias_sizes[0], nh = bias_sizes[1], nq = bias_sizes[2];
-    b.dbias = dbias;
-    b.db_sq = nq > 1 ? kp : 0;
-    b.db_sh = nh > 1 ? nq * kp : 0;
-    b.db_sb = nb > 1 ? nh * nq * kp : 0;
-    b.db_head_per_query = bview.head_per_query;
-    const bool own_head = heads == 1 || (nh > 1 && (bview.head_per_query || p.group == 1));
-    const bool own_batch = batch == 1 || nb > 1;
-    b.db_mode = nq == 1 ? kDbiasRowSum : (own_head && own_batch ? kDbiasStore : kDbiasAdd);
-    e = cudaMemsetAsync(dbias, 0, static_cast<size_t>(nb * nh * nq * kp) * 4, st);
+    e = cudaMemsetAsync(dbias, 0, static_cast<size_t>(nb * nh * nq * kd) * 4, st);
     if (e != cudaSuccess) return cuda_fail(e, "dbias zeroing failed");
+    if (kd > 1 || k_len == 1) {
+      b.dbias = dbias;
+      b.db_sq = nq > 1 ? kd : 0;
+      b.db_sh = nh > 1 ? nq * kd : 0;
+      b.db_sb = nb > 1 ? nh * nq * kd : 0;
+      b.db_kd = static_cast<int>(kd);
+      // dbias has the bias's sizes: a head dim of `heads` is one row per
+      // query head even where the bias itself is read with stride 0
+      const int db_hpq = nh == heads ? 1 : 0;
+      b.db_head_per_query = db_hpq;
+      const bool own_head = heads == 1 || (nh > 1 && (db_hpq || p.group == 1));
+      const bool own_batch = batch == 1 || nb > 1;
+      b.db_mode = nq == 1 ? kDbiasRowSum : (own_head && own_batch ? kDbiasStore : kDbiasAdd);
+    }
+    // else: a bias with one value for every key adds the same amount to every
+    // score of a row, which softmax ignores; its gradient, the sum of dS over
+    // the row's keys, is exactly 0 (sum_k P (dP - D) = D - D), and the zeroed
+    // dbias is the result.
   }
   if ((s = run_backward(b, workspace, lay, st)) != SMA_OK) return s;
   return ok();

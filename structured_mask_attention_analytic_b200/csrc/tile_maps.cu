@@ -135,7 +135,7 @@ constexpr int kSummaryWarps = 8;
 
 __global__ void __launch_bounds__(kSummaryWarps * 32)
 mask_summary_kernel(const uint8_t* __restrict__ mask, int64_t m0, int64_t m1, int64_t m2,
-                    int64_t s0, int64_t s1, int64_t s2, int Lk, int QT, int KT,
+                    int64_t s0, int64_t s1, int64_t s2, int kd, int Lk, int QT, int KT,
                     uint8_t* __restrict__ codes) {
   const int lane = threadIdx.x & 31;
   const int64_t tile = static_cast<int64_t>(blockIdx.x) * kSummaryWarps + (threadIdx.x >> 5);
@@ -153,14 +153,28 @@ mask_summary_kernel(const uint8_t* __restrict__ mask, int64_t m0, int64_t m1, in
   const int nvalid_cols = max(0, min(16, Lk - k0));
   const int64_t rows_left = m2 - static_cast<int64_t>(qt) * kTile;
   const int rows = static_cast<int>(rows_left < kTile ? rows_left : kTile);
-  const uint8_t* base = mask + i0 * s0 + i1 * s1 + (static_cast<int64_t>(qt) * kTile) * s2 +
-                        static_cast<int64_t>(kt) * kTile + vec * 16;
+  const uint8_t* base = mask + i0 * s0 + i1 * s1 + (static_cast<int64_t>(qt) * kTile) * s2;
+  // rows of kd columns (round_up(Lk, 128), Lk, or 1 for every key): whole
+  // 16-byte chunks as vectors, the rest column by column inside the row
+  const bool whole = k0 + 16 <= kd;
   bool all_true = nvalid_cols == 16;
   bool any_true = false;
 #pragma unroll 4
   for (int r = lane >> 3; r < rows; r += 4) {
-    const uint4 v = *reinterpret_cast<const uint4*>(base + r * s2);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const uint8_t* mrow = base + r * s2;
+    uint32_t w[4];
+    if (whole) {
+      const uint4 v = *reinterpret_cast<const uint4*>(mrow + k0);
+      w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        w[e] = 0u;
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          w[e] |= static_cast<uint32_t>(mrow[aux_col(k0 + 4 * e + t, kd)]) << (8 * t);
+      }
+    }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       // per-byte nonzero -> 0xff
@@ -266,7 +280,8 @@ cudaError_t launch_mask_tile_summary(const uint8_t* mask, const int64_t sizes[4]
   if (n_tiles == 0) return cudaSuccess;
   const int64_t blocks = ceil_div(n_tiles, kSummaryWarps);
   mask_summary_kernel<<<static_cast<unsigned>(blocks), kSummaryWarps * 32, 0, stream>>>(
-      mask, sizes[0], sizes[1], sizes[2], strides[0], strides[1], strides[2], Lk, QT, KT, codes);
+      mask, sizes[0], sizes[1], sizes[2], strides[0], strides[1], strides[2],
+      static_cast<int>(sizes[3]), Lk, QT, KT, codes);
   return cudaGetLastError();
 }
 

@@ -79,7 +79,7 @@ struct RowCtx {
   const uint8_t* brow;  // bias row
   const uint8_t* prow;  // pre-mask row or null
   int pk;               // pre-mask length
-  int Lk, Kpad;
+  int Lk, Kcols;
 };
 
 template <int DT>
@@ -87,11 +87,16 @@ __device__ __forceinline__ void row_keys(const RowCtx& rc, int c, uint32_t (&key
                                          bool (&valid)[kPerThread], bool (&pm)[kPerThread]) {
   using T = KeyTraits<DT>;
   uint32_t u[kPerThread];
-  if (c < rc.Kpad) {
+  if (c + kPerThread <= rc.Kcols) {
     load_bits8<DT>(rc.brow, c, u);
-  } else {
+  } else {  // the row's last columns (rows of Lk columns need not end on a chunk)
 #pragma unroll
-    for (int e = 0; e < kPerThread; ++e) u[e] = 0;
+    for (int e = 0; e < kPerThread; ++e) {
+      const int k = c + e;
+      if (k >= rc.Kcols) u[e] = 0;
+      else if (DT == SMA_FP32) u[e] = reinterpret_cast<const uint32_t*>(rc.brow)[k];
+      else u[e] = reinterpret_cast<const uint16_t*>(rc.brow)[k];
+    }
   }
 #pragma unroll
   for (int e = 0; e < kPerThread; ++e) {
@@ -129,8 +134,9 @@ topk_mask_kernel(const TopkProblem p) {
                       (p.p_sizes[2] > 1 ? i2 : 0) * p.p_strides[2];
   rc.pk = p.pre == nullptr ? 0 : static_cast<int>(p.p_sizes[3]);
   rc.Lk = p.Lk;
-  rc.Kpad = p.Kpad;
-  uint8_t* orow = p.out + row * p.Kpad;
+  rc.Kcols = p.Kcols;
+  uint8_t* orow = p.out + row * p.Kcols;
+  const bool out8 = (reinterpret_cast<uintptr_t>(orow) & 7u) == 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const bool take_all = p.window >= p.Lk;
@@ -198,7 +204,7 @@ topk_mask_kernel(const TopkProblem p) {
   // Output pass: key > T, or key == T among the first `remaining` in index order.
   const uint32_t thr = prefix;
   uint32_t eq_before = 0;  // running count of key == T in earlier steps
-  for (int c0 = 0; c0 < p.Kpad; c0 += kRowStep) {
+  for (int c0 = 0; c0 < p.Kcols; c0 += kRowStep) {
     const int c = c0 + threadIdx.x * kPerThread;
     uint32_t key[kPerThread];
     bool valid[kPerThread], pm[kPerThread];
@@ -239,11 +245,15 @@ topk_mask_kernel(const TopkProblem p) {
       }
       out[e] = (keep && pm[e]) ? 1 : 0;
     }
-    if (c < p.Kpad) {
+    if (c + kPerThread <= p.Kcols && out8) {
       uint2 v;
       v.x = out[0] | (out[1] << 8) | (out[2] << 16) | (static_cast<uint32_t>(out[3]) << 24);
       v.y = out[4] | (out[5] << 8) | (out[6] << 16) | (static_cast<uint32_t>(out[7]) << 24);
       *reinterpret_cast<uint2*>(orow + c) = v;
+    } else {  // unaligned rows (Lk columns) and the row's last columns
+#pragma unroll
+      for (int e = 0; e < kPerThread; ++e)
+        if (c + e < p.Kcols) orow[c + e] = out[e];
     }
     eq_before += step_total;
   }
@@ -332,8 +342,13 @@ __device__ __forceinline__ void pre_lanes(uint32_t p4, uint32_t& m0, uint32_t& m
 }
 
 // Block-wide exclusive scan (one barrier); consecutive calls alternate `buf`.
+// After the barrier every warp scans the NT / 32 warp totals itself (lane w
+// holds warp w's), so each thread spends one shared load and a few shuffles
+// on them instead of reading all of them.
 template <int NT>
 __device__ __forceinline__ uint32_t scan_excl(uint32_t v, uint32_t* buf, uint32_t* total) {
+  constexpr int NW = NT / 32;
+  static_assert(NW <= 32, "one warp scans the warp totals");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t incl = v;
 #pragma unroll
@@ -343,14 +358,15 @@ __device__ __forceinline__ uint32_t scan_excl(uint32_t v, uint32_t* buf, uint32_
   }
   if (lane == 31) buf[warp] = incl;
   __syncthreads();
-  uint32_t base = 0, tot = 0;
+  const uint32_t wv = lane < NW ? buf[lane] : 0u;
+  uint32_t wincl = wv;
 #pragma unroll
-  for (int w = 0; w < NT / 32; ++w) {
-    const uint32_t sw = buf[w];
-    base += w < warp ? sw : 0u;
-    tot += sw;
+  for (int o = 1; o < NW; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, wincl, o);
+    if (lane >= o) wincl += t;
   }
-  *total = tot;
+  const uint32_t base = __shfl_sync(0xffffffffu, wincl - wv, warp);
+  *total = __shfl_sync(0xffffffffu, wincl, NW - 1);
   return base + incl - v;
 }
 
@@ -408,7 +424,7 @@ topk16_kernel(const TopkProblem p) {
   const int pk = p.pre == nullptr ? 0 : static_cast<int>(p.p_sizes[3]);
   const int Lk = p.Lk;
   const int c0 = SPAN * threadIdx.x;
-  const bool mine = c0 < p.Kpad;  // Kpad is a multiple of 128, so spans never straddle it
+  const bool mine = c0 < p.Kcols;  // Kcols is a multiple of 128 here, so spans never straddle it
 
   // ---- values
   uint32_t x[WORDS];
@@ -565,9 +581,7 @@ topk16_kernel(const TopkProblem p) {
         c = __reduce_add_sync(0xffffffffu, c) >> 4;
         if (lane == 0) s_red[red][warp] = c;
         __syncthreads();
-        uint32_t all = 0;
-#pragma unroll
-        for (int v2 = 0; v2 < NW; ++v2) all += s_red[red][v2];
+        const uint32_t all = __reduce_add_sync(0xffffffffu, lane < NW ? s_red[red][lane] : 0u);
         red ^= 1;
         return all;
       });
@@ -591,7 +605,7 @@ topk16_kernel(const TopkProblem p) {
   // below it, and are then cleared with the pre-mask.
   const bool and_pre = prow != nullptr && (take_all || T <= key16(H::kSentinel));
   if (!mine) return;
-  uint8_t* orow = p.out + static_cast<int64_t>(row) * p.Kpad + c0;
+  uint8_t* orow = p.out + static_cast<int64_t>(row) * p.Kcols + c0;
 #pragma unroll
   for (int i = 0; i < SPAN / 16; ++i) {
     uint32_t pmw[8];
@@ -651,7 +665,8 @@ cudaError_t launch_topk(const TopkProblem& p, cudaStream_t stream) {
   const bool few = rows < 2 * num_sms();
   // The register-resident kernel stores 16 bytes at a time.
   const bool out16 = (reinterpret_cast<uintptr_t>(p.out) & 15u) == 0;
-  if (p.bias_dtype != SMA_FP32 && p.Kpad <= 16384 && out16) {
+  // It also takes whole 128-column rows (the padded key dim) only.
+  if (p.bias_dtype != SMA_FP32 && p.Kcols <= 16384 && p.Kcols % kTile == 0 && out16) {
     if (p.bias_dtype == SMA_BF16) {
       if (few) topk16_kernel<SMA_BF16, 1024><<<grid, 1024, 0, stream>>>(p);
       else topk16_kernel<SMA_BF16, 512><<<grid, 512, 0, stream>>>(p);

@@ -246,7 +246,7 @@ def _aux_args(t, k_len):
     if t is None:
         return ctypes.c_void_p(0), None, None
     if t.dim() != 4:
-        raise ValueError("mask/bias must be 4D ({B|1}, {H|KVH|1}, {Lq|1}, round_up(Lk,128))")
+        raise ValueError("mask/bias must be 4D ({B|1}, {H|KVH|1}, {Lq|1}, {round_up(Lk,128)|Lk|1})")
     return _ptr(t), nat.i64_array(t.shape), nat.i64_array(t.stride())
 
 
@@ -275,10 +275,11 @@ def masked_attn_fwd(q, k, v, mask=None, bias=None, is_causal: bool = False, scal
                     return_lse: bool = True, workspace=None):
     """Attention forward with a broadcastable 4D bool mask and/or additive bias.
 
-    mask / bias follow ``({B|1}, {H|KVH|1}, {Lq|1}, round_up(Lk, 128))`` with a
-    contiguous last dim; broadcast dims may have any stride (they are read
-    with stride 0).  ``q_len == 1`` takes the grouped-head decode path.
-    Returns ``(out, lse)``."""
+    mask / bias follow ``({B|1}, {H|KVH|1}, {Lq|1}, {round_up(Lk, 128)|Lk|1})``
+    with a contiguous last dim; broadcast dims may have any stride (they are
+    read with stride 0), and a key dim of 1 is one value for every key.  No
+    padding or expansion is made: the kernels read each form in place.
+    ``q_len == 1`` takes the grouped-head decode path.  Returns ``(out, lse)``."""
     _require_cuda(q, k, v, mask, bias)
     b, lq, h, dh = q.shape
     lk, kvh = k.shape[1], k.shape[2]
@@ -319,7 +320,7 @@ def masked_attn_bwd(q, k, v, out, lse, dout, mask=None, bias=None, is_causal: bo
     ``out`` and ``lse`` are that call's results, ``dout`` the upstream
     gradient.  Returns ``(dq, dk, dv)``, or ``(dq, dk, dv, dbias)`` with
     ``return_dbias`` (or a ``dbias`` buffer): float32 at the bias's shape,
-    reduced over the dims the bias broadcasts along."""
+    reduced over the dims the bias broadcasts along (a key dim of 1 too)."""
     _require_cuda(q, k, v, out, lse, dout, mask, bias)
     b, lq, h, dh = q.shape
     lk, kvh = k.shape[1], k.shape[2]
@@ -515,7 +516,8 @@ def dynamic_topk_mask(bias: torch.Tensor, k_len: int, window_size: int, pre_mask
                       out=None) -> torch.Tensor:
     """Bool keep mask of ``bias``'s shape: per row the ``window_size`` largest
     entries among the first ``k_len`` columns after the pre-mask, and'ed with
-    the pre-mask."""
+    the pre-mask.  The bias's key dim is ``round_up(k_len, 128)`` or
+    ``k_len``."""
     _require_cuda(bias, pre_mask)
     if bias.dim() != 4:
         raise ValueError("bias must be 4D")
@@ -551,3 +553,15 @@ def selftest_wait_timeout(timeout_ns: int, out: torch.Tensor) -> None:
     if out.dtype != torch.int64 or out.numel() < 2:
         raise ValueError("out must be a CUDA int64 tensor with 2 elements")
     nat.check(_lib().sma_selftest_wait_timeout(int(timeout_ns), _ptr(out), _stream(out)))
+
+
+def selftest_exp2(x: torch.Tensor) -> torch.Tensor:
+    """Diagnostic: the softmax's FMA-pipe 2^x for a CUDA float32 tensor with
+    an even number of elements (see ``sma_selftest_exp2``)."""
+    _require_cuda(x)
+    if x.dtype != torch.float32 or x.numel() % 2:
+        raise ValueError("x must be a CUDA float32 tensor with an even number of elements")
+    x = x.contiguous()
+    out = torch.empty_like(x)
+    nat.check(_lib().sma_selftest_exp2(_ptr(x), _ptr(out), x.numel(), _stream(x)))
+    return out

@@ -117,7 +117,8 @@ def _masked_call(**over):
     (dict(qs=[256 * 4 * 128, 4 * 128 + 1, 128]), nat.SMA_ERR_INVALID_ARG, "16 bytes"),
     (dict(heads=3), nat.SMA_ERR_INVALID_ARG, "multiple"),
     (dict(head_dim=80), nat.SMA_ERR_UNSUPPORTED, "head_dim"),
-    (dict(mask=0x60000, msz=[1, 1, 256, 200], mst=[0, 0, 200, 1]), nat.SMA_ERR_INVALID_ARG, "round_up"),
+    (dict(mask=0x60000, msz=[1, 1, 256, 230], mst=[0, 0, 240, 1]), nat.SMA_ERR_INVALID_ARG, "round_up"),
+    (dict(mask=0x60000, msz=[1, 1, 256, 200], mst=[0, 0, 208, 2]), nat.SMA_ERR_INVALID_ARG, "contiguous"),
     (dict(mask=0x60000, msz=[1, 3, 256, 256], mst=[0, 0, 256, 1]), nat.SMA_ERR_INVALID_ARG, "head dim"),
     (dict(mask=0x60000, msz=[2, 1, 7, 256], mst=[256, 0, 256, 1]), nat.SMA_ERR_INVALID_ARG, "query dim"),
     (dict(mask=0x60000, msz=[1, 1, 256, 256], mst=[0, 0, 1, 256]), nat.SMA_ERR_INVALID_ARG, "contiguous"),
@@ -129,17 +130,44 @@ def test_masked_attn_validation(over, status, msg):
     assert msg in nat.load().sma_last_error().decode()
 
 
+@pytest.mark.parametrize("kd,kst", [(256, 1), (200, 1), (1, 1), (1, 0), (1, 7)], ids=str)
+@pytest.mark.parametrize("which", ["mask", "bias"])
+def test_masked_attn_accepts_the_three_key_dims(kd, kst, which):
+    """Key dim round_up(Lk, 128) = 256, Lk = 200, or 1 (any stride: one value
+    for every key).  An accepted call reaches the workspace check, which runs
+    after every shape check and before any CUDA call; a 16-byte workspace then
+    stops it, so the fake pointers are never used."""
+    rows = 208 if kd == 200 else kd    # 16-byte-multiple row strides
+    over = {which: 0x60000, which[0] + "sz": [1, 1, 256, kd], which[0] + "st": [0, 0, rows, kst],
+            "wsb": 16}
+    assert _masked_call(**over) == nat.SMA_ERR_WORKSPACE
+    assert "workspace" in nat.load().sma_last_error().decode()
+
+
 def test_topk_validation():
     lib = nat.load()
     bad_window = lib.dynamic_topk_mask(0, ctypes.c_void_p(0x10000), nat.i64_array([1, 1, 1, 256]),
                                        nat.i64_array([256, 256, 256, 1]), 200, None, None, None, 0,
                                        ctypes.c_void_p(0x20000), None)
     assert bad_window == nat.SMA_ERR_INVALID_ARG
-    bad_k = lib.dynamic_topk_mask(0, ctypes.c_void_p(0x10000), nat.i64_array([1, 1, 1, 200]),
-                                  nat.i64_array([200, 200, 200, 1]), 200, None, None, None, 8,
+    bad_k = lib.dynamic_topk_mask(0, ctypes.c_void_p(0x10000), nat.i64_array([1, 1, 1, 230]),
+                                  nat.i64_array([240, 240, 240, 1]), 200, None, None, None, 8,
                                   ctypes.c_void_p(0x20000), None)
     assert bad_k == nat.SMA_ERR_INVALID_ARG
     assert "round_up" in lib.sma_last_error().decode()
+    one = lib.dynamic_topk_mask(0, ctypes.c_void_p(0x10000), nat.i64_array([1, 1, 1, 1]),
+                                nat.i64_array([8, 8, 8, 1]), 200, None, None, None, 8,
+                                ctypes.c_void_p(0x20000), None)
+    assert one == nat.SMA_ERR_INVALID_ARG
+    assert "one column per key" in lib.sma_last_error().decode()
+    # key dims 256 and 200 pass the shape checks; the misaligned output
+    # pointer, checked last before the launch, then stops the call
+    for kd in (256, 200):
+        st = lib.dynamic_topk_mask(0, ctypes.c_void_p(0x10000), nat.i64_array([1, 1, 2, kd]),
+                                   nat.i64_array([512, 512, 256, 1]), 200, None, None, None, 8,
+                                   ctypes.c_void_p(0x20001), None)
+        assert st == nat.SMA_ERR_INVALID_ARG
+        assert "8-byte aligned" in lib.sma_last_error().decode()
     bad_pm = lib.dynamic_topk_mask(0, ctypes.c_void_p(0x10000), nat.i64_array([2, 1, 1, 256]),
                                    nat.i64_array([256, 256, 256, 1]), 200, ctypes.c_void_p(0x30000),
                                    nat.i64_array([3, 1, 1, 200]), nat.i64_array([200, 0, 0, 1]), 8,

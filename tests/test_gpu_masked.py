@@ -7,7 +7,7 @@ import torch
 import structured_mask_attention_analytic_b200 as sma
 import workloads as wl
 from oracle import attention as at
-from tests._helpers import assert_attention_close, f64, sample_tiles
+from tests._helpers import TOL, assert_attention_close, f64, sample_tiles
 
 pytestmark = pytest.mark.gpu
 
@@ -80,6 +80,11 @@ def test_padding_columns_never_matter():
 
 
 def test_stride0_equals_explicit_expand():
+    """A stride-0 view of a broadcast mask/bias is read exactly as the compact
+    tensor (bit-identical results); its contiguous expansion has a bias row
+    per query, which the softmax adds itself instead of the tensor cores
+    (rounding differs), so it agrees within the attention tolerance, and all
+    three match the oracle."""
     rng = wl.rng_for(10)
     q, k, v = _qkv(rng, B, LQ, LK, H, KVH, D)
     base_m = torch.from_numpy(rng.random((1, 1, LQ, KP)) < 0.8).cuda()
@@ -89,8 +94,13 @@ def test_stride0_equals_explicit_expand():
     o2, l2 = sma.masked_attn_fwd(qc, kc, vc, base_m.expand(B, H, LQ, KP).contiguous(),
                                  base_b.expand(B, H, LQ, KP).contiguous())
     o3, l3 = sma.masked_attn_fwd(qc, kc, vc, base_m, base_b)
-    assert torch.equal(o1, o2) and torch.equal(o1, o3)
-    assert torch.equal(l1, l2) and torch.equal(l1, l3)
+    assert torch.equal(o1, o3) and torch.equal(l1, l3)
+    mx, mn = TOL[torch.bfloat16]
+    err = (o1.double() - o2.double()).abs()
+    assert err.max().item() <= mx and err.mean().item() <= mn
+    ref_o, ref_l = _oracle(q, k, v, base_m.cpu(), base_b.cpu(), False)
+    for o, l in ((o1, l1), (o2, l2)):
+        assert_attention_close(o, l, ref_o, ref_l, torch.bfloat16, what="stride 0")
 
 
 def test_fully_masked_rows_are_zero():
@@ -219,3 +229,20 @@ def test_query_broadcast_bias_large_values(bshape, dtype, d):
     if dead:
         heads = slice(1 * (H // KVH), 2 * (H // KVH))
         assert (out[1, :, heads] == 0).all() and torch.isneginf(lse[1, heads]).all()
+
+
+@pytest.mark.parametrize("h,kvh,lq,bshape", [(4, 4, 300, (2, 4, 1)), (16, 2, 40, (2, 2, 1)),
+                                             (8, 2, 300, (1, 1, 1)), (8, 8, 24, (1, 8, 1))], ids=str)
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("fp16", 64)])
+def test_query_broadcast_bias_through_the_tensor_cores(h, kvh, lq, bshape, dtype, d):
+    """A bias row shared by every query of S (and by the query heads a tile
+    pair holds) is added by one more K step of the Q K^T product: one head
+    per KV head with a bias per head, head-packed short queries with a bias
+    per KV head (key ranges split over SMs and merged), and a single row."""
+    rng = wl.rng_for(18)
+    lk = 3000
+    kp = sma.round_up_k(lk)
+    q, k, v = _qkv(rng, 2, lq, lk, h, kvh, d, dtype)
+    mask = torch.from_numpy(rng.random((2, 1, lq, kp)) < 0.7)
+    bias = (wl.normal(rng, bshape + (kp,), "fp32") * 4.0).to(q.dtype)
+    _run(q, k, v, mask, bias, True, what=f"tc bias {h}/{kvh} lq={lq} {bshape} {dtype}")
