@@ -414,7 +414,8 @@ sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
  *          lists); offsets that break a bound, are not ascending or exceed
  *          the totals raise SMA_ERR_DEVICE_INPUT in the device error word and
  *          leave that sequence's rows unwritten.
- * dtype    SMA_BF16 / SMA_FP16; head_dim 64 or 128.
+ * dtype    SMA_BF16 / SMA_FP16 (tensor cores) or SMA_FP32 (FFMA
+ *          arithmetic, no TF32); head_dim 64 or 128.
  * ---------------------------------------------------------------------- */
 
 sma_status varlen_attn_fwd_workspace_size(int32_t batch, int32_t max_q, int32_t max_k, size_t* bytes);
@@ -440,8 +441,8 @@ sma_status varlen_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t 
  * lse are that forward's results for the same arguments (lse required);
  * dout, dq [total_q, heads, d], dk, dv [total_k, kv_heads, d] with strides[2]
  * = {row, head}.  Keys of a sequence that none of its queries keeps get zero
- * dK / dV; rows with no kept key get zero dQ.  bf16 / fp16 only
- * (SMA_ERR_UNSUPPORTED for SMA_FP32); offsets as in varlen_attn_fwd. */
+ * dK / dV; rows with no kept key get zero dQ.  bf16 / fp16 on the tensor
+ * cores, fp32 with FFMA arithmetic; offsets as in varlen_attn_fwd. */
 sma_status varlen_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
                            int32_t head_dim, int32_t total_q, int32_t total_k, int32_t max_q,
                            int32_t max_k, float scale, int32_t is_causal, const int32_t* cu_seqlens_q,

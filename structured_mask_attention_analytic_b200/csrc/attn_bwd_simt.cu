@@ -15,7 +15,9 @@
 // of the transposed list, queries in chunks of 32 staged through shared
 // memory (Q, dO, lse, D); writes dK and dV.
 // The keep rule and bias of each (query, key) pair are evaluated exactly as
-// in the forward; on FULL pairs only the key-length bound applies.
+// in the forward; on FULL pairs only the key-length bound applies.  Packed
+// sequences (varlen): batch entry b is sequence b, its query and key rows
+// offset by the cumulative arrays, its per-row data at [H, total_q].
 #include "device_common.cuh"
 #include "kernels.h"
 
@@ -35,9 +37,10 @@ struct RowKeep {
 };
 
 template <int POLICY>
-__device__ __forceinline__ RowKeep row_keep(const AttnProblem& p, int b, int h, int hk, int q) {
+__device__ __forceinline__ RowKeep row_keep(const AttnProblem& p, int b, int h, int hk, int q,
+                                            const SeqRows& sr) {
   RowKeep r{};
-  r.valid = q < p.Lq;
+  r.valid = q < sr.lq;
   r.causal_lim = 0x7fffffff;
   if (!r.valid) return r;
   if (POLICY == kPolicyDflash) {
@@ -62,15 +65,16 @@ __device__ __forceinline__ RowKeep row_keep(const AttnProblem& p, int b, int h, 
       r.brow = reinterpret_cast<const uint8_t*>(p.bias.ptr) +
                (b * p.bias.sb + hb * p.bias.sh + static_cast<int64_t>(q) * p.bias.sq) * esz;
     }
-    if (p.causal) r.causal_lim = q + p.Lk - p.Lq;
+    if (p.causal) r.causal_lim = q + sr.lk - sr.lq;
   }
   return r;
 }
 
 // Is key k kept for the row (PARTIAL tiles evaluate the whole rule)?
 template <int POLICY>
-__device__ __forceinline__ bool keeps(const AttnProblem& p, const RowKeep& r, int k, bool partial) {
-  if (!r.valid || k >= p.Lk) return false;
+__device__ __forceinline__ bool keeps(const AttnProblem& p, const RowKeep& r, int k, bool partial,
+                                     const SeqRows& sr) {
+  if (!r.valid || k >= sr.lk) return false;
   if (!partial) return true;
   if (POLICY == kPolicyDflash) return (k >= r.clo && k < r.chi) || (k >= r.dlo && k < r.dhi);
   return k <= r.causal_lim && (r.mrow == nullptr || r.mrow[aux_col(k, p.mask.kd)] != 0);
@@ -93,7 +97,8 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dq_kernel(const BwdP
   const int hk = h / p.group;
   const int r = threadIdx.x >> 1, hf = threadIdx.x & 1;
   const int q = qt * kTile + r;
-  const RowKeep rk = row_keep<POLICY>(p, b, h, hk, q);
+  const SeqRows sr = seq_rows<POLICY>(p, b);  // packed sequences: this sequence's rows
+  const RowKeep rk = row_keep<POLICY>(p, b, h, hk, q, sr);
 
   const int lb = p.lists.LB > 1 ? b : 0;
   int lh = 0;
@@ -109,14 +114,15 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dq_kernel(const BwdP
   float qr[E], gr[E], acc[E];
   float lse2 = -INFINITY, dd = 0.f;
   if (rk.valid) {
-    const float l = p.lse[(static_cast<int64_t>(b) * p.H + h) * p.Lq + q];
+    const float l = p.lse[row_index<POLICY>(p, b, h, sr, q)];
     lse2 = l * kLog2e;
-    dd = bp.dvec[(static_cast<int64_t>(b) * p.H + h) * p.Lq + q];
+    dd = bp.dvec[row_index<POLICY>(p, b, h, sr, q)];
   }
 #pragma unroll
   for (int e = 0; e < E; ++e) {
-    const int64_t qi = b * p.q_sb + static_cast<int64_t>(q) * p.q_sr + h * p.q_sh + 2 * e + hf;
-    const int64_t gi = b * bp.do_sb + static_cast<int64_t>(q) * bp.do_sr + h * bp.do_sh + 2 * e + hf;
+    const int64_t qi = b * p.q_sb + static_cast<int64_t>(sr.q_off + q) * p.q_sr + h * p.q_sh + 2 * e + hf;
+    const int64_t gi =
+        b * bp.do_sb + static_cast<int64_t>(sr.q_off + q) * bp.do_sr + h * bp.do_sh + 2 * e + hf;
     qr[e] = rk.valid ? Q[qi] * p.scale_log2 : 0.f;
     gr[e] = rk.valid ? G[gi] : 0.f;
     acc[e] = 0.f;
@@ -135,9 +141,9 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dq_kernel(const BwdP
         const int kk = i / D, e = i - kk * D;
         const int k = c0 + kk;
         float kv = 0.f, vv = 0.f;
-        if (k < p.Lk) {
-          kv = K[b * p.k_sb + static_cast<int64_t>(k) * p.k_sr + hk * p.k_sh + e];
-          vv = V[b * p.v_sb + static_cast<int64_t>(k) * p.v_sr + hk * p.v_sh + e];
+        if (k < sr.lk) {
+          kv = K[b * p.k_sb + static_cast<int64_t>(sr.k_off + k) * p.k_sr + hk * p.k_sh + e];
+          vv = V[b * p.v_sb + static_cast<int64_t>(sr.k_off + k) * p.v_sr + hk * p.v_sh + e];
         }
         sk[kk][e] = kv;
         sv[kk][e] = vv;
@@ -153,13 +159,13 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dq_kernel(const BwdP
         s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
         dp += __shfl_xor_sync(0xffffffffu, dp, 1);
         const int k = c0 + kk;
-        if (POLICY != kPolicyDflash && rk.brow != nullptr && k < p.Lk)
+        if (POLICY != kPolicyDflash && rk.brow != nullptr && k < sr.lk)
           s2 = fmaf(load_any_as_float(rk.brow, p.bias.dtype, aux_col(k, p.bias.kd)), kLog2e, s2);
-        const bool keep = keeps<POLICY>(p, rk, k, partial) && lse2 != -INFINITY;
+        const bool keep = keeps<POLICY>(p, rk, k, partial, sr) && lse2 != -INFINITY;
         const float ds = ds_of(s2, lse2, dp, dd, keep);
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] = fmaf(ds, sk[kk][2 * e + hf], acc[e]);
-        if (dbrow != nullptr && hf == 0 && k < p.Lk && k < bp.db_kd) {
+        if (dbrow != nullptr && hf == 0 && k < sr.lk && k < bp.db_kd) {
           if (bp.db_mode == kDbiasStore) dbrow[k] = ds;
           else if (ds != 0.f) atomicAdd(dbrow + k, ds);
         }
@@ -167,7 +173,10 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dq_kernel(const BwdP
     }
   }
   if (rk.valid) {
-    float* A = bp.dq_acc + ((static_cast<int64_t>(b) * p.Lq + q) * p.H + h) * D;
+    // [B, Lq, H, d], or [total_q, H, d] for packed sequences
+    const int64_t arow = POLICY == kPolicyVarlen ? static_cast<int64_t>(sr.q_off) + q
+                                                 : static_cast<int64_t>(b) * p.Lq + q;
+    float* A = bp.dq_acc + (arow * p.H + h) * D;
 #pragma unroll
     for (int e = 0; e < E; ++e) A[2 * e + hf] = acc[e];
   }
@@ -183,7 +192,8 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dkv_kernel(const Bwd
   const int kt = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int r = threadIdx.x >> 1, hf = threadIdx.x & 1;
   const int k = kt * kTile + r;
-  const bool key_valid = k < p.Lk;
+  const SeqRows sr = seq_rows<POLICY>(p, b);  // packed sequences: this sequence's rows
+  const bool key_valid = k < sr.lk;
   const float* Q = reinterpret_cast<const float*>(p.q);
   const float* K = reinterpret_cast<const float*>(p.k);
   const float* V = reinterpret_cast<const float*>(p.v);
@@ -191,8 +201,10 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dkv_kernel(const Bwd
   float kr[E], vr[E], dk[E], dv[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
-    kr[e] = key_valid ? K[b * p.k_sb + static_cast<int64_t>(k) * p.k_sr + hk * p.k_sh + 2 * e + hf] : 0.f;
-    vr[e] = key_valid ? V[b * p.v_sb + static_cast<int64_t>(k) * p.v_sr + hk * p.v_sh + 2 * e + hf] : 0.f;
+    kr[e] = key_valid ? K[b * p.k_sb + static_cast<int64_t>(sr.k_off + k) * p.k_sr + hk * p.k_sh + 2 * e + hf]
+                      : 0.f;
+    vr[e] = key_valid ? V[b * p.v_sb + static_cast<int64_t>(sr.k_off + k) * p.v_sr + hk * p.v_sh + 2 * e + hf]
+                      : 0.f;
     dk[e] = 0.f;
     dv[e] = 0.f;
   }
@@ -213,9 +225,9 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dkv_kernel(const Bwd
           const int qq = i / D, e = i - qq * D;
           const int q = c0 + qq;
           float qv = 0.f, gv = 0.f;
-          if (q < p.Lq) {
-            qv = Q[b * p.q_sb + static_cast<int64_t>(q) * p.q_sr + h * p.q_sh + e];
-            gv = G[b * bp.do_sb + static_cast<int64_t>(q) * bp.do_sr + h * bp.do_sh + e];
+          if (q < sr.lq) {
+            qv = Q[b * p.q_sb + static_cast<int64_t>(sr.q_off + q) * p.q_sr + h * p.q_sh + e];
+            gv = G[b * bp.do_sb + static_cast<int64_t>(sr.q_off + q) * bp.do_sr + h * bp.do_sh + e];
           }
           sq[qq][e] = qv;
           sg[qq][e] = gv;
@@ -223,9 +235,9 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dkv_kernel(const Bwd
         if (threadIdx.x < kBsChunk) {
           const int q = c0 + threadIdx.x;
           float l2 = -INFINITY, dd = 0.f;
-          if (q < p.Lq) {
-            l2 = p.lse[(static_cast<int64_t>(b) * p.H + h) * p.Lq + q] * kLog2e;
-            dd = bp.dvec[(static_cast<int64_t>(b) * p.H + h) * p.Lq + q];
+          if (q < sr.lq) {
+            l2 = p.lse[row_index<POLICY>(p, b, h, sr, q)] * kLog2e;
+            dd = bp.dvec[row_index<POLICY>(p, b, h, sr, q)];
           }
           sl[threadIdx.x] = l2;
           sd[threadIdx.x] = dd;
@@ -242,10 +254,10 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dkv_kernel(const Bwd
           s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
           dp += __shfl_xor_sync(0xffffffffu, dp, 1);
           s2 *= p.scale_log2;
-          const RowKeep rk = row_keep<POLICY>(p, b, h, hk, q);
+          const RowKeep rk = row_keep<POLICY>(p, b, h, hk, q, sr);
           if (POLICY != kPolicyDflash && rk.brow != nullptr && key_valid)
             s2 = fmaf(load_any_as_float(rk.brow, p.bias.dtype, aux_col(k, p.bias.kd)), kLog2e, s2);
-          const bool keep = key_valid && keeps<POLICY>(p, rk, k, partial) && sl[qq] != -INFINITY;
+          const bool keep = key_valid && keeps<POLICY>(p, rk, k, partial, sr) && sl[qq] != -INFINITY;
           const float pr = keep ? exp2f(s2 - sl[qq]) : 0.f;
           const float ds = pr * (dp - sd[qq]);
 #pragma unroll
@@ -262,8 +274,9 @@ __global__ void __launch_bounds__(kBsThreads) attn_bwd_simt_dkv_kernel(const Bwd
     float* DV = reinterpret_cast<float*>(bp.dv);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      DK[b * bp.dk_sb + static_cast<int64_t>(k) * bp.dk_sr + hk * bp.dk_sh + 2 * e + hf] = dk[e] * bp.scale;
-      DV[b * bp.dv_sb + static_cast<int64_t>(k) * bp.dv_sr + hk * bp.dv_sh + 2 * e + hf] = dv[e];
+      DK[b * bp.dk_sb + static_cast<int64_t>(sr.k_off + k) * bp.dk_sr + hk * bp.dk_sh + 2 * e + hf] =
+          dk[e] * bp.scale;
+      DV[b * bp.dv_sb + static_cast<int64_t>(sr.k_off + k) * bp.dv_sr + hk * bp.dv_sh + 2 * e + hf] = dv[e];
     }
   }
 }
@@ -283,11 +296,14 @@ cudaError_t launch_typed(const BwdProblem& p, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_attn_bwd_simt(const BwdProblem& p, cudaStream_t stream) {
-  if (p.f.d == 128)
-    return p.f.policy == kPolicyDflash ? launch_typed<128, kPolicyDflash>(p, stream)
-                                       : launch_typed<128, kPolicyExplicit>(p, stream);
-  return p.f.policy == kPolicyDflash ? launch_typed<64, kPolicyDflash>(p, stream)
-                                     : launch_typed<64, kPolicyExplicit>(p, stream);
+  if (p.f.d == 128) {
+    if (p.f.policy == kPolicyDflash) return launch_typed<128, kPolicyDflash>(p, stream);
+    if (p.f.policy == kPolicyVarlen) return launch_typed<128, kPolicyVarlen>(p, stream);
+    return launch_typed<128, kPolicyExplicit>(p, stream);
+  }
+  if (p.f.policy == kPolicyDflash) return launch_typed<64, kPolicyDflash>(p, stream);
+  if (p.f.policy == kPolicyVarlen) return launch_typed<64, kPolicyVarlen>(p, stream);
+  return launch_typed<64, kPolicyExplicit>(p, stream);
 }
 
 }  // namespace sma

@@ -5,7 +5,8 @@
 //
 // One CTA per (batch, query head, 128-row query tile); two threads per row,
 // each owning the even or odd half of head_dim; keys in chunks of 32 staged
-// through shared memory.
+// through shared memory.  Packed sequences (varlen): batch entry b is
+// sequence b, its rows offset by the cumulative arrays.
 #include "device_common.cuh"
 #include "gather.cuh"
 #include "kernels.h"
@@ -26,7 +27,8 @@ attn_simt_kernel(const AttnProblem p) {
   const int hk = h / p.group;
   const int r = threadIdx.x >> 1, hf = threadIdx.x & 1;
   const int q = qt * kTile + r;
-  const bool row_valid = q < p.Lq;
+  const SeqRows sr = seq_rows<POLICY>(p, b);  // packed sequences: this sequence's rows
+  const bool row_valid = q < sr.lq;
 
   const int lb = p.lists.LB > 1 ? b : 0;
   int lh = 0;
@@ -41,7 +43,8 @@ attn_simt_kernel(const AttnProblem p) {
   float qr[E], o[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
-    qr[e] = row_valid ? Q[b * p.q_sb + static_cast<int64_t>(q) * p.q_sr + h * p.q_sh + 2 * e + hf] *
+    qr[e] = row_valid ? Q[b * p.q_sb + static_cast<int64_t>(sr.q_off + q) * p.q_sr + h * p.q_sh +
+                          2 * e + hf] *
                             p.scale_log2
                       : 0.f;
     o[e] = 0.f;
@@ -79,7 +82,7 @@ attn_simt_kernel(const AttnProblem p) {
     if (p.gather.idx != nullptr)  // compacted keys: the row's limit on the compacted index
       causal_lim = row_valid ? gather_row_limit(p, static_cast<int64_t>(lb) * p.lists.LH + lh, q) - 1 : -1;
     else if (p.causal)
-      causal_lim = q + p.Lk - p.Lq;
+      causal_lim = q + sr.lk - sr.lq;
   }
 
   float m = -INFINITY, l = 0.f;
@@ -93,9 +96,9 @@ attn_simt_kernel(const AttnProblem p) {
         const int kk = i / D, e = i - kk * D;
         const int k = c0 + kk;
         float kv = 0.f, vv = 0.f;
-        if (k < p.Lk) {
-          kv = K[b * p.k_sb + static_cast<int64_t>(k) * p.k_sr + hk * p.k_sh + e];
-          vv = V[b * p.v_sb + static_cast<int64_t>(k) * p.v_sr + hk * p.v_sh + e];
+        if (k < sr.lk) {
+          kv = K[b * p.k_sb + static_cast<int64_t>(sr.k_off + k) * p.k_sr + hk * p.k_sh + e];
+          vv = V[b * p.v_sb + static_cast<int64_t>(sr.k_off + k) * p.v_sr + hk * p.v_sh + e];
         }
         sk[kk][e] = kv;
         sv[kk][e] = vv;
@@ -110,14 +113,14 @@ attn_simt_kernel(const AttnProblem p) {
         for (int e = 0; e < E; ++e) acc = fmaf(qr[e], sk[kk][2 * e + hf], acc);
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
         const int k = c0 + kk;
-        if (POLICY != kPolicyDflash && p.has_bias && k < p.Lk)
+        if (POLICY != kPolicyDflash && p.has_bias && k < sr.lk)
           acc = fmaf(load_any_as_float(brow, p.bias.dtype, aux_col(k, p.bias.kd)), kLog2e, acc);
         bool keep = row_valid;
         if (partial) {
           if (POLICY == kPolicyDflash) {
             keep = keep && ((k >= clo && k < chi) || (k >= dlo && k < dhi));
           } else {
-            keep = keep && k < p.Lk && k <= causal_lim && (!p.has_mask || mrow[aux_col(k, p.mask.kd)] != 0);
+            keep = keep && k < sr.lk && k <= causal_lim && (!p.has_mask || mrow[aux_col(k, p.mask.kd)] != 0);
           }
         }
         s[kk] = keep ? acc : -INFINITY;
@@ -145,10 +148,9 @@ attn_simt_kernel(const AttnProblem p) {
     const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e)
-      O[b * p.o_sb + static_cast<int64_t>(q) * p.o_sr + h * p.o_sh + 2 * e + hf] = o[e] * inv;
+      O[b * p.o_sb + static_cast<int64_t>(sr.q_off + q) * p.o_sr + h * p.o_sh + 2 * e + hf] = o[e] * inv;
     if (hf == 0 && p.lse != nullptr)
-      p.lse[(static_cast<int64_t>(b) * p.H + h) * p.Lq + q] =
-          l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+      p.lse[row_index<POLICY>(p, b, h, sr, q)] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
   }
 }
 
@@ -160,11 +162,15 @@ cudaError_t launch_attn_simt(const AttnProblem& p, cudaStream_t stream) {
   if (p.d == 128) {
     if (p.policy == kPolicyDflash)
       attn_simt_kernel<128, kPolicyDflash><<<grid, kSimtThreads, 0, stream>>>(p);
+    else if (p.policy == kPolicyVarlen)
+      attn_simt_kernel<128, kPolicyVarlen><<<grid, kSimtThreads, 0, stream>>>(p);
     else
       attn_simt_kernel<128, kPolicyExplicit><<<grid, kSimtThreads, 0, stream>>>(p);
   } else {
     if (p.policy == kPolicyDflash)
       attn_simt_kernel<64, kPolicyDflash><<<grid, kSimtThreads, 0, stream>>>(p);
+    else if (p.policy == kPolicyVarlen)
+      attn_simt_kernel<64, kPolicyVarlen><<<grid, kSimtThreads, 0, stream>>>(p);
     else
       attn_simt_kernel<64, kPolicyExplicit><<<grid, kSimtThreads, 0, stream>>>(p);
   }

@@ -162,6 +162,38 @@ struct BwdProblem {
   int db_mode = 0;  // kDbias* below
 };
 
+#ifdef __CUDACC__
+// Rows of one sequence (batch entry b): its first query / key row and its
+// lengths.  Packed sequences (varlen) take them from the cumulative offsets;
+// malformed offsets give an empty sequence (nothing of it is read or
+// written; the list kernel reports them).  Padded batches: row 0, Lq, Lk.
+struct SeqRows {
+  int q_off, lq, k_off, lk;
+};
+template <int POLICY>
+__device__ __forceinline__ SeqRows seq_rows(const AttnProblem& p, int b) {
+  SeqRows s{0, p.Lq, 0, p.Lk};
+  if (POLICY == kPolicyVarlen) {
+    s.q_off = p.cu_q[b];
+    s.lq = p.cu_q[b + 1] - s.q_off;
+    s.k_off = p.cu_k[b];
+    s.lk = p.cu_k[b + 1] - s.k_off;
+    if (s.lq < 0 || s.lq > p.Lq || s.q_off < 0 || s.q_off + s.lq > p.total_q || s.lk < 0 ||
+        s.lk > p.Lk || s.k_off < 0 || s.k_off + s.lk > p.total_k)
+      s = SeqRows{0, 0, 0, 0};
+  }
+  return s;
+}
+// Index of (b, h, q) in the per-row float arrays (lse, rowsum(dO * O)):
+// [B, H, Lq], or [H, total_q] for packed sequences.
+template <int POLICY>
+__device__ __forceinline__ int64_t row_index(const AttnProblem& p, int b, int h, const SeqRows& s,
+                                             int q) {
+  return POLICY == kPolicyVarlen ? static_cast<int64_t>(h) * p.total_q + s.q_off + q
+                                 : (static_cast<int64_t>(b) * p.H + h) * p.Lq + q;
+}
+#endif
+
 // How the backward writes dbias: not at all; one store per element (every
 // element of dS has its own dbias element); one atomic add per element
 // (several heads or batch rows share an element); one atomic add of each

@@ -1166,8 +1166,6 @@ sma_status varlen_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
                            const int64_t v_strides[2], void* out, const int64_t o_strides[2],
                            float* lse, void* workspace, size_t workspace_bytes, void* stream) {
   if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
-  if (dtype == SMA_FP32)
-    return fail(SMA_ERR_UNSUPPORTED, "varlen attention runs on the tensor cores: bf16 or fp16 only");
   sma_status s = check_heads(heads, kv_heads, head_dim);
   if (s != SMA_OK) return s;
   if (batch < 1 || total_q < 1 || total_k < 1 || max_q < 1 || max_k < 1)
@@ -1221,6 +1219,11 @@ sma_status varlen_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   e = launch_varlen_lists(p, at<int32_t>(workspace, lay.nf), at<int32_t>(workspace, lay.fi),
                           at<int32_t>(workspace, lay.np), at<int32_t>(workspace, lay.pi), st);
   if (e != cudaSuccess) return cuda_fail(e, "tile list launch failed");
+  if (dtype == SMA_FP32) {
+    e = launch_attn_simt(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch failed");
+    return ok();
+  }
   char msg[256];
   const int rc = launch_attn_tc(p, st, msg, sizeof(msg));
   if (rc != SMA_OK) return fail(rc, "%s", msg);
@@ -1253,8 +1256,6 @@ sma_status varlen_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   sma_status s = check_heads(heads, kv_heads, head_dim);
   if (s != SMA_OK) return s;
-  if (dtype == SMA_FP32)
-    return fail(SMA_ERR_UNSUPPORTED, "varlen attention runs on the tensor cores: bf16 or fp16 only");
   if (batch < 1 || total_q < 1 || total_k < 1 || max_q < 1 || max_k < 1)
     return fail(SMA_ERR_INVALID_ARG, "batch, totals and maxima must be >= 1");
   if (is_causal != 0 && is_causal != 1) return fail(SMA_ERR_INVALID_ARG, "is_causal must be 0 or 1");

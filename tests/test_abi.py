@@ -253,14 +253,20 @@ def test_backward_workspace_and_validation_on_host():
             ctypes.c_void_p(0x90000), nat.i64_array(ks), ctypes.c_void_p(dbias),
             ctypes.c_void_p(0xa0000), 1 << 30, None)
 
-    # packed batches have no fp32 backward: rejected before anything runs
+    # packed batches: an unknown dtype code is rejected before anything runs
     s2 = nat.i64_array([1024, 128])
+    assert lib.varlen_attn_bwd(9, 2, 8, 2, 128, 100, 100, 64, 64, ctypes.c_float(0.0), 0,
+                               ctypes.c_void_p(0x10000), ctypes.c_void_p(0x11000),
+                               *([ctypes.c_void_p(0x20000), s2] * 4), ctypes.c_void_p(0x70000),
+                               *([ctypes.c_void_p(0x20000), s2] * 4), ctypes.c_void_p(0xa0000),
+                               1 << 30, None) == nat.SMA_ERR_INVALID_ARG
+    assert "unknown dtype" in lib.sma_last_error().decode()
+    # fp32 packed gradients are accepted up to the workspace check (too small here)
     assert lib.varlen_attn_bwd(2, 2, 8, 2, 128, 100, 100, 64, 64, ctypes.c_float(0.0), 0,
                                ctypes.c_void_p(0x10000), ctypes.c_void_p(0x11000),
                                *([ctypes.c_void_p(0x20000), s2] * 4), ctypes.c_void_p(0x70000),
                                *([ctypes.c_void_p(0x20000), s2] * 4), ctypes.c_void_p(0xa0000),
-                               1 << 30, None) == nat.SMA_ERR_UNSUPPORTED
-    assert "bf16 or fp16" in lib.sma_last_error().decode()
+                               16, None) == nat.SMA_ERR_WORKSPACE
     assert call(lse=0) == nat.SMA_ERR_INVALID_ARG
     assert "lse" in lib.sma_last_error().decode()
     assert call(dbias=0xb0000) == nat.SMA_ERR_INVALID_ARG  # no bias to take the gradient of
@@ -284,8 +290,8 @@ def test_varlen_validation_on_host():
                              ctypes.c_void_p(0x20000), nat.i64_array([256, 128]),
                              ctypes.c_void_p(0x30000), nat.i64_array([256, 128]),
                              ctypes.c_void_p(0x40000), nat.i64_array([512, 128]), None,
-                             ctypes.c_void_p(0x50000), 1 << 20, None)
-    assert st == nat.SMA_ERR_UNSUPPORTED
+                             ctypes.c_void_p(0x50000), 16, None)
+    assert st == nat.SMA_ERR_WORKSPACE   # fp32 is accepted; the 16-byte workspace is not
     st = lib.varlen_attn_fwd(0, 2, 4, 2, 128, 100, 100, 60, 60, ctypes.c_float(0.0), 0,
                              ctypes.c_void_p(0), ctypes.c_void_p(0x200),
                              ctypes.c_void_p(0x10000), nat.i64_array([512, 128]),

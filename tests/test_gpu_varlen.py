@@ -1,5 +1,6 @@
-"""GPU: varlen_attn_fwd (packed variable-length sequences on the tensor-core
-kernel) agrees with the float64 oracle; pad / unpad are exact inverses;
+"""GPU: varlen_attn_fwd / varlen_attn_bwd (packed variable-length sequences:
+bf16 / fp16 on the tensor-core kernels, fp32 on the FFMA kernels) agree with
+the float64 oracle; pad / unpad are exact inverses;
 malformed offsets are reported without writing outside the tensors."""
 import numpy as np
 import pytest
@@ -102,17 +103,37 @@ def test_malformed_offsets_are_reported():
 
 # Gradient agreement as for the padded backward: relative to m = max(1,
 # max |ref|) of each tensor, max-abs <= 2.5e-2 m and mean-abs <= 2.5e-3 m.
+# fp32 inputs (FFMA arithmetic): max-abs <= 1e-4 m and mean-abs <= 1e-5 m.
 def _close_grad(name, got, ref):
     g = f64(got)
     m = max(1.0, float(np.abs(ref).max()))
+    tmax, tmean = (1e-4, 1e-5) if got.dtype == torch.float32 else (2.5e-2, 2.5e-3)
     err = np.abs(g - ref)
     assert np.isfinite(g).all(), f"{name}: non-finite"
-    assert err.max() <= 2.5e-2 * m, f"{name}: max abs err {err.max():.3e} (scale {m:.2f})"
-    assert err.mean() <= 2.5e-3 * m, f"{name}: mean abs err {err.mean():.3e} (scale {m:.2f})"
+    assert err.max() <= tmax * m, f"{name}: max abs err {err.max():.3e} (scale {m:.2f})"
+    assert err.mean() <= tmean * m, f"{name}: mean abs err {err.mean():.3e} (scale {m:.2f})"
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("D,dtype", [(128, "bf16"), (64, "bf16"), (128, "fp16")])
+@pytest.mark.parametrize("D", [64, 128])
+def test_varlen_fp32_forward(causal, D):
+    """fp32 packed sequences on the FFMA kernel: the fp32 bound (1e-4 max-abs)
+    over ragged lengths, an empty sequence and causal rows with no key."""
+    rng = wl.rng_for(55)
+    lq = [300, 1, 0, 129, 77, 200]
+    lk = [300, 5, 7, 260, 40, 128]
+    cu_q, cu_k, q, k, v = _case(rng, lq, lk, 4, 2, D, "fp32")
+    out, lse = sma.varlen_attn_fwd(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(cu_q).cuda(),
+                                   torch.from_numpy(cu_k).cuda(), max(lq), max(lk), causal)
+    torch.cuda.synchronize()
+    assert sma.device_status() == 0
+    ref_o, ref_l = at.varlen_attention(f64(q), f64(k), f64(v), cu_q, cu_k, causal)
+    _check(out, lse, ref_o, ref_l, q.dtype, f"varlen fp32 causal={causal} D={D}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("D,dtype", [(128, "bf16"), (64, "bf16"), (128, "fp16"), (64, "fp32"),
+                                     (128, "fp32")])
 def test_varlen_backward(causal, D, dtype):
     """dQ, dK, dV of packed sequences against the float64 gradients of each
     sequence on its own: lengths spanning several tiles and ragged tails, one
