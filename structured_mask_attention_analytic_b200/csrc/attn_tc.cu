@@ -773,9 +773,9 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
         }
         if (m_ref == -INFINITY) m_ref = m_new;
         const float msub = m_ref == -INFINITY ? 0.f : m_ref;
-        float ls8[8];
+        float2 ls4[4];  // this tile's row sum, four chains of pairs
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ls8[e] = 0.f;
+        for (int e = 0; e < 4; ++e) ls4[e] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < kTile / 32; ++c) {
           uint32_t pk[16];
@@ -783,18 +783,15 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
           for (int e = 0; e < 16; ++e) {
             const float2 t = fma2(make_float2(x[32 * c + 2 * e], x[32 * c + 2 * e + 1]),
                                   make_float2(exp_scale, exp_scale), make_float2(-msub, -msub));
-            float p0, p1;
+            float2 pp;
             if (exp2_pair_on_fma(e)) {
-              const float2 pp = exp2_fma2(t);
-              p0 = pp.x;
-              p1 = pp.y;
+              pp = exp2_fma2(t);
             } else {
-              p0 = fast_exp2(t.x);
-              p1 = fast_exp2(t.y);
+              pp.x = fast_exp2(t.x);
+              pp.y = fast_exp2(t.y);
             }
-            ls8[(2 * e) & 7] += p0;
-            ls8[(2 * e + 1) & 7] += p1;
-            pk[e] = DT == SMA_BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+            ls4[e & 3] = add2(ls4[e & 3], pp);
+            pk[e] = DT == SMA_BF16 ? pack_bf16x2(pp.x, pp.y) : pack_f16x2(pp.x, pp.y);
           }
           // P columns [16c, 16c+16) of the packed pairs
           asm volatile(
@@ -806,11 +803,10 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
               "r"(pk[12]), "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
               : "memory");
         }
-#pragma unroll
-        for (int w2 = 4; w2 >= 1; w2 >>= 1)
-#pragma unroll
-          for (int e = 0; e < w2; ++e) ls8[e] += ls8[e + w2];
-        l_sum += ls8[0];
+        {
+          const float2 a2 = add2(add2(ls4[0], ls4[1]), add2(ls4[2], ls4[3]));
+          l_sum += a2.x + a2.y;
+        }
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(bar(L::kPBar + qi));

@@ -436,8 +436,9 @@ __device__ __forceinline__ float2 exp2_fma2(float2 t) {
   float2 p = fma2(f, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
   p = fma2(p, f, make_float2(kExp2C1, kExp2C1));
   p = fma2(p, f, make_float2(kExp2C0, kExp2C0));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
+  // n << 23 added to the exponent field as one integer multiply-add
+  return make_float2(__uint_as_float(__float_as_uint(j.x) * 8388608u + __float_as_uint(p.x)),
+                     __uint_as_float(__float_as_uint(j.y) * 8388608u + __float_as_uint(p.y)));
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
