@@ -17,7 +17,8 @@
  *   sparse_attn_fwd    masked_attn_fwd over only the keys a query-broadcast
  *                      mask keeps (index gather), e.g. a top-k mask.
  *   dfa_attn_bwd,      gradients dQ, dK, dV of the two attention forwards.
- *   masked_attn_bwd
+ *   masked_attn_bwd    (and masked_attn_bwd_deterministic: dbias summed in a
+ *                      fixed order)
  *   varlen_attn_fwd    attention over packed variable-length sequences, with
  *                      varlen_pad / varlen_unpad.
  *
@@ -378,8 +379,8 @@ sma_status masked_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t 
  * bias value for every key of a row) the sum over the row's keys is exactly
  * 0 (sum_k P (dP - D) = D - D): the call writes zeros.
  * The call zeroes dbias first; sums over broadcast dims use fp32 atomic
- * adds, so their rounding order is not fixed.  Needs a bias (
- * SMA_ERR_INVALID_ARG otherwise). */
+ * adds, so their rounding order is not fixed (masked_attn_bwd_deterministic
+ * fixes it).  Needs a bias (SMA_ERR_INVALID_ARG otherwise). */
 sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
                            int32_t q_len, int32_t k_len, int32_t head_dim, float scale,
                            int32_t is_causal, const void* q, const int64_t q_strides[3],
@@ -393,6 +394,38 @@ sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
                            void* dk, const int64_t dk_strides[3], void* dv,
                            const int64_t dv_strides[3], float* dbias, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/* Bytes of the second workspace masked_attn_bwd_deterministic needs for a
+ * bias of sizes bias_sizes (b', h', q', kd): the fixed-order partial sums,
+ * batch * heads * R * kd * 4 with R = q_len for a bias with a query dim (or
+ * dtype SMA_FP32), else ceil(q_len / G) (G = 64 at head_dim 128, 32 at 64).
+ * 0 when every dbias element already has a single writer (a bias with its
+ * own element for each batch row, query head and query). */
+sma_status masked_attn_bwd_dbias_workspace_size(int32_t dtype, int32_t batch, int32_t heads,
+                                                int32_t kv_heads, int32_t q_len, int32_t head_dim,
+                                                const int64_t bias_sizes[4], size_t* bytes);
+
+/* masked_attn_bwd with a dbias that is bitwise the same on every call with
+ * the same inputs.  The page (PR #190, Changes: dbias reduced over the
+ * broadcast dims) fixes the sums but no order; this entry point fixes one:
+ * every element of the partial buffer (dbias_workspace, device, at least
+ * masked_attn_bwd_dbias_workspace_size bytes, caller-owned) has exactly one
+ * writer, per batch row, query head and query (or group of G queries), and
+ * one kernel then adds the partials of each dbias element in increasing
+ * (batch, head, partial row) order.  dQ / dK / dV are those of
+ * masked_attn_bwd.  SMA_ERR_WORKSPACE if dbias_workspace is smaller than the
+ * query says. */
+sma_status masked_attn_bwd_deterministic(
+    int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads, int32_t q_len, int32_t k_len,
+    int32_t head_dim, float scale, int32_t is_causal, const void* q, const int64_t q_strides[3],
+    const void* k, const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
+    const uint8_t* mask, const int64_t mask_sizes[4], const int64_t mask_strides[4],
+    const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+    const int64_t bias_strides[4], const void* out, const int64_t o_strides[3], const float* lse,
+    const void* dout, const int64_t do_strides[3], void* dq, const int64_t dq_strides[3], void* dk,
+    const int64_t dk_strides[3], void* dv, const int64_t dv_strides[3], float* dbias,
+    void* workspace, size_t workspace_bytes, void* dbias_workspace, size_t dbias_workspace_bytes,
+    void* stream);
 
 /* ------------------------------------------------------------------------
  * Variable-length (packed) batches.

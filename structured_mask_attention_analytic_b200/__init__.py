@@ -22,6 +22,7 @@ from .ops import (  # noqa: F401
     mask_tile_summary,
     masked_attn_bwd,
     masked_attn_bwd_workspace_size,
+    masked_attn_bwd_dbias_workspace_size,
     masked_attn_fwd,
     masked_attn_fwd_workspace_size,
     round_up_k,

@@ -88,6 +88,16 @@ _SIGNATURES = {
                                 c_vp, c_i64p, c_vp, c_vp, c_i64p,
                                 c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
                                 c_vp, c_vp, c_size, c_vp]),
+    "masked_attn_bwd_dbias_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64p,
+                                                     c_sizep]),
+    "masked_attn_bwd_deterministic": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.c_float,
+                                              c_i32,
+                                              c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
+                                              c_vp, c_i64p, c_i64p,
+                                              c_vp, c_i32, c_i64p, c_i64p,
+                                              c_vp, c_i64p, c_vp, c_vp, c_i64p,
+                                              c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
+                                              c_vp, c_vp, c_size, c_vp, c_size, c_vp]),
     "varlen_attn_fwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_sizep]),
     "varlen_attn_fwd": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.c_float,
                                 c_i32, c_vp, c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,

@@ -570,11 +570,16 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           break;
         }
         tc_fence_after();
-        // dbias: this thread's query row of dS over the tile's 128 keys
+        // dbias: this thread's query row of dS over the tile's 128 keys (the
+        // fixed-order mode: the warp's row q / 32 of the partial buffer, if
+        // that group of 32 queries starts inside the query length)
         float* dbrow = nullptr;
-        if (POLICY != kPolicyDflash && p.db_mode != kDbiasNone)
-          dbrow = p.dbias + w.b * p.db_sb + (p.db_head_per_query ? h : w.hk) * p.db_sh +
-                  static_cast<int64_t>(row_valid ? q : 0) * p.db_sq + k0;
+        if (POLICY != kPolicyDflash && p.db_mode != kDbiasNone) {
+          const int64_t qrow = p.db_mode == kDbiasGroupStore ? (q >> 5) : (row_valid ? q : 0);
+          if (p.db_mode != kDbiasGroupStore || (q >> 5) * 32 < p.f.Lq)
+            dbrow = p.dbias + w.b * p.db_sb + (p.db_head_per_query ? h : w.hk) * p.db_sh +
+                    qrow * p.db_sq + k0;
+        }
         auto phase_b = [&](auto mode_tag) {
           constexpr int MODE = decltype(mode_tag)::value;
 #pragma unroll
@@ -622,7 +627,7 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
                   }
                 }
               }
-            } else if (MODE == kDbiasRowSum) {
+            } else if (MODE == kDbiasRowSum || MODE == kDbiasGroupStore) {
               // Column sums over the warp's 32 query rows (rows past Lq hold
               // 0): halving exchanges, after which lane l holds column l.
 #pragma unroll
@@ -635,7 +640,10 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
                   dsv[i] = keep + __shfl_xor_sync(0xffffffffu, send, wd);
                 }
               }
-              if (k0 + 32 * c + lane < p.db_kd) atomicAdd(dbrow + 32 * c + lane, dsv[0]);
+              if (k0 + 32 * c + lane < p.db_kd) {
+                if (MODE == kDbiasRowSum) atomicAdd(dbrow + 32 * c + lane, dsv[0]);
+                else if (dbrow != nullptr) dbrow[32 * c + lane] = dsv[0];
+              }
             }
           }
         };
@@ -645,6 +653,8 @@ attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           phase_b(std::integral_constant<int, kDbiasStore>{});
         else if (p.db_mode == kDbiasAdd)
           phase_b(std::integral_constant<int, kDbiasAdd>{});
+        else if (p.db_mode == kDbiasGroupStore)
+          phase_b(std::integral_constant<int, kDbiasGroupStore>{});
         else
           phase_b(std::integral_constant<int, kDbiasRowSum>{});
         fence_async_shared();
@@ -1317,6 +1327,9 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         if (POLICY != kPolicyDflash && p.db_mode != kDbiasNone)
           dbcol = p.dbias + w.b * p.db_sb + (p.db_head_per_query ? h : w.hk) * p.db_sh +
                   (db_key ? key : 0);
+        // the fixed-order mode stores the sum over the thread's 64 queries in
+        // row (q0 + qb) / 64 of the partial buffer, if those start inside Lq
+        const bool db_grp = q0 + qb < p.f.Lq;
         auto phase_b = [&](auto mode_tag) {
           constexpr int MODE = decltype(mode_tag)::value;
           float rsum = 0.f;
@@ -1341,7 +1354,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
               const float s0 = s01.x, s1 = s01.y, s2 = s23.x, s3 = s23.y;
               pk[e >> 1] = DT == SMA_BF16 ? pack_bf16x2(s0, s1) : pack_f16x2(s0, s1);
               pk[(e >> 1) + 1] = DT == SMA_BF16 ? pack_bf16x2(s2, s3) : pack_f16x2(s2, s3);
-              if (MODE == kDbiasRowSum) {
+              if (MODE == kDbiasRowSum || MODE == kDbiasGroupStore) {
                 rsum += (s0 + s1) + (s2 + s3);  // rows past Lq have P = 0, so dS = 0
               } else if (MODE != kDbiasNone) {
                 const float sv[4] = {s0, s1, s2, s3};
@@ -1361,6 +1374,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
                            pk[4 * v4 + 2], pk[4 * v4 + 3]);
           }
           if (MODE == kDbiasRowSum && db_key) atomicAdd(dbcol, rsum);
+          if (MODE == kDbiasGroupStore && db_key && db_grp) dbcol[((q0 + qb) >> 6) * p.db_sq] = rsum;
         };
         if (POLICY == kPolicyDflash || p.db_mode == kDbiasNone)
           phase_b(std::integral_constant<int, kDbiasNone>{});
@@ -1368,6 +1382,8 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           phase_b(std::integral_constant<int, kDbiasStore>{});
         else if (p.db_mode == kDbiasAdd)
           phase_b(std::integral_constant<int, kDbiasAdd>{});
+        else if (p.db_mode == kDbiasGroupStore)
+          phase_b(std::integral_constant<int, kDbiasGroupStore>{});
         else
           phase_b(std::integral_constant<int, kDbiasRowSum>{});
         fence_async_shared();
@@ -1681,6 +1697,41 @@ cudaError_t launch_transpose_lists(const BwdProblem& p, uint8_t* codes, cudaStre
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   transpose_lists_kernel<<<dim3(p.f.KT, static_cast<unsigned>(rows)), kTrThreads, 0, stream>>>(p, codes);
+  return cudaGetLastError();
+}
+
+// Fixed-order dbias (see kernels.h): one thread per output element, the
+// partial rows summed in increasing (b, h, r) order.
+__global__ void dbias_reduce_kernel(const float* __restrict__ part, int B, int H, int R,
+                                    float* __restrict__ out, int nb, int nh, int nq, int kd) {
+  const int64_t total = static_cast<int64_t>(nb) * nh * nq * kd;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= total) return;
+  const int k = static_cast<int>(t % kd);
+  int64_t rest = t / kd;
+  const int qo = static_cast<int>(rest % nq);
+  rest /= nq;
+  const int ho = static_cast<int>(rest % nh);
+  const int bo = static_cast<int>(rest / nh);
+  const int b0 = nb == 1 ? 0 : bo, b1 = nb == 1 ? B : bo + 1;
+  const int g = H / nh;
+  const int h0 = nh == 1 ? 0 : (nh == H ? ho : ho * g);
+  const int h1 = nh == 1 ? H : (nh == H ? ho + 1 : ho * g + g);
+  const int r0 = nq == 1 ? 0 : qo, r1 = nq == 1 ? R : qo + 1;
+  float acc = 0.f;
+  for (int b = b0; b < b1; ++b)
+    for (int h = h0; h < h1; ++h)
+      for (int r = r0; r < r1; ++r)
+        acc += part[((static_cast<int64_t>(b) * H + h) * R + r) * kd + k];
+  out[t] = acc;
+}
+
+cudaError_t launch_dbias_reduce(const float* part, int B, int H, int R, float* out, int nb, int nh,
+                                int nq, int kd, cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>(nb) * nh * nq * kd;
+  if (total == 0) return cudaSuccess;
+  dbias_reduce_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(
+      part, B, H, R, out, nb, nh, nq, kd);
   return cudaGetLastError();
 }
 

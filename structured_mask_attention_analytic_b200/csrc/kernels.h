@@ -197,8 +197,16 @@ __device__ __forceinline__ int64_t row_index(const AttnProblem& p, int b, int h,
 // How the backward writes dbias: not at all; one store per element (every
 // element of dS has its own dbias element); one atomic add per element
 // (several heads or batch rows share an element); one atomic add of each
-// thread's sum over its queries (dbias broadcast over the queries).
-enum DbiasMode { kDbiasNone = 0, kDbiasStore = 1, kDbiasAdd = 2, kDbiasRowSum = 3 };
+// thread's sum over its queries (dbias broadcast over the queries); or, for
+// the fixed-order (deterministic) dbias, one store of each thread's sum over
+// its group of kDbiasGroupRows queries into row q / kDbiasGroupRows of a
+// partial buffer (every partial element has exactly one writer).
+enum DbiasMode { kDbiasNone = 0, kDbiasStore = 1, kDbiasAdd = 2, kDbiasRowSum = 3,
+                 kDbiasGroupStore = 4 };
+// Query rows summed per partial row by the tensor-core backward kernels:
+// the transposed kernel (head dim 128) sums each thread's 64 queries, the
+// head-dim-64 kernel each warp's 32.
+constexpr int dbias_group_rows(int head_dim) { return head_dim == 128 ? 64 : 32; }
 
 // Single-query (decode) problem after the grouped-head swap: for each
 // (b, kv head) the `group` query heads are the rows.
@@ -303,6 +311,14 @@ cudaError_t launch_bwd_prep(const BwdProblem& p, cudaStream_t stream);
 cudaError_t launch_transpose_lists(const BwdProblem& p, uint8_t* codes, cudaStream_t stream);
 int launch_attn_bwd(const BwdProblem& p, cudaStream_t stream, char* msg, size_t msg_len);
 cudaError_t launch_dq_convert(const BwdProblem& p, cudaStream_t stream);
+// Fixed-order dbias: out[b', h', q', k] (the bias's broadcast shape, kd key
+// columns) = the sum, in increasing (b, h, r) order, of part[b][h][r][k]
+// ([B, H, R, kd]) over the batch rows, query heads and partial rows that
+// element (b', h', q') gathers: every b when nb == 1, else b'; every head
+// when nh == 1, heads [h' g, h' g + g) when nh is the KV head count and g =
+// H / nh > 1, else h'; every r when nq == 1, else r = q'.
+cudaError_t launch_dbias_reduce(const float* part, int B, int H, int R, float* out, int nb, int nh,
+                                int nq, int kd, cudaStream_t stream);
 // fp32 FFMA backward (dQ accumulator, dK, dV, dbias), after launch_bwd_prep
 // and launch_transpose_lists; launch_dq_convert follows.
 cudaError_t launch_attn_bwd_simt(const BwdProblem& p, cudaStream_t stream);

@@ -1028,19 +1028,59 @@ sma_status masked_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t 
   return ok();
 }
 
-sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
-                           int32_t q_len, int32_t k_len, int32_t head_dim, float scale,
-                           int32_t is_causal, const void* q, const int64_t q_strides[3],
-                           const void* k, const int64_t k_strides[3], const void* v,
-                           const int64_t v_strides[3], const uint8_t* mask,
-                           const int64_t mask_sizes[4], const int64_t mask_strides[4],
-                           const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
-                           const int64_t bias_strides[4], const void* out,
-                           const int64_t o_strides[3], const float* lse, const void* dout,
-                           const int64_t do_strides[3], void* dq, const int64_t dq_strides[3],
-                           void* dk, const int64_t dk_strides[3], void* dv,
-                           const int64_t dv_strides[3], float* dbias, void* workspace,
-                           size_t workspace_bytes, void* stream) {
+// Partial buffer of the fixed-order dbias: [batch, heads, R, kd] fp32, R the
+// partial rows per (batch, head): the query rows (a bias with a query dim, or
+// the fp32 kernels, which store per element), else one row per group of
+// dbias_group_rows(head_dim) queries.  0 bytes where every dbias element
+// already has a single writer (a bias with its own element for each
+// (batch, head, query)).
+struct DetDbias {
+  int R = 0;
+  size_t bytes = 0;
+};
+static DetDbias det_dbias_layout(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                                 int32_t q_len, int32_t head_dim, const int64_t bias_sizes[4]) {
+  DetDbias d;
+  const int64_t nb = bias_sizes[0], nh = bias_sizes[1], nq = bias_sizes[2], kd = bias_sizes[3];
+  const int group = heads / kv_heads;
+  const bool own_head = heads == 1 || (nh > 1 && (nh == heads || group == 1));
+  const bool own_batch = batch == 1 || nb > 1;
+  if (nq > 1 && own_head && own_batch) return d;
+  const int G = dbias_group_rows(head_dim);
+  d.R = (nq > 1 || dtype == SMA_FP32) ? q_len : static_cast<int>(ceil_div(q_len, G));
+  d.bytes = static_cast<size_t>(batch) * heads * d.R * kd * 4;
+  return d;
+}
+
+sma_status masked_attn_bwd_dbias_workspace_size(int32_t dtype, int32_t batch, int32_t heads,
+                                                int32_t kv_heads, int32_t q_len, int32_t head_dim,
+                                                const int64_t bias_sizes[4], size_t* bytes) {
+  if (bytes == nullptr || bias_sizes == nullptr)
+    return fail(SMA_ERR_INVALID_ARG, "bias_sizes / bytes is NULL");
+  if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  sma_status s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (batch < 1 || q_len < 1) return fail(SMA_ERR_INVALID_ARG, "batch and q_len must be >= 1");
+  for (int i = 0; i < 4; ++i)
+    if (bias_sizes[i] < 1) return fail(SMA_ERR_INVALID_ARG, "bias sizes must be >= 1");
+  *bytes = det_dbias_layout(dtype, batch, heads, kv_heads, q_len, head_dim, bias_sizes).bytes;
+  return ok();
+}
+
+static sma_status masked_bwd_impl(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                                  int32_t q_len, int32_t k_len, int32_t head_dim, float scale,
+                                  int32_t is_causal, const void* q, const int64_t q_strides[3],
+                                  const void* k, const int64_t k_strides[3], const void* v,
+                                  const int64_t v_strides[3], const uint8_t* mask,
+                                  const int64_t mask_sizes[4], const int64_t mask_strides[4],
+                                  const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+                                  const int64_t bias_strides[4], const void* out,
+                                  const int64_t o_strides[3], const float* lse, const void* dout,
+                                  const int64_t do_strides[3], void* dq, const int64_t dq_strides[3],
+                                  void* dk, const int64_t dk_strides[3], void* dv,
+                                  const int64_t dv_strides[3], float* dbias, void* workspace,
+                                  size_t workspace_bytes, bool deterministic, void* det_ws,
+                                  size_t det_bytes, void* stream) {
   if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   sma_status s = check_heads(heads, kv_heads, head_dim);
   if (s != SMA_OK) return s;
@@ -1076,6 +1116,13 @@ sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   const BwdLayout lay = bwd_layout(mg.codes_bytes, static_cast<int64_t>(mg.LB) * mg.LH, QT, KT,
                                    batch, heads, q_len, head_dim);
   if ((s = check_workspace(workspace, workspace_bytes, lay.total)) != SMA_OK) return s;
+  // fixed-order dbias partials (0 bytes: not used; a bias with a key dim of
+  // 1 has the zero gradient, written without them)
+  DetDbias det;
+  if (deterministic && dbias != nullptr && bias != nullptr && (bias_sizes[3] > 1 || k_len == 1)) {
+    det = det_dbias_layout(dtype, batch, heads, kv_heads, q_len, head_dim, bias_sizes);
+    if ((s = check_workspace(det_ws, det_bytes, det.bytes)) != SMA_OK) return s;
+  }
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
@@ -1139,6 +1186,18 @@ sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
       const bool own_head = heads == 1 || (nh > 1 && (db_hpq || p.group == 1));
       const bool own_batch = batch == 1 || nb > 1;
       b.db_mode = nq == 1 ? kDbiasRowSum : (own_head && own_batch ? kDbiasStore : kDbiasAdd);
+      if (det.bytes > 0) {
+        // every partial element has one writer; the reduce kernel then sums
+        // the partials in a fixed order
+        e = cudaMemsetAsync(det_ws, 0, det.bytes, st);
+        if (e != cudaSuccess) return cuda_fail(e, "dbias partial zeroing failed");
+        b.dbias = static_cast<float*>(det_ws);
+        b.db_sq = kd;
+        b.db_sh = static_cast<int64_t>(det.R) * kd;
+        b.db_sb = static_cast<int64_t>(heads) * det.R * kd;
+        b.db_head_per_query = 1;
+        b.db_mode = nq == 1 && dtype != SMA_FP32 ? kDbiasGroupStore : kDbiasStore;
+      }
     }
     // else: a bias with one value for every key adds the same amount to every
     // score of a row, which softmax ignores; its gradient, the sum of dS over
@@ -1146,7 +1205,51 @@ sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
     // dbias is the result.
   }
   if ((s = run_backward(b, workspace, lay, st)) != SMA_OK) return s;
+  if (det.bytes > 0) {
+    e = launch_dbias_reduce(static_cast<const float*>(det_ws), batch, heads, det.R, dbias,
+                            static_cast<int>(bias_sizes[0]), static_cast<int>(bias_sizes[1]),
+                            static_cast<int>(bias_sizes[2]), static_cast<int>(bias_sizes[3]), st);
+    if (e != cudaSuccess) return cuda_fail(e, "dbias reduction launch failed");
+  }
   return ok();
+}
+
+sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t q_len, int32_t k_len, int32_t head_dim, float scale,
+                           int32_t is_causal, const void* q, const int64_t q_strides[3],
+                           const void* k, const int64_t k_strides[3], const void* v,
+                           const int64_t v_strides[3], const uint8_t* mask,
+                           const int64_t mask_sizes[4], const int64_t mask_strides[4],
+                           const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+                           const int64_t bias_strides[4], const void* out,
+                           const int64_t o_strides[3], const float* lse, const void* dout,
+                           const int64_t do_strides[3], void* dq, const int64_t dq_strides[3],
+                           void* dk, const int64_t dk_strides[3], void* dv,
+                           const int64_t dv_strides[3], float* dbias, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  return masked_bwd_impl(dtype, batch, heads, kv_heads, q_len, k_len, head_dim, scale, is_causal, q,
+                         q_strides, k, k_strides, v, v_strides, mask, mask_sizes, mask_strides, bias,
+                         bias_dtype, bias_sizes, bias_strides, out, o_strides, lse, dout, do_strides,
+                         dq, dq_strides, dk, dk_strides, dv, dv_strides, dbias, workspace,
+                         workspace_bytes, false, nullptr, 0, stream);
+}
+
+sma_status masked_attn_bwd_deterministic(
+    int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads, int32_t q_len, int32_t k_len,
+    int32_t head_dim, float scale, int32_t is_causal, const void* q, const int64_t q_strides[3],
+    const void* k, const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
+    const uint8_t* mask, const int64_t mask_sizes[4], const int64_t mask_strides[4],
+    const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+    const int64_t bias_strides[4], const void* out, const int64_t o_strides[3], const float* lse,
+    const void* dout, const int64_t do_strides[3], void* dq, const int64_t dq_strides[3], void* dk,
+    const int64_t dk_strides[3], void* dv, const int64_t dv_strides[3], float* dbias,
+    void* workspace, size_t workspace_bytes, void* dbias_workspace, size_t dbias_workspace_bytes,
+    void* stream) {
+  return masked_bwd_impl(dtype, batch, heads, kv_heads, q_len, k_len, head_dim, scale, is_causal, q,
+                         q_strides, k, k_strides, v, v_strides, mask, mask_sizes, mask_strides, bias,
+                         bias_dtype, bias_sizes, bias_strides, out, o_strides, lse, dout, do_strides,
+                         dq, dq_strides, dk, dk_strides, dv, dv_strides, dbias, workspace,
+                         workspace_bytes, true, dbias_workspace, dbias_workspace_bytes, stream);
 }
 
 sma_status varlen_attn_fwd_workspace_size(int32_t batch, int32_t max_q, int32_t max_k, size_t* bytes) {

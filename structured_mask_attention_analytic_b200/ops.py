@@ -314,13 +314,24 @@ def masked_attn_bwd_workspace_size(batch, heads, kv_heads, q_len, k_len, head_di
     return n.value
 
 
+def masked_attn_bwd_dbias_workspace_size(dtype, batch, heads, kv_heads, q_len, head_dim, bias_shape) -> int:
+    n = ctypes.c_size_t()
+    nat.check(_lib().masked_attn_bwd_dbias_workspace_size(
+        _DTYPE[dtype], batch, heads, kv_heads, q_len, head_dim, nat.i64_array(bias_shape), ctypes.byref(n)))
+    return n.value
+
+
 def masked_attn_bwd(q, k, v, out, lse, dout, mask=None, bias=None, is_causal: bool = False, scale=None,
-                    dq=None, dk=None, dv=None, workspace=None, return_dbias: bool = False, dbias=None):
+                    dq=None, dk=None, dv=None, workspace=None, return_dbias: bool = False, dbias=None,
+                    deterministic: bool = False, dbias_workspace=None):
     """Gradients of ``masked_attn_fwd`` (same mask / bias / causal / scale):
     ``out`` and ``lse`` are that call's results, ``dout`` the upstream
     gradient.  Returns ``(dq, dk, dv)``, or ``(dq, dk, dv, dbias)`` with
     ``return_dbias`` (or a ``dbias`` buffer): float32 at the bias's shape,
-    reduced over the dims the bias broadcasts along (a key dim of 1 too)."""
+    reduced over the dims the bias broadcasts along (a key dim of 1 too).
+    ``deterministic``: dbias through ``masked_attn_bwd_deterministic`` (the
+    same bits on every call), with a partial-sum buffer of
+    ``masked_attn_bwd_dbias_workspace_size`` bytes (allocated if not given)."""
     _require_cuda(q, k, v, out, lse, dout, mask, bias)
     b, lq, h, dh = q.shape
     lk, kvh = k.shape[1], k.shape[2]
@@ -341,15 +352,22 @@ def masked_attn_bwd(q, k, v, out, lse, dout, mask=None, bias=None, is_causal: bo
             dbias = torch.empty(tuple(bias.shape), dtype=torch.float32, device=q.device)
         elif dbias.dtype != torch.float32 or tuple(dbias.shape) != tuple(bias.shape) or not dbias.is_contiguous():
             raise ValueError("dbias must be contiguous float32 with the bias's shape")
-    nat.check(_lib().masked_attn_bwd(
-        _dtype_code(q), b, h, kvh, lq, lk, dh, ctypes.c_float(0.0 if scale is None else float(scale)),
-        1 if is_causal else 0,
-        _ptr(q), _strides3(q), _ptr(k), _strides3(k), _ptr(v), _strides3(v),
-        mp, msz, mst,
-        bp, _dtype_code(bias) if bias is not None else 0, bsz, bst,
-        _ptr(out), _strides3(out), _ptr(lse), _ptr(dout), _strides3(dout),
-        _ptr(dq), _strides3(dq), _ptr(dk), _strides3(dk), _ptr(dv), _strides3(dv),
-        _ptr(dbias) if want_db else ctypes.c_void_p(0), _ptr(workspace), workspace.numel(), _stream(q)))
+    args = (_dtype_code(q), b, h, kvh, lq, lk, dh, ctypes.c_float(0.0 if scale is None else float(scale)),
+            1 if is_causal else 0,
+            _ptr(q), _strides3(q), _ptr(k), _strides3(k), _ptr(v), _strides3(v),
+            mp, msz, mst,
+            bp, _dtype_code(bias) if bias is not None else 0, bsz, bst,
+            _ptr(out), _strides3(out), _ptr(lse), _ptr(dout), _strides3(dout),
+            _ptr(dq), _strides3(dq), _ptr(dk), _strides3(dk), _ptr(dv), _strides3(dv),
+            _ptr(dbias) if want_db else ctypes.c_void_p(0), _ptr(workspace), workspace.numel())
+    if deterministic and want_db:
+        db_bytes = masked_attn_bwd_dbias_workspace_size(q.dtype, b, h, kvh, lq, dh, list(bias.shape))
+        if dbias_workspace is None:
+            dbias_workspace = torch.empty(max(db_bytes, 1), dtype=torch.uint8, device=q.device)
+        nat.check(_lib().masked_attn_bwd_deterministic(*args, _ptr(dbias_workspace), dbias_workspace.numel(),
+                                                       _stream(q)))
+    else:
+        nat.check(_lib().masked_attn_bwd(*args, _stream(q)))
     return (dq, dk, dv, dbias) if want_db else (dq, dk, dv)
 
 
