@@ -156,10 +156,25 @@ def attention(q, k, v, *, keep=None, keep_rows=None, bias=None, scale=None,
     return out, lse
 
 
-def varlen_attention(q, k, v, cu_q, cu_k, causal: bool = False, scale=None):
+def varlen_seq_aux(aux, b: int, lq: int, lk: int, n_heads: int, n_kv_heads: int):
+    """Sequence b's part of a mask / bias given in the padded per-sequence
+    layout ``(b', h', q', K)`` (reading R33 of the packed path): batch row b
+    (or the only one), query rows ``[0, lq)`` (or the only one) and key
+    columns ``[0, lk)``, as an array broadcasting against ``[1, H, lq, lk]``."""
+    a = np.asarray(aux)
+    a = a[b:b + 1] if a.shape[0] > 1 else a
+    a = a[:, :, :lq] if a.shape[2] > 1 else a
+    if a.shape[-1] > 1:
+        a = a[..., :lk]
+    return aux_view(a, n_heads, n_kv_heads, lk)
+
+
+def varlen_attention(q, k, v, cu_q, cu_k, causal: bool = False, scale=None, mask=None, bias=None):
     """Packed variable-length sequences: sequence b is rows ``cu_q[b]:cu_q[b+1]``
     of q (``[total_q, H, d]``) and ``cu_k[b]:cu_k[b+1]`` of k / v and attends
-    only its own keys, bottom-right causal within the sequence when ``causal``.
+    only its own keys, bottom-right causal within the sequence when ``causal``,
+    and, when given, the keys its part of ``mask`` keeps, with its part of
+    ``bias`` added (both in the padded per-sequence layout, ``varlen_seq_aux``).
 
     The packed form behind flash-sparse-attention PR #197's varlen function
     and pad / unpad helpers (Changes list); each sequence is the dense
@@ -168,14 +183,20 @@ def varlen_attention(q, k, v, cu_q, cu_k, causal: bool = False, scale=None):
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
+    n_heads, n_kv = q.shape[1], k.shape[1]
     out = np.zeros(q.shape)
     lse = np.full((q.shape[1], q.shape[0]), -np.inf)
     for b in range(len(cu_q) - 1):
         q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
         if q1 == q0 or k1 == k0:
             continue
-        keep = causal_keep(q1 - q0, k1 - k0)[None, None] if causal else None
-        o, l = attention(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], keep=keep, scale=scale)
+        lq, lk = q1 - q0, k1 - k0
+        keep = causal_keep(lq, lk)[None, None] if causal else None
+        if mask is not None:
+            m = varlen_seq_aux(mask, b, lq, lk, n_heads, n_kv).astype(bool)
+            keep = m if keep is None else (keep & m)
+        bb = varlen_seq_aux(bias, b, lq, lk, n_heads, n_kv).astype(np.float64) if bias is not None else None
+        o, l = attention(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], keep=keep, bias=bb, scale=scale)
         out[q0:q1] = o[0]
         lse[:, q0:q1] = l[0]
     return out, lse

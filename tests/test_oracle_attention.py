@@ -252,6 +252,50 @@ def test_varlen_equals_block_diagonal_mask(causal):
     np.testing.assert_allclose(lse[fin], ref_lse[0][fin], atol=1e-13)
 
 
+@pytest.mark.parametrize("mshape,bshape", [((5, 1, 1, 8), (1, 4, 5, 8)), ((1, 2, 5, 8), (5, 2, 1, 1)),
+                                           ((5, 4, 5, 8), None), (None, (1, 1, 5, 6))], ids=str)
+def test_varlen_mask_bias_equal_the_block_diagonal_problem(mshape, bshape):
+    """A packed batch with a mask / bias in the padded per-sequence layout
+    equals one problem over the packed rows whose keep mask is block-diagonal
+    and, inside block b, sequence b's mask rows / columns [0, len) (bias
+    likewise), for batch-, head- (H or KVH) and query-broadcast shapes and a
+    key dim that is padded, exact or 1."""
+    rng = np.random.default_rng(22)
+    lq, lk = [3, 0, 5, 1, 4], [4, 2, 5, 0, 2]
+    cu_q, cu_k = np.cumsum([0] + lq), np.cumsum([0] + lk)
+    H, KVH, D = 4, 2, 3
+    q = rng.standard_normal((cu_q[-1], H, D))
+    k = rng.standard_normal((cu_k[-1], KVH, D))
+    v = rng.standard_normal((cu_k[-1], KVH, D))
+    mask = rng.random(mshape) < 0.7 if mshape else None
+    bias = rng.standard_normal(bshape) if bshape else None
+    out, lse = at.varlen_attention(q, k, v, cu_q, cu_k, True, mask=mask, bias=bias)
+    tq, tk = cu_q[-1], cu_k[-1]
+    keep = np.zeros((H, tq, tk), bool)
+    dense_bias = np.zeros((H, tq, tk))
+    for b in range(len(lq)):
+        for h in range(H):
+            for i in range(lq[b]):
+                for j in range(lk[b]):
+                    ok = j <= i + lk[b] - lq[b]          # bottom-right causal
+                    if mask is not None:
+                        mb = mask[b if mask.shape[0] > 1 else 0]
+                        mh = mb[h if mask.shape[1] == H else (h // (H // KVH) if mask.shape[1] > 1 else 0)]
+                        mr = mh[i if mask.shape[2] > 1 else 0]
+                        ok = ok and bool(mr[j if mask.shape[3] > 1 else 0])
+                    keep[h, cu_q[b] + i, cu_k[b] + j] = ok
+                    if bias is not None:
+                        bb = bias[b if bias.shape[0] > 1 else 0]
+                        bh = bb[h if bias.shape[1] == H else (h // (H // KVH) if bias.shape[1] > 1 else 0)]
+                        br = bh[i if bias.shape[2] > 1 else 0]
+                        dense_bias[h, cu_q[b] + i, cu_k[b] + j] = br[j if bias.shape[3] > 1 else 0]
+    ref, ref_lse = at.attention(q[None], k[None], v[None], keep=keep[None], bias=dense_bias[None])
+    np.testing.assert_allclose(out, ref[0], atol=1e-12)
+    np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(ref_lse[0]))
+    fin = ~np.isneginf(lse)
+    np.testing.assert_allclose(lse[fin], ref_lse[0][fin], atol=1e-12)
+
+
 def test_key_dim_forms_of_mask_and_bias(qkv):
     """The three key dims of PR #190's interface (padded to a multiple of 128
     there; padded, Lk, or 1 which the interface expands).  A mask/bias of key
