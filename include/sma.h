@@ -437,7 +437,8 @@ sma_status masked_attn_bwd_deterministic(
  * cu_seqlens_q[b+1]) of the packed queries and [cu_seqlens_k[b],
  * cu_seqlens_k[b+1]) of the packed keys (int32 [batch + 1], ascending, on the
  * device); it attends only its own keys, bottom-right causal per sequence
- * when is_causal (key k kept iff k <= q + len_k - len_q).  No mask or bias.
+ * when is_causal (key k kept iff k <= q + len_k - len_q).  No mask or bias
+ * here (varlen_masked_attn_fwd below takes them).
  *
  * q, out   [total_q, heads, d]; k, v [total_k, kv_heads, d]; strides[2] =
  *          {row, head} in elements, d contiguous, 16-byte multiples.
@@ -486,6 +487,48 @@ sma_status varlen_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
                            void* dq, const int64_t dq_strides[2], void* dk,
                            const int64_t dk_strides[2], void* dv, const int64_t dv_strides[2],
                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Packed batches with a mask and / or bias (reading R33: PR #197's varlen
+ * function sits next to the mask creation it centralises, so a packed batch
+ * takes the same mask / bias as the padded call).  They come in the padded
+ * per-sequence layout of masked_attn_fwd for the problem [batch, max_q,
+ * heads, max_k]: sizes (B|1, H|KVH|1, max_q|1, round_up(max_k, 128)|max_k|1),
+ * element (b, h, q, k) for query q and key k of sequence b (both
+ * sequence-local), any of mask / bias NULL.  Everything else, including the
+ * causal rule, as varlen_attn_fwd / varlen_attn_bwd; dbias (nullable) as in
+ * masked_attn_bwd, at the bias's sizes with sequence-local rows and columns.
+ * The workspaces also hold the mask's tile codes: query them with the mask's
+ * sizes (NULL: none). */
+sma_status varlen_masked_attn_fwd_workspace_size(int32_t batch, int32_t heads, int32_t kv_heads,
+                                                 int32_t max_q, int32_t max_k, int32_t head_dim,
+                                                 const int64_t mask_sizes[4], size_t* bytes);
+
+sma_status varlen_masked_attn_fwd(
+    int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads, int32_t head_dim, int32_t total_q,
+    int32_t total_k, int32_t max_q, int32_t max_k, float scale, int32_t is_causal,
+    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const void* q,
+    const int64_t q_strides[2], const void* k, const int64_t k_strides[2], const void* v,
+    const int64_t v_strides[2], const uint8_t* mask, const int64_t mask_sizes[4],
+    const int64_t mask_strides[4], const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+    const int64_t bias_strides[4], void* out, const int64_t o_strides[2], float* lse,
+    void* workspace, size_t workspace_bytes, void* stream);
+
+sma_status varlen_masked_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t kv_heads,
+                                                 int32_t total_q, int32_t max_q, int32_t max_k,
+                                                 int32_t head_dim, const int64_t mask_sizes[4],
+                                                 size_t* bytes);
+
+sma_status varlen_masked_attn_bwd(
+    int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads, int32_t head_dim, int32_t total_q,
+    int32_t total_k, int32_t max_q, int32_t max_k, float scale, int32_t is_causal,
+    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const void* q,
+    const int64_t q_strides[2], const void* k, const int64_t k_strides[2], const void* v,
+    const int64_t v_strides[2], const uint8_t* mask, const int64_t mask_sizes[4],
+    const int64_t mask_strides[4], const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+    const int64_t bias_strides[4], const void* out, const int64_t o_strides[2], const float* lse,
+    const void* dout, const int64_t do_strides[2], void* dq, const int64_t dq_strides[2], void* dk,
+    const int64_t dk_strides[2], void* dv, const int64_t dv_strides[2], float* dbias,
+    void* workspace, size_t workspace_bytes, void* stream);
 
 /* pad: padded [batch, max_len, heads, d] (strides[3] = batch, row, head) from
  * packed rows, zero past each sequence's length; unpad: the reverse (rows

@@ -107,6 +107,19 @@ _SIGNATURES = {
                                 c_i32, c_vp, c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
                                 c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
                                 c_vp, c_size, c_vp]),
+    "varlen_masked_attn_fwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64p,
+                                                      c_sizep]),
+    "varlen_masked_attn_fwd": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
+                                       ctypes.c_float, c_i32, c_vp, c_vp, c_vp, c_i64p, c_vp, c_i64p,
+                                       c_vp, c_i64p, c_vp, c_i64p, c_i64p, c_vp, c_i32, c_i64p, c_i64p,
+                                       c_vp, c_i64p, c_vp, c_vp, c_size, c_vp]),
+    "varlen_masked_attn_bwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
+                                                      c_i64p, c_sizep]),
+    "varlen_masked_attn_bwd": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
+                                       ctypes.c_float, c_i32, c_vp, c_vp, c_vp, c_i64p, c_vp, c_i64p,
+                                       c_vp, c_i64p, c_vp, c_i64p, c_i64p, c_vp, c_i32, c_i64p, c_i64p,
+                                       c_vp, c_i64p, c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp, c_i64p,
+                                       c_vp, c_i64p, c_vp, c_vp, c_size, c_vp]),
     "varlen_pad": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp]),
     "varlen_unpad": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64p, c_vp, c_i64p, c_vp]),
     "sparse_attn_fwd_workspace_size": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64p,

@@ -37,9 +37,10 @@
 //               keep, additive bias, stride-0 broadcast dims), plus
 //               bottom-right causal masking; the bias is added on every kept
 //               tile, the mask read on PARTIAL tiles only.
-//   Varlen   -- packed sequences: the explicit policy without mask or bias,
-//               each unit's rows offset to its sequence and bounded by its
-//               lengths (bottom-right causal per sequence).
+//   Varlen   -- packed sequences: the explicit policy with each unit's rows
+//               offset to its sequence and bounded by its lengths
+//               (bottom-right causal per sequence); a mask / bias is read in
+//               the padded per-sequence layout at sequence-local (q, k).
 //   Gather   -- the explicit policy over keys compacted by a query-broadcast
 //               mask (PR #197 top-k masks): K/V/bias are the compacted
 //               operands and each row's causal bound is a limit on the
@@ -613,7 +614,10 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
       const float bias_mul = kLog2e / p.scale_log2;
       // With compacted keys every PARTIAL tile is cut by the row limit.
       const int causal_off = POLICY == kPolicyGather ? -(1 << 30) : w.lk - w.lq;
-      const bool mask_bcast_q = POLICY == kPolicyExplicit && p.has_mask && p.mask.sq == 0;
+      // explicit masks: the padded policy, and packed sequences (their mask in
+      // the padded per-sequence layout, rows and columns sequence-local)
+      constexpr bool kMasks = POLICY == kPolicyExplicit || POLICY == kPolicyVarlen;
+      const bool mask_bcast_q = kMasks && p.has_mask && p.mask.sq == 0;
       // Mask / bias rows hold kd columns: round_up(Lk, 128), Lk, or 1.  Vector
       // loads start at most at the row's last aligned chunk (a 16-byte block
       // that holds column kd - 1), so none leaves the row's memory; columns
@@ -701,7 +705,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
             if (k0 + kTile > w.lk) lim = min(lim, w.lk - k0);
             if (p.causal && k0 + kTile - 1 > qfirst + causal_off)
               lim = min(lim, causal_lim - k0 + 1);
-            if (POLICY == kPolicyExplicit && mask_row1) {
+            if (kMasks && mask_row1) {
 #pragma unroll
               for (int c = 0; c < kTile; ++c) x[c] = (row_keep1 && c < lim) ? x[c] : -INFINITY;
             } else if (mask_bcast_q) {
@@ -717,7 +721,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
                 const bool keep = ((bits[c & 3] >> (c >> 2)) & 1u) != 0u && c < lim;
                 x[c] = keep ? x[c] : -INFINITY;
               }
-            } else if (POLICY == kPolicyExplicit && p.has_mask) {
+            } else if (kMasks && p.has_mask) {
 #pragma unroll
               for (int c = 0; c < kTile; c += 16) {
                 const uint4 mv = *reinterpret_cast<const uint4*>(mrow + min(k0 + c, mask_vlast16));

@@ -1252,6 +1252,60 @@ sma_status masked_attn_bwd_deterministic(
                          workspace_bytes, true, dbias_workspace, dbias_workspace_bytes, stream);
 }
 
+// Mask / bias of a packed batch, in the padded per-sequence layout
+// (b', h', q', kd) as masked_attn_fwd takes them for a [batch, max_q, ...,
+// max_k] problem; rows and columns are sequence-local.  All NULL: none.
+struct VarlenAux {
+  const uint8_t* mask = nullptr;
+  const int64_t* mask_sizes = nullptr;
+  const int64_t* mask_strides = nullptr;
+  const void* bias = nullptr;
+  int32_t bias_dtype = 0;
+  const int64_t* bias_sizes = nullptr;
+  const int64_t* bias_strides = nullptr;
+  float* dbias = nullptr;  // backward only
+};
+
+// List geometry of a packed batch: one list row per (sequence, list head,
+// query tile); with a mask the list heads follow the mask's head dim as in
+// masked_attn_fwd, and the tile codes of the mask lead the workspace.
+struct VarlenLists {
+  int LH = 1, head_mode = 0, codes_qt = 0;
+  size_t codes_bytes = 0;
+};
+static VarlenLists varlen_lists_geom(int32_t batch, int32_t heads, int32_t kv_heads, int32_t max_q,
+                                     int32_t max_k, int32_t head_dim, const int64_t* mask_sizes) {
+  VarlenLists v;
+  if (mask_sizes == nullptr) return v;
+  const MaskedGeom mg = masked_geom(batch, heads, kv_heads, max_q < 2 ? 2 : max_q, max_k, head_dim,
+                                    mask_sizes);
+  v.LH = mg.LH;
+  v.head_mode = mg.head_mode;
+  v.codes_qt = mg.codes_qt;
+  v.codes_bytes = mg.codes_bytes;
+  return v;
+}
+
+// Validates the mask / bias of a packed batch against the padded
+// per-sequence problem [batch, max_q, heads, max_k].
+static sma_status check_varlen_aux(const VarlenAux& ax, int32_t batch, int32_t heads,
+                                   int32_t kv_heads, int32_t max_q, int32_t max_k, AuxView* mview,
+                                   AuxView* bview) {
+  sma_status s;
+  if (ax.mask != nullptr &&
+      (s = check_aux("mask", ax.mask, ax.mask_sizes, ax.mask_strides, 1, batch, heads, kv_heads,
+                     max_q, max_k, true, mview)) != SMA_OK)
+    return s;
+  if (ax.bias != nullptr) {
+    if (!valid_dtype(ax.bias_dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown bias dtype %d", ax.bias_dtype);
+    if ((s = check_aux("bias", ax.bias, ax.bias_sizes, ax.bias_strides, elem_size(ax.bias_dtype),
+                       batch, heads, kv_heads, max_q, max_k, true, bview)) != SMA_OK)
+      return s;
+    bview->dtype = ax.bias_dtype;
+  }
+  return SMA_OK;
+}
+
 sma_status varlen_attn_fwd_workspace_size(int32_t batch, int32_t max_q, int32_t max_k, size_t* bytes) {
   if (bytes == nullptr) return fail(SMA_ERR_INVALID_ARG, "bytes is NULL");
   if (batch < 1 || max_q < 1 || max_k < 1)
@@ -1261,13 +1315,36 @@ sma_status varlen_attn_fwd_workspace_size(int32_t batch, int32_t max_q, int32_t 
   return ok();
 }
 
-sma_status varlen_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
-                           int32_t head_dim, int32_t total_q, int32_t total_k, int32_t max_q,
-                           int32_t max_k, float scale, int32_t is_causal, const int32_t* cu_seqlens_q,
-                           const int32_t* cu_seqlens_k, const void* q, const int64_t q_strides[2],
-                           const void* k, const int64_t k_strides[2], const void* v,
-                           const int64_t v_strides[2], void* out, const int64_t o_strides[2],
-                           float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+// Tile lists of a packed batch: causal / length geometry per sequence, and
+// with a mask its tile codes (summarised first into the workspace's head).
+static cudaError_t launch_varlen_aux_lists(const AttnProblem& p, const VarlenAux& ax,
+                                           const AuxView& mview, const VarlenLists& vl,
+                                           void* workspace, const ListsLayout& lay,
+                                           cudaStream_t st) {
+  int32_t* nf = at<int32_t>(workspace, lay.nf);
+  int32_t* np = at<int32_t>(workspace, lay.np);
+  int32_t* fi = at<int32_t>(workspace, lay.fi);
+  int32_t* pi = at<int32_t>(workspace, lay.pi);
+  if (ax.mask == nullptr && ax.bias == nullptr) return launch_varlen_lists(p, nf, fi, np, pi, st);
+  uint8_t* codes = nullptr;
+  if (ax.mask != nullptr) {
+    codes = at<uint8_t>(workspace, 0);
+    const int64_t folded[4] = {mview.sb, mview.sh, mview.sq, 1};
+    const cudaError_t e = launch_mask_tile_summary(ax.mask, ax.mask_sizes, folded, p.Lk, codes, st);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_explicit_lists(p, codes, vl.codes_qt, nf, fi, np, pi, st);
+}
+
+static sma_status varlen_fwd_impl(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                                  int32_t head_dim, int32_t total_q, int32_t total_k, int32_t max_q,
+                                  int32_t max_k, float scale, int32_t is_causal,
+                                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                  const void* q, const int64_t q_strides[2], const void* k,
+                                  const int64_t k_strides[2], const void* v,
+                                  const int64_t v_strides[2], void* out, const int64_t o_strides[2],
+                                  float* lse, void* workspace, size_t workspace_bytes,
+                                  const VarlenAux& ax, void* stream) {
   if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   sma_status s = check_heads(heads, kv_heads, head_dim);
   if (s != SMA_OK) return s;
@@ -1286,9 +1363,16 @@ sma_status varlen_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   if ((s = check_operand("k", k, ks, dtype, total_k)) != SMA_OK) return s;
   if ((s = check_operand("v", v, vs, dtype, total_k)) != SMA_OK) return s;
   if ((s = check_operand("out", out, os, dtype, total_q)) != SMA_OK) return s;
-  size_t need = 0;
-  if ((s = varlen_attn_fwd_workspace_size(batch, max_q, max_k, &need)) != SMA_OK) return s;
-  if ((s = check_workspace(workspace, workspace_bytes, need)) != SMA_OK) return s;
+  AuxView mview, bview;
+  if ((s = check_varlen_aux(ax, batch, heads, kv_heads, max_q, max_k, &mview, &bview)) != SMA_OK)
+    return s;
+  const bool has_mask = ax.mask != nullptr, has_bias = ax.bias != nullptr;
+  const VarlenLists vl = varlen_lists_geom(batch, heads, kv_heads, max_q, max_k, head_dim,
+                                           has_mask ? ax.mask_sizes : nullptr);
+  const ListsLayout lay = lists_layout(vl.codes_bytes,
+                                       static_cast<int64_t>(batch) * vl.LH * ceil_div(max_q, kTile),
+                                       static_cast<int>(ceil_div(max_k, kTile)));
+  if ((s = check_workspace(workspace, workspace_bytes, lay.end)) != SMA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   int* err = device_error_word(&e);
@@ -1313,15 +1397,17 @@ sma_status varlen_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   p.total_q = total_q;
   p.total_k = total_k;
   p.err = err;
-  const ListsLayout lay = lists_layout(0, static_cast<int64_t>(batch) * p.QT, p.KT);
-  p.lists.LB = batch; p.lists.LH = 1; p.lists.head_mode = 0;
+  p.has_mask = has_mask;
+  p.has_bias = has_bias;
+  if (has_mask) p.mask = mview;
+  if (has_bias) p.bias = bview;
+  p.lists.LB = batch; p.lists.LH = vl.LH; p.lists.head_mode = vl.head_mode;
   p.lists.num_full = at<int32_t>(workspace, lay.nf);
   p.lists.num_part = at<int32_t>(workspace, lay.np);
   p.lists.full_idx = at<int32_t>(workspace, lay.fi);
   p.lists.part_idx = at<int32_t>(workspace, lay.pi);
-  e = launch_varlen_lists(p, at<int32_t>(workspace, lay.nf), at<int32_t>(workspace, lay.fi),
-                          at<int32_t>(workspace, lay.np), at<int32_t>(workspace, lay.pi), st);
-  if (e != cudaSuccess) return cuda_fail(e, "tile list launch failed");
+  if ((e = launch_varlen_aux_lists(p, ax, mview, vl, workspace, lay, st)) != cudaSuccess)
+    return cuda_fail(e, "tile list launch failed");
   if (dtype == SMA_FP32) {
     e = launch_attn_simt(p, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch failed");
@@ -1331,6 +1417,50 @@ sma_status varlen_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   const int rc = launch_attn_tc(p, st, msg, sizeof(msg));
   if (rc != SMA_OK) return fail(rc, "%s", msg);
   return ok();
+}
+
+sma_status varlen_attn_fwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t head_dim, int32_t total_q, int32_t total_k, int32_t max_q,
+                           int32_t max_k, float scale, int32_t is_causal, const int32_t* cu_seqlens_q,
+                           const int32_t* cu_seqlens_k, const void* q, const int64_t q_strides[2],
+                           const void* k, const int64_t k_strides[2], const void* v,
+                           const int64_t v_strides[2], void* out, const int64_t o_strides[2],
+                           float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  return varlen_fwd_impl(dtype, batch, heads, kv_heads, head_dim, total_q, total_k, max_q, max_k,
+                         scale, is_causal, cu_seqlens_q, cu_seqlens_k, q, q_strides, k, k_strides, v,
+                         v_strides, out, o_strides, lse, workspace, workspace_bytes, VarlenAux{},
+                         stream);
+}
+
+sma_status varlen_masked_attn_fwd_workspace_size(int32_t batch, int32_t heads, int32_t kv_heads,
+                                                 int32_t max_q, int32_t max_k, int32_t head_dim,
+                                                 const int64_t mask_sizes[4], size_t* bytes) {
+  if (bytes == nullptr) return fail(SMA_ERR_INVALID_ARG, "bytes is NULL");
+  sma_status s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (batch < 1 || max_q < 1 || max_k < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, max_q and max_k must be >= 1");
+  const VarlenLists vl = varlen_lists_geom(batch, heads, kv_heads, max_q, max_k, head_dim, mask_sizes);
+  *bytes = lists_layout(vl.codes_bytes, static_cast<int64_t>(batch) * vl.LH * ceil_div(max_q, kTile),
+                        static_cast<int>(ceil_div(max_k, kTile))).end;
+  return ok();
+}
+
+sma_status varlen_masked_attn_fwd(
+    int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads, int32_t head_dim, int32_t total_q,
+    int32_t total_k, int32_t max_q, int32_t max_k, float scale, int32_t is_causal,
+    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const void* q,
+    const int64_t q_strides[2], const void* k, const int64_t k_strides[2], const void* v,
+    const int64_t v_strides[2], const uint8_t* mask, const int64_t mask_sizes[4],
+    const int64_t mask_strides[4], const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+    const int64_t bias_strides[4], void* out, const int64_t o_strides[2], float* lse,
+    void* workspace, size_t workspace_bytes, void* stream) {
+  VarlenAux ax;
+  ax.mask = mask; ax.mask_sizes = mask_sizes; ax.mask_strides = mask_strides;
+  ax.bias = bias; ax.bias_dtype = bias_dtype; ax.bias_sizes = bias_sizes; ax.bias_strides = bias_strides;
+  return varlen_fwd_impl(dtype, batch, heads, kv_heads, head_dim, total_q, total_k, max_q, max_k,
+                         scale, is_causal, cu_seqlens_q, cu_seqlens_k, q, q_strides, k, k_strides, v,
+                         v_strides, out, o_strides, lse, workspace, workspace_bytes, ax, stream);
 }
 
 sma_status varlen_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t total_q,
@@ -1346,16 +1476,18 @@ sma_status varlen_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t 
   return ok();
 }
 
-sma_status varlen_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
-                           int32_t head_dim, int32_t total_q, int32_t total_k, int32_t max_q,
-                           int32_t max_k, float scale, int32_t is_causal, const int32_t* cu_seqlens_q,
-                           const int32_t* cu_seqlens_k, const void* q, const int64_t q_strides[2],
-                           const void* k, const int64_t k_strides[2], const void* v,
-                           const int64_t v_strides[2], const void* out, const int64_t o_strides[2],
-                           const float* lse, const void* dout, const int64_t do_strides[2],
-                           void* dq, const int64_t dq_strides[2], void* dk,
-                           const int64_t dk_strides[2], void* dv, const int64_t dv_strides[2],
-                           void* workspace, size_t workspace_bytes, void* stream) {
+static sma_status varlen_bwd_impl(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                                  int32_t head_dim, int32_t total_q, int32_t total_k, int32_t max_q,
+                                  int32_t max_k, float scale, int32_t is_causal,
+                                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                  const void* q, const int64_t q_strides[2], const void* k,
+                                  const int64_t k_strides[2], const void* v,
+                                  const int64_t v_strides[2], const void* out,
+                                  const int64_t o_strides[2], const float* lse, const void* dout,
+                                  const int64_t do_strides[2], void* dq, const int64_t dq_strides[2],
+                                  void* dk, const int64_t dk_strides[2], void* dv,
+                                  const int64_t dv_strides[2], void* workspace,
+                                  size_t workspace_bytes, const VarlenAux& ax, void* stream) {
   if (!valid_dtype(dtype)) return fail(SMA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   sma_status s = check_heads(heads, kv_heads, head_dim);
   if (s != SMA_OK) return s;
@@ -1379,18 +1511,25 @@ sma_status varlen_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   if ((s = check_grad_operands(dtype, total_q, total_k, out, os, lse, dout, gs, dq, dqs, dk, dks, dv,
                                dvs)) != SMA_OK)
     return s;
-  size_t need = 0;
-  if ((s = varlen_attn_bwd_workspace_size(batch, heads, total_q, max_q, max_k, head_dim, &need)) !=
-      SMA_OK)
+  if (ax.dbias != nullptr && ax.bias == nullptr)
+    return fail(SMA_ERR_INVALID_ARG, "dbias needs the bias (it takes the bias's shape)");
+  if (ax.dbias != nullptr && (reinterpret_cast<uintptr_t>(ax.dbias) & 15u) != 0)
+    return fail(SMA_ERR_INVALID_ARG, "dbias must be 16-byte aligned");
+  AuxView mview, bview;
+  if ((s = check_varlen_aux(ax, batch, heads, kv_heads, max_q, max_k, &mview, &bview)) != SMA_OK)
     return s;
-  if ((s = check_workspace(workspace, workspace_bytes, need)) != SMA_OK) return s;
+  const bool has_mask = ax.mask != nullptr, has_bias = ax.bias != nullptr;
+  const VarlenLists vl = varlen_lists_geom(batch, heads, kv_heads, max_q, max_k, head_dim,
+                                           has_mask ? ax.mask_sizes : nullptr);
+  const int QT = static_cast<int>(ceil_div(max_q, kTile));
+  const int KT = static_cast<int>(ceil_div(max_k, kTile));
+  const BwdLayout lay = bwd_layout(vl.codes_bytes, static_cast<int64_t>(batch) * vl.LH, QT, KT, 1,
+                                   heads, total_q, head_dim);
+  if ((s = check_workspace(workspace, workspace_bytes, lay.total)) != SMA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   int* err = device_error_word(&e);
   if (err == nullptr) return cuda_fail(e, "device error word unavailable");
-  const int QT = static_cast<int>(ceil_div(max_q, kTile));
-  const int KT = static_cast<int>(ceil_div(max_k, kTile));
-  const BwdLayout lay = bwd_layout(0, batch, QT, KT, 1, heads, total_q, head_dim);
   BwdProblem b{};
   AttnProblem& p = b.f;
   p.dtype = dtype;
@@ -1412,17 +1551,95 @@ sma_status varlen_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
   p.total_q = total_q;
   p.total_k = total_k;
   p.err = err;
-  p.lists.LB = batch; p.lists.LH = 1; p.lists.head_mode = 0;
+  p.has_mask = has_mask;
+  p.has_bias = has_bias;
+  if (has_mask) p.mask = mview;
+  if (has_bias) p.bias = bview;
+  p.lists.LB = batch; p.lists.LH = vl.LH; p.lists.head_mode = vl.head_mode;
   int32_t* nf = at<int32_t>(workspace, lay.fl.nf);
   int32_t* np = at<int32_t>(workspace, lay.fl.np);
   int32_t* fi = at<int32_t>(workspace, lay.fl.fi);
   int32_t* pi = at<int32_t>(workspace, lay.fl.pi);
   p.lists.num_full = nf; p.lists.num_part = np; p.lists.full_idx = fi; p.lists.part_idx = pi;
-  e = launch_varlen_lists(p, nf, fi, np, pi, st);
-  if (e != cudaSuccess) return cuda_fail(e, "tile list launch failed");
+  if ((e = launch_varlen_aux_lists(p, ax, mview, vl, workspace, lay.fl, st)) != cudaSuccess)
+    return cuda_fail(e, "tile list launch failed");
   set_grads(b, dout, gs, dq, dqs, dk, dks, dv, dvs, sc);
+  if (ax.dbias != nullptr) {
+    // as masked_attn_bwd: contiguous fp32 at the bias's sizes, rows and
+    // columns sequence-local
+    const int64_t kd = ax.bias_sizes[3];
+    const int64_t nb = ax.bias_sizes[0], nh = ax.bias_sizes[1], nq = ax.bias_sizes[2];
+    e = cudaMemsetAsync(ax.dbias, 0, static_cast<size_t>(nb * nh * nq * kd) * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "dbias zeroing failed");
+    if (kd > 1 || max_k == 1) {
+      b.dbias = ax.dbias;
+      b.db_sq = nq > 1 ? kd : 0;
+      b.db_sh = nh > 1 ? nq * kd : 0;
+      b.db_sb = nb > 1 ? nh * nq * kd : 0;
+      b.db_kd = static_cast<int>(kd);
+      const int db_hpq = nh == heads ? 1 : 0;
+      b.db_head_per_query = db_hpq;
+      const bool own_head = heads == 1 || (nh > 1 && (db_hpq || p.group == 1));
+      const bool own_batch = batch == 1 || nb > 1;
+      b.db_mode = nq == 1 ? kDbiasRowSum : (own_head && own_batch ? kDbiasStore : kDbiasAdd);
+    }
+  }
   if ((s = run_backward(b, workspace, lay, st)) != SMA_OK) return s;
   return ok();
+}
+
+sma_status varlen_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads,
+                           int32_t head_dim, int32_t total_q, int32_t total_k, int32_t max_q,
+                           int32_t max_k, float scale, int32_t is_causal, const int32_t* cu_seqlens_q,
+                           const int32_t* cu_seqlens_k, const void* q, const int64_t q_strides[2],
+                           const void* k, const int64_t k_strides[2], const void* v,
+                           const int64_t v_strides[2], const void* out, const int64_t o_strides[2],
+                           const float* lse, const void* dout, const int64_t do_strides[2],
+                           void* dq, const int64_t dq_strides[2], void* dk,
+                           const int64_t dk_strides[2], void* dv, const int64_t dv_strides[2],
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  return varlen_bwd_impl(dtype, batch, heads, kv_heads, head_dim, total_q, total_k, max_q, max_k,
+                         scale, is_causal, cu_seqlens_q, cu_seqlens_k, q, q_strides, k, k_strides, v,
+                         v_strides, out, o_strides, lse, dout, do_strides, dq, dq_strides, dk,
+                         dk_strides, dv, dv_strides, workspace, workspace_bytes, VarlenAux{}, stream);
+}
+
+sma_status varlen_masked_attn_bwd_workspace_size(int32_t batch, int32_t heads, int32_t kv_heads,
+                                                 int32_t total_q, int32_t max_q, int32_t max_k,
+                                                 int32_t head_dim, const int64_t mask_sizes[4],
+                                                 size_t* bytes) {
+  if (bytes == nullptr) return fail(SMA_ERR_INVALID_ARG, "bytes is NULL");
+  sma_status s = check_heads(heads, kv_heads, head_dim);
+  if (s != SMA_OK) return s;
+  if (batch < 1 || total_q < 1 || max_q < 1 || max_k < 1)
+    return fail(SMA_ERR_INVALID_ARG, "batch, total_q and maxima must be >= 1");
+  const VarlenLists vl = varlen_lists_geom(batch, heads, kv_heads, max_q, max_k, head_dim, mask_sizes);
+  *bytes = bwd_layout(vl.codes_bytes, static_cast<int64_t>(batch) * vl.LH,
+                      static_cast<int>(ceil_div(max_q, kTile)), static_cast<int>(ceil_div(max_k, kTile)),
+                      1, heads, total_q, head_dim)
+               .total;
+  return ok();
+}
+
+sma_status varlen_masked_attn_bwd(
+    int32_t dtype, int32_t batch, int32_t heads, int32_t kv_heads, int32_t head_dim, int32_t total_q,
+    int32_t total_k, int32_t max_q, int32_t max_k, float scale, int32_t is_causal,
+    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const void* q,
+    const int64_t q_strides[2], const void* k, const int64_t k_strides[2], const void* v,
+    const int64_t v_strides[2], const uint8_t* mask, const int64_t mask_sizes[4],
+    const int64_t mask_strides[4], const void* bias, int32_t bias_dtype, const int64_t bias_sizes[4],
+    const int64_t bias_strides[4], const void* out, const int64_t o_strides[2], const float* lse,
+    const void* dout, const int64_t do_strides[2], void* dq, const int64_t dq_strides[2], void* dk,
+    const int64_t dk_strides[2], void* dv, const int64_t dv_strides[2], float* dbias,
+    void* workspace, size_t workspace_bytes, void* stream) {
+  VarlenAux ax;
+  ax.mask = mask; ax.mask_sizes = mask_sizes; ax.mask_strides = mask_strides;
+  ax.bias = bias; ax.bias_dtype = bias_dtype; ax.bias_sizes = bias_sizes; ax.bias_strides = bias_strides;
+  ax.dbias = dbias;
+  return varlen_bwd_impl(dtype, batch, heads, kv_heads, head_dim, total_q, total_k, max_q, max_k,
+                         scale, is_causal, cu_seqlens_q, cu_seqlens_k, q, q_strides, k, k_strides, v,
+                         v_strides, out, o_strides, lse, dout, do_strides, dq, dq_strides, dk,
+                         dk_strides, dv, dv_strides, workspace, workspace_bytes, ax, stream);
 }
 
 static sma_status check_pad_args(int32_t dtype, int32_t batch, int32_t max_len, int32_t heads,

@@ -12,7 +12,8 @@
 //   own broadcast shape (flash-sparse-attention PR #190 contract), one
 //   streaming pass over the mask.
 // * explicit_lists_kernel -- lists for masked_attn_fwd from those codes plus
-//   causal and key-length geometry.
+//   causal and key-length geometry (per sequence for packed batches with a
+//   mask or bias).
 #include "device_common.cuh"
 #include "kernels.h"
 
@@ -213,9 +214,23 @@ __global__ void __launch_bounds__(kMapThreads)
 explicit_lists_kernel(AttnProblem p, const uint8_t* __restrict__ codes, int codes_qt,
                       int32_t* num_full, int32_t* full_idx, int32_t* num_part, int32_t* part_idx) {
   const int qt = blockIdx.x, lh = blockIdx.y, lb = blockIdx.z;
+  // query / key lengths: the problem's, or for packed sequences (cu_q set;
+  // list batch row lb is sequence lb) the sequence's, whose malformed
+  // offsets are reported and leave it empty
+  int Lq = p.Lq, Lk = p.Lk;
+  if (p.cu_q != nullptr) {
+    Lq = p.cu_q[lb + 1] - p.cu_q[lb];
+    Lk = p.cu_k[lb + 1] - p.cu_k[lb];
+    if (Lq < 0 || Lk < 0 || Lq > p.Lq || Lk > p.Lk || p.cu_q[lb] < 0 || p.cu_k[lb] < 0 ||
+        p.cu_q[lb + 1] > p.total_q || p.cu_k[lb + 1] > p.total_k) {
+      if (threadIdx.x == 0 && qt == 0 && lh == 0) report_error(p.err, SMA_ERR_DEVICE_INPUT);
+      Lq = 0;
+      Lk = 0;
+    }
+  }
   const int q0 = qt * kTile;
-  const int q1 = min(q0 + kTile, p.Lq);
-  const int off = p.Lk - p.Lq;
+  const int q1 = min(q0 + kTile, Lq);
+  const int off = Lk - Lq;
   // mask code rows used by this list
   int mh0 = 0, mh1 = -1;  // mask head indices (before stride folding)
   if (p.has_mask) {
@@ -235,8 +250,9 @@ explicit_lists_kernel(AttnProblem p, const uint8_t* __restrict__ codes, int code
 
   auto code_of = [&](int kt) -> int {
     const int k0 = kt * kTile;
-    const int k1 = min(k0 + kTile, p.Lk);
-    int c = ((kt + 1) * kTile <= p.Lk) ? SMA_TILE_FULL : SMA_TILE_PARTIAL;
+    if (q0 >= Lq || k0 >= Lk) return SMA_TILE_EMPTY;
+    const int k1 = min(k0 + kTile, Lk);
+    int c = ((kt + 1) * kTile <= Lk) ? SMA_TILE_FULL : SMA_TILE_PARTIAL;
     if (p.causal) {
       int cc;
       if (k1 - 1 <= q0 + off) cc = SMA_TILE_FULL;

@@ -432,13 +432,21 @@ def _cu(t: torch.Tensor, batch=None) -> torch.Tensor:
 
 
 def varlen_attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
-                    is_causal: bool = False, scale=None, out=None, return_lse: bool = True, workspace=None):
+                    is_causal: bool = False, scale=None, out=None, return_lse: bool = True, workspace=None,
+                    mask=None, bias=None):
     """Attention over packed variable-length sequences.
 
     q ``[total_q, H, d]``, k/v ``[total_k, KVH, d]``; sequence b is rows
     ``cu_seqlens_q[b]:cu_seqlens_q[b+1]`` of q (keys likewise) and attends
     only its own keys (bottom-right causal per sequence when ``is_causal``).
-    Returns ``(out, lse)``, lse float32 ``[H, total_q]``."""
+    ``mask`` / ``bias``: 4D in the padded per-sequence layout of
+    ``masked_attn_fwd`` for ``[batch, max_seqlen_q, H, max_seqlen_k]``
+    (element ``(b, h, q, k)`` for sequence-local q and k), through
+    ``varlen_masked_attn_fwd``.  Returns ``(out, lse)``, lse float32
+    ``[H, total_q]``."""
+    if mask is not None or bias is not None:
+        return _varlen_masked_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, is_causal,
+                                  scale, out, return_lse, workspace, mask, bias)
     _require_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k)
     total_q, h, dh = q.shape
     total_k, kvh = k.shape[0], k.shape[1]
@@ -461,13 +469,49 @@ def varlen_attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
     return out, lse
 
 
+def _varlen_masked_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_q, max_k, is_causal, scale, out, return_lse,
+                       workspace, mask, bias):
+    _require_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k, mask, bias)
+    total_q, h, dh = q.shape
+    total_k, kvh = k.shape[0], k.shape[1]
+    b = cu_seqlens_q.shape[0] - 1
+    cq, ck = _cu(cu_seqlens_q), _cu(cu_seqlens_k, b)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k and v must share a dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((h, total_q), dtype=torch.float32, device=q.device) if return_lse else None
+    n = ctypes.c_size_t()
+    ms = nat.i64_array(mask.shape) if mask is not None else None
+    nat.check(_lib().varlen_masked_attn_fwd_workspace_size(b, h, kvh, int(max_q), int(max_k), dh, ms,
+                                                           ctypes.byref(n)))
+    if workspace is None:
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=q.device)
+    mp, msz, mst = _aux_args(mask, max_k)
+    bp, bsz, bst = _aux_args(bias, max_k)
+    nat.check(_lib().varlen_masked_attn_fwd(
+        _dtype_code(q), b, h, kvh, dh, total_q, total_k, int(max_q), int(max_k),
+        ctypes.c_float(0.0 if scale is None else float(scale)), 1 if is_causal else 0,
+        _ptr(cq), _ptr(ck), _ptr(q), _strides2(q), _ptr(k), _strides2(k), _ptr(v), _strides2(v),
+        mp, msz, mst, bp, _dtype_code(bias) if bias is not None else 0, bsz, bst,
+        _ptr(out), _strides2(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(q)))
+    return out, lse
+
+
 def varlen_attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
                     max_seqlen_k: int, is_causal: bool = False, scale=None, dq=None, dk=None, dv=None,
-                    workspace=None):
-    """Gradients of ``varlen_attn_fwd`` (same sequences, causal flag and
-    scale): ``out`` and ``lse`` are that call's results, ``dout`` the upstream
-    gradient ``[total_q, H, d]``.  Returns ``(dq, dk, dv)`` in the packed
-    layouts of q and k."""
+                    workspace=None, mask=None, bias=None, return_dbias: bool = False, dbias=None):
+    """Gradients of ``varlen_attn_fwd`` (same sequences, mask / bias, causal
+    flag and scale): ``out`` and ``lse`` are that call's results, ``dout`` the
+    upstream gradient ``[total_q, H, d]``.  Returns ``(dq, dk, dv)`` in the
+    packed layouts of q and k, or ``(dq, dk, dv, dbias)`` with
+    ``return_dbias`` (or a ``dbias`` buffer): float32 at the bias's shape."""
+    if mask is not None or bias is not None:
+        return _varlen_masked_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                                  max_seqlen_k, is_causal, scale, dq, dk, dv, workspace, mask, bias,
+                                  return_dbias, dbias)
+    if return_dbias or dbias is not None:
+        raise ValueError("dbias needs a bias")
     _require_cuda(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k)
     total_q, h, dh = q.shape
     total_k, kvh = k.shape[0], k.shape[1]
@@ -490,6 +534,45 @@ def varlen_attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seq
         _ptr(out), _strides2(out), _ptr(lse), _ptr(dout), _strides2(dout), _ptr(dq), _strides2(dq),
         _ptr(dk), _strides2(dk), _ptr(dv), _strides2(dv), _ptr(workspace), workspace.numel(), _stream(q)))
     return dq, dk, dv
+
+
+def _varlen_masked_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_q, max_k, is_causal, scale,
+                       dq, dk, dv, workspace, mask, bias, return_dbias, dbias):
+    _require_cuda(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, mask, bias)
+    total_q, h, dh = q.shape
+    total_k, kvh = k.shape[0], k.shape[1]
+    b = cu_seqlens_q.shape[0] - 1
+    cq, ck = _cu(cu_seqlens_q), _cu(cu_seqlens_k, b)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (h, total_q) or not lse.is_contiguous():
+        raise ValueError("lse must be the forward's contiguous float32 [heads, total_q]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(k) if dv is None else dv
+    want_db = return_dbias or dbias is not None
+    if want_db:
+        if bias is None:
+            raise ValueError("dbias needs a bias")
+        if dbias is None:
+            dbias = torch.empty(tuple(bias.shape), dtype=torch.float32, device=q.device)
+        elif dbias.dtype != torch.float32 or tuple(dbias.shape) != tuple(bias.shape) or not dbias.is_contiguous():
+            raise ValueError("dbias must be contiguous float32 with the bias's shape")
+    n = ctypes.c_size_t()
+    ms = nat.i64_array(mask.shape) if mask is not None else None
+    nat.check(_lib().varlen_masked_attn_bwd_workspace_size(b, h, kvh, total_q, int(max_q), int(max_k), dh, ms,
+                                                           ctypes.byref(n)))
+    if workspace is None:
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=q.device)
+    mp, msz, mst = _aux_args(mask, max_k)
+    bp, bsz, bst = _aux_args(bias, max_k)
+    nat.check(_lib().varlen_masked_attn_bwd(
+        _dtype_code(q), b, h, kvh, dh, total_q, total_k, int(max_q), int(max_k),
+        ctypes.c_float(0.0 if scale is None else float(scale)), 1 if is_causal else 0,
+        _ptr(cq), _ptr(ck), _ptr(q), _strides2(q), _ptr(k), _strides2(k), _ptr(v), _strides2(v),
+        mp, msz, mst, bp, _dtype_code(bias) if bias is not None else 0, bsz, bst,
+        _ptr(out), _strides2(out), _ptr(lse), _ptr(dout), _strides2(dout), _ptr(dq), _strides2(dq),
+        _ptr(dk), _strides2(dk), _ptr(dv), _strides2(dv), _ptr(dbias) if want_db else ctypes.c_void_p(0),
+        _ptr(workspace), workspace.numel(), _stream(q)))
+    return (dq, dk, dv, dbias) if want_db else (dq, dk, dv)
 
 
 def varlen_pad(packed: torch.Tensor, cu_seqlens: torch.Tensor, max_len: int) -> torch.Tensor:
