@@ -230,9 +230,12 @@ decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap m
           smem8<DT>(kt + (c * D + e0) * L::kEsz, kf);
 #pragma unroll
           for (int r = 0; r < G; ++r) {
-            float d = 0.f;
+            // two products per instruction (fp32 pairs), the halves added last
+            float2 d2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) d = fmaf(qf[r][e], kf[e], d);
+            for (int e = 0; e < 8; e += 2)
+              d2 = fma2(make_float2(qf[r][e], qf[r][e + 1]), make_float2(kf[e], kf[e + 1]), d2);
+            float d = d2.x + d2.y;
 #pragma unroll
             for (int off = 1; off < LPK; off <<= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
             const bool keep = s_keep[(s * G + r) * T + c] != 0;
@@ -261,7 +264,11 @@ decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap m
           l[r] = l[r] * alpha + ps;
           m[r] = m_new;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) o[r][e] *= alpha;
+          for (int e = 0; e < 8; e += 2) {
+            const float2 oo = mul2(make_float2(o[r][e], o[r][e + 1]), make_float2(alpha, alpha));
+            o[r][e] = oo.x;
+            o[r][e + 1] = oo.y;
+          }
         }
 #pragma unroll
         for (int st = 0; st < kSub; ++st) {
@@ -271,7 +278,12 @@ decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap m
 #pragma unroll
           for (int r = 0; r < G; ++r)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) o[r][e] = fmaf(sc[st][r], vf[e], o[r][e]);
+            for (int e = 0; e < 8; e += 2) {
+              const float2 oo = fma2(make_float2(sc[st][r], sc[st][r]), make_float2(vf[e], vf[e + 1]),
+                                     make_float2(o[r][e], o[r][e + 1]));
+              o[r][e] = oo.x;
+              o[r][e + 1] = oo.y;
+            }
         }
       }
       __syncwarp();
