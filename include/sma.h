@@ -398,7 +398,7 @@ sma_status masked_attn_bwd(int32_t dtype, int32_t batch, int32_t heads, int32_t 
 /* Bytes of the second workspace masked_attn_bwd_deterministic needs for a
  * bias of sizes bias_sizes (b', h', q', kd): the fixed-order partial sums,
  * batch * heads * R * kd * 4 with R = q_len for a bias with a query dim (or
- * dtype SMA_FP32), else ceil(q_len / G) (G = 64 at head_dim 128, 32 at 64).
+ * dtype SMA_FP32), else ceil(q_len / 64) (query groups of 64 rows).
  * 0 when every dbias element already has a single writer (a bias with its
  * own element for each batch row, query head and query). */
 sma_status masked_attn_bwd_dbias_workspace_size(int32_t dtype, int32_t batch, int32_t heads,

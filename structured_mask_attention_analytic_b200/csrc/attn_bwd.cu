@@ -8,35 +8,22 @@
 //   dV = P^T dO              dP = dO V^T          D = rowsum(dO * O)
 //   dS = P * (dP - D)        dQ = scale * dS K    dK = scale * dS^T Q
 //
-// One persistent CTA per SM walks units (batch, KV head, 128-key tile).  A
-// unit loops over the (query head of the group, 128-row query tile) pairs
-// that attend its key tile -- the transposed tile lists -- accumulating dK
-// and dV in TMEM over the whole group; each pair's dQ contribution is added
-// into an fp32 accumulator in global memory.
+// One kernel serves head dims 64 and 128 (attn_bwd_t_kernel below).  One
+// persistent CTA per SM walks units (batch, KV head, 128-key tile).  A unit
+// loops over the (query head of the group, 128-row query tile) pairs that
+// attend its key tile -- the transposed tile lists -- accumulating dK and dV
+// in TMEM over the whole group; each pair's dQ tile is added into an fp32
+// accumulator in global memory by bulk tensor reductions from shared memory.
+// The products are formed transposed (key rows in TMEM lanes), so P^T can
+// stay in TMEM as dV's A operand and dS^T, stored once in shared memory,
+// serves both dK (read K-major) and dQ (read MN-major); the layout of TMEM
+// and shared memory and the warp roles are given with the kernel.
 //
-// Per pair, five 128-row products on the tensor cores (bf16/f16 operands
-// from shared memory, fp32 accumulators in TMEM):
-//   S  = Q K^T        A = Q  (K-major)      B = K  (K-major)       -> cols [0, 128)
-//   dP = dO V^T       A = dO (K-major)      B = V  (K-major)       -> cols [128, 256)
-//   dV += P^T dO      A = P^T (MN-major)    B = dO (MN-major)      -> cols [256, 256+D)
-//   dK += dS^T Q      A = dS^T (MN-major)   B = Q  (MN-major)      -> cols [256+D, 256+2D)
-//   dQ  = dS K        A = dS (K-major)      B = K  (MN-major)      -> cols [128, 128+D)
-// P and dS are written by the compute warps into shared memory in the same
-// 128-byte swizzled layout TMA gives a [128][128] tile, so one tile serves as
-// both a K-major operand and (transposed) an MN-major one.  dQ reuses dP's
-// columns once dS is formed.
-//
-// Warp roles (320 threads):
-//   warps 0-3  compute: row r of a query tile; phase A forms P from S (mask,
-//              bias, lse) and stores it; phase B forms dS = P (dP - D) and
-//              stores it.  dS uses P as stored (rounded to the operand type,
-//              as the dV product sees it).
-//   warps 4-7  dQ drain (TMEM -> vector atomic adds into the fp32 dQ
-//              accumulator) and the unit's dK / dV epilogue.
-//   warp  8    TMA producer: K, V once per unit; Q (2 stages), dO (1 stage)
-//   warp  9    MMA issuer (one elected lane), in the order
-//              S(0) dP(0) | dV(p) S(p+1) | dK(p) dQ(p) | dP(p+1) ..., the two
-//              products of each group issued with their k-steps interleaved.
+// The bias gradient is dS itself for a full bias and dS summed over the
+// broadcast query axis otherwise.  Such sums are added with atomics by
+// default; in the deterministic mode each 64-query group's sum is stored to
+// its own slot and a second kernel (dbias_reduce_kernel) adds the slots in a
+// fixed order, so dbias is bit-identical from run to run.
 // Every mbarrier wait is bounded; on expiry the CTA raises its abort flag,
 // drains its own copies and products, frees TMEM and returns.
 #include <cstdio>
@@ -49,36 +36,7 @@
 namespace sma {
 namespace {
 
-constexpr int kBwdThreads = 320;
-constexpr int kBLoadWarp = 8;
-constexpr int kBMmaWarp = 9;
 constexpr uint32_t kBTmemCols = 512;
-
-template <int D>
-struct BLayout {
-  static constexpr uint32_t kChunk = kTile * 128;   // 64 columns x 128 rows, 128B-swizzled
-  static constexpr uint32_t kTileD = kTile * D * 2;  // [128][D] 16-bit tile
-  static constexpr uint32_t kTileK = kTile * kTile * 2;  // [128][128] 16-bit tile (P, dS)
-  static constexpr int kChunksD = D / 64;
-  static constexpr uint32_t kK = 0;
-  static constexpr uint32_t kV = kK + kTileD;
-  static constexpr uint32_t kQ = kV + kTileD;       // 2 stages
-  static constexpr uint32_t kDO = kQ + 2 * kTileD;  // 1 stage
-  static constexpr uint32_t kP = kDO + kTileD;
-  static constexpr uint32_t kDS = kP + kTileK;
-  static constexpr uint32_t kBars = kDS + kTileK;
-  enum : int {
-    kKVFull = 0, kKVEmpty, kQFull, kQEmpty = kQFull + 2, kOFull = kQEmpty + 2, kOEmpty,
-    kSFull, kPDone, kDPFull, kDSDone, kDQFull, kDQFree, kPFree, kDSFree, kAccDone, kAccFree,
-    kDrain, kNumBars
-  };
-  static constexpr uint32_t kTmemSlot = kBars + 8 * kNumBars;
-  static constexpr uint32_t kAbort = kTmemSlot + 4;
-  static constexpr uint32_t kBytes = kAbort + 4;
-  static constexpr uint32_t kAlloc = kBytes + 1024;  // base rounded up to 1024
-  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
-  static_assert(kAlloc <= 232448, "shared memory budget");
-};
 
 // Transposed-list row of the query heads g of a unit.
 __device__ __forceinline__ int64_t bwd_row(const BwdProblem& p, int b, int hk, int g) {
@@ -198,571 +156,8 @@ __device__ __forceinline__ float2 unpack2(uint32_t w) {
   return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }
 
-template <int D, int POLICY, int DT>
-__global__ void __launch_bounds__(kBwdThreads, 1)
-attn_bwd_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
-                const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-                const __grid_constant__ CUtensorMap map_do, int n_units) {
-  using L = BLayout<D>;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const uint32_t sbase = smem_u32(smem);
-  auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * static_cast<uint32_t>(i); };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    mbar_init(bar(L::kKVFull), 1);
-    mbar_init(bar(L::kKVEmpty), 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(L::kQFull + s), 1);
-      mbar_init(bar(L::kQEmpty + s), 1);
-    }
-    mbar_init(bar(L::kOFull), 1);
-    mbar_init(bar(L::kOEmpty), 1);
-    mbar_init(bar(L::kSFull), 1);
-    mbar_init(bar(L::kPDone), 128);
-    mbar_init(bar(L::kDPFull), 1);
-    mbar_init(bar(L::kDSDone), 128);
-    mbar_init(bar(L::kDQFull), 1);
-    mbar_init(bar(L::kDQFree), 128);
-    mbar_init(bar(L::kPFree), 1);
-    mbar_init(bar(L::kDSFree), 1);
-    mbar_init(bar(L::kAccDone), 1);
-    mbar_init(bar(L::kAccFree), 128);
-    mbar_init(bar(L::kDrain), 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == kBMmaWarp) {
-    tmem_alloc(smem_u32(tmem_slot), kBTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == kBLoadWarp) {
-    // ------------------------------------------------------------ producer
-    if (elect_one()) {
-      tma_prefetch_map(&map_q);
-      tma_prefetch_map(&map_k);
-      tma_prefetch_map(&map_v);
-      tma_prefetch_map(&map_do);
-    }
-    __syncwarp();
-    uint32_t kv_it = 0, q_it = 0, o_it = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const BUnit w = bwd_unit(p, u);
-      if (w.n_pairs == 0) continue;
-      if (kv_it > 0 && !mbar_wait_warp(bar(L::kKVEmpty), (kv_it - 1) & 1, abort_flag, p.f.err)) {
-        ok = false;
-        break;
-      }
-      if (elect_one()) {
-        mbar_arrive_expect_tx(bar(L::kKVFull), 2 * L::kTileD);
-        for (int c = 0; c < L::kChunksD; ++c) {
-          tma_load_4d(sbase + L::kK + c * L::kChunk, &map_k, bar(L::kKVFull), c * 64, w.hk,
-                      w.k_off + w.kt * kTile, w.bt);
-          tma_load_4d(sbase + L::kV + c * L::kChunk, &map_v, bar(L::kKVFull), c * 64, w.hk,
-                      w.k_off + w.kt * kTile, w.bt);
-        }
-      }
-      __syncwarp();
-      ++kv_it;
-      PairWalk pw;
-      pw.begin(p, w);
-      for (int i = 0; i < w.n_pairs && ok; ++i, pw.next(p, w)) {
-        bool partial;
-        const int qt = pw.qtile(p, w, &partial);
-        const int h = pw.head(w);
-        const int s = q_it & 1;
-        const uint32_t use = q_it >> 1;
-        if (use > 0 && !mbar_wait_warp(bar(L::kQEmpty + s), (use - 1) & 1, abort_flag, p.f.err)) {
-          ok = false;
-          break;
-        }
-        if (elect_one()) {
-          mbar_arrive_expect_tx(bar(L::kQFull + s), L::kTileD);
-          for (int c = 0; c < L::kChunksD; ++c)
-            tma_load_4d(sbase + L::kQ + s * L::kTileD + c * L::kChunk, &map_q, bar(L::kQFull + s),
-                        c * 64, h, w.q_off + qt * kTile, w.bt);
-        }
-        __syncwarp();
-        ++q_it;
-        if (o_it > 0 && !mbar_wait_warp(bar(L::kOEmpty), (o_it - 1) & 1, abort_flag, p.f.err)) {
-          ok = false;
-          break;
-        }
-        if (elect_one()) {
-          mbar_arrive_expect_tx(bar(L::kOFull), L::kTileD);
-          for (int c = 0; c < L::kChunksD; ++c)
-            tma_load_4d(sbase + L::kDO + c * L::kChunk, &map_do, bar(L::kOFull), c * 64, h,
-                        w.q_off + qt * kTile, w.bt);
-        }
-        __syncwarp();
-        ++o_it;
-      }
-    }
-    if (!ok) {
-      // every copy this warp issued must land before the CTA exits
-      if (kv_it > 0) bdrain_wait(bar(L::kKVFull), (kv_it - 1) & 1, p.f.err);
-      for (uint32_t t = 0; t < 2; ++t) {
-        if (q_it > t) {
-          const uint32_t nn = q_it - 1 - t;
-          bdrain_wait(bar(L::kQFull + (nn & 1)), (nn >> 1) & 1, p.f.err);
-        }
-      }
-      if (o_it > 0) bdrain_wait(bar(L::kOFull), (o_it - 1) & 1, p.f.err);
-    }
-  } else if (warp == kBMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t fmt = DT == SMA_BF16 ? 1u : 0u;
-    constexpr uint32_t idesc_s = mma_idesc_f16(fmt, 128, 128, 0, 0);  // S, dP
-    constexpr uint32_t idesc_t = mma_idesc_f16(fmt, 128, D, 1, 1);    // dV, dK
-    constexpr uint32_t idesc_q = mma_idesc_f16(fmt, 128, D, 0, 1);    // dQ
-    auto with_lo = [](uint64_t d, uint32_t add) -> uint64_t {
-      return (d & 0xffffffff00000000ull) | static_cast<uint32_t>(static_cast<uint32_t>(d) + add);
-    };
-    // Two independent products issued with their k-steps interleaved: each
-    // k-step of a chain depends on the previous one through its accumulator,
-    // so alternating two chains keeps the tensor pipe busy.
-    auto issue_s_dp = [&](uint32_t q_addr, bool with_s, bool with_dp) {
-      const uint64_t qd = smem_desc_sw128(q_addr, 16, 1024);
-      const uint64_t kd = smem_desc_sw128(sbase + L::kK, 16, 1024);
-      const uint64_t od = smem_desc_sw128(sbase + L::kDO, 16, 1024);
-      const uint64_t vd = smem_desc_sw128(sbase + L::kV, 16, 1024);
-#pragma unroll
-      for (int s = 0; s < D / 16; ++s) {
-        const uint32_t off = ((s >> 2) * L::kChunk + (s & 3) * 32) >> 4;
-        if (with_s) tc_mma_ss(tmem + L::kColS, with_lo(qd, off), with_lo(kd, off), idesc_s, s > 0 ? 1u : 0u);
-        if (with_dp) tc_mma_ss(tmem + L::kColDP, with_lo(od, off), with_lo(vd, off), idesc_s, s > 0 ? 1u : 0u);
-      }
-    };
-    // dV += P^T dO interleaved with S(next) = Q(next) K^T (when there is one)
-    auto issue_dv_s = [&](bool acc, bool with_s, uint32_t q_addr) {
-      const uint64_t ad = smem_desc_sw128(sbase + L::kP, L::kChunk, 1024);
-      const uint64_t bd = smem_desc_sw128(sbase + L::kDO, L::kChunk, 1024);
-      const uint64_t qd = smem_desc_sw128(q_addr, 16, 1024);
-      const uint64_t kd = smem_desc_sw128(sbase + L::kK, 16, 1024);
-#pragma unroll
-      for (int s = 0; s < kTile / 16; ++s) {
-        const uint32_t off = (s * 2048) >> 4;
-        tc_mma_ss(tmem + L::kColDV, with_lo(ad, off), with_lo(bd, off), idesc_t, (acc || s > 0) ? 1u : 0u);
-        if (with_s && s < D / 16) {
-          const uint32_t so = ((s >> 2) * L::kChunk + (s & 3) * 32) >> 4;
-          tc_mma_ss(tmem + L::kColS, with_lo(qd, so), with_lo(kd, so), idesc_s, s > 0 ? 1u : 0u);
-        }
-      }
-    };
-    // dK += dS^T Q interleaved with dQ = dS K
-    auto issue_dk_dq = [&](bool acc, uint32_t q_addr) {
-      const uint64_t ad = smem_desc_sw128(sbase + L::kDS, L::kChunk, 1024);
-      const uint64_t bd = smem_desc_sw128(q_addr, L::kChunk, 1024);
-      const uint64_t sd = smem_desc_sw128(sbase + L::kDS, 16, 1024);
-      const uint64_t kd = smem_desc_sw128(sbase + L::kK, L::kChunk, 1024);
-#pragma unroll
-      for (int s = 0; s < kTile / 16; ++s) {
-        const uint32_t off = (s * 2048) >> 4;
-        const uint32_t aoff = ((s >> 2) * L::kChunk + (s & 3) * 32) >> 4;
-        tc_mma_ss(tmem + L::kColDK, with_lo(ad, off), with_lo(bd, off), idesc_t, (acc || s > 0) ? 1u : 0u);
-        tc_mma_ss(tmem + L::kColDP, with_lo(sd, aoff), with_lo(kd, off), idesc_q, s > 0 ? 1u : 0u);
-      }
-    };
-    uint32_t kv_it = 0, q_it = 0, o_it = 0, pit = 0, uit = 0;
-    bool ok = true;
-    auto wait = [&](int b_, uint32_t parity) -> bool {
-      if (!mbar_wait_warp(bar(b_), parity, abort_flag, p.f.err)) ok = false;
-      return ok;
-    };
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const BUnit w = bwd_unit(p, u);
-      const int n = w.n_pairs;
-      if (n == 0) continue;
-      if (!wait(L::kKVFull, kv_it & 1)) break;
-      ++kv_it;
-      // S(0) and dP(0)
-      if (!wait(L::kQFull + (q_it & 1), (q_it >> 1) & 1)) break;
-      if (!wait(L::kOFull, o_it & 1)) break;
-      if (pit > 0 && !wait(L::kDQFree, (pit - 1) & 1)) break;
-      tc_fence_after();
-      if (elect_one()) {
-        issue_s_dp(sbase + L::kQ + (q_it & 1) * L::kTileD, true, true);
-        tc_commit(bar(L::kSFull));
-        tc_commit(bar(L::kDPFull));
-      }
-      __syncwarp();
-      for (int i = 0; i < n && ok; ++i) {
-        const int qs = q_it & 1;  // Q stage of pair i
-        const bool more = i + 1 < n;
-        const uint32_t nq = q_it + 1;
-        // dV += P^T dO, with S(i+1) alongside (S's columns are free once P(i) is formed)
-        if (!wait(L::kPDone, pit & 1)) break;
-        if (i == 0 && uit > 0 && !wait(L::kAccFree, (uit - 1) & 1)) break;
-        if (more && !wait(L::kQFull + (nq & 1), (nq >> 1) & 1)) break;
-        tc_fence_after();
-        if (elect_one()) {
-          issue_dv_s(i > 0, more, sbase + L::kQ + (nq & 1) * L::kTileD);
-          tc_commit(bar(L::kPFree));
-          tc_commit(bar(L::kOEmpty));
-          if (more) tc_commit(bar(L::kSFull));
-        }
-        __syncwarp();
-        ++o_it;
-        // dK += dS^T Q and dQ = dS K (into dP's columns)
-        if (!wait(L::kDSDone, pit & 1)) break;
-        tc_fence_after();
-        if (elect_one()) {
-          issue_dk_dq(i > 0, sbase + L::kQ + qs * L::kTileD);
-          tc_commit(bar(L::kDQFull));
-          tc_commit(bar(L::kDSFree));
-          tc_commit(bar(L::kQEmpty + qs));
-        }
-        __syncwarp();
-        ++q_it;
-        ++pit;
-        // dP(i+1) once dO(i+1) is in and dQ(i) has left TMEM
-        if (more) {
-          if (!wait(L::kOFull, o_it & 1)) break;
-          if (!wait(L::kDQFree, (pit - 1) & 1)) break;
-          tc_fence_after();
-          if (elect_one()) {
-            issue_s_dp(0, false, true);
-            tc_commit(bar(L::kDPFull));
-          }
-          __syncwarp();
-        }
-      }
-      if (!ok) break;
-      if (elect_one()) {
-        tc_commit(bar(L::kAccDone));
-        tc_commit(bar(L::kKVEmpty));
-      }
-      __syncwarp();
-      ++uit;
-    }
-    if (!ok) {
-      if (elect_one()) tc_commit(bar(L::kDrain));
-      __syncwarp();
-      bdrain_wait(bar(L::kDrain), 0, p.f.err);
-    }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ compute (P, dS)
-    const int r = warp * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t s_col = tmem + lane_off + L::kColS;
-    const uint32_t dp_col = tmem + lane_off + L::kColDP;
-    const float scale_log2 = p.f.scale_log2;
-    const float bias_mul = kLog2e / p.f.scale_log2;
-    uint32_t pit = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const BUnit w = bwd_unit(p, u);
-      if (w.n_pairs == 0) continue;
-      const int k0 = w.kt * kTile;
-      PairWalk pw;
-      pw.begin(p, w);
-      for (int i = 0; i < w.n_pairs && ok; ++i, pw.next(p, w)) {
-        bool partial;
-        const int qt = pw.qtile(p, w, &partial);
-        const int h = pw.head(w);
-        const int q = qt * kTile + r;
-        const bool row_valid = q < w.lq;
-        float neg_lse2 = -INFINITY, drow = 0.f;
-        if (row_valid) {
-          const float l = p.f.lse[qrow(p, w, h, q)];
-          neg_lse2 = l == -INFINITY ? -INFINITY : -l * kLog2e;
-          drow = p.dvec[qrow(p, w, h, q)];
-        }
-        const bool live = row_valid && neg_lse2 != -INFINITY;
-        // per-row mask parameters (as in the forward)
-        int clo = 0, chi = 0, dlo = 0, dhi = 0, lim = kTile;
-        const uint8_t* mrow = nullptr;
-        const uint8_t* brow = nullptr;
-        if (POLICY == kPolicyDflash) {
-          if (row_valid) {
-            const int j = q / p.f.bs, ii = q - j * p.f.bs;
-            int a = p.f.anchors[static_cast<int64_t>(w.b) * p.f.N + j];
-            a = a < 0 ? 0 : (a > p.f.Lc ? p.f.Lc : a);
-            chi = a;
-            clo = p.f.window > 0 ? max(0, a + ii - p.f.window + 1) : 0;
-            if (clo > chi) clo = chi;
-            const int base = p.f.Lc + j * p.f.bs;
-            dlo = base + (p.f.window > 0 ? max(0, ii - p.f.window + 1) : 0);
-            dhi = base + (p.f.causal_in_block ? ii + 1 : p.f.bs);
-          }
-        } else {
-          const int qq = row_valid ? q : 0;
-          if (p.f.has_mask) {
-            const int hm = p.f.mask.head_per_query ? h : w.hk;
-            mrow = reinterpret_cast<const uint8_t*>(p.f.mask.ptr) + w.b * p.f.mask.sb +
-                   hm * p.f.mask.sh + static_cast<int64_t>(qq) * p.f.mask.sq;
-          }
-          if (p.f.has_bias) {
-            const int hb = p.f.bias.head_per_query ? h : w.hk;
-            const int esz = p.f.bias.dtype == SMA_FP32 ? 4 : 2;
-            brow = reinterpret_cast<const uint8_t*>(p.f.bias.ptr) +
-                   (w.b * p.f.bias.sb + hb * p.f.bias.sh + static_cast<int64_t>(qq) * p.f.bias.sq) * esz;
-          }
-          if (k0 + kTile > w.lk) lim = min(lim, w.lk - k0);
-          if (p.f.causal) lim = min(lim, q + w.lk - w.lq - k0 + 1);
-        }
-
-        // ---- phase A: P from S
-        if (!mbar_wait(bar(L::kSFull), pit & 1, abort_flag, p.f.err)) { ok = false; break; }
-        if (pit > 0 && !mbar_wait(bar(L::kPFree), (pit - 1) & 1, abort_flag, p.f.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < kTile / 32; ++c) {
-          uint32_t xr[32];
-          tmem_ld32_at(s_col + 32 * c, xr);
-          tc_wait_ld();
-          float x[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(xr[e]);
-          if (POLICY != kPolicyDflash && p.f.has_bias) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              x[e] = fmaf(load_any_as_float(brow, p.f.bias.dtype, aux_col(k0 + 32 * c + e, p.f.bias.kd)),
-                          bias_mul, x[e]);
-          }
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pv[2];
-#pragma unroll
-            for (int z = 0; z < 2; ++z) {
-              const int cc = 32 * c + e + z;
-              bool keep = live;
-              if (partial) {
-                if (POLICY == kPolicyDflash) {
-                  const int k = k0 + cc;
-                  keep = keep && ((k >= clo && k < chi) || (k >= dlo && k < dhi));
-                } else {
-                  keep = keep && cc < lim && (!p.f.has_mask || mrow[aux_col(k0 + cc, p.f.mask.kd)] != 0);
-                }
-              }
-              pv[z] = keep ? fast_exp2(fmaf(x[e + z], scale_log2, neg_lse2)) : 0.f;
-            }
-            pk[e >> 1] = DT == SMA_BF16 ? pack_bf16x2(pv[0], pv[1]) : pack_f16x2(pv[0], pv[1]);
-          }
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            st_shared_v4(sw128_unit(sbase + L::kP, r, 4 * c + v4), pk[4 * v4], pk[4 * v4 + 1],
-                         pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        }
-        fence_async_shared();
-        tc_fence_before();
-        mbar_arrive(bar(L::kPDone));
-
-        // ---- phase B: dS = P (dP - D)
-        if (!mbar_wait(bar(L::kDPFull), pit & 1, abort_flag, p.f.err)) { ok = false; break; }
-        if (pit > 0 && !mbar_wait(bar(L::kDSFree), (pit - 1) & 1, abort_flag, p.f.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // dbias: this thread's query row of dS over the tile's 128 keys (the
-        // fixed-order mode: the warp's row q / 32 of the partial buffer, if
-        // that group of 32 queries starts inside the query length)
-        float* dbrow = nullptr;
-        if (POLICY != kPolicyDflash && p.db_mode != kDbiasNone) {
-          const int64_t qrow = p.db_mode == kDbiasGroupStore ? (q >> 5) : (row_valid ? q : 0);
-          if (p.db_mode != kDbiasGroupStore || (q >> 5) * 32 < p.f.Lq)
-            dbrow = p.dbias + w.b * p.db_sb + (p.db_head_per_query ? h : w.hk) * p.db_sh +
-                    qrow * p.db_sq + k0;
-        }
-        auto phase_b = [&](auto mode_tag) {
-          constexpr int MODE = decltype(mode_tag)::value;
-#pragma unroll
-          for (int c = 0; c < kTile / 32; ++c) {
-            uint32_t yr[32];
-            tmem_ld32_at(dp_col + 32 * c, yr);
-            tc_wait_ld();
-            uint32_t pk[16];
-            float dsv[32];
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
-              const uint4 pp = ld_shared_v4(sw128_unit(sbase + L::kP, r, 4 * c + v4));
-              const uint32_t pw4[4] = {pp.x, pp.y, pp.z, pp.w};
-#pragma unroll
-              for (int z = 0; z < 4; ++z) {
-                const int e = 8 * v4 + 2 * z;
-                const float2 pf = unpack2<DT>(pw4[z]);
-                const float d0 = pf.x * (__uint_as_float(yr[e]) - drow);
-                const float d1 = pf.y * (__uint_as_float(yr[e + 1]) - drow);
-                pk[4 * v4 + z] = DT == SMA_BF16 ? pack_bf16x2(d0, d1) : pack_f16x2(d0, d1);
-                dsv[e] = d0;
-                dsv[e + 1] = d1;
-              }
-            }
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              st_shared_v4(sw128_unit(sbase + L::kDS, r, 4 * c + v4), pk[4 * v4], pk[4 * v4 + 1],
-                           pk[4 * v4 + 2], pk[4 * v4 + 3]);
-            if (MODE == kDbiasStore || MODE == kDbiasAdd) {
-              if (row_valid && k0 + kTile <= p.db_kd && p.db_kd % 4 == 0) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  const float4 v =
-                      make_float4(dsv[4 * j], dsv[4 * j + 1], dsv[4 * j + 2], dsv[4 * j + 3]);
-                  float4* dst = reinterpret_cast<float4*>(dbrow + 32 * c + 4 * j);
-                  if (MODE == kDbiasStore) *dst = v;
-                  else atomicAdd(dst, v);
-                }
-              } else if (row_valid) {  // a dbias row of Lk columns: element by element, inside it
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                  if (k0 + 32 * c + e < p.db_kd) {
-                    if (MODE == kDbiasStore) dbrow[32 * c + e] = dsv[e];
-                    else atomicAdd(dbrow + 32 * c + e, dsv[e]);
-                  }
-                }
-              }
-            } else if (MODE == kDbiasRowSum || MODE == kDbiasGroupStore) {
-              // Column sums over the warp's 32 query rows (rows past Lq hold
-              // 0): halving exchanges, after which lane l holds column l.
-#pragma unroll
-              for (int wd = 16; wd >= 1; wd >>= 1) {
-                const bool upper = (lane & wd) != 0;
-#pragma unroll
-                for (int i = 0; i < wd; ++i) {
-                  const float send = upper ? dsv[i] : dsv[i + wd];
-                  const float keep = upper ? dsv[i + wd] : dsv[i];
-                  dsv[i] = keep + __shfl_xor_sync(0xffffffffu, send, wd);
-                }
-              }
-              if (k0 + 32 * c + lane < p.db_kd) {
-                if (MODE == kDbiasRowSum) atomicAdd(dbrow + 32 * c + lane, dsv[0]);
-                else if (dbrow != nullptr) dbrow[32 * c + lane] = dsv[0];
-              }
-            }
-          }
-        };
-        if (POLICY == kPolicyDflash || p.db_mode == kDbiasNone)
-          phase_b(std::integral_constant<int, kDbiasNone>{});
-        else if (p.db_mode == kDbiasStore)
-          phase_b(std::integral_constant<int, kDbiasStore>{});
-        else if (p.db_mode == kDbiasAdd)
-          phase_b(std::integral_constant<int, kDbiasAdd>{});
-        else if (p.db_mode == kDbiasGroupStore)
-          phase_b(std::integral_constant<int, kDbiasGroupStore>{});
-        else
-          phase_b(std::integral_constant<int, kDbiasRowSum>{});
-        fence_async_shared();
-        tc_fence_before();
-        mbar_arrive(bar(L::kDSDone));
-        ++pit;
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ dQ drain, dK / dV epilogue
-    const int wq = warp - 4;
-    const int r = wq * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t dq_col = tmem + lane_off + L::kColDP;
-    const uint32_t dv_col = tmem + lane_off + L::kColDV;
-    const uint32_t dk_col = tmem + lane_off + L::kColDK;
-    typedef typename std::conditional<DT == SMA_BF16, __nv_bfloat16, __half>::type OutT;
-    uint32_t pit = 0, uit = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const BUnit w = bwd_unit(p, u);
-      const int key = w.kt * kTile + r;
-      OutT* dvrow = reinterpret_cast<OutT*>(p.dv) + w.bt * p.dv_sb + static_cast<int64_t>(w.k_off + key) * p.dv_sr +
-                    w.hk * p.dv_sh;
-      OutT* dkrow = reinterpret_cast<OutT*>(p.dk) + w.bt * p.dk_sb + static_cast<int64_t>(w.k_off + key) * p.dk_sr +
-                    w.hk * p.dk_sh;
-      if (w.n_pairs == 0) {  // keys no query attends: zero gradients
-        if (key < w.lk) {
-          for (int e = 0; e < D / 8; ++e) {
-            reinterpret_cast<uint4*>(dvrow)[e] = make_uint4(0, 0, 0, 0);
-            reinterpret_cast<uint4*>(dkrow)[e] = make_uint4(0, 0, 0, 0);
-          }
-        }
-        continue;
-      }
-      PairWalk pw;
-      pw.begin(p, w);
-      for (int i = 0; i < w.n_pairs && ok; ++i, pw.next(p, w)) {
-        bool partial;
-        const int qt = pw.qtile(p, w, &partial);
-        const int h = pw.head(w);
-        const int q = qt * kTile + r;
-        if (!mbar_wait(bar(L::kDQFull), pit & 1, abort_flag, p.f.err)) { ok = false; break; }
-        tc_fence_after();
-        float4* acc = reinterpret_cast<float4*>(
-            p.dq_acc + ((static_cast<int64_t>(w.bt) * (p.f.cu_q != nullptr ? p.f.total_q : p.f.Lq) +
-                         w.q_off + q) * p.f.H + h) * D);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32_at(dq_col + 32 * c, v);
-          tc_wait_ld();
-          if (c == D / 32 - 1) {
-            tc_fence_before();
-            mbar_arrive(bar(L::kDQFree));
-          }
-          if (q < w.lq) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              atomicAdd(acc + 8 * c + e,
-                        make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                    __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
-          }
-        }
-        ++pit;
-      }
-      if (!ok) break;
-      if (!mbar_wait(bar(L::kAccDone), uit & 1, abort_flag, p.f.err)) { ok = false; break; }
-      tc_fence_after();
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which == 0 ? dv_col : dk_col;
-        const float mul = which == 0 ? 1.f : p.scale;
-        OutT* dst = which == 0 ? dvrow : dkrow;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32_at(col + 32 * c, v);
-          tc_wait_ld();
-          if (key < w.lk) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float a = __uint_as_float(v[2 * e]) * mul;
-              const float bq = __uint_as_float(v[2 * e + 1]) * mul;
-              pk[e] = DT == SMA_BF16 ? pack_bf16x2(a, bq) : pack_f16x2(a, bq);
-            }
-            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(bar(L::kAccFree));
-      ++uit;
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == kBMmaWarp) tmem_dealloc(tmem, kBTmemCols);
-}
-
-
 // ---------------------------------------------------------------------------
-// Head dim 128: the transposed form.  The compute threads own key rows:
+// The transposed form (head dim 64 or 128).  The compute threads own key rows:
 //   S^T  = K Q^T        A = K (K-major)        B = Q (K-major)        SS
 //   dP^T = V dO^T       A = V (K-major)        B = dO (K-major)       SS
 //   dV  += P^T dO       A = P^T from TMEM      B = dO (MN-major)      TS
@@ -813,16 +208,18 @@ constexpr int kTCtrlRegs = 112;
 static_assert(256 * kTLaunchRegs + 128 * kTDrainRegs + 128 * kTCtrlRegs <= kBwdTThreads * kTLaunchRegs,
               "register split must fit the launch allocation");
 
+template <int D_>
 struct TLayout {
-  static constexpr int D = 128;
+  static constexpr int D = D_;
+  static constexpr int kChunks = D / 64;              // 128-byte-swizzled column chunks of a tile
   static constexpr uint32_t kChunk = kTile * 128;
   static constexpr uint32_t kTileD = kTile * D * 2;
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = kK + kTileD;
   static constexpr uint32_t kQ = kV + kTileD;        // 2 stages
   static constexpr uint32_t kDO = kQ + 2 * kTileD;   // 1 stage
-  static constexpr uint32_t kDS = kDO + kTileD;      // dS^T [key][query]
-  static constexpr uint32_t kAux = kDS + kTileD;     // 2 stages of kAuxBytes
+  static constexpr uint32_t kDS = kDO + kTileD;      // dS^T [key][query], 128 x 128 at any D
+  static constexpr uint32_t kAux = kDS + kTile * kTile * 2;  // 2 stages of kAuxBytes
   static constexpr uint32_t kAuxBytes = 6 * kTile * 4;  // nl, dd, clo, chi, dlo, dhi
   // dQ staging for the bulk reductions: per drain warp 32 rows x 32 floats
   static constexpr uint32_t kStage = (kAux + 2 * kAuxBytes + 1023) / 1024 * 1024;
@@ -849,14 +246,13 @@ __host__ __device__ constexpr uint32_t pcol(int q) {
   return static_cast<uint32_t>((q & ~63) + (q & 63) / 2);
 }
 
-template <int POLICY, int DT>
+template <int D, int POLICY, int DT>
 __global__ void __launch_bounds__(kBwdTThreads, 1)
 attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
                   const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                   const __grid_constant__ CUtensorMap map_do, const __grid_constant__ CUtensorMap map_dq,
                   int n_units) {
-  using L = TLayout;
-  constexpr int D = L::D;
+  using L = TLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned by offsetting the shared array itself, so that pointers
   // derived from it keep the shared state space (shared loads, not generic)
@@ -928,7 +324,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
       }
       if (elect_one()) {
         mbar_arrive_expect_tx(bar(L::kKVFull), 2 * L::kTileD);
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < L::kChunks; ++c) {
           tma_load_4d(sbase + L::kK + c * L::kChunk, &map_k, bar(L::kKVFull), c * 64, w.hk,
                       w.k_off + w.kt * kTile, w.bt);
           tma_load_4d(sbase + L::kV + c * L::kChunk, &map_v, bar(L::kKVFull), c * 64, w.hk,
@@ -951,7 +347,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         }
         if (elect_one()) {
           mbar_arrive_expect_tx(bar(L::kQFull + s), L::kTileD);
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sbase + L::kQ + s * L::kTileD + c * L::kChunk, &map_q, bar(L::kQFull + s),
                         c * 64, h, w.q_off + qt * kTile, w.bt);
         }
@@ -963,7 +359,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         }
         if (elect_one()) {
           mbar_arrive_expect_tx(bar(L::kOFull), L::kTileD);
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sbase + L::kDO + c * L::kChunk, &map_do, bar(L::kOFull), c * 64, h,
                         w.q_off + qt * kTile, w.bt);
         }
@@ -1504,11 +900,11 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
   if (warp == kTMmaWarp) tmem_dealloc(tmem, kBTmemCols);
 }
 
-template <int POLICY, int DT>
+template <int D, int POLICY, int DT>
 cudaError_t launch_bwd_t(const BwdProblem& p, const CUtensorMap& mq, const CUtensorMap& mk,
                          const CUtensorMap& mv, const CUtensorMap& mdo, const CUtensorMap& mdq,
                          cudaStream_t stream) {
-  auto kern = attn_bwd_t_kernel<POLICY, DT>;
+  auto kern = attn_bwd_t_kernel<D, POLICY, DT>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaFuncAttributes fa;
@@ -1517,14 +913,14 @@ cudaError_t launch_bwd_t(const BwdProblem& p, const CUtensorMap& mq, const CUten
     // The setmaxnreg split assumes exactly kTLaunchRegs registers per thread.
     if (fa.numRegs != kTLaunchRegs) return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(TLayout::kAlloc));
+                             static_cast<int>(TLayout<D>::kAlloc));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int n_units = p.f.B * p.f.KVH * p.f.KT;
   if (n_units == 0) return cudaSuccess;
   const int grid = n_units < num_sms() ? n_units : num_sms();
-  kern<<<grid, kBwdTThreads, TLayout::kAlloc, stream>>>(p, mq, mk, mv, mdo, mdq, n_units);
+  kern<<<grid, kBwdTThreads, TLayout<D>::kAlloc, stream>>>(p, mq, mk, mv, mdo, mdq, n_units);
   return cudaGetLastError();
 }
 
@@ -1645,25 +1041,6 @@ __global__ void dq_convert_kernel(const BwdProblem p) {
   }
 }
 
-template <int D, int POLICY, int DT>
-cudaError_t launch_bwd_typed(const BwdProblem& p, const CUtensorMap& mq, const CUtensorMap& mk,
-                             const CUtensorMap& mv, const CUtensorMap& mdo, cudaStream_t stream) {
-  using L = BLayout<D>;
-  auto kern = attn_bwd_kernel<D, POLICY, DT>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(L::kAlloc));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  const int n_units = p.f.B * p.f.KVH * p.f.KT;
-  if (n_units == 0) return cudaSuccess;
-  const int grid = n_units < num_sms() ? n_units : num_sms();
-  kern<<<grid, kBwdThreads, L::kAlloc, stream>>>(p, mq, mk, mv, mdo, n_units);
-  return cudaGetLastError();
-}
-
 }  // namespace
 
 // Packed batches are one batch entry of total_q rows for the row-wise kernels
@@ -1765,20 +1142,19 @@ int launch_attn_bwd(const BwdProblem& p, cudaStream_t stream, char* msg, size_t 
       !encode_map(&mdo, p.dout, f.dtype, f.d, f.H, lq, nb, p.do_sh, p.do_sr, p.do_sb, msg, msg_len))
     return SMA_ERR_CUDA;
   CUtensorMap mdq;
-  if (f.d == 128 && !encode_map_f32(&mdq, p.dq_acc, f.d, f.H, lq, nb, 32, 32, msg, msg_len))
-    return SMA_ERR_CUDA;
+  if (!encode_map_f32(&mdq, p.dq_acc, f.d, f.H, lq, nb, 32, 32, msg, msg_len)) return SMA_ERR_CUDA;
   cudaError_t e = cudaErrorInvalidValue;
   const bool bf = f.dtype == SMA_BF16;
   if (f.policy == kPolicyDflash) {
-    if (f.d == 128) e = bf ? launch_bwd_t<kPolicyDflash, SMA_BF16>(p, mq, mk, mv, mdo, mdq, stream)
-                           : launch_bwd_t<kPolicyDflash, SMA_FP16>(p, mq, mk, mv, mdo, mdq, stream);
-    else e = bf ? launch_bwd_typed<64, kPolicyDflash, SMA_BF16>(p, mq, mk, mv, mdo, stream)
-                : launch_bwd_typed<64, kPolicyDflash, SMA_FP16>(p, mq, mk, mv, mdo, stream);
+    if (f.d == 128) e = bf ? launch_bwd_t<128, kPolicyDflash, SMA_BF16>(p, mq, mk, mv, mdo, mdq, stream)
+                           : launch_bwd_t<128, kPolicyDflash, SMA_FP16>(p, mq, mk, mv, mdo, mdq, stream);
+    else e = bf ? launch_bwd_t<64, kPolicyDflash, SMA_BF16>(p, mq, mk, mv, mdo, mdq, stream)
+                : launch_bwd_t<64, kPolicyDflash, SMA_FP16>(p, mq, mk, mv, mdo, mdq, stream);
   } else {
-    if (f.d == 128) e = bf ? launch_bwd_t<kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, mdo, mdq, stream)
-                           : launch_bwd_t<kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, mdo, mdq, stream);
-    else e = bf ? launch_bwd_typed<64, kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, mdo, stream)
-                : launch_bwd_typed<64, kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, mdo, stream);
+    if (f.d == 128) e = bf ? launch_bwd_t<128, kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, mdo, mdq, stream)
+                           : launch_bwd_t<128, kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, mdo, mdq, stream);
+    else e = bf ? launch_bwd_t<64, kPolicyExplicit, SMA_BF16>(p, mq, mk, mv, mdo, mdq, stream)
+                : launch_bwd_t<64, kPolicyExplicit, SMA_FP16>(p, mq, mk, mv, mdo, mdq, stream);
   }
   if (e != cudaSuccess) {
     snprintf(msg, msg_len, "attention backward launch failed: %s", cudaGetErrorString(e));

@@ -203,10 +203,9 @@ __device__ __forceinline__ int64_t row_index(const AttnProblem& p, int b, int h,
 // partial buffer (every partial element has exactly one writer).
 enum DbiasMode { kDbiasNone = 0, kDbiasStore = 1, kDbiasAdd = 2, kDbiasRowSum = 3,
                  kDbiasGroupStore = 4 };
-// Query rows summed per partial row by the tensor-core backward kernels:
-// the transposed kernel (head dim 128) sums each thread's 64 queries, the
-// head-dim-64 kernel each warp's 32.
-constexpr int dbias_group_rows(int head_dim) { return head_dim == 128 ? 64 : 32; }
+// Query rows summed per partial row by the tensor-core backward kernel (the
+// transposed kernel, both head dims): each thread's 64 queries.
+constexpr int dbias_group_rows(int) { return 64; }
 
 // Single-query (decode) problem after the grouped-head swap: for each
 // (b, kv head) the `group` query heads are the rows.

@@ -339,15 +339,15 @@ def test_sparse_workspace_includes_key_range_segments_for_short_queries():
 
 
 def test_deterministic_dbias_workspace_query():
-    """Partial rows per (batch, head): query groups of 64 (head dim 128) or
-    32 (64) for a query-broadcast bias, every query for a bias with a query
-    dim or fp32 operands; nothing when each dbias element has one writer."""
+    """Partial rows per (batch, head): query groups of 64 (either head dim)
+    for a query-broadcast bias, every query for a bias with a query dim or
+    fp32 operands; nothing when each dbias element has one writer."""
     lib = nat.load()
     n = ctypes.c_size_t()
     q = lambda dt, hd, shape: lib.masked_attn_bwd_dbias_workspace_size(  # noqa: E731
         dt, 4, 16, 8, 1000, hd, nat.i64_array(shape), ctypes.byref(n))
     assert q(nat.SMA_BF16, 128, [4, 8, 1, 1024]) == 0 and n.value == 4 * 16 * 16 * 1024 * 4
-    assert q(nat.SMA_BF16, 64, [1, 1, 1, 1000]) == 0 and n.value == 4 * 16 * 32 * 1000 * 4
+    assert q(nat.SMA_BF16, 64, [1, 1, 1, 1000]) == 0 and n.value == 4 * 16 * 16 * 1000 * 4
     assert q(nat.SMA_FP32, 64, [1, 1, 1, 1000]) == 0 and n.value == 4 * 16 * 1000 * 1000 * 4
     assert q(nat.SMA_BF16, 128, [1, 8, 1000, 1024]) == 0 and n.value == 4 * 16 * 1000 * 1024 * 4
     assert q(nat.SMA_BF16, 128, [4, 16, 1000, 1024]) == 0 and n.value == 0
