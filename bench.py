@@ -166,8 +166,9 @@ def kernel_source_sha256() -> str:
 
 
 def measured_traffic(workload_name: str):
-    """(bytes per launch, profile file) from profiles/attn_tc_<workload>_traffic.md
-    if it was captured on the current kernel sources, else (None, reason)."""
+    """(bytes per launch, summary path) from the committed ncu traffic summary
+    of the workload's attention launch, if it was captured on the current
+    kernel sources, else (None, reason)."""
     path = os.path.join(ROOT, "profiles", f"attn_tc_{workload_name}_traffic.md")
     if not os.path.exists(path):
         return None, "no ncu traffic summary for this workload"
