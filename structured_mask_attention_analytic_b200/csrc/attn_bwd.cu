@@ -169,10 +169,14 @@ __device__ __forceinline__ float2 unpack2(uint32_t w) {
 // read MN-major it is dS itself (queries contiguous), so dQ comes out with
 // query rows in TMEM.
 // That halves the operand traffic the products and the compute threads put
-// on shared memory.  Two 128-column TMEM regions alternate between pairs:
-// pair i puts S^T / P^T and later dQ in region X_i, dP^T in Y_i; pair i+1
-// swaps them, so S^T(i+1) is issued as soon as dS^T(i) is formed (ahead of
-// dK(i) and dQ(i)), and dP^T(i+1) once dQ(i) has been drained.
+// on shared memory.  Two 128-column TMEM regions X alternate between pairs:
+// pair i puts S^T / P^T and later dQ in region X_i, dP^T in Y_i.  At head
+// dim 128 (dV and dK take the other 256 columns) Y_i is X_{i+1}: S^T(i+1)
+// is issued as soon as dS^T(i) is formed (ahead of dK(i) and dQ(i)), and
+// dP^T(i+1) once dQ(i) has been drained.  At head dim 64 dV and dK take 128
+// columns and Y has the last 128 of its own: S^T(i+1) is issued once dQ(i-1)
+// has left X_{i+1} (while pair i is still forming P^T and dS^T), and
+// dP^T(i+1) once dS^T(i) is formed.
 // The producer stages, per pair, -lse * log2(e) and rowsum(dO * O) of the
 // 128 queries (and, for DFlash, each query's kept key intervals) in shared
 // memory next to the Q stage.
@@ -227,14 +231,20 @@ struct TLayout {
   static constexpr uint32_t kBars = kStage + 4 * kStageWarp;
   enum : int {
     kKVFull = 0, kKVEmpty, kQFull, kQEmpty = kQFull + 2, kAuxFull = kQEmpty + 2,
-    kOFull = kAuxFull + 2, kOEmpty, kSFull, kPDone, kDPFull, kDSDone, kDQFull, kDQFree, kDSFree,
+    kOFull = kAuxFull + 2, kOEmpty, kSFull, kSFull1, kPDone, kDPFull, kDSDone, kDQFull, kDQFree, kDSFree,
     kAccDone, kAccFree, kDrain, kNumBars
   };
   static constexpr uint32_t kTmemSlot = kBars + 8 * kNumBars;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kBytes = kAbort + 4;
   static constexpr uint32_t kAlloc = kBytes + 1024;
-  static constexpr uint32_t kColDV = 256, kColDK = 384;
+  // TMEM: S^T / P^T / dQ regions X at columns 0 and 128 (alternating by
+  // pair), dV and dK accumulators, and dP^T in Y.  At head dim 128 the four
+  // 128-column regions fill TMEM and Y is the other X region; at head dim 64
+  // dV and dK take 64 columns each and Y has a region of its own (columns
+  // 384-511), so S^T of the next pair can go in while this pair is in flight.
+  static constexpr bool kOwnY = D == 64;
+  static constexpr uint32_t kColDV = 256, kColDK = D == 64 ? 320 : 384, kColY = 384;
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
@@ -281,6 +291,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     mbar_init(bar(L::kOFull), 1);
     mbar_init(bar(L::kOEmpty), 1);
     mbar_init(bar(L::kSFull), 1);
+    mbar_init(bar(L::kSFull1), 1);
     mbar_init(bar(L::kPDone), 256);
     mbar_init(bar(L::kDPFull), 1);
     mbar_init(bar(L::kDSDone), 256);
@@ -508,21 +519,24 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
       if (!wait(L::kKVFull, kv_it & 1)) break;
       ++kv_it;
       {  // S^T(0), dP^T(0)
-        const uint32_t X = (pit & 1) ? 128u : 0u, Y = 128u - X;
+        const uint32_t X = (pit & 1) ? 128u : 0u, Y = L::kOwnY ? L::kColY : 128u - X;
         if (!wait(L::kQFull + (q_it & 1), (q_it >> 1) & 1)) break;
         if (!wait(L::kOFull, o_it & 1)) break;
-        if (pit > 0 && !wait(L::kDQFree, (pit - 1) & 1)) break;  // Y held dQ of the last pair
+        // Head dim 128: Y held dQ of the last pair.  Own Y: X held dQ two
+        // pairs back, waited for during the last pair.
+        if (!L::kOwnY && pit > 0 && !wait(L::kDQFree, (pit - 1) & 1)) break;
         tc_fence_after();
         if (elect_one()) {
           issue_st_dpt(X, Y, sbase + L::kQ + (q_it & 1) * L::kTileD);
-          tc_commit(bar(L::kSFull));
+          tc_commit(bar(L::kSFull + (pit & 1)));
           tc_commit(bar(L::kDPFull));
         }
         __syncwarp();
       }
       for (int i = 0; i < n && ok; ++i) {
-        const uint32_t X = (pit & 1) ? 128u : 0u, Y = 128u - X;
+        const uint32_t X = (pit & 1) ? 128u : 0u, Y = L::kOwnY ? L::kColY : 128u - X;
         const int qs = q_it & 1;
+        const uint32_t nq = q_it + 1;
         // dV += P^T dO
         if (!wait(L::kPDone, pit & 1)) break;
         if (i == 0 && uit > 0 && !wait(L::kAccFree, (uit - 1) & 1)) break;
@@ -533,16 +547,32 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         }
         __syncwarp();
         ++o_it;
-        // dS^T(i) is formed: Y is free (dP^T(i) consumed), so S^T(i+1) goes
-        // first, then dK += dS^T Q and dQ = dS K (into X, after dV read P^T)
+        if (L::kOwnY) {
+          // S^T(i+1) into the other X region as soon as dQ(i-1) has left it,
+          // while this pair's dS^T is still being formed.  The wait is taken
+          // after a unit's last pair too, so that a unit's first pair finds
+          // its X region free.
+          if (pit > 0 && !wait(L::kDQFree, (pit - 1) & 1)) break;
+          if (i + 1 < n) {
+            if (!wait(L::kQFull + (nq & 1), (nq >> 1) & 1)) break;
+            tc_fence_after();
+            if (elect_one()) {
+              issue_t(128u - X, sbase + L::kK, sbase + L::kQ + (nq & 1) * L::kTileD);
+              tc_commit(bar(L::kSFull + ((pit + 1) & 1)));
+            }
+            __syncwarp();
+          }
+        }
+        // dS^T(i) is formed.  Head dim 128: Y is free (dP^T(i) consumed), so
+        // S^T(i+1) goes there first.  Then dK += dS^T Q and dQ = dS K (into
+        // X, after dV read P^T).
         if (!wait(L::kDSDone, pit & 1)) break;
-        const uint32_t nq = q_it + 1;
-        if (i + 1 < n && !wait(L::kQFull + (nq & 1), (nq >> 1) & 1)) break;
+        if (!L::kOwnY && i + 1 < n && !wait(L::kQFull + (nq & 1), (nq >> 1) & 1)) break;
         tc_fence_after();
         if (elect_one()) {
-          if (i + 1 < n) {
+          if (!L::kOwnY && i + 1 < n) {
             issue_t(Y, sbase + L::kK, sbase + L::kQ + (nq & 1) * L::kTileD);
-            tc_commit(bar(L::kSFull));
+            tc_commit(bar(L::kSFull + ((pit + 1) & 1)));
           }
           issue_dk_dq(X, sbase + L::kQ + qs * L::kTileD, i > 0);
           tc_commit(bar(L::kDQFull));
@@ -553,12 +583,13 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         ++q_it;
         ++pit;
         if (i + 1 < n) {
-          // dP^T(i+1) into X once dQ(i) is drained
+          // dP^T(i+1): head dim 128 into X once dQ(i) is drained (pair i+1's
+          // Y); own Y once dP^T(i) is consumed (dS^T(i) formed, above)
           if (!wait(L::kOFull, o_it & 1)) break;
-          if (!wait(L::kDQFree, (pit - 1) & 1)) break;
+          if (!L::kOwnY && !wait(L::kDQFree, (pit - 1) & 1)) break;
           tc_fence_after();
           if (elect_one()) {
-            issue_t(X, sbase + L::kV, sbase + L::kDO);
+            issue_t(L::kOwnY ? L::kColY : X, sbase + L::kV, sbase + L::kDO);
             tc_commit(bar(L::kDPFull));
           }
           __syncwarp();
@@ -599,7 +630,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         const int qt = pw.qtile(p, w, &partial);
         const int h = pw.head(w);
         const int q0 = qt * kTile;
-        const uint32_t X = (pit & 1) ? 128u : 0u, Y = 128u - X;
+        const uint32_t X = (pit & 1) ? 128u : 0u, Y = L::kOwnY ? L::kColY : 128u - X;
         const uint32_t xcol = tmem + lane_off + X, ycol = tmem + lane_off + Y;
         const int s = q_it & 1;
         const float* nl = aux_f(s, 0);
@@ -626,7 +657,8 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           }
         }
         if (!mbar_wait(bar(L::kAuxFull + s), (q_it >> 1) & 1, abort_flag, p.f.err)) { ok = false; break; }
-        if (!mbar_wait(bar(L::kSFull), pit & 1, abort_flag, p.f.err)) { ok = false; break; }
+        // S^T of pair pit completes SFull + (pit & 1) (one barrier per X region)
+        if (!mbar_wait(bar(L::kSFull + (pit & 1)), (pit >> 1) & 1, abort_flag, p.f.err)) { ok = false; break; }
         tc_fence_after();
         // ---- phase A: P^T = exp2(S^T * scale * log2 e - lse * log2 e), packed into X
         // FULL and PARTIAL pairs run separate copies of the loop, so that a
