@@ -161,15 +161,16 @@ __device__ __forceinline__ float2 unpack2(uint32_t w) {
 //   S^T  = K Q^T        A = K (K-major)        B = Q (K-major)        SS
 //   dP^T = V dO^T       A = V (K-major)        B = dO (K-major)       SS
 //   dV  += P^T dO       A = P^T from TMEM      B = dO (MN-major)      TS
-//   dK  += dS^T Q       A = dS^T (K-major)     B = Q (MN-major)       SS
+//   dK  += dS^T Q       A = dS^T from TMEM     B = Q (MN-major)       TS
 //   dQ   = dS K         A = dS (MN-major)      B = K (MN-major)       SS
 // P^T goes to TMEM as packed 16-bit pairs over S^T's columns (pcol below),
-// as the forward's P does, so dV reads its A operand from TMEM.
-// dS^T is written to shared memory only: read K-major it is dK's A operand,
-// read MN-major it is dS itself (queries contiguous), so dQ comes out with
-// query rows in TMEM.
-// That halves the operand traffic the products and the compute threads put
-// on shared memory.  Two 128-column TMEM regions X alternate between pairs:
+// as the forward's P does, so dV reads its A operand from TMEM; dS^T is
+// packed beside it (dscol) for dK.  dS^T is also written once to shared
+// memory, where read MN-major it is dS itself (queries contiguous), so dQ
+// comes out with query rows in TMEM.  Shared-memory bandwidth is what binds
+// this kernel at head dim 128 (the products read 8 KB of operands per
+// 128x128x16 step from it), so operands come from TMEM wherever the layout
+// allows.  Two 128-column TMEM regions X alternate between pairs:
 // pair i puts S^T / P^T and later dQ in region X_i, dP^T in Y_i.  At head
 // dim 128 (dV and dK take the other 256 columns) Y_i is X_{i+1}: S^T(i+1)
 // is issued as soon as dS^T(i) is formed (ahead of dK(i) and dQ(i)), and
@@ -255,6 +256,10 @@ struct TLayout {
 __host__ __device__ constexpr uint32_t pcol(int q) {
   return static_cast<uint32_t>((q & ~63) + (q & 63) / 2);
 }
+// Packed dS^T column of query column q: the other half of the same 64
+// columns (queries 0-63 -> columns 32-63, queries 64-127 -> 96-127), again
+// written only by the thread that read them.
+__host__ __device__ constexpr uint32_t dscol(int q) { return pcol(q) + 32u; }
 
 template <int D, int POLICY, int DT>
 __global__ void __launch_bounds__(kBwdTThreads, 1)
@@ -490,19 +495,22 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         tc_mma_ts(tmem + dcol, tmem + acol + pcol(16 * s), with_lo(bd, (s * 2048) >> 4), idesc_ts,
                   (acc || s > 0) ? 1u : 0u);
     };
-    // dK += dS^T Q (A = the dS^T tile, K-major) interleaved with dQ = dS K
-    // (A = the same tile read MN-major: dS with queries contiguous)
+    // dK += dS^T Q (A = dS^T packed in TMEM beside P^T, queries 16 s ..
+    // 16 s + 15 at dscol(16 s)), then dQ = dS K (A = the dS^T tile in shared
+    // memory read MN-major: dS with queries contiguous).  dQ's first step
+    // overwrites all of X, so every dK step is issued before it: one
+    // thread's MMAs run in order.
     auto issue_dk_dq = [&](uint32_t xcol, uint32_t q_addr, bool acc) {
       const uint64_t qd = smem_desc_sw128(q_addr, L::kChunk, 1024);
       const uint64_t kd = smem_desc_sw128(sbase + L::kK, L::kChunk, 1024);
-      const uint64_t st = smem_desc_sw128(sbase + L::kDS, 16, 1024);
       const uint64_t sd = smem_desc_sw128(sbase + L::kDS, L::kChunk, 1024);
+#pragma unroll
+      for (int s = 0; s < kTile / 16; ++s)
+        tc_mma_ts(tmem + L::kColDK, tmem + xcol + dscol(16 * s), with_lo(qd, (s * 2048) >> 4), idesc_ts,
+                  (acc || s > 0) ? 1u : 0u);
 #pragma unroll
       for (int s = 0; s < kTile / 16; ++s) {
         const uint32_t off = (s * 2048) >> 4;
-        const uint32_t koff = ((s >> 2) * L::kChunk + (s & 3) * 32) >> 4;
-        tc_mma_ss(tmem + L::kColDK, with_lo(st, koff), with_lo(qd, off), idesc_ts,
-                  (acc || s > 0) ? 1u : 0u);
         tc_mma_ss(tmem + xcol, with_lo(sd, off), with_lo(kd, off), idesc_dq, s > 0 ? 1u : 0u);
       }
     };
@@ -800,6 +808,8 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
             for (int v4 = 0; v4 < 4; ++v4)
               st_shared_v4(sw128_unit(sbase + L::kDS, r, cq / 8 + v4), pk[4 * v4], pk[4 * v4 + 1],
                            pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            // and packed into X beside P^T: dK's A operand
+            tmem_st16_at(xcol + dscol(cq), pk);
           }
           if (MODE == kDbiasRowSum && db_key) atomicAdd(dbcol, rsum);
           if (MODE == kDbiasGroupStore && db_key && db_grp) dbcol[((q0 + qb) >> 6) * p.db_sq] = rsum;
@@ -815,6 +825,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         else
           phase_b(std::integral_constant<int, kDbiasRowSum>{});
         fence_async_shared();
+        tc_wait_st();
         tc_fence_before();
         mbar_arrive(bar(L::kDSDone));
         ++pit;
