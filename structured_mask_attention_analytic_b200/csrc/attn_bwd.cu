@@ -173,8 +173,9 @@ __device__ __forceinline__ float2 unpack2(uint32_t w) {
 // allows.  Two 128-column TMEM regions X alternate between pairs:
 // pair i puts S^T / P^T and later dQ in region X_i, dP^T in Y_i.  At head
 // dim 128 (dV and dK take the other 256 columns) Y_i is X_{i+1}: S^T(i+1)
-// is issued as soon as dS^T(i) is formed (ahead of dK(i) and dQ(i)), and
-// dP^T(i+1) once dQ(i) has been drained.  At head dim 64 dV and dK take 128
+// is issued as soon as the compute threads have read dP^T(i) into
+// registers (early in forming dS^T(i)), and dP^T(i+1) once dQ(i) has been
+// drained.  At head dim 64 dV and dK take 128
 // columns and Y has the last 128 of its own: S^T(i+1) is issued once dQ(i-1)
 // has left X_{i+1} (while pair i is still forming P^T and dS^T), and
 // dP^T(i+1) once dS^T(i) is formed.
@@ -232,7 +233,7 @@ struct TLayout {
   static constexpr uint32_t kBars = kStage + 4 * kStageWarp;
   enum : int {
     kKVFull = 0, kKVEmpty, kQFull, kQEmpty = kQFull + 2, kAuxFull = kQEmpty + 2,
-    kOFull = kAuxFull + 2, kOEmpty, kSFull, kSFull1, kPDone, kDPFull, kDSDone, kDQFull, kDQFree, kDSFree,
+    kOFull = kAuxFull + 2, kOEmpty, kSFull, kSFull1, kPDone, kDPFull, kDPRead, kDSDone, kDQFull, kDQFree, kDSFree,
     kAccDone, kAccFree, kDrain, kNumBars
   };
   static constexpr uint32_t kTmemSlot = kBars + 8 * kNumBars;
@@ -299,6 +300,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     mbar_init(bar(L::kSFull1), 1);
     mbar_init(bar(L::kPDone), 256);
     mbar_init(bar(L::kDPFull), 1);
+    mbar_init(bar(L::kDPRead), 256);
     mbar_init(bar(L::kDSDone), 256);
     mbar_init(bar(L::kDQFull), 1);
     mbar_init(bar(L::kDQFree), 128);
@@ -555,7 +557,20 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         }
         __syncwarp();
         ++o_it;
-        if (L::kOwnY) {
+        if (!L::kOwnY) {
+          // Head dim 128: Y is free once the compute threads have read
+          // dP^T(i), early in forming dS^T(i): S^T(i+1) goes there then.
+          if (!wait(L::kDPRead, pit & 1)) break;
+          if (i + 1 < n) {
+            if (!wait(L::kQFull + (nq & 1), (nq >> 1) & 1)) break;
+            tc_fence_after();
+            if (elect_one()) {
+              issue_t(Y, sbase + L::kK, sbase + L::kQ + (nq & 1) * L::kTileD);
+              tc_commit(bar(L::kSFull + ((pit + 1) & 1)));
+            }
+            __syncwarp();
+          }
+        } else {
           // S^T(i+1) into the other X region as soon as dQ(i-1) has left it,
           // while this pair's dS^T is still being formed.  The wait is taken
           // after a unit's last pair too, so that a unit's first pair finds
@@ -571,17 +586,11 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
             __syncwarp();
           }
         }
-        // dS^T(i) is formed.  Head dim 128: Y is free (dP^T(i) consumed), so
-        // S^T(i+1) goes there first.  Then dK += dS^T Q and dQ = dS K (into
-        // X, after dV read P^T).
+        // dS^T(i) is formed: dK += dS^T Q and dQ = dS K (into X, after dV
+        // read P^T)
         if (!wait(L::kDSDone, pit & 1)) break;
-        if (!L::kOwnY && i + 1 < n && !wait(L::kQFull + (nq & 1), (nq >> 1) & 1)) break;
         tc_fence_after();
         if (elect_one()) {
-          if (!L::kOwnY && i + 1 < n) {
-            issue_t(Y, sbase + L::kK, sbase + L::kQ + (nq & 1) * L::kTileD);
-            tc_commit(bar(L::kSFull + ((pit + 1) & 1)));
-          }
           issue_dk_dq(X, sbase + L::kQ + qs * L::kTileD, i > 0);
           tc_commit(bar(L::kDQFull));
           tc_commit(bar(L::kDSFree));
@@ -769,11 +778,10 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         auto phase_b = [&](auto mode_tag) {
           constexpr int MODE = decltype(mode_tag)::value;
           float rsum = 0.f;
-#pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
+          // dS^T of query chunk c from its 32 dP^T columns yr
+          auto chunk = [&](int c, const uint32_t* yr) {
             const int cq = qb + 32 * c;
-            uint32_t yr[32], pr[16];
-            tmem_ld32_at(ycol + cq, yr);
+            uint32_t pr[16];
             tmem_ld16_at(xcol + pcol(cq), pr);
             tc_wait_ld();
             uint32_t pk[16];
@@ -810,6 +818,26 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
                            pk[4 * v4 + 2], pk[4 * v4 + 3]);
             // and packed into X beside P^T: dK's A operand
             tmem_st16_at(xcol + dscol(cq), pk);
+          };
+          // Head dim 128: all 64 of this thread's dP^T columns first, so that
+          // Y is released (DPRead) for the next pair's S^T while dS is still
+          // being formed.  Own Y: one 32-column chunk at a time.
+          if (!L::kOwnY) {
+            uint32_t yr2[64];
+            tmem_ld32_at(ycol + qb, yr2);
+            tmem_ld32_at(ycol + qb + 32, yr2 + 32);
+            tc_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar(L::kDPRead));
+            chunk(0, yr2);
+            chunk(1, yr2 + 32);
+          } else {
+#pragma unroll 1
+            for (int c = 0; c < 2; ++c) {
+              uint32_t ych[32];
+              tmem_ld32_at(ycol + qb + 32 * c, ych);
+              chunk(c, ych);
+            }
           }
           if (MODE == kDbiasRowSum && db_key) atomicAdd(dbcol, rsum);
           if (MODE == kDbiasGroupStore && db_key && db_grp) dbcol[((q0 + qb) >> 6) * p.db_sq] = rsum;
