@@ -91,8 +91,11 @@ decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap m
   const int rg = blockIdx.y - hk * row_groups;
   const int b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int k_begin = split * p.chunk;
-  const int k_end = min(p.Lk, k_begin + p.chunk);
+  // split s takes key tiles [s nt / splits, (s + 1) nt / splits): shares
+  // differ by at most one tile, and every range starts on a tile boundary
+  const int nt_all = (p.Lk + T - 1) / T;
+  const int k_begin = static_cast<int>(static_cast<int64_t>(split) * nt_all / p.splits) * T;
+  const int k_end = min(p.Lk, static_cast<int>(static_cast<int64_t>(split + 1) * nt_all / p.splits) * T);
   const int n_tiles = k_end > k_begin ? (k_end - k_begin + T - 1) / T : 0;
   auto full = [&](int s) { return smem_u32(bars + s); };
   auto empty = [&](int s) { return smem_u32(bars + kRing + s); };
@@ -126,8 +129,8 @@ decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap m
       }
       // bias / keep values of this tile for the CTA's G query heads: each lane
       // takes 8 consecutive keys of one row with one vector load per operand
-      // (keys are 8-aligned and rows 16-byte aligned; chunks start on a
-      // multiple of 128 keys).
+      // (keys are 8-aligned and rows 16-byte aligned; ranges start on a
+      // tile boundary, a multiple of 32 keys).
       constexpr int kGroups = T / 8;
 #pragma unroll
       for (int i0 = 0; i0 < G * kGroups; i0 += 32) {

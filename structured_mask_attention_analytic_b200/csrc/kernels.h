@@ -228,7 +228,7 @@ struct DecodeProblem {
   // bias itself.
   int bias_tc = 0;
   uint32_t bias_tc_a = 0;
-  int splits, chunk;       // split-KV: keys [s*chunk, min((s+1)*chunk, Lk)), chunk % 128 == 0
+  int splits, chunk;       // split-KV: split s takes key tiles [s nt / splits, (s+1) nt / splits); chunk unused
   float* part_o;           // [B, H, splits, d]
   float* part_ml;          // [B, H, splits, 2]  (max in log2 units, sum)
   int* err;

@@ -4,6 +4,7 @@
 // sma_device_status, whose job is to synchronise).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -244,17 +245,27 @@ MaskedGeom masked_geom(int32_t B, int32_t H, int32_t KVH, int32_t Lq, int32_t Lk
   g.KT = static_cast<int>(ceil_div(Lk, kTile));
   g.decode = Lq == 1;
   if (g.decode) {
-    // split-KV: up to about two CTAs per SM of a 148-SM part (one wave), each
-    // streaming a chunk of at least 1024 keys
+    // split-KV: the kernel runs two CTAs per SM and a split takes an even
+    // share of the key tiles (kernel side).  The split count minimises the
+    // estimated time: waves of CTAs over the 2 x SM-count slots times the
+    // 64-key steps of a split, plus two steps of fixed cost per CTA; splits
+    // keep at least 512 keys, at most 64.
     const int rows_groups = (group + 7) / 8;
     const int64_t base_ctas = static_cast<int64_t>(B) * KVH * rows_groups;
-    int splits = static_cast<int>(296 / base_ctas);
-    const int max_splits = static_cast<int>(ceil_div(Lk, 1024));
-    if (splits > max_splits) splits = max_splits;
-    if (splits > 64) splits = 64;
-    if (splits < 1) splits = 1;
+    const int64_t slots = 2 * static_cast<int64_t>(num_sms());
+    const int64_t steps = ceil_div(Lk, 64);
+    const int max_splits = static_cast<int>(std::min<int64_t>(64, std::max<int64_t>(1, ceil_div(Lk, 512))));
+    int splits = 1;
+    int64_t best = -1;
+    for (int sp = 1; sp <= max_splits; ++sp) {
+      const int64_t cost = ceil_div(base_ctas * sp, slots) * (ceil_div(steps, sp) + 2);
+      if (best < 0 || cost < best) {
+        best = cost;
+        splits = sp;
+      }
+    }
     g.splits = splits;
-    g.chunk = static_cast<int>(round_up(ceil_div(Lk, splits), kTile));
+    g.chunk = 0;  // the kernel derives each split's key range
     g.part_o = 0;
     g.part_ml = align256(static_cast<size_t>(B) * H * splits * d * 4);
     g.total = align256(g.part_ml + static_cast<size_t>(B) * H * splits * 2 * 4);
