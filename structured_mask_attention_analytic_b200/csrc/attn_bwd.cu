@@ -333,7 +333,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     __syncwarp();
     uint32_t kv_it = 0, q_it = 0, o_it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
       const BUnit w = bwd_unit(p, u);
       if (w.n_pairs == 0) continue;
       if (kv_it > 0 && !mbar_wait_warp(bar(L::kKVEmpty), (kv_it - 1) & 1, abort_flag, p.f.err)) {
@@ -402,7 +402,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     // flight while the stage is still in use.
     uint32_t q_it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
       const BUnit w = bwd_unit(p, u);
       if (w.n_pairs == 0) continue;
       PairWalk pw;
@@ -522,7 +522,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
       if (!mbar_wait_warp(bar(b_), parity, abort_flag, p.f.err)) ok = false;
       return ok;
     };
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
       const BUnit w = bwd_unit(p, u);
       const int n = w.n_pairs;
       if (n == 0) continue;
@@ -636,7 +636,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     const float bias_mul = kLog2e / p.f.scale_log2;
     uint32_t pit = 0, q_it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
       const BUnit w = bwd_unit(p, u);
       if (w.n_pairs == 0) continue;
       const int key = w.kt * kTile + r;
@@ -872,7 +872,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     uint32_t pit = 0, uit = 0;
     bool ok = true;
     bool bulk_pending = false;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
       const BUnit w = bwd_unit(p, u);
       const int key = w.kt * kTile + r;
       OutT* dvrow = reinterpret_cast<OutT*>(p.dv) + w.bt * p.dv_sb + static_cast<int64_t>(w.k_off + key) * p.dv_sr +

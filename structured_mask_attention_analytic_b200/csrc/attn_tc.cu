@@ -269,7 +269,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
     __syncwarp();
     uint32_t kv_k = 0, kv_v = 0, q_it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
       const Unit w = decode_unit<POLICY>(p, u);
       const int n = w.n;
       if (n == 0) continue;
@@ -400,7 +400,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
                   (first && s == 0) ? 0u : 1u);
       }
     };
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
       const Unit w = decode_unit<POLICY>(p, u);
       const int n = w.n;
       const int nq = 1 + w.h1valid;
@@ -512,7 +512,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
     const uint32_t two_cols = (p.bias_tc_a >> 16) != 0u ? 1u : 0u;  // A has a nonzero lo column
     uint32_t kv_k = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
       const Unit w = decode_unit<POLICY>(p, u);
       const int n = w.n;
       if (n == 0) continue;
@@ -556,7 +556,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
     const uint32_t o_col = tmem + lane_off + (qi == 0 ? L::kColO0 : L::kColO1);
     uint32_t it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
       const Unit w = decode_unit<POLICY>(p, u);
       if (qi == 1 && !w.h1valid) continue;
       const int qfirst = w.q0 + qi * w.q1off;  // first query of this tile

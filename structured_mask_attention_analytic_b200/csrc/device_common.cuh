@@ -441,6 +441,18 @@ __device__ __forceinline__ float2 exp2_fma2(float2 t) {
                      __uint_as_float(__float_as_uint(j.y) * 8388608u + __float_as_uint(p.y)));
 }
 
+// Persistent CTAs take work units in snake order: round r gives CTA c the
+// unit r G + c for even r and r G + (G - 1 - c) for odd r (G = gridDim.x).
+// Units are listed from most to least work (later query tiles first in the
+// forward, earlier key tiles first in the backward), so a CTA that took a
+// heavy unit in one round takes a light one in the next and the CTAs finish
+// together; plain round robin gave CTA 0 up to 1.3x the mean work.  Indices
+// grow with r for every c, so a CTA stops at its first index past the end.
+__device__ __forceinline__ int snake_unit(int r) {
+  const int g = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  return r * g + ((r & 1) ? (g - 1 - c) : c);
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
