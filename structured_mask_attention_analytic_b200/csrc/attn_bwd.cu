@@ -269,6 +269,12 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
                   const __grid_constant__ CUtensorMap map_do, const __grid_constant__ CUtensorMap map_dq,
                   int n_units) {
   using L = TLayout<D>;
+  // Head dim 128, DFlash: the dS pass releases Y as soon as it has read
+  // dP^T, and the next pair's S^T is issued then.  The explicit-mask kernel
+  // keeps the later hand-over: the extra registers it needs there spill and
+  // cost more than the earlier start gains (packed-sequence backward 9.3 ->
+  // 9.8 ms).
+  constexpr bool kEarlyY = !L::kOwnY && POLICY == kPolicyDflash;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned by offsetting the shared array itself, so that pointers
   // derived from it keep the shared state space (shared loads, not generic)
@@ -285,6 +291,9 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
   };
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // units are listed by key tile, which orders them by work except across
+  // packed sequences of different lengths
+  const bool snake = p.f.cu_q == nullptr;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::kKVFull), 1);
@@ -333,7 +342,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     __syncwarp();
     uint32_t kv_it = 0, q_it = 0, o_it = 0;
     bool ok = true;
-    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
+    for (int rnd = 0, u = snake_unit(0, snake); u < n_units && ok; u = snake_unit(++rnd, snake)) {
       const BUnit w = bwd_unit(p, u);
       if (w.n_pairs == 0) continue;
       if (kv_it > 0 && !mbar_wait_warp(bar(L::kKVEmpty), (kv_it - 1) & 1, abort_flag, p.f.err)) {
@@ -402,7 +411,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     // flight while the stage is still in use.
     uint32_t q_it = 0;
     bool ok = true;
-    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
+    for (int rnd = 0, u = snake_unit(0, snake); u < n_units && ok; u = snake_unit(++rnd, snake)) {
       const BUnit w = bwd_unit(p, u);
       if (w.n_pairs == 0) continue;
       PairWalk pw;
@@ -522,7 +531,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
       if (!mbar_wait_warp(bar(b_), parity, abort_flag, p.f.err)) ok = false;
       return ok;
     };
-    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
+    for (int rnd = 0, u = snake_unit(0, snake); u < n_units && ok; u = snake_unit(++rnd, snake)) {
       const BUnit w = bwd_unit(p, u);
       const int n = w.n_pairs;
       if (n == 0) continue;
@@ -557,9 +566,9 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
         }
         __syncwarp();
         ++o_it;
-        if (!L::kOwnY) {
-          // Head dim 128: Y is free once the compute threads have read
-          // dP^T(i), early in forming dS^T(i): S^T(i+1) goes there then.
+        if (kEarlyY) {
+          // Head dim 128, DFlash: Y is free once the compute threads have
+          // read dP^T(i), early in forming dS^T(i): S^T(i+1) goes there then.
           if (!wait(L::kDPRead, pit & 1)) break;
           if (i + 1 < n) {
             if (!wait(L::kQFull + (nq & 1), (nq >> 1) & 1)) break;
@@ -570,7 +579,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
             }
             __syncwarp();
           }
-        } else {
+        } else if (L::kOwnY) {
           // S^T(i+1) into the other X region as soon as dQ(i-1) has left it,
           // while this pair's dS^T is still being formed.  The wait is taken
           // after a unit's last pair too, so that a unit's first pair finds
@@ -587,10 +596,17 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
           }
         }
         // dS^T(i) is formed: dK += dS^T Q and dQ = dS K (into X, after dV
-        // read P^T)
+        // read P^T).  Head dim 128 with explicit masks: S^T(i+1) goes into Y
+        // first, Y being free now (dP^T(i) consumed).
         if (!wait(L::kDSDone, pit & 1)) break;
+        constexpr bool kLateY = !L::kOwnY && !kEarlyY;
+        if (kLateY && i + 1 < n && !wait(L::kQFull + (nq & 1), (nq >> 1) & 1)) break;
         tc_fence_after();
         if (elect_one()) {
+          if (kLateY && i + 1 < n) {
+            issue_t(Y, sbase + L::kK, sbase + L::kQ + (nq & 1) * L::kTileD);
+            tc_commit(bar(L::kSFull + ((pit + 1) & 1)));
+          }
           issue_dk_dq(X, sbase + L::kQ + qs * L::kTileD, i > 0);
           tc_commit(bar(L::kDQFull));
           tc_commit(bar(L::kDSFree));
@@ -636,7 +652,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     const float bias_mul = kLog2e / p.f.scale_log2;
     uint32_t pit = 0, q_it = 0;
     bool ok = true;
-    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
+    for (int rnd = 0, u = snake_unit(0, snake); u < n_units && ok; u = snake_unit(++rnd, snake)) {
       const BUnit w = bwd_unit(p, u);
       if (w.n_pairs == 0) continue;
       const int key = w.kt * kTile + r;
@@ -819,10 +835,10 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
             // and packed into X beside P^T: dK's A operand
             tmem_st16_at(xcol + dscol(cq), pk);
           };
-          // Head dim 128: all 64 of this thread's dP^T columns first, so that
-          // Y is released (DPRead) for the next pair's S^T while dS is still
-          // being formed.  Own Y: one 32-column chunk at a time.
-          if (!L::kOwnY) {
+          // kEarlyY: all 64 of this thread's dP^T columns first, so that Y is
+          // released (DPRead) for the next pair's S^T while dS is still being
+          // formed.  Otherwise one 32-column chunk at a time.
+          if (kEarlyY) {
             uint32_t yr2[64];
             tmem_ld32_at(ycol + qb, yr2);
             tmem_ld32_at(ycol + qb + 32, yr2 + 32);
@@ -872,7 +888,7 @@ attn_bwd_t_kernel(const BwdProblem p, const __grid_constant__ CUtensorMap map_q,
     uint32_t pit = 0, uit = 0;
     bool ok = true;
     bool bulk_pending = false;
-    for (int rnd = 0, u = snake_unit(0); u < n_units && ok; u = snake_unit(++rnd)) {
+    for (int rnd = 0, u = snake_unit(0, snake); u < n_units && ok; u = snake_unit(++rnd, snake)) {
       const BUnit w = bwd_unit(p, u);
       const int key = w.kt * kTile + r;
       OutT* dvrow = reinterpret_cast<OutT*>(p.dv) + w.bt * p.dv_sb + static_cast<int64_t>(w.k_off + key) * p.dv_sr +

@@ -448,9 +448,11 @@ __device__ __forceinline__ float2 exp2_fma2(float2 t) {
 // heavy unit in one round takes a light one in the next and the CTAs finish
 // together; plain round robin gave CTA 0 up to 1.3x the mean work.  Indices
 // grow with r for every c, so a CTA stops at its first index past the end.
-__device__ __forceinline__ int snake_unit(int r) {
+// Where the list is not ordered by work (packed sequences of mixed lengths
+// in the backward), `snake` false keeps plain round robin.
+__device__ __forceinline__ int snake_unit(int r, bool snake = true) {
   const int g = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-  return r * g + ((r & 1) ? (g - 1 - c) : c);
+  return r * g + ((snake && (r & 1)) ? (g - 1 - c) : c);
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
