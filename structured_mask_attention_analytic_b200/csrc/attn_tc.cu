@@ -70,11 +70,11 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kProducerRegs == kThreads * kLaunch
               "register split must equal the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 
-// Exponentials of a softmax row: MUFU ex2 (16 per clock per SM) would take as
-// long as the row's two products on the tensor cores, so the pairs of each
-// 32-column chunk selected here are computed on the FMA pipe instead
-// (exp2_fma2): 5 of 16 pairs, about 31 %.
-__device__ __forceinline__ constexpr bool exp2_pair_on_fma(int e) { return e % 3 == 2; }
+// Exponentials of a softmax row run on MUFU ex2.  MUFU (16 per clock per
+// SM) takes as long as the row's two products on the tensor cores, so a third
+// of them once went to the FMA pipe (exp2_fma2).  Since the units are dealt in
+// snake order that is 1-2 % slower in short runs and 1 % slower over 50 steps
+// under the power cap (measured), so every exponential is on MUFU again.
 
 template <int D, bool BTC = false>
 struct Layout {
@@ -788,12 +788,8 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
             const float2 t = fma2(make_float2(x[32 * c + 2 * e], x[32 * c + 2 * e + 1]),
                                   make_float2(exp_scale, exp_scale), make_float2(-msub, -msub));
             float2 pp;
-            if (exp2_pair_on_fma(e)) {
-              pp = exp2_fma2(t);
-            } else {
-              pp.x = fast_exp2(t.x);
-              pp.y = fast_exp2(t.y);
-            }
+            pp.x = fast_exp2(t.x);
+            pp.y = fast_exp2(t.y);
             ls4[e & 3] = add2(ls4[e & 3], pp);
             pk[e] = DT == SMA_BF16 ? pack_bf16x2(pp.x, pp.y) : pack_f16x2(pp.x, pp.y);
           }
@@ -823,8 +819,7 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
       OutT* orow = reinterpret_cast<OutT*>(p.o) + (POLICY == kPolicyVarlen ? 0 : w.b) * p.o_sb +
                    static_cast<int64_t>(w.q_off + q) * p.o_sr +
                    h * p.o_sh;
-      // A row that kept no key has max -inf (its sum is not 0: exp2_fma2 of
-      // -inf is 2^-125).
+      // A row that kept no key has max -inf (and sum 0).
       const bool live = m_ref != -INFINITY;
       const float inv_l = live ? 1.0f / l_sum : 0.f;
       // Key-range segment: unnormalised O and (max, sum) go to the partials.
