@@ -887,10 +887,10 @@ attn_tc_kernel(const AttnProblem p, const __grid_constant__ CUtensorMap map_q,
 //   O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,
 //   lse = ln 2 * (M + log2 sum_s 2^(m_s - M) l_s).
 // One warp per row: lane s reads segment s's (m_s, l_s) (at most 32
-// segments), the warp reduces M and the sum, then every lane accumulates its
-// D / 32 columns over the segments, eight independent loads at a time.  A
-// segment that kept no key of the row (l_s = 0) may not have written O_s and
-// is never read.
+// segments) while every lane loads its D / 32 columns of all segments' O_s;
+// the warp reduces M and the sum, then each lane accumulates its columns.  A
+// segment that kept no key of the row (l_s = 0) may not have written O_s:
+// its loaded values are discarded (weight 0, selected out).
 template <int D, int DT>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnProblem p) {
   typedef typename std::conditional<DT == SMA_BF16, __nv_bfloat16, __half>::type OutT;
@@ -902,6 +902,28 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnProblem p) 
   const float2 v = lane < ns
                        ? reinterpret_cast<const float2*>(p.part_ml)[static_cast<int64_t>(lane) * p.part_rows + row]
                        : make_float2(-INFINITY, 0.f);
+  // Every segment's O columns are loaded at once, before the weights are
+  // known (one memory round trip for the whole row); a segment that kept no
+  // key may not have written them, so its values are dropped by a select,
+  // never multiplied.
+  const float* src = p.part_o + row * D + lane * kPer;
+  const int64_t seg_stride = p.part_rows * D;
+  float vals[32][kPer];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) vals[i][e] = 0.f;
+    if (i < ns) {
+      const float* sp = src + i * seg_stride;
+      if (kPer == 4) {
+        const float4 a = *reinterpret_cast<const float4*>(sp);
+        vals[i][0] = a.x; vals[i][1] = a.y; vals[i][2] = a.z; vals[i][3] = a.w;
+      } else {
+        const float2 a = *reinterpret_cast<const float2*>(sp);
+        vals[i][0] = a.x; vals[i][1] = a.y;
+      }
+    }
+  }
   const bool live = v.y > 0.f;
   float mx = live ? v.x : -INFINITY;
 #pragma unroll
@@ -913,33 +935,11 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnProblem p) 
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-  const float* src = p.part_o + row * D + lane * kPer;
-  const int64_t seg_stride = p.part_rows * D;
-  constexpr int kGroup = 8;
-  for (int s0 = 0; s0 < ns; s0 += kGroup) {
-    float ws[kGroup];
-    float vals[kGroup][kPer];
 #pragma unroll
-    for (int i = 0; i < kGroup; ++i) {
-      ws[i] = __shfl_sync(0xffffffffu, wgt, (s0 + i) & 31);
-      if (s0 + i >= ns) ws[i] = 0.f;
+  for (int i = 0; i < 32; ++i) {
+    const float w_i = __shfl_sync(0xffffffffu, wgt, i);  // 0 for segments without keys
 #pragma unroll
-      for (int e = 0; e < kPer; ++e) vals[i][e] = 0.f;
-      if (ws[i] != 0.f) {
-        const float* sp = src + (s0 + i) * seg_stride;
-        if (kPer == 4) {
-          const float4 a = *reinterpret_cast<const float4*>(sp);
-          vals[i][0] = a.x; vals[i][1] = a.y; vals[i][2] = a.z; vals[i][3] = a.w;
-        } else {
-          const float2 a = *reinterpret_cast<const float2*>(sp);
-          vals[i][0] = a.x; vals[i][1] = a.y;
-        }
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kGroup; ++i)
-#pragma unroll
-      for (int e = 0; e < kPer; ++e) acc[e] = fmaf(ws[i], vals[i][e], acc[e]);
+    for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w_i, w_i != 0.f ? vals[i][e] : 0.f, acc[e]);
   }
   const float inv = l > 0.f ? 1.0f / l : 0.f;
   const int q = static_cast<int>(row % p.Lq);
