@@ -15,7 +15,9 @@
 // across CTAs (split-KV); a second kernel merges the per-chunk (max, sum,
 // unnormalised O) triples.
 //
-// Consumer lane layout: a key row is read by d/8 lanes, 8 elements each.
+// Consumer lane layout: a key row is read by d/8 lanes, 8 elements each; the
+// G dot products of a key are summed over those lanes in transposed form, so
+// that each lane ends with one head's score and keeps that head's softmax.
 #include <cudaTypedefs.h>
 
 #include <cstdio>
@@ -205,16 +207,21 @@ decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap m
 #pragma unroll
       for (int e = 0; e < 8; ++e) qf[r][e] *= p.scale_log2;
     }
-    float m[G], l[G], o[G][8];
+    // Each lane keeps the online softmax of one query head of the CTA: head
+    // hsel, the top log2(G) bits of its lane index within the key slot.
+    constexpr int LG = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
+    constexpr int LL = LPK == 8 ? 3 : 4;
+    static_assert(LPK == (1 << LL) && G == (1 << LG) && LG <= LL, "lane layout");
+    const int hsel = dl >> (LL - LG);
+    const int hbase = slot * LPK;  // first lane of this key slot
+    float m_own = -INFINITY, l_own = 0.f;
+    float o[G][8];
 #pragma unroll
-    for (int r = 0; r < G; ++r) {
-      m[r] = -INFINITY;
-      l[r] = 0.f;
+    for (int r = 0; r < G; ++r)
 #pragma unroll
       for (int e = 0; e < 8; ++e) o[r][e] = 0.f;
-    }
-    // Per tile: every score of this warp's keys first, then one max / sum /
-    // rescale per row, then the P.V pass -- no branch, so the G rows overlap.
+    // Per tile: the own head's score of every key of this warp first, then one
+    // max / sum / rescale, then the P.V pass -- no branch.
     constexpr int kSteps = T / (kConsumerWarps * KPW);
     constexpr int kSub = kSteps < 4 ? kSteps : 4;  // key-steps per online-softmax update
     bool ok = true;
@@ -225,12 +232,13 @@ decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap m
       const uint8_t* vt = kt + kTileBytes;
 #pragma unroll
       for (int st0 = 0; st0 < kSteps; st0 += kSub) {
-        float sc[kSub][G];
+        float sc[kSub];  // the own head's scores, then probabilities
 #pragma unroll
         for (int st = 0; st < kSub; ++st) {
           const int c = ((st0 + st) * kConsumerWarps + warp) * KPW + slot;
           float kf[8];
           smem8<DT>(kt + (c * D + e0) * L::kEsz, kf);
+          float d[G];
 #pragma unroll
           for (int r = 0; r < G; ++r) {
             // two products per instruction (fp32 pairs), the halves added last
@@ -238,37 +246,58 @@ decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap m
 #pragma unroll
             for (int e = 0; e < 8; e += 2)
               d2 = fma2(make_float2(qf[r][e], qf[r][e + 1]), make_float2(kf[e], kf[e + 1]), d2);
-            float d = d2.x + d2.y;
-#pragma unroll
-            for (int off = 1; off < LPK; off <<= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-            const bool keep = s_keep[(s * G + r) * T + c] != 0;
-            sc[st][r] = keep ? d + s_bias[(s * G + r) * T + c] : -INFINITY;
+            d[r] = d2.x + d2.y;
           }
+          // Sum over the LPK lanes of the key, transposed: step i (lane
+          // offset LPK >> (i + 1)) keeps the half of the remaining heads that
+          // the lane's bit selects and adds the partner's partial sums of it
+          // (log2 G exchanges in place of G butterflies); a butterfly over
+          // the remaining offsets completes the one head left.
+#pragma unroll
+          for (int i = 0; i < LG; ++i) {
+            const int off = LPK >> (i + 1);
+            const bool up = (dl & off) != 0;
+            const int n = G >> i;
+#pragma unroll
+            for (int j = 0; j < (G >> (i + 1)); ++j) {
+              const float mine = up ? d[j + n / 2] : d[j];
+              const float give = up ? d[j] : d[j + n / 2];
+              d[j] = mine + __shfl_xor_sync(0xffffffffu, give, off);
+            }
+          }
+          float v = d[0];
+#pragma unroll
+          for (int off = LPK >> (LG + 1); off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+          const bool keep = s_keep[(s * G + hsel) * T + c] != 0;
+          sc[st] = keep ? v + s_bias[(s * G + hsel) * T + c] : -INFINITY;
+        }
+        // the own head over these keys of every slot of the warp
+        float mx = sc[0];
+#pragma unroll
+        for (int st = 1; st < kSub; ++st) mx = fmaxf(mx, sc[st]);
+#pragma unroll
+        for (int off = LPK; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float m_new = fmaxf(m_own, mx);
+        const bool dead = m_new == -INFINITY;
+        const float alpha = dead ? 1.f : fast_exp2(m_own - m_new);  // exp2(-inf) = 0
+        const float msub = dead ? 0.f : m_new;
+        float ps = 0.f;
+#pragma unroll
+        for (int st = 0; st < kSub; ++st) {
+          sc[st] = fast_exp2(sc[st] - msub);
+          ps += sc[st];
         }
 #pragma unroll
+        for (int off = LPK; off < 32; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+        l_own = l_own * alpha + ps;
+        m_own = m_new;
+        // every head's rescale factor, from a lane of this slot that owns it
+#pragma unroll
         for (int r = 0; r < G; ++r) {
-          float mx = sc[0][r];
-#pragma unroll
-          for (int st = 1; st < kSub; ++st) mx = fmaxf(mx, sc[st][r]);
-#pragma unroll
-          for (int off = LPK; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-          const float m_new = fmaxf(m[r], mx);
-          const bool dead = m_new == -INFINITY;
-          const float alpha = dead ? 1.f : fast_exp2(m[r] - m_new);  // exp2(-inf) = 0
-          const float msub = dead ? 0.f : m_new;
-          float ps = 0.f;
-#pragma unroll
-          for (int st = 0; st < kSub; ++st) {
-            sc[st][r] = fast_exp2(sc[st][r] - msub);
-            ps += sc[st][r];
-          }
-#pragma unroll
-          for (int off = LPK; off < 32; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-          l[r] = l[r] * alpha + ps;
-          m[r] = m_new;
+          const float a_r = __shfl_sync(0xffffffffu, alpha, hbase + (r << (LL - LG)));
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
-            const float2 oo = mul2(make_float2(o[r][e], o[r][e + 1]), make_float2(alpha, alpha));
+            const float2 oo = mul2(make_float2(o[r][e], o[r][e + 1]), make_float2(a_r, a_r));
             o[r][e] = oo.x;
             o[r][e + 1] = oo.y;
           }
@@ -279,14 +308,16 @@ decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap m
           float vf[8];
           smem8<DT>(vt + (c * D + e0) * L::kEsz, vf);
 #pragma unroll
-          for (int r = 0; r < G; ++r)
+          for (int r = 0; r < G; ++r) {
+            const float p_r = __shfl_sync(0xffffffffu, sc[st], hbase + (r << (LL - LG)));
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
-              const float2 oo = fma2(make_float2(sc[st][r], sc[st][r]), make_float2(vf[e], vf[e + 1]),
+              const float2 oo = fma2(make_float2(p_r, p_r), make_float2(vf[e], vf[e + 1]),
                                      make_float2(o[r][e], o[r][e + 1]));
               o[r][e] = oo.x;
               o[r][e + 1] = oo.y;
             }
+          }
         }
       }
       __syncwarp();
@@ -306,12 +337,10 @@ decode_split_kernel(const DecodeProblem p, const __grid_constant__ CUtensorMap m
 #pragma unroll
         for (int e = 0; e < 8; ++e) s_o[(warp * G + r) * D + e0 + e] = o[r][e];
     }
-    if (lane == 0) {
-#pragma unroll
-      for (int r = 0; r < G; ++r) {
-        s_ml[(warp * G + r) * 2] = m[r];
-        s_ml[(warp * G + r) * 2 + 1] = l[r];
-      }
+    // (max, sum) of each head from the first lane of slot 0 that owns it
+    if (slot == 0 && (dl & ((1 << (LL - LG)) - 1)) == 0) {
+      s_ml[(warp * G + hsel) * 2] = m_own;
+      s_ml[(warp * G + hsel) * 2 + 1] = l_own;
     }
   }
   __syncthreads();
