@@ -354,3 +354,35 @@ def test_deterministic_dbias_workspace_query():
     assert q(nat.SMA_BF16, 96, [4, 8, 1, 1024]) == nat.SMA_ERR_UNSUPPORTED
     assert lib.masked_attn_bwd_dbias_workspace_size(nat.SMA_BF16, 4, 16, 8, 1000, 128, None,
                                                     ctypes.byref(n)) == nat.SMA_ERR_INVALID_ARG
+
+
+def _decode_splits(batch, heads, kv_heads, k_len, sms=148):
+    """The split-KV cost model restated: waves of CTAs over two per SM times
+    the 64-key steps of a split plus two of fixed cost; splits keep at least
+    512 keys, at most 64; the first minimum wins."""
+    group = heads // kv_heads
+    base = batch * kv_heads * ((group + 7) // 8)
+    steps = -(-k_len // 64)
+    best, best_s = None, 1
+    for sp in range(1, min(64, max(1, -(-k_len // 512))) + 1):
+        cost = -(-base * sp // (2 * sms)) * (-(-steps // sp) + 2)
+        if best is None or cost < best:
+            best, best_s = cost, sp
+    return best_s
+
+
+def test_decode_workspace_follows_the_split_cost_model():
+    """Single-query calls: the workspace holds fp32 O and (max, sum) for each
+    (batch, head, split); the split count fills the CTA slots (9 splits of
+    16384 keys for 8 x 8 KV heads: 576 CTAs, two waves of 296; 37 for one
+    row of 8 KV heads over 32768 keys).  No GPU is present here, so the
+    library assumes a 148-SM part."""
+    lib = nat.load()
+    n = ctypes.c_size_t()
+    a256 = lambda x: -(-x // 256) * 256  # noqa: E731
+    for (b, h, kvh, lk, want) in [(8, 32, 8, 16384, 9), (1, 32, 8, 32768, 37), (1, 8, 8, 1000, 2)]:
+        sp = _decode_splits(b, h, kvh, lk)
+        assert sp == want
+        assert lib.masked_attn_fwd_workspace_size(b, h, kvh, 1, lk, 128, None, ctypes.byref(n)) == 0
+        part_ml = a256(b * h * sp * 128 * 4)
+        assert n.value == a256(part_ml + b * h * sp * 2 * 4)
