@@ -103,14 +103,6 @@ sma_status sma_device_status(void* stream, int32_t* device_error);
  * method; it checks the failure-reporting path without faulting the GPU. */
 sma_status sma_selftest_wait_timeout(int64_t timeout_ns, int64_t* dev_out, void* stream);
 
-/* Diagnostic: dev_out[i] = 2^dev_in[i] (device float32 arrays of n floats,
- * n even) as the attention softmax computes it on the FMA pipe for part of
- * each row: t = round(t) + f, 2^f from a cubic (relative error <= 7.5e-5 on
- * f in [-1/2, 1/2]), 2^round(t) added to the exponent field.  Arguments below
- * -125 are clamped to -125 (so -inf gives 2^-125, not 0).  Not part of the
- * method; it lets a test compare this exponential with CUDA's. */
-sma_status sma_selftest_exp2(const float* dev_in, float* dev_out, int64_t n, void* stream);
-
 /* ------------------------------------------------------------------------
  * DFlash mask description.
  *

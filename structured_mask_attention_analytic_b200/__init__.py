@@ -26,7 +26,6 @@ from .ops import (  # noqa: F401
     masked_attn_fwd,
     masked_attn_fwd_workspace_size,
     round_up_k,
-    selftest_exp2,
     selftest_wait_timeout,
     sparse_attn_fwd,
     sparse_attn_fwd_workspace_size,

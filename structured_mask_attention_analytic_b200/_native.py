@@ -55,7 +55,6 @@ _SIGNATURES = {
     "sma_abi_version": (c_i32, []),
     "sma_device_status": (c_i32, [c_vp, c_i32p]),
     "sma_selftest_wait_timeout": (c_i32, [ctypes.c_int64, c_vp, c_vp]),
-    "sma_selftest_exp2": (c_i32, [c_vp, c_vp, ctypes.c_int64, c_vp]),
     "dfa_block_map_dims": (c_i32, [ctypes.POINTER(DfaMaskDesc), c_i32p, c_i32p]),
     "dfa_block_map": (c_i32, [ctypes.POINTER(DfaMaskDesc), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "dfa_attn_fwd_workspace_size": (c_i32, [ctypes.POINTER(DfaMaskDesc), c_i32, c_i32, c_i32, c_sizep]),

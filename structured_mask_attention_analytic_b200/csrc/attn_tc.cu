@@ -72,9 +72,10 @@ constexpr uint32_t kTmemCols = 512;
 
 // Exponentials of a softmax row run on MUFU ex2.  MUFU (16 per clock per
 // SM) takes as long as the row's two products on the tensor cores, so a third
-// of them once went to the FMA pipe (exp2_fma2).  Since the units are dealt in
-// snake order that is 1-2 % slower in short runs and 1 % slower over 50 steps
-// under the power cap (measured), so every exponential is on MUFU again.
+// of them once went to the FMA pipe (a cubic for 2^f and an integer add into
+// the exponent field).  Since the units are dealt in snake order that is 1-2 %
+// slower in short runs and 1 % slower over 50 steps under the power cap
+// (measured), so every exponential is on MUFU.
 
 template <int D, bool BTC = false>
 struct Layout {

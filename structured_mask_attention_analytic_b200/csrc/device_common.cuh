@@ -412,35 +412,6 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
   return r;
 }
 
-// 2^t for a pair of arguments on the FMA and integer pipes, leaving the
-// MUFU unit (ex2.approx, 16 results per clock per SM) to the other columns
-// of a softmax row.  t = n + f with n = round(t): adding 1.5 * 2^23 rounds t
-// to an integer held in the low mantissa bits; f = t - n lies in [-1/2, 1/2];
-// 2^f is a cubic whose coefficients fit_exp2_poly.py derives (relative error
-// at most 7.5e-5 over [-1/2, 1/2] in float32, against 2^-9 for rounding P to
-// bf16); 2^n is added to the exponent field (the low bits of the rounded sum,
-// shifted left by 23, are n << 23).  Arguments are clamped at -125 from
-// below: -inf gives 2^-125 (2.4e-38) rather than 0, so a softmax using this
-// must tell an empty row by its max (-inf), not by its sum.  Arguments up to
-// +127 are exact in range.
-constexpr float kExp2C0 = 9.999280572e-01f;
-constexpr float kExp2C1 = 6.932609677e-01f;
-constexpr float kExp2C2 = 2.426111251e-01f;
-constexpr float kExp2C3 = 5.517166480e-02f;
-__device__ __forceinline__ float2 exp2_fma2(float2 t) {
-  t.x = fmaxf(t.x, -125.f);
-  t.y = fmaxf(t.y, -125.f);
-  const float2 magic = make_float2(12582912.f, 12582912.f);
-  const float2 j = add2(t, magic);
-  const float2 f = sub2(t, sub2(j, magic));
-  float2 p = fma2(f, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
-  p = fma2(p, f, make_float2(kExp2C1, kExp2C1));
-  p = fma2(p, f, make_float2(kExp2C0, kExp2C0));
-  // n << 23 added to the exponent field as one integer multiply-add
-  return make_float2(__uint_as_float(__float_as_uint(j.x) * 8388608u + __float_as_uint(p.x)),
-                     __uint_as_float(__float_as_uint(j.y) * 8388608u + __float_as_uint(p.y)));
-}
-
 // Persistent CTAs take work units in snake order: round r gives CTA c the
 // unit r G + c for even r and r G + (G - 1 - c) for odd r (G = gridDim.x).
 // Units are listed from most to least work (later query tiles first in the

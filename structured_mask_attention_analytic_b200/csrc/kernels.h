@@ -328,8 +328,6 @@ int set_last_error(int code, const char* message);
 
 cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, int* err, int64_t* out,
                                          cudaStream_t stream);
-// out[i] = the softmax's FMA-pipe 2^in[i] for n (even) floats on the device.
-cudaError_t launch_exp2_fma_selftest(const float* in, float* out, int64_t n, cudaStream_t stream);
 
 // Device error word in the current context (looked up once per context).
 int* device_error_word(cudaError_t* status);

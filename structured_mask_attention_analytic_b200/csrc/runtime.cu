@@ -108,28 +108,6 @@ cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, int* err, int64_t*
   return cudaGetLastError();
 }
 
-namespace {
-// out[i] = exp2_fma2 of in[i] (pairs), the FMA-pipe exponential of the
-// attention softmax.
-__global__ void exp2_fma_selftest_kernel(const float* in, float* out, int64_t n_pairs) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n_pairs) return;
-  const float2 r = exp2_fma2(make_float2(in[2 * i], in[2 * i + 1]));
-  out[2 * i] = r.x;
-  out[2 * i + 1] = r.y;
-}
-}  // namespace
-
-cudaError_t launch_exp2_fma_selftest(const float* in, float* out, int64_t n,
-                                     cudaStream_t stream) {
-  const int64_t pairs = n / 2;
-  if (pairs == 0) return cudaSuccess;
-  const int block = 256;
-  exp2_fma_selftest_kernel<<<static_cast<unsigned>((pairs + block - 1) / block), block, 0,
-                             stream>>>(in, out, pairs);
-  return cudaGetLastError();
-}
-
 int num_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;

@@ -459,16 +459,6 @@ sma_status sma_selftest_wait_timeout(int64_t timeout_ns, int64_t* dev_out, void*
   return ok();
 }
 
-sma_status sma_selftest_exp2(const float* dev_in, float* dev_out, int64_t n, void* stream) {
-  if (dev_in == nullptr || dev_out == nullptr) return fail(SMA_ERR_INVALID_ARG, "NULL pointer");
-  if (n < 0 || (n & 1) != 0) return fail(SMA_ERR_INVALID_ARG, "n must be even and >= 0");
-  if ((reinterpret_cast<uintptr_t>(dev_in) & 3u) != 0 || (reinterpret_cast<uintptr_t>(dev_out) & 3u) != 0)
-    return fail(SMA_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
-  cudaError_t e = launch_exp2_fma_selftest(dev_in, dev_out, n, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "self-test launch failed");
-  return ok();
-}
-
 sma_status dfa_block_map_dims(const dfa_mask_desc* desc, int32_t* q_tiles, int32_t* kv_tiles) {
   sma_status s = check_desc(desc);
   if (s != SMA_OK) return s;

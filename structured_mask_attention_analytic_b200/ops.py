@@ -654,15 +654,3 @@ def selftest_wait_timeout(timeout_ns: int, out: torch.Tensor) -> None:
     if out.dtype != torch.int64 or out.numel() < 2:
         raise ValueError("out must be a CUDA int64 tensor with 2 elements")
     nat.check(_lib().sma_selftest_wait_timeout(int(timeout_ns), _ptr(out), _stream(out)))
-
-
-def selftest_exp2(x: torch.Tensor) -> torch.Tensor:
-    """Diagnostic: the softmax's FMA-pipe 2^x for a CUDA float32 tensor with
-    an even number of elements (see ``sma_selftest_exp2``)."""
-    _require_cuda(x)
-    if x.dtype != torch.float32 or x.numel() % 2:
-        raise ValueError("x must be a CUDA float32 tensor with an even number of elements")
-    x = x.contiguous()
-    out = torch.empty_like(x)
-    nat.check(_lib().sma_selftest_exp2(_ptr(x), _ptr(out), x.numel(), _stream(x)))
-    return out
