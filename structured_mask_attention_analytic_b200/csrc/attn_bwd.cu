@@ -1011,7 +1011,40 @@ cudaError_t launch_bwd_t(const BwdProblem& p, const CUtensorMap& mq, const CUten
   return cudaGetLastError();
 }
 
-// rowsum(dO * O) per (b, h, q) and the zeroed dQ accumulator; one warp per row.
+// n consecutive elements (2 or 4) of a row as floats, one vector load.
+template <int DT>
+__device__ __forceinline__ void load_vec_as_float(const void* base, int n, float (&f)[4]) {
+  if (DT == SMA_FP32) {
+    if (n == 4) {
+      const float4 a = *reinterpret_cast<const float4*>(base);
+      f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    } else {
+      const float2 a = *reinterpret_cast<const float2*>(base);
+      f[0] = a.x; f[1] = a.y;
+    }
+  } else {
+    uint32_t w[2];
+    if (n == 4) {
+      const uint2 a = *reinterpret_cast<const uint2*>(base);
+      w[0] = a.x; w[1] = a.y;
+    } else {
+      w[0] = *reinterpret_cast<const uint32_t*>(base);
+      w[1] = 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float2 v = unpack2<DT>(w[i]);
+      f[2 * i] = v.x;
+      f[2 * i + 1] = v.y;
+    }
+  }
+}
+
+// D = rowsum(dO * O) of one (b, q, h) row per warp, and the row's fp32 dQ
+// accumulator zeroed.  At head dim 64 or 128 each lane takes d / 32
+// consecutive elements with one vector load per operand (scalar loads if a
+// row is not aligned for them) and zeroes its part of the accumulator with
+// one vector store.
 template <int DT>
 __global__ void bwd_prep_kernel(const BwdProblem p) {
   const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -1023,17 +1056,33 @@ __global__ void bwd_prep_kernel(const BwdProblem p) {
   const int q = static_cast<int>(bq % p.f.Lq);
   const int b = static_cast<int>(bq / p.f.Lq);
   const int d = p.f.d;
-  const void* orow = reinterpret_cast<const uint8_t*>(p.f.o) +
-                     (b * p.f.o_sb + static_cast<int64_t>(q) * p.f.o_sr + h * p.f.o_sh) * (DT == SMA_FP32 ? 4 : 2);
-  const void* grow = reinterpret_cast<const uint8_t*>(p.dout) +
-                     (b * p.do_sb + static_cast<int64_t>(q) * p.do_sr + h * p.do_sh) * (DT == SMA_FP32 ? 4 : 2);
+  constexpr int kEs = DT == SMA_FP32 ? 4 : 2;
+  const uint8_t* orow = reinterpret_cast<const uint8_t*>(p.f.o) +
+                        (b * p.f.o_sb + static_cast<int64_t>(q) * p.f.o_sr + h * p.f.o_sh) * kEs;
+  const uint8_t* grow = reinterpret_cast<const uint8_t*>(p.dout) +
+                        (b * p.do_sb + static_cast<int64_t>(q) * p.do_sr + h * p.do_sh) * kEs;
+  float* acc = p.dq_acc + gw * d;
+  const int per = d >> 5;
+  const bool vec = (d == 64 || d == 128) &&
+                   ((reinterpret_cast<uintptr_t>(orow) | reinterpret_cast<uintptr_t>(grow)) &
+                    static_cast<uintptr_t>(per * kEs - 1)) == 0;
   float s = 0.f;
-  for (int e = lane; e < d; e += 32) s += load_as_float<DT>(orow, e) * load_as_float<DT>(grow, e);
+  if (vec) {
+    float of[4], gf[4];
+    load_vec_as_float<DT>(orow + lane * per * kEs, per, of);
+    load_vec_as_float<DT>(grow + lane * per * kEs, per, gf);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (i < per) s = fmaf(of[i], gf[i], s);
+    if (per == 4) reinterpret_cast<float4*>(acc)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+    else reinterpret_cast<float2*>(acc)[lane] = make_float2(0.f, 0.f);
+  } else {
+    for (int e = lane; e < d; e += 32) s += load_as_float<DT>(orow, e) * load_as_float<DT>(grow, e);
+    for (int e = lane; e < d; e += 32) acc[e] = 0.f;
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane == 0) p.dvec[(static_cast<int64_t>(b) * p.f.H + h) * p.f.Lq + q] = s;
-  float* acc = p.dq_acc + gw * d;
-  for (int e = lane; e < d; e += 32) acc[e] = 0.f;
 }
 
 // codes[row][qt][kt] from the forward lists (2 = FULL, 1 = PARTIAL); the
@@ -1101,30 +1150,56 @@ __global__ void __launch_bounds__(kTrThreads) transpose_lists_kernel(const BwdPr
   }
 }
 
-// dQ = scale * accumulator, in the output dtype; one thread per 4 elements.
+// dQ = scale * accumulator in the output dtype, one (b, q, h) row per warp:
+// at head dim 64 or 128 each lane converts d / 32 consecutive elements with
+// one vector load and one vector store (scalar stores if the dQ row is not
+// aligned for them).
 template <int DT>
 __global__ void dq_convert_kernel(const BwdProblem p) {
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int d4 = p.f.d / 4;
-  const int64_t total = static_cast<int64_t>(p.f.B) * p.f.Lq * p.f.H * d4;
-  if (t >= total) return;
-  const int e = static_cast<int>(t % d4) * 4;
-  const int64_t row = t / d4;  // (b, q, h)
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = static_cast<int64_t>(p.f.B) * p.f.Lq * p.f.H;
+  if (row >= rows) return;
   const int h = static_cast<int>(row % p.f.H);
   const int64_t bq = row / p.f.H;
   const int q = static_cast<int>(bq % p.f.Lq);
   const int b = static_cast<int>(bq / p.f.Lq);
-  const float4 a = reinterpret_cast<const float4*>(p.dq_acc + row * p.f.d + e)[0];
-  const int64_t off = b * p.dq_sb + static_cast<int64_t>(q) * p.dq_sr + h * p.dq_sh + e;
-  if (DT == SMA_FP32) {
-    float* dst = reinterpret_cast<float*>(p.dq) + off;
-    dst[0] = a.x * p.scale; dst[1] = a.y * p.scale; dst[2] = a.z * p.scale; dst[3] = a.w * p.scale;
+  const int d = p.f.d;
+  constexpr int kEs = DT == SMA_FP32 ? 4 : 2;
+  const float* src = p.dq_acc + row * d;
+  const int64_t off = b * p.dq_sb + static_cast<int64_t>(q) * p.dq_sr + h * p.dq_sh;
+  uint8_t* dst = reinterpret_cast<uint8_t*>(p.dq) + off * kEs;
+  const int per = d >> 5;
+  const bool vec = (d == 64 || d == 128) &&
+                   (reinterpret_cast<uintptr_t>(dst) & static_cast<uintptr_t>(per * kEs - 1)) == 0;
+  if (vec) {
+    float a[4];
+    if (per == 4) {
+      const float4 v = reinterpret_cast<const float4*>(src)[lane];
+      a[0] = v.x; a[1] = v.y; a[2] = v.z; a[3] = v.w;
+    } else {
+      const float2 v = reinterpret_cast<const float2*>(src)[lane];
+      a[0] = v.x; a[1] = v.y; a[2] = 0.f; a[3] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] *= p.scale;
+    uint8_t* dl = dst + lane * per * kEs;
+    if (DT == SMA_FP32) {
+      if (per == 4) *reinterpret_cast<float4*>(dl) = make_float4(a[0], a[1], a[2], a[3]);
+      else *reinterpret_cast<float2*>(dl) = make_float2(a[0], a[1]);
+    } else {
+      const uint32_t w0 = DT == SMA_BF16 ? pack_bf16x2(a[0], a[1]) : pack_f16x2(a[0], a[1]);
+      const uint32_t w1 = DT == SMA_BF16 ? pack_bf16x2(a[2], a[3]) : pack_f16x2(a[2], a[3]);
+      if (per == 4) *reinterpret_cast<uint2*>(dl) = make_uint2(w0, w1);
+      else *reinterpret_cast<uint32_t*>(dl) = w0;
+    }
   } else {
-    const uint32_t w0 = DT == SMA_BF16 ? pack_bf16x2(a.x * p.scale, a.y * p.scale)
-                                       : pack_f16x2(a.x * p.scale, a.y * p.scale);
-    const uint32_t w1 = DT == SMA_BF16 ? pack_bf16x2(a.z * p.scale, a.w * p.scale)
-                                       : pack_f16x2(a.z * p.scale, a.w * p.scale);
-    *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.dq) + off) = make_uint2(w0, w1);
+    for (int e = lane; e < d; e += 32) {
+      const float v = src[e] * p.scale;
+      if (DT == SMA_FP32) reinterpret_cast<float*>(dst)[e] = v;
+      else if (DT == SMA_BF16) reinterpret_cast<__nv_bfloat16*>(dst)[e] = __float2bfloat16_rn(v);
+      else reinterpret_cast<__half*>(dst)[e] = __float2half_rn(v);
+    }
   }
 }
 
@@ -1201,8 +1276,8 @@ cudaError_t launch_dbias_reduce(const float* part, int B, int H, int R, float* o
 
 cudaError_t launch_dq_convert(const BwdProblem& pin, cudaStream_t stream) {
   const BwdProblem p = flat_view(pin);
-  const int64_t total = static_cast<int64_t>(p.f.B) * p.f.Lq * p.f.H * (p.f.d / 4);
-  const unsigned grid = static_cast<unsigned>((total + 255) / 256);
+  const int64_t rows = static_cast<int64_t>(p.f.B) * p.f.Lq * p.f.H;  // one warp each
+  const unsigned grid = static_cast<unsigned>((rows * 32 + 255) / 256);
   if (p.f.dtype == SMA_BF16) dq_convert_kernel<SMA_BF16><<<grid, 256, 0, stream>>>(p);
   else if (p.f.dtype == SMA_FP16) dq_convert_kernel<SMA_FP16><<<grid, 256, 0, stream>>>(p);
   else dq_convert_kernel<SMA_FP32><<<grid, 256, 0, stream>>>(p);
