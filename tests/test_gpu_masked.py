@@ -136,6 +136,19 @@ def test_decode_small(bshape, mshape, d):
     _run(q, k, v, mask, bias, False, what=f"decode {bshape} {mshape}")
 
 
+@pytest.mark.parametrize("heads,kv_heads", [(8, 8), (8, 4), (8, 1), (6, 2), (12, 2)], ids=str)
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_query_head_groups(heads, kv_heads, d):
+    """Groups of 1, 2, 8 query heads per KV head (and 3, 6, which leave rows
+    of the CTA's head block empty): each lane of a key sums and keeps the
+    softmax of one head of its block, so every block size is checked."""
+    rng = wl.rng_for(14)
+    q, k, v = _qkv(rng, 2, 1, 1500, heads, kv_heads, d)
+    bias = wl.normal(rng, (2, heads, 1, 1536), "bf16")
+    mask = torch.from_numpy(rng.random((2, 1, 1, 1536)) < 0.8)
+    _run(q, k, v, mask, bias, False, what=f"decode H={heads} KVH={kv_heads} d={d}")
+
+
 def test_decode_equals_unswapped_rows():
     """The grouped-head decode path gives the same rows as the general path
     run on a 2-row query whose first row is the decode query."""
