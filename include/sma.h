@@ -261,7 +261,10 @@ sma_status mask_tile_summary(const uint8_t* mask, const int64_t mask_sizes[4],
  * split-KV partials of the single-query path, and for other short-query
  * problems the partials of the key-range split: each unit's key tiles cut
  * into segments run on separate SMs, merged by a second kernel).  mask_sizes may be NULL when
- * no mask will be passed. */
+ * no mask will be passed.  The single-query split count follows the current
+ * device's SM count (148 when no device is current), so query the size with
+ * the device that will run the call current; a smaller workspace is refused
+ * with SMA_ERR_WORKSPACE. */
 sma_status masked_attn_fwd_workspace_size(int32_t batch, int32_t heads, int32_t kv_heads,
                                           int32_t q_len, int32_t k_len, int32_t head_dim,
                                           const int64_t mask_sizes[4], size_t* bytes);
